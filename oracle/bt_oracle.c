@@ -1,0 +1,304 @@
+/*
+ * CPU oracle for the ternary-weight FWHT-1024 path -- TEST INFRASTRUCTURE.
+ *
+ * Plain, slow, obviously correct FP64 C. Only the tests, the smoke check and
+ * the benchmark's CPU-baseline leg may load it; the CUDA library never does,
+ * and this file shares no code, header, table or constant with it.
+ *
+ * What each function follows (pages cited by title and section):
+ *
+ *  - oracle_pack / oracle_unpack: the base-3 byte code of the Bonsai low-bit
+ *    course (adenzhou1350.github.io/learn/bonsai-low-bit), section
+ *    "先用五个数字理解 1.6bit": trit t in {-1,0,1} maps to digit t+1, five
+ *    digits form code = sum_i (t_i + 1) * 3^i with i = 0 the first trit, and
+ *    t_i = floor(code / 3^i) mod 3 - 1 restores them (example: [-1,0,1,-1,1]
+ *    -> 183). Groups of 128 weights along K (one FP16 scale each, "g128",
+ *    Ternary Bonsai 2 27B release summary, section 三值权重怎么压缩到 1.76
+ *    bit) are packed as 26 bytes: 25 full bytes plus one byte holding the
+ *    group's last 3 trits and two zero-valued pad trits (digit 1).
+ *    The plain 2-bit layout stores digit t+1 in bits [2i, 2i+1] of byte
+ *    i/4, 32 bytes per group; digit 3 is invalid.
+ *
+ *  - oracle_hadamard: H[i][j] = (-1)^popcount(i & j), the closed form of the
+ *    Sylvester recursion H_2n = [[H, H], [H, -H]] printed (with H4) in the
+ *    TensorSharp blog (2kiu.com/news/5337570), section 3.2.
+ *
+ *  - oracle_rotate_matrix: x'_b = (1/sqrt(1024)) * H_1024 * (S . x_b) for every
+ *    1024-long block b of each row, R = (1/sqrt n) H_n S from the release
+ *    summary, section 三值权重怎么压缩到 1.76 bit ("f(x) = W(Rx)").
+ *    Explicit matrix-vector product, O(n^2) per block.
+ *
+ *  - oracle_rotate_butterfly: the same rotation by the in-place butterfly
+ *    (pairs (a, b) -> (a + b, a - b) at half-widths 1, 2, ..., n/2, then
+ *    divide by sqrt n), as described in the TensorSharp blog, section 5.2.
+ *    It exists so large inputs finish; tests tie it to the matrix form.
+ *
+ *  - oracle_gemv: y[m][n] = sum_k w[n][k] * x'[m][k] with
+ *    w[n][k] = scale[n][k/128] * t[n][k] (dense dequantisation, FP64), and the
+ *    acceptance bound B[m][n] = 2e-3 * sum_k |w[n][k] x'[m][k]| + 1e-5.
+ *    Naive triple loop.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORACLE_GROUP 128
+#define ORACLE_BLOCK 1024
+
+enum { ORACLE_LAYOUT_BASE3 = 0, ORACLE_LAYOUT_2BIT = 1 };
+
+enum {
+    ORACLE_OK = 0,
+    ORACLE_BAD_SHAPE = 1,
+    ORACLE_BAD_TRIT = 2,
+    ORACLE_BAD_CODE = 3,
+    ORACLE_BAD_PAD = 4,
+    ORACLE_BAD_LAYOUT = 5
+};
+
+int oracle_bytes_per_group(int layout)
+{
+    if (layout == ORACLE_LAYOUT_BASE3) return 26;
+    if (layout == ORACLE_LAYOUT_2BIT) return 32;
+    return -1;
+}
+
+/* ---- scalar conversions (bit patterns -> double) ---- */
+
+double oracle_f16_to_double(uint16_t h)
+{
+    int sign = (h >> 15) & 1;
+    int expo = (h >> 10) & 0x1f;
+    int mant = h & 0x3ff;
+    double v;
+    if (expo == 0) {
+        v = ldexp((double)mant, -24);              /* subnormal: mant * 2^-24 */
+    } else if (expo == 31) {
+        v = mant ? NAN : INFINITY;
+    } else {
+        v = ldexp((double)(1024 + mant), expo - 25); /* (1 + mant/1024) 2^(e-15) */
+    }
+    return sign ? -v : v;
+}
+
+double oracle_bf16_to_double(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return (double)f;
+}
+
+void oracle_f16_array_to_double(const uint16_t* h, int64_t n, double* out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_f16_to_double(h[i]);
+}
+
+void oracle_bf16_array_to_double(const uint16_t* b, int64_t n, double* out)
+{
+    for (int64_t i = 0; i < n; ++i) out[i] = oracle_bf16_to_double(b[i]);
+}
+
+/* ---- packing ---- */
+
+static int pow3(int i)
+{
+    int p = 1;
+    while (i-- > 0) p *= 3;
+    return p;
+}
+
+int oracle_pack(int layout, const int8_t* trits, int64_t N, int64_t K, uint8_t* codes)
+{
+    if (K % ORACLE_GROUP != 0 || N < 0 || K < 0) return ORACLE_BAD_SHAPE;
+    int bpg = oracle_bytes_per_group(layout);
+    if (bpg < 0) return ORACLE_BAD_LAYOUT;
+    int64_t groups = K / ORACLE_GROUP;
+    for (int64_t i = 0; i < N * K; ++i)
+        if (trits[i] < -1 || trits[i] > 1) return ORACLE_BAD_TRIT;
+
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t g = 0; g < groups; ++g) {
+            const int8_t* t = trits + n * K + g * ORACLE_GROUP;
+            uint8_t* out = codes + (n * groups + g) * bpg;
+            if (layout == ORACLE_LAYOUT_BASE3) {
+                /* byte b holds trits 5b .. 5b+4; positions past 127 are pads (trit 0) */
+                for (int b = 0; b < 26; ++b) {
+                    int code = 0;
+                    for (int i = 0; i < 5; ++i) {
+                        int k = 5 * b + i;
+                        int trit = (k < ORACLE_GROUP) ? t[k] : 0;
+                        code += (trit + 1) * pow3(i);
+                    }
+                    out[b] = (uint8_t)code;
+                }
+            } else {
+                for (int b = 0; b < 32; ++b) {
+                    int code = 0;
+                    for (int i = 0; i < 4; ++i) code |= (t[4 * b + i] + 1) << (2 * i);
+                    out[b] = (uint8_t)code;
+                }
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+int oracle_unpack(int layout, const uint8_t* codes, int64_t N, int64_t K, int8_t* trits)
+{
+    if (K % ORACLE_GROUP != 0 || N < 0 || K < 0) return ORACLE_BAD_SHAPE;
+    int bpg = oracle_bytes_per_group(layout);
+    if (bpg < 0) return ORACLE_BAD_LAYOUT;
+    int64_t groups = K / ORACLE_GROUP;
+    for (int64_t n = 0; n < N; ++n) {
+        for (int64_t g = 0; g < groups; ++g) {
+            const uint8_t* in = codes + (n * groups + g) * bpg;
+            int8_t* t = trits + n * K + g * ORACLE_GROUP;
+            if (layout == ORACLE_LAYOUT_BASE3) {
+                for (int b = 0; b < 26; ++b) {
+                    int code = in[b];
+                    if (code >= 243) return ORACLE_BAD_CODE;
+                    for (int i = 0; i < 5; ++i) {
+                        int digit = (code / pow3(i)) % 3;
+                        int k = 5 * b + i;
+                        if (k < ORACLE_GROUP) t[k] = (int8_t)(digit - 1);
+                        else if (digit != 1) return ORACLE_BAD_PAD;
+                    }
+                }
+            } else {
+                for (int b = 0; b < 32; ++b) {
+                    for (int i = 0; i < 4; ++i) {
+                        int digit = (in[b] >> (2 * i)) & 3;
+                        if (digit == 3) return ORACLE_BAD_CODE;
+                        t[4 * b + i] = (int8_t)(digit - 1);
+                    }
+                }
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ---- Hadamard and the rotation R = (1/sqrt n) H_n S ---- */
+
+static int parity_of_and(int64_t i, int64_t j)
+{
+    uint64_t v = (uint64_t)(i & j);
+    int p = 0;
+    while (v) { p ^= 1; v &= v - 1; }
+    return p;
+}
+
+/* H[i][j] = (-1)^popcount(i & j), n a power of two (n x n, int8, row-major). */
+int oracle_hadamard(int64_t n, int8_t* H)
+{
+    if (n < 1 || (n & (n - 1)) != 0) return ORACLE_BAD_SHAPE;
+    for (int64_t i = 0; i < n; ++i)
+        for (int64_t j = 0; j < n; ++j) H[i * n + j] = parity_of_and(i, j) ? -1 : 1;
+    return ORACLE_OK;
+}
+
+/* Explicit matrix form: xr[m][b*n + i] = (1/sqrt n) sum_j H[i][j] S[j] x[m][b*n + j]. */
+int oracle_rotate_matrix(const double* x, const int8_t* S, int64_t M, int64_t K, double* xr)
+{
+    const int64_t n = ORACLE_BLOCK;
+    if (K % n != 0 || M < 0) return ORACLE_BAD_SHAPE;
+    int8_t* H = (int8_t*)malloc((size_t)(n * n));
+    if (!H) return ORACLE_BAD_SHAPE;
+    oracle_hadamard(n, H);
+    const double inv_sqrt_n = 1.0 / sqrt((double)n);
+    int64_t nblocks = K / n;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t b = 0; b < nblocks; ++b) {
+            const double* xb = x + m * K + b * n;
+            double* ob = xr + m * K + b * n;
+            for (int64_t i = 0; i < n; ++i) {
+                double acc = 0.0;
+                for (int64_t j = 0; j < n; ++j) acc += (double)H[i * n + j] * ((double)S[j] * xb[j]);
+                ob[i] = acc * inv_sqrt_n;
+            }
+        }
+    }
+    free(H);
+    return ORACLE_OK;
+}
+
+/* Butterfly form of the same rotation. */
+int oracle_rotate_butterfly(const double* x, const int8_t* S, int64_t M, int64_t K, double* xr)
+{
+    const int64_t n = ORACLE_BLOCK;
+    if (K % n != 0 || M < 0) return ORACLE_BAD_SHAPE;
+    const double inv_sqrt_n = 1.0 / sqrt((double)n);
+    int64_t nblocks = K / n;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t b = 0; b < nblocks; ++b) {
+            double v[ORACLE_BLOCK];
+            const double* xb = x + m * K + b * n;
+            for (int64_t j = 0; j < n; ++j) v[j] = (double)S[j] * xb[j];
+            for (int64_t half = 1; half < n; half *= 2) {
+                for (int64_t start = 0; start < n; start += 2 * half) {
+                    for (int64_t j = start; j < start + half; ++j) {
+                        double a = v[j], c = v[j + half];
+                        v[j] = a + c;
+                        v[j + half] = a - c;
+                    }
+                }
+            }
+            double* ob = xr + m * K + b * n;
+            for (int64_t j = 0; j < n; ++j) ob[j] = v[j] * inv_sqrt_n;
+        }
+    }
+    return ORACLE_OK;
+}
+
+/* ---- dequantisation and the product ---- */
+
+int oracle_dequant(const int8_t* trits, const uint16_t* scales, int64_t N, int64_t K, double* W)
+{
+    if (K % ORACLE_GROUP != 0) return ORACLE_BAD_SHAPE;
+    int64_t groups = K / ORACLE_GROUP;
+    for (int64_t n = 0; n < N; ++n)
+        for (int64_t k = 0; k < K; ++k)
+            W[n * K + k] = oracle_f16_to_double(scales[n * groups + k / ORACLE_GROUP]) * (double)trits[n * K + k];
+    return ORACLE_OK;
+}
+
+/*
+ * y[m][n] = sum_k w[n][k] xr[m][k]; bound[m][n] = 2e-3 sum_k |w[n][k] xr[m][k]| + 1e-5.
+ * trits int8 [N][K], scales fp16 bits [N][K/128], xr double [M][K], y/bound double [M][N].
+ * bound may be NULL.
+ */
+int oracle_gemv(const int8_t* trits, const uint16_t* scales, const double* xr,
+                int64_t M, int64_t N, int64_t K, double* y, double* bound)
+{
+    if (K % ORACLE_GROUP != 0) return ORACLE_BAD_SHAPE;
+    int64_t groups = K / ORACLE_GROUP;
+#pragma omp parallel for collapse(2) schedule(static)
+    for (int64_t m = 0; m < M; ++m) {
+        for (int64_t n = 0; n < N; ++n) {
+            double acc = 0.0, mag = 0.0;
+            for (int64_t k = 0; k < K; ++k) {
+                double w = oracle_f16_to_double(scales[n * groups + k / ORACLE_GROUP]) * (double)trits[n * K + k];
+                double p = w * xr[m * K + k];
+                acc += p;
+                mag += fabs(p);
+            }
+            y[m * N + n] = acc;
+            if (bound) bound[m * N + n] = 2e-3 * mag + 1e-5;
+        }
+    }
+    return ORACLE_OK;
+}
+
+int oracle_threads(void)
+{
+#ifdef _OPENMP
+    extern int omp_get_max_threads(void);
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
