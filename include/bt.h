@@ -1,0 +1,162 @@
+/*
+ * bt.h -- C ABI of libbt.so: ternary-weight GEMV/GEMM behind a block-wise
+ * Walsh-Hadamard activation rotation, for NVIDIA B200 (sm_100a).
+ *
+ * The path computes y = W (R x). R = (1/sqrt(1024)) H_1024 S is applied to
+ * every 1024-long block of each activation row: H_1024 is the Walsh-Hadamard
+ * matrix in Sylvester (natural) order, S a fixed +-1 diagonal. W holds trits
+ * t in {-1, 0, +1} and one FP16 scale per 128 consecutive weights of a row
+ * (g128), w = s * t. Sources: the Ternary Bonsai 2 27B release summary
+ * (linlog.top/article/1481), section 三值权重怎么压缩到 1.76 bit, for R,
+ * g128 and f(x) = W(Rx); the Bonsai low-bit course
+ * (adenzhou1350.github.io/learn/bonsai-low-bit), section
+ * 先用五个数字理解 1.6bit, for the base-3 byte code; the TensorSharp blog
+ * (2kiu.com/news/5337570), section 3.2, for the Hadamard ordering (H4).
+ *
+ * Conventions shared by every entry point
+ *  - Pointers marked "device" are CUDA device memory owned by the caller.
+ *    The library never allocates, frees or synchronises, and keeps no
+ *    mutable global state.
+ *  - Work is enqueued on `stream` (a cudaStream_t passed as void*; NULL is
+ *    the legacy default stream) and runs asynchronously.
+ *  - Arguments are validated on the host before anything is launched; a
+ *    non-zero bt_status means nothing was enqueued (except BT_ERR_CUDA,
+ *    returned when a launch itself failed).
+ *  - Errors found on the device are OR-ed into the caller's int32 word
+ *    `dev_err` (device memory, nullable) as BT_DEVERR_* bits. Kernels never
+ *    trap and never spin without a bound.
+ *  - Row-major everywhere. Activations are [M][K], outputs [M][N], trits
+ *    [N][K], codes [N][row bytes], scales [N][K/128] as FP16 bit patterns.
+ *  - Reentrant; calls on one stream are ordered, calls on different streams
+ *    must not share a workspace.
+ */
+#ifndef BT_H
+#define BT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    BT_OK = 0,
+    BT_ERR_INVALID_ARG = 1,   /* NULL pointer, bad enum value            */
+    BT_ERR_SHAPE = 2,         /* size constraint violated                */
+    BT_ERR_ALIGN = 3,         /* pointer not aligned as required         */
+    BT_ERR_WORKSPACE = 4,     /* workspace missing or too small          */
+    BT_ERR_UNSUPPORTED = 5,   /* valid request this build does not serve */
+    BT_ERR_CUDA = 6           /* a CUDA launch or query failed           */
+} bt_status;
+
+/* Bits OR-ed into *dev_err by kernels. */
+#define BT_DEVERR_INVALID_TRIT 0x1   /* bt_pack: a trit outside {-1,0,1}           */
+#define BT_DEVERR_INVALID_CODE 0x2   /* base-3 byte >= 243, or 2-bit field == 3    */
+#define BT_DEVERR_INVALID_PAD  0x4   /* bt_unpack: a pad trit of a base-3 group != 0 */
+#define BT_DEVERR_TIMEOUT      0x8   /* a bounded pipeline wait gave up            */
+
+typedef enum {
+    /* Base-3, 5 trits per byte, code = sum_i (t_i + 1) 3^i with trit i at the
+     * lower k. Per row and per group of 128 weights: 25 full bytes, then one
+     * byte with the group's last 3 trits and two pad trits of value 0
+     * (digit 1), so the last byte is in [108, 134]. 26 bytes per group. */
+    BT_LAYOUT_B3 = 0,
+    /* Plain 2 bits per trit: digit t + 1 in bits [2i, 2i+1] of byte i/4 (4
+     * trits per byte, lowest k in the low bits); 32 bytes per group. */
+    BT_LAYOUT_2BIT = 1
+} bt_layout;
+
+typedef enum { BT_F32 = 0, BT_BF16 = 1 } bt_dtype;
+
+const char* bt_status_string(int status);
+int bt_version(void);
+
+/* Bytes of one packed row: K/128 * 26 (base-3) or K/128 * 32 (2-bit).
+ * -1 if K is not a positive multiple of 128 or layout is unknown. Every
+ * packed row is therefore a multiple of 2 bytes (base-3) or 32 bytes. */
+int64_t bt_codes_row_bytes(int layout, int64_t K);
+
+/*
+ * bt_pack: trits (device, int8 [N][K]) -> codes (device, uint8
+ * [N][bt_codes_row_bytes]). K % 128 == 0, N >= 0. Every byte of `codes` is
+ * written. A trit outside {-1,0,1} is packed as 0 and sets
+ * BT_DEVERR_INVALID_TRIT. Source: base-3 byte code, Bonsai low-bit course,
+ * section 先用五个数字理解 1.6bit; group of 128 and FP16 scale, release
+ * summary, section 三值权重怎么压缩到 1.76 bit.
+ */
+bt_status bt_pack(int layout, const int8_t* trits, int64_t N, int64_t K,
+                  uint8_t* codes, int32_t* dev_err, void* stream);
+
+/*
+ * bt_unpack: inverse of bt_pack (device in, device out). Invalid codes set
+ * BT_DEVERR_INVALID_CODE and decode as zeros; a non-zero base-3 pad trit
+ * sets BT_DEVERR_INVALID_PAD. A test and debug helper.
+ */
+bt_status bt_unpack(int layout, const uint8_t* codes, int64_t N, int64_t K,
+                    int8_t* trits, int32_t* dev_err, void* stream);
+
+/*
+ * bt_fwht1024: x_rot = R x block-wise, R = (1/32) H_1024 S.
+ *  x_bf16    device, bf16 bit patterns [M][K], 16-byte aligned
+ *  sign1024  device, int8 [1024], every entry +1 or -1 (other values are
+ *            treated as +1 when >= 0 and -1 when < 0)
+ *  K % 1024 == 0, M >= 0
+ *  out_dtype BT_F32 (float [M][K]) or BT_BF16 (bf16 [M][K], round to
+ *            nearest even); x_rot 16-byte aligned, must not overlap x
+ * FP32 arithmetic; the 1/32 factor is exact. Source: release summary,
+ * section 三值权重怎么压缩到 1.76 bit (R, blockwise, n = 1024); butterfly as
+ * in the TensorSharp blog, section 5.2.
+ */
+bt_status bt_fwht1024(const uint16_t* x_bf16, const int8_t* sign1024, int64_t M, int64_t K,
+                      int out_dtype, void* x_rot, void* stream);
+
+/*
+ * bt_gemv: decode path, y[m][n] = sum_g s[n][g] sum_{k in g} t[n][k] x'[m][k],
+ * 1 <= M <= 16.
+ *  layout    BT_LAYOUT_B3 or BT_LAYOUT_2BIT
+ *  codes     device [N][bt_codes_row_bytes(layout, K)], 16-byte aligned
+ *  scales    device fp16 bits [N][K/128], 4-byte aligned
+ *  x         device [M][K]. If sign1024 != NULL, x is the raw activation in
+ *            bf16 (x_dtype must be BT_BF16) and the rotation is applied
+ *            first (K % 1024 == 0). If sign1024 == NULL, x is already
+ *            rotated, in x_dtype (BT_F32 or BT_BF16), K % 128 == 0.
+ *  y         device [M][N] in y_dtype (BT_F32 or BT_BF16), 16-byte aligned
+ *  workspace device, >= bt_gemv_workspace_bytes(...), 256-byte aligned.
+ *            Scratch only; its contents need no initialisation and are
+ *            meaningless after the call.
+ *  dev_err   nullable; invalid codes set BT_DEVERR_INVALID_CODE (their
+ *            contribution is then unspecified but finite).
+ * Numerics: the rotated activation feeds FP16 tensor-core products with FP32
+ * accumulation (one power-of-two exponent per 128 activations keeps it in
+ * range); y satisfies |y - y_exact| <= 2e-3 * sum_k |w x'| + 1e-5.
+ * Source: fused unpack and group scale inside the matrix product, release
+ * summary, section 三值权重怎么压缩到 1.76 bit.
+ */
+size_t bt_gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K);
+bt_status bt_gemv(int layout, const uint8_t* codes, const uint16_t* scales,
+                  const void* x, int x_dtype, const int8_t* sign1024,
+                  int64_t M, int64_t N, int64_t K, int y_dtype, void* y,
+                  void* workspace, size_t workspace_bytes, int32_t* dev_err, void* stream);
+
+/*
+ * bt_gemm: prefill path, Y = X' W^T with W = s * t decoded into FP16 tiles
+ * in shared memory and multiplied on the tcgen05 tensor cores, FP32
+ * accumulation, bf16 output [M][N] (round to nearest even).
+ *  M % 128 == 0, N % 128 == 0, K % 128 == 0 (K % 1024 == 0 when rotating).
+ *  Arguments as for bt_gemv (y is bf16). The rotated activation is rounded
+ *  to FP16 after scaling each row by a power of two chosen from its largest
+ *  magnitude.
+ * Source: pp512 prompt processing, release summary, section 实测吞吐.
+ */
+size_t bt_gemm_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K);
+bt_status bt_gemm(int layout, const uint8_t* codes, const uint16_t* scales,
+                  const void* x, int x_dtype, const int8_t* sign1024,
+                  int64_t M, int64_t N, int64_t K, void* y_bf16,
+                  void* workspace, size_t workspace_bytes, int32_t* dev_err, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BT_H */

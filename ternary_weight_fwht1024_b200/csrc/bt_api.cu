@@ -1,0 +1,177 @@
+// C ABI of libbt.so: host-side validation and dispatch (declared in include/bt.h).
+#include "bt_internal.cuh"
+
+namespace bt {
+cudaError_t launch_pack(int layout, const int8_t* trits, int64_t N, int64_t K, uint8_t* codes,
+                        int32_t* dev_err, cudaStream_t stream);
+cudaError_t launch_unpack(int layout, const uint8_t* codes, int64_t N, int64_t K, int8_t* trits,
+                          int32_t* dev_err, cudaStream_t stream);
+cudaError_t launch_fwht1024(const uint16_t* x, const int8_t* sign, int64_t M, int64_t K,
+                            int out_dtype, void* out, int num_sms, cudaStream_t stream);
+size_t gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num_sms);
+cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales, const void* x,
+                        int x_dtype, const int8_t* sign, int64_t M, int64_t N, int64_t K, int y_dtype,
+                        void* y, void* workspace, int32_t* dev_err, int num_sms, cudaStream_t stream);
+size_t gemm_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num_sms);
+cudaError_t launch_gemm(int layout, const uint8_t* codes, const uint16_t* scales, const void* x,
+                        int x_dtype, const int8_t* sign, int64_t M, int64_t N, int64_t K, void* y,
+                        void* workspace, int32_t* dev_err, int num_sms, cudaStream_t stream);
+}  // namespace bt
+
+namespace {
+
+constexpr int kVersion = 1;
+constexpr int kDefaultSms = 148;   // B200; used when no device can be queried
+
+int current_sm_count() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return kDefaultSms; }
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+        cudaGetLastError();
+        return kDefaultSms;
+    }
+    return sms;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+bool valid_layout(int layout) { return layout == BT_LAYOUT_B3 || layout == BT_LAYOUT_2BIT; }
+bool valid_dtype(int d) { return d == BT_F32 || d == BT_BF16; }
+int64_t group_bytes(int layout) { return layout == BT_LAYOUT_B3 ? 26 : 32; }
+
+bt_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BT_OK : BT_ERR_CUDA; }
+
+// Shared validation of the product entry points.
+bt_status check_product_args(int layout, const uint8_t* codes, const uint16_t* scales, const void* x,
+                             int x_dtype, const int8_t* sign, int64_t M, int64_t N, int64_t K,
+                             const void* y) {
+    if (!valid_layout(layout) || !valid_dtype(x_dtype)) return BT_ERR_INVALID_ARG;
+    if (M < 0 || N < 0 || K < 0) return BT_ERR_SHAPE;
+    if (K % 128 != 0) return BT_ERR_SHAPE;
+    if (sign && (K % 1024 != 0 || x_dtype != BT_BF16)) return sign && x_dtype != BT_BF16 ? BT_ERR_INVALID_ARG : BT_ERR_SHAPE;
+    if (K > (int64_t(1) << 30) || N > (int64_t(1) << 30)) return BT_ERR_SHAPE;
+    if (M == 0 || N == 0) return BT_OK;
+    if (!y) return BT_ERR_INVALID_ARG;
+    if (K > 0 && (!codes || !scales || !x)) return BT_ERR_INVALID_ARG;
+    if (!aligned(codes, 16) || !aligned(scales, 4) || !aligned(x, 16) || !aligned(y, 16) || !aligned(sign, 16))
+        return BT_ERR_ALIGN;
+    return BT_OK;
+}
+
+// y = 0 for K = 0 (the empty sum)
+__global__ void zero_kernel(uint8_t* p, int64_t bytes) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < bytes; i += (int64_t)gridDim.x * blockDim.x)
+        p[i] = 0;
+}
+
+cudaError_t launch_zero(void* p, int64_t bytes, cudaStream_t s) {
+    if (bytes <= 0) return cudaSuccess;
+    int blocks = static_cast<int>((bytes + 255) / 256);
+    if (blocks > 1024) blocks = 1024;
+    zero_kernel<<<blocks, 256, 0, s>>>(static_cast<uint8_t*>(p), bytes);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* bt_status_string(int status) {
+    switch (status) {
+        case BT_OK: return "ok";
+        case BT_ERR_INVALID_ARG: return "invalid argument (NULL pointer or bad enum)";
+        case BT_ERR_SHAPE: return "shape constraint violated";
+        case BT_ERR_ALIGN: return "pointer misaligned";
+        case BT_ERR_WORKSPACE: return "workspace missing or too small";
+        case BT_ERR_UNSUPPORTED: return "unsupported request";
+        case BT_ERR_CUDA: return "CUDA launch or query failed";
+        default: return "unknown status";
+    }
+}
+
+int bt_version(void) { return kVersion; }
+
+int64_t bt_codes_row_bytes(int layout, int64_t K) {
+    if (!valid_layout(layout) || K <= 0 || K % 128 != 0) return -1;
+    return (K / 128) * group_bytes(layout);
+}
+
+bt_status bt_pack(int layout, const int8_t* trits, int64_t N, int64_t K, uint8_t* codes,
+                  int32_t* dev_err, void* stream) {
+    if (!valid_layout(layout)) return BT_ERR_INVALID_ARG;
+    if (N < 0 || K < 0 || K % 128 != 0) return BT_ERR_SHAPE;
+    if (N == 0 || K == 0) return BT_OK;
+    if (!trits || !codes) return BT_ERR_INVALID_ARG;
+    if (!aligned(trits, 4) || !aligned(dev_err, 4)) return BT_ERR_ALIGN;
+    return from_cuda(bt::launch_pack(layout, trits, N, K, codes, dev_err, static_cast<cudaStream_t>(stream)));
+}
+
+bt_status bt_unpack(int layout, const uint8_t* codes, int64_t N, int64_t K, int8_t* trits,
+                    int32_t* dev_err, void* stream) {
+    if (!valid_layout(layout)) return BT_ERR_INVALID_ARG;
+    if (N < 0 || K < 0 || K % 128 != 0) return BT_ERR_SHAPE;
+    if (N == 0 || K == 0) return BT_OK;
+    if (!trits || !codes) return BT_ERR_INVALID_ARG;
+    if (!aligned(trits, 4) || !aligned(dev_err, 4)) return BT_ERR_ALIGN;
+    return from_cuda(bt::launch_unpack(layout, codes, N, K, trits, dev_err, static_cast<cudaStream_t>(stream)));
+}
+
+bt_status bt_fwht1024(const uint16_t* x_bf16, const int8_t* sign1024, int64_t M, int64_t K,
+                      int out_dtype, void* x_rot, void* stream) {
+    if (!valid_dtype(out_dtype)) return BT_ERR_INVALID_ARG;
+    if (M < 0 || K < 0 || K % 1024 != 0) return BT_ERR_SHAPE;
+    if (M == 0 || K == 0) return BT_OK;
+    if (!x_bf16 || !sign1024 || !x_rot) return BT_ERR_INVALID_ARG;
+    if (!aligned(x_bf16, 16) || !aligned(sign1024, 16) || !aligned(x_rot, 16)) return BT_ERR_ALIGN;
+    return from_cuda(bt::launch_fwht1024(x_bf16, sign1024, M, K, out_dtype, x_rot, current_sm_count(),
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+size_t bt_gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K) {
+    if (!valid_layout(layout) || M < 1 || M > 16 || N < 1 || K < 128 || K % 128 != 0) return 0;
+    return bt::gemv_workspace_bytes(layout, M, N, K, current_sm_count());
+}
+
+bt_status bt_gemv(int layout, const uint8_t* codes, const uint16_t* scales, const void* x, int x_dtype,
+                  const int8_t* sign1024, int64_t M, int64_t N, int64_t K, int y_dtype, void* y,
+                  void* workspace, size_t workspace_bytes, int32_t* dev_err, void* stream) {
+    bt_status st = check_product_args(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y);
+    if (st != BT_OK) return st;
+    if (!valid_dtype(y_dtype)) return BT_ERR_INVALID_ARG;
+    if (M > 16) return BT_ERR_SHAPE;
+    if (M == 0 || N == 0) return BT_OK;
+    if (!aligned(dev_err, 4)) return BT_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (K == 0) return from_cuda(launch_zero(y, M * N * (y_dtype == BT_BF16 ? 2 : 4), s));
+    const int sms = current_sm_count();
+    const size_t need = bt::gemv_workspace_bytes(layout, M, N, K, sms);
+    if (!workspace || workspace_bytes < need) return BT_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return BT_ERR_ALIGN;
+    return from_cuda(bt::launch_gemv(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y_dtype, y,
+                                     workspace, dev_err, sms, s));
+}
+
+size_t bt_gemm_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K) {
+    if (!valid_layout(layout) || M < 128 || M % 128 != 0 || N < 128 || N % 128 != 0 || K < 128 || K % 128 != 0)
+        return 0;
+    return bt::gemm_workspace_bytes(layout, M, N, K, current_sm_count());
+}
+
+bt_status bt_gemm(int layout, const uint8_t* codes, const uint16_t* scales, const void* x, int x_dtype,
+                  const int8_t* sign1024, int64_t M, int64_t N, int64_t K, void* y_bf16,
+                  void* workspace, size_t workspace_bytes, int32_t* dev_err, void* stream) {
+    bt_status st = check_product_args(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y_bf16);
+    if (st != BT_OK) return st;
+    if (M == 0 || N == 0) return BT_OK;
+    if (M % 128 != 0 || N % 128 != 0) return BT_ERR_SHAPE;
+    if (!aligned(dev_err, 4)) return BT_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (K == 0) return from_cuda(launch_zero(y_bf16, M * N * 2, s));
+    const int sms = current_sm_count();
+    const size_t need = bt::gemm_workspace_bytes(layout, M, N, K, sms);
+    if (!workspace || workspace_bytes < need) return BT_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return BT_ERR_ALIGN;
+    return from_cuda(bt::launch_gemm(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y_bf16,
+                                     workspace, dev_err, sms, s));
+}
+
+}  // extern "C"

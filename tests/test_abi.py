@@ -1,0 +1,119 @@
+"""The C ABI on the host: libbt.so loads, exports every entry point that
+include/bt.h declares, and rejects bad arguments before launching anything.
+No GPU is needed: every call below fails host-side validation."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import ternary_weight_fwht1024_b200 as bt
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    import __graft_entry__
+    __graft_entry__.build()
+    return bt.load()
+
+
+def _declared_functions():
+    text = open(os.path.join(ROOT, "include", "bt.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(bt_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_binding_symbols():
+    assert _declared_functions() == sorted(bt.SYMBOLS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_version_and_status_strings(lib):
+    assert lib.bt_version() >= 1
+    assert bt.status_string(0) == "ok"
+    for s in range(1, 7):
+        assert bt.status_string(s) != "unknown status"
+    assert bt.status_string(99) == "unknown status"
+
+
+def test_codes_row_bytes(lib):
+    assert bt.codes_row_bytes(bt.LAYOUT_B3, 1024) == 208
+    assert bt.codes_row_bytes(bt.LAYOUT_B3, 5120) == 1040
+    assert bt.codes_row_bytes(bt.LAYOUT_B3, 17408) == 3536
+    assert bt.codes_row_bytes(bt.LAYOUT_2BIT, 5120) == 1280
+    assert bt.codes_row_bytes(bt.LAYOUT_B3, 100) == -1
+    assert bt.codes_row_bytes(bt.LAYOUT_B3, 0) == -1
+    assert bt.codes_row_bytes(5, 1024) == -1
+
+
+P = ctypes.c_void_p
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def test_pack_validation(lib):
+    good = _fake(1 << 20)
+    assert lib.bt_pack(7, good, 4, 128, good, None, None) == 1          # bad layout
+    assert lib.bt_pack(0, good, 4, 100, good, None, None) == 2          # K % 128
+    assert lib.bt_pack(0, good, -1, 128, good, None, None) == 2         # N < 0
+    assert lib.bt_pack(0, None, 4, 128, good, None, None) == 1          # NULL
+    assert lib.bt_pack(0, _fake((1 << 20) + 1), 4, 128, good, None, None) == 3  # align
+    assert lib.bt_pack(0, None, 0, 128, None, None, None) == 0          # empty: no-op
+
+
+def test_fwht_validation(lib):
+    good = _fake(1 << 20)
+    assert lib.bt_fwht1024(good, good, 1, 1000, 0, good, None) == 2
+    assert lib.bt_fwht1024(good, good, 1, 1024, 5, good, None) == 1
+    assert lib.bt_fwht1024(None, good, 1, 1024, 0, good, None) == 1
+    assert lib.bt_fwht1024(_fake((1 << 20) + 8), good, 1, 1024, 0, good, None) == 3
+    assert lib.bt_fwht1024(good, good, 0, 1024, 0, good, None) == 0
+
+
+def test_gemv_validation(lib):
+    g = _fake(1 << 20)
+    args = lambda **kw: [kw.get("layout", 0), g, g, g, kw.get("xd", 1), kw.get("sign", g),
+                         kw.get("M", 1), kw.get("N", 256), kw.get("K", 1024), kw.get("yd", 0),
+                         kw.get("y", g), kw.get("ws", None), kw.get("wsb", 0), None, None]
+    assert lib.bt_gemv(*args(layout=3)) == 1
+    assert lib.bt_gemv(*args(M=17)) == 2
+    assert lib.bt_gemv(*args(K=1000)) == 2
+    assert lib.bt_gemv(*args(K=1152)) == 2            # rotation needs K % 1024
+    assert lib.bt_gemv(*args(xd=0)) == 1              # raw activations must be bf16
+    assert lib.bt_gemv(*args(yd=4)) == 1
+    assert lib.bt_gemv(*args(y=None)) == 1
+    assert lib.bt_gemv(*args(y=_fake((1 << 20) + 4))) == 3
+    assert lib.bt_gemv(*args()) == 4                  # no workspace
+    need = lib.bt_gemv_workspace_bytes(0, 1, 256, 1024)
+    assert need > 0
+    assert lib.bt_gemv(*args(ws=_fake(1 << 24), wsb=need - 1)) == 4
+    assert lib.bt_gemv(*args(ws=_fake((1 << 24) + 16), wsb=need)) == 3
+    assert lib.bt_gemv(*args(M=0)) == 0
+    assert lib.bt_gemv_workspace_bytes(0, 17, 256, 1024) == 0
+
+
+def test_gemm_validation(lib):
+    g = _fake(1 << 20)
+    args = lambda **kw: [kw.get("layout", 0), g, g, g, 1, g, kw.get("M", 512), kw.get("N", 5120),
+                         kw.get("K", 5120), g, kw.get("ws", None), kw.get("wsb", 0), None, None]
+    assert lib.bt_gemm(*args(M=100)) == 2
+    assert lib.bt_gemm(*args(N=1000)) == 2
+    assert lib.bt_gemm(*args(K=1000)) == 2
+    assert lib.bt_gemm(*args()) == 4
+    assert lib.bt_gemm_workspace_bytes(0, 512, 5120, 5120) > 0
+    assert lib.bt_gemm_workspace_bytes(0, 100, 5120, 5120) == 0
+
+
+def test_binding_refuses_cpu_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        bt.pack(torch.zeros((2, 128), dtype=torch.int8))
