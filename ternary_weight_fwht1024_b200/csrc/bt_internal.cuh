@@ -39,9 +39,9 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 }
 
 __device__ __forceinline__ uint32_t lop3_or_and(uint32_t a, uint32_t b, uint32_t m) {
-    // (a | b) & m in one LOP3
+    // (a | b) & m in one LOP3 (truth table: (0xF0 | 0xCC) & 0xAA = 0xA8)
     uint32_t r;
-    asm("lop3.b32 %0, %1, %2, %3, 0xE0;" : "=r"(r) : "r"(a), "r"(b), "r"(m));
+    asm("lop3.b32 %0, %1, %2, %3, 0xA8;" : "=r"(r) : "r"(a), "r"(b), "r"(m));
     return r;
 }
 
