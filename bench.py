@@ -1,0 +1,409 @@
+"""Benchmark: packed-ternary decode GEMV (with the FWHT-1024 rotation) on B200.
+
+One step = one decode token through the 5120x5120 / 5120x17408 / 17408x5120
+triple at M = 1: for each matrix, bt_gemv rotates the bf16 activation block-wise
+(R = H_1024 S / 32) and multiplies by the base-3 packed ternary weights with
+g128 FP16 scales. The weights are synthetic and seeded (the pages' 27B model
+is not available); twelve distinct copies of the triple (537 MB, over four
+times the 126 MB L2) are used in turn so every step streams from HBM.
+
+`value` = packed weight bytes (codes + scales) per step / device time per step.
+The same JSON line carries the prefill GEMM (pp512: M = 512 on the same
+triple) in TFLOP/s, the 2-bit layout twin, the end-to-end figure through the
+public API with host buffers, a roofline block and the CPU oracle baseline.
+
+`--impl reference` times the CPU oracle (the only reference this method has)
+on a bounded sample of the same workload and prints the same metric.
+Multi-GPU (`--gpus N` under torchrun): independent replicas, weak scaling.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "packed-ternary GEMV weight GB/s (% of HBM peak); pp512 GEMM TFLOP/s"
+L2_BYTES = 126 * 1024 * 1024
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d.get("hbm_gbs", 6545.0), "bf16_tflops": d.get("bf16_tflops", 1627.8),
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", 1395.0), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines: list[str] = []
+        self._t = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._t = threading.Thread(target=self._read, daemon=True)
+            self._t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------- inputs ---
+
+def _layer_tensors(bt, torch, dev, layout, idx, L, with_x=False):
+    import workloads
+    inp = workloads.layer_inputs("C1", L, index=idx, with_x=with_x)
+    codes = bt.pack(torch.from_numpy(inp["trits"]).to(dev), layout)
+    scales = torch.from_numpy(inp["scales"].view(np.int16)).to(dev)
+    return codes, scales, inp
+
+
+def _weight_bytes(L, layout):
+    per_group = (26 if layout == 0 else 32) + 2
+    return L.N * (L.K // 128) * per_group
+
+
+# ---------------------------------------------------------------- GPU arm ---
+
+def run_gpu(args, rank, world):
+    import torch
+    import torch.distributed as dist
+    import ternary_weight_fwht1024_b200 as bt
+    import workloads
+
+    dev = torch.device("cuda", int(os.environ.get("LOCAL_RANK", 0)))
+    torch.cuda.set_device(dev)
+    bt.load()
+    peaks = _peaks()
+    triple = workloads.TRIPLE
+    sign = torch.from_numpy(workloads.sign1024()).to(dev)
+    copies = max(4, math.ceil(4 * L2_BYTES / sum(_weight_bytes(L, 0) for L in triple)))
+
+    def build(layout):
+        base = [_layer_tensors(bt, torch, dev, layout, i, L)[:2] for i, L in enumerate(triple)]
+        reps = [[(c.clone(), s.clone()) for c, s in base] for _ in range(copies)]
+        del base
+        return reps
+
+    stream = torch.cuda.Stream(device=dev)
+    M = 1
+    g = workloads.rng(2 * 1_000_003 + 99)
+    xs_host = [torch.from_numpy(workloads.activations_bf16_bits(g, M, L.K, True).view(np.int16)).pin_memory()
+               for L in triple]
+    xs = [h.to(dev).view(torch.bfloat16) for h in xs_host]
+    ys = [torch.empty((M, L.N), dtype=torch.float32, device=dev) for L in triple]
+    ws = torch.empty(max(bt.gemv_workspace_bytes(l, M, L.N, L.K) for L in triple for l in (0, 1)),
+                     dtype=torch.uint8, device=dev)
+
+    def graphs_for(reps, layout, with_events=False):
+        gs = []
+        with torch.cuda.stream(stream):
+            for r in range(copies):
+                for i, L in enumerate(triple):  # warm the code path before capture
+                    bt.gemv(reps[r][i][0], reps[r][i][1], xs[i], sign, L.N, layout, out=ys[i], ws=ws)
+            torch.cuda.synchronize()
+            for r in range(copies):
+                gr = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gr, stream=stream):
+                    for i, L in enumerate(triple):
+                        bt.gemv(reps[r][i][0], reps[r][i][1], xs[i], sign, L.N, layout, out=ys[i], ws=ws)
+                gs.append(gr)
+        return gs
+
+    def timed(gs, steps, warmup, per_call_events=False):
+        with torch.cuda.stream(stream):
+            for w in range(warmup):
+                gs[w % copies].replay()
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            st = torch.cuda.Event(enable_timing=True)
+            en = torch.cuda.Event(enable_timing=True)
+            st.record(stream)
+            for k in range(steps):
+                gs[(warmup + k) % copies].replay()
+            en.record(stream)
+            torch.cuda.synchronize()
+        ms = st.elapsed_time(en) / steps
+        if world > 1:
+            t = torch.tensor([ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    # ---- base-3 (headline) ----
+    reps3 = build(0)
+    gs3 = graphs_for(reps3, 0)
+    with ClockSampler(dev.index) as clk:
+        time.sleep(0.5)  # let the sampler start before the timed region
+        ms3 = timed(gs3, args.steps, args.warmup)
+    bytes3 = sum(_weight_bytes(L, 0) for L in triple)
+    io_bytes = sum(M * L.K * 2 + M * L.N * 4 for L in triple)
+
+    # per-call durations of the dominant call (bt_gemv = prep + GEMV kernels)
+    per_layer_us = []
+    with torch.cuda.stream(stream):
+        for i, L in enumerate(triple):
+            evs = []
+            for r in range(copies):
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                bt.gemv(reps3[r][i][0], reps3[r][i][1], xs[i], sign, L.N, 0, out=ys[i], ws=ws)
+                b.record(stream)
+                evs.append((a, b))
+            torch.cuda.synchronize()
+            per_layer_us.append(float(np.mean([a.elapsed_time(b) for a, b in evs[2:]])) * 1e3)
+    del gs3
+
+    # ---- e2e through the public API with host buffers ----
+    y_host = [torch.empty((M, L.N), dtype=torch.float32).pin_memory() for L in triple]
+    with torch.cuda.stream(stream):
+        for w in range(args.warmup):
+            for i, L in enumerate(triple):
+                xs[i].view(torch.int16).copy_(xs_host[i], non_blocking=True)
+                bt.gemv(reps3[w % copies][i][0], reps3[w % copies][i][1], xs[i], sign, L.N, 0, out=ys[i], ws=ws)
+                y_host[i].copy_(ys[i], non_blocking=True)
+        torch.cuda.synchronize()
+        st = torch.cuda.Event(enable_timing=True)
+        en = torch.cuda.Event(enable_timing=True)
+        st.record(stream)
+        for k in range(args.steps):
+            r = (args.warmup + k) % copies
+            for i, L in enumerate(triple):
+                xs[i].view(torch.int16).copy_(xs_host[i], non_blocking=True)
+                bt.gemv(reps3[r][i][0], reps3[r][i][1], xs[i], sign, L.N, 0, out=ys[i], ws=ws)
+                y_host[i].copy_(ys[i], non_blocking=True)
+        en.record(stream)
+        torch.cuda.synchronize()
+    e2e_ms = st.elapsed_time(en) / args.steps
+    del reps3
+
+    # ---- 2-bit layout twin ----
+    reps2 = build(1)
+    gs2 = graphs_for(reps2, 1)
+    ms2 = timed(gs2, args.steps, args.warmup)
+    bytes2 = sum(_weight_bytes(L, 1) for L in triple)
+    del gs2, reps2
+
+    # ---- prefill GEMM pp512 ----
+    gemm = None
+    try:
+        Mg = 512
+        gm = [_layer_tensors(bt, torch, dev, 0, i, L)[:2] for i, L in enumerate(triple)]
+        Xs = [torch.randn((Mg, L.K), device=dev).to(torch.bfloat16) for L in triple]
+        Ys = [torch.empty((Mg, L.N), dtype=torch.bfloat16, device=dev) for L in triple]
+        wsg = torch.empty(max(bt.gemm_workspace_bytes(0, Mg, L.N, L.K) for L in triple), dtype=torch.uint8,
+                          device=dev)
+        with torch.cuda.stream(stream):
+            for i, L in enumerate(triple):
+                bt.gemm(gm[i][0], gm[i][1], Xs[i], sign, L.N, 0, out=Ys[i], ws=wsg)
+            torch.cuda.synchronize()
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                for i, L in enumerate(triple):
+                    bt.gemm(gm[i][0], gm[i][1], Xs[i], sign, L.N, 0, out=Ys[i], ws=wsg)
+            gms = timed([gr] * copies, args.steps, args.warmup)
+        flops = sum(2.0 * Mg * L.N * L.K for L in triple)
+        tf = flops / (gms * 1e-3) / 1e12
+        gemm = {"value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(gms, 4),
+                "workload": "pp512 triple, base-3", "frac_of_peak": round(tf / peaks["bf16_tflops"], 4),
+                "peak": peaks["bf16_tflops"], "peak_kind": f"bf16 burst, {peaks['src']}"}
+    except Exception as e:  # the prefill path is reported, not required for the headline
+        gemm = {"value": None, "error": str(e)[:200]}
+
+    gbs = bytes3 / (ms3 * 1e-3) / 1e9 * world
+    dom_bytes = [(_weight_bytes(L, 0) + M * L.K * 2 + M * L.N * 4) for L in triple]
+    achieved = sum(dom_bytes) / (sum(per_layer_us) * 1e-6) / 1e9
+    out = {
+        "metric": METRIC,
+        "value": round(gbs, 2),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms3, 5),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f16 tensor-core products of base-3 trits, f32 accumulate",
+        "data": "synthetic (seeded trits P(0)=0.4, g128 fp16 scales, bf16 activations with 0.1% x20 outliers)",
+        "config": {"workload": "decode GEMV M=1 on the 5120x5120 / 5120x17408 / 17408x5120 triple, base-3 g128, "
+                               "FWHT-1024 fused",
+                   "M": M, "layout": "base-3 5 trits/byte, 26 B + 2 B scale per 128 weights",
+                   "l2": f"{copies} distinct weight copies rotated ({copies * bytes3 / 1e6:.0f} MB > 126 MB L2)",
+                   "graph": "each step is one CUDA graph replay of three bt_gemv calls",
+                   "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
+        "pct_of_hbm_peak": round(100 * gbs / world / peaks["hbm_gbs"], 2),
+        "per_call_us": {L.name: round(u, 2) for L, u in zip(triple, per_layer_us)},
+        "layout_2bit": {"value": round(bytes2 / (ms2 * 1e-3) / 1e9 * world, 2), "unit": "GB/s",
+                        "ms_per_step": round(ms2, 5), "bytes_per_step": bytes2},
+        "tokens_per_s_triple": round(1e3 / ms3 * world, 1),
+        "gemm": gemm,
+        "e2e": {"value": round(bytes3 / (e2e_ms * 1e-3) / 1e9 * world, 2), "unit": "GB/s",
+                "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": sum(M * L.K * 2 for L in triple),
+                "d2h_bytes_per_step": sum(M * L.N * 4 for L in triple)},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": round(achieved / peaks["hbm_gbs"], 4),
+                     "traffic": None,
+                     "kernel": "bt_gemv call (gemv_prep + gemv kernels), average over the three layers",
+                     "peak_kind": f"HBM copy, {peaks['src']}"},
+        "gpu_launches": args.steps * len(triple) * 2,
+        "clocks": clk.summary(),
+    }
+    if rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    return out
+
+
+# ---------------------------------------------------------------- CPU arm ---
+
+def cpu_baseline(budget_s: float):
+    """The FP64 oracle (rotation + dense dequantise + naive matmul) on host cores,
+    on a bounded row sample of each decode matrix; GB/s of packed weights."""
+    import oracle
+    import workloads
+    oracle.build()
+    t_total, b_total, rows_done = 0.0, 0, []
+    for idx, L in enumerate(workloads.TRIPLE):
+        inp = workloads.layer_inputs("C1", L, index=idx)
+        xr = oracle.rotate_bf16(inp["x"], inp["sign"])
+        t0 = time.perf_counter()
+        oracle.gemv(inp["trits"][:32], inp["scales"][:32], xr)        # calibration
+        per_row = (time.perf_counter() - t0) / 32
+        rows = int(min(L.N, max(32, budget_s / 3.0 / max(per_row, 1e-9))))
+        t0 = time.perf_counter()
+        oracle.gemv(inp["trits"][:rows], inp["scales"][:rows], xr)
+        t_total += time.perf_counter() - t0
+        b_total += _weight_bytes(workloads.Layer(L.name, L.K, rows), 0)
+        rows_done.append(f"{L.name}:{rows}/{L.N} rows")
+    return {"value": round(b_total / t_total / 1e9, 4), "unit": "GB/s", "cores": oracle.threads(),
+            "kind": "oracle", "sample": "decode triple M=1 incl. rotation of x, " + ", ".join(rows_done)
+            + f", {t_total:.1f} s"}
+
+
+def run_reference(args):
+    """The CPU oracle as the reference arm, on the same metric and workload."""
+    import oracle
+    import workloads
+    oracle.build()
+    triple = workloads.TRIPLE
+    inputs = [workloads.layer_inputs("C1", L, index=i) for i, L in enumerate(triple)]
+    budget_rows = [L.N for L in triple]  # the oracle covers the whole triple in about a second
+    def step():
+        b = 0
+        for inp, L, r in zip(inputs, triple, budget_rows):
+            xr = oracle.rotate_bf16(inp["x"], inp["sign"])
+            oracle.gemv(inp["trits"][:r], inp["scales"][:r], xr)
+            b += _weight_bytes(workloads.Layer(L.name, L.K, r), 0)
+        return b
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    tot = 0
+    for _ in range(args.steps):
+        tot += step()
+    dt = time.perf_counter() - t0
+    v = tot / dt / 1e9
+    sample = "decode triple M=1, " + ", ".join(f"{L.name}:{r}/{L.N} rows" for L, r in zip(triple, budget_rows))
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": "decode GEMV M=1 on the 5120x5120 / 5120x17408 / 17408x5120 triple, base-3 g128, "
+                               "FWHT-1024 fused", "M": 1},
+        "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": oracle.threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        out = run_gpu(args, rank, world)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -8,37 +8,47 @@
 //
 // Two kernels, chained with programmatic dependent launch:
 //
-//  1. gemv_prep: rotates x (when a sign vector is given) and writes, per row m
-//     and 128-group g, the activations in the order the tensor-core fragments
-//     want them ("slots"), as FP16 scaled by 2^(24 - 2 i - e_g). e_g is a
-//     power-of-two exponent chosen from the group's largest |x'|, i the
-//     position of the trit's 2-bit field inside a 16-bit half (see 2.). It
-//     also writes corr_g = sum_k x~_k (the FP16-rounded activations, back in
-//     real units) and 2^e_g.
+//  1. gemv_prep (one CTA per row m and 1024-block): rotates x (when a sign
+//     vector is given) and writes, per row m and 128-group g, the
+//     activations in the order the tensor-core fragments consume them
+//     ("slots"), as FP16 scaled by 2^(24 - 2 i - e_g). e_g is a power-of-two
+//     exponent chosen from the group's largest |x'|; i is the position of the
+//     trit's 2-bit field inside a 16-bit half (see 2.). It also writes
+//     corr_g = sum_k x~_k (the FP16-rounded activations, in real units) and
+//     2^e_g.
 //
-//  2. gemv: a persistent kernel. Each warp owns a contiguous run of (16-row
-//     tile pair, group) units and streams the packed bytes straight from HBM
-//     into registers. Base-3 bytes go through a 256-entry table in shared
-//     memory, replicated per lane so the gathers are conflict-free, that
-//     turns a byte into its five base-3 digits d = t + 1 as 2-bit fields;
-//     2-bit bytes already are such fields. One LOP3 per two weights then
-//     isolates field i of two bytes into the two halves of a register. Read
-//     as FP16, the half is the subnormal d * 4^i * 2^-24, exact. An
-//     m16n8k16 tensor-core MMA against the slot-ordered activations gives
-//     D = 2^-e sum_k d_k x~_k in FP32, and the group contributes
-//     s * (2^e D - corr) = s * sum_k t_k x~_k. The MMA's A operand is the
-//     weights (16 rows); its 8 columns are the activation rows m.
-//     Units that split a tile across warps leave FP32 partials; the warp
-//     that finishes a tile last (atomic counter) adds them in a fixed order,
-//     so results are deterministic.
+//  2. gemv (persistent, one CTA per SM): each warp owns a contiguous run of
+//     (32-row tile pair, group) units and streams the packed bytes straight
+//     from HBM into registers (L2 bulk prefetch of the run, one group of
+//     register double buffering). Base-3 bytes go through a 256-entry table
+//     in shared memory, replicated per lane so the gathers are conflict-free,
+//     that turns a byte into its five base-3 digits d = t + 1 as 2-bit fields;
+//     2-bit bytes already are such fields. One LOP3 per two weights isolates
+//     field i of two bytes into the two halves of a register; read as FP16,
+//     each half is the subnormal d * 4^i * 2^-24, exactly. An m16n8k16
+//     tensor-core MMA against the slot-ordered activations gives
+//     D = 2^-e sum_k d_k x~_k in FP32, and the group adds
+//     s * (2^e D - corr) = s * sum_k t_k x~_k. The MMA's A operand is 16 weight
+//     rows; its 8 columns are activation rows m.
+//     A tile split across warps leaves FP32 partials; the warp that finishes
+//     it last (atomic counter) adds them in a fixed order, so results are
+//     deterministic run to run.
 #include "bt_internal.cuh"
 
 namespace bt {
 
-constexpr int kGemvWarps = 16;
-constexpr int kGemvTiles = 2;        // 16-row tiles per unit (share the activation fragments)
-constexpr int kPrepWarps = 4;
+#ifndef BT_GEMV_WARPS
+#define BT_GEMV_WARPS 16
+#endif
+#ifndef BT_GEMV_TILES
+#define BT_GEMV_TILES 2
+#endif
+constexpr int kGemvWarps = BT_GEMV_WARPS;  // warps per CTA (one CTA per SM)
+constexpr int kGemvTiles = BT_GEMV_TILES;  // 16-row tiles per unit (share the activation fragments)
+constexpr int kPrepThreads = 256;    // 8 warps: one per group of a 1024-block
 constexpr int kLutBytes = 256 * 256; // 256 codes x (128 B low table + 128 B high table)
+constexpr int kZeroBytes = 512;      // zero fragment area (>= NT * 32)
+constexpr size_t kBsmemMax = 128 * 1024;
 
 // field mask: 2-bit field i of both 16-bit halves
 __host__ __device__ constexpr uint32_t fmask(int i) {
@@ -104,27 +114,24 @@ struct PrepArgs {
 };
 
 template <int LAYOUT>
-__global__ void __launch_bounds__(kPrepWarps * 32) gemv_prep_kernel(PrepArgs a) {
+__global__ void __launch_bounds__(kPrepThreads) gemv_prep_kernel(PrepArgs a) {
     constexpr int NT = LAYOUT == BT_LAYOUT_B3 ? kB3Mmas : k2bMmas;
-    __shared__ __align__(16) float tiles[kPrepWarps][32 * kTileStride];
+    __shared__ __align__(16) float xs[32 * kTileStride];
     pdl_launch_dependents();
     pdl_wait();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t gtid = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    for (int64_t i = gtid; i < a.P; i += (int64_t)gridDim.x * blockDim.x) a.counters[i] = 0;
+    if (blockIdx.x == 0)
+        for (int i = threadIdx.x; i < a.P; i += blockDim.x) a.counters[i] = 0;
 
-    float* tile = tiles[warp];
     const int nblocks = (a.G + 7) / 8;
-    const int64_t total = (int64_t)a.M * nblocks;
-    for (int64_t wb = (int64_t)blockIdx.x * kPrepWarps + warp; wb < total;
-         wb += (int64_t)gridDim.x * kPrepWarps) {
-        const int m = static_cast<int>(wb / nblocks), b = static_cast<int>(wb % nblocks);
-        const int64_t k0 = (int64_t)b * kBlock;
-        const int ng = min(8, a.G - 8 * b);
+    const int m = blockIdx.x / nblocks, b = blockIdx.x % nblocks;
+    const int64_t k0 = (int64_t)b * kBlock;
+    const int ng = min(8, a.G - 8 * b);
+    if (warp == 0) {
         float v[32];
         if (a.sign) {
             load_signed_bf16_block(reinterpret_cast<const uint16_t*>(a.x) + (int64_t)m * a.K + k0, a.sign, v);
-            fwht1024_warp(v, tile);
+            fwht1024_warp(v, xs);
         } else {
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
@@ -139,50 +146,51 @@ __global__ void __launch_bounds__(kPrepWarps * 32) gemv_prep_kernel(PrepArgs a) 
             }
         }
 #pragma unroll
-        for (int j = 0; j < 32; ++j) tile[32 * j + lane] = v[j];
-        __syncwarp();
+        for (int j = 0; j < 32; ++j) xs[32 * j + lane] = v[j];  // element 32 j + lane
+    }
+    __syncthreads();
+    const int q = warp;  // group within the block
+    if (q >= ng) return;
+    float v4[4];
+    float amax = 0.f;
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-            if (q >= ng) break;
-            float amax = 0.f;
+    for (int r = 0; r < 4; ++r) {
+        v4[r] = xs[128 * q + 32 * r + lane];
+        amax = fmaxf(amax, fabsf(v4[r]));
+    }
 #pragma unroll
-            for (int r = 0; r < 4; ++r) amax = fmaxf(amax, fabsf(v[4 * q + r]));
+    for (int s = 16; s > 0; s >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, s));
+    int E = amax > 0.f ? ilogbf(amax) + 1 : -100;  // amax < 2^E
+    E = max(-100, min(100, E));
+    const int e = 9 + E;
+    float corr = 0.f;
 #pragma unroll
-            for (int s = 16; s > 0; s >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, s));
-            int E = amax > 0.f ? ilogbf(amax) + 1 : -100;  // amax < 2^E
-            E = max(-100, min(100, E));
-            const int e = 9 + E;
-            float corr = 0.f;
+    for (int r = 0; r < 4; ++r) {
+        const int k = 32 * r + lane;
+        const int i = LAYOUT == BT_LAYOUT_B3 ? b3_field_of(k) : tb_field_of(k);
+        const __half hv = __float2half_rn(v4[r] * exp2i(24 - 2 * i - e));
+        corr += __half2float(hv) * exp2i(e + 2 * i - 24);
+    }
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int k = 32 * r + lane;
-                const int i = LAYOUT == BT_LAYOUT_B3 ? b3_field_of(k) : tb_field_of(k);
-                const __half hv = __float2half_rn(v[4 * q + r] * exp2i(24 - 2 * i - e));
-                corr += __half2float(hv) * exp2i(e + 2 * i - 24);
-            }
+    for (int s = 16; s > 0; s >>= 1) corr += __shfl_xor_sync(0xffffffffu, corr, s);
+    const int64_t gidx = (int64_t)m * a.G + 8 * b + q;
+    if (lane == 0) a.meta[gidx] = make_float2(corr, exp2i(e));
+    uint32_t* dst = a.bslots + gidx * (NT * 8);
+    const float* xg = xs + 128 * q;
+    for (int widx = lane; widx < NT * 8; widx += 32) {
+        const int t = widx >> 3, c = (widx >> 1) & 3, hp = widx & 1;
+        uint32_t word = 0;
 #pragma unroll
-            for (int s = 16; s > 0; s >>= 1) corr += __shfl_xor_sync(0xffffffffu, corr, s);
-            const int64_t gidx = (int64_t)m * a.G + 8 * b + q;
-            if (lane == 0) a.meta[gidx] = make_float2(corr, exp2i(e));
-            uint32_t* dst = a.bslots + gidx * (NT * 8);
-            const float* xs = tile + 128 * q;
-            for (int widx = lane; widx < NT * 8; widx += 32) {
-                const int t = widx >> 3, c = (widx >> 1) & 3, hp = widx & 1;
-                uint32_t word = 0;
-#pragma unroll
-                for (int u = 0; u < 2; ++u) {
-                    int i = 0;
-                    const int k = LAYOUT == BT_LAYOUT_B3 ? b3_slot(t, c, 2 * hp + u, &i)
-                                                         : tb_slot(t, c, 2 * hp + u, &i);
-                    if (k >= 0) {
-                        const __half hv = __float2half_rn(xs[k] * exp2i(24 - 2 * i - e));
-                        word |= static_cast<uint32_t>(__half_as_ushort(hv)) << (16 * u);
-                    }
-                }
-                dst[widx] = word;
+        for (int u = 0; u < 2; ++u) {
+            int i = 0;
+            const int k = LAYOUT == BT_LAYOUT_B3 ? b3_slot(t, c, 2 * hp + u, &i)
+                                                 : tb_slot(t, c, 2 * hp + u, &i);
+            if (k >= 0) {
+                const __half hv = __float2half_rn(xg[k] * exp2i(24 - 2 * i - e));
+                word |= static_cast<uint32_t>(__half_as_ushort(hv)) << (16 * u);
             }
         }
-        __syncwarp();
+        dst[widx] = word;
     }
 }
 
@@ -198,107 +206,412 @@ struct GemvArgs {
     void* y;
     int y_bf16;
     int M, N, G;
-    int64_t row_bytes;
+    uint32_t row_bytes;
     int64_t U;               // P * G units
     int64_t chunk;           // units per warp
     int32_t* dev_err;
 };
 
-__device__ __forceinline__ uint32_t lds_u32(const uint8_t* base, uint32_t off) {
-    return *reinterpret_cast<const uint32_t*>(base + off);
+extern __shared__ __align__(1024) uint8_t gemv_smem[];
+
+// Table lookup at byte offset `off` of the dynamic shared memory (the table
+// sits at its start); indexing the symbol lets the compiler fold the base.
+__device__ __forceinline__ uint32_t lut_u32(uint32_t off) {
+    return *reinterpret_cast<const uint32_t*>(gemv_smem + off);
 }
 
-// Decode one row's six bytes 6c..6c+5 of a base-3 group into 15 registers.
-// W0, W1: the aligned 8-byte window holding them; o8 = 8 * (offset in window).
-__device__ __forceinline__ void b3_decode_pairs(uint32_t W0, uint32_t W1, uint32_t o8, uint32_t lane4,
-                                                const uint8_t* lut, uint32_t (&R)[15], uint32_t& err) {
+__device__ __forceinline__ uint32_t smem_u32addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint32_t lds_u32(uint32_t addr) {
+    uint32_t r;
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(r) : "r"(addr));
+    return r;
+}
+__device__ __forceinline__ uint2 lds_u64(uint32_t addr) {
+    uint2 r;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(addr));
+    return r;
+}
+
+// Registers a warp holds for one group: packed bytes and scales of its rows.
+template <int LAYOUT>
+struct CodeStage {
+    uint32_t w[kGemvTiles][LAYOUT == BT_LAYOUT_B3 ? 5 : 4];
+    uint32_t s[kGemvTiles][2];
+};
+
+// Byte offsets (from a.codes / a.scales) for one parity of groups j0, j0+2, ...
+struct StagePtr {
+    uint32_t og[kGemvTiles], oh[kGemvTiles];  // aligned windows (base-3) or 8-byte chunks (2-bit)
+    uint32_t o12[kGemvTiles];                 // base-3 pair 12 (bytes 24, 25)
+    uint32_t osg[kGemvTiles], osh[kGemvTiles];// scale element offsets
+};
+
+template <int LAYOUT>
+__device__ __forceinline__ void load_stage(CodeStage<LAYOUT>& S, const GemvArgs& a, const StagePtr& P) {
+#pragma unroll
+    for (int tt = 0; tt < kGemvTiles; ++tt) {
+        if constexpr (LAYOUT == BT_LAYOUT_B3) {
+            S.w[tt][0] = ldg_stream_u32(a.codes + P.og[tt]);
+            S.w[tt][1] = ldg_stream_u32(a.codes + P.og[tt] + 4);
+            S.w[tt][2] = ldg_stream_u32(a.codes + P.oh[tt]);
+            S.w[tt][3] = ldg_stream_u32(a.codes + P.oh[tt] + 4);
+            S.w[tt][4] = ldg_stream_u16(a.codes + P.o12[tt]);
+        } else {
+            const uint2 x0 = ldg_stream_u64(a.codes + P.og[tt]);
+            const uint2 x1 = ldg_stream_u64(a.codes + P.oh[tt]);
+            S.w[tt][0] = x0.x; S.w[tt][1] = x0.y; S.w[tt][2] = x1.x; S.w[tt][3] = x1.y;
+        }
+        S.s[tt][0] = ldg_stream_u16(a.scales + P.osg[tt]);
+        S.s[tt][1] = ldg_stream_u16(a.scales + P.osh[tt]);
+    }
+}
+
+__device__ __forceinline__ void advance2(StagePtr& P, int group_bytes) {
+#pragma unroll
+    for (int tt = 0; tt < kGemvTiles; ++tt) {
+        P.og[tt] += 2 * group_bytes;
+        P.oh[tt] += 2 * group_bytes;
+        P.o12[tt] += 2 * group_bytes;
+        P.osg[tt] += 2;
+        P.osh[tt] += 2;
+    }
+}
+
+// Decode one row's bytes 6c..6c+5 of a base-3 group into 15 registers.
+__device__ __forceinline__ void b3_decode_pairs(uint32_t W0, uint32_t W1, uint32_t o8, uint32_t lane_addr,
+                                                uint32_t (&R)[15], uint32_t& err) {
     const uint32_t lo = __funnelshift_r(W0, W1, o8);
     const uint32_t hi = W1 >> o8;
 #pragma unroll
     for (int q = 0; q < 3; ++q) {
         const uint32_t src = q == 2 ? hi : lo;
         const uint32_t b = q == 1 ? 2u : 0u;
-        const uint32_t aA = prmt(src, lane4, 0x5504u | (b << 4));
-        const uint32_t aB = prmt(src, lane4, 0x5504u | ((b + 1) << 4));
-        const uint32_t va = lds_u32(lut, aA);
-        const uint32_t vb = lds_u32(lut, aB + 128);
+        // address = table + code * 256 + lane * 4 (+128 for the high table)
+        const uint32_t va = lut_u32(prmt(src, lane_addr, 0x5504u | (b << 4)));
+        const uint32_t vb = lut_u32(prmt(src, lane_addr, 0x5504u | ((b + 1) << 4)) + 128);
         err = lop3_or3(err, va, vb);
 #pragma unroll
         for (int i = 0; i < 5; ++i) R[5 * q + i] = lop3_or_and(va, vb, fmask(i));
     }
 }
 
+struct LaneCtx {
+    uint32_t lane_addr;          // lane * 4: byte offset of this lane's table column
+    uint32_t mG[3], mH[3];       // pair-12 field masks for rows g and g+8
+    uint32_t bbase[2], bstride[2];        // activation fragment base/stride per column tile (shared)
+    uint32_t mbase[2][2], mstride[2][2];  // meta base/stride per column tile and column
+};
+
+// One group j for the warp's tiles: activation fragments, decode, MMA, scale.
+template <int LAYOUT, int MT, bool BSMEM, bool M1>
+__device__ __forceinline__ void process_group(const GemvArgs& a, const CodeStage<LAYOUT>& S, int j,
+                                              uint32_t o8g, uint32_t o8h, const LaneCtx& cx,
+                                              float (&acc)[kGemvTiles][MT][4], uint32_t& err) {
+    constexpr int NT = LAYOUT == BT_LAYOUT_B3 ? kB3Mmas : k2bMmas;
+    const int lane = threadIdx.x & 31, g = lane >> 2, c = lane & 3;
+    uint32_t bf[MT][NT][2];
+    float pm[MT][2], cm[MT][2];
+    if constexpr (BSMEM) {
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const uint32_t ba = cx.bbase[mt] + static_cast<uint32_t>(j) * cx.bstride[mt];
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                const uint2 v = lds_u64(ba + 32 * t);
+                bf[mt][t][0] = v.x;
+                bf[mt][t][1] = v.y;
+            }
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                if (M1 && r == 1) { cm[mt][1] = 0.f; pm[mt][1] = 0.f; continue; }
+                const uint2 md = lds_u64(cx.mbase[mt][r] + static_cast<uint32_t>(j) * cx.mstride[mt][r]);
+                cm[mt][r] = __uint_as_float(md.x);
+                pm[mt][r] = __uint_as_float(md.y);
+            }
+        }
+    } else {
+        const int G = a.G;
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            const int m = mt * 8 + g;
+            const uint32_t* bp = a.bslots + (((int64_t)m * G + j) * NT) * 8 + c * 2;
+#pragma unroll
+            for (int t = 0; t < NT; ++t) {
+                uint2 v = make_uint2(0u, 0u);
+                if (m < a.M) v = ldg_u64(bp + t * 8);
+                bf[mt][t][0] = v.x;
+                bf[mt][t][1] = v.y;
+            }
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int mm = mt * 8 + 2 * c + r;
+                float2 md = make_float2(0.f, 0.f);
+                if (mm < a.M) md = __ldg(a.meta + (int64_t)mm * G + j);
+                cm[mt][r] = md.x;
+                pm[mt][r] = md.y;
+            }
+        }
+        if (j + 1 < G) {
+            // the next group's fragment lines and meta into L1
+            constexpr int lines = (NT * 32 + 127) / 128;
+            if (lane < a.M * (lines + 1)) {
+                const int mm = lane / (lines + 1), l = lane % (lines + 1);
+                if (l < lines)
+                    prefetch_l1(reinterpret_cast<const uint8_t*>(a.bslots + (((int64_t)mm * G + j + 1) * NT) * 8) + 128 * l);
+                else
+                    prefetch_l1(a.meta + (int64_t)mm * G + j + 1);
+            }
+        }
+    }
+#pragma unroll
+    for (int tt = 0; tt < kGemvTiles; ++tt) {
+        const float sg = f16_bits_to_f32(S.s[tt][0]);
+        const float sh = f16_bits_to_f32(S.s[tt][1]);
+        uint32_t Rg[16], Rh[16], QG[3], QH[3];
+        if constexpr (LAYOUT == BT_LAYOUT_B3) {
+            uint32_t r15[15];
+            b3_decode_pairs(S.w[tt][0], S.w[tt][1], o8g, cx.lane_addr, r15, err);
+#pragma unroll
+            for (int i = 0; i < 15; ++i) Rg[i] = r15[i];
+            b3_decode_pairs(S.w[tt][2], S.w[tt][3], o8h, cx.lane_addr, r15, err);
+#pragma unroll
+            for (int i = 0; i < 15; ++i) Rh[i] = r15[i];
+            Rg[15] = Rh[15] = 0u;
+            const uint32_t w12 = S.w[tt][4];
+            const uint32_t va = lut_u32(prmt(w12, cx.lane_addr, 0x5504u));
+            const uint32_t vb = lut_u32(prmt(w12, cx.lane_addr, 0x5514u) + 128);
+            err = lop3_or3(err, va, vb);
+#pragma unroll
+            for (int i = 0; i < 3; ++i) {
+                QG[i] = lop3_or_and(va, vb, cx.mG[i]);
+                QH[i] = lop3_or_and(va, vb, cx.mH[i]);
+            }
+        } else {
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const uint32_t w = S.w[tt][r];
+                const uint32_t w12s = w >> 12;
+                uint32_t* Rr = r < 2 ? Rg : Rh;
+                const int base = (r & 1) * 8;
+#pragma unroll
+                for (int f = 0; f < 6; ++f) Rr[base + f] = w & fmask(f);
+                Rr[base + 6] = w12s & fmask(0);
+                Rr[base + 7] = w12s & fmask(1);
+                err |= w & (w >> 1);
+            }
+#pragma unroll
+            for (int i = 0; i < 3; ++i) QG[i] = QH[i] = 0u;
+        }
+#pragma unroll
+        for (int mt = 0; mt < MT; ++mt) {
+            float d[4] = {0.f, 0.f, 0.f, 0.f};
+            if constexpr (LAYOUT == BT_LAYOUT_B3) {
+#pragma unroll
+                for (int t = 0; t < 7; ++t)
+                    mma_f16_16816(d, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1], bf[mt][t][0],
+                                  bf[mt][t][1], d);
+                mma_f16_16816(d, Rg[14], Rh[14], QG[0], QH[0], bf[mt][7][0], bf[mt][7][1], d);
+                mma_f16_16816(d, QG[1], QH[1], QG[2], QH[2], bf[mt][NT - 1][0], bf[mt][NT - 1][1], d);
+            } else {
+#pragma unroll
+                for (int t = 0; t < NT; ++t)
+                    mma_f16_16816(d, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1], bf[mt][t][0],
+                                  bf[mt][t][1], d);
+            }
+            acc[tt][mt][0] = fmaf(sg, fmaf(d[0], pm[mt][0], -cm[mt][0]), acc[tt][mt][0]);
+            acc[tt][mt][2] = fmaf(sh, fmaf(d[2], pm[mt][0], -cm[mt][0]), acc[tt][mt][2]);
+            if (!M1) {
+                acc[tt][mt][1] = fmaf(sg, fmaf(d[1], pm[mt][1], -cm[mt][1]), acc[tt][mt][1]);
+                acc[tt][mt][3] = fmaf(sh, fmaf(d[3], pm[mt][1], -cm[mt][1]), acc[tt][mt][3]);
+            }
+        }
+    }
+}
+
+// L2 prefetch of one segment: lane l covers row l of the tile pair.
+__device__ __forceinline__ void prefetch_segment(const GemvArgs& a, int p, int j0, int j1, int group_bytes) {
+    const uintptr_t base = reinterpret_cast<uintptr_t>(a.codes);
+    const uintptr_t lo_lim = (base + 15) & ~uintptr_t(15);
+    const uintptr_t hi_lim = (base + (uintptr_t)a.N * a.row_bytes) & ~uintptr_t(15);
+    for (int r = threadIdx.x & 31; r < kGemvTiles * 16; r += 32) {
+        const int n = p * (kGemvTiles * 16) + r;
+        if (n >= a.N) break;
+        const uintptr_t row = base + (uintptr_t)n * a.row_bytes;
+        uintptr_t s = (row + (uintptr_t)j0 * group_bytes) & ~uintptr_t(15);
+        uintptr_t e = (row + (uintptr_t)j1 * group_bytes + 15) & ~uintptr_t(15);
+        if (s < lo_lim) s = lo_lim;
+        if (e > hi_lim) e = hi_lim;
+        if (e > s) prefetch_l2_bulk(reinterpret_cast<const void*>(s), static_cast<uint32_t>(e - s));
+        prefetch_l2(a.scales + (int64_t)n * a.G + j0);
+        prefetch_l2(a.scales + (int64_t)n * a.G + (j1 - 1));
+    }
+}
+
+// Block-wide copy global -> shared with eight loads in flight per thread.
 template <typename T>
+__device__ __forceinline__ void copy_to_smem(T* dst, const T* src, int n) {
+    constexpr int U = 8;
+    for (int base = 0; base < n; base += U * blockDim.x) {
+        T v[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = base + u * blockDim.x + threadIdx.x;
+            if (i < n) v[u] = __ldcg(src + i);
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int i = base + u * blockDim.x + threadIdx.x;
+            if (i < n) dst[i] = v[u];
+        }
+    }
+}
+
+__device__ __forceinline__ void fence_acq_rel_gpu() {
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
 __device__ __forceinline__ void store_y(void* y, int bf16, int64_t idx, float v) {
     if (bf16) reinterpret_cast<__nv_bfloat16*>(y)[idx] = __float2bfloat16_rn(v);
     else reinterpret_cast<float*>(y)[idx] = v;
 }
 
-template <int LAYOUT, int MT>
+template <int LAYOUT, int MT, bool BSMEM, bool M1>
 __global__ void __launch_bounds__(kGemvWarps * 32, 1) gemv_kernel(GemvArgs a) {
-    constexpr int NT = LAYOUT == BT_LAYOUT_B3 ? kB3Mmas : k2bMmas;
     constexpr int TL = kGemvTiles;
-    extern __shared__ __align__(16) uint8_t lut[];
+    constexpr int NT = LAYOUT == BT_LAYOUT_B3 ? kB3Mmas : k2bMmas;
+    constexpr int GB = LAYOUT == BT_LAYOUT_B3 ? kB3GroupBytes : k2bGroupBytes;
+    uint8_t* smem = gemv_smem;
+    uint8_t* lut = smem;                                              // base-3 only
+    uint8_t* sB = smem + (LAYOUT == BT_LAYOUT_B3 ? kLutBytes : 0);    // zero area, meta, slots
     pdl_launch_dependents();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, c = lane & 3;
-
-    if (LAYOUT == BT_LAYOUT_B3) {
-        // table row = code (256 B): [0,128) low table, [128,256) high table,
-        // one 4-byte entry per lane. Entry: the five digits as 2-bit fields
-        // at bits 2i (low) or 16 + 2i (high); bit 31 flags codes >= 243.
-        uint32_t* lut32 = reinterpret_cast<uint32_t*>(lut);
-        for (int idx = threadIdx.x; idx < 256 * 64; idx += blockDim.x) {
-            const int code = idx >> 6, hi = (idx >> 5) & 1;
-            uint32_t val = 0x80000000u;
-            if (code < 243) {
-                uint32_t f = 0;
-                int r = code;
-#pragma unroll
-                for (int i = 0; i < 5; ++i) { f |= static_cast<uint32_t>(r % 3) << (2 * i); r /= 3; }
-                val = hi ? (f << 16) : f;
-            }
-            lut32[idx] = val;
-        }
-        __syncthreads();
-    }
+    const int G = a.G;
 
     const int64_t wglobal = (int64_t)blockIdx.x * kGemvWarps + warp;
     const int64_t u_begin = wglobal * a.chunk;
     const int64_t u_end = min(a.U, u_begin + a.chunk);
-    pdl_wait();
+    // The weights do not depend on the previous kernel: start streaming the
+    // first segment into L2 before waiting for it.
+    if (u_begin < u_end) {
+        const int p0 = static_cast<int>(u_begin / G);
+        const int j00 = static_cast<int>(u_begin - (int64_t)p0 * G);
+        const int64_t j10 = (int64_t)j00 + (u_end - u_begin);
+        prefetch_segment(a, p0, j00, static_cast<int>(j10 < G ? j10 : G), GB);
+    }
 
-    const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
-    // pair-12 field masks (base-3): even c -> fields 0,1,2; odd c -> 3,4,none.
-    uint32_t mq[3];
-    mq[0] = (c & 1) ? fmask(3) : fmask(0);
-    mq[1] = (c & 1) ? fmask(4) : fmask(1);
-    mq[2] = (c & 1) ? 0u : fmask(2);
-    uint32_t mG[3], mH[3];
+    if constexpr (LAYOUT == BT_LAYOUT_B3) {
+        // table row = code (256 B): [0,128) low table, [128,256) high table,
+        // one 4-byte entry per lane. Entry: the five digits as 2-bit fields
+        // at bits 2i (low) or 16 + 2i (high); bit 31 flags codes >= 243.
+        for (int code = threadIdx.x; code < 256; code += blockDim.x) {
+            uint32_t f = 0x80000000u;
+            if (code < 243) {
+                f = 0;
+                int r = code;
 #pragma unroll
-    for (int i = 0; i < 3; ++i) { mG[i] = c < 2 ? mq[i] : 0u; mH[i] = c < 2 ? 0u : mq[i]; }
+                for (int i = 0; i < 5; ++i) { f |= static_cast<uint32_t>(r % 3) << (2 * i); r /= 3; }
+            }
+            const uint32_t fh = code < 243 ? (f << 16) : f;
+            uint4* row = reinterpret_cast<uint4*>(lut + code * 256);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) row[v] = make_uint4(f, f, f, f);
+#pragma unroll
+            for (int v = 8; v < 16; ++v) row[v] = make_uint4(fh, fh, fh, fh);
+        }
+    }
+    const uint32_t zero_area = smem_u32addr(sB);
+    const uint32_t meta_area = zero_area + kZeroBytes;
+    const uint32_t slot_area = meta_area + static_cast<uint32_t>(a.M * G * 8);
+    {
+        uint4* z = reinterpret_cast<uint4*>(sB);
+        for (int i = threadIdx.x; i < kZeroBytes / 16; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
+    }
+    pdl_wait();
+    if constexpr (BSMEM) {
+        // meta [M][G] float2, then slots [M][G][NT*32 B]
+        const float2* gm = a.meta;
+        float2* sm = reinterpret_cast<float2*>(sB + kZeroBytes);
+        copy_to_smem<float2>(sm, gm, a.M * G);
+        const uint4* gb = reinterpret_cast<const uint4*>(a.bslots);
+        uint4* sb = reinterpret_cast<uint4*>(sB + kZeroBytes + a.M * G * 8);
+        copy_to_smem<uint4>(sb, gb, a.M * G * NT * 2);  // NT * 32 bytes per (m, g)
+    }
+    __syncthreads();
+
+    LaneCtx cx;
+    cx.lane_addr = static_cast<uint32_t>(lane) * 4u;
+    {
+        // pair-12 field masks (base-3): even c -> fields 0,1,2; odd c -> 3,4,none.
+        uint32_t mq[3];
+        mq[0] = (c & 1) ? fmask(3) : fmask(0);
+        mq[1] = (c & 1) ? fmask(4) : fmask(1);
+        mq[2] = (c & 1) ? 0u : fmask(2);
+#pragma unroll
+        for (int i = 0; i < 3; ++i) { cx.mG[i] = c < 2 ? mq[i] : 0u; cx.mH[i] = c < 2 ? 0u : mq[i]; }
+    }
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+        const int m = mt * 8 + g;
+        const bool okm = m < a.M;
+        cx.bbase[mt] = okm ? slot_area + static_cast<uint32_t>(m * G * NT * 32 + c * 8) : zero_area + c * 8;
+        cx.bstride[mt] = okm ? NT * 32 : 0;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int mm = mt * 8 + 2 * c + r;
+            const bool ok = mm < a.M;
+            cx.mbase[mt][r] = ok ? meta_area + static_cast<uint32_t>(mm * G * 8) : zero_area;
+            cx.mstride[mt][r] = ok ? 8 : 0;
+        }
+    }
 
     uint32_t err = 0;
-    const int G = a.G;
     int64_t u = u_begin;
+    bool first_segment = true;
     while (u < u_end) {
         const int p = static_cast<int>(u / G);
         const int j0 = static_cast<int>(u - (int64_t)p * G);
         const int64_t j1_64 = (int64_t)j0 + (u_end - u);
         const int j1 = static_cast<int>(j1_64 < G ? j1_64 : (int64_t)G);
+        if (!first_segment) prefetch_segment(a, p, j0, j1, GB);
 
-        const uint8_t* rowg[TL];
-        const uint8_t* rowh[TL];
-        const uint16_t* scg[TL];
-        const uint16_t* sch[TL];
+        // offsets of groups j0 (stage 0) and j0 + 1 (stage 1); base-3 window
+        // shifts for each stage (a +26-byte step flips the 4-byte alignment)
+        StagePtr P0, P1;
+        uint32_t o8g0 = 0, o8h0 = 0, o8g1 = 0, o8h1 = 0;
 #pragma unroll
         for (int tt = 0; tt < TL; ++tt) {
-            const int ng = min(a.N - 1, (p * TL + tt) * 16 + g);
-            const int nh = min(a.N - 1, (p * TL + tt) * 16 + g + 8);
-            rowg[tt] = a.codes + (int64_t)ng * a.row_bytes;
-            rowh[tt] = a.codes + (int64_t)nh * a.row_bytes;
-            scg[tt] = a.scales + (int64_t)ng * G;
-            sch[tt] = a.scales + (int64_t)nh * G;
+            const uint32_t ng = static_cast<uint32_t>(min(a.N - 1, (p * TL + tt) * 16 + g));
+            const uint32_t nh = static_cast<uint32_t>(min(a.N - 1, (p * TL + tt) * 16 + g + 8));
+            const uint32_t rg = ng * a.row_bytes, rh = nh * a.row_bytes;
+#pragma unroll
+            for (int s = 0; s < 2; ++s) {
+                StagePtr& P = s ? P1 : P0;
+                const uint32_t js = static_cast<uint32_t>(j0 + s) * GB;
+                if constexpr (LAYOUT == BT_LAYOUT_B3) {
+                    const uint32_t ug = rg + js + 6u * c, uh = rh + js + 6u * c;  // codes are 16-aligned
+                    P.og[tt] = ug & ~3u;
+                    P.oh[tt] = uh & ~3u;
+                    P.o12[tt] = (c < 2 ? rg : rh) + js + 24u;
+                    if (tt == 0) {
+                        // rows 8 and 16 apart share their 4-byte alignment
+                        // (8 * row_bytes is a multiple of 4), so tile 0's
+                        // shifts hold for tile 1 as well
+                        if (s == 0) { o8g0 = (ug & 3u) * 8u; o8h0 = (uh & 3u) * 8u; }
+                        else { o8g1 = (ug & 3u) * 8u; o8h1 = (uh & 3u) * 8u; }
+                    }
+                } else {
+                    P.og[tt] = rg + js + 8u * c;
+                    P.oh[tt] = rh + js + 8u * c;
+                    P.o12[tt] = 0;
+                }
+            }
+            P0.osg[tt] = ng * G + j0;
+            P0.osh[tt] = nh * G + j0;
+            P1.osg[tt] = P0.osg[tt] + 1;
+            P1.osh[tt] = P0.osh[tt] + 1;
         }
         float acc[TL][MT][4];
 #pragma unroll
@@ -308,108 +621,18 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1) gemv_kernel(GemvArgs a) {
 #pragma unroll
                 for (int r = 0; r < 4; ++r) acc[tt][mt][r] = 0.f;
 
-        for (int j = j0; j < j1; ++j) {
-            // activation fragments and group constants, shared by the tiles
-            uint32_t bf[MT][NT][2];
-            float pm[MT][2], cm[MT][2];
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                const int m = mt * 8 + g;
-                const uint32_t* bp = a.bslots + (((int64_t)m * G + j) * NT) * 8 + c * 2;
-#pragma unroll
-                for (int t = 0; t < NT; ++t) {
-                    uint2 v = make_uint2(0u, 0u);
-                    if (m < a.M) v = ldg_u64(bp + t * 8);
-                    bf[mt][t][0] = v.x;
-                    bf[mt][t][1] = v.y;
-                }
-#pragma unroll
-                for (int r = 0; r < 2; ++r) {
-                    const int mm = mt * 8 + 2 * c + r;
-                    float2 md = make_float2(0.f, 0.f);
-                    if (mm < a.M) md = __ldg(a.meta + (int64_t)mm * G + j);
-                    cm[mt][r] = md.x;
-                    pm[mt][r] = md.y;
-                }
-            }
-#pragma unroll
-            for (int tt = 0; tt < TL; ++tt) {
-                const float sg = f16_bits_to_f32(__ldg(scg[tt] + j));
-                const float sh = f16_bits_to_f32(__ldg(sch[tt] + j));
-                uint32_t Rg[16], Rh[16];
-                uint32_t QG[3], QH[3];
-                if (LAYOUT == BT_LAYOUT_B3) {
-                    // bytes 6c..6c+5 of the group lie in the aligned 8-byte window
-                    // starting at (address & ~3); rows may differ in alignment
-                    const int64_t off = (int64_t)j * kB3GroupBytes + 6 * c;
-                    const uintptr_t ag = reinterpret_cast<uintptr_t>(rowg[tt] + off);
-                    const uintptr_t ah = reinterpret_cast<uintptr_t>(rowh[tt] + off);
-                    const uint32_t o8g = static_cast<uint32_t>(ag & 3) * 8u;
-                    const uint32_t o8h = static_cast<uint32_t>(ah & 3) * 8u;
-                    const uint8_t* pg = reinterpret_cast<const uint8_t*>(ag & ~uintptr_t(3));
-                    const uint8_t* ph = reinterpret_cast<const uint8_t*>(ah & ~uintptr_t(3));
-                    const uint32_t g0 = ldg_u32(pg), g1 = ldg_u32(pg + 4);
-                    const uint32_t h0 = ldg_u32(ph), h1 = ldg_u32(ph + 4);
-                    const uint8_t* pp = (c < 2 ? rowg[tt] : rowh[tt]) + (int64_t)j * kB3GroupBytes + 24;
-                    const uint32_t w12 = ldg_u16(pp);
-                    uint32_t r15[15];
-                    b3_decode_pairs(g0, g1, o8g, lane4, lut, r15, err);
-#pragma unroll
-                    for (int i = 0; i < 15; ++i) Rg[i] = r15[i];
-                    b3_decode_pairs(h0, h1, o8h, lane4, lut, r15, err);
-#pragma unroll
-                    for (int i = 0; i < 15; ++i) Rh[i] = r15[i];
-                    Rg[15] = Rh[15] = 0u;
-                    const uint32_t va = lds_u32(lut, prmt(w12, lane4, 0x5504u));
-                    const uint32_t vb = lds_u32(lut, prmt(w12, lane4, 0x5514u) + 128);
-                    err = lop3_or3(err, va, vb);
-#pragma unroll
-                    for (int i = 0; i < 3; ++i) {
-                        QG[i] = lop3_or_and(va, vb, mG[i]);
-                        QH[i] = lop3_or_and(va, vb, mH[i]);
-                    }
-                } else {
-                    const int64_t off = (int64_t)j * k2bGroupBytes + 8 * c;
-                    const uint2 wg = ldg_u64(rowg[tt] + off);
-                    const uint2 wh = ldg_u64(rowh[tt] + off);
-                    const uint32_t ws[4] = {wg.x, wg.y, wh.x, wh.y};
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) {
-                        const uint32_t w = ws[r];
-                        const uint32_t w12s = w >> 12;
-                        uint32_t* R = r < 2 ? Rg : Rh;
-                        const int base = (r & 1) * 8;
-#pragma unroll
-                        for (int f = 0; f < 6; ++f) R[base + f] = w & fmask(f);
-                        R[base + 6] = w12s & fmask(0);
-                        R[base + 7] = w12s & fmask(1);
-                        err |= w & (w >> 1);
-                    }
-#pragma unroll
-                    for (int i = 0; i < 3; ++i) QG[i] = QH[i] = 0u;
-                }
-#pragma unroll
-                for (int mt = 0; mt < MT; ++mt) {
-                    float d[4] = {0.f, 0.f, 0.f, 0.f};
-                    if (LAYOUT == BT_LAYOUT_B3) {
-#pragma unroll
-                        for (int t = 0; t < 7; ++t)
-                            mma_f16_16816(d, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1],
-                                          bf[mt][t][0], bf[mt][t][1], d);
-                        mma_f16_16816(d, Rg[14], Rh[14], QG[0], QH[0], bf[mt][7][0], bf[mt][7][1], d);
-                        mma_f16_16816(d, QG[1], QH[1], QG[2], QH[2], bf[mt][NT - 1][0], bf[mt][NT - 1][1], d);
-                    } else {
-#pragma unroll
-                        for (int t = 0; t < NT; ++t)
-                            mma_f16_16816(d, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1],
-                                          bf[mt][t][0], bf[mt][t][1], d);
-                    }
-                    acc[tt][mt][0] = fmaf(sg, fmaf(d[0], pm[mt][0], -cm[mt][0]), acc[tt][mt][0]);
-                    acc[tt][mt][1] = fmaf(sg, fmaf(d[1], pm[mt][1], -cm[mt][1]), acc[tt][mt][1]);
-                    acc[tt][mt][2] = fmaf(sh, fmaf(d[2], pm[mt][0], -cm[mt][0]), acc[tt][mt][2]);
-                    acc[tt][mt][3] = fmaf(sh, fmaf(d[3], pm[mt][1], -cm[mt][1]), acc[tt][mt][3]);
-                }
-            }
+        // two register stages: the next group's bytes are in flight while
+        // this one is decoded
+        CodeStage<LAYOUT> S0, S1;
+        load_stage(S0, a, P0);
+        for (int j = j0; j < j1; j += 2) {
+            if (j + 1 < j1) load_stage(S1, a, P1);
+            advance2(P0, GB);
+            process_group<LAYOUT, MT, BSMEM, M1>(a, S0, j, o8g0, o8h0, cx, acc, err);
+            if (j + 1 >= j1) break;
+            if (j + 2 < j1) load_stage(S0, a, P0);
+            advance2(P1, GB);
+            process_group<LAYOUT, MT, BSMEM, M1>(a, S1, j + 1, o8g1, o8h1, cx, acc, err);
         }
 
         // ---- write the segment: whole tile -> y, part of a tile -> partials + fixup
@@ -423,10 +646,10 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1) gemv_kernel(GemvArgs a) {
                     for (int r = 0; r < 4; ++r) {
                         const int n = (p * TL + tt) * 16 + g + (r >> 1) * 8;
                         const int m = mt * 8 + 2 * c + (r & 1);
-                        if (n < a.N && m < a.M) store_y<float>(a.y, a.y_bf16, (int64_t)m * a.N + n, acc[tt][mt][r]);
+                        if (n < a.N && m < a.M) store_y(a.y, a.y_bf16, (int64_t)m * a.N + n, acc[tt][mt][r]);
                     }
         } else {
-            const int slot = (u == u_begin) ? 0 : 1;
+            const int slot = first_segment ? 0 : 1;
             float* part = a.partials + ((wglobal * 2 + slot) * (TL * 16)) * a.M;
 #pragma unroll
             for (int tt = 0; tt < TL; ++tt)
@@ -438,7 +661,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1) gemv_kernel(GemvArgs a) {
                         const int m = mt * 8 + 2 * c + (r & 1);
                         if (m < a.M) __stcg(part + row * a.M + m, acc[tt][mt][r]);
                     }
-            __threadfence();
+            // release this warp's partials, then count the segment in
+            fence_acq_rel_gpu();
             __syncwarp();
             const int64_t w_lo = ((int64_t)p * G) / a.chunk;
             const int64_t w_hi = ((int64_t)(p + 1) * G - 1) / a.chunk;
@@ -449,42 +673,36 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1) gemv_kernel(GemvArgs a) {
             }
             last = __shfl_sync(0xffffffffu, last, 0);
             if (last) {
-                __threadfence();
-                float sum[TL][MT][4];
+                // the last segment of the tile adds all partials in segment
+                // order; lane l owns row l (loads of all segments in flight)
+                fence_acq_rel_gpu();
+                const int nseg = static_cast<int>(w_hi - w_lo) + 1;
+                for (int row = lane; row < TL * 16; row += 32) {
+                    const int n = p * TL * 16 + row;
+                    for (int m = 0; m < a.M; ++m) {
+                        float sum = 0.f;
+                        for (int s0 = 0; s0 < nseg; s0 += 8) {
+                            float v[8];
 #pragma unroll
-                for (int tt = 0; tt < TL; ++tt)
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) sum[tt][mt][r] = 0.f;
-                for (int64_t w = w_lo; w <= w_hi; ++w) {
-                    const int ws = ((w * a.chunk) / G == p) ? 0 : 1;
-                    const float* pw = a.partials + ((w * 2 + ws) * (TL * 16)) * a.M;
-#pragma unroll
-                    for (int tt = 0; tt < TL; ++tt)
-#pragma unroll
-                        for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                            for (int r = 0; r < 4; ++r) {
-                                const int row = tt * 16 + g + (r >> 1) * 8;
-                                const int m = mt * 8 + 2 * c + (r & 1);
-                                if (m < a.M) sum[tt][mt][r] += __ldcg(pw + row * a.M + m);
+                            for (int s1 = 0; s1 < 8; ++s1) {
+                                const int64_t w = w_lo + s0 + s1;
+                                v[s1] = 0.f;
+                                if (s0 + s1 < nseg) {
+                                    const int ws = (w * a.chunk >= (int64_t)p * G) ? 0 : 1;  // w starts in p
+                                    v[s1] = __ldcg(a.partials + ((w * 2 + ws) * (TL * 16) + row) * a.M + m);
+                                }
                             }
-                }
 #pragma unroll
-                for (int tt = 0; tt < TL; ++tt)
-#pragma unroll
-                    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-                        for (int r = 0; r < 4; ++r) {
-                            const int n = (p * TL + tt) * 16 + g + (r >> 1) * 8;
-                            const int m = mt * 8 + 2 * c + (r & 1);
-                            if (n < a.N && m < a.M) store_y<float>(a.y, a.y_bf16, (int64_t)m * a.N + n, sum[tt][mt][r]);
+                            for (int s1 = 0; s1 < 8; ++s1) sum += v[s1];
                         }
+                        if (n < a.N) store_y(a.y, a.y_bf16, (int64_t)m * a.N + n, sum);
+                    }
+                }
                 if (lane == 0) a.counters[p] = 0;
             }
         }
         u += j1 - j0;
+        first_segment = false;
     }
 
     int bad = 0;
@@ -499,6 +717,8 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1) gemv_kernel(GemvArgs a) {
 struct GemvPlan {
     int NT, MT, P, grid, warps_total, prep_grid;
     int64_t G, U, chunk;
+    bool bsmem;
+    size_t smem;
     size_t off_bslots, off_meta, off_counters, off_partials, total;
 };
 
@@ -516,19 +736,15 @@ static GemvPlan make_gemv_plan(int layout, int64_t M, int64_t N, int64_t K, int 
     const int64_t min_chunk = 4;
     int64_t warps_needed = (pl.U + min_chunk - 1) / min_chunk;
     if (warps_needed < 1) warps_needed = 1;
-    if (warps_needed >= max_warps) {
-        pl.grid = num_sms;
-    } else {
-        pl.grid = static_cast<int>((warps_needed + kGemvWarps - 1) / kGemvWarps);
-    }
+    pl.grid = warps_needed >= max_warps ? num_sms
+                                        : static_cast<int>((warps_needed + kGemvWarps - 1) / kGemvWarps);
     pl.warps_total = pl.grid * kGemvWarps;
     pl.chunk = (pl.U + pl.warps_total - 1) / pl.warps_total;
     if (pl.chunk < 1) pl.chunk = 1;
-    const int64_t nblocks = (pl.G + 7) / 8;
-    int64_t pg = (M * nblocks + kPrepWarps - 1) / kPrepWarps;
-    if (pg < 1) pg = 1;
-    if (pg > (int64_t)num_sms * 4) pg = (int64_t)num_sms * 4;
-    pl.prep_grid = static_cast<int>(pg);
+    pl.prep_grid = static_cast<int>(M * ((pl.G + 7) / 8));
+    const size_t bbytes = (size_t)M * pl.G * (pl.NT * 32 + 8);
+    pl.bsmem = M <= 8 && bbytes <= kBsmemMax;
+    pl.smem = (layout == BT_LAYOUT_B3 ? kLutBytes : 0) + kZeroBytes + (pl.bsmem ? bbytes : 0);
     size_t off = 0;
     pl.off_bslots = off;
     off = align_up(off + (size_t)M * pl.G * pl.NT * 32, 256);
@@ -546,23 +762,31 @@ size_t gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num
     return make_gemv_plan(layout, M, N, K, num_sms).total;
 }
 
-template <int LAYOUT, int MT>
+template <int LAYOUT, int MT, bool BSMEM, bool M1>
 static cudaError_t launch_gemv_t(const GemvArgs& ga, const GemvPlan& pl, cudaStream_t stream) {
-    const size_t smem = LAYOUT == BT_LAYOUT_B3 ? kLutBytes : 0;
-    cudaError_t e = cudaFuncSetAttribute(gemv_kernel<LAYOUT, MT>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    auto kern = gemv_kernel<LAYOUT, MT, BSMEM, M1>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)pl.smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(pl.grid);
     cfg.blockDim = dim3(kGemvWarps * 32);
-    cfg.dynamicSmemBytes = smem;
+    cfg.dynamicSmemBytes = pl.smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemv_kernel<LAYOUT, MT>, ga);
+    return cudaLaunchKernelEx(&cfg, kern, ga);
+}
+
+template <int LAYOUT>
+static cudaError_t dispatch_gemv(const GemvArgs& ga, const GemvPlan& pl, cudaStream_t s) {
+    if (ga.M == 1 && pl.bsmem) return launch_gemv_t<LAYOUT, 1, true, true>(ga, pl, s);
+    if (pl.MT == 1)
+        return pl.bsmem ? launch_gemv_t<LAYOUT, 1, true, false>(ga, pl, s)
+                        : launch_gemv_t<LAYOUT, 1, false, false>(ga, pl, s);
+    return launch_gemv_t<LAYOUT, 2, false, false>(ga, pl, s);
 }
 
 cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales, const void* x,
@@ -584,9 +808,9 @@ cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales
     pa.counters = reinterpret_cast<int*>(ws + pl.off_counters);
     pa.P = pl.P;
     if (layout == BT_LAYOUT_B3)
-        gemv_prep_kernel<BT_LAYOUT_B3><<<pl.prep_grid, kPrepWarps * 32, 0, stream>>>(pa);
+        gemv_prep_kernel<BT_LAYOUT_B3><<<pl.prep_grid, kPrepThreads, 0, stream>>>(pa);
     else
-        gemv_prep_kernel<BT_LAYOUT_2BIT><<<pl.prep_grid, kPrepWarps * 32, 0, stream>>>(pa);
+        gemv_prep_kernel<BT_LAYOUT_2BIT><<<pl.prep_grid, kPrepThreads, 0, stream>>>(pa);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
@@ -602,15 +826,12 @@ cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales
     ga.M = static_cast<int>(M);
     ga.N = static_cast<int>(N);
     ga.G = static_cast<int>(pl.G);
-    ga.row_bytes = (K / kGroup) * (layout == BT_LAYOUT_B3 ? kB3GroupBytes : k2bGroupBytes);
+    ga.row_bytes = static_cast<uint32_t>((K / kGroup) * (layout == BT_LAYOUT_B3 ? kB3GroupBytes : k2bGroupBytes));
     ga.U = pl.U;
     ga.chunk = pl.chunk;
     ga.dev_err = dev_err;
-    if (layout == BT_LAYOUT_B3)
-        return pl.MT == 1 ? launch_gemv_t<BT_LAYOUT_B3, 1>(ga, pl, stream)
-                          : launch_gemv_t<BT_LAYOUT_B3, 2>(ga, pl, stream);
-    return pl.MT == 1 ? launch_gemv_t<BT_LAYOUT_2BIT, 1>(ga, pl, stream)
-                      : launch_gemv_t<BT_LAYOUT_2BIT, 2>(ga, pl, stream);
+    return layout == BT_LAYOUT_B3 ? dispatch_gemv<BT_LAYOUT_B3>(ga, pl, stream)
+                                  : dispatch_gemv<BT_LAYOUT_2BIT>(ga, pl, stream);
 }
 
 }  // namespace bt
