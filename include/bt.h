@@ -140,6 +140,31 @@ bt_status bt_gemv(int layout, const uint8_t* codes, const uint16_t* scales,
                   void* workspace, size_t workspace_bytes, int32_t* dev_err, void* stream);
 
 /*
+ * bt_gemv_noalloc: bt_gemv for callers that cannot allocate device memory --
+ * code that runs where cudaMalloc is unavailable or not allowed (inside a
+ * custom allocator or memory-pool callback, in a runtime that has handed all
+ * device memory to its own arena, or under a fixed memory budget decided
+ * before the call). The paper has no counterpart; it is an interface
+ * convenience of this library.
+ * Arguments and results are those of bt_gemv without the workspace: the
+ * scratch is a 4 MiB array in the library's own device memory, reserved on
+ * every GPU that loads libbt.so until the process exits. Requests whose
+ * bt_gemv_workspace_bytes exceeds 4 MiB (for example M = 16 on 17408-row
+ * matrices) are rejected with BT_ERR_WORKSPACE before anything is launched.
+ * The first call on a device looks up the array's device address (once per
+ * device, with that device current); make that first call before any stream
+ * capture. All calls share the one array and it keeps the last call's
+ * contents (everything that must start at zero is cleared by the call), so
+ * calls that may overlap on the GPU -- on different streams, or from
+ * different host threads -- race and must be serialised by the caller.
+ * Never calls cudaMalloc, cudaFree or any allocating routine.
+ */
+bt_status bt_gemv_noalloc(int layout, const uint8_t* codes, const uint16_t* scales,
+                          const void* x, int x_dtype, const int8_t* sign1024,
+                          int64_t M, int64_t N, int64_t K, int y_dtype, void* y,
+                          int32_t* dev_err, void* stream);
+
+/*
  * bt_gemm: prefill path, Y = X' W^T with W = s * t decoded into FP16 tiles
  * in shared memory and multiplied on the tcgen05 tensor cores, FP32
  * accumulation, bf16 output [M][N] (round to nearest even).

@@ -30,7 +30,8 @@ DEVERR_TIMEOUT = 0x8
 # Exported entry points, as declared in include/bt.h.
 SYMBOLS = (
     "bt_status_string", "bt_version", "bt_codes_row_bytes", "bt_pack", "bt_unpack",
-    "bt_fwht1024", "bt_gemv_workspace_bytes", "bt_gemv", "bt_gemm_workspace_bytes", "bt_gemm",
+    "bt_fwht1024", "bt_gemv_workspace_bytes", "bt_gemv", "bt_gemv_noalloc", "bt_gemm_workspace_bytes",
+    "bt_gemm",
 )
 
 _lock = threading.Lock()
@@ -64,10 +65,11 @@ def load() -> ctypes.CDLL:
             lib.bt_gemv_workspace_bytes.argtypes = [I, I64, I64, I64]
             lib.bt_gemv_workspace_bytes.restype = SZ
             lib.bt_gemv.argtypes = [I, P, P, P, I, P, I64, I64, I64, I, P, P, SZ, P, P]
+            lib.bt_gemv_noalloc.argtypes = [I, P, P, P, I, P, I64, I64, I64, I, P, P, P]
             lib.bt_gemm_workspace_bytes.argtypes = [I, I64, I64, I64]
             lib.bt_gemm_workspace_bytes.restype = SZ
             lib.bt_gemm.argtypes = [I, P, P, P, I, P, I64, I64, I64, P, P, SZ, P, P]
-            for name in ("bt_pack", "bt_unpack", "bt_fwht1024", "bt_gemv", "bt_gemm"):
+            for name in ("bt_pack", "bt_unpack", "bt_fwht1024", "bt_gemv", "bt_gemv_noalloc", "bt_gemm"):
                 getattr(lib, name).restype = I
             _lib = lib
     return _lib
@@ -168,6 +170,25 @@ def gemv(codes: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, sign: torch
     _check("bt_gemv", load().bt_gemv(layout, _ptr(codes), _ptr(scales), _ptr(x), _x_dtype(x), _ptr(sign),
                                       M, N, K, y_dtype, _ptr(out), _ptr(ws), ws.numel(), _ptr(dev_err),
                                       _stream(x.device)))
+    return out
+
+
+def gemv_noalloc(codes: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, sign: torch.Tensor | None, N: int,
+                 layout: int = LAYOUT_B3, y_dtype: int = F32, out: torch.Tensor | None = None,
+                 dev_err: torch.Tensor | None = None) -> torch.Tensor:
+    """bt_gemv without a caller-provided workspace (scratch lives in libbt.so).
+
+    For callers that cannot allocate device memory at call time. Calls share
+    one 4 MiB scratch array per GPU: calls that may overlap on the GPU race.
+    `out` may be passed to avoid allocating the result here as well.
+    """
+    _require_cuda(codes, scales, x, sign, out, dev_err)
+    M, K = x.shape
+    if out is None:
+        out = torch.empty((M, N), dtype=torch.float32 if y_dtype == F32 else torch.bfloat16, device=x.device)
+    _check("bt_gemv_noalloc", load().bt_gemv_noalloc(layout, _ptr(codes), _ptr(scales), _ptr(x), _x_dtype(x),
+                                                      _ptr(sign), M, N, K, y_dtype, _ptr(out), _ptr(dev_err),
+                                                      _stream(x.device)))
     return out
 
 

@@ -12,6 +12,8 @@ size_t gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num
 cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales, const void* x,
                         int x_dtype, const int8_t* sign, int64_t M, int64_t N, int64_t K, int y_dtype,
                         void* y, void* workspace, int32_t* dev_err, int num_sms, cudaStream_t stream);
+size_t gemv_noalloc_max_bytes();
+cudaError_t gemv_noalloc_scratch(void** out);
 size_t gemm_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num_sms);
 cudaError_t launch_gemm(int layout, const uint8_t* codes, const uint16_t* scales, const void* x,
                         int x_dtype, const int8_t* sign, int64_t M, int64_t N, int64_t K, void* y,
@@ -148,6 +150,25 @@ bt_status bt_gemv(int layout, const uint8_t* codes, const uint16_t* scales, cons
     if (!aligned(workspace, 256)) return BT_ERR_ALIGN;
     return from_cuda(bt::launch_gemv(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y_dtype, y,
                                      workspace, dev_err, sms, s));
+}
+
+bt_status bt_gemv_noalloc(int layout, const uint8_t* codes, const uint16_t* scales, const void* x,
+                          int x_dtype, const int8_t* sign1024, int64_t M, int64_t N, int64_t K, int y_dtype,
+                          void* y, int32_t* dev_err, void* stream) {
+    bt_status st = check_product_args(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y);
+    if (st != BT_OK) return st;
+    if (!valid_dtype(y_dtype)) return BT_ERR_INVALID_ARG;
+    if (M > 16) return BT_ERR_SHAPE;
+    if (M == 0 || N == 0) return BT_OK;
+    if (!aligned(dev_err, 4)) return BT_ERR_ALIGN;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (K == 0) return from_cuda(launch_zero(y, M * N * (y_dtype == BT_BF16 ? 2 : 4), s));
+    const int sms = current_sm_count();
+    if (bt::gemv_workspace_bytes(layout, M, N, K, sms) > bt::gemv_noalloc_max_bytes()) return BT_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    if (bt::gemv_noalloc_scratch(&scratch) != cudaSuccess) { cudaGetLastError(); return BT_ERR_CUDA; }
+    return from_cuda(bt::launch_gemv(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y_dtype, y,
+                                     scratch, dev_err, sms, s));
 }
 
 size_t bt_gemm_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K) {

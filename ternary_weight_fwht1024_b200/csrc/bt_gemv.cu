@@ -35,6 +35,8 @@
 //     deterministic run to run.
 #include "bt_internal.cuh"
 
+#include <mutex>
+
 namespace bt {
 
 #ifndef BT_GEMV_WARPS
@@ -832,6 +834,38 @@ cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales
     ga.dev_err = dev_err;
     return layout == BT_LAYOUT_B3 ? dispatch_gemv<BT_LAYOUT_B3>(ga, pl, stream)
                                   : dispatch_gemv<BT_LAYOUT_2BIT>(ga, pl, stream);
+}
+
+// ------------------------------------------------ allocation-free variant ---
+//
+// Scratch for bt_gemv_noalloc: a fixed array in device memory, reserved by
+// every GPU that loads the library for as long as the process lives. Host
+// code only ever sees a stand-in for `noalloc_scratch`, so its device address
+// is looked up once per device with cudaGetSymbolAddress (with that device
+// current) and cached; the first call on a device does this lookup.
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
+static __device__ __align__(256) uint8_t noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+static std::mutex g_scratch_mutex;
+static void* g_scratch_ptr[kMaxDevices];
+
+size_t gemv_noalloc_max_bytes() { return kNoAllocScratchBytes; }
+
+cudaError_t gemv_noalloc_scratch(void** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_scratch_mutex);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, noalloc_scratch);
+        if (e != cudaSuccess) return e;
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return cudaSuccess;
 }
 
 }  // namespace bt
