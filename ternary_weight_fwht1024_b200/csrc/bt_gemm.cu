@@ -1,10 +1,598 @@
-// Prefill GEMM (placeholder until the tcgen05 kernel lands).
+// Prefill GEMM on the tcgen05 tensor cores: Y = X' W^T, M % 128 == 0.
+//
+// pp512 prompt processing (release summary of Ternary Bonsai 2 27B, section
+// 实测吞吐) is a dense contraction, so it runs on the 5th-generation tensor
+// cores with the packed weights decoded to FP16 tiles in shared memory and
+// never materialised in HBM (section 三值权重怎么压缩到 1.76 bit: unpack and
+// group scale fused inside the matrix product).
+//
+// Two kernels:
+//
+//  1. gemm_prep (one CTA per activation row): rotates the row block-wise
+//     (x' = H_1024 S x / 32, when a sign vector is given), picks a power of
+//     two 2^e_m from the row's largest |x'|, and writes x' * 2^-e_m as FP16 in
+//     the per-group slot order the weight decoder produces (below), plus
+//     2^e_m.
+//
+//  2. gemm: one 128 x BN output tile per CTA, one 128-wide K group per
+//     pipeline stage (two stages).
+//       warp 0      TMA: the activation tile (two 64-column panels, 128-byte
+//                   swizzle) into shared memory;
+//       warp 1      allocates TMEM, one elected thread issues
+//                   tcgen05.mma.cta_group::1.kind::f16 (M 128, N BN, K 16) x 8
+//                   per stage into an FP32 accumulator in TMEM and commits
+//                   each stage to its "empty" barrier;
+//       warps 2-9   decode the packed weights of the stage (one row per
+//                   thread) to FP16 s*t -- exact -- and store them in the
+//                   tensor cores' K-major 128-byte-swizzled layout; then
+//                   they read the accumulator back (tcgen05.ld) and write
+//                   bf16 Y scaled by 2^e_m.
+//     A group's 128 trits are laid out in "slot" order: slot 2w + h holds
+//     half h of decoded word w. For base-3, word w < 60 is digit w % 5 of
+//     bytes (2p, 2p+1), p = w / 5; words 60-62 are digits 0-2 of bytes
+//     (24, 25); word 63 is digits 3 and 4 of byte 24 (byte 25's digits 3
+//     and 4 are the group's two pad trits). For 2-bit, word 8q + f is trits
+//     f and 8 + f of the group's 32-bit word q. The activations are written
+//     in the same order, so the contraction over each group is unchanged.
+//     Decoding a word: OR the two digits' 2-bit fields into FP16 1024 + d 4^i
+//     (exact), one HFMA2 makes it d - 1 = t (exact), one HMUL2 makes s t.
+// Waits on barriers are bounded: a wait that runs out sets BT_DEVERR_TIMEOUT,
+// the CTA skips the rest of its work and still releases its TMEM.
 #include "bt_internal.cuh"
 
+#include <cuda.h>
+
 namespace bt {
-size_t gemm_workspace_bytes(int, int64_t M, int64_t, int64_t K, int) { return (size_t)M * K * 2 + 4096; }
-cudaError_t launch_gemm(int, const uint8_t*, const uint16_t*, const void*, int, const int8_t*, int64_t,
-                        int64_t, int64_t, void*, void*, int32_t*, int, cudaStream_t) {
-    return cudaErrorNotSupported;
+
+constexpr int kGemmBM = 128;
+constexpr int kGemmBK = 128;             // one weight group per stage
+constexpr int kGemmDecWarps = 8;         // decoder / epilogue warps
+constexpr int kGemmThreads = (2 + kGemmDecWarps) * 32;
+constexpr int kGemmLutBytes = 256 * 64;  // 8 copies x (low, high) x 4 bytes per code
+constexpr uint32_t kSpinLimit = 1u << 26;
+
+// ---------------------------------------------------------------- helpers ----
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
+}
+// Bounded wait on the given phase parity; false when the limit ran out.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    for (uint32_t it = 0; it < kSpinLimit; ++it) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+        if (ok) return true;
+    }
+    return false;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        :: "r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void fence_proxy_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row atoms
+// 1024 bytes apart (SBO), version 1 (Blackwell).
+__device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t addr) {
+    uint64_t d = 0;
+    d |= static_cast<uint64_t>((addr >> 4) & 0x3FFFu);
+    d |= static_cast<uint64_t>(1u) << 16;              // leading byte offset (unused for this layout) = 16 B
+    d |= static_cast<uint64_t>(1024u >> 4) << 32;      // stride byte offset
+    d |= static_cast<uint64_t>(1u) << 46;              // descriptor version
+    d |= static_cast<uint64_t>(2u) << 61;              // SWIZZLE_128B
+    return d;
+}
+
+// Instruction descriptor, kind::f16: FP16 A and B (both K-major), FP32 D.
+__host__ __device__ constexpr uint32_t idesc_f16(int M, int N) {
+    return (1u << 4)                                   // D format F32
+         | (0u << 7) | (0u << 10)                      // A, B format F16
+         | (static_cast<uint32_t>(N >> 3) << 17)
+         | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void tc_mma(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        :: "r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
+}
+__device__ __forceinline__ void tc_commit(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :: "r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+        "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]),
+          "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]),
+          "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c) {
+    uint32_t r;
+    asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
+    return r;
+}
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+    uint32_t r;
+    asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+__host__ __device__ constexpr uint32_t gfmask(int i) { return (3u << (2 * i)) | (3u << (2 * i + 16)); }
+
+// FP16 constants turning (1024 + d 4^i) into d - 1: multiply by 4^-i, add
+// -(1024 4^-i + 1); both are exact in FP16 for i <= 5.
+__device__ __forceinline__ uint32_t h2_mul_of(int i) {
+    const uint32_t h = __half_as_ushort(__float2half_rn(ldexpf(1.f, -2 * i)));
+    return h | (h << 16);
+}
+__device__ __forceinline__ uint32_t h2_add_of(int i) {
+    const uint32_t h = __half_as_ushort(__float2half_rn(-(ldexpf(1024.f, -2 * i) + 1.f)));
+    return h | (h << 16);
+}
+
+// ------------------------------------------------------------------ prep ----
+
+struct GemmPrepArgs {
+    const void* x;
+    int x_bf16;
+    const int8_t* sign;   // nullable: x already rotated
+    int M, K, G;
+    int layout;
+    __half* xt;           // [M][K] FP16, slot order within each group
+    float* rowscale;      // [M] 2^e_m
+};
+
+__device__ __forceinline__ int gemm_slot_k(int layout, int slot) {
+    const int w = slot >> 1, h = slot & 1;
+    if (layout == BT_LAYOUT_B3) {
+        if (w < 60) return 10 * (w / 5) + 5 * h + (w % 5);
+        if (w < 63) return 120 + 5 * h + (w - 60);
+        return 123 + h;
+    }
+    return 16 * (w >> 3) + 8 * h + (w & 7);
+}
+
+constexpr int kGemmPrepWarps = 8;
+
+__global__ void __launch_bounds__(kGemmPrepWarps * 32) gemm_prep_kernel(GemmPrepArgs a) {
+    extern __shared__ __align__(16) float rowbuf[];   // K floats, then tiles
+    float* tiles = rowbuf + a.K;                        // kGemmPrepWarps x 32 x 36
+    __shared__ float red[kGemmPrepWarps];
+    pdl_launch_dependents();
+    pdl_wait();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m = blockIdx.x;
+    const int nblocks = (a.K + kBlock - 1) / kBlock;
+    float amax = 0.f;
+    for (int b = warp; b < nblocks; b += kGemmPrepWarps) {
+        const int64_t k0 = (int64_t)b * kBlock;
+        float v[32];
+        if (a.sign) {
+            load_signed_bf16_block(reinterpret_cast<const uint16_t*>(a.x) + (int64_t)m * a.K + k0, a.sign, v);
+            fwht1024_warp(v, tiles + warp * 32 * kTileStride);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int64_t idx = k0 + 32 * j + lane;
+                float val = 0.f;
+                if (idx < a.K) {
+                    const int64_t off = (int64_t)m * a.K + idx;
+                    val = a.x_bf16 ? bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(a.x)[off])
+                                   : reinterpret_cast<const float*>(a.x)[off];
+                }
+                v[j] = val;
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const int64_t idx = k0 + 32 * j + lane;
+            if (idx < a.K) rowbuf[idx] = v[j];
+            amax = fmaxf(amax, fabsf(v[j]));
+        }
+    }
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, s));
+    if (lane == 0) red[warp] = amax;
+    __syncthreads();
+    amax = 0.f;
+    for (int w = 0; w < kGemmPrepWarps; ++w) amax = fmaxf(amax, red[w]);
+    // 2^e with max |x'| 2^-e < 2^15 keeps FP16 finite with margin
+    int e = amax > 0.f ? ilogbf(amax) + 1 - 15 : 0;
+    e = max(-110, min(110, e));
+    const float inv = __int_as_float((127 - e) << 23);
+    if (threadIdx.x == 0) a.rowscale[m] = __int_as_float((127 + e) << 23);
+    __half* dst = a.xt + (int64_t)m * a.K;
+    for (int idx = threadIdx.x; idx < a.K; idx += blockDim.x) {
+        const int g = idx >> 7, slot = idx & 127;
+        dst[idx] = __float2half_rn(rowbuf[g * kGroup + gemm_slot_k(a.layout, slot)] * inv);
+    }
+}
+
+// ------------------------------------------------------------------ GEMM ----
+
+struct GemmArgs {
+    const uint8_t* codes;
+    const uint16_t* scales;
+    const float* rowscale;
+    __nv_bfloat16* y;
+    int M, N, K, G;
+    int64_t row_bytes;
+    int32_t* dev_err;
+};
+
+template <int LAYOUT, int BN, int STAGES>
+struct GemmSmem {
+    static constexpr int kA = kGemmBM * kGemmBK * 2;   // 32 KB: two 64-column panels
+    static constexpr int kB = BN * kGemmBK * 2;
+    static constexpr int kStage = kA + kB;
+    static constexpr int kLut = LAYOUT == BT_LAYOUT_B3 ? kGemmLutBytes : 0;
+    static constexpr int kBars = 1024;                  // barriers, TMEM address, flags
+    static constexpr int kTotal = STAGES * kStage + kLut + kBars + 1024;  // + alignment slack
+};
+
+template <int LAYOUT, int BN, int STAGES>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
+    using SM = GemmSmem<LAYOUT, BN, STAGES>;
+    extern __shared__ uint8_t gsm_raw[];
+    uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* stages = base;
+    uint8_t* lut = base + STAGES * SM::kStage;
+    uint8_t* ctl = lut + SM::kLut;
+    uint64_t* full = reinterpret_cast<uint64_t*>(ctl);
+    uint64_t* empty = full + STAGES;
+    uint64_t* accf = empty + STAGES;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int m0 = blockIdx.y * kGemmBM, n0 = blockIdx.x * BN;
+    const int ktiles = a.G;
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(smem_addr(full + s), 1 + kGemmDecWarps);
+            mbar_init(smem_addr(empty + s), 1);
+        }
+        mbar_init(smem_addr(accf), 1);
+        *abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (LAYOUT == BT_LAYOUT_B3) {
+        // digits of each code as 2-bit fields, 8 copies per code (low table,
+        // then high table with the fields in the upper half)
+        for (int idx = threadIdx.x; idx < 256 * 16; idx += blockDim.x) {
+            const int code = idx >> 4, hi = (idx >> 3) & 1;
+            uint32_t f = 0x80000000u;
+            if (code < 243) {
+                f = 0;
+                int r = code;
+                for (int i = 0; i < 5; ++i) { f |= static_cast<uint32_t>(r % 3) << (2 * i); r /= 3; }
+                if (hi) f <<= 16;
+            }
+            reinterpret_cast<uint32_t*>(lut)[idx] = f;
+        }
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(smem_addr(tmem_slot)), "r"(BN <= 128 ? 128 : 256) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    pdl_wait();  // the activations come from the prep kernel
+
+    int bad = 0;
+    if (warp == 0) {
+        // ---------------- TMA producer: activation tiles
+        if (lane == 0) {
+            for (int kt = 0; kt < ktiles; ++kt) {
+                const int s = kt % STAGES;
+                if (kt >= STAGES && !mbar_wait(smem_addr(empty + s), ((kt / STAGES) - 1) & 1)) {
+                    bad = BT_DEVERR_TIMEOUT; *abort_flag = 1; break;
+                }
+                if (*abort_flag) break;
+                const uint32_t dst = smem_addr(stages + s * SM::kStage);
+                mbar_arrive_tx(smem_addr(full + s), SM::kA);
+                tma_load_2d(dst, &amap, kt * kGemmBK, m0, smem_addr(full + s));
+                tma_load_2d(dst + SM::kA / 2, &amap, kt * kGemmBK + 64, m0, smem_addr(full + s));
+            }
+        }
+    } else if (warp == 1) {
+        // ---------------- MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idesc = idesc_f16(kGemmBM, BN);
+            for (int kt = 0; kt < ktiles; ++kt) {
+                const int s = kt % STAGES;
+                if (!mbar_wait(smem_addr(full + s), (kt / STAGES) & 1)) {
+                    bad = BT_DEVERR_TIMEOUT; *abort_flag = 1; break;
+                }
+                if (*abort_flag) break;
+                tc_fence_after();
+                const uint32_t sa = smem_addr(stages + s * SM::kStage);
+                const uint32_t sb = sa + SM::kA;
+#pragma unroll
+                for (int k = 0; k < kGemmBK / 16; ++k) {
+                    const uint32_t pa = sa + (k >> 2) * (SM::kA / 2) + (k & 3) * 32;
+                    const uint32_t pb = sb + (k >> 2) * (SM::kB / 2) + (k & 3) * 32;
+                    tc_mma(tmem, smem_desc_sw128(pa), smem_desc_sw128(pb), idesc, (kt > 0 || k > 0) ? 1u : 0u);
+                }
+                tc_commit(smem_addr(empty + s));
+            }
+            tc_commit(smem_addr(accf));
+        }
+    } else {
+        // ---------------- decoders: one weight row per thread
+        const int t = threadIdx.x - 64;                 // 0 .. 255
+        const int n = n0 + t;
+        const bool active = t < BN;
+        const int nr = active ? n : n0;                 // rows beyond BN do no work
+        const uint8_t* rowp = a.codes + (int64_t)nr * a.row_bytes;
+        const uint16_t* srow = a.scales + (int64_t)nr * a.G;
+        const uint8_t* lut_lane = lut + (lane & 7) * 4;   // this lane's copy of the table
+        uint32_t hm[6], ha[6];
+#pragma unroll
+        for (int i = 0; i < 6; ++i) { hm[i] = h2_mul_of(i); ha[i] = h2_add_of(i); }
+        const uint32_t hm34 = (hm[3] & 0xFFFFu) | (hm[4] & 0xFFFF0000u);
+        const uint32_t ha34 = (ha[3] & 0xFFFFu) | (ha[4] & 0xFFFF0000u);
+        uint32_t err = 0;
+        for (int kt = 0; kt < ktiles; ++kt) {
+            const int s = kt % STAGES;
+            if (kt >= STAGES && !mbar_wait(smem_addr(empty + s), ((kt / STAGES) - 1) & 1)) {
+                bad = BT_DEVERR_TIMEOUT; *abort_flag = 1; break;
+            }
+            if (*abort_flag) break;
+            if (active) {
+                const uint32_t s1 = srow[kt];
+                const uint32_t s2 = s1 | (s1 << 16);
+                uint8_t* bst = stages + s * SM::kStage + SM::kA;
+                // row t of the B tile: panel p (slots 64p..64p+63), 8-row atoms
+                const uint32_t row_off = static_cast<uint32_t>((t >> 3) * 1024 + (t & 7) * 128);
+                uint32_t words[64];
+                if constexpr (LAYOUT == BT_LAYOUT_B3) {
+                    const uint8_t* gp = rowp + (int64_t)kt * kB3GroupBytes;
+#pragma unroll
+                    for (int p = 0; p < 13; ++p) {
+                        const uint32_t pr = __ldg(reinterpret_cast<const unsigned short*>(gp + 2 * p));
+                        const uint32_t va = *reinterpret_cast<const uint32_t*>(lut_lane + (pr & 0xFFu) * 64u);
+                        const uint32_t vb = *reinterpret_cast<const uint32_t*>(lut_lane + (pr >> 8) * 64u + 32u);
+                        err |= va | vb;
+                        const int nw = p < 12 ? 5 : 3;
+#pragma unroll
+                        for (int i = 0; i < nw; ++i) {
+                            const uint32_t f = lop3_or_and(va, vb, gfmask(i)) | 0x64006400u;
+                            words[5 * p + i] = hmul2_u32(hfma2_u32(f, hm[i], ha[i]), s2);
+                        }
+                        if (p == 12) {
+                            const uint32_t f = (va & 0x0C0u) | ((va & 0x300u) << 16) | 0x64006400u;
+                            words[63] = hmul2_u32(hfma2_u32(f, hm34, ha34), s2);
+                        }
+                    }
+                } else {
+                    const uint4* gp = reinterpret_cast<const uint4*>(rowp + (int64_t)kt * k2bGroupBytes);
+                    const uint4 q0 = __ldg(gp), q1 = __ldg(gp + 1);
+                    const uint32_t q[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+                    for (int w = 0; w < 8; ++w) {
+                        // fields 0-4 of each half in place, fields 5-7 after a
+                        // 10-bit shift: a field at bits 10-11 would reach into
+                        // the FP16 exponent of 1024 + d 4^i
+                        const uint32_t x = q[w], x10 = x >> 10;
+                        err |= x & (x >> 1) & 0x55555555u;
+#pragma unroll
+                        for (int f = 0; f < 8; ++f) {
+                            const uint32_t fl = (f < 5 ? (x & gfmask(f)) : (x10 & gfmask(f - 5))) | 0x64006400u;
+                            const int i = f < 5 ? f : f - 5;
+                            words[8 * w + f] = hmul2_u32(hfma2_u32(fl, hm[i], ha[i]), s2);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int c = 0; c < 16; ++c) {
+                    const int panel = c >> 3, chunk = c & 7;
+                    uint8_t* dst = bst + panel * (SM::kB / 2) + row_off + ((chunk ^ (t & 7)) << 4);
+                    *reinterpret_cast<uint4*>(dst) =
+                        make_uint4(words[4 * c], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
+                }
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(smem_addr(full + s));
+        }
+        if (LAYOUT == BT_LAYOUT_B3 ? (err >> 31) : (err != 0)) bad |= BT_DEVERR_INVALID_CODE;
+
+        // ---------------- epilogue: TMEM -> bf16 Y (rows m0 + 32 (warp % 4) + lane)
+        if (!*abort_flag && !mbar_wait(smem_addr(accf), 0)) { bad |= BT_DEVERR_TIMEOUT; *abort_flag = 1; }
+        tc_fence_after();
+        const int quarter = warp & 3;
+        const bool do_epi = warp >= 2 && warp < 6 && !*abort_flag;   // one warp per TMEM lane quarter
+        if (do_epi) {
+            const int m = m0 + quarter * 32 + lane;
+            const float rs = a.rowscale[m];
+#pragma unroll 1
+            for (int c0 = 0; c0 < BN; c0 += 32) {
+                uint32_t r[32];
+                tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + c0, r);
+                uint32_t packed[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[2 * j]) * rs,
+                                                                    __uint_as_float(r[2 * j + 1]) * rs);
+                    packed[j] = *reinterpret_cast<const uint32_t*>(&b2);
+                }
+                uint4* out = reinterpret_cast<uint4*>(a.y + (int64_t)m * a.N + n0 + c0);
+#pragma unroll
+                for (int v = 0; v < 4; ++v)
+                    out[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+            }
+        }
+    }
+    bad = __reduce_or_sync(0xffffffffu, bad);
+    if (lane == 0) report(a.dev_err, bad);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
+                     :: "r"(tmem), "r"(BN <= 128 ? 128 : 256) : "memory");
+    }
+}
+
+// ------------------------------------------------------------------ host ----
+
+static size_t gemm_align(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+size_t gemm_workspace_bytes(int, int64_t M, int64_t, int64_t K, int) {
+    return gemm_align((size_t)M * K * 2, 256) + gemm_align((size_t)M * 4, 256);
+}
+
+static int pick_bn(int64_t M, int64_t N, int num_sms) {
+    const int cands[5] = {256, 224, 192, 160, 128};
+    int best = 128;
+    double best_eff = -1.0;
+    for (int bn : cands) {
+        if (N % bn) continue;
+        const int64_t tiles = (M / kGemmBM) * (N / bn);
+        const int64_t waves = (tiles + num_sms - 1) / num_sms;
+        const double eff = (double)tiles / (double)(waves * num_sms);
+        if (eff > best_eff + 1e-9) { best_eff = eff; best = bn; }
+    }
+    return best;
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    }
+    return fn;
+}
+
+template <int LAYOUT, int BN, int STAGES>
+static cudaError_t launch_gemm_t(const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t stream) {
+    using SM = GemmSmem<LAYOUT, BN, STAGES>;
+    auto kern = gemm_kernel<LAYOUT, BN, STAGES>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kTotal);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(ga.N / BN, ga.M / kGemmBM);
+    cfg.blockDim = dim3(kGemmThreads);
+    cfg.dynamicSmemBytes = SM::kTotal;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, amap, ga);
+}
+
+template <int LAYOUT>
+static cudaError_t dispatch_gemm(int bn, const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t s) {
+    switch (bn) {
+        case 256: return launch_gemm_t<LAYOUT, 256, 2>(amap, ga, s);
+        case 224: return launch_gemm_t<LAYOUT, 224, 2>(amap, ga, s);
+        case 192: return launch_gemm_t<LAYOUT, 192, 2>(amap, ga, s);
+        case 160: return launch_gemm_t<LAYOUT, 160, 2>(amap, ga, s);
+        default: return launch_gemm_t<LAYOUT, 128, 3>(amap, ga, s);
+    }
+}
+
+cudaError_t launch_gemm(int layout, const uint8_t* codes, const uint16_t* scales, const void* x, int x_dtype,
+                        const int8_t* sign, int64_t M, int64_t N, int64_t K, void* y, void* workspace,
+                        int32_t* dev_err, int num_sms, cudaStream_t stream) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return cudaErrorNotSupported;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    __half* xt = reinterpret_cast<__half*>(ws);
+    float* rowscale = reinterpret_cast<float*>(ws + gemm_align((size_t)M * K * 2, 256));
+
+    GemmPrepArgs pa{};
+    pa.x = x;
+    pa.x_bf16 = x_dtype == BT_BF16;
+    pa.sign = sign;
+    pa.M = static_cast<int>(M);
+    pa.K = static_cast<int>(K);
+    pa.G = static_cast<int>(K / kGroup);
+    pa.layout = layout;
+    pa.xt = xt;
+    pa.rowscale = rowscale;
+    const size_t prep_smem = (size_t)K * 4 + (size_t)kGemmPrepWarps * 32 * kTileStride * 4;
+    cudaError_t e = cudaFuncSetAttribute(gemm_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)prep_smem);
+    if (e != cudaSuccess) return e;
+    gemm_prep_kernel<<<static_cast<unsigned>(M), kGemmPrepWarps * 32, prep_smem, stream>>>(pa);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+
+    CUtensorMap amap;
+    const cuuint64_t gdim[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+    const cuuint64_t gstride[1] = {static_cast<cuuint64_t>(K) * 2};
+    const cuuint32_t box[2] = {64, kGemmBM};
+    const cuuint32_t estride[2] = {1, 1};
+    if (enc(&amap, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, xt, gdim, gstride, box, estride,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return cudaErrorInvalidValue;
+
+    GemmArgs ga{};
+    ga.codes = codes;
+    ga.scales = scales;
+    ga.rowscale = rowscale;
+    ga.y = static_cast<__nv_bfloat16*>(y);
+    ga.M = static_cast<int>(M);
+    ga.N = static_cast<int>(N);
+    ga.K = static_cast<int>(K);
+    ga.G = static_cast<int>(K / kGroup);
+    ga.row_bytes = (K / kGroup) * (layout == BT_LAYOUT_B3 ? kB3GroupBytes : k2bGroupBytes);
+    ga.dev_err = dev_err;
+    const int bn = pick_bn(M, N, num_sms);
+    return layout == BT_LAYOUT_B3 ? dispatch_gemm<BT_LAYOUT_B3>(bn, amap, ga, stream)
+                                  : dispatch_gemm<BT_LAYOUT_2BIT>(bn, amap, ga, stream);
+}
+
 }  // namespace bt

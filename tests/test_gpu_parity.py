@@ -205,3 +205,73 @@ def test_gemv_flags_invalid_codes(layout):
     torch.cuda.synchronize()
     assert int(err.item()) & bt.DEVERR_INVALID_CODE
     assert torch.isfinite(y).all()
+
+
+# ---------------------------------------------------------------- GEMM ----
+
+def run_gemm(trits, scales, x_bits, sign, layout=bt.LAYOUT_B3, x_f32=None):
+    codes = bt.pack(T(trits), layout)
+    if x_f32 is None:
+        x = T(x_bits, "bf16")
+        sg = T(sign)
+    else:
+        x = torch.from_numpy(x_f32.astype(np.float32)).to(DEV)
+        sg = None
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    y = bt.gemm(codes, T(scales), x, sg, trits.shape[0], layout, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    return f64(y)
+
+
+@pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
+@pytest.mark.parametrize("M,N,K", [(128, 256, 1024), (256, 384, 2048), (128, 128, 3072)])
+def test_gemm_small_full(layout, M, N, K):
+    case = workloads.random_case(8000 + N + K, M, N, K)
+    _, y_ref, b = oracle.forward(case["trits"], case["scales"], case["x"], case["sign"])
+    y = run_gemm(case["trits"], case["scales"], case["x"], case["sign"], layout)
+    check(y, y_ref, b, extra=np.abs(y_ref) * 2.0 ** -8)
+
+
+@pytest.mark.parametrize("idx,layer", list(enumerate(workloads.TRIPLE)))
+def test_gemm_prefill_triple_sampled_rows(idx, layer):
+    # the pp512 shapes at full N and K; the oracle computes 8 sampled rows of Y
+    case = workloads.layer_inputs("C3", layer, index=idx)
+    y = run_gemm(case["trits"], case["scales"], case["x"], case["sign"])
+    rows = np.sort(workloads.rng(9000 + idx).choice(512, size=8, replace=False))
+    xr = oracle.rotate_bf16(case["x"][rows], case["sign"])
+    y_ref, b = oracle.gemv(case["trits"], case["scales"], xr)
+    check(y[rows], y_ref, b, extra=np.abs(y_ref) * 2.0 ** -8)
+
+
+def test_gemm_2bit_prefill_shape_sampled():
+    layer = workloads.TRIPLE[0]
+    case = workloads.layer_inputs("C4", layer, M=512, index=0)
+    y = run_gemm(case["trits"], case["scales"], case["x"], case["sign"], bt.LAYOUT_2BIT)
+    rows = np.array([0, 77, 300, 511])
+    xr = oracle.rotate_bf16(case["x"][rows], case["sign"])
+    y_ref, b = oracle.gemv(case["trits"], case["scales"], xr)
+    check(y[rows], y_ref, b, extra=np.abs(y_ref) * 2.0 ** -8)
+
+
+@pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
+def test_gemm_prerotated_ragged_blocks(layout):
+    M, N, K = 128, 256, 1152
+    case = workloads.random_case(8500, M, N, K)
+    xr = workloads.rng(8501).standard_normal((M, K)) * 2.0
+    xr32 = xr.astype(np.float32).astype(np.float64)
+    y_ref, b = oracle.gemv(case["trits"], case["scales"], xr32)
+    y = run_gemm(case["trits"], case["scales"], None, None, layout, x_f32=xr32)
+    check(y, y_ref, b, extra=np.abs(y_ref) * 2.0 ** -8)
+
+
+def test_gemm_special_cases():
+    M, N, K = 128, 128, 1024
+    case = workloads.random_case(8600, M, N, K)
+    z = np.zeros_like(case["trits"])
+    y0 = run_gemm(z, case["scales"], case["x"], case["sign"])
+    assert np.all(y0 == 0)
+    z[3, 999] = -1
+    _, y_ref, b = oracle.forward(z, case["scales"], case["x"], case["sign"])
+    y1 = run_gemm(z, case["scales"], case["x"], case["sign"])
+    check(y1, y_ref, b, extra=np.abs(y_ref) * 2.0 ** -8)
