@@ -40,51 +40,16 @@
 // the CTA skips the rest of its work and still releases its TMEM.
 #include "bt_internal.cuh"
 
-#include <cuda.h>
-
 namespace bt {
 
 constexpr int kGemmBM = 128;
 constexpr int kGemmBK = 128;             // one weight group per stage
 constexpr int kGemmDecWarps = 8;         // decoder / epilogue warps
 constexpr int kGemmThreads = (2 + kGemmDecWarps) * 32;
-constexpr int kGemmLutBytes = 256 * 64;  // 8 copies x (low, high) x 4 bytes per code
-constexpr uint32_t kSpinLimit = 1u << 26;
+constexpr int kGemmLutCopies = 16;
+constexpr int kGemmLutBytes = 256 * kGemmLutCopies * 8;  // 16 copies x (low, high) x 4 bytes per code
 
 // ---------------------------------------------------------------- helpers ----
-
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(bar), "r"(count) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" :: "r"(bar) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive_tx(uint32_t bar, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
-}
-// Bounded wait on the given phase parity; false when the limit ran out.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
-    for (uint32_t it = 0; it < kSpinLimit; ++it) {
-        uint32_t ok;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
-        if (ok) return true;
-    }
-    return false;
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
-        :: "r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar) : "memory");
-}
 
 __device__ __forceinline__ void fence_proxy_async_smem() {
     asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -295,10 +260,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (LAYOUT == BT_LAYOUT_B3) {
-        // digits of each code as 2-bit fields, 8 copies per code (low table,
+        // digits of each code as 2-bit fields, 16 copies per code (low table,
         // then high table with the fields in the upper half)
-        for (int idx = threadIdx.x; idx < 256 * 16; idx += blockDim.x) {
-            const int code = idx >> 4, hi = (idx >> 3) & 1;
+        for (int idx = threadIdx.x; idx < 256 * 2 * kGemmLutCopies; idx += blockDim.x) {
+            const int code = idx / (2 * kGemmLutCopies), hi = (idx / kGemmLutCopies) & 1;
             uint32_t f = 0x80000000u;
             if (code < 243) {
                 f = 0;
@@ -366,33 +331,52 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
         const int nr = active ? n : n0;                 // rows beyond BN do no work
         const uint8_t* rowp = a.codes + (int64_t)nr * a.row_bytes;
         const uint16_t* srow = a.scales + (int64_t)nr * a.G;
-        const uint8_t* lut_lane = lut + (lane & 7) * 4;   // this lane's copy of the table
+        const uint8_t* lut_lane = lut + (lane & (kGemmLutCopies - 1)) * 4;   // this lane's copy of the table
+        constexpr uint32_t kRow = 8 * kGemmLutCopies;                         // table bytes per code
         uint32_t hm[6], ha[6];
 #pragma unroll
         for (int i = 0; i < 6; ++i) { hm[i] = h2_mul_of(i); ha[i] = h2_add_of(i); }
         const uint32_t hm34 = (hm[3] & 0xFFFFu) | (hm[4] & 0xFFFF0000u);
         const uint32_t ha34 = (ha[3] & 0xFFFFu) | (ha[4] & 0xFFFF0000u);
         uint32_t err = 0;
+        // the next group's packed bytes and scale are loaded one stage ahead
+        constexpr int NW = LAYOUT == BT_LAYOUT_B3 ? 13 : 8;
+        uint32_t cur[NW], nxt[NW], s_cur = 0, s_nxt = 0;
+        auto load_group = [&](int kt, uint32_t (&dst)[NW], uint32_t& sc) {
+            if (!active || kt >= ktiles) return;
+            if constexpr (LAYOUT == BT_LAYOUT_B3) {
+                const unsigned short* gp = reinterpret_cast<const unsigned short*>(rowp + (int64_t)kt * kB3GroupBytes);
+#pragma unroll
+                for (int p = 0; p < 13; ++p) dst[p] = __ldg(gp + p);
+            } else {
+                const uint4* gp = reinterpret_cast<const uint4*>(rowp + (int64_t)kt * k2bGroupBytes);
+                const uint4 q0 = __ldg(gp), q1 = __ldg(gp + 1);
+                dst[0] = q0.x; dst[1] = q0.y; dst[2] = q0.z; dst[3] = q0.w;
+                dst[4] = q1.x; dst[5] = q1.y; dst[6] = q1.z; dst[7] = q1.w;
+            }
+            sc = srow[kt];
+        };
+        load_group(0, cur, s_cur);
         for (int kt = 0; kt < ktiles; ++kt) {
             const int s = kt % STAGES;
+            load_group(kt + 1, nxt, s_nxt);
             if (kt >= STAGES && !mbar_wait(smem_addr(empty + s), ((kt / STAGES) - 1) & 1)) {
                 bad = BT_DEVERR_TIMEOUT; *abort_flag = 1; break;
             }
             if (*abort_flag) break;
             if (active) {
-                const uint32_t s1 = srow[kt];
+                const uint32_t s1 = s_cur;
                 const uint32_t s2 = s1 | (s1 << 16);
                 uint8_t* bst = stages + s * SM::kStage + SM::kA;
                 // row t of the B tile: panel p (slots 64p..64p+63), 8-row atoms
                 const uint32_t row_off = static_cast<uint32_t>((t >> 3) * 1024 + (t & 7) * 128);
                 uint32_t words[64];
                 if constexpr (LAYOUT == BT_LAYOUT_B3) {
-                    const uint8_t* gp = rowp + (int64_t)kt * kB3GroupBytes;
 #pragma unroll
                     for (int p = 0; p < 13; ++p) {
-                        const uint32_t pr = __ldg(reinterpret_cast<const unsigned short*>(gp + 2 * p));
-                        const uint32_t va = *reinterpret_cast<const uint32_t*>(lut_lane + (pr & 0xFFu) * 64u);
-                        const uint32_t vb = *reinterpret_cast<const uint32_t*>(lut_lane + (pr >> 8) * 64u + 32u);
+                        const uint32_t pr = cur[p];
+                        const uint32_t va = *reinterpret_cast<const uint32_t*>(lut_lane + (pr & 0xFFu) * kRow);
+                        const uint32_t vb = *reinterpret_cast<const uint32_t*>(lut_lane + (pr >> 8) * kRow + kRow / 2);
                         err |= va | vb;
                         const int nw = p < 12 ? 5 : 3;
 #pragma unroll
@@ -406,15 +390,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
                         }
                     }
                 } else {
-                    const uint4* gp = reinterpret_cast<const uint4*>(rowp + (int64_t)kt * k2bGroupBytes);
-                    const uint4 q0 = __ldg(gp), q1 = __ldg(gp + 1);
-                    const uint32_t q[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
 #pragma unroll
                     for (int w = 0; w < 8; ++w) {
                         // fields 0-4 of each half in place, fields 5-7 after a
                         // 10-bit shift: a field at bits 10-11 would reach into
                         // the FP16 exponent of 1024 + d 4^i
-                        const uint32_t x = q[w], x10 = x >> 10;
+                        const uint32_t x = cur[w], x10 = x >> 10;
                         err |= x & (x >> 1) & 0x55555555u;
 #pragma unroll
                         for (int f = 0; f < 8; ++f) {
@@ -432,6 +413,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
                         make_uint4(words[4 * c], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
                 }
             }
+#pragma unroll
+            for (int i = 0; i < NW; ++i) cur[i] = nxt[i];
+            s_cur = s_nxt;
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_addr(full + s));
@@ -496,22 +480,6 @@ static int pick_bn(int64_t M, int64_t N, int num_sms) {
     return best;
 }
 
-typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-static EncodeTiledFn encode_fn() {
-    static EncodeTiledFn fn = nullptr;
-    if (!fn) {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<EncodeTiledFn>(p);
-    }
-    return fn;
-}
-
 template <int LAYOUT, int BN, int STAGES>
 static cudaError_t launch_gemm_t(const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t stream) {
     using SM = GemmSmem<LAYOUT, BN, STAGES>;
@@ -545,7 +513,7 @@ static cudaError_t dispatch_gemm(int bn, const CUtensorMap& amap, const GemmArgs
 cudaError_t launch_gemm(int layout, const uint8_t* codes, const uint16_t* scales, const void* x, int x_dtype,
                         const int8_t* sign, int64_t M, int64_t N, int64_t K, void* y, void* workspace,
                         int32_t* dev_err, int num_sms, cudaStream_t stream) {
-    EncodeTiledFn enc = encode_fn();
+    EncodeTiledFn enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
     uint8_t* ws = static_cast<uint8_t*>(workspace);
     __half* xt = reinterpret_cast<__half*>(ws);

@@ -508,20 +508,18 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1) gemv_kernel(GemvArgs a) {
         // table row = code (256 B): [0,128) low table, [128,256) high table,
         // one 4-byte entry per lane. Entry: the five digits as 2-bit fields
         // at bits 2i (low) or 16 + 2i (high); bit 31 flags codes >= 243.
-        for (int code = threadIdx.x; code < 256; code += blockDim.x) {
+        // consecutive threads fill consecutive 16-byte chunks (conflict-free)
+        for (int idx = threadIdx.x; idx < 256 * 16; idx += blockDim.x) {
+            const int code = idx >> 4, v = idx & 15;
             uint32_t f = 0x80000000u;
             if (code < 243) {
                 f = 0;
                 int r = code;
 #pragma unroll
                 for (int i = 0; i < 5; ++i) { f |= static_cast<uint32_t>(r % 3) << (2 * i); r /= 3; }
+                if (v >= 8) f <<= 16;
             }
-            const uint32_t fh = code < 243 ? (f << 16) : f;
-            uint4* row = reinterpret_cast<uint4*>(lut + code * 256);
-#pragma unroll
-            for (int v = 0; v < 8; ++v) row[v] = make_uint4(f, f, f, f);
-#pragma unroll
-            for (int v = 8; v < 16; ++v) row[v] = make_uint4(fh, fh, fh, fh);
+            reinterpret_cast<uint4*>(lut)[idx] = make_uint4(f, f, f, f);
         }
     }
     const uint32_t zero_area = smem_u32addr(sB);
@@ -714,6 +712,392 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1) gemv_kernel(GemvArgs a) {
     if (lane == 0) report(a.dev_err, bad);
 }
 
+// ----------------------------------------------- GEMV, TMA-fed variant -----
+//
+// Used when K % 1024 == 0 and M <= 8. Work item = (64-row tile quad Q,
+// 1024-block b). One producer warp streams each item's packed bytes
+// ([64 rows][RB bytes], RB = 208 base-3 or 256 2-bit) and scales
+// ([64 rows][8]) into a ring of shared-memory stages with 2D tensor copies,
+// well ahead of use. Sixteen consumer warps split the item: warp w decodes
+// group w % 8 of the block for the 32 rows of tile pair w / 8 (two 16-row
+// tiles, two independent MMA chains sharing one set of activation
+// fragments), so no warp waits on HBM. Each CTA owns a contiguous run of
+// items; a tile quad's partial sums are reduced through shared memory in a
+// fixed order, and a quad split across CTAs is finished by the CTA that
+// completes it last (atomic counter), in segment order.
+
+constexpr int kTmaConsumers = 16;
+constexpr int kTmaThreads = (kTmaConsumers + 1) * 32;
+constexpr int kTmaRows = 64;
+constexpr int kRedBytes = kTmaConsumers * 32 * 8 * 4;   // [warp][32 rows][8 cols] floats
+
+// The five base-3 digits of every byte value as 2-bit fields (bit 31 marks
+// values >= 243), the source of the shared-memory table.
+struct B3FieldTable {
+    uint32_t v[256];
+    constexpr B3FieldTable() : v() {
+        for (int code = 0; code < 256; ++code) {
+            uint32_t f = 0x80000000u;
+            if (code < 243) {
+                f = 0;
+                int r = code;
+                for (int i = 0; i < 5; ++i) { f |= static_cast<uint32_t>(r % 3) << (2 * i); r /= 3; }
+            }
+            v[code] = f;
+        }
+    }
+};
+__constant__ B3FieldTable c_b3_fields = B3FieldTable();
+
+struct GemvTmaArgs {
+    const uint32_t* bslots;
+    const float2* meta;
+    float* partials;         // [grid][2][64][M]
+    int* counters;           // [quads]
+    void* y;
+    int y_bf16;
+    int M, N, G, nb, stages;
+    int64_t items;           // quads * nb
+    int64_t chunk;           // items per CTA
+    int32_t* dev_err;
+};
+
+template <int LAYOUT>
+struct TmaGeom {
+    static constexpr int RB = LAYOUT == BT_LAYOUT_B3 ? 8 * kB3GroupBytes : 8 * k2bGroupBytes;  // 208 / 256
+    static constexpr int kCodes = kTmaRows * RB;
+    static constexpr int kScales = kTmaRows * 16;
+    static constexpr int kStage = kCodes + kScales;
+};
+
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+    uint16_t r;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(r) : "r"(addr));
+    return r;
+}
+
+__device__ __forceinline__ void consumer_bar() {
+    asm volatile("bar.sync 1, %0;" :: "n"(kTmaConsumers * 32) : "memory");
+}
+
+template <int LAYOUT, bool BSMEM, bool M1>
+__global__ void __launch_bounds__(kTmaThreads, 1)
+gemv_tma_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant__ CUtensorMap smap, GemvTmaArgs a) {
+    using GE = TmaGeom<LAYOUT>;
+    constexpr int NT = LAYOUT == BT_LAYOUT_B3 ? kB3Mmas : k2bMmas;
+    const int S = a.stages;
+    uint8_t* smem = gemv_smem;
+    uint8_t* lut = smem;
+    uint8_t* sB = smem + (LAYOUT == BT_LAYOUT_B3 ? kLutBytes : 0);
+    const int M = a.M, G = a.G, nb = a.nb;
+    const uint32_t bbytes = BSMEM ? static_cast<uint32_t>(M * G * (NT * 32 + 8)) : 0u;
+    uint8_t* stages = sB + ((kZeroBytes + bbytes + 1023) & ~1023u);
+    float* red = reinterpret_cast<float*>(stages + S * GE::kStage);
+    uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red) + kRedBytes);
+    uint64_t* empty = full + S;
+    volatile int* flags = reinterpret_cast<volatile int*>(empty + S);   // [0] abort, [1] last-segment vote
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t i0 = (int64_t)blockIdx.x * a.chunk;
+    const int64_t i1 = min(a.items, i0 + a.chunk);
+    const int nitems = static_cast<int>(i1 > i0 ? i1 - i0 : 0);
+    const int Q0 = static_cast<int>(i0 / nb), b0 = static_cast<int>(i0 % nb);
+
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < S; ++s) {
+            mbar_init(smem_addr(full + s), 1);
+            mbar_init(smem_addr(empty + s), kTmaConsumers);
+        }
+        flags[0] = 0;
+        flags[1] = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if constexpr (LAYOUT == BT_LAYOUT_B3) {
+        for (int idx = threadIdx.x; idx < 256 * 16; idx += blockDim.x) {
+            const int code = idx >> 4, v = idx & 15;
+            uint32_t f = c_b3_fields.v[code];
+            if (v >= 8 && code < 243) f <<= 16;
+            reinterpret_cast<uint4*>(lut)[idx] = make_uint4(f, f, f, f);
+        }
+    }
+    for (int i = threadIdx.x; i < kZeroBytes / 16; i += blockDim.x)
+        reinterpret_cast<uint4*>(sB)[i] = make_uint4(0, 0, 0, 0);
+    __syncthreads();
+
+    int bad = 0;
+    if (warp == kTmaConsumers) {
+        // ---------------- producer: the weights do not depend on the previous
+        // kernel, so streaming starts before the dependency wait
+        if (lane == 0) {
+            int Q = Q0, b = b0;
+            for (int it = 0; it < nitems; ++it) {
+                const int s = it % S;
+                if (it >= S && !mbar_wait(smem_addr(empty + s), ((it / S) - 1) & 1)) {
+                    bad = BT_DEVERR_TIMEOUT; flags[0] = 1; break;
+                }
+                if (flags[0]) break;
+                const uint32_t dst = smem_addr(stages + s * GE::kStage);
+                mbar_arrive_tx(smem_addr(full + s), GE::kStage);
+                tma_load_2d(dst, &cmap, b * GE::RB, Q * kTmaRows, smem_addr(full + s));
+                tma_load_2d(dst + GE::kCodes, &smap, b * 8, Q * kTmaRows, smem_addr(full + s));
+                if (++b == nb) { b = 0; ++Q; }
+            }
+        }
+        pdl_wait();
+    } else {
+        // ---------------- consumers
+        const int q = warp & 7, h = warp >> 3;
+        const int g = lane >> 2, c = lane & 3;
+        pdl_wait();
+        if constexpr (BSMEM) {
+            float2* smeta = reinterpret_cast<float2*>(sB + kZeroBytes);
+            for (int i = threadIdx.x; i < M * G; i += kTmaConsumers * 32) smeta[i] = __ldcg(a.meta + i);
+            const uint4* gb = reinterpret_cast<const uint4*>(a.bslots);
+            uint4* sb = reinterpret_cast<uint4*>(sB + kZeroBytes + M * G * 8);
+            const int n16 = M * G * NT * 2;
+            for (int base = 0; base < n16; base += 8 * kTmaConsumers * 32) {
+                uint4 v[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int i = base + u * kTmaConsumers * 32 + threadIdx.x;
+                    if (i < n16) v[u] = __ldcg(gb + i);
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int i = base + u * kTmaConsumers * 32 + threadIdx.x;
+                    if (i < n16) sb[i] = v[u];
+                }
+            }
+            consumer_bar();
+        }
+        const uint32_t zero_area = smem_u32addr(sB);
+        const uint32_t meta_area = zero_area + kZeroBytes;
+        const uint32_t slot_area = meta_area + static_cast<uint32_t>(M * G * 8);
+        const int m = g;                                  // activation row of this lane's fragment column
+        const bool okm = m < M;
+        const uint32_t bbase = okm ? slot_area + static_cast<uint32_t>(m * G * NT * 32 + c * 8) : zero_area + c * 8;
+        const uint32_t bstride = okm ? NT * 32 : 0;
+        uint32_t mbase[2], mstride[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int mm = 2 * c + r;
+            const bool ok = mm < M;
+            mbase[r] = ok ? meta_area + static_cast<uint32_t>(mm * G * 8) : zero_area;
+            mstride[r] = ok ? 8 : 0;
+        }
+        uint32_t mq[3];
+        mq[0] = (c & 1) ? fmask(3) : fmask(0);
+        mq[1] = (c & 1) ? fmask(4) : fmask(1);
+        mq[2] = (c & 1) ? 0u : fmask(2);
+        uint32_t mG[3], mH[3];
+#pragma unroll
+        for (int i = 0; i < 3; ++i) { mG[i] = c < 2 ? mq[i] : 0u; mH[i] = c < 2 ? 0u : mq[i]; }
+        const uint32_t lane4 = static_cast<uint32_t>(lane) * 4u;
+        // this warp's byte offset inside a stage row, and the base-3 window shift
+        const uint32_t off = LAYOUT == BT_LAYOUT_B3 ? static_cast<uint32_t>(q * kB3GroupBytes + 6 * c)
+                                                    : static_cast<uint32_t>(q * k2bGroupBytes + 8 * c);
+        const uint32_t o8 = LAYOUT == BT_LAYOUT_B3 ? (off & 3u) * 8u : 0u;
+        const uint32_t a4 = LAYOUT == BT_LAYOUT_B3 ? (off & ~3u) : off;
+
+        uint32_t err = 0;
+        float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+        int seg_start = 0;                                 // item index where the open segment began
+        int Q = Q0, b = b0;
+        for (int it = 0; it < nitems; ++it) {
+            const int s = it % S;
+            const int j = 8 * b + q;
+            // an aborted CTA keeps walking its items (no waits, no work) so that
+            // every consumer warp still meets every barrier below
+            bool ok = !flags[0];
+            if (ok && !mbar_wait(smem_addr(full + s), (it / S) & 1)) { bad = BT_DEVERR_TIMEOUT; flags[0] = 1; ok = false; }
+            if (ok) {
+                const uint32_t st = smem_u32addr(stages + s * GE::kStage);
+                const uint32_t sc = st + GE::kCodes;
+                uint32_t w[2][5];
+                float sgv[2], shv[2];
+#pragma unroll
+                for (int tt = 0; tt < 2; ++tt) {
+                    const int rg = h * 32 + tt * 16 + g, rh = rg + 8;
+                    sgv[tt] = f16_bits_to_f32(lds_u16(sc + rg * 16 + 2 * q));
+                    shv[tt] = f16_bits_to_f32(lds_u16(sc + rh * 16 + 2 * q));
+                    if constexpr (LAYOUT == BT_LAYOUT_B3) {
+                        w[tt][0] = lds_u32(st + rg * GE::RB + a4);
+                        w[tt][1] = lds_u32(st + rg * GE::RB + a4 + 4);
+                        w[tt][2] = lds_u32(st + rh * GE::RB + a4);
+                        w[tt][3] = lds_u32(st + rh * GE::RB + a4 + 4);
+                        w[tt][4] = lds_u16(st + (c < 2 ? rg : rh) * GE::RB + q * kB3GroupBytes + 24);
+                    } else {
+                        const uint2 x0 = lds_u64(st + rg * GE::RB + a4);
+                        const uint2 x1 = lds_u64(st + rh * GE::RB + a4);
+                        w[tt][0] = x0.x; w[tt][1] = x0.y; w[tt][2] = x1.x; w[tt][3] = x1.y; w[tt][4] = 0;
+                    }
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_addr(empty + s));   // the stage may be refilled
+
+                // activation fragments and group constants
+                uint32_t bf[NT][2];
+                float pm[2], cm[2];
+                if constexpr (BSMEM) {
+                    const uint32_t ba = bbase + static_cast<uint32_t>(j) * bstride;
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) {
+                        const uint2 v = lds_u64(ba + 32 * t);
+                        bf[t][0] = v.x;
+                        bf[t][1] = v.y;
+                    }
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        if (M1 && r == 1) { cm[1] = 0.f; pm[1] = 0.f; continue; }
+                        const uint2 md = lds_u64(mbase[r] + static_cast<uint32_t>(j) * mstride[r]);
+                        cm[r] = __uint_as_float(md.x);
+                        pm[r] = __uint_as_float(md.y);
+                    }
+                } else {
+                    const uint32_t* bp = a.bslots + (((int64_t)m * G + j) * NT) * 8 + c * 2;
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) {
+                        uint2 v = make_uint2(0u, 0u);
+                        if (okm) v = ldg_u64(bp + t * 8);
+                        bf[t][0] = v.x;
+                        bf[t][1] = v.y;
+                    }
+#pragma unroll
+                    for (int r = 0; r < 2; ++r) {
+                        const int mm = 2 * c + r;
+                        float2 md = make_float2(0.f, 0.f);
+                        if (mm < M) md = __ldg(a.meta + (int64_t)mm * G + j);
+                        cm[r] = md.x;
+                        pm[r] = md.y;
+                    }
+                }
+#pragma unroll
+                for (int tt = 0; tt < 2; ++tt) {
+                    uint32_t Rg[16], Rh[16], QG[3], QH[3];
+                    if constexpr (LAYOUT == BT_LAYOUT_B3) {
+                        uint32_t r15[15];
+                        b3_decode_pairs(w[tt][0], w[tt][1], o8, lane4, r15, err);
+#pragma unroll
+                        for (int k = 0; k < 15; ++k) Rg[k] = r15[k];
+                        b3_decode_pairs(w[tt][2], w[tt][3], o8, lane4, r15, err);
+#pragma unroll
+                        for (int k = 0; k < 15; ++k) Rh[k] = r15[k];
+                        Rg[15] = Rh[15] = 0u;
+                        const uint32_t va = lut_u32(prmt(w[tt][4], lane4, 0x5504u));
+                        const uint32_t vb = lut_u32(prmt(w[tt][4], lane4, 0x5514u) + 128);
+                        err = lop3_or3(err, va, vb);
+#pragma unroll
+                        for (int k = 0; k < 3; ++k) {
+                            QG[k] = lop3_or_and(va, vb, mG[k]);
+                            QH[k] = lop3_or_and(va, vb, mH[k]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int r = 0; r < 4; ++r) {
+                            const uint32_t x = w[tt][r];
+                            const uint32_t x12 = x >> 12;
+                            uint32_t* Rr = r < 2 ? Rg : Rh;
+                            const int base = (r & 1) * 8;
+#pragma unroll
+                            for (int f = 0; f < 6; ++f) Rr[base + f] = x & fmask(f);
+                            Rr[base + 6] = x12 & fmask(0);
+                            Rr[base + 7] = x12 & fmask(1);
+                            err |= x & (x >> 1);
+                        }
+#pragma unroll
+                        for (int k = 0; k < 3; ++k) QG[k] = QH[k] = 0u;
+                    }
+                    float d[4] = {0.f, 0.f, 0.f, 0.f};
+                    if constexpr (LAYOUT == BT_LAYOUT_B3) {
+#pragma unroll
+                        for (int t = 0; t < 7; ++t)
+                            mma_f16_16816(d, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1], bf[t][0], bf[t][1], d);
+                        mma_f16_16816(d, Rg[14], Rh[14], QG[0], QH[0], bf[7][0], bf[7][1], d);
+                        mma_f16_16816(d, QG[1], QH[1], QG[2], QH[2], bf[NT - 1][0], bf[NT - 1][1], d);
+                    } else {
+#pragma unroll
+                        for (int t = 0; t < NT; ++t)
+                            mma_f16_16816(d, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1], bf[t][0], bf[t][1], d);
+                    }
+                    acc[tt][0] = fmaf(sgv[tt], fmaf(d[0], pm[0], -cm[0]), acc[tt][0]);
+                    acc[tt][2] = fmaf(shv[tt], fmaf(d[2], pm[0], -cm[0]), acc[tt][2]);
+                    if (!M1) {
+                        acc[tt][1] = fmaf(sgv[tt], fmaf(d[1], pm[1], -cm[1]), acc[tt][1]);
+                        acc[tt][3] = fmaf(shv[tt], fmaf(d[3], pm[1], -cm[1]), acc[tt][3]);
+                    }
+                }
+            }  // ok
+
+            // ---- close the quad's segment at a quad boundary or at the end
+            const int Qcur = Q;
+            const int bcur = b;
+            if (++b == nb) { b = 0; ++Q; }
+            const bool boundary = (it + 1 == nitems) || (Q != Qcur);
+            if (boundary) {
+                float* rw = red + warp * 32 * 8;                 // [32 rows][8 cols]
+#pragma unroll
+                for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) {
+                        const int row = tt * 16 + g + (r >> 1) * 8, col = 2 * c + (r & 1);
+                        rw[row * 8 + col] = acc[tt][r];
+                    }
+                consumer_bar();
+                const int64_t seg_i0 = i0 + seg_start;
+                const bool whole = (seg_i0 % nb == 0) && (bcur == nb - 1);
+                const int tid = threadIdx.x;
+                float* part = a.partials + (((int64_t)blockIdx.x * 2 + (seg_start == 0 ? 0 : 1)) * kTmaRows) * M;
+                for (int e = tid; e < kTmaRows * M; e += kTmaConsumers * 32) {
+                    const int row = e / M, col = e % M;
+                    const int hh = row >> 5, lr = row & 31;
+                    float sum = 0.f;
+#pragma unroll
+                    for (int qq = 0; qq < 8; ++qq) sum += red[((hh * 8 + qq) * 32 + lr) * 8 + col];
+                    const int n = Qcur * kTmaRows + row;
+                    if (whole) {
+                        if (n < a.N) store_y(a.y, a.y_bf16, (int64_t)col * a.N + n, sum);
+                    } else {
+                        __stcg(part + row * M + col, sum);
+                    }
+                }
+                if (!whole) {
+                    fence_acq_rel_gpu();
+                    consumer_bar();
+                    const int64_t c_lo = ((int64_t)Qcur * nb) / a.chunk;
+                    const int64_t c_hi = ((int64_t)(Qcur + 1) * nb - 1) / a.chunk;
+                    if (tid == 0) {
+                        const int old = atomicAdd(a.counters + Qcur, 1);
+                        flags[1] = (old == static_cast<int>(c_hi - c_lo)) ? 1 : 0;
+                    }
+                    consumer_bar();
+                    if (flags[1]) {
+                        fence_acq_rel_gpu();
+                        for (int e = tid; e < kTmaRows * M; e += kTmaConsumers * 32) {
+                            const int row = e / M, col = e % M;
+                            float sum = 0.f;
+                            for (int64_t cc = c_lo; cc <= c_hi; ++cc) {
+                                const int sl = (cc * a.chunk >= (int64_t)Qcur * nb) ? 0 : 1;   // cc starts in Q
+                                sum += __ldcg(a.partials + ((cc * 2 + sl) * kTmaRows + row) * M + col);
+                            }
+                            const int n = Qcur * kTmaRows + row;
+                            if (n < a.N) store_y(a.y, a.y_bf16, (int64_t)col * a.N + n, sum);
+                        }
+                        if (tid == 0) a.counters[Qcur] = 0;
+                    }
+                }
+                consumer_bar();
+#pragma unroll
+                for (int tt = 0; tt < 2; ++tt) acc[tt][0] = acc[tt][1] = acc[tt][2] = acc[tt][3] = 0.f;
+                seg_start = it + 1;
+            }
+        }
+        if (LAYOUT == BT_LAYOUT_B3) { if (err >> 31) bad |= BT_DEVERR_INVALID_CODE; }
+        else if (err & 0x55555555u) bad |= BT_DEVERR_INVALID_CODE;
+    }
+    bad = __reduce_or_sync(0xffffffffu, bad);
+    if (lane == 0) report(a.dev_err, bad);
+}
+
 // ------------------------------------------------------------ host ---------
 
 struct GemvPlan {
@@ -755,9 +1139,78 @@ static GemvPlan make_gemv_plan(int layout, int64_t M, int64_t N, int64_t K, int 
     pl.off_counters = off;
     off = align_up(off + (size_t)pl.P * sizeof(int), 256);
     pl.off_partials = off;
+    // partials: enough for either kernel (the TMA-fed one needs grid x 2 x 32 x M)
     off = align_up(off + (size_t)pl.warps_total * 2 * kGemvTiles * 16 * M * sizeof(float), 256);
     pl.total = off;
     return pl;
+}
+
+// TMA-fed variant: applies to M <= 8, K % 1024 == 0, 16-byte aligned scales,
+// and activation fragments that fit next to the table and the stage ring.
+struct TmaPlan {
+    bool use, bsmem;
+    int grid, nb, stages;
+    int64_t items, chunk;
+    size_t smem;
+};
+
+static TmaPlan make_tma_plan(int layout, int64_t M, int64_t N, int64_t K, const void* scales, int num_sms) {
+    TmaPlan t{};
+    const int NT = layout == BT_LAYOUT_B3 ? kB3Mmas : k2bMmas;
+    const int G = static_cast<int>(K / kGroup);
+    t.use = M <= 8 && K % kBlock == 0 && (reinterpret_cast<uintptr_t>(scales) & 15) == 0;
+    if (!t.use) return t;
+    t.nb = static_cast<int>(K / kBlock);
+    const int64_t quads = (N + kTmaRows - 1) / kTmaRows;
+    t.items = quads * t.nb;
+    t.grid = static_cast<int>(t.items < num_sms ? t.items : num_sms);
+    t.chunk = (t.items + t.grid - 1) / t.grid;
+    const int RB = layout == BT_LAYOUT_B3 ? 8 * kB3GroupBytes : 8 * k2bGroupBytes;
+    const size_t stage = (size_t)kTmaRows * RB + kTmaRows * 16;
+    const size_t limit = 227 * 1024;
+    const size_t lutb = layout == BT_LAYOUT_B3 ? kLutBytes : 0;
+    const size_t bbytes = align_up(kZeroBytes + (size_t)M * G * (NT * 32 + 8), 1024);
+    const size_t nob = align_up(kZeroBytes, 1024);
+    t.use = false;
+    for (int st : {6, 5, 4, 3}) {      // prefer activation fragments in shared memory, then more stages
+        const size_t with_b = lutb + bbytes + (size_t)st * stage + kRedBytes + 256;
+        if (with_b <= limit) { t.use = true; t.bsmem = true; t.stages = st; t.smem = with_b; break; }
+    }
+    if (!t.use) {
+        for (int st : {6, 5, 4, 3}) {
+            const size_t wo = lutb + nob + (size_t)st * stage + kRedBytes + 256;
+            if (wo <= limit) { t.use = true; t.bsmem = false; t.stages = st; t.smem = wo; break; }
+        }
+    }
+    return t;
+}
+
+template <int LAYOUT, bool BSMEM, bool M1>
+static cudaError_t launch_gemv_tma_t(const CUtensorMap& cmap, const CUtensorMap& smap, const GemvTmaArgs& ta,
+                                     const TmaPlan& tp, cudaStream_t stream) {
+    auto kern = gemv_tma_kernel<LAYOUT, BSMEM, M1>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tp.smem);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(tp.grid);
+    cfg.blockDim = dim3(kTmaThreads);
+    cfg.dynamicSmemBytes = tp.smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, cmap, smap, ta);
+}
+
+template <int LAYOUT>
+static cudaError_t dispatch_gemv_tma(const CUtensorMap& cmap, const CUtensorMap& smap, const GemvTmaArgs& ta,
+                                     const TmaPlan& tp, cudaStream_t s) {
+    if (tp.bsmem)
+        return ta.M == 1 ? launch_gemv_tma_t<LAYOUT, true, true>(cmap, smap, ta, tp, s)
+                         : launch_gemv_tma_t<LAYOUT, true, false>(cmap, smap, ta, tp, s);
+    return launch_gemv_tma_t<LAYOUT, false, false>(cmap, smap, ta, tp, s);
 }
 
 size_t gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num_sms) {
@@ -815,6 +1268,47 @@ cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales
         gemv_prep_kernel<BT_LAYOUT_2BIT><<<pl.prep_grid, kPrepThreads, 0, stream>>>(pa);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
+
+    const TmaPlan tp = make_tma_plan(layout, M, N, K, scales, num_sms);
+    EncodeTiledFn enc = tp.use ? tensor_map_encoder() : nullptr;
+    if (tp.use && enc) {
+        const int RB = layout == BT_LAYOUT_B3 ? 8 * kB3GroupBytes : 8 * k2bGroupBytes;
+        const cuuint64_t row_bytes = (K / kGroup) * (layout == BT_LAYOUT_B3 ? kB3GroupBytes : k2bGroupBytes);
+        CUtensorMap cmap, smap;
+        const cuuint64_t cdim[2] = {row_bytes, static_cast<cuuint64_t>(N)};
+        const cuuint64_t cstr[1] = {row_bytes};
+        const cuuint32_t cbox[2] = {static_cast<cuuint32_t>(RB), kTmaRows};
+        const cuuint64_t sdim[2] = {static_cast<cuuint64_t>(pl.G), static_cast<cuuint64_t>(N)};
+        const cuuint64_t sstr[1] = {static_cast<cuuint64_t>(pl.G) * 2};
+        const cuuint32_t sbox[2] = {8, kTmaRows};
+        const cuuint32_t one[2] = {1, 1};
+        const bool okc = enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), cdim, cstr, cbox,
+                             one, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+        const bool oks = okc && enc(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t*>(scales), sdim,
+                                    sstr, sbox, one, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+        if (oks) {
+            GemvTmaArgs ta{};
+            ta.bslots = pa.bslots;
+            ta.meta = pa.meta;
+            ta.partials = reinterpret_cast<float*>(ws + pl.off_partials);
+            ta.counters = pa.counters;
+            ta.y = y;
+            ta.y_bf16 = y_dtype == BT_BF16;
+            ta.M = static_cast<int>(M);
+            ta.N = static_cast<int>(N);
+            ta.G = static_cast<int>(pl.G);
+            ta.nb = tp.nb;
+            ta.stages = tp.stages;
+            ta.items = tp.items;
+            ta.chunk = tp.chunk;
+            ta.dev_err = dev_err;
+            return layout == BT_LAYOUT_B3 ? dispatch_gemv_tma<BT_LAYOUT_B3>(cmap, smap, ta, tp, stream)
+                                          : dispatch_gemv_tma<BT_LAYOUT_2BIT>(cmap, smap, ta, tp, stream);
+        }
+    }
 
     GemvArgs ga{};
     ga.codes = codes;
