@@ -125,8 +125,10 @@ bt_status bt_fwht1024(const uint16_t* x_bf16, const int8_t* sign1024, int64_t M,
  *  workspace device, >= bt_gemv_workspace_bytes(...), 256-byte aligned.
  *            Scratch only; its contents need no initialisation and are
  *            meaningless after the call.
- *  dev_err   nullable; invalid codes set BT_DEVERR_INVALID_CODE (their
- *            contribution is then unspecified but finite).
+ *  dev_err   nullable. When given, the packed codes are validated on the
+ *            fly and invalid ones set BT_DEVERR_INVALID_CODE (their
+ *            contribution is then unspecified but finite); when NULL the
+ *            check is skipped (it costs one ALU op per byte pair).
  * Numerics: the rotated activation feeds FP16 tensor-core products with FP32
  * accumulation (one power-of-two exponent per 128 activations keeps it in
  * range); y satisfies |y - y_exact| <= 2e-3 * sum_k |w x'| + 1e-5.

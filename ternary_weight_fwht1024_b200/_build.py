@@ -14,7 +14,7 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
     "-O3", "-lineinfo", "-std=c++17", "-shared", "-Xcompiler", "-fPIC",
-    "--expt-relaxed-constexpr", "-Xptxas", "-v",
+    "--expt-relaxed-constexpr", "-Xptxas", "-v", "-Xlinker", "--no-undefined",
 ]
 
 

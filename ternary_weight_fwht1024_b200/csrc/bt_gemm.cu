@@ -15,7 +15,8 @@
 //     2^e_m.
 //
 //  2. gemm: one 128 x BN output tile per CTA, one 128-wide K group per
-//     pipeline stage (two stages).
+//     pipeline stage; a 4-stage ring of activation tiles (TMA) and a
+//     2-stage ring of decoded weight tiles.
 //       warp 0      TMA: the activation tile (two 64-column panels, 128-byte
 //                   swizzle) into shared memory;
 //       warp 1      allocates TMEM, one elected thread issues
@@ -46,8 +47,8 @@ constexpr int kGemmBM = 128;
 constexpr int kGemmBK = 128;             // one weight group per stage
 constexpr int kGemmDecWarps = 8;         // decoder / epilogue warps
 constexpr int kGemmThreads = (2 + kGemmDecWarps) * 32;
-constexpr int kGemmLutCopies = 16;
-constexpr int kGemmLutBytes = 256 * kGemmLutCopies * 8;  // 16 copies x (low, high) x 4 bytes per code
+constexpr int kGemmLutCopies = 8;
+constexpr int kGemmLutBytes = 256 * kGemmLutCopies * 8;  // 8 copies x (low, high) x 4 bytes per code
 
 // ---------------------------------------------------------------- helpers ----
 
@@ -223,12 +224,15 @@ struct GemmArgs {
 
 template <int LAYOUT, int BN, int STAGES>
 struct GemmSmem {
+    // activation ring (TMA) is deeper than the weight ring (decoded in the
+    // CTA): activation tiles come from L2/HBM and need the longer lead
+    static constexpr int kAStages = 4;
+    static constexpr int kBStages = STAGES;
     static constexpr int kA = kGemmBM * kGemmBK * 2;   // 32 KB: two 64-column panels
     static constexpr int kB = BN * kGemmBK * 2;
-    static constexpr int kStage = kA + kB;
     static constexpr int kLut = LAYOUT == BT_LAYOUT_B3 ? kGemmLutBytes : 0;
     static constexpr int kBars = 1024;                  // barriers, TMEM address, flags
-    static constexpr int kTotal = STAGES * kStage + kLut + kBars + 1024;  // + alignment slack
+    static constexpr int kTotal = kAStages * kA + kBStages * kB + kLut + kBars + 1024;  // + alignment slack
 };
 
 template <int LAYOUT, int BN, int STAGES>
@@ -237,12 +241,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
     using SM = GemmSmem<LAYOUT, BN, STAGES>;
     extern __shared__ uint8_t gsm_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~uintptr_t(1023));
-    uint8_t* stages = base;
-    uint8_t* lut = base + STAGES * SM::kStage;
+    constexpr int SA = SM::kAStages, SB = SM::kBStages;
+    uint8_t* a_ring = base;
+    uint8_t* b_ring = base + SA * SM::kA;
+    uint8_t* lut = b_ring + SB * SM::kB;
     uint8_t* ctl = lut + SM::kLut;
-    uint64_t* full = reinterpret_cast<uint64_t*>(ctl);
-    uint64_t* empty = full + STAGES;
-    uint64_t* accf = empty + STAGES;
+    uint64_t* fullA = reinterpret_cast<uint64_t*>(ctl);
+    uint64_t* emptyA = fullA + SA;
+    uint64_t* fullB = emptyA + SA;
+    uint64_t* emptyB = fullB + SB;
+    uint64_t* accf = emptyB + SB;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -251,26 +259,32 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
     const int ktiles = a.G;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
-            mbar_init(smem_addr(full + s), 1 + kGemmDecWarps);
-            mbar_init(smem_addr(empty + s), 1);
+        for (int s = 0; s < SA; ++s) {
+            mbar_init(smem_addr(fullA + s), 1);
+            mbar_init(smem_addr(emptyA + s), 1);
+        }
+        for (int s = 0; s < SB; ++s) {
+            mbar_init(smem_addr(fullB + s), kGemmDecWarps);
+            mbar_init(smem_addr(emptyB + s), 1);
         }
         mbar_init(smem_addr(accf), 1);
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (LAYOUT == BT_LAYOUT_B3) {
-        // digits of each code as 2-bit fields, 16 copies per code (low table,
+        // digits of each code as 2-bit fields, 8 copies per code (low table,
         // then high table with the fields in the upper half)
         for (int idx = threadIdx.x; idx < 256 * 2 * kGemmLutCopies; idx += blockDim.x) {
             const int code = idx / (2 * kGemmLutCopies), hi = (idx / kGemmLutCopies) & 1;
-            uint32_t f = 0x80000000u;
+            // fields plus the FP16 exponent bits of 1024 (0x6400) in the same
+            // half, so one LOP3 yields 1024 + d 4^i
+            uint32_t f = 0x80000000u | 0x6400u;
             if (code < 243) {
-                f = 0;
+                f = 0x6400u;
                 int r = code;
                 for (int i = 0; i < 5; ++i) { f |= static_cast<uint32_t>(r % 3) << (2 * i); r /= 3; }
-                if (hi) f <<= 16;
             }
+            if (hi) f = (f & 0xFFFFu) << 16 | (f & 0x80000000u);
             reinterpret_cast<uint32_t*>(lut)[idx] = f;
         }
     }
@@ -289,15 +303,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
         // ---------------- TMA producer: activation tiles
         if (lane == 0) {
             for (int kt = 0; kt < ktiles; ++kt) {
-                const int s = kt % STAGES;
-                if (kt >= STAGES && !mbar_wait(smem_addr(empty + s), ((kt / STAGES) - 1) & 1)) {
+                const int s = kt % SA;
+                if (kt >= SA && !mbar_wait(smem_addr(emptyA + s), ((kt / SA) - 1) & 1)) {
                     bad = BT_DEVERR_TIMEOUT; *abort_flag = 1; break;
                 }
                 if (*abort_flag) break;
-                const uint32_t dst = smem_addr(stages + s * SM::kStage);
-                mbar_arrive_tx(smem_addr(full + s), SM::kA);
-                tma_load_2d(dst, &amap, kt * kGemmBK, m0, smem_addr(full + s));
-                tma_load_2d(dst + SM::kA / 2, &amap, kt * kGemmBK + 64, m0, smem_addr(full + s));
+                const uint32_t dst = smem_addr(a_ring + s * SM::kA);
+                mbar_arrive_tx(smem_addr(fullA + s), SM::kA);
+                tma_load_2d(dst, &amap, kt * kGemmBK, m0, smem_addr(fullA + s));
+                tma_load_2d(dst + SM::kA / 2, &amap, kt * kGemmBK + 64, m0, smem_addr(fullA + s));
             }
         }
     } else if (warp == 1) {
@@ -305,21 +319,23 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
         if (lane == 0) {
             constexpr uint32_t idesc = idesc_f16(kGemmBM, BN);
             for (int kt = 0; kt < ktiles; ++kt) {
-                const int s = kt % STAGES;
-                if (!mbar_wait(smem_addr(full + s), (kt / STAGES) & 1)) {
+                const int s_a = kt % SA, s_b = kt % SB;
+                if (!mbar_wait(smem_addr(fullA + s_a), (kt / SA) & 1) ||
+                    !mbar_wait(smem_addr(fullB + s_b), (kt / SB) & 1)) {
                     bad = BT_DEVERR_TIMEOUT; *abort_flag = 1; break;
                 }
                 if (*abort_flag) break;
                 tc_fence_after();
-                const uint32_t sa = smem_addr(stages + s * SM::kStage);
-                const uint32_t sb = sa + SM::kA;
+                const uint32_t sa = smem_addr(a_ring + s_a * SM::kA);
+                const uint32_t sb = smem_addr(b_ring + s_b * SM::kB);
 #pragma unroll
                 for (int k = 0; k < kGemmBK / 16; ++k) {
                     const uint32_t pa = sa + (k >> 2) * (SM::kA / 2) + (k & 3) * 32;
                     const uint32_t pb = sb + (k >> 2) * (SM::kB / 2) + (k & 3) * 32;
                     tc_mma(tmem, smem_desc_sw128(pa), smem_desc_sw128(pb), idesc, (kt > 0 || k > 0) ? 1u : 0u);
                 }
-                tc_commit(smem_addr(empty + s));
+                tc_commit(smem_addr(emptyA + s_a));
+                tc_commit(smem_addr(emptyB + s_b));
             }
             tc_commit(smem_addr(accf));
         }
@@ -358,16 +374,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
         };
         load_group(0, cur, s_cur);
         for (int kt = 0; kt < ktiles; ++kt) {
-            const int s = kt % STAGES;
+            const int s = kt % SB;
             load_group(kt + 1, nxt, s_nxt);
-            if (kt >= STAGES && !mbar_wait(smem_addr(empty + s), ((kt / STAGES) - 1) & 1)) {
+            if (kt >= SB && !mbar_wait(smem_addr(emptyB + s), ((kt / SB) - 1) & 1)) {
                 bad = BT_DEVERR_TIMEOUT; *abort_flag = 1; break;
             }
             if (*abort_flag) break;
             if (active) {
                 const uint32_t s1 = s_cur;
                 const uint32_t s2 = s1 | (s1 << 16);
-                uint8_t* bst = stages + s * SM::kStage + SM::kA;
+                uint8_t* bst = b_ring + s * SM::kB;
                 // row t of the B tile: panel p (slots 64p..64p+63), 8-row atoms
                 const uint32_t row_off = static_cast<uint32_t>((t >> 3) * 1024 + (t & 7) * 128);
                 uint32_t words[64];
@@ -377,15 +393,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
                         const uint32_t pr = cur[p];
                         const uint32_t va = *reinterpret_cast<const uint32_t*>(lut_lane + (pr & 0xFFu) * kRow);
                         const uint32_t vb = *reinterpret_cast<const uint32_t*>(lut_lane + (pr >> 8) * kRow + kRow / 2);
-                        err |= va | vb;
+                        err |= (va | vb) & 0x80000000u;
                         const int nw = p < 12 ? 5 : 3;
 #pragma unroll
                         for (int i = 0; i < nw; ++i) {
-                            const uint32_t f = lop3_or_and(va, vb, gfmask(i)) | 0x64006400u;
+                            const uint32_t f = lop3_or_and(va, vb, gfmask(i) | 0x64006400u);
                             words[5 * p + i] = hmul2_u32(hfma2_u32(f, hm[i], ha[i]), s2);
                         }
                         if (p == 12) {
-                            const uint32_t f = (va & 0x0C0u) | ((va & 0x300u) << 16) | 0x64006400u;
+                            const uint32_t f = (va & 0x64C0u) | ((va & 0x300u) << 16) | 0x64000000u;
                             words[63] = hmul2_u32(hfma2_u32(f, hm34, ha34), s2);
                         }
                     }
@@ -418,7 +434,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
             s_cur = s_nxt;
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(full + s));
+            if (lane == 0) mbar_arrive(smem_addr(fullB + s));
         }
         if (LAYOUT == BT_LAYOUT_B3 ? (err >> 31) : (err != 0)) bad |= BT_DEVERR_INVALID_CODE;
 
@@ -467,7 +483,7 @@ size_t gemm_workspace_bytes(int, int64_t M, int64_t, int64_t K, int) {
 }
 
 static int pick_bn(int64_t M, int64_t N, int num_sms) {
-    const int cands[5] = {256, 224, 192, 160, 128};
+    const int cands[2] = {160, 128};
     int best = 128;
     double best_eff = -1.0;
     for (int bn : cands) {
@@ -501,13 +517,7 @@ static cudaError_t launch_gemm_t(const CUtensorMap& amap, const GemmArgs& ga, cu
 
 template <int LAYOUT>
 static cudaError_t dispatch_gemm(int bn, const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t s) {
-    switch (bn) {
-        case 256: return launch_gemm_t<LAYOUT, 256, 2>(amap, ga, s);
-        case 224: return launch_gemm_t<LAYOUT, 224, 2>(amap, ga, s);
-        case 192: return launch_gemm_t<LAYOUT, 192, 2>(amap, ga, s);
-        case 160: return launch_gemm_t<LAYOUT, 160, 2>(amap, ga, s);
-        default: return launch_gemm_t<LAYOUT, 128, 3>(amap, ga, s);
-    }
+    return bn == 160 ? launch_gemm_t<LAYOUT, 160, 2>(amap, ga, s) : launch_gemm_t<LAYOUT, 128, 2>(amap, ga, s);
 }
 
 cudaError_t launch_gemm(int layout, const uint8_t* codes, const uint16_t* scales, const void* x, int x_dtype,

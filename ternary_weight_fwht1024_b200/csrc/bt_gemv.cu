@@ -281,7 +281,9 @@ __device__ __forceinline__ void advance2(StagePtr& P, int group_bytes) {
     }
 }
 
-// Decode one row's bytes 6c..6c+5 of a base-3 group into 15 registers.
+// Decode one row's bytes 6c..6c+5 of a base-3 group into 15 registers
+// (CHECK: also OR the table entries into err, whose bit 31 flags codes >= 243).
+template <bool CHECK = true>
 __device__ __forceinline__ void b3_decode_pairs(uint32_t W0, uint32_t W1, uint32_t o8, uint32_t lane_addr,
                                                 uint32_t (&R)[15], uint32_t& err) {
     const uint32_t lo = __funnelshift_r(W0, W1, o8);
@@ -293,7 +295,7 @@ __device__ __forceinline__ void b3_decode_pairs(uint32_t W0, uint32_t W1, uint32
         // address = table + code * 256 + lane * 4 (+128 for the high table)
         const uint32_t va = lut_u32(prmt(src, lane_addr, 0x5504u | (b << 4)));
         const uint32_t vb = lut_u32(prmt(src, lane_addr, 0x5504u | ((b + 1) << 4)) + 128);
-        err = lop3_or3(err, va, vb);
+        if (CHECK) err = lop3_or3(err, va, vb);
 #pragma unroll
         for (int i = 0; i < 5; ++i) R[5 * q + i] = lop3_or_and(va, vb, fmask(i));
     }
@@ -780,7 +782,7 @@ __device__ __forceinline__ void consumer_bar() {
     asm volatile("bar.sync 1, %0;" :: "n"(kTmaConsumers * 32) : "memory");
 }
 
-template <int LAYOUT, bool BSMEM, bool M1>
+template <int LAYOUT, bool BSMEM, bool M1, bool CHECK>
 __global__ void __launch_bounds__(kTmaThreads, 1)
 gemv_tma_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant__ CUtensorMap smap, GemvTmaArgs a) {
     using GE = TmaGeom<LAYOUT>;
@@ -830,9 +832,10 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant_
         // kernel, so streaming starts before the dependency wait
         if (lane == 0) {
             int Q = Q0, b = b0;
+            int s = 0;
+            uint32_t ph = 0;                 // parity of the current pass over the ring
             for (int it = 0; it < nitems; ++it) {
-                const int s = it % S;
-                if (it >= S && !mbar_wait(smem_addr(empty + s), ((it / S) - 1) & 1)) {
+                if (it >= S && !mbar_wait(smem_addr(empty + s), ph ^ 1u)) {
                     bad = BT_DEVERR_TIMEOUT; flags[0] = 1; break;
                 }
                 if (flags[0]) break;
@@ -841,6 +844,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant_
                 tma_load_2d(dst, &cmap, b * GE::RB, Q * kTmaRows, smem_addr(full + s));
                 tma_load_2d(dst + GE::kCodes, &smap, b * 8, Q * kTmaRows, smem_addr(full + s));
                 if (++b == nb) { b = 0; ++Q; }
+                if (++s == S) { s = 0; ph ^= 1u; }
             }
         }
         pdl_wait();
@@ -903,13 +907,14 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant_
         float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
         int seg_start = 0;                                 // item index where the open segment began
         int Q = Q0, b = b0;
+        int s = 0;
+        uint32_t ph = 0;
         for (int it = 0; it < nitems; ++it) {
-            const int s = it % S;
             const int j = 8 * b + q;
             // an aborted CTA keeps walking its items (no waits, no work) so that
             // every consumer warp still meets every barrier below
             bool ok = !flags[0];
-            if (ok && !mbar_wait(smem_addr(full + s), (it / S) & 1)) { bad = BT_DEVERR_TIMEOUT; flags[0] = 1; ok = false; }
+            if (ok && !mbar_wait(smem_addr(full + s), ph)) { bad = BT_DEVERR_TIMEOUT; flags[0] = 1; ok = false; }
             if (ok) {
                 const uint32_t st = smem_u32addr(stages + s * GE::kStage);
                 const uint32_t sc = st + GE::kCodes;
@@ -976,16 +981,16 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant_
                     uint32_t Rg[16], Rh[16], QG[3], QH[3];
                     if constexpr (LAYOUT == BT_LAYOUT_B3) {
                         uint32_t r15[15];
-                        b3_decode_pairs(w[tt][0], w[tt][1], o8, lane4, r15, err);
+                        b3_decode_pairs<CHECK>(w[tt][0], w[tt][1], o8, lane4, r15, err);
 #pragma unroll
                         for (int k = 0; k < 15; ++k) Rg[k] = r15[k];
-                        b3_decode_pairs(w[tt][2], w[tt][3], o8, lane4, r15, err);
+                        b3_decode_pairs<CHECK>(w[tt][2], w[tt][3], o8, lane4, r15, err);
 #pragma unroll
                         for (int k = 0; k < 15; ++k) Rh[k] = r15[k];
                         Rg[15] = Rh[15] = 0u;
                         const uint32_t va = lut_u32(prmt(w[tt][4], lane4, 0x5504u));
                         const uint32_t vb = lut_u32(prmt(w[tt][4], lane4, 0x5514u) + 128);
-                        err = lop3_or3(err, va, vb);
+                        if (CHECK) err = lop3_or3(err, va, vb);
 #pragma unroll
                         for (int k = 0; k < 3; ++k) {
                             QG[k] = lop3_or_and(va, vb, mG[k]);
@@ -1002,23 +1007,35 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant_
                             for (int f = 0; f < 6; ++f) Rr[base + f] = x & fmask(f);
                             Rr[base + 6] = x12 & fmask(0);
                             Rr[base + 7] = x12 & fmask(1);
-                            err |= x & (x >> 1);
+                            if (CHECK) err |= x & (x >> 1);
                         }
 #pragma unroll
                         for (int k = 0; k < 3; ++k) QG[k] = QH[k] = 0u;
                     }
-                    float d[4] = {0.f, 0.f, 0.f, 0.f};
+                    // two accumulator chains (even / odd MMA steps) halve the
+                    // dependent MMA latency per tile
+                    float d[4] = {0.f, 0.f, 0.f, 0.f}, e4[4] = {0.f, 0.f, 0.f, 0.f};
                     if constexpr (LAYOUT == BT_LAYOUT_B3) {
 #pragma unroll
-                        for (int t = 0; t < 7; ++t)
-                            mma_f16_16816(d, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1], bf[t][0], bf[t][1], d);
-                        mma_f16_16816(d, Rg[14], Rh[14], QG[0], QH[0], bf[7][0], bf[7][1], d);
+                        for (int t = 0; t < 7; ++t) {
+                            if (t & 1)
+                                mma_f16_16816(e4, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1], bf[t][0], bf[t][1], e4);
+                            else
+                                mma_f16_16816(d, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1], bf[t][0], bf[t][1], d);
+                        }
+                        mma_f16_16816(e4, Rg[14], Rh[14], QG[0], QH[0], bf[7][0], bf[7][1], e4);
                         mma_f16_16816(d, QG[1], QH[1], QG[2], QH[2], bf[NT - 1][0], bf[NT - 1][1], d);
                     } else {
 #pragma unroll
-                        for (int t = 0; t < NT; ++t)
-                            mma_f16_16816(d, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1], bf[t][0], bf[t][1], d);
+                        for (int t = 0; t < NT; ++t) {
+                            if (t & 1)
+                                mma_f16_16816(e4, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1], bf[t][0], bf[t][1], e4);
+                            else
+                                mma_f16_16816(d, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1], bf[t][0], bf[t][1], d);
+                        }
                     }
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) d[r] += e4[r];
                     acc[tt][0] = fmaf(sgv[tt], fmaf(d[0], pm[0], -cm[0]), acc[tt][0]);
                     acc[tt][2] = fmaf(shv[tt], fmaf(d[2], pm[0], -cm[0]), acc[tt][2]);
                     if (!M1) {
@@ -1027,6 +1044,8 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant_
                     }
                 }
             }  // ok
+
+            if (++s == S) { s = 0; ph ^= 1u; }
 
             // ---- close the quad's segment at a quad boundary or at the end
             const int Qcur = Q;
@@ -1145,6 +1164,10 @@ static GemvPlan make_gemv_plan(int layout, int64_t M, int64_t N, int64_t K, int 
     return pl;
 }
 
+size_t gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num_sms) {
+    return make_gemv_plan(layout, M, N, K, num_sms).total;
+}
+
 // TMA-fed variant: applies to M <= 8, K % 1024 == 0, 16-byte aligned scales,
 // and activation fragments that fit next to the table and the stage ring.
 struct TmaPlan {
@@ -1185,10 +1208,10 @@ static TmaPlan make_tma_plan(int layout, int64_t M, int64_t N, int64_t K, const 
     return t;
 }
 
-template <int LAYOUT, bool BSMEM, bool M1>
+template <int LAYOUT, bool BSMEM, bool M1, bool CHECK>
 static cudaError_t launch_gemv_tma_t(const CUtensorMap& cmap, const CUtensorMap& smap, const GemvTmaArgs& ta,
                                      const TmaPlan& tp, cudaStream_t stream) {
-    auto kern = gemv_tma_kernel<LAYOUT, BSMEM, M1>;
+    auto kern = gemv_tma_kernel<LAYOUT, BSMEM, M1, CHECK>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tp.smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
@@ -1204,17 +1227,22 @@ static cudaError_t launch_gemv_tma_t(const CUtensorMap& cmap, const CUtensorMap&
     return cudaLaunchKernelEx(&cfg, kern, cmap, smap, ta);
 }
 
+template <int LAYOUT, bool CHECK>
+static cudaError_t dispatch_gemv_tma_c(const CUtensorMap& cmap, const CUtensorMap& smap, const GemvTmaArgs& ta,
+                                       const TmaPlan& tp, cudaStream_t s) {
+    if (tp.bsmem)
+        return ta.M == 1 ? launch_gemv_tma_t<LAYOUT, true, true, CHECK>(cmap, smap, ta, tp, s)
+                         : launch_gemv_tma_t<LAYOUT, true, false, CHECK>(cmap, smap, ta, tp, s);
+    return launch_gemv_tma_t<LAYOUT, false, false, CHECK>(cmap, smap, ta, tp, s);
+}
+
+// Code validation costs an ALU op per byte pair; it runs when the caller
+// passes an error word to report into.
 template <int LAYOUT>
 static cudaError_t dispatch_gemv_tma(const CUtensorMap& cmap, const CUtensorMap& smap, const GemvTmaArgs& ta,
                                      const TmaPlan& tp, cudaStream_t s) {
-    if (tp.bsmem)
-        return ta.M == 1 ? launch_gemv_tma_t<LAYOUT, true, true>(cmap, smap, ta, tp, s)
-                         : launch_gemv_tma_t<LAYOUT, true, false>(cmap, smap, ta, tp, s);
-    return launch_gemv_tma_t<LAYOUT, false, false>(cmap, smap, ta, tp, s);
-}
-
-size_t gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num_sms) {
-    return make_gemv_plan(layout, M, N, K, num_sms).total;
+    return ta.dev_err ? dispatch_gemv_tma_c<LAYOUT, true>(cmap, smap, ta, tp, s)
+                      : dispatch_gemv_tma_c<LAYOUT, false>(cmap, smap, ta, tp, s);
 }
 
 template <int LAYOUT, int MT, bool BSMEM, bool M1>

@@ -275,3 +275,17 @@ def test_gemm_special_cases():
     _, y_ref, b = oracle.forward(z, case["scales"], case["x"], case["sign"])
     y1 = run_gemm(z, case["scales"], case["x"], case["sign"])
     check(y1, y_ref, b, extra=np.abs(y_ref) * 2.0 ** -8)
+
+
+@pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
+def test_gemv_unchecked_equals_checked(layout):
+    # without an error word the code check is compiled out; results must not change
+    case = workloads.layer_inputs("C1", workloads.TRIPLE[2], index=2)
+    codes = bt.pack(T(case["trits"]), layout)
+    x, sign, sc = T(case["x"], "bf16"), T(case["sign"]), T(case["scales"])
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    a = bt.gemv(codes, sc, x, sign, case["N"], layout, dev_err=err)
+    b = bt.gemv(codes, sc, x, sign, case["N"], layout)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert torch.equal(a, b)
