@@ -102,6 +102,23 @@ class ClockSampler:
         return {"sm_mhz": float(np.median(sm)), "sm_max_mhz": mx, "reasons": sorted(reasons), "samples": len(sm)}
 
 
+# ------------------------------------------------------- multi-rank timing ---
+
+def max_over_ranks(ms: float, world: int, dist=None, device=None) -> float:
+    """The slowest rank's time: every rank calls this once per timed region."""
+    if world <= 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_rate(units_per_rank: float, ms: float, world: int) -> float:
+    """Units per second over all ranks (weak scaling: each rank does its own units)."""
+    return units_per_rank * world / (ms * 1e-3)
+
+
 # ----------------------------------------------------------------- inputs ---
 
 def _layer_tensors(bt, torch, dev, layout, idx, L, with_x=False):
@@ -179,12 +196,7 @@ def run_gpu(args, rank, world):
                 gs[(warmup + k) % copies].replay()
             en.record(stream)
             torch.cuda.synchronize()
-        ms = st.elapsed_time(en) / steps
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return max_over_ranks(st.elapsed_time(en) / steps, world, dist, dev)
 
     # ---- base-3 (headline) ----
     reps3 = build(0)
@@ -220,6 +232,9 @@ def run_gpu(args, rank, world):
                 bt.gemv(reps3[w % copies][i][0], reps3[w % copies][i][1], xs[i], sign, L.N, 0, out=ys[i], ws=ws)
                 y_host[i].copy_(ys[i], non_blocking=True)
         torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
         st = torch.cuda.Event(enable_timing=True)
         en = torch.cuda.Event(enable_timing=True)
         st.record(stream)
@@ -231,7 +246,7 @@ def run_gpu(args, rank, world):
                 y_host[i].copy_(ys[i], non_blocking=True)
         en.record(stream)
         torch.cuda.synchronize()
-    e2e_ms = st.elapsed_time(en) / args.steps
+    e2e_ms = max_over_ranks(st.elapsed_time(en) / args.steps, world, dist, dev)
     del reps3
 
     # ---- 2-bit layout twin ----
@@ -267,7 +282,38 @@ def run_gpu(args, rank, world):
     except Exception as e:  # the prefill path is reported, not required for the headline
         gemm = {"value": None, "error": str(e)[:200]}
 
-    gbs = bytes3 / (ms3 * 1e-3) / 1e9 * world
+    # ---- 27B-equivalent decode sweep: 64 stacks x 2 triples = 384 matrices
+    sweep = None
+    if not args.no_sweep:
+        try:
+            sweep = run_sweep(bt, torch, dev, stream, sign, args, world, dist)
+        except Exception as e:
+            sweep = {"error": str(e)[:200]}
+
+    # ---- standalone rotation sweep
+    fwht = {}
+    try:
+        for Mf in (1, 16, 512):
+            for Kf in (1024, 5120, 17408):
+                xf = torch.randn((Mf, Kf), device=dev).to(torch.bfloat16)
+                with torch.cuda.stream(stream):
+                    for _ in range(3):
+                        bt.fwht1024(xf, sign)
+                    torch.cuda.synchronize()
+                    a_ = torch.cuda.Event(enable_timing=True)
+                    b_ = torch.cuda.Event(enable_timing=True)
+                    reps = 50
+                    a_.record(stream)
+                    for _ in range(reps):
+                        bt.fwht1024(xf, sign)
+                    b_.record(stream)
+                    torch.cuda.synchronize()
+                us = a_.elapsed_time(b_) * 1e3 / reps
+                fwht[f"M{Mf}xK{Kf}"] = {"us": round(us, 2), "GB/s": round(Mf * Kf * 6 / (us * 1e-6) / 1e9, 1)}
+    except Exception as e:
+        fwht = {"error": str(e)[:200]}
+
+    gbs = whole_job_rate(bytes3, ms3, world) / 1e9
     dom_bytes = [(_weight_bytes(L, 0) + M * L.K * 2 + M * L.N * 4) for L in triple]
     achieved = sum(dom_bytes) / (sum(per_layer_us) * 1e-6) / 1e9
     out = {
@@ -295,6 +341,8 @@ def run_gpu(args, rank, world):
                         "ms_per_step": round(ms2, 5), "bytes_per_step": bytes2},
         "tokens_per_s_triple": round(1e3 / ms3 * world, 1),
         "gemm": gemm,
+        "sweep_27b": sweep,
+        "fwht_sweep": fwht,
         "e2e": {"value": round(bytes3 / (e2e_ms * 1e-3) / 1e9 * world, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": sum(M * L.K * 2 for L in triple),
                 "d2h_bytes_per_step": sum(M * L.N * 4 for L in triple)},
@@ -308,6 +356,66 @@ def run_gpu(args, rank, world):
     }
     if rank == 0 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(args.cpu_seconds)
+    return out
+
+
+def run_sweep(bt, torch, dev, stream, sign, args, world, dist):
+    """Decode token through 64 stacks x 2 triples (384 matrices, 26.2e9 weights, 5.7 GB
+    base-3): one seeded triple generated on the host and cloned on the device to 128
+    distinct copies at distinct addresses; one token step = 384 bt_gemv calls replayed
+    from CUDA graphs."""
+    import workloads
+    triple = workloads.TRIPLE
+    uniq = []
+    for i, L in enumerate(triple):
+        inp = workloads.layer_inputs("C2", L, index=i, with_x=False)
+        uniq.append((bt.pack(torch.from_numpy(inp["trits"]).to(dev), 0),
+                     torch.from_numpy(inp["scales"].view(np.int16)).to(dev)))
+    n_triples = 128
+    mats = [[(c.clone(), s.clone()) for c, s in uniq] for _ in range(n_triples)]
+    del uniq
+    weight_bytes = n_triples * sum(_weight_bytes(L, 0) for L in triple)
+    out = {"weights": int(n_triples * sum(L.N * L.K for L in triple)), "bytes_per_token": weight_bytes,
+           "matrices": 3 * n_triples}
+    for M in (1, 4, 16):
+        g = workloads.rng(3 * 1_000_003 + 1000 + M)
+        xs = [torch.from_numpy(workloads.activations_bf16_bits(g, M, L.K, True).view(np.int16)).to(dev)
+              .view(torch.bfloat16) for L in triple]
+        ys = [torch.empty((M, L.N), device=dev) for L in triple]
+        ws = torch.empty(max(bt.gemv_workspace_bytes(0, M, L.N, L.K) for L in triple), dtype=torch.uint8,
+                         device=dev)
+        graphs = []
+        with torch.cuda.stream(stream):
+            for i, L in enumerate(triple):
+                bt.gemv(mats[0][i][0], mats[0][i][1], xs[i], sign, L.N, 0, out=ys[i], ws=ws)
+            torch.cuda.synchronize()
+            per_graph = 16
+            for g0 in range(0, n_triples, per_graph):
+                gr = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gr, stream=stream):
+                    for t in range(g0, g0 + per_graph):
+                        for i, L in enumerate(triple):
+                            bt.gemv(mats[t][i][0], mats[t][i][1], xs[i], sign, L.N, 0, out=ys[i], ws=ws)
+                graphs.append(gr)
+            for gr in graphs:
+                gr.replay()
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            a_ = torch.cuda.Event(enable_timing=True)
+            b_ = torch.cuda.Event(enable_timing=True)
+            tokens = 3
+            a_.record(stream)
+            for _ in range(tokens):
+                for gr in graphs:
+                    gr.replay()
+            b_.record(stream)
+            torch.cuda.synchronize()
+        ms = max_over_ranks(a_.elapsed_time(b_) / tokens, world, dist, dev)
+        out[f"M{M}"] = {"ms_per_token_step": round(ms, 3), "tokens_per_s": round(whole_job_rate(M, ms, world), 1),
+                        "weight_GB/s": round(whole_job_rate(weight_bytes, ms, world) / 1e9, 1)}
+        del graphs
+    out["roofline_tokens_per_s_M1"] = round(_peaks()["hbm_gbs"] * 1e9 / weight_bytes, 1)
     return out
 
 
@@ -337,17 +445,34 @@ def cpu_baseline(budget_s: float):
             + f", {t_total:.1f} s"}
 
 
+def reference_rows(per_row_s, Ns, step_budget_s):
+    """Rows of each matrix one oracle step covers: the whole matrix when the
+    step fits its time budget, else the same fraction of every matrix."""
+    full = sum(p * n for p, n in zip(per_row_s, Ns))
+    frac = min(1.0, step_budget_s / max(full, 1e-12))
+    return [max(8, min(n, int(n * frac))) for n in Ns]
+
+
 def run_reference(args):
-    """The CPU oracle as the reference arm, on the same metric and workload."""
+    """The CPU oracle as the reference arm, on the same metric and workload:
+    each step is the rotation of x plus the FP64 GEMV of a row sample of every
+    matrix, sized so that warm-up plus timed steps take about `ref_seconds`."""
     import oracle
     import workloads
     oracle.build()
     triple = workloads.TRIPLE
     inputs = [workloads.layer_inputs("C1", L, index=i) for i, L in enumerate(triple)]
-    budget_rows = [L.N for L in triple]  # the oracle covers the whole triple in about a second
+    per_row = []
+    for inp in inputs:
+        xr = oracle.rotate_bf16(inp["x"], inp["sign"])
+        t0 = time.perf_counter()
+        oracle.gemv(inp["trits"][:64], inp["scales"][:64], xr)
+        per_row.append((time.perf_counter() - t0) / 64)
+    rows = reference_rows(per_row, [L.N for L in triple], args.ref_seconds / (args.steps + args.warmup))
+
     def step():
         b = 0
-        for inp, L, r in zip(inputs, triple, budget_rows):
+        for inp, L, r in zip(inputs, triple, rows):
             xr = oracle.rotate_bf16(inp["x"], inp["sign"])
             oracle.gemv(inp["trits"][:r], inp["scales"][:r], xr)
             b += _weight_bytes(workloads.Layer(L.name, L.K, r), 0)
@@ -360,9 +485,11 @@ def run_reference(args):
         tot += step()
     dt = time.perf_counter() - t0
     v = tot / dt / 1e9
-    sample = "decode triple M=1, " + ", ".join(f"{L.name}:{r}/{L.N} rows" for L, r in zip(triple, budget_rows))
+    sample = ("decode triple M=1 incl. rotation of x, rows per step " +
+              ", ".join(f"{L.name}:{r}/{L.N}" for L, r in zip(triple, rows)))
     return {
-        "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": 1,
+        "impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", 1)),
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 3),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": "decode GEMV M=1 on the 5120x5120 / 5120x17408 / 17408x5120 triple, base-3 g128, "
@@ -370,6 +497,7 @@ def run_reference(args):
         "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": oracle.threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "note": "FP64 CPU oracle on rank 0's host cores; other ranks exit without work",
     }
 
 
@@ -380,7 +508,10 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--ref-seconds", type=float, default=90.0,
+                    help="CPU time the reference arm spends over warm-up + timed steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the 384-matrix 27B-equivalent sweep")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank = int(os.environ.get("RANK", 0))
