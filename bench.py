@@ -207,20 +207,28 @@ def run_gpu(args, rank, world):
     bytes3 = sum(_weight_bytes(L, 0) for L in triple)
     io_bytes = sum(M * L.K * 2 + M * L.N * 4 for L in triple)
 
-    # per-call durations of the dominant call (bt_gemv = prep + GEMV kernels)
+    # per-call durations of the dominant call (one bt_gemv: main kernel + chunk reduction),
+    # from a CUDA graph of `copies` calls of one layer over the rotating weight copies
     per_layer_us = []
     with torch.cuda.stream(stream):
         for i, L in enumerate(triple):
-            evs = []
-            for r in range(copies):
-                a = torch.cuda.Event(enable_timing=True)
-                b = torch.cuda.Event(enable_timing=True)
-                a.record(stream)
-                bt.gemv(reps3[r][i][0], reps3[r][i][1], xs[i], sign, L.N, 0, out=ys[i], ws=ws)
-                b.record(stream)
-                evs.append((a, b))
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                for r in range(copies):
+                    bt.gemv(reps3[r][i][0], reps3[r][i][1], xs[i], sign, L.N, 0, out=ys[i], ws=ws)
+            for _ in range(3):
+                gr.replay()
             torch.cuda.synchronize()
-            per_layer_us.append(float(np.mean([a.elapsed_time(b) for a, b in evs[2:]])) * 1e3)
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            reps_t = 20
+            a.record(stream)
+            for _ in range(reps_t):
+                gr.replay()
+            b.record(stream)
+            torch.cuda.synchronize()
+            per_layer_us.append(a.elapsed_time(b) * 1e3 / (reps_t * copies))
+            del gr
     del gs3
 
     # ---- e2e through the public API with host buffers ----
@@ -290,25 +298,31 @@ def run_gpu(args, rank, world):
         except Exception as e:
             sweep = {"error": str(e)[:200]}
 
-    # ---- standalone rotation sweep
+    # ---- standalone rotation sweep (graphs of 20 calls; the largest inputs are L2-resident)
     fwht = {}
     try:
         for Mf in (1, 16, 512):
             for Kf in (1024, 5120, 17408):
                 xf = torch.randn((Mf, Kf), device=dev).to(torch.bfloat16)
+                of = torch.empty((Mf, Kf), dtype=torch.float32, device=dev)
                 with torch.cuda.stream(stream):
-                    for _ in range(3):
-                        bt.fwht1024(xf, sign)
+                    bt.fwht1024(xf, sign, out=of)
+                    torch.cuda.synchronize()
+                    gr = torch.cuda.CUDAGraph()
+                    with torch.cuda.graph(gr, stream=stream):
+                        for _ in range(20):
+                            bt.fwht1024(xf, sign, out=of)
+                    gr.replay()
                     torch.cuda.synchronize()
                     a_ = torch.cuda.Event(enable_timing=True)
                     b_ = torch.cuda.Event(enable_timing=True)
-                    reps = 50
                     a_.record(stream)
-                    for _ in range(reps):
-                        bt.fwht1024(xf, sign)
+                    for _ in range(10):
+                        gr.replay()
                     b_.record(stream)
                     torch.cuda.synchronize()
-                us = a_.elapsed_time(b_) * 1e3 / reps
+                    del gr
+                us = a_.elapsed_time(b_) * 1e3 / 200
                 fwht[f"M{Mf}xK{Kf}"] = {"us": round(us, 2), "GB/s": round(Mf * Kf * 6 / (us * 1e-6) / 1e9, 1)}
     except Exception as e:
         fwht = {"error": str(e)[:200]}
@@ -349,9 +363,9 @@ def run_gpu(args, rank, world):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(achieved / peaks["hbm_gbs"], 4),
                      "traffic": None,
-                     "kernel": "bt_gemv call (gemv_prep + gemv kernels), average over the three layers",
+                     "kernel": "bt_gemv call (table-lookup GEMV kernel + chunk reduction), weighted over the three layers",
                      "peak_kind": f"HBM copy, {peaks['src']}"},
-        "gpu_launches": args.steps * len(triple) * 2,
+        "gpu_launches": args.steps * len(triple) * 2,  # GEMV + chunk-sum kernels per bt_gemv call
         "clocks": clk.summary(),
     }
     if rank == 0 and not args.no_cpu_baseline:

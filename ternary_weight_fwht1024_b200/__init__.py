@@ -132,14 +132,19 @@ def unpack(codes: torch.Tensor, K: int, layout: int = LAYOUT_B3,
     return trits
 
 
-def fwht1024(x: torch.Tensor, sign: torch.Tensor, out_dtype: int = F32) -> torch.Tensor:
+def fwht1024(x: torch.Tensor, sign: torch.Tensor, out_dtype: int = F32,
+             out: torch.Tensor | None = None) -> torch.Tensor:
     """x' = (1/32) H_1024 (S . x) per 1024-block; x bf16 [M, K]."""
-    _require_cuda(x, sign)
+    _require_cuda(x, sign, out)
     if x.dtype != torch.bfloat16:
         raise TypeError("x must be bfloat16")
     xc = x.contiguous()
     M, K = xc.shape
-    out = torch.empty((M, K), dtype=torch.float32 if out_dtype == F32 else torch.bfloat16, device=x.device)
+    if out is None:
+        out = torch.empty((M, K), dtype=torch.float32 if out_dtype == F32 else torch.bfloat16, device=x.device)
+    elif out.dtype != (torch.float32 if out_dtype == F32 else torch.bfloat16) or tuple(out.shape) != (M, K) \
+            or not out.is_contiguous():
+        raise ValueError("out must be a contiguous [M, K] tensor of the output dtype")
     _check("bt_fwht1024", load().bt_fwht1024(_ptr(xc), _ptr(sign), M, K, out_dtype, _ptr(out), _stream(x.device)))
     return out
 

@@ -1164,8 +1164,21 @@ static GemvPlan make_gemv_plan(int layout, int64_t M, int64_t N, int64_t K, int 
     return pl;
 }
 
+// Single-row calls with K a multiple of 512 take the table-lookup kernel
+// (bt_gemv_lut.cu); the workspace covers either path.
+bool gemv_lut_applies(int64_t M, int64_t K, const void* scales);
+size_t gemv_lut_workspace_bytes(int64_t N, int64_t K);
+cudaError_t launch_gemv_lut(int layout, const uint8_t* codes, const uint16_t* scales, const void* x, int x_dtype,
+                            const int8_t* sign, int64_t N, int64_t K, int y_dtype, void* y, void* workspace,
+                            int32_t* dev_err, int num_sms, cudaStream_t stream);
+
 size_t gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num_sms) {
-    return make_gemv_plan(layout, M, N, K, num_sms).total;
+    size_t need = make_gemv_plan(layout, M, N, K, num_sms).total;
+    if (M == 1 && K % 1024 == 0) {
+        const size_t lut = align_up(gemv_lut_workspace_bytes(N, K), 256);
+        if (lut > need) need = lut;
+    }
+    return need;
 }
 
 // TMA-fed variant: applies to M <= 8, K % 1024 == 0, 16-byte aligned scales,
@@ -1276,6 +1289,9 @@ cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales
                         int x_dtype, const int8_t* sign, int64_t M, int64_t N, int64_t K, int y_dtype,
                         void* y, void* workspace, int32_t* dev_err, int num_sms,
                         cudaStream_t stream) {
+    if (gemv_lut_applies(M, K, scales))
+        return launch_gemv_lut(layout, codes, scales, x, x_dtype, sign, N, K, y_dtype, y, workspace, dev_err,
+                               num_sms, stream);
     const GemvPlan pl = make_gemv_plan(layout, M, N, K, num_sms);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
 
