@@ -58,7 +58,8 @@ constexpr int kLutDepth = 2;                         // sets in flight per warp
 constexpr int kLutCBoxB3 = 112;                      // box bytes per row: 104 + up to 8 of alignment
 constexpr int kLutCBox2b = 128;
 constexpr int kLutSlotMax = kLutSet * kLutCBox2b + kLutSet * 16;  // codes box + scale box (8 halves/row)
-constexpr int kLutBarOffset = kLutXsOffset + 5 * 4 * 32 * 4;
+constexpr int kLutTileOffset = kLutXsOffset + 5 * 4 * 32 * 4;   // FWHT exchange tile, 32 x 36 f32
+constexpr int kLutBarOffset = kLutTileOffset + 32 * kTileStride * 4;
 constexpr int kLutRingOffset = kLutBarOffset + kLutWarps * kLutDepth * 8;
 constexpr int kLutSmem = kLutRingOffset + kLutWarps * kLutDepth * kLutSlotMax;
 constexpr int kLutMinRows = 64;                      // fewest rows worth a table build
@@ -188,28 +189,41 @@ __device__ __forceinline__ void lut_scatter(const float* xr, int h, float* xs) {
     }
 }
 
-// Tables for the current chunk. Base-3: code c = a + 27 b (a: trits 0-2,
-// b: trits 3-4); task (b, k) writes the 27 entries of that b for byte k of
-// every lane. Codes 243-255 are not base-3 codes and read 0. 2-bit: code
-// c = lo + 16 hi, digits 2 bits wide; entries with a digit 3 read 0. (An
-// invalid code thus contributes nothing; the checked kernel reports it.)
+// Entries for codes that are not valid (base-3 codes 243-255, 2-bit codes
+// with a field of 3) read 0, so an invalid code contributes nothing (the
+// checked kernel reports it). They never change: zeroed once per launch.
+template <int LAYOUT>
+__device__ __forceinline__ void lut_zero_invalid(float* table) {
+    if (LAYOUT == BT_LAYOUT_B3) {
+        for (int t = threadIdx.x; t < 2 * 13 * 64; t += kLutThreads) {
+            const int r = t / (13 * 64), u = t - r * 13 * 64;
+            table[r * (kLutRegion / 4) + 243 * 64 + u] = 0.f;
+        }
+    } else {
+        for (int t = threadIdx.x; t < 2 * 256 * 64; t += kLutThreads) {
+            const int c = (t >> 6) & 255;
+            if (c & (c >> 1) & 0x55) table[t] = 0.f;
+        }
+    }
+}
+
+// Tables for the current chunk: entry(c) = sum_i (d_i(c) - 1) x'_i over the
+// trits of byte slot (L, k). Warp w serves k = w % 4 for every lane and a
+// quarter of the high digits. Base-3: c = a + 27 b (a: trits 0-2, b: trits
+// 3-4), warp takes b = w / 4 + 4 j and writes the 27 entries of each b.
+// 2-bit: c = lo + 16 hi (two 2-bit digits each), warp takes hi = w / 4 + 4 j
+// and writes the entries whose digits are all valid.
 template <int LAYOUT>
 __device__ __forceinline__ void lut_build(const float* xs, float* table) {
     const int warp = threadIdx.x >> 5, L = threadIdx.x & 31;
+    const int k = warp & 3, q = warp >> 2;
+    const float x0 = xs[(0 * 4 + k) * 32 + L], x1 = xs[(1 * 4 + k) * 32 + L], x2 = xs[(2 * 4 + k) * 32 + L],
+                x3 = xs[(3 * 4 + k) * 32 + L];
+    float* col = table + (k >> 1) * (kLutRegion / 4) + L + 32 * (k & 1);
     if (LAYOUT == BT_LAYOUT_B3) {
-        for (int task = warp; task < 40; task += kLutWarps) {
-            const int b = task >> 2, k = task & 3;
-            const float x0 = xs[(0 * 4 + k) * 32 + L], x1 = xs[(1 * 4 + k) * 32 + L],
-                        x2 = xs[(2 * 4 + k) * 32 + L], x3 = xs[(3 * 4 + k) * 32 + L],
-                        x4 = xs[(4 * 4 + k) * 32 + L];
-            float* col = table + (k >> 1) * (kLutRegion / 4) + L + 32 * (k & 1);
-            if (b == 9) {
-#pragma unroll
-                for (int a = 0; a < 13; ++a) col[(243 + a) * 64] = 0.f;
-                continue;
-            }
-            const float d3 = (float)(b % 3) - 1.f, d4 = (float)(b / 3) - 1.f;
-            const float base = d3 * x3 + d4 * x4;
+        const float x4 = xs[(4 * 4 + k) * 32 + L];
+        for (int b = q; b < 9; b += 4) {
+            const float base = (float)(b % 3 - 1) * x3 + (float)(b / 3 - 1) * x4;
 #pragma unroll
             for (int d2 = 0; d2 < 3; ++d2) {
                 const float s2 = base + (float)(d2 - 1) * x2;
@@ -224,19 +238,17 @@ __device__ __forceinline__ void lut_build(const float* xs, float* table) {
             }
         }
     } else {
-        for (int task = warp; task < 64; task += kLutWarps) {
-            const int hi = task >> 2, k = task & 3;
-            const float x0 = xs[(0 * 4 + k) * 32 + L], x1 = xs[(1 * 4 + k) * 32 + L],
-                        x2 = xs[(2 * 4 + k) * 32 + L], x3 = xs[(3 * 4 + k) * 32 + L];
-            float* col = table + (k >> 1) * (kLutRegion / 4) + L + 32 * (k & 1);
+        for (int hi = q; hi < 16; hi += 4) {
             const int e2 = hi & 3, e3 = hi >> 2;
-            const bool bad_hi = e2 == 3 || e3 == 3;
+            if (e2 == 3 || e3 == 3) continue;
             const float base = (float)(e2 - 1) * x2 + (float)(e3 - 1) * x3;
 #pragma unroll
-            for (int lo = 0; lo < 16; ++lo) {
-                const int e0 = lo & 3, e1 = lo >> 2;
-                const float v = (bad_hi || e0 == 3 || e1 == 3) ? 0.f : base + (float)(e0 - 1) * x0 + (float)(e1 - 1) * x1;
-                col[(16 * hi + lo) * 64] = v;
+            for (int e1 = 0; e1 < 3; ++e1) {
+                const float s1 = base + (float)(e1 - 1) * x1;
+                const int c = 16 * hi + 4 * e1;
+                col[(c + 0) * 64] = s1 - x0;
+                col[(c + 1) * 64] = s1;
+                col[(c + 2) * 64] = s1 + x0;
             }
         }
     }
@@ -356,6 +368,7 @@ gemv_lut_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant_
                 lut_issue_set(rg, &cmap, &smap, issued + d, cx, sx, w_lo + (int64_t)d * kLutSet);
         if (chunk < a.nchunk) issued += min(kLutDepth, nsets);
     }
+    lut_zero_invalid<LAYOUT>(table);
     pdl_wait();
     pdl_launch_dependents();
 
@@ -378,7 +391,7 @@ gemv_lut_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant_
         if (!first && ok) issued += min(kLutDepth, nsets);
         first = false;
         if (new_blk) {
-            if (warp == 0) lut_rotate_block(a, blk, xf, xr, table /* FWHT exchange tile */);
+            if (warp == 0) lut_rotate_block(a, blk, xf, xr, reinterpret_cast<float*>(lut_smem + kLutTileOffset));
             cur_blk = blk;
             __syncthreads();
         }
