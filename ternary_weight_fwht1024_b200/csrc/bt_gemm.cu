@@ -23,11 +23,12 @@
 //                   tcgen05.mma.cta_group::1.kind::f16 (M 128, N BN, K 16) x 8
 //                   per stage into an FP32 accumulator in TMEM and commits
 //                   each stage to its "empty" barrier;
-//       warps 2-9   decode the packed weights of the stage (one row per
-//                   thread) to FP16 s*t -- exact -- and store them in the
-//                   tensor cores' K-major 128-byte-swizzled layout; then
-//                   they read the accumulator back (tcgen05.ld) and write
-//                   bf16 Y scaled by 2^e_m.
+//       warps 2..   decode the packed weights of the stage to FP16 s*t --
+//                   exact -- and store them in the tensor cores' K-major
+//                   128-byte-swizzled layout: two threads per weight row,
+//                   one per 64-column panel (BN / 16 warps); then warps 2-5
+//                   read the accumulator back (tcgen05.ld) and write bf16 Y
+//                   scaled by 2^e_m.
 //     A group's 128 trits are laid out in "slot" order: slot 2w + h holds
 //     half h of decoded word w. For base-3, word w < 60 is digit w % 5 of
 //     bytes (2p, 2p+1), p = w / 5; words 60-62 are digits 0-2 of bytes
@@ -45,8 +46,9 @@ namespace bt {
 
 constexpr int kGemmBM = 128;
 constexpr int kGemmBK = 128;             // one weight group per stage
-constexpr int kGemmDecWarps = 8;         // decoder / epilogue warps
-constexpr int kGemmThreads = (2 + kGemmDecWarps) * 32;
+// decoder warps: two threads per weight row of the BN-row tile
+__host__ __device__ constexpr int gemm_dec_warps(int bn) { return bn / 16; }
+__host__ __device__ constexpr int gemm_threads(int bn) { return (2 + gemm_dec_warps(bn)) * 32; }
 constexpr int kGemmLutCopies = 8;
 constexpr int kGemmLutBytes = 256 * kGemmLutCopies * 8;  // 8 copies x (low, high) x 4 bytes per code
 
@@ -236,7 +238,7 @@ struct GemmSmem {
 };
 
 template <int LAYOUT, int BN, int STAGES>
-__global__ void __launch_bounds__(kGemmThreads, 1)
+__global__ void __launch_bounds__(gemm_threads(BN), 1)
 gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
     using SM = GemmSmem<LAYOUT, BN, STAGES>;
     extern __shared__ uint8_t gsm_raw[];
@@ -264,7 +266,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
             mbar_init(smem_addr(emptyA + s), 1);
         }
         for (int s = 0; s < SB; ++s) {
-            mbar_init(smem_addr(fullB + s), kGemmDecWarps);
+            mbar_init(smem_addr(fullB + s), gemm_dec_warps(BN));
             mbar_init(smem_addr(emptyB + s), 1);
         }
         mbar_init(smem_addr(accf), 1);
@@ -340,13 +342,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
             tc_commit(smem_addr(accf));
         }
     } else {
-        // ---------------- decoders: one weight row per thread
-        const int t = threadIdx.x - 64;                 // 0 .. 255
+        // ---------------- decoders: thread (panel h, row t) decodes the 64
+        // slots of weight row t that land in panel h
+        const int tt = threadIdx.x - 64;                // 0 .. 2 BN - 1
+        const int h = tt / BN, t = tt - h * BN;
         const int n = n0 + t;
-        const bool active = t < BN;
-        const int nr = active ? n : n0;                 // rows beyond BN do no work
-        const uint8_t* rowp = a.codes + (int64_t)nr * a.row_bytes;
-        const uint16_t* srow = a.scales + (int64_t)nr * a.G;
+        const uint8_t* rowp = a.codes + (int64_t)n * a.row_bytes;
+        const uint16_t* srow = a.scales + (int64_t)n * a.G;
         const uint8_t* lut_lane = lut + (lane & (kGemmLutCopies - 1)) * 4;   // this lane's copy of the table
         constexpr uint32_t kRow = 8 * kGemmLutCopies;                         // table bytes per code
         uint32_t hm[6], ha[6];
@@ -355,20 +357,21 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
         const uint32_t hm34 = (hm[3] & 0xFFFFu) | (hm[4] & 0xFFFF0000u);
         const uint32_t ha34 = (ha[3] & 0xFFFFu) | (ha[4] & 0xFFFF0000u);
         uint32_t err = 0;
-        // the next group's packed bytes and scale are loaded one stage ahead
-        constexpr int NW = LAYOUT == BT_LAYOUT_B3 ? 13 : 8;
+        // Base-3: slots 0-63 (words 0-31) come from byte pairs 0-6, slots
+        // 64-127 (words 32-63) from pairs 6-12; pair 6 feeds both. 2-bit:
+        // panel h is the group's 32-bit words 4h .. 4h + 3.
+        constexpr int NW = LAYOUT == BT_LAYOUT_B3 ? 7 : 4;
         uint32_t cur[NW], nxt[NW], s_cur = 0, s_nxt = 0;
         auto load_group = [&](int kt, uint32_t (&dst)[NW], uint32_t& sc) {
-            if (!active || kt >= ktiles) return;
+            if (kt >= ktiles) return;
             if constexpr (LAYOUT == BT_LAYOUT_B3) {
-                const unsigned short* gp = reinterpret_cast<const unsigned short*>(rowp + (int64_t)kt * kB3GroupBytes);
+                const unsigned short* gp =
+                    reinterpret_cast<const unsigned short*>(rowp + (int64_t)kt * kB3GroupBytes) + 6 * h;
 #pragma unroll
-                for (int p = 0; p < 13; ++p) dst[p] = __ldg(gp + p);
+                for (int p = 0; p < 7; ++p) dst[p] = __ldg(gp + p);
             } else {
-                const uint4* gp = reinterpret_cast<const uint4*>(rowp + (int64_t)kt * k2bGroupBytes);
-                const uint4 q0 = __ldg(gp), q1 = __ldg(gp + 1);
-                dst[0] = q0.x; dst[1] = q0.y; dst[2] = q0.z; dst[3] = q0.w;
-                dst[4] = q1.x; dst[5] = q1.y; dst[6] = q1.z; dst[7] = q1.w;
+                const uint4 q = __ldg(reinterpret_cast<const uint4*>(rowp + (int64_t)kt * k2bGroupBytes) + h);
+                dst[0] = q.x; dst[1] = q.y; dst[2] = q.z; dst[3] = q.w;
             }
             sc = srow[kt];
         };
@@ -380,34 +383,58 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
                 bad = BT_DEVERR_TIMEOUT; *abort_flag = 1; break;
             }
             if (*abort_flag) break;
-            if (active) {
+            {
                 const uint32_t s1 = s_cur;
                 const uint32_t s2 = s1 | (s1 << 16);
-                uint8_t* bst = b_ring + s * SM::kB;
-                // row t of the B tile: panel p (slots 64p..64p+63), 8-row atoms
+                uint8_t* bst = b_ring + s * SM::kB + h * (SM::kB / 2);
+                // row t of panel h: 8-row atoms of 1024 bytes, 128 bytes per row
                 const uint32_t row_off = static_cast<uint32_t>((t >> 3) * 1024 + (t & 7) * 128);
-                uint32_t words[64];
+                uint32_t words[32];
                 if constexpr (LAYOUT == BT_LAYOUT_B3) {
-#pragma unroll
-                    for (int p = 0; p < 13; ++p) {
-                        const uint32_t pr = cur[p];
-                        const uint32_t va = *reinterpret_cast<const uint32_t*>(lut_lane + (pr & 0xFFu) * kRow);
-                        const uint32_t vb = *reinterpret_cast<const uint32_t*>(lut_lane + (pr >> 8) * kRow + kRow / 2);
+                    auto pair_fields = [&](int j, uint32_t& va, uint32_t& vb) {
+                        const uint32_t pr = cur[j];
+                        va = *reinterpret_cast<const uint32_t*>(lut_lane + (pr & 0xFFu) * kRow);
+                        vb = *reinterpret_cast<const uint32_t*>(lut_lane + (pr >> 8) * kRow + kRow / 2);
                         err |= (va | vb) & 0x80000000u;
-                        const int nw = p < 12 ? 5 : 3;
+                    };
+                    if (h == 0) {
 #pragma unroll
-                        for (int i = 0; i < nw; ++i) {
-                            const uint32_t f = lop3_or_and(va, vb, gfmask(i) | 0x64006400u);
-                            words[5 * p + i] = hmul2_u32(hfma2_u32(f, hm[i], ha[i]), s2);
+                        for (int p = 0; p < 7; ++p) {
+                            uint32_t va, vb;
+                            pair_fields(p, va, vb);
+#pragma unroll
+                            for (int i = 0; i < 5; ++i) {
+                                const int w = 5 * p + i;
+                                if (w < 32) {
+                                    const uint32_t f = lop3_or_and(va, vb, gfmask(i) | 0x64006400u);
+                                    words[w] = hmul2_u32(hfma2_u32(f, hm[i], ha[i]), s2);
+                                }
+                            }
                         }
-                        if (p == 12) {
-                            const uint32_t f = (va & 0x64C0u) | ((va & 0x300u) << 16) | 0x64000000u;
-                            words[63] = hmul2_u32(hfma2_u32(f, hm34, ha34), s2);
+                    } else {
+#pragma unroll
+                        for (int j = 0; j < 7; ++j) {
+                            const int p = 6 + j;
+                            uint32_t va, vb;
+                            pair_fields(j, va, vb);
+                            const int nw = p < 12 ? 5 : 3;
+#pragma unroll
+                            for (int i = 0; i < nw; ++i) {
+                                const int w = 5 * p + i;
+                                if (w >= 32) {
+                                    const uint32_t f = lop3_or_and(va, vb, gfmask(i) | 0x64006400u);
+                                    words[w - 32] = hmul2_u32(hfma2_u32(f, hm[i], ha[i]), s2);
+                                }
+                            }
+                            if (p == 12) {
+                                const uint32_t f = (va & 0x64C0u) | ((va & 0x300u) << 16) | 0x64000000u;
+                                words[31] = hmul2_u32(hfma2_u32(f, hm34, ha34), s2);
+                            }
                         }
                     }
                 } else {
 #pragma unroll
-                    for (int w = 0; w < 8; ++w) {
+                    for (int w = 0; w < 4; ++w) {
                         // fields 0-4 of each half in place, fields 5-7 after a
                         // 10-bit shift: a field at bits 10-11 would reach into
                         // the FP16 exponent of 1024 + d 4^i
@@ -422,9 +449,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
                     }
                 }
 #pragma unroll
-                for (int c = 0; c < 16; ++c) {
-                    const int panel = c >> 3, chunk = c & 7;
-                    uint8_t* dst = bst + panel * (SM::kB / 2) + row_off + ((chunk ^ (t & 7)) << 4);
+                for (int c = 0; c < 8; ++c) {
+                    uint8_t* dst = bst + row_off + ((c ^ (t & 7)) << 4);
                     *reinterpret_cast<uint4*>(dst) =
                         make_uint4(words[4 * c], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
                 }
@@ -504,7 +530,7 @@ static cudaError_t launch_gemm_t(const CUtensorMap& amap, const GemmArgs& ga, cu
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(ga.N / BN, ga.M / kGemmBM);
-    cfg.blockDim = dim3(kGemmThreads);
+    cfg.blockDim = dim3(gemm_threads(BN));
     cfg.dynamicSmemBytes = SM::kTotal;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
