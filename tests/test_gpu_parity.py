@@ -170,6 +170,49 @@ def test_gemv_prerotated_ragged_groups(layout, N, K):
     check(run_gemv(case, layout, rotate=False, x_f32=xr32), y_ref, b)
 
 
+# Single-row (M = 1) calls with K % 1024 == 0 take the table-lookup kernel:
+# one K chunk of 512 per CTA and row slices, or, with more chunks than SMs,
+# CTAs that walk chunks. These cases cover its branches.
+
+@pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
+@pytest.mark.parametrize("N,K", [(1, 1024), (3, 2048), (17, 1024), (77, 3072), (1000, 17408)])
+def test_gemv_m1_prerotated_f32(layout, N, K):
+    case = workloads.random_case(2400 + N + K, 1, N, K)
+    xr = workloads.rng(2500 + N).standard_normal((1, K)) * 3.0
+    xr32 = xr.astype(np.float32).astype(np.float64)
+    y_ref, b = oracle.gemv(case["trits"], case["scales"], xr32)
+    check(run_gemv(case, layout, rotate=False, x_f32=xr32), y_ref, b)
+
+
+@pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
+def test_gemv_m1_prerotated_bf16(layout):
+    N, K = 300, 5120
+    case = workloads.random_case(2600, 1, N, K)
+    xbits = workloads.activations_bf16_bits(workloads.rng(2601), 1, K, True)
+    xr = oracle.bf16_to_f64(xbits)
+    y_ref, b = oracle.gemv(case["trits"], case["scales"], xr)
+    codes = bt.pack(T(case["trits"]), layout)
+    y = bt.gemv(codes, T(case["scales"]), T(xbits, "bf16"), None, N, layout)
+    check(f64(y), y_ref, b)
+
+
+@pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
+def test_gemv_m1_walks_chunks(layout):
+    # 76 blocks = 152 chunks of 512: more chunks than SMs, so CTAs walk chunks
+    N, K = 40, 76 * 1024
+    case = workloads.random_case(2700, 1, N, K)
+    _, y_ref, b = oracle.forward(case["trits"], case["scales"], case["x"], case["sign"])
+    check(run_gemv(case, layout), y_ref, b)
+
+
+@pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
+def test_gemv_m1_bf16_output(layout):
+    case = workloads.random_case(2800, 1, 5120, 5120)
+    _, y_ref, b = oracle.forward(case["trits"], case["scales"], case["x"], case["sign"])
+    y = run_gemv(case, layout, y_dtype=bt.BF16)
+    check(y, y_ref, b, extra=np.abs(y_ref) * 2.0 ** -8)
+
+
 def test_gemv_bf16_output():
     case = workloads.random_case(4000, 4, 512, 2048)
     _, y_ref, b = oracle.forward(case["trits"], case["scales"], case["x"], case["sign"])
