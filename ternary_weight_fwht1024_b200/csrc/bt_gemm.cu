@@ -365,10 +365,29 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
         auto load_group = [&](int kt, uint32_t (&dst)[NW], uint32_t& sc) {
             if (kt >= ktiles) return;
             if constexpr (LAYOUT == BT_LAYOUT_B3) {
-                const unsigned short* gp =
-                    reinterpret_cast<const unsigned short*>(rowp + (int64_t)kt * kB3GroupBytes) + 6 * h;
+                // bytes [s, s + 14) through the 8-byte aligned window of 16 or
+                // 24 bytes that holds them (alignment taken from the address:
+                // rows are only 2-byte aligned when K % 512 != 0). Every word
+                // of the window shares its aligned 8 bytes with a byte of the
+                // row, so no load leaves the buffer's last aligned block.
+                const uintptr_t sa = reinterpret_cast<uintptr_t>(rowp) + (uintptr_t)(kt * kB3GroupBytes + 12 * h);
+                const int sh = (int)(sa & 7);                // 0, 2, 4 or 6
+                const uint2* wp = reinterpret_cast<const uint2*>(sa - (uintptr_t)sh);
+                const uint2 x0 = __ldg(wp), x1 = __ldg(wp + 1);
+                const uint2 x2 = sh > 2 ? __ldg(wp + 2) : make_uint2(0u, 0u);
+                const uint32_t w6[6] = {x0.x, x0.y, x1.x, x1.y, x2.x, x2.y};
+                // 32-bit words at byte offsets sh, sh + 4, sh + 8, sh + 12
+                uint32_t v[4];
+                const uint32_t bits = 8u * (uint32_t)(sh & 3);
+                const bool up = sh >= 4;
 #pragma unroll
-                for (int p = 0; p < 7; ++p) dst[p] = __ldg(gp + p);
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t lo = up ? w6[i + 1] : w6[i];
+                    const uint32_t hi = up ? w6[i + 2] : w6[i + 1];
+                    v[i] = __funnelshift_r(lo, hi, bits);
+                }
+#pragma unroll
+                for (int p = 0; p < 7; ++p) dst[p] = (p & 1) ? (v[p >> 1] >> 16) : (v[p >> 1] & 0xFFFFu);
             } else {
                 const uint4 q = __ldg(reinterpret_cast<const uint4*>(rowp + (int64_t)kt * k2bGroupBytes) + h);
                 dst[0] = q.x; dst[1] = q.y; dst[2] = q.z; dst[3] = q.w;
