@@ -224,11 +224,18 @@ struct GemmArgs {
     int32_t* dev_err;
 };
 
+#ifndef BT_GEMM_ASTAGES
+#define BT_GEMM_ASTAGES 2
+#endif
+#ifndef BT_GEMM_BSTAGES
+#define BT_GEMM_BSTAGES 3
+#endif
+
 template <int LAYOUT, int BN, int STAGES>
 struct GemmSmem {
     // activation ring (TMA) is deeper than the weight ring (decoded in the
     // CTA): activation tiles come from L2/HBM and need the longer lead
-    static constexpr int kAStages = 4;
+    static constexpr int kAStages = BT_GEMM_ASTAGES;
     static constexpr int kBStages = STAGES;
     static constexpr int kA = kGemmBM * kGemmBK * 2;   // 32 KB: two 64-column panels
     static constexpr int kB = BN * kGemmBK * 2;
@@ -361,7 +368,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
         // 64-127 (words 32-63) from pairs 6-12; pair 6 feeds both. 2-bit:
         // panel h is the group's 32-bit words 4h .. 4h + 3.
         constexpr int NW = LAYOUT == BT_LAYOUT_B3 ? 7 : 4;
-        uint32_t cur[NW], nxt[NW], s_cur = 0, s_nxt = 0;
         auto load_group = [&](int kt, uint32_t (&dst)[NW], uint32_t& sc) {
             if (kt >= ktiles) return;
             if constexpr (LAYOUT == BT_LAYOUT_B3) {
@@ -394,16 +400,17 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
             }
             sc = srow[kt];
         };
-        load_group(0, cur, s_cur);
-        for (int kt = 0; kt < ktiles; ++kt) {
+        // Stage kt decodes group kt from registers loaded two stages earlier:
+        // the loop is unrolled by two over two named buffers, so no register
+        // copy waits on a load in flight.
+        auto stage = [&](int kt, const uint32_t (&cw)[NW], uint32_t scv) -> bool {
             const int s = kt % SB;
-            load_group(kt + 1, nxt, s_nxt);
             if (kt >= SB && !mbar_wait(smem_addr(emptyB + s), ((kt / SB) - 1) & 1)) {
-                bad = BT_DEVERR_TIMEOUT; *abort_flag = 1; break;
+                bad = BT_DEVERR_TIMEOUT; *abort_flag = 1; return false;
             }
-            if (*abort_flag) break;
+            if (*abort_flag) return false;
             {
-                const uint32_t s1 = s_cur;
+                const uint32_t s1 = scv;
                 const uint32_t s2 = s1 | (s1 << 16);
                 uint8_t* bst = b_ring + s * SM::kB + h * (SM::kB / 2);
                 // row t of panel h: 8-row atoms of 1024 bytes, 128 bytes per row
@@ -411,7 +418,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
                 uint32_t words[32];
                 if constexpr (LAYOUT == BT_LAYOUT_B3) {
                     auto pair_fields = [&](int j, uint32_t& va, uint32_t& vb) {
-                        const uint32_t pr = cur[j];
+                        const uint32_t pr = cw[j];
                         va = *reinterpret_cast<const uint32_t*>(lut_lane + (pr & 0xFFu) * kRow);
                         vb = *reinterpret_cast<const uint32_t*>(lut_lane + (pr >> 8) * kRow + kRow / 2);
                         err |= (va | vb) & 0x80000000u;
@@ -457,7 +464,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
                         // fields 0-4 of each half in place, fields 5-7 after a
                         // 10-bit shift: a field at bits 10-11 would reach into
                         // the FP16 exponent of 1024 + d 4^i
-                        const uint32_t x = cur[w], x10 = x >> 10;
+                        const uint32_t x = cw[w], x10 = x >> 10;
                         err |= x & (x >> 1) & 0x55555555u;
 #pragma unroll
                         for (int f = 0; f < 8; ++f) {
@@ -474,12 +481,20 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
                         make_uint4(words[4 * c], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
                 }
             }
-#pragma unroll
-            for (int i = 0; i < NW; ++i) cur[i] = nxt[i];
-            s_cur = s_nxt;
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) mbar_arrive(smem_addr(fullB + s));
+            return true;
+        };
+        uint32_t bufA[NW], bufB[NW], sA = 0, sB = 0;
+        load_group(0, bufA, sA);
+        load_group(1, bufB, sB);
+        for (int kt = 0; kt < ktiles; kt += 2) {
+            if (!stage(kt, bufA, sA)) break;
+            load_group(kt + 2, bufA, sA);
+            if (kt + 1 >= ktiles) break;
+            if (!stage(kt + 1, bufB, sB)) break;
+            load_group(kt + 3, bufB, sB);
         }
         if (LAYOUT == BT_LAYOUT_B3 ? (err >> 31) : (err != 0)) bad |= BT_DEVERR_INVALID_CODE;
 
@@ -528,6 +543,9 @@ size_t gemm_workspace_bytes(int, int64_t M, int64_t, int64_t K, int) {
 }
 
 static int pick_bn(int64_t M, int64_t N, int num_sms) {
+#ifdef BT_GEMM_BN_FORCE
+    if (N % BT_GEMM_BN_FORCE == 0) return BT_GEMM_BN_FORCE;
+#endif
     const int cands[2] = {160, 128};
     int best = 128;
     double best_eff = -1.0;
@@ -562,7 +580,8 @@ static cudaError_t launch_gemm_t(const CUtensorMap& amap, const GemmArgs& ga, cu
 
 template <int LAYOUT>
 static cudaError_t dispatch_gemm(int bn, const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t s) {
-    return bn == 160 ? launch_gemm_t<LAYOUT, 160, 2>(amap, ga, s) : launch_gemm_t<LAYOUT, 128, 2>(amap, ga, s);
+    return bn == 160 ? launch_gemm_t<LAYOUT, 160, BT_GEMM_BSTAGES>(amap, ga, s)
+                     : launch_gemm_t<LAYOUT, 128, BT_GEMM_BSTAGES>(amap, ga, s);
 }
 
 cudaError_t launch_gemm(int layout, const uint8_t* codes, const uint16_t* scales, const void* x, int x_dtype,
