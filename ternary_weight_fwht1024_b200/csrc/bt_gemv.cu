@@ -1313,7 +1313,10 @@ cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
 
-    const TmaPlan tp = make_tma_plan(layout, M, N, K, scales, num_sms);
+    // The TMA-fed kernel takes up to 8 activation rows (one n8 MMA column
+    // block); 9-16 rows run as two launches over the same prepared
+    // fragments, each streaming the weights once.
+    const TmaPlan tp = make_tma_plan(layout, M < 8 ? M : 8, N, K, scales, num_sms);
     EncodeTiledFn enc = tp.use ? tensor_map_encoder() : nullptr;
     if (tp.use && enc) {
         const int RB = layout == BT_LAYOUT_B3 ? 8 * kB3GroupBytes : 8 * k2bGroupBytes;
@@ -1334,23 +1337,31 @@ cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales
                                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
         if (oks) {
-            GemvTmaArgs ta{};
-            ta.bslots = pa.bslots;
-            ta.meta = pa.meta;
-            ta.partials = reinterpret_cast<float*>(ws + pl.off_partials);
-            ta.counters = pa.counters;
-            ta.y = y;
-            ta.y_bf16 = y_dtype == BT_BF16;
-            ta.M = static_cast<int>(M);
-            ta.N = static_cast<int>(N);
-            ta.G = static_cast<int>(pl.G);
-            ta.nb = tp.nb;
-            ta.stages = tp.stages;
-            ta.items = tp.items;
-            ta.chunk = tp.chunk;
-            ta.dev_err = dev_err;
-            return layout == BT_LAYOUT_B3 ? dispatch_gemv_tma<BT_LAYOUT_B3>(cmap, smap, ta, tp, stream)
-                                          : dispatch_gemv_tma<BT_LAYOUT_2BIT>(cmap, smap, ta, tp, stream);
+            for (int64_t m0 = 0; m0 < M; m0 += 8) {
+                // each launch waits for the previous one (programmatic
+                // dependency) before it touches the partials; tile counters
+                // are back at zero when a launch ends
+                GemvTmaArgs ta{};
+                ta.bslots = pa.bslots + m0 * pl.G * pl.NT * 8;
+                ta.meta = pa.meta + m0 * pl.G;
+                ta.partials = reinterpret_cast<float*>(ws + pl.off_partials);
+                ta.counters = pa.counters;
+                ta.y = static_cast<uint8_t*>(y) + m0 * N * (y_dtype == BT_BF16 ? 2 : 4);
+                ta.y_bf16 = y_dtype == BT_BF16;
+                ta.M = static_cast<int>(M - m0 < 8 ? M - m0 : 8);
+                ta.N = static_cast<int>(N);
+                ta.G = static_cast<int>(pl.G);
+                ta.nb = tp.nb;
+                ta.stages = tp.stages;
+                ta.items = tp.items;
+                ta.chunk = tp.chunk;
+                ta.dev_err = dev_err;
+                const cudaError_t e2 = layout == BT_LAYOUT_B3
+                                           ? dispatch_gemv_tma<BT_LAYOUT_B3>(cmap, smap, ta, tp, stream)
+                                           : dispatch_gemv_tma<BT_LAYOUT_2BIT>(cmap, smap, ta, tp, stream);
+                if (e2 != cudaSuccess) return e2;
+            }
+            return cudaSuccess;
         }
     }
 
