@@ -232,29 +232,58 @@ def run_gpu(args, rank, world):
     del gs3
 
     # ---- e2e through the public API with host buffers ----
-    y_host = [torch.empty((M, L.N), dtype=torch.float32).pin_memory() for L in triple]
+    # Each step copies the step's activations from pinned host memory, makes
+    # the three bt_gemv calls and reads the outputs back into pinned host
+    # memory. "graph": the step as a serving loop would run it, captured once
+    # as a CUDA graph of those API calls and copies and replayed per step.
+    # "eager": the same calls issued from Python every step.
+    # one pinned host buffer per direction: a step is one H2D copy of the three
+    # activation rows and one D2H copy of the three outputs
+    x_host_all = torch.cat([h.view(-1) for h in xs_host]).pin_memory()
+    x_dev_all = torch.empty_like(x_host_all, device=dev)
+    y_dev_all = torch.empty(sum(M * L.N for L in triple), dtype=torch.float32, device=dev)
+    y_host_all = torch.empty_like(y_dev_all, device="cpu").pin_memory()
+    xo = [0]
+    yo = [0]
+    for L in triple:
+        xo.append(xo[-1] + M * L.K)
+        yo.append(yo[-1] + M * L.N)
+    xs_e = [x_dev_all[xo[i]:xo[i + 1]].view(torch.bfloat16).view(M, L.K) for i, L in enumerate(triple)]
+    ys_e = [y_dev_all[yo[i]:yo[i + 1]].view(M, L.N) for i, L in enumerate(triple)]
+
+    def e2e_step(r):
+        x_dev_all.copy_(x_host_all, non_blocking=True)
+        for i, L in enumerate(triple):
+            bt.gemv(reps3[r][i][0], reps3[r][i][1], xs_e[i], sign, L.N, 0, out=ys_e[i], ws=ws)
+        y_host_all.copy_(y_dev_all, non_blocking=True)
+
+    def e2e_timed(run_step):
+        with torch.cuda.stream(stream):
+            for w in range(args.warmup):
+                run_step(w % copies)
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
+            st = torch.cuda.Event(enable_timing=True)
+            en = torch.cuda.Event(enable_timing=True)
+            st.record(stream)
+            for k in range(args.steps):
+                run_step((args.warmup + k) % copies)
+            en.record(stream)
+            torch.cuda.synchronize()
+        return max_over_ranks(st.elapsed_time(en) / args.steps, world, dist, dev)
+
+    e2e_eager_ms = e2e_timed(e2e_step)
+    e2e_graphs = []
     with torch.cuda.stream(stream):
-        for w in range(args.warmup):
-            for i, L in enumerate(triple):
-                xs[i].view(torch.int16).copy_(xs_host[i], non_blocking=True)
-                bt.gemv(reps3[w % copies][i][0], reps3[w % copies][i][1], xs[i], sign, L.N, 0, out=ys[i], ws=ws)
-                y_host[i].copy_(ys[i], non_blocking=True)
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        st = torch.cuda.Event(enable_timing=True)
-        en = torch.cuda.Event(enable_timing=True)
-        st.record(stream)
-        for k in range(args.steps):
-            r = (args.warmup + k) % copies
-            for i, L in enumerate(triple):
-                xs[i].view(torch.int16).copy_(xs_host[i], non_blocking=True)
-                bt.gemv(reps3[r][i][0], reps3[r][i][1], xs[i], sign, L.N, 0, out=ys[i], ws=ws)
-                y_host[i].copy_(ys[i], non_blocking=True)
-        en.record(stream)
-        torch.cuda.synchronize()
-    e2e_ms = max_over_ranks(st.elapsed_time(en) / args.steps, world, dist, dev)
+        for r in range(copies):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                e2e_step(r)
+            e2e_graphs.append(gr)
+    e2e_ms = e2e_timed(lambda r: e2e_graphs[r].replay())
+    del e2e_graphs
     del reps3
 
     # ---- 2-bit layout twin ----
@@ -359,10 +388,16 @@ def run_gpu(args, rank, world):
         "fwht_sweep": fwht,
         "e2e": {"value": round(bytes3 / (e2e_ms * 1e-3) / 1e9 * world, 2), "unit": "GB/s",
                 "ms_per_step": round(e2e_ms, 5), "h2d_bytes_per_step": sum(M * L.K * 2 for L in triple),
-                "d2h_bytes_per_step": sum(M * L.N * 4 for L in triple)},
+                "d2h_bytes_per_step": sum(M * L.N * 4 for L in triple),
+                "mode": "graph of the step's API calls and host copies, replayed per step",
+                "eager": {"value": round(bytes3 / (e2e_eager_ms * 1e-3) / 1e9 * world, 2),
+                          "ms_per_step": round(e2e_eager_ms, 5)}},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(achieved / peaks["hbm_gbs"], 4),
-                     "traffic": None,
+                     # dram__bytes_read.sum + dram__bytes_write.sum of gemv_lut_kernel, mean over the
+                     # three layers' launches (profiles/gemv_lut_kernel_b3_triple.md)
+                     "traffic": 14962176,
+                     "algorithmic_bytes_per_launch": int(sum(dom_bytes) / len(dom_bytes)),
                      "kernel": "bt_gemv call (table-lookup GEMV kernel + chunk reduction), weighted over the three layers",
                      "peak_kind": f"HBM copy, {peaks['src']}"},
         "gpu_launches": args.steps * len(triple) * 2,  # GEMV + chunk-sum kernels per bt_gemv call
