@@ -25,8 +25,9 @@
 //                   each stage to its "empty" barrier;
 //       warps 2..   decode the packed weights of the stage to FP16 s*t --
 //                   exact -- and store them in the tensor cores' K-major
-//                   128-byte-swizzled layout: two threads per weight row,
-//                   one per 64-column panel (BN / 16 warps); then warps 2-5
+//                   128-byte-swizzled layout: BT_GEMM_TPR (2) threads per
+//                   weight row, each one 128 / TPR-slot part of the group
+//                   (BN TPR / 32 warps); then warps 2-5
 //                   read the accumulator back (tcgen05.ld) and write bf16 Y
 //                   scaled by 2^e_m.
 //     A group's 128 trits are laid out in "slot" order: slot 2w + h holds
@@ -46,8 +47,13 @@ namespace bt {
 
 constexpr int kGemmBM = 128;
 constexpr int kGemmBK = 128;             // one weight group per stage
-// decoder warps: two threads per weight row of the BN-row tile
-__host__ __device__ constexpr int gemm_dec_warps(int bn) { return bn / 16; }
+// decoder warps: TPR threads per weight row of the BN-row tile, each decoding
+// 128 / TPR of a group's slots
+#ifndef BT_GEMM_TPR
+#define BT_GEMM_TPR 2
+#endif
+constexpr int kGemmTpr = BT_GEMM_TPR;
+__host__ __device__ constexpr int gemm_dec_warps(int bn) { return bn * kGemmTpr / 32; }
 __host__ __device__ constexpr int gemm_threads(int bn) { return (2 + gemm_dec_warps(bn)) * 32; }
 constexpr int kGemmLutCopies = 8;
 constexpr int kGemmLutBytes = 256 * kGemmLutCopies * 8;  // 8 copies x (low, high) x 4 bytes per code
@@ -132,6 +138,67 @@ __device__ __forceinline__ uint32_t h2_mul_of(int i) {
 __device__ __forceinline__ uint32_t h2_add_of(int i) {
     const uint32_t h = __half_as_ushort(__float2half_rn(-(ldexpf(1024.f, -2 * i) + 1.f)));
     return h | (h << 16);
+}
+
+// Words per decoder thread and packed words it reads, per layout.
+template <int LAYOUT>
+struct GemmPart {
+    static constexpr int WPT = 64 / kGemmTpr;
+    static constexpr int NW = LAYOUT == BT_LAYOUT_B3 ? (kGemmTpr == 2 ? 7 : 4) : WPT / 8;
+};
+
+// Decode part QQ of one group (WPT words of FP16 pairs s t, slot order) from
+// the part's packed words. Base-3 word w < 60 is digit w % 5 of byte pair
+// w / 5; words 60-62 are digits 0-2 of pair 12, word 63 digits 3-4 of byte
+// 24. 2-bit: word 8 q + f holds fields f and 8 + f of the group's 32-bit
+// word q.
+template <int LAYOUT, int QQ>
+__device__ __forceinline__ void gemm_decode_part(const uint32_t (&cw)[GemmPart<LAYOUT>::NW], uint32_t s2,
+                                                 uint32_t (&words)[GemmPart<LAYOUT>::WPT], const uint8_t* lut_lane,
+                                                 const uint32_t (&hm)[6], const uint32_t (&ha)[6], uint32_t hm34,
+                                                 uint32_t ha34, uint32_t& err) {
+    constexpr int WPT = GemmPart<LAYOUT>::WPT, NW = GemmPart<LAYOUT>::NW;
+    constexpr int W0 = WPT * QQ, W1 = W0 + WPT, P0 = W0 / 5;
+    constexpr uint32_t kRow = 8 * kGemmLutCopies;
+    if constexpr (LAYOUT == BT_LAYOUT_B3) {
+#pragma unroll
+        for (int j = 0; j < NW; ++j) {
+            const int p = P0 + j;
+            if (p > 12) continue;
+            const uint32_t pr = cw[j];
+            const uint32_t va = *reinterpret_cast<const uint32_t*>(lut_lane + (pr & 0xFFu) * kRow);
+            const uint32_t vb = *reinterpret_cast<const uint32_t*>(lut_lane + (pr >> 8) * kRow + kRow / 2);
+            err |= (va | vb) & 0x80000000u;
+            const int nw = p < 12 ? 5 : 3;
+#pragma unroll
+            for (int i = 0; i < nw; ++i) {
+                const int w = 5 * p + i;
+                if (w >= W0 && w < W1) {
+                    const uint32_t f = lop3_or_and(va, vb, gfmask(i) | 0x64006400u);
+                    words[w - W0] = hmul2_u32(hfma2_u32(f, hm[i], ha[i]), s2);
+                }
+            }
+            if (p == 12 && W1 == 64) {
+                const uint32_t f = (va & 0x64C0u) | ((va & 0x300u) << 16) | 0x64000000u;
+                words[63 - W0] = hmul2_u32(hfma2_u32(f, hm34, ha34), s2);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int w = 0; w < NW; ++w) {
+            // fields 0-4 of each half in place, fields 5-7 after a 10-bit
+            // shift: a field at bits 10-11 would reach into the FP16
+            // exponent of 1024 + d 4^i
+            const uint32_t x = cw[w], x10 = x >> 10;
+            err |= x & (x >> 1) & 0x55555555u;
+#pragma unroll
+            for (int f = 0; f < 8; ++f) {
+                const uint32_t fl = (f < 5 ? (x & gfmask(f)) : (x10 & gfmask(f - 5))) | 0x64006400u;
+                const int i = f < 5 ? f : f - 5;
+                words[8 * w + f] = hmul2_u32(hfma2_u32(fl, hm[i], ha[i]), s2);
+            }
+        }
+    }
 }
 
 // ------------------------------------------------------------------ prep ----
@@ -349,54 +416,68 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
             tc_commit(smem_addr(accf));
         }
     } else {
-        // ---------------- decoders: thread (panel h, row t) decodes the 64
-        // slots of weight row t that land in panel h
-        const int tt = threadIdx.x - 64;                // 0 .. 2 BN - 1
-        const int h = tt / BN, t = tt - h * BN;
+        // ---------------- decoders: thread (part qq, row t) decodes the 128 /
+        // TPR slots of weight row t with index 128 qq / TPR and up; they lie
+        // in panel h (64-slot halves of the group)
+        constexpr int TPR = kGemmTpr;
+        constexpr int WPT = GemmPart<LAYOUT>::WPT;      // 32-bit words per thread
+        const int tt = threadIdx.x - 64;                // 0 .. TPR BN - 1
+        const int qq = tt / BN, t = tt - qq * BN;
+        const int h = qq * WPT / 32;                    // panel
         const int n = n0 + t;
         const uint8_t* rowp = a.codes + (int64_t)n * a.row_bytes;
         const uint16_t* srow = a.scales + (int64_t)n * a.G;
         const uint8_t* lut_lane = lut + (lane & (kGemmLutCopies - 1)) * 4;   // this lane's copy of the table
-        constexpr uint32_t kRow = 8 * kGemmLutCopies;                         // table bytes per code
         uint32_t hm[6], ha[6];
 #pragma unroll
         for (int i = 0; i < 6; ++i) { hm[i] = h2_mul_of(i); ha[i] = h2_add_of(i); }
         const uint32_t hm34 = (hm[3] & 0xFFFFu) | (hm[4] & 0xFFFF0000u);
         const uint32_t ha34 = (ha[3] & 0xFFFFu) | (ha[4] & 0xFFFF0000u);
         uint32_t err = 0;
-        // Base-3: slots 0-63 (words 0-31) come from byte pairs 0-6, slots
-        // 64-127 (words 32-63) from pairs 6-12; pair 6 feeds both. 2-bit:
-        // panel h is the group's 32-bit words 4h .. 4h + 3.
-        constexpr int NW = LAYOUT == BT_LAYOUT_B3 ? 7 : 4;
+        // Base-3: word w < 60 is digit w % 5 of byte pair w / 5; words 60-63
+        // come from pair 12. The words of part qq, [WPT qq, WPT qq + WPT), use
+        // the pairs from WPT qq / 5 on: 7 pairs for TPR = 2, 4 for TPR = 4.
+        // 2-bit: part qq is the group's 32-bit words WPT qq / 8 and on.
+        constexpr int NW = GemmPart<LAYOUT>::NW;
+        const int p_lo = (WPT * qq) / 5;
         auto load_group = [&](int kt, uint32_t (&dst)[NW], uint32_t& sc) {
             if (kt >= ktiles) return;
             if constexpr (LAYOUT == BT_LAYOUT_B3) {
-                // bytes [s, s + 14) through the 8-byte aligned window of 16 or
-                // 24 bytes that holds them (alignment taken from the address:
-                // rows are only 2-byte aligned when K % 512 != 0). Every word
-                // of the window shares its aligned 8 bytes with a byte of the
-                // row, so no load leaves the buffer's last aligned block.
-                const uintptr_t sa = reinterpret_cast<uintptr_t>(rowp) + (uintptr_t)(kt * kB3GroupBytes + 12 * h);
+                // the 2 NW bytes from pair p_lo through the 8-byte aligned
+                // window that holds them (alignment taken from the address:
+                // rows are only 2-byte aligned when K % 512 != 0). A window
+                // word is loaded only if it holds a needed byte, so no load
+                // leaves the buffer's last aligned block.
+                constexpr int NB = 2 * NW;                   // 14 or 8 bytes
+                const uintptr_t sa = reinterpret_cast<uintptr_t>(rowp) + (uintptr_t)(kt * kB3GroupBytes + 2 * p_lo);
                 const int sh = (int)(sa & 7);                // 0, 2, 4 or 6
                 const uint2* wp = reinterpret_cast<const uint2*>(sa - (uintptr_t)sh);
-                const uint2 x0 = __ldg(wp), x1 = __ldg(wp + 1);
-                const uint2 x2 = sh > 2 ? __ldg(wp + 2) : make_uint2(0u, 0u);
+                const uint2 x0 = __ldg(wp);
+                const uint2 x1 = sh + NB > 8 ? __ldg(wp + 1) : make_uint2(0u, 0u);
+                const uint2 x2 = sh + NB > 16 ? __ldg(wp + 2) : make_uint2(0u, 0u);
                 const uint32_t w6[6] = {x0.x, x0.y, x1.x, x1.y, x2.x, x2.y};
-                // 32-bit words at byte offsets sh, sh + 4, sh + 8, sh + 12
-                uint32_t v[4];
+                // 32-bit words at byte offsets sh, sh + 4, ...
+                constexpr int NV = (NB + 3) / 4;
+                uint32_t v[NV];
                 const uint32_t bits = 8u * (uint32_t)(sh & 3);
                 const bool up = sh >= 4;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
+                for (int i = 0; i < NV; ++i) {
                     const uint32_t lo = up ? w6[i + 1] : w6[i];
                     const uint32_t hi = up ? w6[i + 2] : w6[i + 1];
                     v[i] = __funnelshift_r(lo, hi, bits);
                 }
 #pragma unroll
-                for (int p = 0; p < 7; ++p) dst[p] = (p & 1) ? (v[p >> 1] >> 16) : (v[p >> 1] & 0xFFFFu);
+                for (int p = 0; p < NW; ++p) dst[p] = (p & 1) ? (v[p >> 1] >> 16) : (v[p >> 1] & 0xFFFFu);
             } else {
-                const uint4 q = __ldg(reinterpret_cast<const uint4*>(rowp + (int64_t)kt * k2bGroupBytes) + h);
-                dst[0] = q.x; dst[1] = q.y; dst[2] = q.z; dst[3] = q.w;
+                const uint32_t* gp = reinterpret_cast<const uint32_t*>(rowp + (int64_t)kt * k2bGroupBytes) + NW * qq;
+                if constexpr (NW == 4) {
+                    const uint4 q = __ldg(reinterpret_cast<const uint4*>(gp));
+                    dst[0] = q.x; dst[1] = q.y; dst[2] = q.z; dst[3] = q.w;
+                } else {
+                    const uint2 q = __ldg(reinterpret_cast<const uint2*>(gp));
+                    dst[0] = q.x; dst[1] = q.y;
+                }
             }
             sc = srow[kt];
         };
@@ -415,68 +496,18 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
                 uint8_t* bst = b_ring + s * SM::kB + h * (SM::kB / 2);
                 // row t of panel h: 8-row atoms of 1024 bytes, 128 bytes per row
                 const uint32_t row_off = static_cast<uint32_t>((t >> 3) * 1024 + (t & 7) * 128);
-                uint32_t words[32];
-                if constexpr (LAYOUT == BT_LAYOUT_B3) {
-                    auto pair_fields = [&](int j, uint32_t& va, uint32_t& vb) {
-                        const uint32_t pr = cw[j];
-                        va = *reinterpret_cast<const uint32_t*>(lut_lane + (pr & 0xFFu) * kRow);
-                        vb = *reinterpret_cast<const uint32_t*>(lut_lane + (pr >> 8) * kRow + kRow / 2);
-                        err |= (va | vb) & 0x80000000u;
-                    };
-                    if (h == 0) {
-#pragma unroll
-                        for (int p = 0; p < 7; ++p) {
-                            uint32_t va, vb;
-                            pair_fields(p, va, vb);
-#pragma unroll
-                            for (int i = 0; i < 5; ++i) {
-                                const int w = 5 * p + i;
-                                if (w < 32) {
-                                    const uint32_t f = lop3_or_and(va, vb, gfmask(i) | 0x64006400u);
-                                    words[w] = hmul2_u32(hfma2_u32(f, hm[i], ha[i]), s2);
-                                }
-                            }
-                        }
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 7; ++j) {
-                            const int p = 6 + j;
-                            uint32_t va, vb;
-                            pair_fields(j, va, vb);
-                            const int nw = p < 12 ? 5 : 3;
-#pragma unroll
-                            for (int i = 0; i < nw; ++i) {
-                                const int w = 5 * p + i;
-                                if (w >= 32) {
-                                    const uint32_t f = lop3_or_and(va, vb, gfmask(i) | 0x64006400u);
-                                    words[w - 32] = hmul2_u32(hfma2_u32(f, hm[i], ha[i]), s2);
-                                }
-                            }
-                            if (p == 12) {
-                                const uint32_t f = (va & 0x64C0u) | ((va & 0x300u) << 16) | 0x64000000u;
-                                words[31] = hmul2_u32(hfma2_u32(f, hm34, ha34), s2);
-                            }
-                        }
-                    }
-                } else {
-#pragma unroll
-                    for (int w = 0; w < 4; ++w) {
-                        // fields 0-4 of each half in place, fields 5-7 after a
-                        // 10-bit shift: a field at bits 10-11 would reach into
-                        // the FP16 exponent of 1024 + d 4^i
-                        const uint32_t x = cw[w], x10 = x >> 10;
-                        err |= x & (x >> 1) & 0x55555555u;
-#pragma unroll
-                        for (int f = 0; f < 8; ++f) {
-                            const uint32_t fl = (f < 5 ? (x & gfmask(f)) : (x10 & gfmask(f - 5))) | 0x64006400u;
-                            const int i = f < 5 ? f : f - 5;
-                            words[8 * w + f] = hmul2_u32(hfma2_u32(fl, hm[i], ha[i]), s2);
-                        }
-                    }
+                uint32_t words[WPT];
+                switch (qq) {
+                    case 0: gemm_decode_part<LAYOUT, 0>(cw, s2, words, lut_lane, hm, ha, hm34, ha34, err); break;
+                    case 1: gemm_decode_part<LAYOUT, 1>(cw, s2, words, lut_lane, hm, ha, hm34, ha34, err); break;
+                    case 2: gemm_decode_part<LAYOUT, 2 % kGemmTpr>(cw, s2, words, lut_lane, hm, ha, hm34, ha34, err); break;
+                    default: gemm_decode_part<LAYOUT, 3 % kGemmTpr>(cw, s2, words, lut_lane, hm, ha, hm34, ha34, err); break;
                 }
+                // 16-byte chunks of the panel row: chunk c0 + c, c0 = first chunk of this part
+                const int c0 = (qq * WPT / 4) & 7;
 #pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    uint8_t* dst = bst + row_off + ((c ^ (t & 7)) << 4);
+                for (int c = 0; c < WPT / 4; ++c) {
+                    uint8_t* dst = bst + row_off + (((c0 + c) ^ (t & 7)) << 4);
                     *reinterpret_cast<uint4*>(dst) =
                         make_uint4(words[4 * c], words[4 * c + 1], words[4 * c + 2], words[4 * c + 3]);
                 }
