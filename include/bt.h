@@ -116,7 +116,8 @@ bt_status bt_fwht1024(const uint16_t* x_bf16, const int8_t* sign1024, int64_t M,
  * 1 <= M <= 16.
  *  layout    BT_LAYOUT_B3 or BT_LAYOUT_2BIT
  *  codes     device [N][bt_codes_row_bytes(layout, K)], 16-byte aligned
- *  scales    device fp16 bits [N][K/128], 4-byte aligned
+ *  scales    device fp16 bits [N][K/128], 4-byte aligned (16-byte aligned
+ *            for the fastest kernels)
  *  x         device [M][K]. If sign1024 != NULL, x is the raw activation in
  *            bf16 (x_dtype must be BT_BF16) and the rotation is applied
  *            first (K % 1024 == 0). If sign1024 == NULL, x is already
@@ -128,10 +129,24 @@ bt_status bt_fwht1024(const uint16_t* x_bf16, const int8_t* sign1024, int64_t M,
  *  dev_err   nullable. When given, the packed codes are validated on the
  *            fly and invalid ones set BT_DEVERR_INVALID_CODE (their
  *            contribution is then unspecified but finite); when NULL the
- *            check is skipped (it costs one ALU op per byte pair).
- * Numerics: the rotated activation feeds FP16 tensor-core products with FP32
+ *            check is skipped (it costs one ALU op per byte pair or word).
+ *            A copy that does not arrive within a bounded wait sets
+ *            BT_DEVERR_TIMEOUT and the affected outputs are unspecified.
+ * Kernels: M = 1 with K % 1024 == 0 and 16-byte aligned scales runs the
+ * table-lookup kernel (per-call tables of the 5- or 4-trit partial dot
+ * products of x', one lookup per packed byte, FP32 throughout) and a kernel
+ * that sums its per-512-column partials; other shapes run a prep kernel
+ * (rotation, FP16 activation fragments) and an mma.sync kernel (M <= 8 per
+ * launch; 9-16 rows take two launches). Consecutive kernels of a call, and
+ * of consecutive calls, overlap through programmatic dependent launch: a
+ * kernel may start reading codes and scales before the preceding kernel in
+ * the stream has finished if that kernel allows it, so codes and scales must
+ * not be written by a kernel that triggers dependent launch early.
+ * Numerics: M = 1: FP32 table entries, scale products and sums. Otherwise
+ * the rotated activation feeds FP16 tensor-core products with FP32
  * accumulation (one power-of-two exponent per 128 activations keeps it in
- * range); y satisfies |y - y_exact| <= 2e-3 * sum_k |w x'| + 1e-5.
+ * range). Either way y satisfies |y - y_exact| <= 2e-3 * sum_k |w x'| + 1e-5,
+ * and repeated calls give bit-identical results.
  * Source: fused unpack and group scale inside the matrix product, release
  * summary, section 三值权重怎么压缩到 1.76 bit.
  */
