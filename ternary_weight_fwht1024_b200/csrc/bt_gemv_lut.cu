@@ -20,8 +20,8 @@
 // set's code bytes ([16 rows][112 B], x rounded down to 16 B so base-3 chunks
 // at 8-byte offsets stay legal) and scales ([16 rows][8 halves]) with two TMA
 // tensor copies into a two-slot ring, completing on the slot's mbarrier. The
-// first sets are requested before the dependency wait, so the rotation and
-// the table build run under their latency.
+// first sets are requested right after the activation loads, so the rotation
+// and the table build run under their latency.
 //
 // Tables. Lane L of a warp reads code word L (bytes 4L..4L+3) of a row chunk,
 // so byte position p = 4L + k is only ever looked up by lane L: its table
@@ -351,8 +351,6 @@ gemv_lut_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant_
     uint32_t issued = 0, done = 0;  // sets requested / consumed by this warp
     bool ok = true;
 
-    // Request the first sets of the first chunk before the dependency wait:
-    // weights are not written by the kernels this launch may overlap.
     auto box_x = [&](int c, int& cx, int& sx, int& coff, int& soff) {
         const int cb = c * CB;
         cx = cb & ~15;
@@ -360,21 +358,12 @@ gemv_lut_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant_
         sx = (4 * c) & ~7;
         soff = 2 * (4 * c - sx);
     };
-    {
-        int cx, sx, coff, soff;
-        box_x(chunk, cx, sx, coff, soff);
-        if (L == 0 && chunk < a.nchunk)
-            for (int d = 0; d < kLutDepth && d < nsets; ++d)
-                lut_issue_set(rg, &cmap, &smap, issued + d, cx, sx, w_lo + (int64_t)d * kLutSet);
-        if (chunk < a.nchunk) issued += min(kLutDepth, nsets);
-    }
     lut_zero_invalid<LAYOUT>(table);
     pdl_wait();
     pdl_launch_dependents();
 
     uint32_t bad = 0;
     int cur_blk = -1;
-    bool first = true;
     for (; chunk < a.nchunk; chunk += cstep) {
         int cx, sx, coff, soff;
         box_x(chunk, cx, sx, coff, soff);
@@ -385,11 +374,14 @@ gemv_lut_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant_
         XFetch xf;
         if (new_blk && warp == 0) lut_fetch_block(a, blk, xf);
         __syncthreads();  // previous chunk's lookups are done with table / xs
-        if (!first && L == 0 && ok)
+        // The first sets of this chunk's rows go out after warp 0 has issued
+        // its activation loads, so those loads do not queue behind the
+        // weight stream; the rotation and the table build run under the
+        // copies' latency.
+        if (L == 0 && ok)
             for (int d = 0; d < kLutDepth && d < nsets; ++d)
                 lut_issue_set(rg, &cmap, &smap, issued + d, cx, sx, w_lo + (int64_t)d * kLutSet);
-        if (!first && ok) issued += min(kLutDepth, nsets);
-        first = false;
+        if (ok) issued += min(kLutDepth, nsets);
         if (new_blk) {
             if (warp == 0) lut_rotate_block(a, blk, xf, xr, reinterpret_cast<float*>(lut_smem + kLutTileOffset));
             cur_blk = blk;
@@ -573,14 +565,14 @@ cudaError_t launch_gemv_lut(int layout, const uint8_t* codes, const uint16_t* sc
     ra.nchunk = la.nchunk;
     ra.y_bf16 = y_dtype == BT_BF16;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)((N + 31) / 32));
-    cfg.blockDim = dim3(256);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
+    cfg.gridDim = dim3((unsigned)((N + 31) / 32));
+    cfg.blockDim = dim3(256);
     return cudaLaunchKernelEx(&cfg, gemv_lut_reduce_kernel, ra);
 }
 
