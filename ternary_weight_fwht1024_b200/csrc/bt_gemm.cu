@@ -577,7 +577,12 @@ static int pick_bn(int64_t M, int64_t N, int num_sms) {
 #ifdef BT_GEMM_BN_FORCE
     if (N % BT_GEMM_BN_FORCE == 0) return BT_GEMM_BN_FORCE;
 #endif
-    const int cands[2] = {160, 128};
+#ifdef BT_GEMM_NO_BN256
+    const int cands[] = {160, 128};
+#else
+    // on equal wave efficiency the wider tile wins: fewer operand bytes per FLOP
+    const int cands[] = {256, 160, 128};
+#endif
     int best = 128;
     double best_eff = -1.0;
     for (int bn : cands) {
@@ -611,6 +616,8 @@ static cudaError_t launch_gemm_t(const CUtensorMap& amap, const GemmArgs& ga, cu
 
 template <int LAYOUT>
 static cudaError_t dispatch_gemm(int bn, const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t s) {
+    // BN = 256: two weight stages (64 KB each) fit beside the activation ring
+    if (bn == 256) return launch_gemm_t<LAYOUT, 256, 2>(amap, ga, s);
     return bn == 160 ? launch_gemm_t<LAYOUT, 160, BT_GEMM_BSTAGES>(amap, ga, s)
                      : launch_gemm_t<LAYOUT, 128, BT_GEMM_BSTAGES>(amap, ga, s);
 }
