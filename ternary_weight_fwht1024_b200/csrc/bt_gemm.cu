@@ -55,8 +55,12 @@ constexpr int kGemmBK = 128;             // one weight group per stage
 constexpr int kGemmTpr = BT_GEMM_TPR;
 __host__ __device__ constexpr int gemm_dec_warps(int bn) { return bn * kGemmTpr / 32; }
 __host__ __device__ constexpr int gemm_threads(int bn) { return (2 + gemm_dec_warps(bn)) * 32; }
-constexpr int kGemmLutCopies = 8;
-constexpr int kGemmLutBytes = 256 * kGemmLutCopies * 8;  // 8 copies x (low, high) x 4 bytes per code
+// Base-3 decode table: per code, one 32-bit word per lane (each lane reads
+// only its own bank, so lookups never conflict) holding the code's five
+// base-3 digits as 2-bit fields plus the FP16 exponent bits of 1024 (0x6400)
+// in both halves; bit 31 marks codes 243-255.
+constexpr int kGemmLutRow = 32 * 4;                       // bytes per code
+constexpr int kGemmLutBytes = 256 * kGemmLutRow;
 
 // ---------------------------------------------------------------- helpers ----
 
@@ -159,22 +163,22 @@ __device__ __forceinline__ void gemm_decode_part(const uint32_t (&cw)[GemmPart<L
                                                  uint32_t ha34, uint32_t& err) {
     constexpr int WPT = GemmPart<LAYOUT>::WPT, NW = GemmPart<LAYOUT>::NW;
     constexpr int W0 = WPT * QQ, W1 = W0 + WPT, P0 = W0 / 5;
-    constexpr uint32_t kRow = 8 * kGemmLutCopies;
     if constexpr (LAYOUT == BT_LAYOUT_B3) {
 #pragma unroll
         for (int j = 0; j < NW; ++j) {
             const int p = P0 + j;
             if (p > 12) continue;
             const uint32_t pr = cw[j];
-            const uint32_t va = *reinterpret_cast<const uint32_t*>(lut_lane + (pr & 0xFFu) * kRow);
-            const uint32_t vb = *reinterpret_cast<const uint32_t*>(lut_lane + (pr >> 8) * kRow + kRow / 2);
+            const uint32_t va = *reinterpret_cast<const uint32_t*>(lut_lane + (pr & 0xFFu) * kGemmLutRow);
+            const uint32_t vb = *reinterpret_cast<const uint32_t*>(lut_lane + (pr >> 8) * kGemmLutRow);
             err |= (va | vb) & 0x80000000u;
+            const uint32_t x = prmt(va, vb, 0x7610u);   // byte 2p's fields low, byte 2p+1's high
             const int nw = p < 12 ? 5 : 3;
 #pragma unroll
             for (int i = 0; i < nw; ++i) {
                 const int w = 5 * p + i;
                 if (w >= W0 && w < W1) {
-                    const uint32_t f = lop3_or_and(va, vb, gfmask(i) | 0x64006400u);
+                    const uint32_t f = x & (gfmask(i) | 0x64006400u);
                     words[w - W0] = hmul2_u32(hfma2_u32(f, hm[i], ha[i]), s2);
                 }
             }
@@ -348,20 +352,17 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (LAYOUT == BT_LAYOUT_B3) {
-        // digits of each code as 2-bit fields, 8 copies per code (low table,
-        // then high table with the fields in the upper half)
-        for (int idx = threadIdx.x; idx < 256 * 2 * kGemmLutCopies; idx += blockDim.x) {
-            const int code = idx / (2 * kGemmLutCopies), hi = (idx / kGemmLutCopies) & 1;
-            // fields plus the FP16 exponent bits of 1024 (0x6400) in the same
-            // half, so one LOP3 yields 1024 + d 4^i
-            uint32_t f = 0x80000000u | 0x6400u;
+        // digits of each code as 2-bit fields with the FP16 exponent bits of
+        // 1024 (0x6400), in both halves, so that field i masked out of a half
+        // reads 1024 + d 4^i; one word per lane
+        for (int idx = threadIdx.x; idx < 256 * 32; idx += blockDim.x) {
+            const int code = idx >> 5;
+            uint32_t f = 0x6400u;
             if (code < 243) {
-                f = 0x6400u;
                 int r = code;
                 for (int i = 0; i < 5; ++i) { f |= static_cast<uint32_t>(r % 3) << (2 * i); r /= 3; }
             }
-            if (hi) f = (f & 0xFFFFu) << 16 | (f & 0x80000000u);
-            reinterpret_cast<uint32_t*>(lut)[idx] = f;
+            reinterpret_cast<uint32_t*>(lut)[idx] = f | (f << 16) | (code < 243 ? 0u : 0x80000000u);
         }
     }
     if (warp == 1) {
@@ -427,7 +428,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
         const int n = n0 + t;
         const uint8_t* rowp = a.codes + (int64_t)n * a.row_bytes;
         const uint16_t* srow = a.scales + (int64_t)n * a.G;
-        const uint8_t* lut_lane = lut + (lane & (kGemmLutCopies - 1)) * 4;   // this lane's copy of the table
+        const uint8_t* lut_lane = lut + lane * 4;       // this lane's column (bank) of the table
         uint32_t hm[6], ha[6];
 #pragma unroll
         for (int i = 0; i < 6; ++i) { hm[i] = h2_mul_of(i); ha[i] = h2_add_of(i); }
