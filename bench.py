@@ -396,7 +396,7 @@ def run_gpu(args, rank, world):
                      "frac": round(achieved / peaks["hbm_gbs"], 4),
                      # dram__bytes_read.sum + dram__bytes_write.sum of gemv_lut_kernel, mean over the
                      # three layers' launches (profiles/gemv_lut_kernel_b3_triple.md)
-                     "traffic": None,
+                     "traffic": 14961664,
                      "algorithmic_bytes_per_launch": int(sum(dom_bytes) / len(dom_bytes)),
                      "kernel": "bt_gemv call (table-lookup GEMV kernel + chunk reduction), weighted over the three layers",
                      "peak_kind": f"HBM copy, {peaks['src']}"},
