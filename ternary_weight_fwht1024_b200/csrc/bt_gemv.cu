@@ -1243,9 +1243,9 @@ static cudaError_t launch_gemv_tma_t(const CUtensorMap& cmap, const CUtensorMap&
 template <int LAYOUT, bool CHECK>
 static cudaError_t dispatch_gemv_tma_c(const CUtensorMap& cmap, const CUtensorMap& smap, const GemvTmaArgs& ta,
                                        const TmaPlan& tp, cudaStream_t s) {
-    if (tp.bsmem)
-        return ta.M == 1 ? launch_gemv_tma_t<LAYOUT, true, true, CHECK>(cmap, smap, ta, tp, s)
-                         : launch_gemv_tma_t<LAYOUT, true, false, CHECK>(cmap, smap, ta, tp, s);
+    // (single-row calls that qualify for this kernel take the table-lookup
+    // kernel instead, so the M = 1 specialisation is not instantiated here)
+    if (tp.bsmem) return launch_gemv_tma_t<LAYOUT, true, false, CHECK>(cmap, smap, ta, tp, s);
     return launch_gemv_tma_t<LAYOUT, false, false, CHECK>(cmap, smap, ta, tp, s);
 }
 
