@@ -96,17 +96,15 @@ __device__ __forceinline__ uint2 lds_u64(uint32_t addr) {
     return v;
 }
 
-// Table lookup at a shared-window byte address. Volatile so the compiler keeps
-// the row loads of the next rows (also volatile) ahead of these lookups.
+// Table lookup at a shared-window byte address. The ring reads above carry a
+// memory clobber (they must stay after the mbarrier wait that publishes the
+// TMA bytes); the table is written before a CTA barrier, so lookups need none.
 __device__ __forceinline__ float lds_f32(uint32_t addr) {
     float v;
     asm volatile("ld.shared.f32 %0, [%1];" : "=f"(v) : "r"(addr));
     return v;
 }
 
-// Raw words of one lane's 32 bf16 activations of a 1024-block and of its 32
-// sign bytes. Fetched before the row loads so that the rotation does not
-// queue behind them. (FP32 activations are read when the block is rotated.)
 struct LutReduceArgs {
     const float* partials;
     void* y;
@@ -115,6 +113,10 @@ struct LutReduceArgs {
     int y_bf16;
 };
 
+// Raw words of one lane's 32 bf16 activations of a 1024-block and of its 32
+// sign bytes. Fetched before the first weight copies are requested, so that
+// the rotation does not queue behind them. (FP32 activations are read when
+// the block is rotated.)
 struct XFetch {
     uint4 q[4];
     uint4 sg[2];
