@@ -370,7 +370,7 @@ def run_gpu(args, rank, world):
         "higher_is_better": True,
         "scaling": "weak",
         "vs_baseline": None,
-        "dtype": "f16 tensor-core products of base-3 trits, f32 accumulate",
+        "dtype": "f32",  # M = 1: FP32 table entries (partial dot products), FP32 scale products and sums
         "data": "synthetic (seeded trits P(0)=0.4, g128 fp16 scales, bf16 activations with 0.1% x20 outliers)",
         "config": {"workload": "decode GEMV M=1 on the 5120x5120 / 5120x17408 / 17408x5120 triple, base-3 g128, "
                                "FWHT-1024 fused",
