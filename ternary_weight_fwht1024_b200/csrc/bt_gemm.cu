@@ -131,6 +131,58 @@ __device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
     return r;
 }
 
+// ---- CTA pair (cta_group::2) helpers
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+// all threads of both CTAs; hardware barrier (the pair is co-scheduled)
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+// TMA load into this CTA's shared memory whose bytes complete on the pair
+// leader's barrier (the peer bit of the barrier address cleared)
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map, int x, int y, uint32_t bar) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];"
+        :: "r"(dst), "l"(map), "r"(x), "r"(y), "r"(bar & 0xFEFFFFFFu) : "memory");
+}
+__device__ __forceinline__ void tc_mma_pair(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+        :: "r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
+}
+// arrive once on the barrier at this offset in both CTAs of the pair when the
+// pair's MMAs issued so far complete
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+    asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
+                 :: "r"(bar), "h"((uint16_t)3) : "memory");
+}
+// arrive on the barrier at this offset in CTA `rank` of the cluster
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar, uint32_t rank) {
+    asm volatile(
+        "{\n\t.reg .b32 ra;\n\t"
+        "mapa.shared::cluster.u32 ra, %0, %1;\n\t"
+        "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}"
+        :: "r"(bar), "r"(rank) : "memory");
+}
+// bounded wait with cluster-scope acquire (arrivals may come from the peer)
+__device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity) {
+    for (uint32_t it = 0; it < kSpinLimit; ++it) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+        if (ok) return true;
+    }
+    return false;
+}
+
 __host__ __device__ constexpr uint32_t gfmask(int i) { return (3u << (2 * i)) | (3u << (2 * i + 16)); }
 
 // FP16 constants turning (1024 + d 4^i) into d - 1: multiply by 4^-i, add
@@ -302,11 +354,10 @@ struct GemmArgs {
 #define BT_GEMM_BSTAGES 3
 #endif
 
-template <int LAYOUT, int BN, int STAGES>
+template <int LAYOUT, int BN, int STAGES, int ASTAGES = BT_GEMM_ASTAGES>
 struct GemmSmem {
-    // activation ring (TMA) is deeper than the weight ring (decoded in the
-    // CTA): activation tiles come from L2/HBM and need the longer lead
-    static constexpr int kAStages = BT_GEMM_ASTAGES;
+    // activation ring (TMA) and ring of decoded weight tiles (BN rows each)
+    static constexpr int kAStages = ASTAGES;
     static constexpr int kBStages = STAGES;
     static constexpr int kA = kGemmBM * kGemmBK * 2;   // 32 KB: two 64-column panels
     static constexpr int kB = BN * kGemmBK * 2;
@@ -315,10 +366,18 @@ struct GemmSmem {
     static constexpr int kTotal = kAStages * kA + kBStages * kB + kLut + kBars + 1024;  // + alignment slack
 };
 
-template <int LAYOUT, int BN, int STAGES>
-__global__ void __launch_bounds__(gemm_threads(BN), 1)
+// PAIR: the two CTAs of a cluster (M tiles 2j, 2j + 1) share one BN-column
+// weight tile. Each decodes half of its rows (BL = BN / 2) into its own
+// shared memory; the leader (rank 0) issues tcgen05.mma.cta_group::2 with
+// M = 256, which reads A and B from both CTAs and accumulates each CTA's 128
+// rows x BN columns in that CTA's TMEM. Activation copies complete on the
+// leader's barrier, the peer's decoders arrive on it remotely, and each
+// commit arrives on the barrier pair in both CTAs.
+template <int LAYOUT, int BN, int STAGES, int ASTAGES = BT_GEMM_ASTAGES, bool PAIR = false>
+__global__ void __launch_bounds__(gemm_threads(PAIR ? BN / 2 : BN), 1)
 gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
-    using SM = GemmSmem<LAYOUT, BN, STAGES>;
+    constexpr int BL = PAIR ? BN / 2 : BN;             // weight rows decoded by this CTA
+    using SM = GemmSmem<LAYOUT, BL, STAGES, ASTAGES>;
     extern __shared__ uint8_t gsm_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~uintptr_t(1023));
     constexpr int SA = SM::kAStages, SB = SM::kBStages;
@@ -335,8 +394,12 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int m0 = blockIdx.y * kGemmBM, n0 = blockIdx.x * BN;
+    // a CTA pair sits along x, so that its two CTAs take the two halves of a
+    // 256-row activation tile against the same weight tile
+    const int m0 = (PAIR ? blockIdx.x : blockIdx.y) * kGemmBM, n0 = (PAIR ? blockIdx.y : blockIdx.x) * BN;
     const int ktiles = a.G;
+    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    const bool leader = rank == 0;
 
     if (threadIdx.x == 0) {
         for (int s = 0; s < SA; ++s) {
@@ -344,7 +407,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
             mbar_init(smem_addr(emptyA + s), 1);
         }
         for (int s = 0; s < SB; ++s) {
-            mbar_init(smem_addr(fullB + s), gemm_dec_warps(BN));
+            mbar_init(smem_addr(fullB + s), (PAIR ? 2 : 1) * gemm_dec_warps(BL));
             mbar_init(smem_addr(emptyB + s), 1);
         }
         mbar_init(smem_addr(accf), 1);
@@ -366,11 +429,18 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
         }
     }
     if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     :: "r"(smem_addr(tmem_slot)), "r"(BN <= 128 ? 128 : 256) : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        if constexpr (PAIR) {
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
+                         :: "r"(smem_addr(tmem_slot)), "r"(BN <= 128 ? 128 : 256) : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                         :: "r"(smem_addr(tmem_slot)), "r"(BN <= 128 ? 128 : 256) : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
     }
     __syncthreads();
+    if constexpr (PAIR) cluster_sync_all();   // both CTAs' barriers exist before any remote arrival
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     pdl_wait();  // the activations come from the prep kernel
@@ -386,19 +456,27 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
                 }
                 if (*abort_flag) break;
                 const uint32_t dst = smem_addr(a_ring + s * SM::kA);
-                mbar_arrive_tx(smem_addr(fullA + s), SM::kA);
-                tma_load_2d(dst, &amap, kt * kGemmBK, m0, smem_addr(fullA + s));
-                tma_load_2d(dst + SM::kA / 2, &amap, kt * kGemmBK + 64, m0, smem_addr(fullA + s));
+                if constexpr (PAIR) {
+                    // the leader's barrier counts both CTAs' activation bytes
+                    if (leader) mbar_arrive_tx(smem_addr(fullA + s), 2 * SM::kA);
+                    tma_load_2d_pair(dst, &amap, kt * kGemmBK, m0, smem_addr(fullA + s));
+                    tma_load_2d_pair(dst + SM::kA / 2, &amap, kt * kGemmBK + 64, m0, smem_addr(fullA + s));
+                } else {
+                    mbar_arrive_tx(smem_addr(fullA + s), SM::kA);
+                    tma_load_2d(dst, &amap, kt * kGemmBK, m0, smem_addr(fullA + s));
+                    tma_load_2d(dst + SM::kA / 2, &amap, kt * kGemmBK + 64, m0, smem_addr(fullA + s));
+                }
             }
         }
     } else if (warp == 1) {
-        // ---------------- MMA issuer
-        if (lane == 0) {
-            constexpr uint32_t idesc = idesc_f16(kGemmBM, BN);
+        // ---------------- MMA issuer (the leader, for a pair)
+        if (lane == 0 && leader) {
+            constexpr uint32_t idesc = idesc_f16(PAIR ? 2 * kGemmBM : kGemmBM, BN);
             for (int kt = 0; kt < ktiles; ++kt) {
                 const int s_a = kt % SA, s_b = kt % SB;
-                if (!mbar_wait(smem_addr(fullA + s_a), (kt / SA) & 1) ||
-                    !mbar_wait(smem_addr(fullB + s_b), (kt / SB) & 1)) {
+                const bool okb = PAIR ? mbar_wait_cluster(smem_addr(fullB + s_b), (kt / SB) & 1)
+                                      : mbar_wait(smem_addr(fullB + s_b), (kt / SB) & 1);
+                if (!mbar_wait(smem_addr(fullA + s_a), (kt / SA) & 1) || !okb) {
                     bad = BT_DEVERR_TIMEOUT; *abort_flag = 1; break;
                 }
                 if (*abort_flag) break;
@@ -409,12 +487,21 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
                 for (int k = 0; k < kGemmBK / 16; ++k) {
                     const uint32_t pa = sa + (k >> 2) * (SM::kA / 2) + (k & 3) * 32;
                     const uint32_t pb = sb + (k >> 2) * (SM::kB / 2) + (k & 3) * 32;
-                    tc_mma(tmem, smem_desc_sw128(pa), smem_desc_sw128(pb), idesc, (kt > 0 || k > 0) ? 1u : 0u);
+                    if constexpr (PAIR)
+                        tc_mma_pair(tmem, smem_desc_sw128(pa), smem_desc_sw128(pb), idesc, (kt > 0 || k > 0) ? 1u : 0u);
+                    else
+                        tc_mma(tmem, smem_desc_sw128(pa), smem_desc_sw128(pb), idesc, (kt > 0 || k > 0) ? 1u : 0u);
                 }
-                tc_commit(smem_addr(emptyA + s_a));
-                tc_commit(smem_addr(emptyB + s_b));
+                if constexpr (PAIR) {
+                    tc_commit_pair(smem_addr(emptyA + s_a));
+                    tc_commit_pair(smem_addr(emptyB + s_b));
+                } else {
+                    tc_commit(smem_addr(emptyA + s_a));
+                    tc_commit(smem_addr(emptyB + s_b));
+                }
             }
-            tc_commit(smem_addr(accf));
+            if constexpr (PAIR) tc_commit_pair(smem_addr(accf));
+            else tc_commit(smem_addr(accf));
         }
     } else {
         // ---------------- decoders: thread (part qq, row t) decodes the 128 /
@@ -422,10 +509,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
         // in panel h (64-slot halves of the group)
         constexpr int TPR = kGemmTpr;
         constexpr int WPT = GemmPart<LAYOUT>::WPT;      // 32-bit words per thread
-        const int tt = threadIdx.x - 64;                // 0 .. TPR BN - 1
-        const int qq = tt / BN, t = tt - qq * BN;
+        const int tt = threadIdx.x - 64;                // 0 .. TPR BL - 1
+        const int qq = tt / BL, t = tt - qq * BL;
         const int h = qq * WPT / 32;                    // panel
-        const int n = n0 + t;
+        const int n = n0 + (int)rank * BL + t;
         const uint8_t* rowp = a.codes + (int64_t)n * a.row_bytes;
         const uint16_t* srow = a.scales + (int64_t)n * a.G;
         const uint8_t* lut_lane = lut + lane * 4;       // this lane's column (bank) of the table
@@ -515,7 +602,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
             }
             fence_proxy_async_smem();
             __syncwarp();
-            if (lane == 0) mbar_arrive(smem_addr(fullB + s));
+            if (lane == 0) {
+                if constexpr (PAIR) mbar_arrive_cluster(smem_addr(fullB + s), 0u);   // the leader's barrier
+                else mbar_arrive(smem_addr(fullB + s));
+            }
             return true;
         };
         uint32_t bufA[NW], bufB[NW], sA = 0, sB = 0;
@@ -560,9 +650,15 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
     if (lane == 0) report(a.dev_err, bad);
     tc_fence_before();
     __syncthreads();
-    if (warp == 1) {
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
-                     :: "r"(tmem), "r"(BN <= 128 ? 128 : 256) : "memory");
+    if constexpr (PAIR) {
+        cluster_sync_all();   // both CTAs are done with the pair's TMEM and barriers
+        if (warp == 1)
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;"
+                         :: "r"(tmem), "r"(BN <= 128 ? 128 : 256) : "memory");
+    } else {
+        if (warp == 1)
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
+                         :: "r"(tmem), "r"(BN <= 128 ? 128 : 256) : "memory");
     }
 }
 
@@ -615,8 +711,46 @@ static cudaError_t launch_gemm_t(const CUtensorMap& amap, const GemmArgs& ga, cu
     return cudaLaunchKernelEx(&cfg, kern, amap, ga);
 }
 
+// CTA-pair launch: clusters of two CTAs along M (M % 256 == 0). Each CTA
+// decodes BN / 2 weight rows, so the rings hold 3 activation stages and 3-4
+// weight stages. The pair has to lie along the grid's x axis: a kernel that
+// uses cta_group::2 launched with clusters of (1, 2, 1) is refused with
+// cudaErrorInvalidClusterSize. Compiled in with -DBT_GEMM_PAIR only: on B200
+// at M = 512 it gives the same bits as the single-CTA kernel but runs slower
+// (about 404 against 503 TFLOP/s over the three prefill layers).
+template <int LAYOUT, int BN, int SB, int SA>
+static cudaError_t launch_gemm_pair_t(const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t stream) {
+    using SM = GemmSmem<LAYOUT, BN / 2, SB, SA>;
+    static_assert(SM::kTotal <= 227 * 1024, "shared memory");
+    auto kern = gemm_kernel<LAYOUT, BN, SB, SA, true>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kTotal);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(ga.M / kGemmBM, ga.N / BN);
+    cfg.blockDim = dim3(gemm_threads(BN / 2));
+    cfg.dynamicSmemBytes = SM::kTotal;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = 2;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kern, amap, ga);
+}
+
 template <int LAYOUT>
 static cudaError_t dispatch_gemm(int bn, const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t s) {
+#ifdef BT_GEMM_PAIR
+    if (ga.M % (2 * kGemmBM) == 0) {
+        if (bn == 256) return launch_gemm_pair_t<LAYOUT, 256, 3, 3>(amap, ga, s);
+        if (bn == 160) return launch_gemm_pair_t<LAYOUT, 160, 4, 3>(amap, ga, s);
+        return launch_gemm_pair_t<LAYOUT, 128, 4, 3>(amap, ga, s);
+    }
+#endif
     // BN = 256: two weight stages (64 KB each) fit beside the activation ring
     if (bn == 256) return launch_gemm_t<LAYOUT, 256, 2>(amap, ga, s);
     return bn == 160 ? launch_gemm_t<LAYOUT, 160, BT_GEMM_BSTAGES>(amap, ga, s)
