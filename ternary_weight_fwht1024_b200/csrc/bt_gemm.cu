@@ -39,6 +39,11 @@
 //     in the same order, so the contraction over each group is unchanged.
 //     Decoding a word: OR the two digits' 2-bit fields into FP16 1024 + d 4^i
 //     (exact), one HFMA2 makes it d - 1 = t (exact), one HMUL2 makes s t.
+//
+//     With M % 256 == 0 the tiles run as CTA pairs (clusters of two along
+//     M): both CTAs decode half of a BN-row weight tile each, and the pair
+//     leader issues tcgen05.mma.cta_group::2 (M 256) over both CTAs' shared
+//     memory, so each decoded weight row serves 256 activation rows.
 // Waits on barriers are bounded: a wait that runs out sets BT_DEVERR_TIMEOUT,
 // the CTA skips the rest of its work and still releases its TMEM.
 #include "bt_internal.cuh"
@@ -371,8 +376,9 @@ struct GemmSmem {
 // shared memory; the leader (rank 0) issues tcgen05.mma.cta_group::2 with
 // M = 256, which reads A and B from both CTAs and accumulates each CTA's 128
 // rows x BN columns in that CTA's TMEM. Activation copies complete on the
-// leader's barrier, the peer's decoders arrive on it remotely, and each
-// commit arrives on the barrier pair in both CTAs.
+// leader's barrier; the peer's decoders arrive on their own barrier, which
+// one relay thread forwards to the leader's; each commit arrives on the
+// barrier pair in both CTAs.
 template <int LAYOUT, int BN, int STAGES, int ASTAGES = BT_GEMM_ASTAGES, bool PAIR = false>
 __global__ void __launch_bounds__(gemm_threads(PAIR ? BN / 2 : BN), 1)
 gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
@@ -407,7 +413,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
             mbar_init(smem_addr(emptyA + s), 1);
         }
         for (int s = 0; s < SB; ++s) {
-            mbar_init(smem_addr(fullB + s), (PAIR ? 2 : 1) * gemm_dec_warps(BL));
+            // a pair leader also counts the one arrival relayed from the peer
+            mbar_init(smem_addr(fullB + s), gemm_dec_warps(BL) + (PAIR && leader ? 1 : 0));
             mbar_init(smem_addr(emptyB + s), 1);
         }
         mbar_init(smem_addr(accf), 1);
@@ -502,6 +509,22 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
             }
             if constexpr (PAIR) tc_commit_pair(smem_addr(accf));
             else tc_commit(smem_addr(accf));
+        }
+        if constexpr (PAIR) {
+            // Relay (the peer's warp 1): once this CTA's decoders have filled
+            // weight stage kt, one cluster-scope arrival tells the leader. The
+            // decoders themselves arrive locally: a cluster-scope release in
+            // their own code would wait for the code loads they keep in flight.
+            if (lane == 0 && !leader) {
+                for (int kt = 0; kt < ktiles; ++kt) {
+                    const int s_b = kt % SB;
+                    if (!mbar_wait(smem_addr(fullB + s_b), (kt / SB) & 1)) {
+                        bad = BT_DEVERR_TIMEOUT; *abort_flag = 1; break;
+                    }
+                    if (*abort_flag) break;
+                    mbar_arrive_cluster(smem_addr(fullB + s_b), 0u);
+                }
+            }
         }
     } else {
         // ---------------- decoders: thread (part qq, row t) decodes the 128 /
@@ -603,8 +626,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
             fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) {
-                if constexpr (PAIR) mbar_arrive_cluster(smem_addr(fullB + s), 0u);   // the leader's barrier
-                else mbar_arrive(smem_addr(fullB + s));
+                mbar_arrive(smem_addr(fullB + s));
             }
             return true;
         };
@@ -715,9 +737,9 @@ static cudaError_t launch_gemm_t(const CUtensorMap& amap, const GemmArgs& ga, cu
 // decodes BN / 2 weight rows, so the rings hold 3 activation stages and 3-4
 // weight stages. The pair has to lie along the grid's x axis: a kernel that
 // uses cta_group::2 launched with clusters of (1, 2, 1) is refused with
-// cudaErrorInvalidClusterSize. Compiled in with -DBT_GEMM_PAIR only: on B200
-// at M = 512 it gives the same bits as the single-CTA kernel but runs slower
-// (about 404 against 503 TFLOP/s over the three prefill layers).
+// cudaErrorInvalidClusterSize. On B200 at M = 512 the pair gives the same bits
+// as the single-CTA kernel at about 540 against 501 TFLOP/s over the three
+// prefill layers (-DBT_GEMM_NO_PAIR builds without it).
 template <int LAYOUT, int BN, int SB, int SA>
 static cudaError_t launch_gemm_pair_t(const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t stream) {
     using SM = GemmSmem<LAYOUT, BN / 2, SB, SA>;
@@ -744,7 +766,7 @@ static cudaError_t launch_gemm_pair_t(const CUtensorMap& amap, const GemmArgs& g
 
 template <int LAYOUT>
 static cudaError_t dispatch_gemm(int bn, const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t s) {
-#ifdef BT_GEMM_PAIR
+#ifndef BT_GEMM_NO_PAIR
     if (ga.M % (2 * kGemmBM) == 0) {
         if (bn == 256) return launch_gemm_pair_t<LAYOUT, 256, 3, 3>(amap, ga, s);
         if (bn == 160) return launch_gemm_pair_t<LAYOUT, 160, 4, 3>(amap, ga, s);
