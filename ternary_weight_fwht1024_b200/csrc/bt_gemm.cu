@@ -740,6 +740,19 @@ static cudaError_t launch_gemm_t(const CUtensorMap& amap, const GemmArgs& ga, cu
 // cudaErrorInvalidClusterSize. On B200 at M = 512 the pair gives the same bits
 // as the single-CTA kernel at about 540 against 501 TFLOP/s over the three
 // prefill layers (-DBT_GEMM_NO_PAIR builds without it).
+// ring depths (weight, activation stages) of the pair kernel per tile width
+#ifndef BT_GEMM_PAIR_SB160
+#define BT_GEMM_PAIR_SB160 4
+#endif
+#ifndef BT_GEMM_PAIR_SA160
+#define BT_GEMM_PAIR_SA160 3
+#endif
+#ifndef BT_GEMM_PAIR_SB256
+#define BT_GEMM_PAIR_SB256 3
+#endif
+#ifndef BT_GEMM_PAIR_SA256
+#define BT_GEMM_PAIR_SA256 3
+#endif
 template <int LAYOUT, int BN, int SB, int SA>
 static cudaError_t launch_gemm_pair_t(const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t stream) {
     using SM = GemmSmem<LAYOUT, BN / 2, SB, SA>;
@@ -768,8 +781,8 @@ template <int LAYOUT>
 static cudaError_t dispatch_gemm(int bn, const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t s) {
 #ifndef BT_GEMM_NO_PAIR
     if (ga.M % (2 * kGemmBM) == 0) {
-        if (bn == 256) return launch_gemm_pair_t<LAYOUT, 256, 3, 3>(amap, ga, s);
-        if (bn == 160) return launch_gemm_pair_t<LAYOUT, 160, 4, 3>(amap, ga, s);
+        if (bn == 256) return launch_gemm_pair_t<LAYOUT, 256, BT_GEMM_PAIR_SB256, BT_GEMM_PAIR_SA256>(amap, ga, s);
+        if (bn == 160) return launch_gemm_pair_t<LAYOUT, 160, BT_GEMM_PAIR_SB160, BT_GEMM_PAIR_SA160>(amap, ga, s);
         return launch_gemm_pair_t<LAYOUT, 128, 4, 3>(amap, ga, s);
     }
 #endif
