@@ -15,8 +15,9 @@
 //     2^e_m.
 //
 //  2. gemm: one 128 x BN output tile per CTA, one 128-wide K group per
-//     pipeline stage; a 4-stage ring of activation tiles (TMA) and a
-//     2-stage ring of decoded weight tiles.
+//     pipeline stage; a 2-stage ring of activation tiles (TMA) and a
+//     3-stage ring of decoded weight tiles (2 at BN = 256; the CTA-pair
+//     form below holds 3 and 3-4).
 //       warp 0      TMA: the activation tile (two 64-column panels, 128-byte
 //                   swizzle) into shared memory;
 //       warp 1      allocates TMEM, one elected thread issues
