@@ -189,6 +189,14 @@ bt_status bt_gemv_noalloc(int layout, const uint8_t* codes, const uint16_t* scal
  *  Arguments as for bt_gemv (y is bf16). The rotated activation is rounded
  *  to FP16 after scaling each row by a power of two chosen from its largest
  *  magnitude.
+ * Kernels: a prep kernel (rotation, row scaling, FP16 in the decoder's K
+ *  order), then the tensor-core kernel, chained by programmatic dependent
+ *  launch. With M % 256 == 0 the output tiles run as clusters of two CTAs
+ *  that share each decoded weight tile (tcgen05 cta_group::2, M = 256 per
+ *  instruction); otherwise one CTA per 128-row tile. Both forms add the same
+ *  products in the same order per output, and repeated calls give
+ *  bit-identical results. Waits are bounded: one that runs out sets
+ *  BT_DEVERR_TIMEOUT and the affected outputs are unspecified.
  * Source: pp512 prompt processing, release summary, section 实测吞吐.
  */
 size_t bt_gemm_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K);
