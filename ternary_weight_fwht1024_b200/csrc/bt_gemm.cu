@@ -26,7 +26,7 @@
 //                   each stage to its "empty" barrier;
 //       warps 2..   decode the packed weights of the stage to FP16 s*t --
 //                   exact -- and store them in the tensor cores' K-major
-//                   128-byte-swizzled layout: BT_GEMM_TPR (2) threads per
+//                   128-byte-swizzled layout: BT_GEMM_TPR (4) threads per
 //                   weight row, each one 128 / TPR-slot part of the group
 //                   (BN TPR / 32 warps); then warps 2-5
 //                   read the accumulator back (tcgen05.ld) and write bf16 Y
@@ -56,7 +56,7 @@ constexpr int kGemmBK = 128;             // one weight group per stage
 // decoder warps: TPR threads per weight row of the BN-row tile, each decoding
 // 128 / TPR of a group's slots
 #ifndef BT_GEMM_TPR
-#define BT_GEMM_TPR 2
+#define BT_GEMM_TPR 4
 #endif
 constexpr int kGemmTpr = BT_GEMM_TPR;
 __host__ __device__ constexpr int gemm_dec_warps(int bn) { return bn * kGemmTpr / 32; }
@@ -693,10 +693,19 @@ size_t gemm_workspace_bytes(int, int64_t M, int64_t, int64_t K, int) {
     return gemm_align((size_t)M * K * 2, 256) + gemm_align((size_t)M * 4, 256);
 }
 
+static bool gemm_pairs(int64_t M) {
+#ifdef BT_GEMM_NO_PAIR
+    return false;
+#else
+    return M % (2 * kGemmBM) == 0;
+#endif
+}
+
 static int pick_bn(int64_t M, int64_t N, int num_sms) {
 #ifdef BT_GEMM_BN_FORCE
     if (N % BT_GEMM_BN_FORCE == 0) return BT_GEMM_BN_FORCE;
 #endif
+    const bool pair = gemm_pairs(M);
 #ifdef BT_GEMM_NO_BN256
     const int cands[] = {160, 128};
 #else
@@ -707,6 +716,7 @@ static int pick_bn(int64_t M, int64_t N, int num_sms) {
     double best_eff = -1.0;
     for (int bn : cands) {
         if (N % bn) continue;
+        if (gemm_threads(pair ? bn / 2 : bn) > 1024) continue;   // a CTA decodes BN (pair: BN / 2) rows
         const int64_t tiles = (M / kGemmBM) * (N / bn);
         const int64_t waves = (tiles + num_sms - 1) / num_sms;
         const double eff = (double)tiles / (double)(waves * num_sms);
@@ -781,14 +791,18 @@ static cudaError_t launch_gemm_pair_t(const CUtensorMap& amap, const GemmArgs& g
 template <int LAYOUT>
 static cudaError_t dispatch_gemm(int bn, const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t s) {
 #ifndef BT_GEMM_NO_PAIR
-    if (ga.M % (2 * kGemmBM) == 0) {
+    if (gemm_pairs(ga.M)) {
         if (bn == 256) return launch_gemm_pair_t<LAYOUT, 256, BT_GEMM_PAIR_SB256, BT_GEMM_PAIR_SA256>(amap, ga, s);
         if (bn == 160) return launch_gemm_pair_t<LAYOUT, 160, BT_GEMM_PAIR_SB160, BT_GEMM_PAIR_SA160>(amap, ga, s);
         return launch_gemm_pair_t<LAYOUT, 128, 4, 3>(amap, ga, s);
     }
 #endif
-    // BN = 256: two weight stages (64 KB each) fit beside the activation ring
-    if (bn == 256) return launch_gemm_t<LAYOUT, 256, 2>(amap, ga, s);
+    // BN = 256: two weight stages (64 KB each) fit beside the activation ring;
+    // with four decoder threads per row its CTA would exceed 1024 threads, and
+    // pick_bn does not choose it
+    if constexpr (gemm_threads(256) <= 1024) {
+        if (bn == 256) return launch_gemm_t<LAYOUT, 256, 2>(amap, ga, s);
+    }
     return bn == 160 ? launch_gemm_t<LAYOUT, 160, BT_GEMM_BSTAGES>(amap, ga, s)
                      : launch_gemm_t<LAYOUT, 128, BT_GEMM_BSTAGES>(amap, ga, s);
 }
