@@ -46,7 +46,7 @@ typedef enum {
     BT_ERR_SHAPE = 2,         /* size constraint violated                */
     BT_ERR_ALIGN = 3,         /* pointer not aligned as required         */
     BT_ERR_WORKSPACE = 4,     /* workspace missing or too small          */
-    BT_ERR_UNSUPPORTED = 5,   /* valid request this build does not serve */
+    BT_ERR_UNSUPPORTED = 5,   /* valid request the library does not serve */
     BT_ERR_CUDA = 6           /* a CUDA launch or query failed           */
 } bt_status;
 
