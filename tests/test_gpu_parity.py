@@ -297,9 +297,11 @@ def test_gemm_2bit_prefill_shape_sampled():
     check(y[rows], y_ref, b, extra=np.abs(y_ref) * 2.0 ** -8)
 
 
+@pytest.mark.parametrize("M", [128, 256])   # 256: CTA pairs
 @pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
-def test_gemm_prerotated_ragged_blocks(layout):
-    M, N, K = 128, 256, 1152
+def test_gemm_prerotated_ragged_blocks(layout, M):
+    # K = 1152: an odd number of K groups, and rows only 2-byte aligned
+    N, K = 256, 1152
     case = workloads.random_case(8500, M, N, K)
     xr = workloads.rng(8501).standard_normal((M, K)) * 2.0
     xr32 = xr.astype(np.float32).astype(np.float64)
@@ -308,8 +310,9 @@ def test_gemm_prerotated_ragged_blocks(layout):
     check(y, y_ref, b, extra=np.abs(y_ref) * 2.0 ** -8)
 
 
-def test_gemm_special_cases():
-    M, N, K = 128, 128, 1024
+@pytest.mark.parametrize("M", [128, 256])
+def test_gemm_special_cases(M):
+    N, K = 128, 1024
     case = workloads.random_case(8600, M, N, K)
     z = np.zeros_like(case["trits"])
     y0 = run_gemm(z, case["scales"], case["x"], case["sign"])
