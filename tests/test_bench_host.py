@@ -88,3 +88,29 @@ def test_reference_arm_prints_one_json_line():
     assert out["impl"] == "reference" and out["unit"] == "GB/s" and out["value"] > 0
     assert out["cpu_baseline"]["kind"] == "oracle"
     assert out["e2e"]["h2d_bytes_per_step"] == 0 and out["e2e"]["d2h_bytes_per_step"] == 0
+
+
+def test_clock_summary_reads_median_and_active_reasons():
+    # index, clocks.sm, clocks.max.sm, power, active mask, hw_slowdown, hw_thermal, sw_thermal, sw_power_cap
+    cs = bench.ClockSampler(0)
+    cs.lines = [
+        "0, 1965, 1965, 700.1, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "0, 1800, 1965, 990.0, 0x0000000000000004, Not Active, Not Active, Not Active, Active",
+        "0, 1900, 1965, 950.0, 0x0000000000000000, Not Active, Not Active, Not Active, Not Active",
+        "garbage line",
+        "0, [N/A], 1965, 1.0, 0x0, Not Active, Not Active, Not Active, Not Active",
+    ]
+    s = cs.summary()
+    assert s["samples"] == 3
+    assert s["sm_mhz"] == 1900.0
+    assert s["sm_max_mhz"] == 1965.0
+    assert s["reasons"] == ["sw_power_cap"]
+
+
+def test_clock_summary_flags_thermal_and_handles_no_samples():
+    cs = bench.ClockSampler(0)
+    cs.lines = ["0, 1500, 1965, 1000.0, 0x48, Active, Not Active, Active, Not Active"]
+    s = cs.summary()
+    assert s["reasons"] == ["hw_slowdown", "sw_thermal_slowdown"]
+    empty = bench.ClockSampler(0)
+    assert empty.summary() == {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
