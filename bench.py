@@ -34,6 +34,10 @@ import numpy as np  # noqa: E402
 
 METRIC = "packed-ternary GEMV weight GB/s (% of HBM peak); pp512 GEMM TFLOP/s"
 L2_BYTES = 126 * 1024 * 1024
+# DRAM bytes (read + write) per launch of the timed GEMV kernel, mean over the
+# three layers, from an ncu capture of the current kernel; None when the kernel
+# has changed since the counters were taken.
+TRAFFIC_PER_LAUNCH = None
 
 
 def _peaks():
@@ -184,7 +188,7 @@ def run_gpu(args, rank, world):
     def timed(gs, steps, warmup, per_call_events=False):
         with torch.cuda.stream(stream):
             for w in range(warmup):
-                gs[w % copies].replay()
+                gs[w % len(gs)].replay()
             torch.cuda.synchronize()
             if world > 1:
                 dist.barrier()
@@ -193,7 +197,7 @@ def run_gpu(args, rank, world):
             en = torch.cuda.Event(enable_timing=True)
             st.record(stream)
             for k in range(steps):
-                gs[(warmup + k) % copies].replay()
+                gs[(warmup + k) % len(gs)].replay()
             en.record(stream)
             torch.cuda.synchronize()
         return max_over_ranks(st.elapsed_time(en) / steps, world, dist, dev)
@@ -293,66 +297,29 @@ def run_gpu(args, rank, world):
     bytes2 = sum(_weight_bytes(L, 1) for L in triple)
     del gs2, reps2
 
-    # ---- prefill GEMM pp512 ----
-    gemm = None
-    try:
-        Mg = 512
-        gm = [_layer_tensors(bt, torch, dev, 0, i, L)[:2] for i, L in enumerate(triple)]
-        Xs = [torch.randn((Mg, L.K), device=dev).to(torch.bfloat16) for L in triple]
-        Ys = [torch.empty((Mg, L.N), dtype=torch.bfloat16, device=dev) for L in triple]
-        wsg = torch.empty(max(bt.gemm_workspace_bytes(0, Mg, L.N, L.K) for L in triple), dtype=torch.uint8,
-                          device=dev)
-        with torch.cuda.stream(stream):
-            for i, L in enumerate(triple):
-                bt.gemm(gm[i][0], gm[i][1], Xs[i], sign, L.N, 0, out=Ys[i], ws=wsg)
-            torch.cuda.synchronize()
-            gr = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gr, stream=stream):
-                for i, L in enumerate(triple):
-                    bt.gemm(gm[i][0], gm[i][1], Xs[i], sign, L.N, 0, out=Ys[i], ws=wsg)
-            gms = timed([gr] * copies, args.steps, args.warmup)
-        flops = sum(2.0 * Mg * L.N * L.K for L in triple)
-        tf = flops / (gms * 1e-3) / 1e12
-        gemm = {"value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(gms, 4),
-                "workload": "pp512 triple, base-3", "frac_of_peak": round(tf / peaks["bf16_tflops"], 4),
-                "peak": peaks["bf16_tflops"], "peak_kind": f"bf16 burst, {peaks['src']}"}
-    except Exception as e:  # the prefill path is reported, not required for the headline
-        gemm = {"value": None, "error": str(e)[:200]}
+    # ---- prefill GEMM pp512, both layouts (seeded C3 / C4 inputs) ----
+    gemm = {}
+    for layout, cfg, name in ((0, "C3", "base-3"), (1, "C4", "2-bit")):
+        try:
+            gemm[name] = run_gemm(bt, torch, dev, stream, sign, layout, cfg, args, timed, peaks)
+        except Exception as e:  # the prefill path is reported, not required for the headline
+            gemm[name] = {"value": None, "error": str(e)[:200]}
 
     # ---- 27B-equivalent decode sweep: 64 stacks x 2 triples = 384 matrices
     sweep = None
     if not args.no_sweep:
-        try:
-            sweep = run_sweep(bt, torch, dev, stream, sign, args, world, dist)
-        except Exception as e:
-            sweep = {"error": str(e)[:200]}
+        sweep = {}
+        for layout, name in ((0, "base-3"), (1, "2-bit")):
+            try:
+                sweep[name] = run_sweep(bt, torch, dev, stream, sign, args, world, dist, layout)
+            except Exception as e:
+                sweep[name] = {"error": str(e)[:200]}
 
-    # ---- standalone rotation sweep (graphs of 20 calls; the largest inputs are L2-resident)
+    # ---- standalone rotation sweep: graphs of calls over distinct buffers; where
+    # one call's input + output is large, enough buffers that the set exceeds 4x L2
     fwht = {}
     try:
-        for Mf in (1, 16, 512):
-            for Kf in (1024, 5120, 17408):
-                xf = torch.randn((Mf, Kf), device=dev).to(torch.bfloat16)
-                of = torch.empty((Mf, Kf), dtype=torch.float32, device=dev)
-                with torch.cuda.stream(stream):
-                    bt.fwht1024(xf, sign, out=of)
-                    torch.cuda.synchronize()
-                    gr = torch.cuda.CUDAGraph()
-                    with torch.cuda.graph(gr, stream=stream):
-                        for _ in range(20):
-                            bt.fwht1024(xf, sign, out=of)
-                    gr.replay()
-                    torch.cuda.synchronize()
-                    a_ = torch.cuda.Event(enable_timing=True)
-                    b_ = torch.cuda.Event(enable_timing=True)
-                    a_.record(stream)
-                    for _ in range(10):
-                        gr.replay()
-                    b_.record(stream)
-                    torch.cuda.synchronize()
-                    del gr
-                us = a_.elapsed_time(b_) * 1e3 / 200
-                fwht[f"M{Mf}xK{Kf}"] = {"us": round(us, 2), "GB/s": round(Mf * Kf * 6 / (us * 1e-6) / 1e9, 1)}
+        fwht = run_fwht_sweep(bt, torch, dev, stream, sign)
     except Exception as e:
         fwht = {"error": str(e)[:200]}
 
@@ -383,7 +350,8 @@ def run_gpu(args, rank, world):
         "layout_2bit": {"value": round(bytes2 / (ms2 * 1e-3) / 1e9 * world, 2), "unit": "GB/s",
                         "ms_per_step": round(ms2, 5), "bytes_per_step": bytes2},
         "tokens_per_s_triple": round(1e3 / ms3 * world, 1),
-        "gemm": gemm,
+        "gemm": gemm.get("base-3"),
+        "gemm_2bit": gemm.get("2-bit"),
         "sweep_27b": sweep,
         "fwht_sweep": fwht,
         "e2e": {"value": round(bytes3 / (e2e_ms * 1e-3) / 1e9 * world, 2), "unit": "GB/s",
@@ -394,9 +362,9 @@ def run_gpu(args, rank, world):
                           "ms_per_step": round(e2e_eager_ms, 5)}},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(achieved / peaks["hbm_gbs"], 4),
-                     # dram__bytes_read.sum + dram__bytes_write.sum of gemv_lut_kernel, mean over the
-                     # three layers' launches (profiles/gemv_lut_kernel_b3_triple.md)
-                     "traffic": 14961664,
+                     # dram__bytes_read.sum + dram__bytes_write.sum of the GEMV kernel per launch, mean
+                     # over the three layers (one ncu capture of this kernel build)
+                     "traffic": TRAFFIC_PER_LAUNCH,
                      "algorithmic_bytes_per_launch": int(sum(dom_bytes) / len(dom_bytes)),
                      "kernel": "bt_gemv call (table-lookup GEMV kernel + chunk reduction), weighted over the three layers",
                      "peak_kind": f"HBM copy, {peaks['src']}"},
@@ -408,22 +376,96 @@ def run_gpu(args, rank, world):
     return out
 
 
-def run_sweep(bt, torch, dev, stream, sign, args, world, dist):
+def run_gemm(bt, torch, dev, stream, sign, layout, cfg, args, timed, peaks):
+    """pp512: M = 512 seeded activations (with their outliers) through the triple,
+    one CUDA graph of three bt_gemm calls per step."""
+    import workloads
+    triple = workloads.TRIPLE
+    Mg = 512
+    ins = [workloads.layer_inputs(cfg, L, M=Mg, index=i) for i, L in enumerate(triple)]
+    gm = [(bt.pack(torch.from_numpy(c["trits"]).to(dev), layout), torch.from_numpy(c["scales"].view(np.int16)).to(dev))
+          for c in ins]
+    Xs = [torch.from_numpy(c["x"].view(np.int16)).to(dev).view(torch.bfloat16) for c in ins]
+    del ins
+    Ys = [torch.empty((Mg, L.N), dtype=torch.bfloat16, device=dev) for L in triple]
+    wsg = torch.empty(max(bt.gemm_workspace_bytes(layout, Mg, L.N, L.K) for L in triple), dtype=torch.uint8,
+                      device=dev)
+    with torch.cuda.stream(stream):
+        for i, L in enumerate(triple):
+            bt.gemm(gm[i][0], gm[i][1], Xs[i], sign, L.N, layout, out=Ys[i], ws=wsg)
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            for i, L in enumerate(triple):
+                bt.gemm(gm[i][0], gm[i][1], Xs[i], sign, L.N, layout, out=Ys[i], ws=wsg)
+        gms = timed([gr], args.steps, args.warmup)
+        del gr
+    flops = sum(2.0 * Mg * L.N * L.K for L in triple)
+    tf = flops / (gms * 1e-3) / 1e12
+    return {"value": round(tf, 2), "unit": "TFLOP/s", "ms_per_step": round(gms, 4),
+            "workload": f"pp512 triple, {'base-3' if layout == 0 else '2-bit'}, seeded {cfg} activations",
+            "frac_of_peak": round(tf / peaks["bf16_tflops"], 4), "peak": peaks["bf16_tflops"],
+            "peak_kind": f"bf16 burst, {peaks['src']}",
+            "l2": "weights (21-26 MB per matrix) re-read from L2 across steps; the activations dominate traffic"}
+
+
+def run_fwht_sweep(bt, torch, dev, stream, sign):
+    """bt_fwht1024 at M in {1, 16, 512} x K in {1024, 5120, 17408}, FP32 output: per
+    size, a CUDA graph of calls over distinct input/output buffers (as many as
+    keep the set above 4x L2, at most 20). GB/s counts bf16 in + FP32 out."""
+    import workloads
+    out = {}
+    for Mf in (1, 16, 512):
+        for Kf in (1024, 5120, 17408):
+            per = Mf * Kf * 6
+            nbuf = max(1, min(20, math.ceil(4 * L2_BYTES / per)))
+            resident = nbuf * per > 4 * L2_BYTES
+            g = workloads.rng(5 * 1_000_003 + Mf * 7 + Kf)
+            xb = torch.from_numpy(workloads.activations_bf16_bits(g, Mf, Kf, True).view(np.int16)).to(dev) \
+                .view(torch.bfloat16)
+            xs = [xb.clone() for _ in range(nbuf)]
+            os_ = [torch.empty((Mf, Kf), dtype=torch.float32, device=dev) for _ in range(nbuf)]
+            calls = 20
+            with torch.cuda.stream(stream):
+                bt.fwht1024(xs[0], sign, out=os_[0])
+                torch.cuda.synchronize()
+                gr = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gr, stream=stream):
+                    for c in range(calls):
+                        bt.fwht1024(xs[c % nbuf], sign, out=os_[c % nbuf])
+                gr.replay()
+                torch.cuda.synchronize()
+                a_ = torch.cuda.Event(enable_timing=True)
+                b_ = torch.cuda.Event(enable_timing=True)
+                a_.record(stream)
+                for _ in range(10):
+                    gr.replay()
+                b_.record(stream)
+                torch.cuda.synchronize()
+                del gr
+            us = a_.elapsed_time(b_) * 1e3 / (10 * calls)
+            out[f"M{Mf}xK{Kf}"] = {"us": round(us, 2), "GB/s": round(per / (us * 1e-6) / 1e9, 1),
+                                   "buffers": nbuf, "hbm_resident": resident}
+            del xs, os_
+    return out
+
+
+def run_sweep(bt, torch, dev, stream, sign, args, world, dist, layout=0):
     """Decode token through 64 stacks x 2 triples (384 matrices, 26.2e9 weights, 5.7 GB
-    base-3): one seeded triple generated on the host and cloned on the device to 128
-    distinct copies at distinct addresses; one token step = 384 bt_gemv calls replayed
-    from CUDA graphs."""
+    base-3 / 7.0 GB 2-bit): one seeded triple generated on the host and cloned on the
+    device to 128 distinct copies at distinct addresses; one token step = 384 bt_gemv
+    calls replayed from CUDA graphs."""
     import workloads
     triple = workloads.TRIPLE
     uniq = []
     for i, L in enumerate(triple):
         inp = workloads.layer_inputs("C2", L, index=i, with_x=False)
-        uniq.append((bt.pack(torch.from_numpy(inp["trits"]).to(dev), 0),
+        uniq.append((bt.pack(torch.from_numpy(inp["trits"]).to(dev), layout),
                      torch.from_numpy(inp["scales"].view(np.int16)).to(dev)))
     n_triples = 128
     mats = [[(c.clone(), s.clone()) for c, s in uniq] for _ in range(n_triples)]
     del uniq
-    weight_bytes = n_triples * sum(_weight_bytes(L, 0) for L in triple)
+    weight_bytes = n_triples * sum(_weight_bytes(L, layout) for L in triple)
     out = {"weights": int(n_triples * sum(L.N * L.K for L in triple)), "bytes_per_token": weight_bytes,
            "matrices": 3 * n_triples}
     for M in (1, 4, 16):
@@ -431,12 +473,12 @@ def run_sweep(bt, torch, dev, stream, sign, args, world, dist):
         xs = [torch.from_numpy(workloads.activations_bf16_bits(g, M, L.K, True).view(np.int16)).to(dev)
               .view(torch.bfloat16) for L in triple]
         ys = [torch.empty((M, L.N), device=dev) for L in triple]
-        ws = torch.empty(max(bt.gemv_workspace_bytes(0, M, L.N, L.K) for L in triple), dtype=torch.uint8,
+        ws = torch.empty(max(bt.gemv_workspace_bytes(layout, M, L.N, L.K) for L in triple), dtype=torch.uint8,
                          device=dev)
         graphs = []
         with torch.cuda.stream(stream):
             for i, L in enumerate(triple):
-                bt.gemv(mats[0][i][0], mats[0][i][1], xs[i], sign, L.N, 0, out=ys[i], ws=ws)
+                bt.gemv(mats[0][i][0], mats[0][i][1], xs[i], sign, L.N, layout, out=ys[i], ws=ws)
             torch.cuda.synchronize()
             per_graph = 16
             for g0 in range(0, n_triples, per_graph):
@@ -444,7 +486,7 @@ def run_sweep(bt, torch, dev, stream, sign, args, world, dist):
                 with torch.cuda.graph(gr, stream=stream):
                     for t in range(g0, g0 + per_graph):
                         for i, L in enumerate(triple):
-                            bt.gemv(mats[t][i][0], mats[t][i][1], xs[i], sign, L.N, 0, out=ys[i], ws=ws)
+                            bt.gemv(mats[t][i][0], mats[t][i][1], xs[i], sign, L.N, layout, out=ys[i], ws=ws)
                 graphs.append(gr)
             for gr in graphs:
                 gr.replay()
@@ -465,6 +507,7 @@ def run_sweep(bt, torch, dev, stream, sign, args, world, dist):
                         "weight_GB/s": round(whole_job_rate(weight_bytes, ms, world) / 1e9, 1)}
         del graphs
     out["roofline_tokens_per_s_M1"] = round(_peaks()["hbm_gbs"] * 1e9 / weight_bytes, 1)
+    del mats
     return out
 
 
@@ -498,8 +541,36 @@ def cpu_baseline(budget_s: float):
     sample = ("decode triple M=1 incl. rotation of x, rows per pass " +
               ", ".join(f"{L.name}:{r}/{L.N}" for L, r in zip(workloads.TRIPLE, rows)) +
               f", {passes} passes, {t_total:.1f} s")
-    return {"value": round(b_total / t_total / 1e9, 4), "unit": "GB/s", "cores": oracle.threads(),
-            "kind": "oracle", "sample": sample}
+    # the same oracle on one host thread, on a row sample of each matrix
+    cores = oracle.threads()
+    oracle.set_threads(1)
+    try:
+        r1 = [max(8, r // max(1, cores)) for r in rows]
+        t1, b1 = 0.0, 0
+        for inp, L, r in zip(inputs, workloads.TRIPLE, r1):
+            t0 = time.perf_counter()
+            xr = oracle.rotate_bf16(inp["x"], inp["sign"])
+            oracle.gemv(inp["trits"][:r], inp["scales"][:r], xr)
+            t1 += time.perf_counter() - t0
+            b1 += _weight_bytes(workloads.Layer(L.name, L.K, r), 0)
+    finally:
+        oracle.set_threads(cores)
+    return {"value": round(b_total / t_total / 1e9, 4), "unit": "GB/s", "cores": cores,
+            "kind": "oracle", "sample": sample, "cpu_model": _cpu_model(),
+            "one_thread": {"value": round(b1 / t1 / 1e9, 4), "unit": "GB/s", "cores": 1,
+                           "sample": "rows per matrix " + ", ".join(f"{L.name}:{r}" for L, r in
+                                                                   zip(workloads.TRIPLE, r1)) + f", {t1:.1f} s"}}
+
+
+def _cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
 
 
 def reference_rows(per_row_s, Ns, step_budget_s):
@@ -552,10 +623,55 @@ def run_reference(args):
         "config": {"workload": "decode GEMV M=1 on the 5120x5120 / 5120x17408 / 17408x5120 triple, base-3 g128, "
                                "FWHT-1024 fused", "M": 1},
         "cpu_baseline": {"value": round(v, 4), "unit": "GB/s", "cores": oracle.threads(), "kind": "oracle",
-                         "sample": sample},
+                         "sample": sample, "cpu_model": _cpu_model()},
         "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
         "note": "FP64 CPU oracle on rank 0's host cores; other ranks exit without work",
     }
+
+
+def run_case(case: str, reps: int):
+    """One small workload for a profiler capture (one kernel of interest, a few
+    launches, a few GB on the device at most); prints one line and exits."""
+    import torch
+    import ternary_weight_fwht1024_b200 as bt
+    import workloads
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    sign = torch.from_numpy(workloads.sign1024()).to(dev)
+    if case.startswith("gemv"):
+        # gemv_m<M>_<layout>: the three decode layers at M rows, seeded C2 inputs
+        M = int(case.split("_")[1][1:])
+        layout = 1 if case.endswith("2bit") else 0
+        for i, L in enumerate(workloads.TRIPLE):
+            inp = workloads.layer_inputs("C2", L, M=M, index=i)
+            codes = bt.pack(torch.from_numpy(inp["trits"]).to(dev), layout)
+            sc = torch.from_numpy(inp["scales"].view(np.int16)).to(dev)
+            x = torch.from_numpy(inp["x"].view(np.int16)).to(dev).view(torch.bfloat16)
+            for _ in range(reps):
+                bt.gemv(codes, sc, x, sign, L.N, layout)
+    elif case.startswith("gemm"):
+        # gemm_<layout>: pp512 on the 5120x5120 layer
+        layout = 1 if case.endswith("2bit") else 0
+        L = workloads.TRIPLE[0]
+        inp = workloads.layer_inputs("C3", L, M=512, index=0)
+        codes = bt.pack(torch.from_numpy(inp["trits"]).to(dev), layout)
+        sc = torch.from_numpy(inp["scales"].view(np.int16)).to(dev)
+        x = torch.from_numpy(inp["x"].view(np.int16)).to(dev).view(torch.bfloat16)
+        for _ in range(reps):
+            bt.gemm(codes, sc, x, sign, L.N, layout)
+    elif case == "fwht":
+        # 512 x 17408 (53 MB in + out) over distinct buffers: 10 of them exceed 4x L2
+        g = workloads.rng(77)
+        xs = [torch.from_numpy(workloads.activations_bf16_bits(g, 512, 17408, True).view(np.int16)).to(dev)
+              .view(torch.bfloat16) for _ in range(10)]
+        outs = [torch.empty((512, 17408), dtype=torch.float32, device=dev) for _ in range(10)]
+        for r in range(reps):
+            for x, o in zip(xs, outs):
+                bt.fwht1024(x, sign, out=o)
+    else:
+        raise SystemExit(f"unknown case {case}")
+    torch.cuda.synchronize()
+    print(json.dumps({"case": case, "reps": reps, "ok": True}))
 
 
 def main():
@@ -569,7 +685,13 @@ def main():
                     help="CPU time the reference arm spends over warm-up + timed steps")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the 384-matrix 27B-equivalent sweep")
+    ap.add_argument("--case", default=None,
+                    help="run one small workload for a profiler capture (gemv_m<M>[_2bit], gemm[_2bit], fwht)")
+    ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
+    if args.case:
+        run_case(args.case, args.reps)
+        return
     args.warmup = max(3, args.warmup)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))

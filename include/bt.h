@@ -168,9 +168,11 @@ bt_status bt_gemv(int layout, const uint8_t* codes, const uint16_t* scales,
  * every GPU that loads libbt.so until the process exits. Requests whose
  * bt_gemv_workspace_bytes exceeds 4 MiB (for example M = 16 on 17408-row
  * matrices) are rejected with BT_ERR_WORKSPACE before anything is launched.
- * The first call on a device looks up the array's device address (once per
- * device, with that device current); make that first call before any stream
- * capture. All calls share the one array and it keeps the last call's
+ * The first call in a CUDA context looks up the array's device address
+ * (for the usual primary context: once per device, with that device
+ * current) and caches it for that context; a context created later on the
+ * same device -- after cudaDeviceReset, or a caller's own context -- gets a
+ * lookup of its own. Make that first call before any stream capture. All calls share the one array and it keeps the last call's
  * contents (everything that must start at zero is cleared by the call), so
  * calls that may overlap on the GPU -- on different streams, or from
  * different host threads -- race and must be serialised by the caller.

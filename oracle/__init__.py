@@ -69,6 +69,7 @@ def _load():
             lib.oracle_f16_array_to_double.argtypes = [P, I64, P]
             lib.oracle_bf16_array_to_double.argtypes = [P, I64, P]
             lib.oracle_threads.restype = ctypes.c_int
+            lib.oracle_set_threads.argtypes = [ctypes.c_int]
             _lib = lib
     return _lib
 
@@ -84,6 +85,11 @@ def _check(rc: int, what: str):
 
 def threads() -> int:
     return _load().oracle_threads()
+
+
+def set_threads(n: int) -> None:
+    """Host threads the oracle's parallel loops use from now on (timing only)."""
+    _load().oracle_set_threads(int(n))
 
 
 def bytes_per_group(layout: int) -> int:

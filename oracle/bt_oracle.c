@@ -302,3 +302,14 @@ int oracle_threads(void)
     return 1;
 #endif
 }
+
+/* Threads the parallel loops above use from now on (timing only). */
+void oracle_set_threads(int n)
+{
+#ifdef _OPENMP
+    extern void omp_set_num_threads(int);
+    if (n > 0) omp_set_num_threads(n);
+#else
+    (void)n;
+#endif
+}

@@ -1390,14 +1390,33 @@ cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales
 // Scratch for bt_gemv_noalloc: a fixed array in device memory, reserved by
 // every GPU that loads the library for as long as the process lives. Host
 // code only ever sees a stand-in for `noalloc_scratch`, so its device address
-// is looked up once per device with cudaGetSymbolAddress (with that device
-// current) and cached; the first call on a device does this lookup.
+// is looked up with cudaGetSymbolAddress in the context that is current on the
+// calling thread. The address belongs to that context's copy of the module,
+// so it is cached per context (not per device ordinal): a context created
+// later on the same device -- after cudaDeviceReset, or a caller's own
+// non-primary context -- gets its own lookup, never a stale address.
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
 static __device__ __align__(256) uint8_t noalloc_scratch[kNoAllocScratchBytes];
 
-constexpr int kMaxDevices = 64;
+constexpr int kMaxContexts = 64;
 static std::mutex g_scratch_mutex;
-static void* g_scratch_ptr[kMaxDevices];
+static CUcontext g_scratch_ctx[kMaxContexts];
+static void* g_scratch_ptr[kMaxContexts];
+static int g_scratch_used = 0;
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+
+static CtxGetCurrentFn ctx_get_current() {
+    static CtxGetCurrentFn fn = nullptr;
+    if (!fn) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<CtxGetCurrentFn>(p);
+    }
+    return fn;
+}
 
 size_t gemv_noalloc_max_bytes() { return kNoAllocScratchBytes; }
 
@@ -1405,15 +1424,34 @@ cudaError_t gemv_noalloc_scratch(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    std::lock_guard<std::mutex> lock(g_scratch_mutex);
-    if (!g_scratch_ptr[dev]) {
-        void* p = nullptr;
-        e = cudaGetSymbolAddress(&p, noalloc_scratch);
-        if (e != cudaSuccess) return e;
-        g_scratch_ptr[dev] = p;
+    CtxGetCurrentFn get = ctx_get_current();
+    CUcontext ctx = nullptr;
+    if (get && get(&ctx) == CUDA_SUCCESS && ctx) {
+        std::lock_guard<std::mutex> lock(g_scratch_mutex);
+        for (int i = 0; i < g_scratch_used; ++i) {
+            if (g_scratch_ctx[i] == ctx) {
+                *out = g_scratch_ptr[i];
+                return cudaSuccess;
+            }
+        }
     }
-    *out = g_scratch_ptr[dev];
+    // first call in this context (or no context yet: the runtime binds the
+    // device's primary context here)
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    ctx = nullptr;
+    if (get && get(&ctx) == CUDA_SUCCESS && ctx) {
+        std::lock_guard<std::mutex> lock(g_scratch_mutex);
+        bool known = false;
+        for (int i = 0; i < g_scratch_used; ++i) known = known || g_scratch_ctx[i] == ctx;
+        if (!known && g_scratch_used < kMaxContexts) {
+            g_scratch_ctx[g_scratch_used] = ctx;
+            g_scratch_ptr[g_scratch_used] = p;
+            ++g_scratch_used;
+        }
+    }
+    *out = p;
     return cudaSuccess;
 }
 

@@ -291,8 +291,22 @@ struct LutRing {
     int cbox;
 };
 
+// The test-only build of the library (BT_TEST_WITHHOLD_COPY, never the
+// product) leaves out one copy -- the second set of CTA 0's warp 0 -- so that
+// the bounded wait on it runs out: the kernel must then set
+// BT_DEVERR_TIMEOUT, let its other copies land and return.
+__device__ __forceinline__ bool lut_withheld(uint32_t n) {
+#ifdef BT_TEST_WITHHOLD_COPY
+    return blockIdx.x == 0 && (threadIdx.x >> 5) == 0 && n == 1;
+#else
+    (void)n;
+    return false;
+#endif
+}
+
 __device__ __forceinline__ void lut_issue_set(const LutRing& rg, const CUtensorMap* cmap, const CUtensorMap* smap,
                                               uint32_t n, int cx, int sx, int64_t r0) {
+    if (lut_withheld(n)) return;
     const uint32_t d = n % kLutDepth;
     const uint32_t dst = rg.ring + d * rg.slot_bytes;
     const uint32_t bar = rg.bar + 8 * d;
@@ -433,10 +447,10 @@ gemv_lut_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant_
             if (L < kLutSet && r0 + L < w_hi) pout[r0 + L] = v;
         }
     }
-    // after a timeout: let the copies still in flight land before exiting
-    for (; done < issued; ++done) {
-        if (!mbar_wait(rg.bar + 8 * (done % kLutDepth), (done / kLutDepth) & 1u)) break;
-    }
+    // after a timeout: let every copy still in flight land before exiting
+    // (each wait is bounded; a set whose wait ran out does not stop the
+    // waits on the sets requested after it)
+    for (; done < issued; ++done) mbar_wait(rg.bar + 8 * (done % kLutDepth), (done / kLutDepth) & 1u);
 
     if (bad) report(a.dev_err, (int)bad);
 }

@@ -188,7 +188,12 @@ __device__ __forceinline__ void load_signed_bf16_block(const uint16_t* xb, const
 
 // ------------------------------------------------ mbarriers and TMA ----
 
-constexpr uint32_t kSpinLimit = 1u << 26;  // bound on every barrier wait
+// Bound on every barrier wait (iterations of try_wait). The test-only build
+// of the library lowers it so that a withheld copy times out quickly.
+#ifndef BT_SPIN_LIMIT
+#define BT_SPIN_LIMIT (1u << 26)
+#endif
+constexpr uint32_t kSpinLimit = BT_SPIN_LIMIT;
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {
     return static_cast<uint32_t>(__cvta_generic_to_shared(p));

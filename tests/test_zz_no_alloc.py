@@ -28,12 +28,22 @@ def _tensors(case, layout):
     return codes, scales, x, sign
 
 
+# (1, 5120, 5120): the single-row kernel; (3, 1000, 3072): one TMA-fed launch;
+# (9, 5120, 5120): two launches that reuse the scratch's counters and partials;
+# (2, 1000, 3200): K not a multiple of 1024, pre-rotated FP32 x, the general
+# register-fed kernel.
 @pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
-@pytest.mark.parametrize("M,N,K", [(1, 5120, 5120), (3, 1000, 3072)])
+@pytest.mark.parametrize("M,N,K", [(1, 5120, 5120), (3, 1000, 3072), (9, 5120, 5120), (2, 1000, 3200)])
 def test_noalloc_matches_workspace_entry_point(layout, M, N, K):
     case = workloads.random_case(7000 + M + layout, M, N, K)
+    assert bt.gemv_workspace_bytes(layout, M, N, K) <= (4 << 20)
     codes, scales, x, sign = _tensors(case, layout)
-    _, y_ref, bound = oracle.forward(case["trits"], case["scales"], case["x"], case["sign"])
+    if K % 1024:
+        xr = workloads.rng(7100 + M).standard_normal((M, K)).astype(np.float32)
+        x, sign = torch.from_numpy(xr).to(x.device), None
+        y_ref, bound = oracle.gemv(case["trits"], case["scales"], xr.astype(np.float64))
+    else:
+        _, y_ref, bound = oracle.forward(case["trits"], case["scales"], case["x"], case["sign"])
     y_ws = bt.gemv(codes, scales, x, sign, N, layout).cpu().numpy().astype(np.float64)
     for _ in range(2):  # two calls in a row share (and reuse) the scratch array
         err = torch.zeros(1, dtype=torch.int32, device=x.device)
