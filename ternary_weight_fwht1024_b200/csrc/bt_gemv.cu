@@ -34,6 +34,7 @@
 //     it last (atomic counter) adds them in a fixed order, so results are
 //     deterministic run to run.
 #include "bt_internal.cuh"
+#include "bt_slots.cuh"
 
 #include <mutex>
 
@@ -51,56 +52,6 @@ constexpr int kPrepThreads = 256;    // 8 warps: one per group of a 1024-block
 constexpr int kLutBytes = 256 * 256; // 256 codes x (128 B low table + 128 B high table)
 constexpr int kZeroBytes = 512;      // zero fragment area (>= NT * 32)
 constexpr size_t kBsmemMax = 128 * 1024;
-
-// field mask: 2-bit field i of both 16-bit halves
-__host__ __device__ constexpr uint32_t fmask(int i) {
-    return (3u << (2 * i)) | (3u << (2 * i + 16));
-}
-
-// ---------------------------------------------------------- slot maps ----
-// Slot (t, c, h): MMA step t of a group, lane c of a quad (threadID_in_group),
-// half h: 0/1 = low/high half of fragment register a0, 2/3 = of a2.
-// Returns the k (0..127) the slot carries, or -1 for an empty slot; *field is
-// the 2-bit field index i of that trit inside its 16-bit half.
-
-__device__ __forceinline__ int b3_slot(int t, int c, int h, int* field) {
-    // lane c decodes byte pairs 3c, 3c+1, 3c+2 (bytes 6c..6c+5) into registers
-    // rho = 5 q + i; pair 12 (bytes 24, 25) is shared by lanes c (fields
-    // {0,1,2} for even c, {3,4} for odd c) and appears as registers Q0..Q2.
-    const int which = h >> 1, hi = h & 1;
-    int rho = -1, qi = -1;
-    if (t < 7) rho = 2 * t + which;
-    else if (t == 7) { if (which == 0) rho = 14; else qi = 0; }
-    else qi = which == 0 ? 1 : 2;
-    if (rho >= 0) {
-        const int q = rho / 5, i = rho % 5, p = 3 * c + q;
-        *field = i;
-        return 10 * p + (hi ? 5 : 0) + i;
-    }
-    const int f = (c & 1) == 0 ? qi : (qi < 2 ? 3 + qi : -1);
-    if (f < 0) return -1;
-    const int k = (hi ? 125 : 120) + f;
-    if (k >= kGroup) return -1;  // the two pad trits
-    *field = f;
-    return k;
-}
-
-__device__ __forceinline__ int tb_slot(int t, int c, int h, int* field) {
-    // lane c holds bytes 8c..8c+7 = two words of 16 trits; register
-    // rho = 8 w + f holds trits f and 8 + f of word w (f < 6 directly, f = 6, 7
-    // after a 12-bit shift, then as field f - 6).
-    const int rho = 2 * t + (h >> 1), hi = h & 1;
-    const int w = rho >> 3, f = rho & 7;
-    *field = f < 6 ? f : f - 6;
-    return 32 * c + 16 * w + (hi ? 8 : 0) + f;
-}
-
-__device__ __forceinline__ int b3_field_of(int k) { return k % 5; }
-__device__ __forceinline__ int tb_field_of(int k) { const int f = k & 7; return f < 6 ? f : f - 6; }
-
-__device__ __forceinline__ float exp2i(int n) {  // 2^n for n in [-126, 127]
-    return __int_as_float((n + 127) << 23);
-}
 
 // ----------------------------------------------------------- prep ----------
 
@@ -165,35 +116,49 @@ __global__ void __launch_bounds__(kPrepThreads) gemv_prep_kernel(PrepArgs a) {
     int E = amax > 0.f ? ilogbf(amax) + 1 : -100;  // amax < 2^E
     E = max(-100, min(100, E));
     const int e = 9 + E;
-    float corr = 0.f;
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int k = 32 * r + lane;
-        const int i = LAYOUT == BT_LAYOUT_B3 ? b3_field_of(k) : tb_field_of(k);
-        const __half hv = __float2half_rn(v4[r] * exp2i(24 - 2 * i - e));
-        corr += __half2float(hv) * exp2i(e + 2 * i - 24);
-    }
-#pragma unroll
-    for (int s = 16; s > 0; s >>= 1) corr += __shfl_xor_sync(0xffffffffu, corr, s);
+    // Lanes 0..3 (c) write their own fragment words -- (t, c) pairs of FP16
+    // slots, as the MMA's B operand expects -- and keep them for the
+    // correction below.
     const int64_t gidx = (int64_t)m * a.G + 8 * b + q;
-    if (lane == 0) a.meta[gidx] = make_float2(corr, exp2i(e));
     uint32_t* dst = a.bslots + gidx * (NT * 8);
     const float* xg = xs + 128 * q;
-    for (int widx = lane; widx < NT * 8; widx += 32) {
-        const int t = widx >> 3, c = (widx >> 1) & 3, hp = widx & 1;
-        uint32_t word = 0;
+    uint32_t bf[NT][2];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            int i = 0;
-            const int k = LAYOUT == BT_LAYOUT_B3 ? b3_slot(t, c, 2 * hp + u, &i)
-                                                 : tb_slot(t, c, 2 * hp + u, &i);
-            if (k >= 0) {
-                const __half hv = __float2half_rn(xg[k] * exp2i(24 - 2 * i - e));
-                word |= static_cast<uint32_t>(__half_as_ushort(hv)) << (16 * u);
+    for (int t = 0; t < NT; ++t) {
+#pragma unroll
+        for (int hp = 0; hp < 2; ++hp) {
+            uint32_t word = 0;
+            if (lane < 4) {
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    int i = 0;
+                    const int k = LAYOUT == BT_LAYOUT_B3 ? b3_slot(t, lane, 2 * hp + u, &i)
+                                                         : tb_slot(t, lane, 2 * hp + u, &i);
+                    if (k >= 0) {
+                        const __half hv = __float2half_rn(xg[k] * exp2i(24 - 2 * i - e));
+                        word |= static_cast<uint32_t>(__half_as_ushort(hv)) << (16 * u);
+                    }
+                }
+                dst[t * 8 + lane * 2 + hp] = word;
             }
+            bf[t][hp] = word;  // zero outside lanes 0..3: only column 0 is fed
         }
-        dst[widx] = word;
     }
+    // corr = 2^e x (the group's tensor-core sum with every digit 1), by the
+    // same MMA chain the GEMV kernels run: a row of zero trits decodes to
+    // exactly these A registers, so its D equals this one bit for bit and
+    // s * (2^e D - corr) is exactly 0.
+    uint32_t Rg[16], Rh[16];
+    float d[4];
+    if constexpr (LAYOUT == BT_LAYOUT_B3) {
+        uint32_t QG[3], QH[3];
+        b3_ones_tile(lane & 3, Rg, Rh, QG, QH);
+        b3_group_mma(Rg, Rh, QG, QH, bf, d);
+    } else {
+        tb_ones_tile(Rg, Rh);
+        tb_group_mma(Rg, Rh, bf, d);
+    }
+    if (lane == 0) a.meta[gidx] = make_float2(d[0] * exp2i(e), exp2i(e));  // lane 0: D[0][0], column 0
 }
 
 // ----------------------------------------------------------- GEMV ----------
@@ -410,20 +375,9 @@ __device__ __forceinline__ void process_group(const GemvArgs& a, const CodeStage
         }
 #pragma unroll
         for (int mt = 0; mt < MT; ++mt) {
-            float d[4] = {0.f, 0.f, 0.f, 0.f};
-            if constexpr (LAYOUT == BT_LAYOUT_B3) {
-#pragma unroll
-                for (int t = 0; t < 7; ++t)
-                    mma_f16_16816(d, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1], bf[mt][t][0],
-                                  bf[mt][t][1], d);
-                mma_f16_16816(d, Rg[14], Rh[14], QG[0], QH[0], bf[mt][7][0], bf[mt][7][1], d);
-                mma_f16_16816(d, QG[1], QH[1], QG[2], QH[2], bf[mt][NT - 1][0], bf[mt][NT - 1][1], d);
-            } else {
-#pragma unroll
-                for (int t = 0; t < NT; ++t)
-                    mma_f16_16816(d, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1], bf[mt][t][0],
-                                  bf[mt][t][1], d);
-            }
+            float d[4];
+            if constexpr (LAYOUT == BT_LAYOUT_B3) b3_group_mma(Rg, Rh, QG, QH, bf[mt], d);
+            else tb_group_mma(Rg, Rh, bf[mt], d);
             acc[tt][mt][0] = fmaf(sg, fmaf(d[0], pm[mt][0], -cm[mt][0]), acc[tt][mt][0]);
             acc[tt][mt][2] = fmaf(sh, fmaf(d[2], pm[mt][0], -cm[mt][0]), acc[tt][mt][2]);
             if (!M1) {
@@ -733,24 +687,6 @@ constexpr int kTmaThreads = (kTmaConsumers + 1) * 32;
 constexpr int kTmaRows = 64;
 constexpr int kRedBytes = kTmaConsumers * 32 * 8 * 4;   // [warp][32 rows][8 cols] floats
 
-// The five base-3 digits of every byte value as 2-bit fields (bit 31 marks
-// values >= 243), the source of the shared-memory table.
-struct B3FieldTable {
-    uint32_t v[256];
-    constexpr B3FieldTable() : v() {
-        for (int code = 0; code < 256; ++code) {
-            uint32_t f = 0x80000000u;
-            if (code < 243) {
-                f = 0;
-                int r = code;
-                for (int i = 0; i < 5; ++i) { f |= static_cast<uint32_t>(r % 3) << (2 * i); r /= 3; }
-            }
-            v[code] = f;
-        }
-    }
-};
-__constant__ B3FieldTable c_b3_fields = B3FieldTable();
-
 struct GemvTmaArgs {
     const uint32_t* bslots;
     const float2* meta;
@@ -1014,28 +950,9 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant_
                     }
                     // two accumulator chains (even / odd MMA steps) halve the
                     // dependent MMA latency per tile
-                    float d[4] = {0.f, 0.f, 0.f, 0.f}, e4[4] = {0.f, 0.f, 0.f, 0.f};
-                    if constexpr (LAYOUT == BT_LAYOUT_B3) {
-#pragma unroll
-                        for (int t = 0; t < 7; ++t) {
-                            if (t & 1)
-                                mma_f16_16816(e4, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1], bf[t][0], bf[t][1], e4);
-                            else
-                                mma_f16_16816(d, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1], bf[t][0], bf[t][1], d);
-                        }
-                        mma_f16_16816(e4, Rg[14], Rh[14], QG[0], QH[0], bf[7][0], bf[7][1], e4);
-                        mma_f16_16816(d, QG[1], QH[1], QG[2], QH[2], bf[NT - 1][0], bf[NT - 1][1], d);
-                    } else {
-#pragma unroll
-                        for (int t = 0; t < NT; ++t) {
-                            if (t & 1)
-                                mma_f16_16816(e4, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1], bf[t][0], bf[t][1], e4);
-                            else
-                                mma_f16_16816(d, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1], bf[t][0], bf[t][1], d);
-                        }
-                    }
-#pragma unroll
-                    for (int r = 0; r < 4; ++r) d[r] += e4[r];
+                    float d[4];
+                    if constexpr (LAYOUT == BT_LAYOUT_B3) b3_group_mma(Rg, Rh, QG, QH, bf, d);
+                    else tb_group_mma(Rg, Rh, bf, d);
                     acc[tt][0] = fmaf(sgv[tt], fmaf(d[0], pm[0], -cm[0]), acc[tt][0]);
                     acc[tt][2] = fmaf(shv[tt], fmaf(d[2], pm[0], -cm[0]), acc[tt][2]);
                     if (!M1) {

@@ -278,18 +278,28 @@ def test_gemv_special_cases_m1_exact(layout, t):
         assert np.array_equal(y1, expect), (y1[n], expect[n])
 
 
-@pytest.mark.parametrize("M", [2, 4, 16])
-def test_gemv_special_cases_batched(M):
-    # M > 1 runs the tensor-core path, whose digit encoding (t + 1) is undone by a
-    # per-group correction term; zero and single-trit weights stay within the bound.
-    N, K = 64, 2048
+@pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
+@pytest.mark.parametrize("M,K", [(2, 2048), (4, 2048), (16, 2048), (3, 1152)])
+def test_gemv_special_cases_batched(layout, M, K):
+    # M > 1 runs the tensor-core path. Weights enter as digits t + 1; the
+    # per-group correction is the same tensor-core sum taken with every digit
+    # 1, so a row of zero trits cancels exactly: y = 0 bit for bit. (K = 1152:
+    # pre-rotated input, the register-fed kernel.) A single trit stays within
+    # the bound.
+    N = 64
     case = workloads.random_case(5100 + M, M, N, K)
     case["trits"] = np.zeros_like(case["trits"])
-    _, y_ref, b = oracle.forward(case["trits"], case["scales"], case["x"], case["sign"])
-    check(run_gemv(case), y_ref, b)
-    case["trits"][17, 1500] = -1
-    _, y_ref, b = oracle.forward(case["trits"], case["scales"], case["x"], case["sign"])
-    check(run_gemv(case), y_ref, b)
+    rotate = K % 1024 == 0
+    xr = workloads.rng(5200 + M).standard_normal((M, K)).astype(np.float32).astype(np.float64)
+    for checked in (True, False):
+        y0 = run_gemv(case, layout, rotate=rotate, x_f32=None if rotate else xr, checked=checked)
+        assert np.all(y0 == 0.0), float(np.max(np.abs(y0)))
+    case["trits"][17, 1000] = -1
+    if rotate:
+        _, y_ref, b = oracle.forward(case["trits"], case["scales"], case["x"], case["sign"])
+    else:
+        y_ref, b = oracle.gemv(case["trits"], case["scales"], xr)
+    check(run_gemv(case, layout, rotate=rotate, x_f32=None if rotate else xr), y_ref, b)
 
 
 def test_gemv_deterministic():
