@@ -167,7 +167,7 @@ def run_gpu(args, rank, world):
                for L in triple]
     xs = [h.to(dev).view(torch.bfloat16) for h in xs_host]
     ys = [torch.empty((M, L.N), dtype=torch.float32, device=dev) for L in triple]
-    ws = torch.empty(max(bt.gemv_workspace_bytes(l, M, L.N, L.K) for L in triple for l in (0, 1)),
+    ws = torch.zeros(max(bt.gemv_workspace_bytes(l, M, L.N, L.K) for L in triple for l in (0, 1)),
                      dtype=torch.uint8, device=dev)
 
     def graphs_for(reps, layout, with_events=False):
@@ -388,7 +388,7 @@ def run_gemm(bt, torch, dev, stream, sign, layout, cfg, args, timed, peaks):
     Xs = [torch.from_numpy(c["x"].view(np.int16)).to(dev).view(torch.bfloat16) for c in ins]
     del ins
     Ys = [torch.empty((Mg, L.N), dtype=torch.bfloat16, device=dev) for L in triple]
-    wsg = torch.empty(max(bt.gemm_workspace_bytes(layout, Mg, L.N, L.K) for L in triple), dtype=torch.uint8,
+    wsg = torch.zeros(max(bt.gemm_workspace_bytes(layout, Mg, L.N, L.K) for L in triple), dtype=torch.uint8,
                       device=dev)
     with torch.cuda.stream(stream):
         for i, L in enumerate(triple):
@@ -473,7 +473,7 @@ def run_sweep(bt, torch, dev, stream, sign, args, world, dist, layout=0):
         xs = [torch.from_numpy(workloads.activations_bf16_bits(g, M, L.K, True).view(np.int16)).to(dev)
               .view(torch.bfloat16) for L in triple]
         ys = [torch.empty((M, L.N), device=dev) for L in triple]
-        ws = torch.empty(max(bt.gemv_workspace_bytes(layout, M, L.N, L.K) for L in triple), dtype=torch.uint8,
+        ws = torch.zeros(max(bt.gemv_workspace_bytes(layout, M, L.N, L.K) for L in triple), dtype=torch.uint8,
                          device=dev)
         graphs = []
         with torch.cuda.stream(stream):

@@ -157,6 +157,57 @@ bt_status bt_gemv(int layout, const uint8_t* codes, const uint16_t* scales,
                   void* workspace, size_t workspace_bytes, int32_t* dev_err, void* stream);
 
 /*
+ * bt_gemv_batched: the single-row (M = 1) product y_p = W_p (R x_p) for a list
+ * of matrices, in one persistent launch per 12 matrices. A matrix's
+ * activation is either given (x, x_dtype) or the output of an earlier matrix
+ * of the list (x_from >= 0: the chained layers of a decode step), so a whole
+ * token's stack of layers -- or matrices that share nothing -- stream their
+ * weights without a gap between them. Each 1024-block of every activation is
+ * rotated once. Source: release summary, sections 三值权重怎么压缩到 1.76 bit
+ * (R, g128, fused unpack and scale) and 已知短板 (the activation transform
+ * is the largest cost outside the product at batch 1).
+ *  layout     BT_LAYOUT_B3 or BT_LAYOUT_2BIT (one layout per call)
+ *  problems   host array of `count` descriptors (1 <= count <= 256):
+ *    codes    device [N][bt_codes_row_bytes(layout, K)], 16-byte aligned
+ *    scales   device fp16 bits [N][K/128], 16-byte aligned
+ *    x        device [1][K], 16-byte aligned, in x_dtype (BT_BF16, or BT_F32
+ *             when sign1024 is NULL); unused when x_from >= 0
+ *    x_from   -1, or the index of an earlier problem whose y (N == this K,
+ *             in y_dtype) is this activation; with sign1024 that y must be
+ *             bf16 (y_dtype BT_BF16)
+ *    y        device [1][N] in y_dtype, 16-byte aligned
+ *    N >= 1;  K % 1024 == 0, at most 27648 (base-3) / 39936 (2-bit): one
+ *             matrix's activation fragments are held in shared memory
+ *             (BT_ERR_UNSUPPORTED beyond)
+ *  sign1024   as for bt_gemv (NULL: every x is already rotated)
+ *  workspace  device, >= bt_gemv_batched_workspace_bytes(...), 256-byte
+ *             aligned. Its first 4096 bytes are counters: they must be zero
+ *             before the first call of any GEMV entry point with this
+ *             workspace (zero-fill it once when it is allocated); every call
+ *             leaves them zero again. The rest is scratch.
+ *  dev_err    as for bt_gemv; a dependency or copy that does not arrive
+ *             within a bounded time sets BT_DEVERR_TIMEOUT.
+ * Matrices of more than one launch (count > 12) depend on earlier launches
+ * through stream order. Numerics and determinism as for bt_gemv at M > 1:
+ * FP16 activations (one power-of-two exponent per 128), FP32 accumulation,
+ * zero trits contribute exactly 0, and results do not depend on the schedule.
+ */
+typedef struct {
+    const uint8_t* codes;
+    const uint16_t* scales;
+    const void* x;
+    int32_t x_dtype;
+    int32_t x_from;
+    void* y;
+    int64_t N;
+    int64_t K;
+} bt_gemv_problem;
+
+size_t bt_gemv_batched_workspace_bytes(int layout, const bt_gemv_problem* problems, int count);
+bt_status bt_gemv_batched(int layout, const bt_gemv_problem* problems, int count, const int8_t* sign1024,
+                          int y_dtype, void* workspace, size_t workspace_bytes, int32_t* dev_err, void* stream);
+
+/*
  * bt_gemv_noalloc: bt_gemv for callers that cannot allocate device memory --
  * code that runs where cudaMalloc is unavailable or not allowed (inside a
  * custom allocator or memory-pool callback, in a runtime that has handed all

@@ -30,9 +30,16 @@ DEVERR_TIMEOUT = 0x8
 # Exported entry points, as declared in include/bt.h.
 SYMBOLS = (
     "bt_status_string", "bt_version", "bt_codes_row_bytes", "bt_pack", "bt_unpack",
-    "bt_fwht1024", "bt_gemv_workspace_bytes", "bt_gemv", "bt_gemv_noalloc", "bt_gemm_workspace_bytes",
-    "bt_gemm",
+    "bt_fwht1024", "bt_gemv_workspace_bytes", "bt_gemv", "bt_gemv_batched_workspace_bytes", "bt_gemv_batched",
+    "bt_gemv_noalloc", "bt_gemm_workspace_bytes", "bt_gemm",
 )
+
+
+class GemvProblem(ctypes.Structure):
+    """bt_gemv_problem (include/bt.h)."""
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("x", ctypes.c_void_p),
+                ("x_dtype", ctypes.c_int32), ("x_from", ctypes.c_int32), ("y", ctypes.c_void_p),
+                ("N", ctypes.c_int64), ("K", ctypes.c_int64)]
 
 _lock = threading.Lock()
 _lib = None
@@ -66,10 +73,15 @@ def load() -> ctypes.CDLL:
             lib.bt_gemv_workspace_bytes.restype = SZ
             lib.bt_gemv.argtypes = [I, P, P, P, I, P, I64, I64, I64, I, P, P, SZ, P, P]
             lib.bt_gemv_noalloc.argtypes = [I, P, P, P, I, P, I64, I64, I64, I, P, P, P]
+            PP = ctypes.POINTER(GemvProblem)
+            lib.bt_gemv_batched_workspace_bytes.argtypes = [I, PP, I]
+            lib.bt_gemv_batched_workspace_bytes.restype = SZ
+            lib.bt_gemv_batched.argtypes = [I, PP, I, P, I, P, SZ, P, P]
             lib.bt_gemm_workspace_bytes.argtypes = [I, I64, I64, I64]
             lib.bt_gemm_workspace_bytes.restype = SZ
             lib.bt_gemm.argtypes = [I, P, P, P, I, P, I64, I64, I64, P, P, SZ, P, P]
-            for name in ("bt_pack", "bt_unpack", "bt_fwht1024", "bt_gemv", "bt_gemv_noalloc", "bt_gemm"):
+            for name in ("bt_pack", "bt_unpack", "bt_fwht1024", "bt_gemv", "bt_gemv_batched", "bt_gemv_noalloc",
+                         "bt_gemm"):
                 getattr(lib, name).restype = I
             _lib = lib
     return _lib
@@ -103,13 +115,21 @@ def codes_row_bytes(layout: int, K: int) -> int:
 
 
 def workspace(nbytes: int, device) -> torch.Tensor:
-    """A cached uint8 scratch buffer of at least nbytes on `device` (current stream use)."""
+    """A cached uint8 workspace of at least nbytes on `device`, one per stream.
+
+    Zero-filled when allocated: its first 4096 bytes are counters that the
+    library keeps at zero between calls (include/bt.h)."""
     key = (torch.device(device), torch.cuda.current_stream(device).cuda_stream)
     buf = _workspaces.get(key)
     if buf is None or buf.numel() < nbytes:
-        buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        buf = torch.zeros(max(nbytes, 4096), dtype=torch.uint8, device=device)
         _workspaces[key] = buf
     return buf
+
+
+def new_workspace(nbytes: int, device) -> torch.Tensor:
+    """A workspace of its own (zero-filled, as every GEMV workspace must start)."""
+    return torch.zeros(max(nbytes, 4096), dtype=torch.uint8, device=device)
 
 
 def pack(trits: torch.Tensor, layout: int = LAYOUT_B3, dev_err: torch.Tensor | None = None) -> torch.Tensor:
@@ -176,6 +196,49 @@ def gemv(codes: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, sign: torch
                                       M, N, K, y_dtype, _ptr(out), _ptr(ws), ws.numel(), _ptr(dev_err),
                                       _stream(x.device)))
     return out
+
+
+def _problem_array(problems):
+    arr = (GemvProblem * len(problems))()
+    for i, p in enumerate(problems):
+        x = p.get("x")
+        x_from = int(p.get("x_from", -1))
+        arr[i].codes = p["codes"].data_ptr()
+        arr[i].scales = p["scales"].data_ptr()
+        arr[i].x = x.data_ptr() if (x is not None and x_from < 0) else None
+        arr[i].x_dtype = _x_dtype(x) if (x is not None and x_from < 0) else BF16
+        arr[i].x_from = x_from
+        arr[i].y = p["y"].data_ptr()
+        arr[i].N = int(p["N"])
+        arr[i].K = int(p["K"])
+    return arr
+
+
+def gemv_batched_workspace_bytes(layout: int, problems) -> int:
+    arr = _problem_array(problems)
+    return int(load().bt_gemv_batched_workspace_bytes(layout, arr, len(problems)))
+
+
+def gemv_batched(problems, sign: torch.Tensor | None, layout: int = LAYOUT_B3, y_dtype: int = F32,
+                 ws: torch.Tensor | None = None, dev_err: torch.Tensor | None = None):
+    """y_p = W_p (R x_p) for a list of single-row problems in one launch (per 12).
+
+    Each problem is a dict with codes, scales, y ([1, N] of y_dtype), N, K and
+    either x ([1, K] bf16, or f32 when sign is None) or x_from (the index of an
+    earlier problem whose y is this x). Returns the list of y tensors."""
+    if not problems:
+        return []
+    dev = problems[0]["y"].device
+    for p in problems:
+        _require_cuda(p["codes"], p["scales"], p.get("x"), p["y"])
+    _require_cuda(sign, ws, dev_err)
+    arr = _problem_array(problems)
+    need = int(load().bt_gemv_batched_workspace_bytes(layout, arr, len(problems)))
+    if ws is None:
+        ws = workspace(need, dev)
+    _check("bt_gemv_batched", load().bt_gemv_batched(layout, arr, len(problems), _ptr(sign), y_dtype, _ptr(ws),
+                                                      ws.numel(), _ptr(dev_err), _stream(dev)))
+    return [p["y"] for p in problems]
 
 
 def gemv_noalloc(codes: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, sign: torch.Tensor | None, N: int,

@@ -8,8 +8,8 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libbt.so")
-SOURCES = ["bt_api.cu", "bt_pack.cu", "bt_fwht.cu", "bt_gemv.cu", "bt_gemv_lut.cu", "bt_gemm.cu"]
-HEADERS = ["bt_internal.cuh", os.path.join("..", "..", "include", "bt.h")]
+SOURCES = ["bt_api.cu", "bt_pack.cu", "bt_fwht.cu", "bt_gemv.cu", "bt_gemv_lut.cu", "bt_decode.cu", "bt_gemm.cu"]
+HEADERS = ["bt_internal.cuh", "bt_slots.cuh", os.path.join("..", "..", "include", "bt.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",
@@ -23,7 +23,7 @@ FLAGS = [
 # bounded wait run out (BT_DEVERR_TIMEOUT) without faulting or hanging the GPU.
 # Nothing but that test loads it.
 WAITTEST_LIB = os.path.join(HERE, "libbt_waittest.so")
-WAITTEST_FLAGS = ["-DBT_TEST_WITHHOLD_COPY", "-DBT_SPIN_LIMIT=4096u"]
+WAITTEST_FLAGS = ["-DBT_TEST_WITHHOLD_COPY", "-DBT_SPIN_LIMIT=4096u", "-DBT_WAIT_NS=20000000ull"]
 
 
 def _stale(lib: str) -> bool:

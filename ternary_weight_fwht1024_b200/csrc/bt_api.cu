@@ -14,6 +14,20 @@ cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales
                         void* y, void* workspace, int32_t* dev_err, int num_sms, cudaStream_t stream);
 size_t gemv_noalloc_max_bytes();
 cudaError_t gemv_noalloc_scratch(void** out);
+struct DecodeProblem {
+    const uint8_t* codes;
+    const uint16_t* scales;
+    const void* x;
+    int x_bf16;
+    int x_from;
+    void* y;
+    int64_t N, K;
+};
+size_t decode_workspace_bytes(const int64_t* Ks, int count);
+bool decode_applies(int64_t M, int64_t K, const void* codes, const void* scales);
+bool decode_k_fits(int layout, int64_t K);
+cudaError_t launch_decode(int layout, const DecodeProblem* problems, int count, const int8_t* sign, int y_dtype,
+                          void* workspace, int32_t* dev_err, int num_sms, cudaStream_t stream);
 size_t gemm_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num_sms);
 cudaError_t launch_gemm(int layout, const uint8_t* codes, const uint16_t* scales, const void* x,
                         int x_dtype, const int8_t* sign, int64_t M, int64_t N, int64_t K, void* y,
@@ -133,6 +147,18 @@ size_t bt_gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K) {
     return bt::gemv_workspace_bytes(layout, M, N, K, current_sm_count());
 }
 
+// One GEMV call on a validated workspace: single-row calls that fit take the
+// persistent decode kernel, the rest the kernels of bt_gemv.cu.
+cudaError_t run_gemv(int layout, const uint8_t* codes, const uint16_t* scales, const void* x, int x_dtype,
+                     const int8_t* sign1024, int64_t M, int64_t N, int64_t K, int y_dtype, void* y, void* ws,
+                     int32_t* dev_err, int sms, cudaStream_t s) {
+    if (bt::decode_applies(M, K, codes, scales) && bt::decode_k_fits(layout, K)) {
+        bt::DecodeProblem p{codes, scales, x, x_dtype == BT_BF16 ? 1 : 0, -1, y, N, K};
+        return bt::launch_decode(layout, &p, 1, sign1024, y_dtype, ws, dev_err, sms, s);
+    }
+    return bt::launch_gemv(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y_dtype, y, ws, dev_err, sms, s);
+}
+
 bt_status bt_gemv(int layout, const uint8_t* codes, const uint16_t* scales, const void* x, int x_dtype,
                   const int8_t* sign1024, int64_t M, int64_t N, int64_t K, int y_dtype, void* y,
                   void* workspace, size_t workspace_bytes, int32_t* dev_err, void* stream) {
@@ -148,8 +174,52 @@ bt_status bt_gemv(int layout, const uint8_t* codes, const uint16_t* scales, cons
     const size_t need = bt::gemv_workspace_bytes(layout, M, N, K, sms);
     if (!workspace || workspace_bytes < need) return BT_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return BT_ERR_ALIGN;
-    return from_cuda(bt::launch_gemv(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y_dtype, y,
-                                     workspace, dev_err, sms, s));
+    return from_cuda(run_gemv(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y_dtype, y, workspace,
+                              dev_err, sms, s));
+}
+
+size_t bt_gemv_batched_workspace_bytes(int layout, const bt_gemv_problem* problems, int count) {
+    if (!valid_layout(layout) || !problems || count < 1) return 0;
+    int64_t Ks[256];
+    if (count > 256) return 0;
+    for (int i = 0; i < count; ++i) Ks[i] = problems[i].K;
+    return bt::decode_workspace_bytes(Ks, count);
+}
+
+bt_status bt_gemv_batched(int layout, const bt_gemv_problem* problems, int count, const int8_t* sign1024,
+                          int y_dtype, void* workspace, size_t workspace_bytes, int32_t* dev_err, void* stream) {
+    if (!valid_layout(layout) || !valid_dtype(y_dtype)) return BT_ERR_INVALID_ARG;
+    if (count < 0 || count > 256) return BT_ERR_SHAPE;
+    if (count == 0) return BT_OK;
+    if (!problems) return BT_ERR_INVALID_ARG;
+    if (!aligned(dev_err, 4) || !aligned(sign1024, 16)) return BT_ERR_ALIGN;
+    bt::DecodeProblem dp[256];
+    for (int i = 0; i < count; ++i) {
+        const bt_gemv_problem& q = problems[i];
+        if (q.N < 1 || q.K < 1024 || q.K % 1024 != 0 || q.K > (int64_t(1) << 30) || q.N > (int64_t(1) << 30))
+            return BT_ERR_SHAPE;
+        if (!bt::decode_k_fits(layout, q.K)) return BT_ERR_UNSUPPORTED;
+        if (!q.codes || !q.scales || !q.y) return BT_ERR_INVALID_ARG;
+        if (!aligned(q.codes, 16) || !aligned(q.scales, 16) || !aligned(q.y, 16)) return BT_ERR_ALIGN;
+        if (q.x_from >= 0) {
+            if (q.x_from >= i) return BT_ERR_INVALID_ARG;             // only earlier outputs
+            if (problems[q.x_from].N != q.K) return BT_ERR_SHAPE;     // that output is this input
+            if (sign1024 && y_dtype != BT_BF16) return BT_ERR_INVALID_ARG;  // rotation reads bf16
+        } else {
+            if (q.x_from != -1) return BT_ERR_INVALID_ARG;
+            if (!q.x || !valid_dtype(q.x_dtype)) return BT_ERR_INVALID_ARG;
+            if (sign1024 && q.x_dtype != BT_BF16) return BT_ERR_INVALID_ARG;
+            if (!aligned(q.x, 16)) return BT_ERR_ALIGN;
+        }
+        dp[i] = bt::DecodeProblem{q.codes, q.scales, q.x, q.x_from >= 0 ? (y_dtype == BT_BF16 ? 1 : 0)
+                                                                        : (q.x_dtype == BT_BF16 ? 1 : 0),
+                                  q.x_from, q.y, q.N, q.K};
+    }
+    const size_t need = bt_gemv_batched_workspace_bytes(layout, problems, count);
+    if (!workspace || workspace_bytes < need) return BT_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return BT_ERR_ALIGN;
+    return from_cuda(bt::launch_decode(layout, dp, count, sign1024, y_dtype, workspace, dev_err, current_sm_count(),
+                                       static_cast<cudaStream_t>(stream)));
 }
 
 bt_status bt_gemv_noalloc(int layout, const uint8_t* codes, const uint16_t* scales, const void* x,
@@ -167,14 +237,19 @@ bt_status bt_gemv_noalloc(int layout, const uint8_t* codes, const uint16_t* scal
     if (bt::gemv_workspace_bytes(layout, M, N, K, sms) > bt::gemv_noalloc_max_bytes()) return BT_ERR_WORKSPACE;
     void* scratch = nullptr;
     if (bt::gemv_noalloc_scratch(&scratch) != cudaSuccess) { cudaGetLastError(); return BT_ERR_CUDA; }
-    return from_cuda(bt::launch_gemv(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y_dtype, y,
-                                     scratch, dev_err, sms, s));
+    return from_cuda(run_gemv(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y_dtype, y, scratch, dev_err,
+                              sms, s));
 }
+
+// Every workspace keeps its first kSyncBytes for the decode kernel's counters
+// (zero between calls); the GEMM's scratch follows them, so one buffer can
+// serve both entry points.
+constexpr size_t kSyncBytes = 4096;
 
 size_t bt_gemm_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K) {
     if (!valid_layout(layout) || M < 128 || M % 128 != 0 || N < 128 || N % 128 != 0 || K < 128 || K % 128 != 0)
         return 0;
-    return bt::gemm_workspace_bytes(layout, M, N, K, current_sm_count());
+    return kSyncBytes + bt::gemm_workspace_bytes(layout, M, N, K, current_sm_count());
 }
 
 bt_status bt_gemm(int layout, const uint8_t* codes, const uint16_t* scales, const void* x, int x_dtype,
@@ -188,11 +263,11 @@ bt_status bt_gemm(int layout, const uint8_t* codes, const uint16_t* scales, cons
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (K == 0) return from_cuda(launch_zero(y_bf16, M * N * 2, s));
     const int sms = current_sm_count();
-    const size_t need = bt::gemm_workspace_bytes(layout, M, N, K, sms);
+    const size_t need = kSyncBytes + bt::gemm_workspace_bytes(layout, M, N, K, sms);
     if (!workspace || workspace_bytes < need) return BT_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return BT_ERR_ALIGN;
     return from_cuda(bt::launch_gemm(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y_bf16,
-                                     workspace, dev_err, sms, s));
+                                     static_cast<uint8_t*>(workspace) + kSyncBytes, dev_err, sms, s));
 }
 
 }  // extern "C"

@@ -53,6 +53,13 @@ constexpr int kLutBytes = 256 * 256; // 256 codes x (128 B low table + 128 B hig
 constexpr int kZeroBytes = 512;      // zero fragment area (>= NT * 32)
 constexpr size_t kBsmemMax = 128 * 1024;
 
+// Bytes of the per-(row, group) constants (corr, 2^e) kept in shared memory,
+// padded to 16 so that the activation fragments after them start on a
+// 16-byte boundary (they are copied in with 16-byte stores).
+__host__ __device__ constexpr uint32_t meta_area_bytes(int M, int G) {
+    return (static_cast<uint32_t>(M * G * 8) + 15u) & ~15u;
+}
+
 // ----------------------------------------------------------- prep ----------
 
 struct PrepArgs {
@@ -480,7 +487,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1) gemv_kernel(GemvArgs a) {
     }
     const uint32_t zero_area = smem_u32addr(sB);
     const uint32_t meta_area = zero_area + kZeroBytes;
-    const uint32_t slot_area = meta_area + static_cast<uint32_t>(a.M * G * 8);
+    const uint32_t slot_area = meta_area + meta_area_bytes(a.M, G);
     {
         uint4* z = reinterpret_cast<uint4*>(sB);
         for (int i = threadIdx.x; i < kZeroBytes / 16; i += blockDim.x) z[i] = make_uint4(0, 0, 0, 0);
@@ -492,7 +499,7 @@ __global__ void __launch_bounds__(kGemvWarps * 32, 1) gemv_kernel(GemvArgs a) {
         float2* sm = reinterpret_cast<float2*>(sB + kZeroBytes);
         copy_to_smem<float2>(sm, gm, a.M * G);
         const uint4* gb = reinterpret_cast<const uint4*>(a.bslots);
-        uint4* sb = reinterpret_cast<uint4*>(sB + kZeroBytes + a.M * G * 8);
+        uint4* sb = reinterpret_cast<uint4*>(sB + kZeroBytes + meta_area_bytes(a.M, G));
         copy_to_smem<uint4>(sb, gb, a.M * G * NT * 2);  // NT * 32 bytes per (m, g)
     }
     __syncthreads();
@@ -728,7 +735,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant_
     uint8_t* lut = smem;
     uint8_t* sB = smem + (LAYOUT == BT_LAYOUT_B3 ? kLutBytes : 0);
     const int M = a.M, G = a.G, nb = a.nb;
-    const uint32_t bbytes = BSMEM ? static_cast<uint32_t>(M * G * (NT * 32 + 8)) : 0u;
+    const uint32_t bbytes = BSMEM ? static_cast<uint32_t>(M * G * NT * 32) + meta_area_bytes(M, G) : 0u;
     uint8_t* stages = sB + ((kZeroBytes + bbytes + 1023) & ~1023u);
     float* red = reinterpret_cast<float*>(stages + S * GE::kStage);
     uint64_t* full = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(red) + kRedBytes);
@@ -793,7 +800,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant_
             float2* smeta = reinterpret_cast<float2*>(sB + kZeroBytes);
             for (int i = threadIdx.x; i < M * G; i += kTmaConsumers * 32) smeta[i] = __ldcg(a.meta + i);
             const uint4* gb = reinterpret_cast<const uint4*>(a.bslots);
-            uint4* sb = reinterpret_cast<uint4*>(sB + kZeroBytes + M * G * 8);
+            uint4* sb = reinterpret_cast<uint4*>(sB + kZeroBytes + meta_area_bytes(M, G));
             const int n16 = M * G * NT * 2;
             for (int base = 0; base < n16; base += 8 * kTmaConsumers * 32) {
                 uint4 v[8];
@@ -812,7 +819,7 @@ gemv_tma_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant_
         }
         const uint32_t zero_area = smem_u32addr(sB);
         const uint32_t meta_area = zero_area + kZeroBytes;
-        const uint32_t slot_area = meta_area + static_cast<uint32_t>(M * G * 8);
+        const uint32_t slot_area = meta_area + meta_area_bytes(M, G);
         const int m = g;                                  // activation row of this lane's fragment column
         const bool okm = m < M;
         const uint32_t bbase = okm ? slot_area + static_cast<uint32_t>(m * G * NT * 32 + c * 8) : zero_area + c * 8;
@@ -1064,7 +1071,7 @@ static GemvPlan make_gemv_plan(int layout, int64_t M, int64_t N, int64_t K, int 
     pl.chunk = (pl.U + pl.warps_total - 1) / pl.warps_total;
     if (pl.chunk < 1) pl.chunk = 1;
     pl.prep_grid = static_cast<int>(M * ((pl.G + 7) / 8));
-    const size_t bbytes = (size_t)M * pl.G * (pl.NT * 32 + 8);
+    const size_t bbytes = (size_t)M * pl.G * pl.NT * 32 + meta_area_bytes((int)M, (int)pl.G);
     pl.bsmem = M <= 8 && bbytes <= kBsmemMax;
     pl.smem = (layout == BT_LAYOUT_B3 ? kLutBytes : 0) + kZeroBytes + (pl.bsmem ? bbytes : 0);
     size_t off = 0;
@@ -1089,11 +1096,19 @@ cudaError_t launch_gemv_lut(int layout, const uint8_t* codes, const uint16_t* sc
                             const int8_t* sign, int64_t N, int64_t K, int y_dtype, void* y, void* workspace,
                             int32_t* dev_err, int num_sms, cudaStream_t stream);
 
+// The first kSyncBytes of every GEMV workspace hold the counters of the
+// single-row decode kernel (bt_decode.cu), which must stay zero between calls;
+// the kernels of this file use the bytes after them.
+constexpr size_t kSyncBytes = 4096;
+size_t decode_workspace_bytes(const int64_t* Ks, int count);
+
 size_t gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num_sms) {
-    size_t need = make_gemv_plan(layout, M, N, K, num_sms).total;
+    size_t need = kSyncBytes + make_gemv_plan(layout, M, N, K, num_sms).total;
     if (M == 1 && K % 1024 == 0) {
-        const size_t lut = align_up(gemv_lut_workspace_bytes(N, K), 256);
+        const size_t lut = kSyncBytes + align_up(gemv_lut_workspace_bytes(N, K), 256);
         if (lut > need) need = lut;
+        const size_t dec = decode_workspace_bytes(&K, 1);
+        if (dec > need) need = dec;
     }
     return need;
 }
@@ -1122,7 +1137,7 @@ static TmaPlan make_tma_plan(int layout, int64_t M, int64_t N, int64_t K, const 
     const size_t stage = (size_t)kTmaRows * RB + kTmaRows * 16;
     const size_t limit = 227 * 1024;
     const size_t lutb = layout == BT_LAYOUT_B3 ? kLutBytes : 0;
-    const size_t bbytes = align_up(kZeroBytes + (size_t)M * G * (NT * 32 + 8), 1024);
+    const size_t bbytes = align_up(kZeroBytes + (size_t)M * G * NT * 32 + meta_area_bytes((int)M, G), 1024);
     const size_t nob = align_up(kZeroBytes, 1024);
     t.use = false;
     for (int st : {6, 5, 4, 3}) {      // prefer activation fragments in shared memory, then more stages
@@ -1206,11 +1221,11 @@ cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales
                         int x_dtype, const int8_t* sign, int64_t M, int64_t N, int64_t K, int y_dtype,
                         void* y, void* workspace, int32_t* dev_err, int num_sms,
                         cudaStream_t stream) {
+    uint8_t* ws = static_cast<uint8_t*>(workspace) + kSyncBytes;
     if (gemv_lut_applies(M, K, scales))
-        return launch_gemv_lut(layout, codes, scales, x, x_dtype, sign, N, K, y_dtype, y, workspace, dev_err,
+        return launch_gemv_lut(layout, codes, scales, x, x_dtype, sign, N, K, y_dtype, y, ws, dev_err,
                                num_sms, stream);
     const GemvPlan pl = make_gemv_plan(layout, M, N, K, num_sms);
-    uint8_t* ws = static_cast<uint8_t*>(workspace);
 
     PrepArgs pa{};
     pa.x = x;

@@ -1,12 +1,17 @@
 """Failure detection on the GPU without a fault: a bounded wait that runs out.
 
-Every mbarrier wait in libbt.so gives up after a fixed number of tries, sets
-BT_DEVERR_TIMEOUT in the caller's error word, lets its copies still in flight
-land and returns, so the context stays usable. This test loads the test-only
-twin of the library (libbt_waittest.so: the table-lookup GEMV never requests
-one set of rows -- the second set of CTA 0's warp 0 -- and gives up after 4096
-tries) and checks that the call returns with the timeout bit set, and that
-the product library still matches the oracle afterwards in the same process.
+Every wait in libbt.so is bounded (a number of tries, or a time on the global
+timer); one that runs out sets BT_DEVERR_TIMEOUT in the caller's error word,
+lets the copies still in flight land and returns, so the context stays
+usable. These tests load the test-only twin of the library
+(libbt_waittest.so), in which one copy is never requested and the bounds are
+short (4096 tries, 20 ms):
+  * the table-lookup GEMV (single row, K beyond the decode kernel's limit):
+    the second set of rows of CTA 0's warp 0;
+  * the persistent decode kernel (single row): the second stage of CTA 0's
+    first team.
+Each test checks that the call returns with the timeout bit set, and that the
+product library still matches the oracle afterwards in the same process.
 Nothing traps, faults or spins without a bound.
 """
 import ctypes
@@ -49,7 +54,7 @@ def test_withheld_copy_times_out_and_the_context_survives():
 
     lib = _waittest_lib()
     need = lib.bt_gemv_workspace_bytes(bt.LAYOUT_B3, 1, N, K)
-    ws = torch.empty(need, dtype=torch.uint8, device=dev)
+    ws = torch.zeros(need, dtype=torch.uint8, device=dev)  # counters start at zero
     stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
     vp = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
     st = lib.bt_gemv(bt.LAYOUT_B3, vp(codes), vp(scales), vp(x), bt.BF16, vp(sign), 1, N, K, bt.F32, vp(y),
@@ -60,6 +65,39 @@ def test_withheld_copy_times_out_and_the_context_survives():
     assert not int(err.item()) & bt.DEVERR_INVALID_CODE
 
     # the context is still usable: the product library gives the oracle's result
+    _, y_ref, bound = oracle.forward(case["trits"], case["scales"], case["x"], case["sign"])
+    err.zero_()
+    y2 = bt.gemv(codes, scales, x, sign, N, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    assert np.all(np.abs(y2.cpu().numpy().astype(np.float64) - y_ref) <= bound)
+
+
+def test_withheld_stage_of_the_decode_kernel_times_out():
+    dev = torch.device("cuda:0")
+    N, K = 5120, 5120          # single row, K % 1024 == 0: the persistent decode kernel
+    case = workloads.random_case(11100, 1, N, K)
+    codes = bt.pack(torch.from_numpy(case["trits"]).to(dev))
+    scales = torch.from_numpy(case["scales"].view(np.int16)).to(dev)
+    x = torch.from_numpy(case["x"].view(np.int16)).to(dev).view(torch.bfloat16)
+    sign = torch.from_numpy(case["sign"]).to(dev)
+    y = torch.empty((1, N), dtype=torch.float32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    lib = _waittest_lib()
+    need = lib.bt_gemv_workspace_bytes(bt.LAYOUT_B3, 1, N, K)
+    ws = torch.zeros(need, dtype=torch.uint8, device=dev)  # counters start at zero
+    stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    vp = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
+    for _ in range(2):         # the counters are back at zero after a call that timed out
+        err.zero_()
+        st = lib.bt_gemv(bt.LAYOUT_B3, vp(codes), vp(scales), vp(x), bt.BF16, vp(sign), 1, N, K, bt.F32, vp(y),
+                         vp(ws), need, vp(err), stream)
+        assert st == 0
+        torch.cuda.synchronize()
+        assert int(err.item()) & bt.DEVERR_TIMEOUT
+    assert int(ws[:4096].count_nonzero().item()) == 0
+
     _, y_ref, bound = oracle.forward(case["trits"], case["scales"], case["x"], case["sign"])
     err.zero_()
     y2 = bt.gemv(codes, scales, x, sign, N, dev_err=err)
