@@ -649,6 +649,18 @@ def run_case(case: str, reps: int):
             x = torch.from_numpy(inp["x"].view(np.int16)).to(dev).view(torch.bfloat16)
             for _ in range(reps):
                 bt.gemv(codes, sc, x, sign, L.N, layout)
+    elif case.startswith("batched"):
+        # batched[_2bit]: the decode triple in one bt_gemv_batched launch, seeded C1 inputs
+        layout = 1 if case.endswith("2bit") else 0
+        probs = []
+        for i, L in enumerate(workloads.TRIPLE):
+            inp = workloads.layer_inputs("C1", L, index=i)
+            probs.append(dict(codes=bt.pack(torch.from_numpy(inp["trits"]).to(dev), layout),
+                              scales=torch.from_numpy(inp["scales"].view(np.int16)).to(dev),
+                              x=torch.from_numpy(inp["x"].view(np.int16)).to(dev).view(torch.bfloat16),
+                              y=torch.empty((1, L.N), device=dev), N=L.N, K=L.K))
+        for _ in range(reps):
+            bt.gemv_batched(probs, sign, layout)
     elif case.startswith("gemm"):
         # gemm_<layout>: pp512 on the 5120x5120 layer
         layout = 1 if case.endswith("2bit") else 0
@@ -686,7 +698,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-sweep", action="store_true", help="skip the 384-matrix 27B-equivalent sweep")
     ap.add_argument("--case", default=None,
-                    help="run one small workload for a profiler capture (gemv_m<M>[_2bit], gemm[_2bit], fwht)")
+                    help="run one small workload for a profiler capture (gemv_m<M>[_2bit], batched[_2bit], "
+                         "gemm[_2bit], fwht)")
     ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
     if args.case:

@@ -63,6 +63,12 @@ constexpr int kDecFragBytes = 320;            // per group: 10 MMA steps (9 or 8
 constexpr int kDecMetaBytes = 8;              // per group: (corr, 2^e)
 constexpr size_t kDecSyncBytes = 4096;        // counters at the start of the workspace
 constexpr int kDecSyncTicket = 0, kDecSyncExit = 1, kDecSyncRot = 2, kDecSyncDone = 2 + kDecMaxProblems;
+// rotation warp's scratch: the FWHT exchange tile (then the rotated block),
+// the block's fragment words [8 groups][10 steps x 8], the slot table
+constexpr int kDecRotTile = 32 * kTileStride * 4;
+constexpr int kDecRotWords = 8 * 80 * 4;
+constexpr int kDecSlotEntries = 10 * 4 * 4;  // (step, lane, half)
+constexpr int kDecRotBytes = kDecRotTile + kDecRotWords + kDecSlotEntries * 2;
 
 // Bound on every wait, in nanoseconds of the global timer. The test-only
 // build of the library shortens it.
@@ -78,6 +84,7 @@ struct DecProblem {
     int32_t tiles, tile_base, job_base, frag_base;  // frag_base: first group in the workspace
     int32_t dep;          // problem whose output x is (-1: none)
     int32_t x_bf16;
+    int32_t has_dependents;  // a later problem of the launch reads this y: count finished tiles
 };
 
 struct DecParams {
@@ -120,7 +127,7 @@ __host__ __device__ inline DecLayout dec_layout(int layout, int gmax, int stages
     L.team_bytes = t;
     L.team0 = layout == BT_LAYOUT_B3 ? kB3LutBytes : 0;
     L.rot = L.team0 + kDecTeams * t;
-    L.total = L.rot + 32 * kTileStride * 4;
+    L.total = L.rot + kDecRotBytes;
     return L;
 }
 
@@ -222,10 +229,27 @@ __device__ __forceinline__ bool dec_withheld(int team, uint32_t sidx) {
 
 // -------------------------------------------------------- rotation warp ----
 
+// Slot table: entry (t, c, h) = k | field << 8 of the trit that slot carries
+// (k = 0xFF: empty slot). Filled once per CTA.
 template <int LAYOUT>
-__device__ void dec_rotate(const DecParams& P, float* xs, int& bad) {
+__device__ __forceinline__ void dec_slot_table(uint16_t* tab) {
     constexpr int NT = LAYOUT == BT_LAYOUT_B3 ? kB3Mmas : k2bMmas;
+    for (int e = threadIdx.x; e < kDecSlotEntries; e += blockDim.x) {
+        const int t = e >> 4, c = (e >> 2) & 3, h = e & 3;
+        int i = 0, k = -1;
+        if (t < NT) k = LAYOUT == BT_LAYOUT_B3 ? b3_slot(t, c, h, &i) : tb_slot(t, c, h, &i);
+        tab[e] = k < 0 ? uint16_t(0xFF) : static_cast<uint16_t>(k | (i << 8));
+    }
+}
+
+template <int LAYOUT>
+__device__ void dec_rotate(const DecParams& P, uint8_t* scratch, int& bad) {
+    constexpr int NT = LAYOUT == BT_LAYOUT_B3 ? kB3Mmas : k2bMmas;
+    constexpr int WPG = NT * 8;  // fragment words per group: (step, lane c, b0/b1)
     const int lane = threadIdx.x & 31;
+    float* xs = reinterpret_cast<float*>(scratch);
+    uint32_t* words = reinterpret_cast<uint32_t*>(scratch + kDecRotTile);
+    const uint16_t* tab = reinterpret_cast<const uint16_t*>(scratch + kDecRotTile + kDecRotWords);
     // A registers of an all-zero-trit row, for the correction term
     uint32_t Og[16], Oh[16], OQg[3], OQh[3];
     if constexpr (LAYOUT == BT_LAYOUT_B3) b3_ones_tile(lane & 3, Og, Oh, OQg, OQh);
@@ -265,6 +289,7 @@ __device__ void dec_rotate(const DecParams& P, float* xs, int& bad) {
                 v[4 * q] = f.x; v[4 * q + 1] = f.y; v[4 * q + 2] = f.z; v[4 * q + 3] = f.w;
             }
         }
+        __syncwarp();  // the previous job's readers of xs and words are done
         if (P.sign) {
             const uint4* sg = reinterpret_cast<const uint4*>(P.sign + 32 * lane);
             const uint4 s0 = __ldg(sg), s1 = __ldg(sg + 1);
@@ -284,8 +309,10 @@ __device__ void dec_rotate(const DecParams& P, float* xs, int& bad) {
         }
         __syncwarp();
 
+        // per group: e from the largest |x'| (every lane ends with all eight)
+        int eg[8];
+#pragma unroll
         for (int q = 0; q < 8; ++q) {
-            const int gidx = pr.frag_base + 8 * b + q;
             float amax = 0.f;
 #pragma unroll
             for (int r = 0; r < 4; ++r) amax = fmaxf(amax, fabsf(xs[128 * q + 32 * r + lane]));
@@ -293,51 +320,56 @@ __device__ void dec_rotate(const DecParams& P, float* xs, int& bad) {
             for (int s = 16; s > 0; s >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, s));
             int E = amax > 0.f ? ilogbf(amax) + 1 : -100;  // amax < 2^E
             E = max(-100, min(100, E));
-            const int e = 9 + E;
-            const float* xg = xs + 128 * q;
+            eg[q] = 9 + E;
+        }
+        // fragment words of the eight groups, spread over the lanes
+        for (int f = lane; f < 8 * WPG; f += 32) {
+            const int q = f / WPG, widx = f - q * WPG;
+            const int t = widx >> 3, c = (widx >> 1) & 3, hp = widx & 1;
+            int e = eg[0];
+#pragma unroll
+            for (int r = 1; r < 8; ++r) e = q == r ? eg[r] : e;
+            uint32_t word = 0;
+#pragma unroll
+            for (int u = 0; u < 2; ++u) {
+                const uint32_t en = tab[(t * 4 + c) * 4 + 2 * hp + u];
+                const int k = en & 0xFF, i = en >> 8;
+                if (k != 0xFF) {
+                    const __half hv = __float2half_rn(xs[128 * q + k] * exp2i(24 - 2 * i - e));
+                    word |= static_cast<uint32_t>(__half_as_ushort(hv)) << (16 * u);
+                }
+            }
+            words[q * 80 + widx] = word;
+        }
+        __syncwarp();
+        // to the workspace as [group][step pair s][lane c][b0(2s), b1(2s), b0(2s+1), b1(2s+1)]
+        for (int f = lane; f < 8 * 20; f += 32) {
+            const int q = f / 20, r = f - q * 20, s2 = r >> 2, c = r & 3;
+            const int t0 = 2 * s2, t1 = 2 * s2 + 1;
+            const uint32_t* wq = words + q * 80;
+            const uint4 w = make_uint4(t0 < NT ? wq[t0 * 8 + 2 * c] : 0u, t0 < NT ? wq[t0 * 8 + 2 * c + 1] : 0u,
+                                       t1 < NT ? wq[t1 * 8 + 2 * c] : 0u, t1 < NT ? wq[t1 * 8 + 2 * c + 1] : 0u);
+            __stcg(reinterpret_cast<uint4*>(P.frag + (size_t)(pr.frag_base + 8 * b + q) * kDecFragBytes) + 4 * s2 + c, w);
+        }
+        // corr per group: the all-digits-1 tile through the tiles' MMA chain
+#pragma unroll 1
+        for (int q = 0; q < 8; ++q) {
             uint32_t bf[NT][2];
 #pragma unroll
             for (int t = 0; t < NT; ++t) {
-#pragma unroll
-                for (int hp = 0; hp < 2; ++hp) {
-                    uint32_t word = 0;
-                    if (lane < 4) {
-#pragma unroll
-                        for (int u = 0; u < 2; ++u) {
-                            int i = 0;
-                            const int k = LAYOUT == BT_LAYOUT_B3 ? b3_slot(t, lane, 2 * hp + u, &i)
-                                                                 : tb_slot(t, lane, 2 * hp + u, &i);
-                            if (k >= 0) {
-                                const __half hv = __float2half_rn(xg[k] * exp2i(24 - 2 * i - e));
-                                word |= static_cast<uint32_t>(__half_as_ushort(hv)) << (16 * u);
-                            }
-                        }
-                    }
-                    bf[t][hp] = word;  // zero outside lanes 0..3: only column 0 is fed
-                }
-            }
-            if (lane < 4) {
-                // [step pair s][lane c][b0(2s), b1(2s), b0(2s+1), b1(2s+1)]
-                uint4* dst = reinterpret_cast<uint4*>(P.frag + (size_t)gidx * kDecFragBytes) + lane;
-#pragma unroll
-                for (int s = 0; s < 5; ++s) {
-                    const int t0 = 2 * s, t1 = 2 * s + 1;
-                    const uint4 w = make_uint4(t0 < NT ? bf[t0][0] : 0u, t0 < NT ? bf[t0][1] : 0u,
-                                               t1 < NT ? bf[t1][0] : 0u, t1 < NT ? bf[t1][1] : 0u);
-                    __stcg(dst + 4 * s, w);
-                }
+                bf[t][0] = lane < 4 ? words[q * 80 + t * 8 + 2 * lane] : 0u;  // only column 0 is fed
+                bf[t][1] = lane < 4 ? words[q * 80 + t * 8 + 2 * lane + 1] : 0u;
             }
             float d[4];
             if constexpr (LAYOUT == BT_LAYOUT_B3) b3_group_mma(Og, Oh, OQg, OQh, bf, d);
             else tb_group_mma(Og, Oh, bf, d);
-            if (lane == 0) __stcg(P.meta + gidx, make_float2(d[0] * exp2i(e), exp2i(e)));  // D[0][0]
+            if (lane == 0) __stcg(P.meta + pr.frag_base + 8 * b + q, make_float2(d[0] * exp2i(eg[q]), exp2i(eg[q])));
         }
         __syncwarp();
         if (lane == 0) {
             __threadfence();
             atomicAdd(P.sync + kDecSyncRot + p, 1);
         }
-        __syncwarp();
     }
 }
 
@@ -354,9 +386,12 @@ __device__ void dec_produce(const DecParams& P, const DecLayout& L, uint8_t* sme
     int tile = blockIdx.x + team * gridDim.x;  // fixed first ticket: its weights go out before the wait
     bool waited = false, ok = true;
     uint32_t sidx = 0;
-    int k = 0;
+    int k = 0, pending = 0;
     while (ok) {
         const bool end = tile >= P.total_tiles;
+        // the next ticket is requested before this tile's stages go out, so
+        // the atomic's round trip overlaps them
+        if (!end && waited) pending = atomicAdd(P.sync + kDecSyncTicket, 1);
         int p = 0, t = 0, nb = 1;
         if (!end) {
             p = find_problem(P, tile);
@@ -387,8 +422,9 @@ __device__ void dec_produce(const DecParams& P, const DecLayout& L, uint8_t* sme
         if (!waited) {
             pdl_wait();  // the ticket counter belongs to this launch only after the previous one ends
             waited = true;
+            pending = atomicAdd(P.sync + kDecSyncTicket, 1);
         }
-        tile = atomicAdd(P.sync + kDecSyncTicket, 1) + kDecTeams * (int)gridDim.x;
+        tile = pending + kDecTeams * (int)gridDim.x;
     }
     // let every copy still in flight land before the CTA may exit
     const uint32_t first = sidx > (uint32_t)S ? sidx - S : 0u;
@@ -529,7 +565,7 @@ __device__ void dec_consume(const DecParams& P, const DecLayout& L, uint8_t* sme
                 }
             }
             __syncwarp();
-            if (lane == 0) {
+            if (lane == 0 && pr.has_dependents) {
                 __threadfence();
                 atomicAdd(P.sync + kDecSyncDone + p, 1);
             }
@@ -552,6 +588,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
     const DecLayout L = dec_layout(LAYOUT, P.gmax, P.stages, P.stage_bytes);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     if constexpr (LAYOUT == BT_LAYOUT_B3) b3_lut_fill(smem, threadIdx.x, blockDim.x);
+    dec_slot_table<LAYOUT>(reinterpret_cast<uint16_t*>(smem + L.rot + kDecRotTile + kDecRotWords));
     if (threadIdx.x < kDecTeams) {
         const uint32_t tb = smem_addr(smem) + L.team0 + threadIdx.x * L.team_bytes;
         const uint32_t full0 = tb + L.bars, empty0 = full0 + 8 * P.stages;
@@ -573,7 +610,7 @@ __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_con
         if (lane == 0) dec_produce<LAYOUT>(P, L, smem, warp - kDecConsumerWarps, bad);
     } else {
         pdl_wait();
-        dec_rotate<LAYOUT>(P, reinterpret_cast<float*>(smem + L.rot), bad);
+        dec_rotate<LAYOUT>(P, smem + L.rot, bad);
     }
     bad = __reduce_or_sync(0xffffffffu, bad);
     if (lane == 0 && bad) report(P.dev_err, bad);
@@ -682,6 +719,8 @@ static cudaError_t dec_launch_group(int layout, const DecodeProblem* all, int fi
             d.x = s.x_from >= 0 ? all[s.x_from].y : s.x;
             d.x_bf16 = s.x_from >= 0 ? y_bf16 : s.x_bf16;
         }
+        d.has_dependents = 0;
+        if (d.dep >= 0) P.p[d.dep].has_dependents = 1;
         tiles += d.tiles;
         jobs += d.nb;
         groups += d.G;

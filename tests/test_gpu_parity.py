@@ -256,18 +256,19 @@ def test_gemv_bf16_output():
 
 @pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
 @pytest.mark.parametrize("t", [1, -1])
-def test_gemv_special_cases_m1_exact(layout, t):
-    # M = 1 runs the table-lookup kernel. A byte of zero trits has the table
-    # entry 0 exactly and a byte with one non-zero trit the entry +-x'_k
-    # exactly, so all-zero weights give y = 0 exactly and a single trit gives
-    # y[n] = t * fl(s * x'_k), with x' the library's own FP32 rotation
-    # (bt_fwht1024 runs the same warp transform).
-    N, K = 64, 2048
+def test_gemv_special_cases_m1_lut_exact(layout, t):
+    # Single-row calls whose K is beyond the decode kernel's limit run the
+    # table-lookup kernel. A byte of zero trits has the table entry 0 exactly
+    # and a byte with one non-zero trit the entry +-x'_k exactly, so all-zero
+    # weights give y = 0 exactly and a single trit gives y[n] = t * fl(s * x'_k),
+    # with x' the library's own FP32 rotation (bt_fwht1024 runs the same warp
+    # transform).
+    N, K = 64, 28 * 1024
     case = workloads.random_case(5000, 1, N, K)
     case["trits"] = np.zeros_like(case["trits"])
     for checked in (True, False):
         assert np.all(run_gemv(case, layout, checked=checked) == 0.0)
-    n, k = 17, 1500
+    n, k = 17, 21500
     case["trits"][n, k] = t
     xr = bt.fwht1024(T(case["x"], "bf16"), T(case["sign"]), bt.F32).cpu().numpy()
     s = np.float32(case["scales"][n, k // 128].view(np.float16))
@@ -276,6 +277,22 @@ def test_gemv_special_cases_m1_exact(layout, t):
     for checked in (True, False):
         y1 = run_gemv(case, layout, checked=checked)[0].astype(np.float32)
         assert np.array_equal(y1, expect), (y1[n], expect[n])
+
+
+@pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
+def test_gemv_special_cases_m1_decode(layout):
+    # Single-row calls with K % 1024 == 0 up to the limit run the persistent
+    # decode kernel (tensor cores, FP16 activations): zero trits cancel to
+    # exactly 0 through the all-digits-1 correction; a single trit is within
+    # the bound.
+    N, K = 64, 2048
+    case = workloads.random_case(5050, 1, N, K)
+    case["trits"] = np.zeros_like(case["trits"])
+    for checked in (True, False):
+        assert np.all(run_gemv(case, layout, checked=checked) == 0.0)
+    case["trits"][17, 1500] = 1
+    _, y_ref, b = oracle.forward(case["trits"], case["scales"], case["x"], case["sign"])
+    check(run_gemv(case, layout), y_ref, b)
 
 
 @pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
