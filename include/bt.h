@@ -132,10 +132,12 @@ bt_status bt_fwht1024(const uint16_t* x_bf16, const int8_t* sign1024, int64_t M,
  *            check is skipped (it costs one ALU op per byte pair or word).
  *            A copy that does not arrive within a bounded wait sets
  *            BT_DEVERR_TIMEOUT and the affected outputs are unspecified.
- * Kernels: M = 1 with K % 1024 == 0 and 16-byte aligned scales runs the
- * table-lookup kernel (per-call tables of the 5- or 4-trit partial dot
- * products of x', one lookup per packed byte, FP32 throughout) and a kernel
- * that sums its per-512-column partials; other shapes run a prep kernel
+ * Kernels: M = 1 with K % 1024 == 0, K <= bt_gemv_batched_max_k and 16-byte
+ * aligned codes and scales runs the persistent decode kernel of
+ * bt_gemv_batched; M = 1 with a larger K runs the table-lookup kernel
+ * (per-call tables of the 5- or 4-trit partial dot products of x', one
+ * lookup per packed byte, FP32 throughout) and a kernel that sums its
+ * per-512-column partials; other shapes run a prep kernel
  * (rotation, FP16 activation fragments) and an mma.sync kernel (M <= 8 per
  * launch; 9-16 rows take two launches). Consecutive kernels of a call, and
  * of consecutive calls, overlap through programmatic dependent launch: a
@@ -176,9 +178,9 @@ bt_status bt_gemv(int layout, const uint8_t* codes, const uint16_t* scales,
  *             in y_dtype) is this activation; with sign1024 that y must be
  *             bf16 (y_dtype BT_BF16)
  *    y        device [1][N] in y_dtype, 16-byte aligned
- *    N >= 1;  K % 1024 == 0, at most 27648 (base-3) / 39936 (2-bit): one
- *             matrix's activation fragments are held in shared memory
- *             (BT_ERR_UNSUPPORTED beyond)
+ *    N >= 1;  K % 1024 == 0, K <= bt_gemv_batched_max_k(layout) (one
+ *             matrix's activation fragments are held in shared memory;
+ *             BT_ERR_UNSUPPORTED beyond)
  *  sign1024   as for bt_gemv (NULL: every x is already rotated)
  *  workspace  device, >= bt_gemv_batched_workspace_bytes(...), 256-byte
  *             aligned. Its first 4096 bytes are counters: they must be zero
@@ -203,6 +205,9 @@ typedef struct {
     int64_t K;
 } bt_gemv_problem;
 
+/* Largest K bt_gemv_batched takes for a layout (-1 for an unknown layout);
+ * single-row bt_gemv calls with a larger K run the table-lookup kernel. */
+int64_t bt_gemv_batched_max_k(int layout);
 size_t bt_gemv_batched_workspace_bytes(int layout, const bt_gemv_problem* problems, int count);
 bt_status bt_gemv_batched(int layout, const bt_gemv_problem* problems, int count, const int8_t* sign1024,
                           int y_dtype, void* workspace, size_t workspace_bytes, int32_t* dev_err, void* stream);

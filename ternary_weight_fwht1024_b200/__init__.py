@@ -30,7 +30,8 @@ DEVERR_TIMEOUT = 0x8
 # Exported entry points, as declared in include/bt.h.
 SYMBOLS = (
     "bt_status_string", "bt_version", "bt_codes_row_bytes", "bt_pack", "bt_unpack",
-    "bt_fwht1024", "bt_gemv_workspace_bytes", "bt_gemv", "bt_gemv_batched_workspace_bytes", "bt_gemv_batched",
+    "bt_fwht1024", "bt_gemv_workspace_bytes", "bt_gemv", "bt_gemv_batched_max_k", "bt_gemv_batched_workspace_bytes",
+    "bt_gemv_batched",
     "bt_gemv_noalloc", "bt_gemm_workspace_bytes", "bt_gemm",
 )
 
@@ -74,6 +75,8 @@ def load() -> ctypes.CDLL:
             lib.bt_gemv.argtypes = [I, P, P, P, I, P, I64, I64, I64, I, P, P, SZ, P, P]
             lib.bt_gemv_noalloc.argtypes = [I, P, P, P, I, P, I64, I64, I64, I, P, P, P]
             PP = ctypes.POINTER(GemvProblem)
+            lib.bt_gemv_batched_max_k.argtypes = [I]
+            lib.bt_gemv_batched_max_k.restype = I64
             lib.bt_gemv_batched_workspace_bytes.argtypes = [I, PP, I]
             lib.bt_gemv_batched_workspace_bytes.restype = SZ
             lib.bt_gemv_batched.argtypes = [I, PP, I, P, I, P, SZ, P, P]
@@ -212,6 +215,10 @@ def _problem_array(problems):
         arr[i].N = int(p["N"])
         arr[i].K = int(p["K"])
     return arr
+
+
+def gemv_batched_max_k(layout: int) -> int:
+    return int(load().bt_gemv_batched_max_k(layout))
 
 
 def gemv_batched_workspace_bytes(layout: int, problems) -> int:

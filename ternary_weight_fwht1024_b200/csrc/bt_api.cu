@@ -26,6 +26,7 @@ struct DecodeProblem {
 size_t decode_workspace_bytes(const int64_t* Ks, int count);
 bool decode_applies(int64_t M, int64_t K, const void* codes, const void* scales);
 bool decode_k_fits(int layout, int64_t K);
+int64_t decode_max_k(int layout);
 cudaError_t launch_decode(int layout, const DecodeProblem* problems, int count, const int8_t* sign, int y_dtype,
                           void* workspace, int32_t* dev_err, int num_sms, cudaStream_t stream);
 size_t gemm_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num_sms);
@@ -176,6 +177,11 @@ bt_status bt_gemv(int layout, const uint8_t* codes, const uint16_t* scales, cons
     if (!aligned(workspace, 256)) return BT_ERR_ALIGN;
     return from_cuda(run_gemv(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y_dtype, y, workspace,
                               dev_err, sms, s));
+}
+
+int64_t bt_gemv_batched_max_k(int layout) {
+    if (!valid_layout(layout)) return -1;
+    return bt::decode_max_k(layout);
 }
 
 size_t bt_gemv_batched_workspace_bytes(int layout, const bt_gemv_problem* problems, int count) {

@@ -56,7 +56,7 @@ constexpr int kDecConsumerWarps = kDecTeams * kDecTeamWarps;
 constexpr int kDecRotWarp = kDecConsumerWarps + kDecTeams;  // warps 16, 17: producers
 constexpr int kDecWarps = kDecRotWarp + 1;
 constexpr int kDecThreads = kDecWarps * 32;
-constexpr int kDecRows = 16;                  // rows per tile (the MMA's M)
+constexpr int kDecRows = 32;                  // rows per tile: two MMA row blocks of 16
 constexpr int kDecQueue = 32;                 // tile ids per team in flight (more than stages)
 constexpr int kDecMaxStages = 24;
 constexpr int kDecFragBytes = 320;            // per group: 10 MMA steps (9 or 8 used) x 4 lanes x 8 B
@@ -181,25 +181,27 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
                  :: "r"(dst), "l"(src), "r"(bytes), "r"(bar) : "memory");
 }
 
+// Shared-memory loads of data that TMA or bulk copies wrote: volatile, so they
+// stay after the barrier wait (itself volatile, with a memory clobber) that
+// publishes the bytes.
 __device__ __forceinline__ uint32_t lds32(uint32_t a) {
     uint32_t v;
-    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a) : "memory");
+    asm volatile("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(a));
     return v;
 }
 __device__ __forceinline__ uint32_t lds16(uint32_t a) {
     uint16_t v;
-    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a) : "memory");
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(v) : "r"(a));
     return v;
 }
 __device__ __forceinline__ uint2 lds64(uint32_t a) {
     uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a) : "memory");
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
     return v;
 }
 __device__ __forceinline__ uint4 lds128(uint32_t a) {
     uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a)
-                 : "memory");
+    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
     return v;
 }
 
@@ -433,19 +435,29 @@ __device__ void dec_produce(const DecParams& P, const DecLayout& L, uint8_t* sme
 
 // ------------------------------------------------------------- consumers ----
 
+extern __shared__ __align__(1024) uint8_t dec_smem[];
+
+// The decode table sits at the start of the dynamic shared memory.
+struct DecLut {
+    __device__ __forceinline__ static uint32_t ld(uint32_t off) {
+        return *reinterpret_cast<const uint32_t*>(dec_smem + off);
+    }
+};
+
 template <int LAYOUT, bool CHECK>
 __device__ void dec_consume(const DecParams& P, const DecLayout& L, uint8_t* smem, int team, int& bad) {
     constexpr int RB = LAYOUT == BT_LAYOUT_B3 ? 8 * kB3GroupBytes : 8 * k2bGroupBytes;
     constexpr int NT = LAYOUT == BT_LAYOUT_B3 ? kB3Mmas : k2bMmas;
     const int S = P.stages;
+    const uint32_t stage_bytes = static_cast<uint32_t>(P.stage_bytes);
+    const int y_bf16 = P.y_bf16;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int q = warp % kDecTeamWarps;
     const int g = lane >> 2, c = lane & 3;
-    const uint32_t lut = smem_addr(smem);
-    const uint32_t tb = lut + L.team0 + team * L.team_bytes;
+    const uint32_t tb = smem_addr(smem) + L.team0 + team * L.team_bytes;
     const uint32_t full0 = tb + L.bars, empty0 = full0 + 8 * S;
     const uint32_t fbar = empty0 + 8 * S, tbar = fbar + 8;
-    const uint32_t frag = tb + L.frag, meta = tb + L.meta;
+    const uint32_t frag = tb + L.frag, meta = tb + L.meta, ring = tb + L.ring;
     float* red = reinterpret_cast<float*>(smem + L.team0 + team * L.team_bytes + L.red);
     volatile int* tq = reinterpret_cast<volatile int*>(smem + L.team0 + team * L.team_bytes + L.tq);
 
@@ -457,7 +469,8 @@ __device__ void dec_consume(const DecParams& P, const DecLayout& L, uint8_t* sme
                                                 : static_cast<uint32_t>(q * k2bGroupBytes + 8 * c);
     const uint32_t o8 = LAYOUT == BT_LAYOUT_B3 ? (off & 3u) * 8u : 0u;
     const uint32_t a4 = LAYOUT == BT_LAYOUT_B3 ? (off & ~3u) : off;
-    const uint32_t rg_off = static_cast<uint32_t>(g * RB), rh_off = static_cast<uint32_t>((g + 8) * RB);
+    const uint32_t o12 = static_cast<uint32_t>(q * kB3GroupBytes + 24 + (c < 2 ? 0 : 8 * RB));
+    const uint32_t frag_lane = frag + c * 16;
 
     pdl_wait();  // x, y and the counters belong to this launch from here on
 
@@ -471,101 +484,123 @@ __device__ void dec_consume(const DecParams& P, const DecLayout& L, uint8_t* sme
 
     uint32_t err = 0, sidx = 0, fph = 0, tph = 0;
     int k = 0, cur = -1;
+    int nb = 0, N = 0, has_dep = 0, tile_base = 0;
+    void* y = nullptr;
     for (;;) {
         uint32_t slot = sidx % S;
         if (!mbar_wait_t(full0 + 8 * slot, (sidx / S) & 1u)) { bad |= BT_DEVERR_TIMEOUT; break; }
         const int tile = tq[k % kDecQueue];
         if (tile < 0) break;
         const int p = find_problem(P, tile);
-        const DecProblem& pr = P.p[p];
-        const int t = tile - pr.tile_base;
         if (p != cur) {
+            nb = P.p[p].nb;
+            N = P.p[p].N;
+            has_dep = P.p[p].has_dependents;
+            tile_base = P.p[p].tile_base;
+            y = P.p[p].y;
+            const int G = P.p[p].G, frag_base = P.p[p].frag_base;
             // every warp of the team is done with the previous fragments
             if (!team_bar(tph)) { bad |= BT_DEVERR_TIMEOUT; break; }
             if (q == 0 && lane == 0) {
-                if (!poll_at_least(P.sync + kDecSyncRot + p, pr.nb)) bad |= BT_DEVERR_TIMEOUT;
+                if (!poll_at_least(P.sync + kDecSyncRot + p, nb)) bad |= BT_DEVERR_TIMEOUT;
                 asm volatile("fence.proxy.async;" ::: "memory");  // rotation results, read by the copy engine
-                const uint32_t fbytes = pr.G * kDecFragBytes, mbytes = pr.G * kDecMetaBytes;
+                const uint32_t fbytes = G * kDecFragBytes, mbytes = G * kDecMetaBytes;
                 mbar_arrive_tx(fbar, fbytes + mbytes);
-                bulk_g2s(frag, P.frag + (size_t)pr.frag_base * kDecFragBytes, fbytes, fbar);
-                bulk_g2s(meta, P.meta + pr.frag_base, mbytes, fbar);
+                bulk_g2s(frag, P.frag + (size_t)frag_base * kDecFragBytes, fbytes, fbar);
+                bulk_g2s(meta, P.meta + frag_base, mbytes, fbar);
             }
             const bool ok = mbar_wait_t(fbar, fph);
             fph ^= 1u;
             if (!ok) { bad |= BT_DEVERR_TIMEOUT; break; }
             cur = p;
         }
-        float acc_g = 0.f, acc_h = 0.f;
+        const int t = tile - tile_base;
+        // rows g, g + 8 (tt = 0) and 16 + g, 24 + g (tt = 1) of the tile
+        float acc[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
         bool ok = true;
-        for (int b = 0; b < pr.nb; ++b) {
+        for (int b = 0; b < nb; ++b) {
             if (b > 0) {
                 slot = sidx % S;
                 if (!mbar_wait_t(full0 + 8 * slot, (sidx / S) & 1u)) { ok = false; break; }
             }
-            const uint32_t st = tb + L.ring + slot * P.stage_bytes;
+            const uint32_t st = ring + slot * stage_bytes;
             const uint32_t sc = st + kDecRows * RB;
-            const float sg = f16_bits_to_f32(lds16(sc + g * 16 + 2 * q));
-            const float sh = f16_bits_to_f32(lds16(sc + (g + 8) * 16 + 2 * q));
-            uint32_t Rg[16], Rh[16], QG[3], QH[3];
-            if constexpr (LAYOUT == BT_LAYOUT_B3) {
-                const uint32_t w0 = lds32(st + rg_off + a4), w1 = lds32(st + rg_off + a4 + 4);
-                const uint32_t w2 = lds32(st + rh_off + a4), w3 = lds32(st + rh_off + a4 + 4);
-                const uint32_t w12 = lds16(st + (c < 2 ? rg_off : rh_off) + q * kB3GroupBytes + 24);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty0 + 8 * slot);  // the stage may be refilled
-                b3_decode_tile<CHECK>(lut, w0, w1, w2, w3, w12, o8, lane4, mG, mH, Rg, Rh, QG, QH, err);
-            } else {
-                const uint2 x0 = lds64(st + rg_off + a4), x1 = lds64(st + rh_off + a4);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(empty0 + 8 * slot);
-                tb_decode_tile<CHECK>(x0, x1, Rg, Rh, err);
+            float sgv[2], shv[2];
+            uint32_t w[2][5];
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt) {
+                const uint32_t rg = static_cast<uint32_t>((16 * tt + g) * RB), rh = rg + 8 * RB;
+                sgv[tt] = f16_bits_to_f32(lds16(sc + (16 * tt + g) * 16 + 2 * q));
+                shv[tt] = f16_bits_to_f32(lds16(sc + (16 * tt + g + 8) * 16 + 2 * q));
+                if constexpr (LAYOUT == BT_LAYOUT_B3) {
+                    w[tt][0] = lds32(st + rg + a4);
+                    w[tt][1] = lds32(st + rg + a4 + 4);
+                    w[tt][2] = lds32(st + rh + a4);
+                    w[tt][3] = lds32(st + rh + a4 + 4);
+                    w[tt][4] = lds16(st + 16 * tt * RB + g * RB + o12);
+                } else {
+                    const uint2 x0 = lds64(st + rg + a4), x1 = lds64(st + rh + a4);
+                    w[tt][0] = x0.x; w[tt][1] = x0.y; w[tt][2] = x1.x; w[tt][3] = x1.y; w[tt][4] = 0;
+                }
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(empty0 + 8 * slot);  // the stage may be refilled
             ++sidx;
+            // activation fragments of group 8 b + q (column 0: lanes with g == 0)
             const int j = 8 * b + q;
             uint32_t bf[NT][2];
-            {
-                const uint32_t fa = frag + j * kDecFragBytes + c * 16;
 #pragma unroll
-                for (int s = 0; s < (NT + 1) / 2; ++s) {
-                    uint4 w = make_uint4(0u, 0u, 0u, 0u);
-                    if (g == 0) w = lds128(fa + s * 64);
-                    bf[2 * s][0] = w.x;
-                    bf[2 * s][1] = w.y;
-                    if (2 * s + 1 < NT) {
-                        bf[2 * s + 1][0] = w.z;
-                        bf[2 * s + 1][1] = w.w;
-                    }
+            for (int s2 = 0; s2 < (NT + 1) / 2; ++s2) {
+                uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                if (g == 0) v = lds128(frag_lane + j * kDecFragBytes + s2 * 64);
+                bf[2 * s2][0] = v.x;
+                bf[2 * s2][1] = v.y;
+                if (2 * s2 + 1 < NT) {
+                    bf[2 * s2 + 1][0] = v.z;
+                    bf[2 * s2 + 1][1] = v.w;
                 }
             }
             const uint2 md = lds64(meta + j * kDecMetaBytes);
             const float cm = __uint_as_float(md.x), pm = __uint_as_float(md.y);
-            float d[4];
-            if constexpr (LAYOUT == BT_LAYOUT_B3) b3_group_mma(Rg, Rh, QG, QH, bf, d);
-            else tb_group_mma(Rg, Rh, bf, d);
-            acc_g = fmaf(sg, fmaf(d[0], pm, -cm), acc_g);
-            acc_h = fmaf(sh, fmaf(d[2], pm, -cm), acc_h);
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt) {
+                uint32_t Rg[16], Rh[16], QG[3], QH[3];
+                float d[4];
+                if constexpr (LAYOUT == BT_LAYOUT_B3) {
+                    b3_decode_tile<CHECK, DecLut>(w[tt][0], w[tt][1], w[tt][2], w[tt][3], w[tt][4], o8, lane4, mG,
+                                                  mH, Rg, Rh, QG, QH, err);
+                    b3_group_mma(Rg, Rh, QG, QH, bf, d);
+                } else {
+                    tb_decode_tile<CHECK>(make_uint2(w[tt][0], w[tt][1]), make_uint2(w[tt][2], w[tt][3]), Rg, Rh,
+                                          err);
+                    tb_group_mma(Rg, Rh, bf, d);
+                }
+                acc[tt][0] = fmaf(sgv[tt], fmaf(d[0], pm, -cm), acc[tt][0]);
+                acc[tt][1] = fmaf(shv[tt], fmaf(d[2], pm, -cm), acc[tt][1]);
+            }
         }
         if (!ok) { bad |= BT_DEVERR_TIMEOUT; break; }
-        // the tile's 16 rows: partial sums of the 8 warps, added in warp order
+        // the tile's rows: partial sums of the 8 warps, added in warp order
         float* rd = red + (k & 1) * (kDecTeamWarps * kDecRows);
         if (c == 0) {
-            rd[q * kDecRows + g] = acc_g;
-            rd[q * kDecRows + g + 8] = acc_h;
+#pragma unroll
+            for (int tt = 0; tt < 2; ++tt) {
+                rd[q * kDecRows + 16 * tt + g] = acc[tt][0];
+                rd[q * kDecRows + 16 * tt + g + 8] = acc[tt][1];
+            }
         }
         if (!team_bar(tph)) { bad |= BT_DEVERR_TIMEOUT; break; }
         if (q == 0) {
-            if (lane < kDecRows) {
-                float sum = 0.f;
+            float sum = 0.f;
 #pragma unroll
-                for (int w = 0; w < kDecTeamWarps; ++w) sum += rd[w * kDecRows + lane];
-                const int n = t * kDecRows + lane;
-                if (n < pr.N) {
-                    if (P.y_bf16) reinterpret_cast<__nv_bfloat16*>(pr.y)[n] = __float2bfloat16_rn(sum);
-                    else reinterpret_cast<float*>(pr.y)[n] = sum;
-                }
+            for (int w2 = 0; w2 < kDecTeamWarps; ++w2) sum += rd[w2 * kDecRows + lane];
+            const int n = t * kDecRows + lane;
+            if (n < N) {
+                if (y_bf16) reinterpret_cast<__nv_bfloat16*>(y)[n] = __float2bfloat16_rn(sum);
+                else reinterpret_cast<float*>(y)[n] = sum;
             }
             __syncwarp();
-            if (lane == 0 && pr.has_dependents) {
+            if (lane == 0 && has_dep) {
                 __threadfence();
                 atomicAdd(P.sync + kDecSyncDone + p, 1);
             }
@@ -579,8 +614,6 @@ __device__ void dec_consume(const DecParams& P, const DecLayout& L, uint8_t* sme
 }
 
 // -------------------------------------------------------------- kernel ----
-
-extern __shared__ __align__(1024) uint8_t dec_smem[];
 
 template <int LAYOUT, bool CHECK>
 __global__ void __launch_bounds__(kDecThreads, 1) decode_kernel(const __grid_constant__ DecParams P) {
@@ -782,6 +815,14 @@ cudaError_t launch_decode(int layout, const DecodeProblem* problems, int count, 
 
 // Largest K the decode kernel takes: the fragments of one matrix sit in each
 // team's shared memory next to the decode table and at least two stages.
+int64_t decode_max_k(int layout) {
+    const int RB = layout == BT_LAYOUT_B3 ? 8 * kB3GroupBytes : 8 * k2bGroupBytes;
+    int64_t best = 0;
+    for (int G = 8; G <= 4096; G += 8)
+        if ((size_t)dec_layout(layout, G, 2, kDecRows * RB + kDecRows * 16).total <= 227 * 1024) best = (int64_t)G * kGroup;
+    return best;
+}
+
 bool decode_k_fits(int layout, int64_t K) {
     const int G = static_cast<int>(K / kGroup);
     const int RB = layout == BT_LAYOUT_B3 ? 8 * kB3GroupBytes : 8 * k2bGroupBytes;

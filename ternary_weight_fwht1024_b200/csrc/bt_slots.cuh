@@ -97,18 +97,12 @@ __device__ __forceinline__ void b3_lut_fill(uint8_t* lut, int tid, int nthreads)
     }
 }
 
-__device__ __forceinline__ uint32_t lds_lut(uint32_t saddr) {
-    uint32_t v;
-    asm("ld.shared.u32 %0, [%1];" : "=r"(v) : "r"(saddr));
-    return v;
-}
-
 // Decode one row's bytes 6c..6c+5 of a base-3 group (window words W0, W1,
-// shifted right by o8 bits) into 15 registers through the table at shared
-// address `lut` (CHECK: OR the entries into err, whose bit 31 flags codes
-// >= 243).
-template <bool CHECK>
-__device__ __forceinline__ void b3_decode6(uint32_t lut, uint32_t W0, uint32_t W1, uint32_t o8, uint32_t lane4,
+// shifted right by o8 bits) into 15 registers through the decode table; LUT
+// reads the table entry at a byte offset (CHECK: OR the entries into err,
+// whose bit 31 flags codes >= 243).
+template <bool CHECK, class LUT>
+__device__ __forceinline__ void b3_decode6(uint32_t W0, uint32_t W1, uint32_t o8, uint32_t lane4,
                                            uint32_t (&R)[15], uint32_t& err) {
     const uint32_t lo = __funnelshift_r(W0, W1, o8);
     const uint32_t hi = W1 >> o8;
@@ -116,9 +110,9 @@ __device__ __forceinline__ void b3_decode6(uint32_t lut, uint32_t W0, uint32_t W
     for (int q = 0; q < 3; ++q) {
         const uint32_t src = q == 2 ? hi : lo;
         const uint32_t b = q == 1 ? 2u : 0u;
-        // address = code * 256 + lane * 4 (+128 for the high table)
-        const uint32_t va = lds_lut(lut + prmt(src, lane4, 0x5504u | (b << 4)));
-        const uint32_t vb = lds_lut(lut + prmt(src, lane4, 0x5504u | ((b + 1) << 4)) + 128);
+        // offset = code * 256 + lane * 4 (+128 for the high table)
+        const uint32_t va = LUT::ld(prmt(src, lane4, 0x5504u | (b << 4)));
+        const uint32_t vb = LUT::ld(prmt(src, lane4, 0x5504u | ((b + 1) << 4)) + 128);
         if (CHECK) err = lop3_or3(err, va, vb);
 #pragma unroll
         for (int i = 0; i < 5; ++i) R[5 * q + i] = lop3_or_and(va, vb, fmask(i));
@@ -128,21 +122,21 @@ __device__ __forceinline__ void b3_decode6(uint32_t lut, uint32_t W0, uint32_t W
 // A fragments of one 16-row tile for one base-3 group: rows g (words wg0/1,
 // shift o8) and g + 8 (wh0/1), and pair 12 (bytes 24, 25) of row g (c < 2) or
 // g + 8 (c >= 2) in w12. mG / mH: the lane's pair-12 field masks.
-template <bool CHECK>
-__device__ __forceinline__ void b3_decode_tile(uint32_t lut, uint32_t wg0, uint32_t wg1, uint32_t wh0, uint32_t wh1,
+template <bool CHECK, class LUT>
+__device__ __forceinline__ void b3_decode_tile(uint32_t wg0, uint32_t wg1, uint32_t wh0, uint32_t wh1,
                                                uint32_t w12, uint32_t o8, uint32_t lane4, const uint32_t (&mG)[3],
                                                const uint32_t (&mH)[3], uint32_t (&Rg)[16], uint32_t (&Rh)[16],
                                                uint32_t (&QG)[3], uint32_t (&QH)[3], uint32_t& err) {
     uint32_t r15[15];
-    b3_decode6<CHECK>(lut, wg0, wg1, o8, lane4, r15, err);
+    b3_decode6<CHECK, LUT>(wg0, wg1, o8, lane4, r15, err);
 #pragma unroll
     for (int k = 0; k < 15; ++k) Rg[k] = r15[k];
-    b3_decode6<CHECK>(lut, wh0, wh1, o8, lane4, r15, err);
+    b3_decode6<CHECK, LUT>(wh0, wh1, o8, lane4, r15, err);
 #pragma unroll
     for (int k = 0; k < 15; ++k) Rh[k] = r15[k];
     Rg[15] = Rh[15] = 0u;
-    const uint32_t va = lds_lut(lut + prmt(w12, lane4, 0x5504u));
-    const uint32_t vb = lds_lut(lut + prmt(w12, lane4, 0x5514u) + 128);
+    const uint32_t va = LUT::ld(prmt(w12, lane4, 0x5504u));
+    const uint32_t vb = LUT::ld(prmt(w12, lane4, 0x5514u) + 128);
     if (CHECK) err = lop3_or3(err, va, vb);
 #pragma unroll
     for (int k = 0; k < 3; ++k) {

@@ -117,3 +117,29 @@ def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):
         bt.pack(torch.zeros((2, 128), dtype=torch.int8))
+
+
+def test_batched_max_k_and_validation(lib):
+    kb3, k2b = bt.gemv_batched_max_k(bt.LAYOUT_B3), bt.gemv_batched_max_k(bt.LAYOUT_2BIT)
+    assert kb3 >= 17408 and kb3 % 1024 == 0 and k2b >= kb3 and k2b % 1024 == 0
+    assert bt.gemv_batched_max_k(7) == -1
+    good = 1 << 20
+
+    def probs(**kw):
+        arr = (bt.GemvProblem * 2)()
+        for i in range(2):
+            arr[i].codes = arr[i].scales = arr[i].x = arr[i].y = good
+            arr[i].x_dtype, arr[i].x_from, arr[i].N, arr[i].K = 1, -1, 64, 1024
+        for k, v in kw.items():
+            setattr(arr[1], k, v)
+        return arr
+    call = lambda a, sign=None: lib.bt_gemv_batched(0, a, 2, sign, 0, None, 0, None, None)  # noqa: E731
+    assert call(probs()) == 4                       # fine but no workspace
+    assert call(probs(K=1000)) == 2                 # K % 1024
+    assert call(probs(K=kb3 + 1024)) == 5           # beyond the limit
+    assert call(probs(x_from=1)) == 1               # only earlier outputs
+    assert call(probs(x_from=0, K=1024, N=64)) == 2  # problem 0's N (64) is not this K
+    assert call(probs(x_from=-2)) == 1
+    assert call(probs(y=good + 8)) == 3             # alignment
+    assert call(probs(x_dtype=0), _fake(good)) == 1  # rotation reads bf16
+    assert lib.bt_gemv_batched(0, probs(), 0, None, 0, None, 0, None, None) == 0  # nothing to do

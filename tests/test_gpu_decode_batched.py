@@ -179,7 +179,7 @@ def test_batched_chain_f32_prerotated():
 
 # the largest K the kernel takes: one matrix's fragments fill most of a
 # team's shared memory (base-3 also holds the 64 KB decode table)
-K_MAX = {bt.LAYOUT_B3: 27648, bt.LAYOUT_2BIT: 39936}
+K_MAX = {layout: bt.gemv_batched_max_k(layout) for layout in (bt.LAYOUT_B3, bt.LAYOUT_2BIT)}
 
 
 @pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
