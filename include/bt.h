@@ -55,6 +55,8 @@ typedef enum {
 #define BT_DEVERR_INVALID_CODE 0x2   /* base-3 byte >= 243, or 2-bit field == 3    */
 #define BT_DEVERR_INVALID_PAD  0x4   /* bt_unpack: a pad trit of a base-3 group != 0 */
 #define BT_DEVERR_TIMEOUT      0x8   /* a bounded pipeline wait gave up            */
+#define BT_DEVERR_RANGE        0x10  /* single-row kernel: a partial sum was non-finite
+                                        or beyond +-2^27 (outputs unspecified)     */
 
 typedef enum {
     /* Base-3, 5 trits per byte, code = sum_i (t_i + 1) 3^i with trit i at the
@@ -124,31 +126,40 @@ bt_status bt_fwht1024(const uint16_t* x_bf16, const int8_t* sign1024, int64_t M,
  *            rotated, in x_dtype (BT_F32 or BT_BF16), K % 128 == 0.
  *  y         device [M][N] in y_dtype (BT_F32 or BT_BF16), 16-byte aligned
  *  workspace device, >= bt_gemv_workspace_bytes(...), 256-byte aligned.
- *            Scratch only; its contents need no initialisation and are
- *            meaningless after the call.
+ *            Single-row calls that the single-row kernel serves (M = 1,
+ *            K % 1024 == 0, 16-byte aligned codes and scales, N <= 258048)
+ *            keep counters and fixed-point accumulators in it: such a
+ *            workspace must be zero-filled before its first use, and every
+ *            call leaves it zero-filled again. Every other call uses its
+ *            workspace as plain scratch; a buffer that served one must be
+ *            zero-filled again before it serves a single-row call.
  *  dev_err   nullable. When given, the packed codes are validated on the
  *            fly and invalid ones set BT_DEVERR_INVALID_CODE (their
  *            contribution is then unspecified but finite); when NULL the
  *            check is skipped (it costs one ALU op per byte pair or word).
  *            A copy that does not arrive within a bounded wait sets
  *            BT_DEVERR_TIMEOUT and the affected outputs are unspecified.
- * Kernels: M = 1 with K % 1024 == 0, K <= bt_gemv_batched_max_k and 16-byte
- * aligned codes and scales runs the persistent decode kernel of
- * bt_gemv_batched; M = 1 with a larger K runs the table-lookup kernel
- * (per-call tables of the 5- or 4-trit partial dot products of x', one
- * lookup per packed byte, FP32 throughout) and a kernel that sums its
- * per-512-column partials; other shapes run a prep kernel
- * (rotation, FP16 activation fragments) and an mma.sync kernel (M <= 8 per
- * launch; 9-16 rows take two launches). Consecutive kernels of a call, and
- * of consecutive calls, overlap through programmatic dependent launch: a
- * kernel may start reading codes and scales before the preceding kernel in
- * the stream has finished if that kernel allows it, so codes and scales must
- * not be written by a kernel that triggers dependent launch early.
- * Numerics: M = 1: FP32 table entries, scale products and sums. Otherwise
- * the rotated activation feeds FP16 tensor-core products with FP32
- * accumulation (one power-of-two exponent per 128 activations keeps it in
- * range). Either way y satisfies |y - y_exact| <= 2e-3 * sum_k |w x'| + 1e-5,
- * and repeated calls give bit-identical results.
+ * Kernels: single rows that TMA can stream (as above) run the persistent
+ * table-lookup kernel of bt_gemv_batched: per-chunk tables of the 5- or
+ * 4-trit partial dot products of x', one lookup per packed byte, FP32 table
+ * entries and products, chunk partials added in 64-bit fixed point (36
+ * fraction bits) by every CTA that streamed them, one launch per call. Other
+ * shapes run a prep kernel (rotation, FP16 activation fragments) and an
+ * mma.sync kernel (M <= 8 per launch; 9-16 rows take two launches).
+ * Consecutive kernels of a call, and of consecutive calls, overlap through
+ * programmatic dependent launch: a kernel may start reading codes and scales
+ * before the preceding kernel in the stream has finished if that kernel
+ * allows it, so codes and scales must not be written by a kernel that
+ * triggers dependent launch early.
+ * Numerics: single-row kernel: FP32 table entries, scale products and chunk
+ * sums, exact integer addition of the chunk partials, one rounding to the
+ * output; zero trits contribute exactly 0. Otherwise the rotated activation
+ * feeds FP16 tensor-core products with FP32 accumulation (one power-of-two
+ * exponent per 128 activations keeps it in range), and the digit offset is
+ * taken out by the same tensor-core sum of an all-zero-trit row, so zero
+ * trits contribute exactly 0 there too. Either way y satisfies
+ * |y - y_exact| <= 2e-3 * sum_k |w x'| + 1e-5, and repeated calls give
+ * bit-identical results.
  * Source: fused unpack and group scale inside the matrix product, release
  * summary, section 三值权重怎么压缩到 1.76 bit.
  */
@@ -160,14 +171,15 @@ bt_status bt_gemv(int layout, const uint8_t* codes, const uint16_t* scales,
 
 /*
  * bt_gemv_batched: the single-row (M = 1) product y_p = W_p (R x_p) for a list
- * of matrices, in one persistent launch per 12 matrices. A matrix's
- * activation is either given (x, x_dtype) or the output of an earlier matrix
- * of the list (x_from >= 0: the chained layers of a decode step), so a whole
- * token's stack of layers -- or matrices that share nothing -- stream their
- * weights without a gap between them. Each 1024-block of every activation is
- * rotated once. Source: release summary, sections 三值权重怎么压缩到 1.76 bit
- * (R, g128, fused unpack and scale) and 已知短板 (the activation transform
- * is the largest cost outside the product at batch 1).
+ * of matrices, in one persistent launch per 12 matrices (or per 258048 output
+ * rows). A matrix's activation is either given (x, x_dtype) or the output of
+ * an earlier matrix of the list (x_from >= 0: the chained layers of a decode
+ * step), so a whole token's stack of layers -- or matrices that share nothing
+ * -- stream their weights without a gap between them. Every CTA takes an
+ * equal contiguous share of the list's (matrix, 512-column chunk, row) items.
+ * Source: release summary, sections 三值权重怎么压缩到 1.76 bit (R, g128,
+ * fused unpack and scale) and 已知短板 (the activation transform is the
+ * largest cost outside the product at batch 1).
  *  layout     BT_LAYOUT_B3 or BT_LAYOUT_2BIT (one layout per call)
  *  problems   host array of `count` descriptors (1 <= count <= 256):
  *    codes    device [N][bt_codes_row_bytes(layout, K)], 16-byte aligned
@@ -178,21 +190,18 @@ bt_status bt_gemv(int layout, const uint8_t* codes, const uint16_t* scales,
  *             in y_dtype) is this activation; with sign1024 that y must be
  *             bf16 (y_dtype BT_BF16)
  *    y        device [1][N] in y_dtype, 16-byte aligned
- *    N >= 1;  K % 1024 == 0, K <= bt_gemv_batched_max_k(layout) (one
- *             matrix's activation fragments are held in shared memory;
- *             BT_ERR_UNSUPPORTED beyond)
+ *    1 <= N <= 258048; K % 1024 == 0
  *  sign1024   as for bt_gemv (NULL: every x is already rotated)
  *  workspace  device, >= bt_gemv_batched_workspace_bytes(...), 256-byte
- *             aligned. Its first 4096 bytes are counters: they must be zero
- *             before the first call of any GEMV entry point with this
- *             workspace (zero-fill it once when it is allocated); every call
- *             leaves them zero again. The rest is scratch.
+ *             aligned; counters and fixed-point accumulators that must be
+ *             zero-filled before the first call and that every call leaves
+ *             zero-filled again (as for single-row bt_gemv calls; after a
+ *             call that reported BT_DEVERR_TIMEOUT the kernel clears them
+ *             as well).
  *  dev_err    as for bt_gemv; a dependency or copy that does not arrive
  *             within a bounded time sets BT_DEVERR_TIMEOUT.
- * Matrices of more than one launch (count > 12) depend on earlier launches
- * through stream order. Numerics and determinism as for bt_gemv at M > 1:
- * FP16 activations (one power-of-two exponent per 128), FP32 accumulation,
- * zero trits contribute exactly 0, and results do not depend on the schedule.
+ * Matrices of different launches depend on one another through stream order.
+ * Numerics and determinism as for single-row bt_gemv calls.
  */
 typedef struct {
     const uint8_t* codes;
@@ -205,9 +214,6 @@ typedef struct {
     int64_t K;
 } bt_gemv_problem;
 
-/* Largest K bt_gemv_batched takes for a layout (-1 for an unknown layout);
- * single-row bt_gemv calls with a larger K run the table-lookup kernel. */
-int64_t bt_gemv_batched_max_k(int layout);
 size_t bt_gemv_batched_workspace_bytes(int layout, const bt_gemv_problem* problems, int count);
 bt_status bt_gemv_batched(int layout, const bt_gemv_problem* problems, int count, const int8_t* sign1024,
                           int y_dtype, void* workspace, size_t workspace_bytes, int32_t* dev_err, void* stream);
@@ -220,10 +226,14 @@ bt_status bt_gemv_batched(int layout, const bt_gemv_problem* problems, int count
  * before the call). The paper has no counterpart; it is an interface
  * convenience of this library.
  * Arguments and results are those of bt_gemv without the workspace: the
- * scratch is a 4 MiB array in the library's own device memory, reserved on
- * every GPU that loads libbt.so until the process exits. Requests whose
- * bt_gemv_workspace_bytes exceeds 4 MiB (for example M = 16 on 17408-row
- * matrices) are rejected with BT_ERR_WORKSPACE before anything is launched.
+ * scratch is an 8 MiB array in the library's own device memory, reserved on
+ * every GPU that loads libbt.so until the process exits. Its first 2 MiB hold
+ * the single-row kernel's counters and accumulators (zero at load, zero again
+ * after every call); the other 6 MiB are scratch for the other kernels.
+ * Requests needing more than their part (bt_gemv_workspace_bytes beyond
+ * 2 MiB for single rows -- more than about 250000 output rows -- or beyond
+ * 6 MiB otherwise, for example M >= 10 on 17408-row matrices) are rejected
+ * with BT_ERR_WORKSPACE before anything is launched.
  * The first call in a CUDA context looks up the array's device address
  * (for the usual primary context: once per device, with that device
  * current) and caches it for that context; a context created later on the

@@ -12,8 +12,8 @@ size_t gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num
 cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales, const void* x,
                         int x_dtype, const int8_t* sign, int64_t M, int64_t N, int64_t K, int y_dtype,
                         void* y, void* workspace, int32_t* dev_err, int num_sms, cudaStream_t stream);
-size_t gemv_noalloc_max_bytes();
-cudaError_t gemv_noalloc_scratch(void** out);
+size_t gemv_noalloc_max_bytes(bool single_row);
+cudaError_t gemv_noalloc_scratch(bool single_row, void** out);
 struct DecodeProblem {
     const uint8_t* codes;
     const uint16_t* scales;
@@ -23,12 +23,11 @@ struct DecodeProblem {
     void* y;
     int64_t N, K;
 };
-size_t decode_workspace_bytes(const int64_t* Ks, int count);
-bool decode_applies(int64_t M, int64_t K, const void* codes, const void* scales);
-bool decode_k_fits(int layout, int64_t K);
-int64_t decode_max_k(int layout);
-cudaError_t launch_decode(int layout, const DecodeProblem* problems, int count, const int8_t* sign, int y_dtype,
-                          void* workspace, int32_t* dev_err, int num_sms, cudaStream_t stream);
+size_t gemv1_workspace_bytes(const int64_t* Ns, int count);
+bool gemv1_applies(int64_t M, int64_t N, int64_t K, const void* codes, const void* scales);
+int64_t gemv1_max_rows();
+cudaError_t launch_gemv1(int layout, const DecodeProblem* problems, int count, const int8_t* sign, int y_dtype,
+                         void* workspace, int32_t* dev_err, int num_sms, cudaStream_t stream);
 size_t gemm_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num_sms);
 cudaError_t launch_gemm(int layout, const uint8_t* codes, const uint16_t* scales, const void* x,
                         int x_dtype, const int8_t* sign, int64_t M, int64_t N, int64_t K, void* y,
@@ -148,14 +147,14 @@ size_t bt_gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K) {
     return bt::gemv_workspace_bytes(layout, M, N, K, current_sm_count());
 }
 
-// One GEMV call on a validated workspace: single-row calls that fit take the
-// persistent decode kernel, the rest the kernels of bt_gemv.cu.
+// One GEMV call on a validated workspace: single rows that TMA can stream
+// take the persistent table-lookup kernel, the rest the kernels of bt_gemv.cu.
 cudaError_t run_gemv(int layout, const uint8_t* codes, const uint16_t* scales, const void* x, int x_dtype,
                      const int8_t* sign1024, int64_t M, int64_t N, int64_t K, int y_dtype, void* y, void* ws,
                      int32_t* dev_err, int sms, cudaStream_t s) {
-    if (bt::decode_applies(M, K, codes, scales) && bt::decode_k_fits(layout, K)) {
+    if (bt::gemv1_applies(M, N, K, codes, scales)) {
         bt::DecodeProblem p{codes, scales, x, x_dtype == BT_BF16 ? 1 : 0, -1, y, N, K};
-        return bt::launch_decode(layout, &p, 1, sign1024, y_dtype, ws, dev_err, sms, s);
+        return bt::launch_gemv1(layout, &p, 1, sign1024, y_dtype, ws, dev_err, sms, s);
     }
     return bt::launch_gemv(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y_dtype, y, ws, dev_err, sms, s);
 }
@@ -179,17 +178,11 @@ bt_status bt_gemv(int layout, const uint8_t* codes, const uint16_t* scales, cons
                               dev_err, sms, s));
 }
 
-int64_t bt_gemv_batched_max_k(int layout) {
-    if (!valid_layout(layout)) return -1;
-    return bt::decode_max_k(layout);
-}
-
 size_t bt_gemv_batched_workspace_bytes(int layout, const bt_gemv_problem* problems, int count) {
-    if (!valid_layout(layout) || !problems || count < 1) return 0;
-    int64_t Ks[256];
-    if (count > 256) return 0;
-    for (int i = 0; i < count; ++i) Ks[i] = problems[i].K;
-    return bt::decode_workspace_bytes(Ks, count);
+    if (!valid_layout(layout) || !problems || count < 1 || count > 256) return 0;
+    int64_t Ns[256];
+    for (int i = 0; i < count; ++i) Ns[i] = problems[i].N;
+    return bt::gemv1_workspace_bytes(Ns, count);
 }
 
 bt_status bt_gemv_batched(int layout, const bt_gemv_problem* problems, int count, const int8_t* sign1024,
@@ -202,9 +195,8 @@ bt_status bt_gemv_batched(int layout, const bt_gemv_problem* problems, int count
     bt::DecodeProblem dp[256];
     for (int i = 0; i < count; ++i) {
         const bt_gemv_problem& q = problems[i];
-        if (q.N < 1 || q.K < 1024 || q.K % 1024 != 0 || q.K > (int64_t(1) << 30) || q.N > (int64_t(1) << 30))
+        if (q.N < 1 || q.K < 1024 || q.K % 1024 != 0 || q.K > (int64_t(1) << 30) || q.N > bt::gemv1_max_rows())
             return BT_ERR_SHAPE;
-        if (!bt::decode_k_fits(layout, q.K)) return BT_ERR_UNSUPPORTED;
         if (!q.codes || !q.scales || !q.y) return BT_ERR_INVALID_ARG;
         if (!aligned(q.codes, 16) || !aligned(q.scales, 16) || !aligned(q.y, 16)) return BT_ERR_ALIGN;
         if (q.x_from >= 0) {
@@ -224,8 +216,8 @@ bt_status bt_gemv_batched(int layout, const bt_gemv_problem* problems, int count
     const size_t need = bt_gemv_batched_workspace_bytes(layout, problems, count);
     if (!workspace || workspace_bytes < need) return BT_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return BT_ERR_ALIGN;
-    return from_cuda(bt::launch_decode(layout, dp, count, sign1024, y_dtype, workspace, dev_err, current_sm_count(),
-                                       static_cast<cudaStream_t>(stream)));
+    return from_cuda(bt::launch_gemv1(layout, dp, count, sign1024, y_dtype, workspace, dev_err, current_sm_count(),
+                                      static_cast<cudaStream_t>(stream)));
 }
 
 bt_status bt_gemv_noalloc(int layout, const uint8_t* codes, const uint16_t* scales, const void* x,
@@ -240,9 +232,11 @@ bt_status bt_gemv_noalloc(int layout, const uint8_t* codes, const uint16_t* scal
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (K == 0) return from_cuda(launch_zero(y, M * N * (y_dtype == BT_BF16 ? 2 : 4), s));
     const int sms = current_sm_count();
-    if (bt::gemv_workspace_bytes(layout, M, N, K, sms) > bt::gemv_noalloc_max_bytes()) return BT_ERR_WORKSPACE;
+    const bool single = bt::gemv1_applies(M, N, K, codes, scales);
+    const size_t need = single ? bt::gemv1_workspace_bytes(&N, 1) : bt::gemv_workspace_bytes(layout, M, N, K, sms);
+    if (need > bt::gemv_noalloc_max_bytes(single)) return BT_ERR_WORKSPACE;
     void* scratch = nullptr;
-    if (bt::gemv_noalloc_scratch(&scratch) != cudaSuccess) { cudaGetLastError(); return BT_ERR_CUDA; }
+    if (bt::gemv_noalloc_scratch(single, &scratch) != cudaSuccess) { cudaGetLastError(); return BT_ERR_CUDA; }
     return from_cuda(run_gemv(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y_dtype, y, scratch, dev_err,
                               sms, s));
 }

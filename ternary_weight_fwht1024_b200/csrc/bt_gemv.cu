@@ -1088,29 +1088,22 @@ static GemvPlan make_gemv_plan(int layout, int64_t M, int64_t N, int64_t K, int 
     return pl;
 }
 
-// Single-row calls with K a multiple of 512 take the table-lookup kernel
-// (bt_gemv_lut.cu); the workspace covers either path.
-bool gemv_lut_applies(int64_t M, int64_t K, const void* scales);
-size_t gemv_lut_workspace_bytes(int64_t N, int64_t K);
-cudaError_t launch_gemv_lut(int layout, const uint8_t* codes, const uint16_t* scales, const void* x, int x_dtype,
-                            const int8_t* sign, int64_t N, int64_t K, int y_dtype, void* y, void* workspace,
-                            int32_t* dev_err, int num_sms, cudaStream_t stream);
-
-// The first kSyncBytes of every GEMV workspace hold the counters of the
-// single-row decode kernel (bt_decode.cu), which must stay zero between calls;
-// the kernels of this file use the bytes after them.
+// Single rows that TMA can stream take the persistent table-lookup kernel
+// (bt_gemv_lut.cu), whose workspace is a zero-kept accumulator area; the
+// kernels of this file use their workspace as plain scratch after the
+// first kSyncBytes.
 constexpr size_t kSyncBytes = 4096;
-size_t decode_workspace_bytes(const int64_t* Ks, int count);
+bool gemv1_applies(int64_t M, int64_t N, int64_t K, const void* codes, const void* scales);
+size_t gemv1_workspace_bytes(const int64_t* Ns, int count);
 
 size_t gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num_sms) {
-    size_t need = kSyncBytes + make_gemv_plan(layout, M, N, K, num_sms).total;
     if (M == 1 && K % 1024 == 0) {
-        const size_t lut = kSyncBytes + align_up(gemv_lut_workspace_bytes(N, K), 256);
-        if (lut > need) need = lut;
-        const size_t dec = decode_workspace_bytes(&K, 1);
-        if (dec > need) need = dec;
+        // the single-row kernel's need (alignment of the pointers is not known here)
+        const size_t one = gemv1_workspace_bytes(&N, 1);
+        const size_t other = kSyncBytes + make_gemv_plan(layout, M, N, K, num_sms).total;
+        return one > other ? one : other;
     }
-    return need;
+    return kSyncBytes + make_gemv_plan(layout, M, N, K, num_sms).total;
 }
 
 // TMA-fed variant: applies to M <= 8, K % 1024 == 0, 16-byte aligned scales,
@@ -1222,9 +1215,6 @@ cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales
                         void* y, void* workspace, int32_t* dev_err, int num_sms,
                         cudaStream_t stream) {
     uint8_t* ws = static_cast<uint8_t*>(workspace) + kSyncBytes;
-    if (gemv_lut_applies(M, K, scales))
-        return launch_gemv_lut(layout, codes, scales, x, x_dtype, sign, N, K, y_dtype, y, ws, dev_err,
-                               num_sms, stream);
     const GemvPlan pl = make_gemv_plan(layout, M, N, K, num_sms);
 
     PrepArgs pa{};
@@ -1327,8 +1317,14 @@ cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales
 // so it is cached per context (not per device ordinal): a context created
 // later on the same device -- after cudaDeviceReset, or a caller's own
 // non-primary context -- gets its own lookup, never a stale address.
-constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;  // 4 MiB
-static __device__ __align__(256) uint8_t noalloc_scratch[kNoAllocScratchBytes];
+// The first 2 MiB serve the single-row kernel, whose counters and
+// accumulators must start at zero: the array starts zeroed and every
+// single-row call leaves its part zero again. The other 6 MiB are plain
+// scratch for the other kernels, so the two kinds of call never disturb one
+// another.
+constexpr size_t kNoAllocSingleBytes = size_t(2) << 20;  // single-row kernel: zero-kept accumulators
+constexpr size_t kNoAllocOtherBytes = size_t(6) << 20;   // the other kernels: plain scratch
+static __device__ __align__(256) uint8_t noalloc_scratch[kNoAllocSingleBytes + kNoAllocOtherBytes];
 
 constexpr int kMaxContexts = 64;
 static std::mutex g_scratch_mutex;
@@ -1350,9 +1346,9 @@ static CtxGetCurrentFn ctx_get_current() {
     return fn;
 }
 
-size_t gemv_noalloc_max_bytes() { return kNoAllocScratchBytes; }
+size_t gemv_noalloc_max_bytes(bool single_row) { return single_row ? kNoAllocSingleBytes : kNoAllocOtherBytes; }
 
-cudaError_t gemv_noalloc_scratch(void** out) {
+cudaError_t gemv_noalloc_scratch(bool single_row, void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -1362,7 +1358,7 @@ cudaError_t gemv_noalloc_scratch(void** out) {
         std::lock_guard<std::mutex> lock(g_scratch_mutex);
         for (int i = 0; i < g_scratch_used; ++i) {
             if (g_scratch_ctx[i] == ctx) {
-                *out = g_scratch_ptr[i];
+                *out = static_cast<uint8_t*>(g_scratch_ptr[i]) + (single_row ? 0 : kNoAllocSingleBytes);
                 return cudaSuccess;
             }
         }
@@ -1383,7 +1379,7 @@ cudaError_t gemv_noalloc_scratch(void** out) {
             ++g_scratch_used;
         }
     }
-    *out = p;
+    *out = static_cast<uint8_t*>(p) + (single_row ? 0 : kNoAllocSingleBytes);
     return cudaSuccess;
 }
 

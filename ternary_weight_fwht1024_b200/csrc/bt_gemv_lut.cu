@@ -1,53 +1,59 @@
-// Decode GEMV for one activation row (M = 1): y = W x' with x' = R x, by table
-// lookup of packed bytes.
+// Decode GEMV for one activation row (M = 1), by table lookup of packed
+// bytes, over a list of matrices in one persistent launch: y_p = W_p (R x_p).
 //
 // One base-3 byte holds five trits of a row of W (Bonsai low-bit course,
 // section "先用五个数字理解 1.6bit"), a 2-bit byte four. Against a fixed
 // activation vector the contribution of one byte, sum_i t_i x'_(5b+i), depends
-// only on the byte's code, so for every byte position of a K chunk the kernel
-// tabulates that sum for all 256 codes once and then streams the rows: one
-// shared-memory lookup and one FP32 add per byte instead of decoding five
-// trits. (The tables hold partial dot products of the rotated activations,
-// so they are rebuilt per call; W is never decoded.)
+// only on the byte's code, so for every byte position of a 512-wide K chunk
+// the kernel tabulates that sum for all 256 codes once and then streams rows:
+// one shared-memory lookup and one FP32 add per byte instead of decoding five
+// trits. W is never decoded. The release summary of Ternary Bonsai 2 27B
+// (section 三值权重怎么压缩到 1.76 bit) fuses unpack and group scale into the
+// product; section 已知短板 names the activation transform as the largest
+// cost outside the product at batch 1, and decode is bound by weight bytes
+// (section 实测吞吐).
 //
-// Work split. K is cut into 512-wide chunks (four g128 groups: 104 bytes of a
-// base-3 row, 128 of a 2-bit row). Each CTA owns one chunk and an equal slice
-// of the rows (with more chunks than SMs, a CTA walks chunks with all rows).
-// It rotates the 1024-block that holds its chunk (the warp FWHT of the
-// Sylvester H_1024, S applied first, scaled by 1/32; TensorSharp blog,
-// sections 3.2 and 5.2), builds the tables and lets each warp stream its own
-// contiguous rows in sets of 16. Each warp is its own producer: lane 0 moves a
-// set's code bytes ([16 rows][112 B], x rounded down to 16 B so base-3 chunks
-// at 8-byte offsets stay legal) and scales ([16 rows][8 halves]) with two TMA
-// tensor copies into a two-slot ring, completing on the slot's mbarrier. The
-// first sets are requested right after the activation loads, so the rotation
-// and the table build run under their latency.
+// Work. The launch's (matrix, 512-chunk, row) items, in that order, are cut
+// into one contiguous range per CTA (one CTA per SM), so every CTA streams the
+// same number of row chunks. A range is a few segments (matrix p, chunk c,
+// rows n0..n1); per segment the CTA rotates the 1024-block holding the chunk
+// (the warp FWHT of the Sylvester H_1024, S applied first, 1/32; TensorSharp
+// blog, sections 3.2 and 5.2) unless it already holds it, builds the chunk's
+// tables, and its 16 warps stream the rows in sets of 16 (set k to warp
+// k % 16), each warp with its own two-slot TMA ring ([16 rows][112 B] of codes,
+// x rounded down to 16 B, and [16 rows][8 halves] of scales). When matrix p's
+// input is an earlier matrix's output, the segment's weights are requested
+// first and the rotation waits until that output is complete.
+//
+// Reduction. A row's chunk partials come from several CTAs. Each is turned
+// into a 64-bit fixed-point integer (36 fraction bits) and added to the row's
+// accumulator with a fire-and-forget red.add: integer sums do not depend on
+// their order, so the result is deterministic with no second kernel. A
+// finisher warp per CTA counts every finished segment into 256-row completion
+// blocks; the CTA that completes a block converts its rows to y (one rounding
+// to FP32 or bf16), zeroes their accumulators and, when a later matrix reads
+// this output, counts the rows done. The accumulators and counters are thus
+// zero again after every call.
 //
 // Tables. Lane L of a warp reads code word L (bytes 4L..4L+3) of a row chunk,
 // so byte position p = 4L + k is only ever looked up by lane L: its table
 // lives in shared-memory bank L and a warp's 32 lookups never conflict. Two
 // 64 KB regions [256 codes][64 slots] of FP32 hold the 128 tables; byte k of
 // lane L sits in region k/2, slot L + 32 (k % 2). One PRMT turns the code byte
-// and a lane constant into the byte offset code * 256 + slot * 4.
-//
-// Scales multiply per row: a base-3 chunk row has four groups of 26 bytes, so
-// a lane's word lies in one group or (lanes 6 and 19) straddles two; the lane
-// applies s_a to bytes 0-1 and s_b to bytes 2-3 of its word.
-//
-// Each warp keeps one FP32 partial per row of its set in every lane and
-// reduces the 32 x 16 block with a butterfly transpose (16 shuffles); lanes i
-// and i + 16 then hold row i. Partials per (chunk, row) go to the workspace
-// and a second kernel, launched as a programmatic dependent, sums the chunks
-// of each row in chunk order, so results are deterministic and the workspace
-// needs no counters or clearing. (Having the last CTA of a row slice do that
-// sum instead costs more on B200: its atomic arrival and the dependent L2
-// reads are each about a microsecond, and one CTA per slice does the work.)
+// and a lane constant into the byte offset code * 256 + slot * 4. Scales
+// multiply per row: a base-3 chunk row has four groups of 26 bytes, so a
+// lane's word lies in one group or (lanes 6 and 19) straddles two; the lane
+// applies s_a to bytes 0-1 and s_b to bytes 2-3 of its word. Each warp keeps
+// one FP32 partial per row of its set in every lane and reduces the 32 x 16
+// block with a butterfly transpose (16 shuffles); lanes i and i + 16 then hold
+// row i.
 #include "bt_internal.cuh"
 
 namespace bt {
 
-constexpr int kLutWarps = 16;
+constexpr int kLutWarps = 16;                        // streaming warps
 constexpr int kLutThreads = kLutWarps * 32;
+constexpr int kLutAllThreads = kLutThreads + 32;     // + the finisher warp
 constexpr int kLutChunk = 512;                      // k per table set
 constexpr int kLutRegion = 256 * 64 * 4;            // [256 codes][64 slots] f32
 constexpr int kLutTableBytes = 2 * kLutRegion;
@@ -59,28 +65,47 @@ constexpr int kLutCBoxB3 = 112;                      // box bytes per row: 104 +
 constexpr int kLutCBox2b = 128;
 constexpr int kLutSlotMax = kLutSet * kLutCBox2b + kLutSet * 16;  // codes box + scale box (8 halves/row)
 constexpr int kLutTileOffset = kLutXsOffset + 5 * 4 * 32 * 4;   // FWHT exchange tile, 32 x 36 f32
+constexpr int kLutSegSlots = 2;                      // finished segments handed to the finisher
 constexpr int kLutBarOffset = kLutTileOffset + 32 * kTileStride * 4;
-constexpr int kLutRingOffset = kLutBarOffset + kLutWarps * kLutDepth * 8;
+constexpr int kLutSegBarOffset = kLutBarOffset + kLutWarps * kLutDepth * 8;
+constexpr int kLutRingOffset = kLutSegBarOffset + 2 * kLutSegSlots * 8 + 64;
 constexpr int kLutSmem = kLutRingOffset + kLutWarps * kLutDepth * kLutSlotMax;
-constexpr int kLutMinRows = 64;                      // fewest rows worth a table build
 
-struct LutArgs {
-    const uint8_t* codes;
-    const uint16_t* scales;
-    const void* x;
-    const int8_t* sign;  // NULL: x is already rotated
-    float* partials;     // [nchunk][N]
-    int32_t* dev_err;
-    int64_t N;
-    int64_t rows_per_part;  // rows of one CTA's slice (multiple of 16)
-    int parts;              // CTAs per chunk (1: a CTA walks chunks)
-    int K;
-    int G;
-    int RB;  // bytes per row of codes
-    int nchunk;
-    int x_bf16;
+constexpr int kLutMaxProblems = 12;                  // per launch (kernel parameters < 4 KB)
+constexpr int kLutBlockRows = 256;                   // rows per completion block
+constexpr size_t kLutSyncBytes = 4096;               // counters at the start of the workspace
+constexpr int kLutSyncExit = 0, kLutSyncAbort = 1, kLutSyncDone = 2, kLutSyncBlocks = 16;
+constexpr int kLutMaxBlocks = (int)(kLutSyncBytes / 4) - kLutSyncBlocks;  // completion blocks per launch
+constexpr float kLutFix = 68719476736.0f;             // 2^36: the accumulators' fixed-point unit
+constexpr float kLutUnfix = 1.0f / 68719476736.0f;    // 2^-36 (exact)
+
+#ifndef BT_WAIT_NS
+#define BT_WAIT_NS 2000000000ull
+#endif
+constexpr uint64_t kLutWaitNs = BT_WAIT_NS;
+
+struct LutProblem {
+    const void* x;          // [1][K] bf16 or f32 (the output of problem `dep` when dep >= 0)
+    void* y;                // [1][N]
+    int64_t rc_base;        // first (chunk, row) item of this matrix in the launch's order
+    int32_t N, K, G, RB, nchunk, x_bf16;
+    int32_t dep;            // problem whose output x is (-1: none)
+    int32_t has_dependents; // a later problem of the launch reads this y
+    int32_t acc_base;       // first accumulator (row) of this matrix
+    int32_t blk_base;       // first completion block of this matrix
 };
 
+struct LutParams {
+    CUtensorMap cmap[kLutMaxProblems];
+    CUtensorMap smap[kLutMaxProblems];
+    LutProblem p[kLutMaxProblems];
+    const int8_t* sign;                // NULL: x already rotated
+    int32_t* dev_err;
+    int* sync;                         // [exits, rows done per matrix ..., completion blocks ...]
+    unsigned long long* acc;           // fixed-point row sums
+    int64_t total_rc;
+    int nprob, y_bf16;
+};
 
 extern __shared__ __align__(1024) uint8_t lut_smem[];
 
@@ -105,14 +130,6 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
     return v;
 }
 
-struct LutReduceArgs {
-    const float* partials;
-    void* y;
-    int64_t N;
-    int nchunk;
-    int y_bf16;
-};
-
 // Raw words of one lane's 32 bf16 activations of a 1024-block and of its 32
 // sign bytes. Fetched before the first weight copies are requested, so that
 // the rotation does not queue behind them. (FP32 activations are read when
@@ -122,39 +139,40 @@ struct XFetch {
     uint4 sg[2];
 };
 
-__device__ __forceinline__ void lut_fetch_block(const LutArgs& a, int blk, XFetch& f) {
+__device__ __forceinline__ void lut_fetch_block(const void* x, int x_bf16, const int8_t* sign, int blk, XFetch& f) {
     const int lane = threadIdx.x & 31;
-    if (!a.x_bf16) return;
+    if (!x_bf16) return;
+    // L2 reads: x may be the output of an earlier matrix of the same launch
     const uint4* src =
-        reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(a.x) + (size_t)blk * kBlock + 32 * lane);
+        reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + (size_t)blk * kBlock + 32 * lane);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) f.q[q] = __ldg(src + q);
-    if (a.sign) {
-        const uint4* sg = reinterpret_cast<const uint4*>(a.sign + 32 * lane);
+    for (int q = 0; q < 4; ++q) f.q[q] = __ldcg(src + q);
+    if (sign) {
+        const uint4* sg = reinterpret_cast<const uint4*>(sign + 32 * lane);
         f.sg[0] = __ldg(sg);
         f.sg[1] = __ldg(sg + 1);
     }
 }
 
 // The rotated (or, without S, copied) block into xr as FP32. Warp 0 only.
-__device__ __forceinline__ void lut_rotate_block(const LutArgs& a, int blk, const XFetch& f, float* xr,
-                                                 float* tile) {
+__device__ __forceinline__ void lut_rotate_block(const void* x, int x_bf16, const int8_t* sign, int blk,
+                                                 const XFetch& f, float* xr, float* tile) {
     const int lane = threadIdx.x & 31;
     float v[32];
-    if (a.x_bf16) {
+    if (x_bf16) {
         const uint32_t* w = reinterpret_cast<const uint32_t*>(f.q);
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = bf16_bits_to_f32((i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu));
     } else {
-        const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(a.x) + (size_t)blk * kBlock +
+        const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(x) + (size_t)blk * kBlock +
                                                             32 * lane);
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-            const float4 t = __ldg(src + q);
+            const float4 t = __ldcg(src + q);
             v[4 * q] = t.x; v[4 * q + 1] = t.y; v[4 * q + 2] = t.z; v[4 * q + 3] = t.w;
         }
     }
-    if (a.sign) {  // the ABI accepts S with bf16 activations only
+    if (sign) {  // the ABI accepts S with bf16 activations only
         const uint32_t* sw = reinterpret_cast<const uint32_t*>(f.sg);
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
@@ -315,14 +333,88 @@ __device__ __forceinline__ void lut_issue_set(const LutRing& rg, const CUtensorM
     tma_load_2d(dst + kLutSet * rg.cbox, smap, sx, (int)r0, bar);
 }
 
+
+// ------------------------------------------------------------ helpers ----
+
+__device__ __forceinline__ uint64_t lut_ns() {
+    uint64_t t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Wait for the phase of the given parity, bounded in time.
+__device__ __forceinline__ bool lut_wait(uint32_t bar, uint32_t parity) {
+    uint64_t t0 = 0;
+    for (uint32_t i = 0;; ++i) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+        if (ok) return true;
+        if ((i & 63) == 63) {
+            const uint64_t now = lut_ns();
+            if (t0 == 0) t0 = now;
+            else if (now - t0 > kLutWaitNs) return false;
+        }
+    }
+}
+
+// Wait until *p >= target (a counter other CTAs raise), bounded in time.
+__device__ __forceinline__ bool lut_poll(const int* p, int target) {
+    const uint64_t t0 = lut_ns();
+    for (;;) {
+        int v;
+        asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+        if (v >= target) return true;
+        if (lut_ns() - t0 > kLutWaitNs) return false;
+        __nanosleep(128);
+    }
+}
+
+__device__ __forceinline__ void red_add_u64(unsigned long long* p, unsigned long long v) {
+    asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" :: "l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ void fence_acq_rel() {
+    asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
+// barrier of the 16 streaming warps (the finisher warp runs on its own)
+__device__ __forceinline__ void stream_bar() {
+    asm volatile("bar.sync 1, %0;" :: "n"(kLutThreads) : "memory");
+}
+
+// One segment of a CTA's range: matrix p, chunk c, rows [n0, n1).
+struct LutSeg {
+    int p, c, n0, n1;
+};
+
+__device__ __forceinline__ bool lut_next_seg(const LutParams& P, int64_t& rc, int64_t rc1, LutSeg& s) {
+    if (rc >= rc1) return false;
+    int p = 0;
+    while (p + 1 < P.nprob && rc >= P.p[p + 1].rc_base) ++p;
+    const int64_t local = rc - P.p[p].rc_base;
+    const int N = P.p[p].N;
+    s.p = p;
+    s.c = static_cast<int>(local / N);
+    s.n0 = static_cast<int>(local - (int64_t)s.c * N);
+    const int64_t end = (int64_t)s.n0 + (rc1 - rc);
+    s.n1 = static_cast<int>(end < N ? end : N);
+    rc += s.n1 - s.n0;
+    return true;
+}
+
+// ------------------------------------------------------------- kernel ----
+
 template <int LAYOUT, bool CHECK>
-__global__ void __launch_bounds__(kLutThreads, 1)
-gemv_lut_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant__ CUtensorMap smap, const LutArgs a) {
+__device__ void lut_stream(const LutParams& P, int64_t rc0, int64_t rc1, uint32_t segfull, uint32_t segempty,
+                           int& bad) {
     float* table = reinterpret_cast<float*>(lut_smem);
     const uint32_t tab_s = smem_addr(lut_smem);
     float* xr = reinterpret_cast<float*>(lut_smem + kLutXrOffset);
     float* xs = reinterpret_cast<float*>(lut_smem + kLutXsOffset);
-
     const int warp = threadIdx.x >> 5, L = threadIdx.x & 31;
     const int CB = LAYOUT == BT_LAYOUT_B3 ? 4 * kB3GroupBytes : 4 * k2bGroupBytes;  // bytes per chunk row
     const bool lane_on = LAYOUT == BT_LAYOUT_B3 ? L < 26 : true;
@@ -346,72 +438,64 @@ gemv_lut_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant_
     // table slots hold zeros
     const int wlane = LAYOUT == BT_LAYOUT_B3 ? (L < 26 ? L : 25) : L;
 
-    // this CTA's chunks and rows
-    int chunk = a.parts > 1 ? (int)(blockIdx.x / a.parts) : (int)blockIdx.x;
-    const int cstep = a.parts > 1 ? a.nchunk : (int)gridDim.x;
-    const int part = a.parts > 1 ? (int)(blockIdx.x % a.parts) : 0;
-    const int64_t row_lo = (int64_t)part * a.rows_per_part;
-    const int64_t row_hi = min(a.N, row_lo + a.rows_per_part);
-    // each warp streams a contiguous share of the rows, in sets of 16
-    const int64_t share = (((row_hi - row_lo) + kLutWarps * kLutSet - 1) / (kLutWarps * kLutSet)) * kLutSet;
-    const int64_t w_lo = min(row_hi, row_lo + warp * share);
-    const int64_t w_hi = min(row_hi, w_lo + share);
-    const int nsets = (int)((w_hi - w_lo + kLutSet - 1) / kLutSet);
-
-    if (L == 0) {
-        for (int d = 0; d < kLutDepth; ++d) mbar_init(rg.bar + 8 * d, 1);
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncwarp();
+    lut_zero_invalid<LAYOUT>(table);
+    pdl_wait();  // x, y, the accumulators and the counters belong to this launch from here on
 
     uint32_t issued = 0, done = 0;  // sets requested / consumed by this warp
     bool ok = true;
+    int cur_p = -1, cur_blk = -1;
+    uint32_t seg_i = 0;
+    int64_t rc = rc0;
+    LutSeg sg;
+    while (lut_next_seg(P, rc, rc1, sg)) {
+        const LutProblem& pr = P.p[sg.p];
+        const int n0 = sg.n0, n1 = sg.n1;
+        unsigned long long* acc = P.acc + pr.acc_base;
+        const int cb = sg.c * CB;
+        const int cx = cb & ~15, coff = cb - cx;
+        const int sx = (4 * sg.c) & ~7, soff = 2 * (4 * sg.c - sx);
+        const int blk = (sg.c * kLutChunk) / kBlock;
+        const bool new_blk = sg.p != cur_p || blk != cur_blk;
+        const int nsets = (n1 - n0 + kLutSet - 1) / kLutSet;
+        const int my = warp < nsets ? (nsets - warp + kLutWarps - 1) / kLutWarps : 0;  // sets warp, warp + 16, ...
 
-    auto box_x = [&](int c, int& cx, int& sx, int& coff, int& soff) {
-        const int cb = c * CB;
-        cx = cb & ~15;
-        coff = cb - cx;
-        sx = (4 * c) & ~7;
-        soff = 2 * (4 * c - sx);
-    };
-    lut_zero_invalid<LAYOUT>(table);
-    pdl_wait();
-    pdl_launch_dependents();
-
-    uint32_t bad = 0;
-    int cur_blk = -1;
-    for (; chunk < a.nchunk; chunk += cstep) {
-        int cx, sx, coff, soff;
-        box_x(chunk, cx, sx, coff, soff);
-        float* pout = a.partials + (int64_t)chunk * a.N;
-
-        const int blk = (chunk * kLutChunk) / kBlock;
-        const bool new_blk = blk != cur_blk;
         XFetch xf;
-        if (new_blk && warp == 0) lut_fetch_block(a, blk, xf);
-        __syncthreads();  // previous chunk's lookups are done with table / xs
-        // The first sets of this chunk's rows go out after warp 0 has issued
-        // its activation loads, so those loads do not queue behind the
-        // weight stream; the rotation and the table build run under the
-        // copies' latency.
-        if (L == 0 && ok)
-            for (int d = 0; d < kLutDepth && d < nsets; ++d)
-                lut_issue_set(rg, &cmap, &smap, issued + d, cx, sx, w_lo + (int64_t)d * kLutSet);
-        if (ok) issued += min(kLutDepth, nsets);
-        if (new_blk) {
-            if (warp == 0) lut_rotate_block(a, blk, xf, xr, reinterpret_cast<float*>(lut_smem + kLutTileOffset));
-            cur_blk = blk;
-            __syncthreads();
+        if (new_blk && warp == 0) {
+            if (sg.p != cur_p && pr.dep >= 0) {
+                // the input is an earlier matrix's output: wait until all its rows are in
+                int okw = 1;
+                if (L == 0) okw = lut_poll(P.sync + kLutSyncDone + pr.dep, P.p[pr.dep].N) ? 1 : 0;
+                if (!__shfl_sync(0xffffffffu, okw, 0)) bad |= BT_DEVERR_TIMEOUT;
+            }
+            lut_fetch_block(pr.x, pr.x_bf16, P.sign, blk, xf);
         }
-        lut_scatter<LAYOUT>(xr, (chunk * kLutChunk - blk * kBlock) / kLutChunk, xs);
-        __syncthreads();
+        stream_bar();  // the previous segment's lookups are done with table / xs
+        // This segment's first sets go out after warp 0 has issued its
+        // activation loads, so those loads do not queue behind the weight
+        // stream; the rotation and the table build run under the copies'
+        // latency.
+        if (L == 0 && ok)
+            for (int d = 0; d < kLutDepth && d < my; ++d)
+                lut_issue_set(rg, &P.cmap[sg.p], &P.smap[sg.p], issued + d, cx, sx,
+                              n0 + (int64_t)kLutSet * (warp + kLutWarps * d));
+        if (ok) issued += min(kLutDepth, my);
+        if (new_blk) {
+            if (warp == 0)
+                lut_rotate_block(pr.x, pr.x_bf16, P.sign, blk, xf, xr,
+                                 reinterpret_cast<float*>(lut_smem + kLutTileOffset));
+            cur_p = sg.p;
+            cur_blk = blk;
+            stream_bar();
+        }
+        lut_scatter<LAYOUT>(xr, (sg.c * kLutChunk - blk * kBlock) / kLutChunk, xs);
+        stream_bar();
         lut_build<LAYOUT>(xs, table);
-        __syncthreads();
+        stream_bar();
 
-        for (int q = 0; q < nsets && ok; ++q) {
+        for (int q = 0; q < my && ok; ++q) {
             const uint32_t n = done;
             const uint32_t d = n % kLutDepth;
-            if (!mbar_wait(rg.bar + 8 * d, (n / kLutDepth) & 1u)) {
+            if (!lut_wait(rg.bar + 8 * d, (n / kLutDepth) & 1u)) {
                 ok = false;
                 bad |= BT_DEVERR_TIMEOUT;
                 break;
@@ -419,7 +503,7 @@ gemv_lut_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant_
             ++done;
             const uint32_t cslot = rg.ring + d * rg.slot_bytes + coff + 4 * wlane;
             const uint32_t sslot = rg.ring + d * rg.slot_bytes + kLutSet * rg.cbox + soff;
-            float acc[kLutSet];
+            float a16[kLutSet];
 #pragma unroll
             for (int i = 0; i < kLutSet; ++i) {
                 const uint32_t cw = lds_u32(cslot + i * rg.cbox);
@@ -435,73 +519,216 @@ gemv_lut_kernel(const __grid_constant__ CUtensorMap cmap, const __grid_constant_
                 const uint2 q4 = lds_u64(sslot + 16 * i);
                 const uint32_t sp = prmt(q4.x, q4.y, ssel);
                 const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&sp));
-                acc[i] = fmaf(sf.y, e2 + e3, sf.x * (e0 + e1));
+                a16[i] = fmaf(sf.y, e2 + e3, sf.x * (e0 + e1));
             }
-            const int64_t r0 = w_lo + (int64_t)q * kLutSet;
-            const float v = lut_transpose_reduce(acc);  // every value read from the slot is consumed here
+            const int r0 = n0 + kLutSet * (warp + kLutWarps * q);
+            const float v = lut_transpose_reduce(a16);  // every value read from the slot is consumed here
             __syncwarp();
-            if (L == 0 && q + kLutDepth < nsets) {
-                lut_issue_set(rg, &cmap, &smap, issued, cx, sx, r0 + kLutDepth * kLutSet);
+            if (L == 0 && q + kLutDepth < my)
+                lut_issue_set(rg, &P.cmap[sg.p], &P.smap[sg.p], issued, cx, sx,
+                              n0 + (int64_t)kLutSet * (warp + kLutWarps * (q + kLutDepth)));
+            if (q + kLutDepth < my) ++issued;
+            if (L < kLutSet && r0 + L < n1) {
+                // the row's chunk partial, in fixed point (36 fraction bits)
+                if (!(fabsf(v) < 0x1p27f)) bad |= BT_DEVERR_RANGE;
+                const long long f = __float2ll_rn(fminf(fmaxf(v, -0x1p27f), 0x1p27f) * kLutFix);
+                red_add_u64(acc + r0 + L, static_cast<unsigned long long>(f));
             }
-            if (q + kLutDepth < nsets) ++issued;
-            if (L < kLutSet && r0 + L < w_hi) pout[r0 + L] = v;
         }
+        // hand the finished segment to the finisher warp
+        __syncwarp();
+        if (L == 0) {
+            const uint32_t sl = seg_i % kLutSegSlots;
+            if (seg_i >= (uint32_t)kLutSegSlots && !lut_wait(segempty + 8 * sl, ((seg_i / kLutSegSlots) - 1) & 1u))
+                bad |= BT_DEVERR_TIMEOUT;
+            mbar_arrive(segfull + 8 * sl);
+        }
+        ++seg_i;
     }
     // after a timeout: let every copy still in flight land before exiting
     // (each wait is bounded; a set whose wait ran out does not stop the
     // waits on the sets requested after it)
-    for (; done < issued; ++done) mbar_wait(rg.bar + 8 * (done % kLutDepth), (done / kLutDepth) & 1u);
-
-    if (bad) report(a.dev_err, (int)bad);
+    for (; done < issued; ++done) lut_wait(rg.bar + 8 * (done % kLutDepth), (done / kLutDepth) & 1u);
 }
 
-// y[r] = sum over chunks c, in order, of partials[c][r]. A CTA of 8 warps
-// takes 32 rows: warp w sums chunks w, w + 8, ... and the eight warp sums
-// are added in warp order.
-__global__ void __launch_bounds__(256) gemv_lut_reduce_kernel(const LutReduceArgs a) {
-    __shared__ float part[8][33];
+// The finisher warp: counts the CTA's finished segments into the completion
+// blocks and converts every block this CTA completes.
+__device__ void lut_finish(const LutParams& P, int64_t rc0, int64_t rc1, uint32_t segfull, uint32_t segempty,
+                           int& bad) {
+    const int L = threadIdx.x & 31;
     pdl_wait();
-    pdl_launch_dependents();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int64_t r = (int64_t)blockIdx.x * 32 + lane;
-    float s = 0.f;
-    if (r < a.N) {
-#pragma unroll 4
-        for (int c = warp; c < a.nchunk; c += 8) s += a.partials[(int64_t)c * a.N + r];
+    int64_t rc = rc0;
+    LutSeg sg;
+    uint32_t seg_i = 0;
+    while (lut_next_seg(P, rc, rc1, sg)) {
+        const uint32_t sl = seg_i % kLutSegSlots;
+        if (!lut_wait(segfull + 8 * sl, (seg_i / kLutSegSlots) & 1u)) {
+            bad |= BT_DEVERR_TIMEOUT;
+            break;
+        }
+        const LutProblem& pr = P.p[sg.p];
+        const int N = pr.N, nchunk = pr.nchunk;
+        // the streaming warps' adds happened before their arrival; this fence
+        // orders them (cumulatively) before the counts below
+        if (L == 0) fence_acq_rel();
+        __syncwarp();
+        for (int blk = sg.n0 / kLutBlockRows; blk * kLutBlockRows < sg.n1; ++blk) {
+            const int b0 = blk * kLutBlockRows, b1 = min(N, b0 + kLutBlockRows);
+            const int part = min(b1, sg.n1) - max(b0, sg.n0);
+            int* cnt = P.sync + kLutSyncBlocks + pr.blk_base + blk;
+            int last = 0;
+            if (L == 0) {
+                last = atomicAdd(cnt, part) + part == (b1 - b0) * nchunk;
+                if (last) fence_acq_rel();  // every other CTA's adds to these rows are visible
+            }
+            last = __shfl_sync(0xffffffffu, last, 0);
+            if (!last) continue;
+            for (int n = b0 + L; n < b1; n += 32) {
+                const unsigned long long u = atomicExch(P.acc + pr.acc_base + n, 0ull);
+                const float v = __ll2float_rn(static_cast<long long>(u)) * kLutUnfix;
+                if (P.y_bf16) reinterpret_cast<__nv_bfloat16*>(pr.y)[n] = __float2bfloat16_rn(v);
+                else reinterpret_cast<float*>(pr.y)[n] = v;
+            }
+            __syncwarp();
+            if (L == 0) {
+                *cnt = 0;
+                if (pr.has_dependents) {
+                    __threadfence();
+                    atomicAdd(P.sync + kLutSyncDone + sg.p, b1 - b0);
+                }
+            }
+        }
+        __syncwarp();
+        if (L == 0) mbar_arrive(segempty + 8 * sl);
+        ++seg_i;
     }
-    part[warp][lane] = s;
-    __syncthreads();
-    if (warp == 0 && r < a.N) {
-        float t = part[0][lane];
-#pragma unroll
-        for (int w = 1; w < 8; ++w) t += part[w][lane];
-        if (a.y_bf16)
-            reinterpret_cast<__nv_bfloat16*>(a.y)[r] = __float2bfloat16_rn(t);
-        else
-            reinterpret_cast<float*>(a.y)[r] = t;
-    }
-}
-
-// ------------------------------------------------------------------ host ----
-
-bool gemv_lut_applies(int64_t M, int64_t K, const void* scales) {
-    // tensor maps need 16-byte aligned bases (codes already are) and row pitches
-    return M == 1 && K > 0 && K % kBlock == 0 && (reinterpret_cast<uintptr_t>(scales) & 15) == 0;
-}
-
-size_t gemv_lut_workspace_bytes(int64_t N, int64_t K) {
-    return (size_t)(K / kLutChunk) * (size_t)N * sizeof(float);
 }
 
 template <int LAYOUT, bool CHECK>
-static cudaError_t launch_lut_main(const CUtensorMap& cmap, const CUtensorMap& smap, const LutArgs& la, int grid,
-                                   cudaStream_t stream) {
+__global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ LutParams P) {
+    const int warp = threadIdx.x >> 5, L = threadIdx.x & 31;
+    const uint32_t segfull = smem_addr(lut_smem + kLutSegBarOffset);
+    const uint32_t segempty = segfull + 8 * kLutSegSlots;
+    // this CTA's contiguous share of the launch's (matrix, chunk, row) items
+    const int64_t rc0 = P.total_rc * blockIdx.x / gridDim.x;
+    const int64_t rc1 = P.total_rc * (blockIdx.x + 1) / gridDim.x;
+
+    if (warp < kLutWarps && L == 0) {
+        const uint32_t bar = smem_addr(lut_smem + kLutBarOffset) + warp * kLutDepth * 8;
+        for (int d = 0; d < kLutDepth; ++d) mbar_init(bar + 8 * d, 1);
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < kLutSegSlots; ++s) {
+            mbar_init(segfull + 8 * s, kLutWarps);
+            mbar_init(segempty + 8 * s, 1);
+        }
+    }
+    if (L == 0) asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    __syncthreads();
+    pdl_launch_dependents();
+
+    int bad = 0;
+    if (warp < kLutWarps) lut_stream<LAYOUT, CHECK>(P, rc0, rc1, segfull, segempty, bad);
+    else lut_finish(P, rc0, rc1, segfull, segempty, bad);
+    bad = __reduce_or_sync(0xffffffffu, bad);
+    if (L == 0 && bad) report(P.dev_err, bad);
+    __shared__ int s_abort;
+    if (threadIdx.x == 0) s_abort = 0;
+    __syncthreads();
+    if (L == 0 && (bad & BT_DEVERR_TIMEOUT)) atomicOr(&s_abort, 1);
+    __syncthreads();
+
+    // Launch end: the last CTA resets the per-matrix counters. After a wait
+    // that ran out somewhere, it also clears every accumulator and completion
+    // counter of the launch, so the workspace is zero again either way.
+    __shared__ int s_last;
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (s_abort) atomicOr(P.sync + kLutSyncAbort, 1);
+        s_last = atomicAdd(P.sync + kLutSyncExit, 1) == (int)gridDim.x - 1;
+        if (s_last) __threadfence();
+    }
+    __syncthreads();
+    if (s_last) {
+        const bool aborted = *reinterpret_cast<volatile int*>(P.sync + kLutSyncAbort) != 0;
+        if (aborted) {
+            const LutProblem& lp = P.p[P.nprob - 1];
+            const int rows = lp.acc_base + lp.N;
+            const int blocks = lp.blk_base + (lp.N + kLutBlockRows - 1) / kLutBlockRows;
+            for (int i = threadIdx.x; i < rows; i += blockDim.x) P.acc[i] = 0ull;
+            for (int i = threadIdx.x; i < blocks; i += blockDim.x) P.sync[kLutSyncBlocks + i] = 0;
+        }
+        if (threadIdx.x == 0) {
+            for (int i = 0; i < P.nprob; ++i) P.sync[kLutSyncDone + i] = 0;
+            P.sync[kLutSyncAbort] = 0;
+            P.sync[kLutSyncExit] = 0;
+            __threadfence();
+        }
+    }
+}
+
+// ---------------------------------------------------------------- host ----
+
+struct DecodeProblem {
+    const uint8_t* codes;
+    const uint16_t* scales;
+    const void* x;
+    int x_bf16;
+    int x_from;  // -1 or an earlier problem index
+    void* y;
+    int64_t N, K;
+};
+
+static size_t lut_align(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// The launches a list is cut into: at most kLutMaxProblems matrices and
+// kLutMaxBlocks completion blocks each.
+template <class F>
+static void lut_for_each_launch(const int64_t* Ns, int count, F&& f) {
+    int first = 0;
+    while (first < count) {
+        int n = 0, blocks = 0;
+        while (first + n < count && n < kLutMaxProblems) {
+            const int b = (int)((Ns[first + n] + kLutBlockRows - 1) / kLutBlockRows);
+            if (n > 0 && blocks + b > kLutMaxBlocks) break;
+            blocks += b;
+            ++n;
+        }
+        f(first, n);
+        first += n;
+    }
+}
+
+size_t gemv1_workspace_bytes(const int64_t* Ns, int count) {
+    size_t need = kLutSyncBytes;
+    lut_for_each_launch(Ns, count, [&](int first, int n) {
+        size_t rows = 0;
+        for (int i = first; i < first + n; ++i) rows += (size_t)Ns[i];
+        const size_t w = kLutSyncBytes + lut_align(rows * 8, 256);
+        if (w > need) need = w;
+    });
+    return need;
+}
+
+// Single rows whose weights TMA can stream: K a multiple of 1024 (so the
+// scale rows are whole 16-byte units), 16-byte aligned codes and scales, and
+// few enough rows for the completion counters of one launch.
+bool gemv1_applies(int64_t M, int64_t N, int64_t K, const void* codes, const void* scales) {
+    return M == 1 && K > 0 && K % kBlock == 0 && (reinterpret_cast<uintptr_t>(scales) & 15) == 0 &&
+           (reinterpret_cast<uintptr_t>(codes) & 15) == 0 &&
+           (N + kLutBlockRows - 1) / kLutBlockRows <= kLutMaxBlocks;
+}
+
+int64_t gemv1_max_rows() { return (int64_t)kLutMaxBlocks * kLutBlockRows; }
+
+template <int LAYOUT, bool CHECK>
+static cudaError_t lut_launch_t(const LutParams& P, int grid, cudaStream_t stream) {
     auto kern = gemv_lut_kernel<LAYOUT, CHECK>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutSmem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kLutThreads);
+    cfg.blockDim = dim3(kLutAllThreads);
     cfg.dynamicSmemBytes = kLutSmem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -509,87 +736,85 @@ static cudaError_t launch_lut_main(const CUtensorMap& cmap, const CUtensorMap& s
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, kern, cmap, smap, la);
+    return cudaLaunchKernelEx(&cfg, kern, P);
 }
 
-cudaError_t launch_gemv_lut(int layout, const uint8_t* codes, const uint16_t* scales, const void* x, int x_dtype,
-                            const int8_t* sign, int64_t N, int64_t K, int y_dtype, void* y, void* workspace,
-                            int32_t* dev_err, int num_sms, cudaStream_t stream) {
-    if (N <= 0) return cudaSuccess;
-    LutArgs la{};
-    la.codes = codes;
-    la.scales = scales;
-    la.x = x;
-    la.sign = sign;
-    la.partials = static_cast<float*>(workspace);
-    la.dev_err = dev_err;
-    la.N = N;
-    la.K = static_cast<int>(K);
-    la.G = static_cast<int>(K / kGroup);
-    la.RB = static_cast<int>(la.G * (layout == BT_LAYOUT_B3 ? kB3GroupBytes : k2bGroupBytes));
-    la.nchunk = static_cast<int>(K / kLutChunk);
-    la.x_bf16 = x_dtype == BT_BF16;
-    // one chunk per CTA, rows split into `parts` slices; more chunks than
-    // SMs: a CTA per SM walks chunks with all rows
-    int64_t grid;
-    if (la.nchunk <= num_sms) {
-        int64_t parts = num_sms / la.nchunk;
-        const int64_t max_parts = (N + kLutMinRows - 1) / kLutMinRows;
-        if (parts > max_parts) parts = max_parts;
-        if (parts < 1) parts = 1;
-        la.rows_per_part = ((N + parts - 1) / parts + kLutSet - 1) / kLutSet * kLutSet;
-        la.parts = (int)((N + la.rows_per_part - 1) / la.rows_per_part);
-        if (la.parts < 1) la.parts = 1;
-        grid = (int64_t)la.nchunk * la.parts;  // parts == 1: CTA c takes chunk c
-    } else {
-        la.parts = 1;
-        la.rows_per_part = N;
-        grid = num_sms;
-    }
-
+static cudaError_t lut_launch_group(int layout, const DecodeProblem* all, int first, int count, const int8_t* sign,
+                                    int y_bf16, uint8_t* ws, int32_t* dev_err, int num_sms, cudaStream_t stream) {
     EncodeTiledFn enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
-    CUtensorMap cmap, smap;
-    const cuuint64_t cdim[2] = {static_cast<cuuint64_t>(la.RB), static_cast<cuuint64_t>(N)};
-    const cuuint64_t cstr[1] = {static_cast<cuuint64_t>(la.RB)};
-    const cuuint32_t cbox[2] = {static_cast<cuuint32_t>(layout == BT_LAYOUT_B3 ? kLutCBoxB3 : kLutCBox2b), kLutSet};
-    const cuuint64_t sdim[2] = {static_cast<cuuint64_t>(la.G), static_cast<cuuint64_t>(N)};
-    const cuuint64_t sstr[1] = {static_cast<cuuint64_t>(la.G) * 2};
-    const cuuint32_t sbox[2] = {8, kLutSet};
-    const cuuint32_t one[2] = {1, 1};
-    if (enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), cdim, cstr, cbox, one,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
-        enc(&smap, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t*>(scales), sdim, sstr, sbox, one,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-        return cudaErrorInvalidValue;
-
-    cudaError_t e;
+    LutParams P{};
+    const int gbytes = layout == BT_LAYOUT_B3 ? kB3GroupBytes : k2bGroupBytes;
+    int64_t rc = 0;
+    int rows = 0, blocks = 0;
+    for (int i = 0; i < count; ++i) {
+        const DecodeProblem& s = all[first + i];
+        LutProblem& d = P.p[i];
+        d.N = static_cast<int32_t>(s.N);
+        d.K = static_cast<int32_t>(s.K);
+        d.G = static_cast<int32_t>(s.K / kGroup);
+        d.RB = d.G * gbytes;
+        d.nchunk = static_cast<int32_t>(s.K / kLutChunk);
+        d.rc_base = rc;
+        d.acc_base = rows;
+        d.blk_base = blocks;
+        d.y = s.y;
+        d.has_dependents = 0;
+        if (s.x_from >= first) {
+            d.dep = s.x_from - first;
+            d.x = all[s.x_from].y;
+            d.x_bf16 = y_bf16;
+            P.p[d.dep].has_dependents = 1;
+        } else {
+            d.dep = -1;
+            d.x = s.x_from >= 0 ? all[s.x_from].y : s.x;
+            d.x_bf16 = s.x_from >= 0 ? y_bf16 : s.x_bf16;
+        }
+        rc += (int64_t)d.nchunk * d.N;
+        rows += d.N;
+        blocks += (d.N + kLutBlockRows - 1) / kLutBlockRows;
+        const cuuint64_t cdim[2] = {static_cast<cuuint64_t>(d.RB), static_cast<cuuint64_t>(s.N)};
+        const cuuint64_t cstr[1] = {static_cast<cuuint64_t>(d.RB)};
+        const cuuint32_t cbox[2] = {static_cast<cuuint32_t>(layout == BT_LAYOUT_B3 ? kLutCBoxB3 : kLutCBox2b), kLutSet};
+        const cuuint64_t sdim[2] = {static_cast<cuuint64_t>(d.G), static_cast<cuuint64_t>(s.N)};
+        const cuuint64_t sstr[1] = {static_cast<cuuint64_t>(d.G) * 2};
+        const cuuint32_t sbox[2] = {8, kLutSet};
+        const cuuint32_t one[2] = {1, 1};
+        if (enc(&P.cmap[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(s.codes), cdim, cstr, cbox, one,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS ||
+            enc(&P.smap[i], CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<uint16_t*>(s.scales), sdim, sstr, sbox, one,
+                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+            return cudaErrorInvalidValue;
+    }
+    P.sign = sign;
+    P.dev_err = dev_err;
+    P.sync = reinterpret_cast<int*>(ws);
+    P.acc = reinterpret_cast<unsigned long long*>(ws + kLutSyncBytes);
+    P.total_rc = rc;
+    P.nprob = count;
+    P.y_bf16 = y_bf16;
+    // one CTA per SM, never more CTAs than (chunk, row) items
+    const int grid = (int)(rc < num_sms ? rc : num_sms);
     if (layout == BT_LAYOUT_B3)
-        e = dev_err ? launch_lut_main<BT_LAYOUT_B3, true>(cmap, smap, la, (int)grid, stream)
-                    : launch_lut_main<BT_LAYOUT_B3, false>(cmap, smap, la, (int)grid, stream);
-    else
-        e = dev_err ? launch_lut_main<BT_LAYOUT_2BIT, true>(cmap, smap, la, (int)grid, stream)
-                    : launch_lut_main<BT_LAYOUT_2BIT, false>(cmap, smap, la, (int)grid, stream);
-    if (e != cudaSuccess) return e;
+        return dev_err ? lut_launch_t<BT_LAYOUT_B3, true>(P, grid, stream)
+                       : lut_launch_t<BT_LAYOUT_B3, false>(P, grid, stream);
+    return dev_err ? lut_launch_t<BT_LAYOUT_2BIT, true>(P, grid, stream)
+                   : lut_launch_t<BT_LAYOUT_2BIT, false>(P, grid, stream);
+}
 
-    LutReduceArgs ra{};
-    ra.partials = la.partials;
-    ra.y = y;
-    ra.N = N;
-    ra.nchunk = la.nchunk;
-    ra.y_bf16 = y_dtype == BT_BF16;
-    cudaLaunchConfig_t cfg{};
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    attr[0].val.programmaticStreamSerializationAllowed = 1;
-    cfg.attrs = attr;
-    cfg.numAttrs = 1;
-    cfg.gridDim = dim3((unsigned)((N + 31) / 32));
-    cfg.blockDim = dim3(256);
-    return cudaLaunchKernelEx(&cfg, gemv_lut_reduce_kernel, ra);
+cudaError_t launch_gemv1(int layout, const DecodeProblem* problems, int count, const int8_t* sign, int y_dtype,
+                         void* workspace, int32_t* dev_err, int num_sms, cudaStream_t stream) {
+    int64_t Ns[256];
+    for (int i = 0; i < count && i < 256; ++i) Ns[i] = problems[i].N;
+    cudaError_t err = cudaSuccess;
+    lut_for_each_launch(Ns, count, [&](int first, int n) {
+        if (err != cudaSuccess) return;
+        err = lut_launch_group(layout, problems, first, n, sign, y_dtype == BT_BF16,
+                               static_cast<uint8_t*>(workspace), dev_err, num_sms, stream);
+    });
+    return err;
 }
 
 }  // namespace bt

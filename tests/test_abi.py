@@ -119,10 +119,7 @@ def test_binding_refuses_cpu_tensors():
         bt.pack(torch.zeros((2, 128), dtype=torch.int8))
 
 
-def test_batched_max_k_and_validation(lib):
-    kb3, k2b = bt.gemv_batched_max_k(bt.LAYOUT_B3), bt.gemv_batched_max_k(bt.LAYOUT_2BIT)
-    assert kb3 >= 17408 and kb3 % 1024 == 0 and k2b >= kb3 and k2b % 1024 == 0
-    assert bt.gemv_batched_max_k(7) == -1
+def test_batched_validation(lib):
     good = 1 << 20
 
     def probs(**kw):
@@ -136,10 +133,14 @@ def test_batched_max_k_and_validation(lib):
     call = lambda a, sign=None: lib.bt_gemv_batched(0, a, 2, sign, 0, None, 0, None, None)  # noqa: E731
     assert call(probs()) == 4                       # fine but no workspace
     assert call(probs(K=1000)) == 2                 # K % 1024
-    assert call(probs(K=kb3 + 1024)) == 5           # beyond the limit
+    assert call(probs(K=76 * 1024)) == 4            # any K % 1024 == 0
+    assert call(probs(N=258049)) == 2               # beyond the rows of one launch's counters
     assert call(probs(x_from=1)) == 1               # only earlier outputs
     assert call(probs(x_from=0, K=1024, N=64)) == 2  # problem 0's N (64) is not this K
     assert call(probs(x_from=-2)) == 1
     assert call(probs(y=good + 8)) == 3             # alignment
     assert call(probs(x_dtype=0), _fake(good)) == 1  # rotation reads bf16
     assert lib.bt_gemv_batched(0, probs(), 0, None, 0, None, 0, None, None) == 0  # nothing to do
+    arr = probs()
+    need = lib.bt_gemv_batched_workspace_bytes(0, arr, 2)
+    assert need == 4096 + 256 * ((2 * 64 * 8 + 255) // 256)  # counters, then one 64-bit accumulator per row

@@ -177,17 +177,12 @@ def test_batched_chain_f32_prerotated():
         check(y.cpu().numpy().astype(np.float64), y_ref, b)
 
 
-# the largest K the kernel takes: one matrix's fragments fill most of a
-# team's shared memory (base-3 also holds the 64 KB decode table)
-K_MAX = {layout: bt.gemv_batched_max_k(layout) for layout in (bt.LAYOUT_B3, bt.LAYOUT_2BIT)}
-
-
 @pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
-@pytest.mark.parametrize("N,K", [(1, 1024), (17, 2048), (1000, 1024), (77, "max")])
+@pytest.mark.parametrize("N,K", [(1, 1024), (17, 2048), (1000, 1024), (77, 76 * 1024), (300, 3072)])
 def test_batched_ragged_and_edge_shapes(layout, N, K):
-    # one row, a ragged last tile, one 1024-block per row, and the largest K
-    if K == "max":
-        K = K_MAX[layout]
+    # one row, a ragged last set, one 1024-block per row, a long row (152
+    # chunks: more chunks than CTAs, so CTAs cover several chunks) and a
+    # list of one
     case = workloads.random_case(12300 + N + K, 1, N, K)
     codes, sc = _weights(case, layout)
     y = torch.empty((1, N), device=DEV)
@@ -198,18 +193,27 @@ def test_batched_ragged_and_edge_shapes(layout, N, K):
     check(y.cpu().numpy().astype(np.float64), y_ref, b)
 
 
-def test_batched_rejects_k_beyond_the_limit():
-    for layout, kmax in K_MAX.items():
-        probs = [dict(codes=torch.zeros((16, bt.codes_row_bytes(layout, kmax + 1024)), dtype=torch.uint8, device=DEV),
-                      scales=torch.zeros((16, (kmax + 1024) // 128), dtype=torch.int16, device=DEV),
-                      x=torch.zeros((1, kmax + 1024), dtype=torch.bfloat16, device=DEV),
-                      y=torch.empty((1, 16), device=DEV), N=16, K=kmax + 1024)]
-        with pytest.raises(bt.BtError) as e:
-            bt.gemv_batched(probs, None, layout)
-        assert e.value.status == 5  # BT_ERR_UNSUPPORTED, nothing launched
+def test_batched_many_small_matrices_one_launch():
+    # twelve independent matrices of different shapes in one launch: segments
+    # of several matrices share CTAs
+    shapes = [(1024, 64), (2048, 333), (1024, 1), (3072, 1500), (1024, 257), (5120, 100),
+              (2048, 2048), (1024, 16), (4096, 999), (1024, 4000), (2048, 31), (1024, 512)]
+    sign_np = workloads.sign1024()
+    cases, probs = [], []
+    for i, (K, N) in enumerate(shapes):
+        c = workloads.random_case(12500 + i, 1, N, K)
+        codes, sc = _weights(c, bt.LAYOUT_B3)
+        probs.append(dict(codes=codes, scales=sc, x=T(c["x"], "bf16"), y=torch.empty((1, N), device=DEV), N=N, K=K))
+        cases.append(c)
+    ys = bt.gemv_batched(probs, T(sign_np))
+    torch.cuda.synchronize()
+    for c, y in zip(cases, ys):
+        _, y_ref, b = oracle.forward(c["trits"], c["scales"], c["x"], sign_np)
+        check(y.cpu().numpy().astype(np.float64), y_ref, b)
 
 
 def test_batched_zero_weights_exact_and_invalid_codes_flagged():
+    # zero trits: every table entry is an exact 0 and integer sums of zeros stay 0
     K, N = 2048, 64
     case = workloads.random_case(12400, 1, N, K)
     sign = T(case["sign"])

@@ -204,9 +204,9 @@ def test_gemv_prerotated_ragged_groups(layout, N, K):
     check(run_gemv(case, layout, rotate=False, x_f32=xr32), y_ref, b)
 
 
-# Single-row (M = 1) calls with K % 1024 == 0 take the table-lookup kernel:
-# one K chunk of 512 per CTA and row slices, or, with more chunks than SMs,
-# CTAs that walk chunks. These cases cover its branches.
+# Single-row (M = 1) calls with K % 1024 == 0 take the persistent
+# table-lookup kernel: every CTA streams an equal contiguous share of the
+# (chunk, row) items, one or several chunks. These cases cover its branches.
 
 @pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
 @pytest.mark.parametrize("N,K", [(1, 1024), (3, 2048), (17, 1024), (77, 3072), (1000, 17408)])
@@ -232,7 +232,7 @@ def test_gemv_m1_prerotated_bf16(layout):
 
 @pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
 def test_gemv_m1_walks_chunks(layout):
-    # 76 blocks = 152 chunks of 512: more chunks than SMs, so CTAs walk chunks
+    # 76 blocks = 152 chunks of 512: more chunks than SMs, so CTAs cover several chunks
     N, K = 40, 76 * 1024
     case = workloads.random_case(2700, 1, N, K)
     _, y_ref, b = oracle.forward(case["trits"], case["scales"], case["x"], case["sign"])
@@ -256,43 +256,30 @@ def test_gemv_bf16_output():
 
 @pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
 @pytest.mark.parametrize("t", [1, -1])
-def test_gemv_special_cases_m1_lut_exact(layout, t):
-    # Single-row calls whose K is beyond the decode kernel's limit run the
-    # table-lookup kernel. A byte of zero trits has the table entry 0 exactly
-    # and a byte with one non-zero trit the entry +-x'_k exactly, so all-zero
-    # weights give y = 0 exactly and a single trit gives y[n] = t * fl(s * x'_k),
-    # with x' the library's own FP32 rotation (bt_fwht1024 runs the same warp
-    # transform).
-    N, K = 64, 28 * 1024
+@pytest.mark.parametrize("K", [2048, 28 * 1024])
+def test_gemv_special_cases_m1_exact(layout, t, K):
+    # M = 1 runs the table-lookup kernel. A byte of zero trits has the table
+    # entry 0 exactly and a byte with one non-zero trit the entry +-x'_k
+    # exactly, and chunk partials are added as exact integers (2^-36 units),
+    # so all-zero weights give y = 0 exactly and a single trit gives
+    # y[n] = t * fl(s * x'_k) (|s x'_k| >= 2^-13 here, so the fixed-point unit
+    # does not round it), with x' the library's own FP32 rotation
+    # (bt_fwht1024 runs the same warp transform).
+    N = 64
     case = workloads.random_case(5000, 1, N, K)
     case["trits"] = np.zeros_like(case["trits"])
     for checked in (True, False):
         assert np.all(run_gemv(case, layout, checked=checked) == 0.0)
-    n, k = 17, 21500
+    n, k = 17, K - 548
     case["trits"][n, k] = t
     xr = bt.fwht1024(T(case["x"], "bf16"), T(case["sign"]), bt.F32).cpu().numpy()
     s = np.float32(case["scales"][n, k // 128].view(np.float16))
     expect = np.zeros(N, dtype=np.float32)
     expect[n] = np.float32(t) * (s * xr[0, k])
+    assert abs(float(expect[n])) >= 2.0 ** -13
     for checked in (True, False):
         y1 = run_gemv(case, layout, checked=checked)[0].astype(np.float32)
         assert np.array_equal(y1, expect), (y1[n], expect[n])
-
-
-@pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
-def test_gemv_special_cases_m1_decode(layout):
-    # Single-row calls with K % 1024 == 0 up to the limit run the persistent
-    # decode kernel (tensor cores, FP16 activations): zero trits cancel to
-    # exactly 0 through the all-digits-1 correction; a single trit is within
-    # the bound.
-    N, K = 64, 2048
-    case = workloads.random_case(5050, 1, N, K)
-    case["trits"] = np.zeros_like(case["trits"])
-    for checked in (True, False):
-        assert np.all(run_gemv(case, layout, checked=checked) == 0.0)
-    case["trits"][17, 1500] = 1
-    _, y_ref, b = oracle.forward(case["trits"], case["scales"], case["x"], case["sign"])
-    check(run_gemv(case, layout), y_ref, b)
 
 
 @pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])

@@ -4,15 +4,12 @@ Every wait in libbt.so is bounded (a number of tries, or a time on the global
 timer); one that runs out sets BT_DEVERR_TIMEOUT in the caller's error word,
 lets the copies still in flight land and returns, so the context stays
 usable. These tests load the test-only twin of the library
-(libbt_waittest.so), in which one copy is never requested and the bounds are
-short (4096 tries, 20 ms):
-  * the table-lookup GEMV (single row, K beyond the decode kernel's limit):
-    the second set of rows of CTA 0's warp 0;
-  * the persistent decode kernel (single row): the second stage of CTA 0's
-    first team.
-Each test checks that the call returns with the timeout bit set, and that the
-product library still matches the oracle afterwards in the same process.
-Nothing traps, faults or spins without a bound.
+(libbt_waittest.so), in which the single-row kernel never requests one set of
+rows -- the second set of CTA 0's warp 0 -- and every wait gives up after
+20 ms. They check that the call returns with the timeout bit set, that the
+workspace's counters are zero again afterwards, and that the product library
+still matches the oracle in the same process. Nothing traps, faults or spins
+without a bound.
 """
 import ctypes
 
@@ -40,9 +37,8 @@ def _waittest_lib():
 
 def test_withheld_copy_times_out_and_the_context_survives():
     dev = torch.device("cuda:0")
-    # 152 chunks of 512 (more than the SMs): every CTA walks chunks with all
-    # 1000 rows, so warp 0 of CTA 0 streams 64 rows (4 sets) per chunk and
-    # its second set is the one left out
+    # 152 chunks of 512: CTA 0's share starts with 1000 rows of chunk 0, so its
+    # warp 0 streams sets 0, 16, 32 and 48 and the second of them is left out
     N, K = 1000, 76 * 1024
     case = workloads.random_case(11000, 1, N, K)
     codes = bt.pack(torch.from_numpy(case["trits"]).to(dev))
@@ -73,9 +69,9 @@ def test_withheld_copy_times_out_and_the_context_survives():
     assert np.all(np.abs(y2.cpu().numpy().astype(np.float64) - y_ref) <= bound)
 
 
-def test_withheld_stage_of_the_decode_kernel_times_out():
+def test_withheld_copy_twice_leaves_a_clean_workspace():
     dev = torch.device("cuda:0")
-    N, K = 5120, 5120          # single row, K % 1024 == 0: the persistent decode kernel
+    N, K = 5120, 5120          # CTA 0's share: 346 rows of chunk 0, sets 0 and 16 for warp 0
     case = workloads.random_case(11100, 1, N, K)
     codes = bt.pack(torch.from_numpy(case["trits"]).to(dev))
     scales = torch.from_numpy(case["scales"].view(np.int16)).to(dev)
