@@ -54,7 +54,13 @@ bool valid_layout(int layout) { return layout == BT_LAYOUT_B3 || layout == BT_LA
 bool valid_dtype(int d) { return d == BT_F32 || d == BT_BF16; }
 int64_t group_bytes(int layout) { return layout == BT_LAYOUT_B3 ? 26 : 32; }
 
-bt_status from_cuda(cudaError_t e) { return e == cudaSuccess ? BT_OK : BT_ERR_CUDA; }
+// A failed launch also leaves its error as the runtime's last error; clear it,
+// so that a later call does not report it as its own.
+bt_status from_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return BT_OK;
+    cudaGetLastError();
+    return BT_ERR_CUDA;
+}
 
 // Shared validation of the product entry points.
 bt_status check_product_args(int layout, const uint8_t* codes, const uint16_t* scales, const void* x,

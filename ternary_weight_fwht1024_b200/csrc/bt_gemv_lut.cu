@@ -605,7 +605,7 @@ __device__ void lut_finish(const LutParams& P, int64_t rc0, int64_t rc1, uint32_
 }
 
 template <int LAYOUT, bool CHECK>
-__global__ void __maxnreg__(112) gemv_lut_kernel(const __grid_constant__ LutParams P) {
+__global__ void __launch_bounds__(kLutAllThreads, 1) gemv_lut_kernel(const __grid_constant__ LutParams P) {
     const int warp = threadIdx.x >> 5, L = threadIdx.x & 31;
     const uint32_t segfull = smem_addr(lut_smem + kLutSegBarOffset);
     const uint32_t segempty = segfull + 8 * kLutSegSlots;
