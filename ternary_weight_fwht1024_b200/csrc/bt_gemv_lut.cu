@@ -68,8 +68,13 @@ constexpr int kLutTileOffset = kLutXsOffset + 5 * 4 * 32 * 4;   // FWHT exchange
 constexpr int kLutSegSlots = 2;                      // finished segments handed to the finisher
 constexpr int kLutBarOffset = kLutTileOffset + 32 * kTileStride * 4;
 constexpr int kLutSegBarOffset = kLutBarOffset + kLutWarps * kLutDepth * 8;
-constexpr int kLutRingOffset = kLutSegBarOffset + 2 * kLutSegSlots * 8 + 64;
+// TMA writes into the ring: every slot starts on a 128-byte boundary
+constexpr int kLutRingOffset = (kLutSegBarOffset + 2 * kLutSegSlots * 8 + 127) & ~127;
 constexpr int kLutSmem = kLutRingOffset + kLutWarps * kLutDepth * kLutSlotMax;
+static_assert(kLutRingOffset % 128 == 0, "ring slots are TMA destinations");
+static_assert((kLutSet * kLutCBoxB3 + kLutSet * 16) % 128 == 0 && (kLutSet * kLutCBox2b + kLutSet * 16) % 128 == 0 &&
+                  (kLutSet * kLutCBoxB3) % 128 == 0 && (kLutSet * kLutCBox2b) % 128 == 0,
+              "slot sizes and the scale boxes inside them keep 128-byte alignment");
 
 constexpr int kLutMaxProblems = 12;                  // per launch (kernel parameters < 4 KB)
 constexpr int kLutBlockRows = 256;                   // rows per completion block
