@@ -13,7 +13,7 @@
 // cost outside the product at batch 1, and decode is bound by weight bytes
 // (section 实测吞吐).
 //
-// Work. The launch's (matrix, 512-chunk, row) items, in that order, are cut
+// Work. A phase's (matrix, 512-chunk, row) items, in that order, are cut
 // into one contiguous range per CTA (one CTA per SM), so every CTA streams the
 // same number of row chunks. A range is a few segments (matrix p, chunk c,
 // rows n0..n1); per segment the CTA rotates the 1024-block holding the chunk
@@ -28,12 +28,19 @@
 // Reduction. A row's chunk partials come from several CTAs. Each is turned
 // into a 64-bit fixed-point integer (36 fraction bits) and added to the row's
 // accumulator with a fire-and-forget red.add: integer sums do not depend on
-// their order, so the result is deterministic with no second kernel. A
-// finisher warp per CTA counts every finished segment into 256-row completion
-// blocks; the CTA that completes a block converts its rows to y (one rounding
+// their order, so the result is deterministic with no second kernel. At the
+// end of its share of a phase a CTA counts the rows it streamed into 256-row
+// completion blocks (one atomic per block it touched, all in flight at
+// once); the CTA that completes a block converts its rows to y (one rounding
 // to FP32 or bf16), zeroes their accumulators and, when a later matrix reads
 // this output, counts the rows done. The accumulators and counters are thus
 // zero again after every call.
+//
+// Phases. Matrices that do not read one another's outputs form one phase and
+// share the grid as one range; a matrix whose input is an earlier output
+// starts a new phase, which every CTA joins after finishing its share of the
+// previous one (its weights are requested, and it waits for the input, at
+// the start of its first segment).
 //
 // Tables. Lane L of a warp reads code word L (bytes 4L..4L+3) of a row chunk,
 // so byte position p = 4L + k is only ever looked up by lane L: its table
@@ -53,7 +60,6 @@ namespace bt {
 
 constexpr int kLutWarps = 16;                        // streaming warps
 constexpr int kLutThreads = kLutWarps * 32;
-constexpr int kLutAllThreads = kLutThreads + 32;     // + the finisher warp
 constexpr int kLutChunk = 512;                      // k per table set
 constexpr int kLutRegion = 256 * 64 * 4;            // [256 codes][64 slots] f32
 constexpr int kLutTableBytes = 2 * kLutRegion;
@@ -65,11 +71,9 @@ constexpr int kLutCBoxB3 = 112;                      // box bytes per row: 104 +
 constexpr int kLutCBox2b = 128;
 constexpr int kLutSlotMax = kLutSet * kLutCBox2b + kLutSet * 16;  // codes box + scale box (8 halves/row)
 constexpr int kLutTileOffset = kLutXsOffset + 5 * 4 * 32 * 4;   // FWHT exchange tile, 32 x 36 f32
-constexpr int kLutSegSlots = 2;                      // finished segments handed to the finisher
 constexpr int kLutBarOffset = kLutTileOffset + 32 * kTileStride * 4;
-constexpr int kLutSegBarOffset = kLutBarOffset + kLutWarps * kLutDepth * 8;
 // TMA writes into the ring: every slot starts on a 128-byte boundary
-constexpr int kLutRingOffset = (kLutSegBarOffset + 2 * kLutSegSlots * 8 + 127) & ~127;
+constexpr int kLutRingOffset = (kLutBarOffset + kLutWarps * kLutDepth * 8 + 127) & ~127;
 constexpr int kLutSmem = kLutRingOffset + kLutWarps * kLutDepth * kLutSlotMax;
 static_assert(kLutRingOffset % 128 == 0, "ring slots are TMA destinations");
 static_assert((kLutSet * kLutCBoxB3 + kLutSet * 16) % 128 == 0 && (kLutSet * kLutCBox2b + kLutSet * 16) % 128 == 0 &&
@@ -81,6 +85,7 @@ constexpr int kLutBlockRows = 256;                   // rows per completion bloc
 constexpr size_t kLutSyncBytes = 4096;               // counters at the start of the workspace
 constexpr int kLutSyncExit = 0, kLutSyncAbort = 1, kLutSyncDone = 2, kLutSyncBlocks = 16;
 constexpr int kLutMaxBlocks = (int)(kLutSyncBytes / 4) - kLutSyncBlocks;  // completion blocks per launch
+constexpr int kLutMaxLast = 64;                      // blocks a CTA converts per round at a phase end
 constexpr float kLutFix = 68719476736.0f;             // 2^36: the accumulators' fixed-point unit
 constexpr float kLutUnfix = 1.0f / 68719476736.0f;    // 2^-36 (exact)
 
@@ -108,8 +113,8 @@ struct LutParams {
     int32_t* dev_err;
     int* sync;                         // [exits, rows done per matrix ..., completion blocks ...]
     unsigned long long* acc;           // fixed-point row sums
-    int64_t total_rc;
-    int nprob, y_bf16;
+    int64_t phase_rc[kLutMaxProblems + 1];  // first item of every phase, then the launch's item count
+    int nprob, nphase, y_bf16;
 };
 
 extern __shared__ __align__(1024) uint8_t lut_smem[];
@@ -382,15 +387,6 @@ __device__ __forceinline__ void red_add_u64(unsigned long long* p, unsigned long
     asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" :: "l"(p), "l"(v) : "memory");
 }
 
-__device__ __forceinline__ void fence_acq_rel() {
-    asm volatile("fence.acq_rel.gpu;" ::: "memory");
-}
-
-// barrier of the 16 streaming warps (the finisher warp runs on its own)
-__device__ __forceinline__ void stream_bar() {
-    asm volatile("bar.sync 1, %0;" :: "n"(kLutThreads) : "memory");
-}
-
 // One segment of a CTA's range: matrix p, chunk c, rows [n0, n1).
 struct LutSeg {
     int p, c, n0, n1;
@@ -414,12 +410,13 @@ __device__ __forceinline__ bool lut_next_seg(const LutParams& P, int64_t& rc, in
 // ------------------------------------------------------------- kernel ----
 
 template <int LAYOUT, bool CHECK>
-__device__ void lut_stream(const LutParams& P, int64_t rc0, int64_t rc1, uint32_t segfull, uint32_t segempty,
-                           int& bad) {
+__global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_constant__ LutParams P) {
     float* table = reinterpret_cast<float*>(lut_smem);
     const uint32_t tab_s = smem_addr(lut_smem);
     float* xr = reinterpret_cast<float*>(lut_smem + kLutXrOffset);
     float* xs = reinterpret_cast<float*>(lut_smem + kLutXsOffset);
+    __shared__ int s_last[kLutMaxLast];   // blocks this CTA completed: (matrix << 20) | block
+    __shared__ int s_nlast, s_flag;
     const int warp = threadIdx.x >> 5, L = threadIdx.x & 31;
     const int CB = LAYOUT == BT_LAYOUT_B3 ? 4 * kB3GroupBytes : 4 * k2bGroupBytes;  // bytes per chunk row
     const bool lane_on = LAYOUT == BT_LAYOUT_B3 ? L < 26 : true;
@@ -443,218 +440,189 @@ __device__ void lut_stream(const LutParams& P, int64_t rc0, int64_t rc1, uint32_
     // table slots hold zeros
     const int wlane = LAYOUT == BT_LAYOUT_B3 ? (L < 26 ? L : 25) : L;
 
+    if (L == 0) {
+        for (int d = 0; d < kLutDepth; ++d) mbar_init(rg.bar + 8 * d, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+    pdl_launch_dependents();
     lut_zero_invalid<LAYOUT>(table);
     pdl_wait();  // x, y, the accumulators and the counters belong to this launch from here on
 
+    int bad = 0;
     uint32_t issued = 0, done = 0;  // sets requested / consumed by this warp
     bool ok = true;
     int cur_p = -1, cur_blk = -1;
-    uint32_t seg_i = 0;
-    int64_t rc = rc0;
-    LutSeg sg;
-    while (lut_next_seg(P, rc, rc1, sg)) {
-        const LutProblem& pr = P.p[sg.p];
-        const int n0 = sg.n0, n1 = sg.n1;
-        unsigned long long* acc = P.acc + pr.acc_base;
-        const int cb = sg.c * CB;
-        const int cx = cb & ~15, coff = cb - cx;
-        const int sx = (4 * sg.c) & ~7, soff = 2 * (4 * sg.c - sx);
-        const int blk = (sg.c * kLutChunk) / kBlock;
-        const bool new_blk = sg.p != cur_p || blk != cur_blk;
-        const int nsets = (n1 - n0 + kLutSet - 1) / kLutSet;
-        const int my = warp < nsets ? (nsets - warp + kLutWarps - 1) / kLutWarps : 0;  // sets warp, warp + 16, ...
+    for (int ph = 0; ph < P.nphase; ++ph) {
+        // this CTA's contiguous share of the phase's (matrix, chunk, row) items
+        const int64_t base = P.phase_rc[ph], span = P.phase_rc[ph + 1] - base;
+        const int64_t rc0 = base + span * blockIdx.x / gridDim.x;
+        const int64_t rc1 = base + span * (blockIdx.x + 1) / gridDim.x;
+        int64_t rc = rc0;
+        LutSeg sg;
+        while (lut_next_seg(P, rc, rc1, sg)) {
+            const LutProblem& pr = P.p[sg.p];
+            const int n0 = sg.n0, n1 = sg.n1;
+            unsigned long long* acc = P.acc + pr.acc_base;
+            const int cb = sg.c * CB;
+            const int cx = cb & ~15, coff = cb - cx;
+            const int sx = (4 * sg.c) & ~7, soff = 2 * (4 * sg.c - sx);
+            const int blk = (sg.c * kLutChunk) / kBlock;
+            const bool new_blk = sg.p != cur_p || blk != cur_blk;
+            const int nsets = (n1 - n0 + kLutSet - 1) / kLutSet;
+            const int my = warp < nsets ? (nsets - warp + kLutWarps - 1) / kLutWarps : 0;  // sets warp, warp + 16, ...
 
-        XFetch xf;
-        if (new_blk && warp == 0) {
-            if (sg.p != cur_p && pr.dep >= 0) {
-                // the input is an earlier matrix's output: wait until all its rows are in
-                int okw = 1;
-                if (L == 0) okw = lut_poll(P.sync + kLutSyncDone + pr.dep, P.p[pr.dep].N) ? 1 : 0;
-                if (!__shfl_sync(0xffffffffu, okw, 0)) bad |= BT_DEVERR_TIMEOUT;
+            XFetch xf;
+            if (new_blk && warp == 0) {
+                if (sg.p != cur_p && pr.dep >= 0) {
+                    // the input is an earlier matrix's output: wait until all its rows are in
+                    int okw = 1;
+                    if (L == 0) okw = lut_poll(P.sync + kLutSyncDone + pr.dep, P.p[pr.dep].N) ? 1 : 0;
+                    if (!__shfl_sync(0xffffffffu, okw, 0)) bad |= BT_DEVERR_TIMEOUT;
+                }
+                lut_fetch_block(pr.x, pr.x_bf16, P.sign, blk, xf);
             }
-            lut_fetch_block(pr.x, pr.x_bf16, P.sign, blk, xf);
-        }
-        stream_bar();  // the previous segment's lookups are done with table / xs
-        // This segment's first sets go out after warp 0 has issued its
-        // activation loads, so those loads do not queue behind the weight
-        // stream; the rotation and the table build run under the copies'
-        // latency.
-        if (L == 0 && ok)
-            for (int d = 0; d < kLutDepth && d < my; ++d)
-                lut_issue_set(rg, &P.cmap[sg.p], &P.smap[sg.p], issued + d, cx, sx,
-                              n0 + (int64_t)kLutSet * (warp + kLutWarps * d));
-        if (ok) issued += min(kLutDepth, my);
-        if (new_blk) {
-            if (warp == 0)
-                lut_rotate_block(pr.x, pr.x_bf16, P.sign, blk, xf, xr,
-                                 reinterpret_cast<float*>(lut_smem + kLutTileOffset));
-            cur_p = sg.p;
-            cur_blk = blk;
-            stream_bar();
-        }
-        lut_scatter<LAYOUT>(xr, (sg.c * kLutChunk - blk * kBlock) / kLutChunk, xs);
-        stream_bar();
-        lut_build<LAYOUT>(xs, table);
-        stream_bar();
+            __syncthreads();  // the previous segment's lookups are done with table / xs
+            // This segment's first sets go out after warp 0 has issued its
+            // activation loads, so those loads do not queue behind the weight
+            // stream; the rotation and the table build run under the copies'
+            // latency.
+            if (L == 0 && ok)
+                for (int d = 0; d < kLutDepth && d < my; ++d)
+                    lut_issue_set(rg, &P.cmap[sg.p], &P.smap[sg.p], issued + d, cx, sx,
+                                  n0 + (int64_t)kLutSet * (warp + kLutWarps * d));
+            if (ok) issued += min(kLutDepth, my);
+            if (new_blk) {
+                if (warp == 0)
+                    lut_rotate_block(pr.x, pr.x_bf16, P.sign, blk, xf, xr,
+                                     reinterpret_cast<float*>(lut_smem + kLutTileOffset));
+                cur_p = sg.p;
+                cur_blk = blk;
+                __syncthreads();
+            }
+            lut_scatter<LAYOUT>(xr, (sg.c * kLutChunk - blk * kBlock) / kLutChunk, xs);
+            __syncthreads();
+            lut_build<LAYOUT>(xs, table);
+            __syncthreads();
 
-        for (int q = 0; q < my && ok; ++q) {
-            const uint32_t n = done;
-            const uint32_t d = n % kLutDepth;
-            if (!lut_wait(rg.bar + 8 * d, (n / kLutDepth) & 1u)) {
-                ok = false;
-                bad |= BT_DEVERR_TIMEOUT;
-                break;
-            }
-            ++done;
-            const uint32_t cslot = rg.ring + d * rg.slot_bytes + coff + 4 * wlane;
-            const uint32_t sslot = rg.ring + d * rg.slot_bytes + kLutSet * rg.cbox + soff;
-            float a16[kLutSet];
+            for (int q = 0; q < my && ok; ++q) {
+                const uint32_t n = done;
+                const uint32_t d = n % kLutDepth;
+                if (!lut_wait(rg.bar + 8 * d, (n / kLutDepth) & 1u)) {
+                    ok = false;
+                    bad |= BT_DEVERR_TIMEOUT;
+                    break;
+                }
+                ++done;
+                const uint32_t cslot = rg.ring + d * rg.slot_bytes + coff + 4 * wlane;
+                const uint32_t sslot = rg.ring + d * rg.slot_bytes + kLutSet * rg.cbox + soff;
+                float a16[kLutSet];
 #pragma unroll
-            for (int i = 0; i < kLutSet; ++i) {
-                const uint32_t cw = lds_u32(cslot + i * rg.cbox);
-                if (CHECK && lane_on) bad |= lut_check<LAYOUT>(cw);
-                const uint32_t o0 = prmt(cw, lanebytes, 0x6604u);
-                const uint32_t o1 = prmt(cw, lanebytes, 0x6615u);
-                const uint32_t o2 = prmt(cw, lanebytes, 0x6624u);
-                const uint32_t o3 = prmt(cw, lanebytes, 0x6635u);
-                const float e0 = lds_f32(tab_s + o0);
-                const float e1 = lds_f32(tab_s + o1);
-                const float e2 = lds_f32(tab_s + kLutRegion + o2);
-                const float e3 = lds_f32(tab_s + kLutRegion + o3);
-                const uint2 q4 = lds_u64(sslot + 16 * i);
-                const uint32_t sp = prmt(q4.x, q4.y, ssel);
-                const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&sp));
-                a16[i] = fmaf(sf.y, e2 + e3, sf.x * (e0 + e1));
-            }
-            const int r0 = n0 + kLutSet * (warp + kLutWarps * q);
-            const float v = lut_transpose_reduce(a16);  // every value read from the slot is consumed here
-            __syncwarp();
-            if (L == 0 && q + kLutDepth < my)
-                lut_issue_set(rg, &P.cmap[sg.p], &P.smap[sg.p], issued, cx, sx,
-                              n0 + (int64_t)kLutSet * (warp + kLutWarps * (q + kLutDepth)));
-            if (q + kLutDepth < my) ++issued;
-            if (L < kLutSet && r0 + L < n1) {
-                // the row's chunk partial, in fixed point (36 fraction bits)
-                if (!(fabsf(v) < 0x1p27f)) bad |= BT_DEVERR_RANGE;
-                const long long f = __float2ll_rn(fminf(fmaxf(v, -0x1p27f), 0x1p27f) * kLutFix);
-                red_add_u64(acc + r0 + L, static_cast<unsigned long long>(f));
+                for (int i = 0; i < kLutSet; ++i) {
+                    const uint32_t cw = lds_u32(cslot + i * rg.cbox);
+                    if (CHECK && lane_on) bad |= lut_check<LAYOUT>(cw);
+                    const uint32_t o0 = prmt(cw, lanebytes, 0x6604u);
+                    const uint32_t o1 = prmt(cw, lanebytes, 0x6615u);
+                    const uint32_t o2 = prmt(cw, lanebytes, 0x6624u);
+                    const uint32_t o3 = prmt(cw, lanebytes, 0x6635u);
+                    const float e0 = lds_f32(tab_s + o0);
+                    const float e1 = lds_f32(tab_s + o1);
+                    const float e2 = lds_f32(tab_s + kLutRegion + o2);
+                    const float e3 = lds_f32(tab_s + kLutRegion + o3);
+                    const uint2 q4 = lds_u64(sslot + 16 * i);
+                    const uint32_t sp = prmt(q4.x, q4.y, ssel);
+                    const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&sp));
+                    a16[i] = fmaf(sf.y, e2 + e3, sf.x * (e0 + e1));
+                }
+                const int r0 = n0 + kLutSet * (warp + kLutWarps * q);
+                const float v = lut_transpose_reduce(a16);  // every value read from the slot is consumed here
+                __syncwarp();
+                if (L == 0 && q + kLutDepth < my)
+                    lut_issue_set(rg, &P.cmap[sg.p], &P.smap[sg.p], issued, cx, sx,
+                                  n0 + (int64_t)kLutSet * (warp + kLutWarps * (q + kLutDepth)));
+                if (q + kLutDepth < my) ++issued;
+                if (L < kLutSet && r0 + L < n1) {
+                    // the row's chunk partial, in fixed point (36 fraction bits)
+                    if (!(fabsf(v) < 0x1p27f)) bad |= BT_DEVERR_RANGE;
+                    const long long f = __float2ll_rn(fminf(fmaxf(v, -0x1p27f), 0x1p27f) * kLutFix);
+                    red_add_u64(acc + r0 + L, static_cast<unsigned long long>(f));
+                }
             }
         }
-        // hand the finished segment to the finisher warp
-        __syncwarp();
-        if (L == 0) {
-            const uint32_t sl = seg_i % kLutSegSlots;
-            if (seg_i >= (uint32_t)kLutSegSlots && !lut_wait(segempty + 8 * sl, ((seg_i / kLutSegSlots) - 1) & 1u))
-                bad |= BT_DEVERR_TIMEOUT;
-            mbar_arrive(segfull + 8 * sl);
+
+        // ---- phase end: count this CTA's rows into the completion blocks and
+        // convert the blocks it completes
+        __threadfence();  // this thread's adds are performed before the counts below
+        if (threadIdx.x == 0) s_nlast = 0;
+        __syncthreads();
+        {
+            int pair = 0;
+            rc = rc0;
+            while (lut_next_seg(P, rc, rc1, sg)) {
+                const LutProblem& pr = P.p[sg.p];
+                for (int b = sg.n0 / kLutBlockRows; b * kLutBlockRows < sg.n1; ++b, ++pair) {
+                    if (pair % kLutThreads != (int)threadIdx.x) continue;
+                    const int b0 = b * kLutBlockRows, b1 = min(pr.N, b0 + kLutBlockRows);
+                    const int part = min(b1, sg.n1) - max(b0, sg.n0);
+                    if (atomicAdd(P.sync + kLutSyncBlocks + pr.blk_base + b, part) + part == (b1 - b0) * pr.nchunk) {
+                        __threadfence();  // every other CTA's adds to these rows are visible
+                        const int slot = atomicAdd(&s_nlast, 1);
+                        if (slot < kLutMaxLast) s_last[slot] = (sg.p << 20) | b;
+                        else bad |= BT_DEVERR_TIMEOUT;  // (cannot happen: a share touches few blocks)
+                    }
+                }
+            }
         }
-        ++seg_i;
+        __syncthreads();
+        const int nlast = min(s_nlast, kLutMaxLast);
+        for (int i = threadIdx.x; i < nlast * kLutBlockRows; i += kLutThreads) {
+            const int e = s_last[i / kLutBlockRows];
+            const LutProblem& pr = P.p[e >> 20];
+            const int n = (e & 0xFFFFF) * kLutBlockRows + i % kLutBlockRows;
+            if (n < pr.N) {
+                unsigned long long* a = P.acc + pr.acc_base + n;
+                const float v = __ll2float_rn(static_cast<long long>(__ldcg(a))) * kLutUnfix;
+                __stcg(a, 0ull);
+                if (P.y_bf16) reinterpret_cast<__nv_bfloat16*>(pr.y)[n] = __float2bfloat16_rn(v);
+                else reinterpret_cast<float*>(pr.y)[n] = v;
+            }
+        }
+        __syncthreads();
+        if ((int)threadIdx.x < nlast) {
+            const int e = s_last[threadIdx.x];
+            const LutProblem& pr = P.p[e >> 20];
+            const int b = e & 0xFFFFF;
+            P.sync[kLutSyncBlocks + pr.blk_base + b] = 0;
+            if (pr.has_dependents) {
+                __threadfence();  // the block's y is visible before it is counted
+                atomicAdd(P.sync + kLutSyncDone + (e >> 20), min(pr.N, (b + 1) * kLutBlockRows) - b * kLutBlockRows);
+            }
+        }
     }
     // after a timeout: let every copy still in flight land before exiting
     // (each wait is bounded; a set whose wait ran out does not stop the
     // waits on the sets requested after it)
     for (; done < issued; ++done) lut_wait(rg.bar + 8 * (done % kLutDepth), (done / kLutDepth) & 1u);
-}
 
-// The finisher warp: counts the CTA's finished segments into the completion
-// blocks and converts every block this CTA completes.
-__device__ void lut_finish(const LutParams& P, int64_t rc0, int64_t rc1, uint32_t segfull, uint32_t segempty,
-                           int& bad) {
-    const int L = threadIdx.x & 31;
-    pdl_wait();
-    int64_t rc = rc0;
-    LutSeg sg;
-    uint32_t seg_i = 0;
-    while (lut_next_seg(P, rc, rc1, sg)) {
-        const uint32_t sl = seg_i % kLutSegSlots;
-        if (!lut_wait(segfull + 8 * sl, (seg_i / kLutSegSlots) & 1u)) {
-            bad |= BT_DEVERR_TIMEOUT;
-            break;
-        }
-        const LutProblem& pr = P.p[sg.p];
-        const int N = pr.N, nchunk = pr.nchunk;
-        // the streaming warps' adds happened before their arrival; this fence
-        // orders them (cumulatively) before the counts below
-        if (L == 0) fence_acq_rel();
-        __syncwarp();
-        for (int blk = sg.n0 / kLutBlockRows; blk * kLutBlockRows < sg.n1; ++blk) {
-            const int b0 = blk * kLutBlockRows, b1 = min(N, b0 + kLutBlockRows);
-            const int part = min(b1, sg.n1) - max(b0, sg.n0);
-            int* cnt = P.sync + kLutSyncBlocks + pr.blk_base + blk;
-            int last = 0;
-            if (L == 0) {
-                last = atomicAdd(cnt, part) + part == (b1 - b0) * nchunk;
-                if (last) fence_acq_rel();  // every other CTA's adds to these rows are visible
-            }
-            last = __shfl_sync(0xffffffffu, last, 0);
-            if (!last) continue;
-            for (int n = b0 + L; n < b1; n += 32) {
-                const unsigned long long u = atomicExch(P.acc + pr.acc_base + n, 0ull);
-                const float v = __ll2float_rn(static_cast<long long>(u)) * kLutUnfix;
-                if (P.y_bf16) reinterpret_cast<__nv_bfloat16*>(pr.y)[n] = __float2bfloat16_rn(v);
-                else reinterpret_cast<float*>(pr.y)[n] = v;
-            }
-            __syncwarp();
-            if (L == 0) {
-                *cnt = 0;
-                if (pr.has_dependents) {
-                    __threadfence();
-                    atomicAdd(P.sync + kLutSyncDone + sg.p, b1 - b0);
-                }
-            }
-        }
-        __syncwarp();
-        if (L == 0) mbar_arrive(segempty + 8 * sl);
-        ++seg_i;
-    }
-}
-
-template <int LAYOUT, bool CHECK>
-__global__ void __launch_bounds__(kLutAllThreads, 1) gemv_lut_kernel(const __grid_constant__ LutParams P) {
-    const int warp = threadIdx.x >> 5, L = threadIdx.x & 31;
-    const uint32_t segfull = smem_addr(lut_smem + kLutSegBarOffset);
-    const uint32_t segempty = segfull + 8 * kLutSegSlots;
-    // this CTA's contiguous share of the launch's (matrix, chunk, row) items
-    const int64_t rc0 = P.total_rc * blockIdx.x / gridDim.x;
-    const int64_t rc1 = P.total_rc * (blockIdx.x + 1) / gridDim.x;
-
-    if (warp < kLutWarps && L == 0) {
-        const uint32_t bar = smem_addr(lut_smem + kLutBarOffset) + warp * kLutDepth * 8;
-        for (int d = 0; d < kLutDepth; ++d) mbar_init(bar + 8 * d, 1);
-    }
-    if (threadIdx.x == 0) {
-        for (int s = 0; s < kLutSegSlots; ++s) {
-            mbar_init(segfull + 8 * s, kLutWarps);
-            mbar_init(segempty + 8 * s, 1);
-        }
-    }
-    if (L == 0) asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    __syncthreads();
-    pdl_launch_dependents();
-
-    int bad = 0;
-    if (warp < kLutWarps) lut_stream<LAYOUT, CHECK>(P, rc0, rc1, segfull, segempty, bad);
-    else lut_finish(P, rc0, rc1, segfull, segempty, bad);
     bad = __reduce_or_sync(0xffffffffu, bad);
     if (L == 0 && bad) report(P.dev_err, bad);
-    __shared__ int s_abort;
-    if (threadIdx.x == 0) s_abort = 0;
+    if (threadIdx.x == 0) s_flag = 0;
     __syncthreads();
-    if (L == 0 && (bad & BT_DEVERR_TIMEOUT)) atomicOr(&s_abort, 1);
+    if (L == 0 && (bad & BT_DEVERR_TIMEOUT)) atomicOr(&s_flag, 1);
     __syncthreads();
 
     // Launch end: the last CTA resets the per-matrix counters. After a wait
     // that ran out somewhere, it also clears every accumulator and completion
     // counter of the launch, so the workspace is zero again either way.
-    __shared__ int s_last;
+    __shared__ int s_lastcta;
     if (threadIdx.x == 0) {
         __threadfence();
-        if (s_abort) atomicOr(P.sync + kLutSyncAbort, 1);
-        s_last = atomicAdd(P.sync + kLutSyncExit, 1) == (int)gridDim.x - 1;
-        if (s_last) __threadfence();
+        if (s_flag) atomicOr(P.sync + kLutSyncAbort, 1);
+        s_lastcta = atomicAdd(P.sync + kLutSyncExit, 1) == (int)gridDim.x - 1;
+        if (s_lastcta) __threadfence();
     }
     __syncthreads();
-    if (s_last) {
+    if (s_lastcta) {
         const bool aborted = *reinterpret_cast<volatile int*>(P.sync + kLutSyncAbort) != 0;
         if (aborted) {
             const LutProblem& lp = P.p[P.nprob - 1];
@@ -663,6 +631,7 @@ __global__ void __launch_bounds__(kLutAllThreads, 1) gemv_lut_kernel(const __gri
             for (int i = threadIdx.x; i < rows; i += blockDim.x) P.acc[i] = 0ull;
             for (int i = threadIdx.x; i < blocks; i += blockDim.x) P.sync[kLutSyncBlocks + i] = 0;
         }
+        __syncthreads();
         if (threadIdx.x == 0) {
             for (int i = 0; i < P.nprob; ++i) P.sync[kLutSyncDone + i] = 0;
             P.sync[kLutSyncAbort] = 0;
@@ -733,7 +702,7 @@ static cudaError_t lut_launch_t(const LutParams& P, int grid, cudaStream_t strea
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(grid);
-    cfg.blockDim = dim3(kLutAllThreads);
+    cfg.blockDim = dim3(kLutThreads);
     cfg.dynamicSmemBytes = kLutSmem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -797,9 +766,13 @@ static cudaError_t lut_launch_group(int layout, const DecodeProblem* all, int fi
     P.dev_err = dev_err;
     P.sync = reinterpret_cast<int*>(ws);
     P.acc = reinterpret_cast<unsigned long long*>(ws + kLutSyncBytes);
-    P.total_rc = rc;
     P.nprob = count;
     P.y_bf16 = y_bf16;
+    // a matrix that reads an output of this launch starts a new phase
+    P.nphase = 0;
+    for (int i = 0; i < count; ++i)
+        if (i == 0 || P.p[i].dep >= 0) P.phase_rc[P.nphase++] = P.p[i].rc_base;
+    P.phase_rc[P.nphase] = rc;
     // one CTA per SM, never more CTAs than (chunk, row) items
     const int grid = (int)(rc < num_sms ? rc : num_sms);
     if (layout == BT_LAYOUT_B3)
