@@ -68,6 +68,9 @@ def _load():
             lib.oracle_bf16_to_double.restype = ctypes.c_double
             lib.oracle_f16_array_to_double.argtypes = [P, I64, P]
             lib.oracle_bf16_array_to_double.argtypes = [P, I64, P]
+            lib.oracle_double_to_f16.argtypes = [ctypes.c_double]
+            lib.oracle_double_to_f16.restype = ctypes.c_uint16
+            lib.oracle_ternarize.argtypes = [P, P, I64, I64, P, P]
             lib.oracle_threads.restype = ctypes.c_int
             lib.oracle_set_threads.argtypes = [ctypes.c_int]
             _lib = lib
@@ -180,3 +183,23 @@ def forward(trits: np.ndarray, scales_bits: np.ndarray, x_bits: np.ndarray, sign
     xr = rotate_bf16(x_bits, sign)
     y, b = gemv(trits, scales_bits, xr)
     return xr, y, b
+
+
+def double_to_f16(v: float) -> int:
+    """FP16 bit pattern of v, round to nearest even."""
+    return int(_load().oracle_double_to_f16(float(v)))
+
+
+def ternarize(W: np.ndarray, sign: np.ndarray):
+    """The offline weight path: (trits int8 [N, K], scales fp16 bits [N, K/128]).
+
+    Rows of W are rotated block-wise by R = (1/32) H_1024 S, then every
+    128-group takes the threshold (of 40 candidates, (j/20) mean|v|) and
+    least-squares FP16 scale with the smallest reconstruction error."""
+    w = np.ascontiguousarray(W, dtype=np.float64)
+    s = np.ascontiguousarray(sign, dtype=np.int8)
+    N, K = w.shape
+    t = np.zeros((N, K), dtype=np.int8)
+    sc = np.zeros((N, K // GROUP), dtype=np.uint16)
+    _check(_load().oracle_ternarize(_ptr(w), _ptr(s), N, K, _ptr(t), _ptr(sc)), "ternarize")
+    return t, sc

@@ -33,6 +33,23 @@
  *    divide by sqrt n), as described in the TensorSharp blog, section 5.2.
  *    It exists so large inputs finish; tests tie it to the matrix form.
  *
+ *  - oracle_ternarize: the offline weight path. Every row of a float W
+ *    [N][K] is first rotated into the fixed basis block-wise, w'_b =
+ *    (1/sqrt 1024) H_1024 (S . w_b) (release summary, section 三值权重怎么压缩到
+ *    1.76 bit: the weights are transformed to R = (1/sqrt n) H_n S before
+ *    ternarisation and the activation gets the same R at inference), so that
+ *    W' R ~ W. Then every group of 128 rotated weights v gets a scale and a
+ *    threshold by the rule of the TensorSharp blog (2kiu.com/news/5337570),
+ *    section 2.1: t_i = 0 where |v_i / s| is below the threshold, sign(v_i)
+ *    elsewhere, with s derived from the mean |v| and the threshold chosen by
+ *    searching candidates for the smallest reconstruction error. Reading
+ *    taken here: candidate thresholds tau_j = (j / 20) * mean|v|, j = 1..40;
+ *    for each, the trits t_i = sign(v_i) where |v_i| >= tau_j, the scale the
+ *    least-squares one for those trits (the mean |v| over the non-zero
+ *    trits), rounded to FP16, and the error sum_i (v_i - s t_i)^2 with that
+ *    FP16 scale; the smallest error wins, the smallest j on ties. A group of
+ *    zeros gets s = 0 and zero trits. All in FP64, sums in index order.
+ *
  *  - oracle_gemv: y[m][n] = sum_k w[n][k] * x'[m][k] with
  *    w[n][k] = scale[n][k/128] * t[n][k] (dense dequantisation, FP64), and the
  *    acceptance bound B[m][n] = 2e-3 * sum_k |w[n][k] x'[m][k]| + 1e-5.
@@ -251,6 +268,87 @@ int oracle_rotate_butterfly(const double* x, const int8_t* S, int64_t M, int64_t
             for (int64_t j = 0; j < n; ++j) ob[j] = v[j] * inv_sqrt_n;
         }
     }
+    return ORACLE_OK;
+}
+
+/* ---- FP16 rounding and the offline ternarisation ---- */
+
+/* double -> FP16 bit pattern, round to nearest, ties to even (overflow -> inf) */
+uint16_t oracle_double_to_f16(double v)
+{
+    uint16_t sign = 0;
+    if (v < 0 || (v == 0 && signbit(v))) { sign = 0x8000; v = -v; }
+    if (isnan(v)) return 0x7E00;
+    if (v == 0) return sign;
+    /* the FP16 grid near v: exponent e with 2^e <= v < 2^(e+1), clamped to
+     * the subnormal range; spacing 2^(e-10) */
+    int e;
+    frexp(v, &e);  /* v = f * 2^e, f in [0.5, 1) -> 2^(e-1) <= v < 2^e */
+    e -= 1;
+    if (e < -14) e = -14;
+    double ulp = ldexp(1.0, e - 10);
+    double q = v / ulp;                /* exact: a power-of-two division */
+    double r = floor(q);
+    double frac = q - r;
+    if (frac > 0.5 || (frac == 0.5 && fmod(r, 2.0) != 0.0)) r += 1.0;
+    double rounded = r * ulp;          /* may carry into the next binade: fine */
+    if (rounded >= 65520.0) return (uint16_t)(sign | 0x7C00);  /* beyond the largest finite half */
+    /* encode */
+    if (rounded < ldexp(1.0, -14)) {   /* subnormal (or the smallest normal after rounding) */
+        int m = (int)(rounded / ldexp(1.0, -24));
+        if (m >= 1024) return (uint16_t)(sign | 0x0400);
+        return (uint16_t)(sign | m);
+    }
+    int ee;
+    double ff = frexp(rounded, &ee);   /* rounded = ff * 2^ee, ff in [0.5, 1) */
+    int m = (int)((ff * 2.0 - 1.0) * 1024.0 + 0.5);
+    int biased = ee - 1 + 15;
+    return (uint16_t)(sign | (biased << 10) | m);
+}
+
+int oracle_ternarize(const double* W, const int8_t* S, int64_t N, int64_t K, int8_t* trits, uint16_t* scales)
+{
+    if (K % ORACLE_BLOCK != 0 || N < 0) return ORACLE_BAD_SHAPE;
+    double* Wr = (double*)malloc((size_t)(N * K) * sizeof(double));
+    if (!Wr && N * K > 0) return ORACLE_BAD_SHAPE;
+    int rc = oracle_rotate_butterfly(W, S, N, K, Wr);
+    if (rc != ORACLE_OK) { free(Wr); return rc; }
+    const int64_t groups = K / ORACLE_GROUP;
+#pragma omp parallel for schedule(static)
+    for (int64_t gi = 0; gi < N * groups; ++gi) {
+        const int64_t n = gi / groups, g = gi % groups;
+        const double* v = Wr + n * K + g * ORACLE_GROUP;
+        int8_t* t = trits + n * K + g * ORACLE_GROUP;
+        double mean = 0.0;
+        for (int i = 0; i < ORACLE_GROUP; ++i) mean += fabs(v[i]);
+        mean = mean / ORACLE_GROUP;
+        int best_j = 0;
+        double best_err = 0.0;
+        uint16_t best_s = 0;
+        for (int j = 1; j <= 40; ++j) {
+            const double tau = ((double)j / 20.0) * mean;
+            double sum = 0.0;
+            int nnz = 0;
+            for (int i = 0; i < ORACLE_GROUP; ++i) {
+                if (fabs(v[i]) >= tau) { sum += fabs(v[i]); ++nnz; }
+            }
+            const uint16_t s16 = nnz ? oracle_double_to_f16(sum / nnz) : 0;
+            const double s = oracle_f16_to_double(s16);
+            double err = 0.0;
+            for (int i = 0; i < ORACLE_GROUP; ++i) {
+                const double q = fabs(v[i]) >= tau ? (v[i] < 0 ? -s : s) : 0.0;
+                const double d = v[i] - q;
+                err += d * d;
+            }
+            if (j == 1 || err < best_err) { best_err = err; best_j = j; best_s = s16; }
+        }
+        if (mean == 0.0) best_s = 0;   /* a group of zeros: no scale, zero trits */
+        const double tau = ((double)best_j / 20.0) * mean;
+        for (int i = 0; i < ORACLE_GROUP; ++i)
+            t[i] = (mean != 0.0 && fabs(v[i]) >= tau) ? (v[i] < 0 ? -1 : 1) : 0;
+        scales[n * groups + g] = best_s;
+    }
+    free(Wr);
     return ORACLE_OK;
 }
 

@@ -258,3 +258,101 @@ def test_forward_is_gemv_of_rotation():
     H = scipy.linalg.hadamard(1024).astype(np.float64)
     ref_xr = np.concatenate([(H @ (s * x[0, b * 1024:(b + 1) * 1024])) / 32.0 for b in range(2)])
     assert np.max(np.abs(xr[0] - ref_xr)) < 1e-12 * np.max(np.abs(ref_xr))
+
+
+# ------------------------------------------------ offline ternarisation ----
+
+def test_double_to_f16_matches_numpy_round_to_nearest_even():
+    g = np.random.default_rng(7)
+    v = g.standard_normal(100000) * np.exp2(g.integers(-30, 17, 100000))
+    edge = [0.0, -0.0, 65504.0, 65519.99, 65520.0, 1e-8, 2.0 ** -24, 2.0 ** -25, 3 * 2.0 ** -26, 2.0 ** -14,
+            -0.999 * 2.0 ** -14, 1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11, 2049.0, 2051.0]
+    v = np.concatenate([v, edge])
+    ours = np.array([oracle.double_to_f16(x) for x in v], dtype=np.uint16)
+    with np.errstate(over="ignore"):
+        ref = v.astype(np.float16).view(np.uint16)
+    assert np.array_equal(ours, ref)
+
+
+def _rotated_basis_weights(v_rot, sign):
+    """Float W whose block-wise rotation R W^T is exactly v_rot: W = S . (H v) / 32
+    with scipy's Hadamard (R^T = S H / 32, H symmetric); exact for these values."""
+    import scipy.linalg
+    H = scipy.linalg.hadamard(1024).astype(np.float64)
+    N, K = v_rot.shape
+    W = np.zeros_like(v_rot)
+    for b in range(K // 1024):
+        blk = v_rot[:, 1024 * b:1024 * (b + 1)]
+        W[:, 1024 * b:1024 * (b + 1)] = (blk @ H.T) / 32.0 * sign[None, :].astype(np.float64)
+    return W
+
+
+def test_ternarize_recovers_a_ternary_target_exactly():
+    # rotated rows that are exactly c * t: the ternariser must return t and c
+    g = np.random.default_rng(11)
+    N, K = 6, 2048
+    sign = workloads.sign1024()
+    t = g.choice([-1, 0, 1], size=(N, K), p=[0.3, 0.4, 0.3]).astype(np.int8)
+    t[2, 128:256] = 0                                   # one all-zero group: scale 0
+    c = 2.0 ** -3
+    W = _rotated_basis_weights(c * t.astype(np.float64), sign)
+    assert np.array_equal(oracle.rotate(W, sign), c * t)   # the construction is exact
+    trits, scales = oracle.ternarize(W, sign)
+    assert np.array_equal(trits, t)
+    expect = np.full((N, K // 128), np.float16(c).view(np.uint16), dtype=np.uint16)
+    expect[2, 1] = 0
+    assert np.array_equal(scales, expect)
+
+
+def test_ternarize_sign_and_power_of_two_equivariance():
+    g = np.random.default_rng(12)
+    W = g.standard_normal((5, 1024)) * 0.05
+    sign = workloads.sign1024()
+    t, s = oracle.ternarize(W, sign)
+    tn, sn = oracle.ternarize(-W, sign)
+    assert np.array_equal(tn, -t) and np.array_equal(sn, s)
+    t4, s4 = oracle.ternarize(W * 4.0, sign)
+    assert np.array_equal(t4, t)
+    assert np.array_equal(oracle.f16_to_f64(s4), 4.0 * oracle.f16_to_f64(s))
+
+
+def _group_errors(v, t, s_bits):
+    s = oracle.f16_to_f64(s_bits)
+    rec = t.reshape(v.shape[0], -1, 128) * s[:, :, None]
+    return ((v.reshape(v.shape[0], -1, 128) - rec) ** 2).sum(axis=2)
+
+
+def test_ternarize_is_no_worse_than_the_half_mean_threshold():
+    # the search includes tau = 0.5 mean|v| (the pages' fixed +-0.5-style rule),
+    # so its error is never above that rule's error, computed here on its own
+    g = np.random.default_rng(13)
+    W = g.standard_normal((8, 2048)) * 0.02
+    W.reshape(-1)[g.choice(W.size, 40, replace=False)] *= 25.0
+    sign = workloads.sign1024()
+    t, s = oracle.ternarize(W, sign)
+    v = oracle.rotate(W, sign)
+    vg = v.reshape(8, -1, 128)
+    tau = 0.5 * np.abs(vg).mean(axis=2, keepdims=True)
+    keep = np.abs(vg) >= tau
+    s_half = np.array([[np.float16((np.abs(vg[n, q])[keep[n, q]]).mean()).view(np.uint16)
+                        for q in range(vg.shape[1])] for n in range(8)], dtype=np.uint16)
+    t_half = (np.sign(vg) * keep).astype(np.int8).reshape(8, 2048)
+    assert np.all(_group_errors(v, t, s) <= _group_errors(v, t_half, s_half) + 1e-18)
+
+
+def test_rotation_lowers_the_ternarisation_error_on_outlier_weights():
+    # the pages' reason for R: spreading outliers before ternarising. Rotated
+    # ternarisation error (in the rotated basis, equal to the error in the
+    # original one since R is orthogonal) against ternarising W as it is (fed
+    # as R^T W, which the ternariser rotates back to W).
+    g = np.random.default_rng(14)
+    N, K = 16, 2048
+    W = g.standard_normal((N, K)) * 0.02
+    W.reshape(-1)[g.choice(W.size, W.size // 100, replace=False)] *= 20.0
+    sign = workloads.sign1024()
+    t, s = oracle.ternarize(W, sign)
+    err_rot = _group_errors(oracle.rotate(W, sign), t, s).sum()
+    Wt = _rotated_basis_weights(W, sign)            # R^T W
+    t0, s0 = oracle.ternarize(Wt, sign)
+    err_plain = _group_errors(oracle.rotate(Wt, sign), t0, s0).sum()
+    assert err_rot < 0.8 * err_plain, (err_rot, err_plain)
