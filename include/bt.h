@@ -273,6 +273,34 @@ bt_status bt_gemm(int layout, const uint8_t* codes, const uint16_t* scales,
                   int64_t M, int64_t N, int64_t K, void* y_bf16,
                   void* workspace, size_t workspace_bytes, int32_t* dev_err, void* stream);
 
+/*
+ * bt_ternarize: the offline weight path, float W -> trits and g128 FP16
+ * scales in the rotated basis, ready for bt_pack. Source: release summary,
+ * section 三值权重怎么压缩到 1.76 bit (every weight tensor is transformed
+ * block-wise to the fixed basis R = (1/sqrt 1024) H_1024 S before it is
+ * ternarised, and the activation gets the same R, f(x) = W(Rx)); TensorSharp
+ * blog, section 2.1 (per-block scale from the mean |w|, threshold chosen by
+ * searching candidates for the smallest reconstruction error).
+ *  W        device float [N][K], 16-byte aligned; K % 1024 == 0
+ *  sign1024 device int8 [1024] (S), 16-byte aligned
+ *  trits    device int8 [N][K] out: each row is R applied to the row of W,
+ *           block-wise, then ternarised per 128 weights
+ *  scales   device fp16 bits [N][K/128] out, 2-byte aligned
+ *  workspace device, >= bt_ternarize_workspace_bytes(N, K) (the rotated
+ *           weights in FP64), 256-byte aligned; scratch
+ * Per group of 128 rotated weights v: candidate thresholds tau_j = (j / 20)
+ * mean|v| for j = 1..40; trits sign(v_i) where |v_i| >= tau_j, else 0; scale
+ * the mean |v_i| over the non-zero trits, rounded to nearest FP16; the
+ * candidate with the smallest sum (v_i - s t_i)^2 wins (the smallest j on
+ * ties); a group of zeros gets scale 0. All in FP64 in the plain order of
+ * operations, so the result is that of the definition, bit for bit. An
+ * offline step: one warp per (row, 1024-block) rotates, one thread per group
+ * searches.
+ */
+size_t bt_ternarize_workspace_bytes(int64_t N, int64_t K);
+bt_status bt_ternarize(const float* W, const int8_t* sign1024, int64_t N, int64_t K, int8_t* trits,
+                       uint16_t* scales, void* workspace, size_t workspace_bytes, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

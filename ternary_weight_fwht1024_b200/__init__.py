@@ -36,7 +36,7 @@ SINGLE_ROW_MAX_N = 258048
 SYMBOLS = (
     "bt_status_string", "bt_version", "bt_codes_row_bytes", "bt_pack", "bt_unpack",
     "bt_fwht1024", "bt_gemv_workspace_bytes", "bt_gemv", "bt_gemv_batched_workspace_bytes", "bt_gemv_batched",
-    "bt_gemv_noalloc", "bt_gemm_workspace_bytes", "bt_gemm",
+    "bt_gemv_noalloc", "bt_gemm_workspace_bytes", "bt_gemm", "bt_ternarize_workspace_bytes", "bt_ternarize",
 )
 
 
@@ -85,8 +85,11 @@ def load() -> ctypes.CDLL:
             lib.bt_gemm_workspace_bytes.argtypes = [I, I64, I64, I64]
             lib.bt_gemm_workspace_bytes.restype = SZ
             lib.bt_gemm.argtypes = [I, P, P, P, I, P, I64, I64, I64, P, P, SZ, P, P]
+            lib.bt_ternarize_workspace_bytes.argtypes = [I64, I64]
+            lib.bt_ternarize_workspace_bytes.restype = SZ
+            lib.bt_ternarize.argtypes = [P, P, I64, I64, P, P, P, SZ, P]
             for name in ("bt_pack", "bt_unpack", "bt_fwht1024", "bt_gemv", "bt_gemv_batched", "bt_gemv_noalloc",
-                         "bt_gemm"):
+                         "bt_gemm", "bt_ternarize"):
                 getattr(lib, name).restype = I
             _lib = lib
     return _lib
@@ -290,3 +293,24 @@ def gemm(codes: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, sign: torch
                                       M, N, K, _ptr(out), _ptr(ws), ws.numel(), _ptr(dev_err),
                                       _stream(x.device)))
     return out
+
+
+def ternarize(W: torch.Tensor, sign: torch.Tensor, ws: torch.Tensor | None = None):
+    """Offline weight path: float W [N, K] -> (trits int8 [N, K], scales fp16 bits [N, K/128]).
+
+    Rows of W are rotated block-wise by R = (1/32) H_1024 S, then every group
+    of 128 takes the threshold and FP16 scale with the smallest reconstruction
+    error; pack the trits with pack() and multiply with gemv()/gemm() as usual."""
+    _require_cuda(W, sign, ws)
+    if W.dtype != torch.float32:
+        raise TypeError("W must be float32")
+    Wc = W.contiguous()
+    N, K = Wc.shape
+    trits = torch.empty((N, K), dtype=torch.int8, device=W.device)
+    scales = torch.empty((N, K // 128), dtype=torch.int16, device=W.device)
+    need = int(load().bt_ternarize_workspace_bytes(N, K))
+    if ws is None:
+        ws = torch.empty(max(need, 256), dtype=torch.uint8, device=W.device)
+    _check("bt_ternarize", load().bt_ternarize(_ptr(Wc), _ptr(sign), N, K, _ptr(trits), _ptr(scales), _ptr(ws),
+                                                ws.numel(), _stream(W.device)))
+    return trits, scales

@@ -8,7 +8,7 @@ import sys
 HERE = os.path.dirname(os.path.abspath(__file__))
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libbt.so")
-SOURCES = ["bt_api.cu", "bt_pack.cu", "bt_fwht.cu", "bt_gemv.cu", "bt_gemv_lut.cu", "bt_gemm.cu"]
+SOURCES = ["bt_api.cu", "bt_pack.cu", "bt_fwht.cu", "bt_gemv.cu", "bt_gemv_lut.cu", "bt_gemm.cu", "bt_ternarize.cu"]
 HEADERS = ["bt_internal.cuh", "bt_slots.cuh", os.path.join("..", "..", "include", "bt.h")]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

@@ -29,6 +29,9 @@ int64_t gemv1_max_rows();
 cudaError_t launch_gemv1(int layout, const DecodeProblem* problems, int count, const int8_t* sign, int y_dtype,
                          void* workspace, int32_t* dev_err, int num_sms, cudaStream_t stream);
 size_t gemm_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num_sms);
+size_t ternarize_workspace_bytes(int64_t N, int64_t K);
+cudaError_t launch_ternarize(const float* W, const int8_t* sign, int64_t N, int64_t K, int8_t* trits,
+                             uint16_t* scales, void* workspace, cudaStream_t stream);
 cudaError_t launch_gemm(int layout, const uint8_t* codes, const uint16_t* scales, const void* x,
                         int x_dtype, const int8_t* sign, int64_t M, int64_t N, int64_t K, void* y,
                         void* workspace, int32_t* dev_err, int num_sms, cudaStream_t stream);
@@ -274,6 +277,23 @@ bt_status bt_gemm(int layout, const uint8_t* codes, const uint16_t* scales, cons
     if (!aligned(workspace, 256)) return BT_ERR_ALIGN;
     return from_cuda(bt::launch_gemm(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y_bf16,
                                      static_cast<uint8_t*>(workspace) + kSyncBytes, dev_err, sms, s));
+}
+
+size_t bt_ternarize_workspace_bytes(int64_t N, int64_t K) {
+    if (N < 0 || K < 0 || K % 1024 != 0) return 0;
+    return bt::ternarize_workspace_bytes(N, K);
+}
+
+bt_status bt_ternarize(const float* W, const int8_t* sign1024, int64_t N, int64_t K, int8_t* trits,
+                       uint16_t* scales, void* workspace, size_t workspace_bytes, void* stream) {
+    if (N < 0 || K < 0 || K % 1024 != 0 || K > (int64_t(1) << 30) || N > (int64_t(1) << 30)) return BT_ERR_SHAPE;
+    if (N == 0 || K == 0) return BT_OK;
+    if (!W || !sign1024 || !trits || !scales) return BT_ERR_INVALID_ARG;
+    if (!aligned(W, 16) || !aligned(sign1024, 16) || !aligned(scales, 2)) return BT_ERR_ALIGN;
+    if (!workspace || workspace_bytes < bt::ternarize_workspace_bytes(N, K)) return BT_ERR_WORKSPACE;
+    if (!aligned(workspace, 256)) return BT_ERR_ALIGN;
+    return from_cuda(bt::launch_ternarize(W, sign1024, N, K, trits, scales, workspace,
+                                          static_cast<cudaStream_t>(stream)));
 }
 
 }  // extern "C"
