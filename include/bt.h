@@ -55,8 +55,6 @@ typedef enum {
 #define BT_DEVERR_INVALID_CODE 0x2   /* base-3 byte >= 243, or 2-bit field == 3    */
 #define BT_DEVERR_INVALID_PAD  0x4   /* bt_unpack: a pad trit of a base-3 group != 0 */
 #define BT_DEVERR_TIMEOUT      0x8   /* a bounded pipeline wait gave up            */
-#define BT_DEVERR_RANGE        0x10  /* single-row kernel: a partial sum was non-finite
-                                        or beyond +-2^27 (outputs unspecified)     */
 
 typedef enum {
     /* Base-3, 5 trits per byte, code = sum_i (t_i + 1) 3^i with trit i at the
@@ -125,35 +123,31 @@ bt_status bt_fwht1024(const uint16_t* x_bf16, const int8_t* sign1024, int64_t M,
  *            first (K % 1024 == 0). If sign1024 == NULL, x is already
  *            rotated, in x_dtype (BT_F32 or BT_BF16), K % 128 == 0.
  *  y         device [M][N] in y_dtype (BT_F32 or BT_BF16), 16-byte aligned
- *  workspace device, >= bt_gemv_workspace_bytes(...), 256-byte aligned.
- *            Single-row calls that the single-row kernel serves (M = 1,
- *            K % 1024 == 0, 16-byte aligned codes and scales, N <= 258048)
- *            keep counters and fixed-point accumulators in it: such a
- *            workspace must be zero-filled before its first use, and every
- *            call leaves it zero-filled again. Every other call uses its
- *            workspace as plain scratch; a buffer that served one must be
- *            zero-filled again before it serves a single-row call.
+ *  workspace device, >= bt_gemv_workspace_bytes(...), 256-byte aligned. Its
+ *            first 4096 bytes are counters of the single-row kernel: zero-
+ *            fill them once, before the first call with this workspace;
+ *            every call leaves them zero again. The rest is scratch.
  *  dev_err   nullable. When given, the packed codes are validated on the
  *            fly and invalid ones set BT_DEVERR_INVALID_CODE (their
  *            contribution is then unspecified but finite); when NULL the
  *            check is skipped (it costs one ALU op per byte pair or word).
  *            A copy that does not arrive within a bounded wait sets
  *            BT_DEVERR_TIMEOUT and the affected outputs are unspecified.
- * Kernels: single rows that TMA can stream (as above) run the persistent
- * table-lookup kernel of bt_gemv_batched: per-chunk tables of the 5- or
- * 4-trit partial dot products of x', one lookup per packed byte, FP32 table
- * entries and products, chunk partials added in 64-bit fixed point (36
- * fraction bits) by every CTA that streamed them, one launch per call. Other
- * shapes run a prep kernel (rotation, FP16 activation fragments) and an
- * mma.sync kernel (M <= 8 per launch; 9-16 rows take two launches).
+ * Kernels: single rows that TMA can stream (M = 1, K % 1024 == 0, 16-byte
+ * aligned codes and scales, N <= 258048) run the persistent table-lookup
+ * kernel of bt_gemv_batched: per-chunk tables of the 5- or 4-trit partial dot
+ * products of x', one lookup per packed byte, FP32 throughout; the partials
+ * of a row's 512-column chunks are added in chunk order by the CTA that
+ * completes the row's block; one launch per call. Other shapes run a prep
+ * kernel (rotation, FP16 activation fragments) and an mma.sync kernel
+ * (M <= 8 per launch; 9-16 rows take two launches).
  * Consecutive kernels of a call, and of consecutive calls, overlap through
  * programmatic dependent launch: a kernel may start reading codes and scales
  * before the preceding kernel in the stream has finished if that kernel
  * allows it, so codes and scales must not be written by a kernel that
  * triggers dependent launch early.
- * Numerics: single-row kernel: FP32 table entries, scale products and chunk
- * sums, exact integer addition of the chunk partials, one rounding to the
- * output; zero trits contribute exactly 0. Otherwise the rotated activation
+ * Numerics: single-row kernel: FP32 table entries, scale products and sums
+ * in a fixed order; zero trits contribute exactly 0. Otherwise the rotated activation
  * feeds FP16 tensor-core products with FP32 accumulation (one power-of-two
  * exponent per 128 activations keeps it in range), and the digit offset is
  * taken out by the same tensor-core sum of an all-zero-trit row, so zero
@@ -193,11 +187,10 @@ bt_status bt_gemv(int layout, const uint8_t* codes, const uint16_t* scales,
  *    1 <= N <= 258048; K % 1024 == 0
  *  sign1024   as for bt_gemv (NULL: every x is already rotated)
  *  workspace  device, >= bt_gemv_batched_workspace_bytes(...), 256-byte
- *             aligned; counters and fixed-point accumulators that must be
- *             zero-filled before the first call and that every call leaves
- *             zero-filled again (as for single-row bt_gemv calls; after a
- *             call that reported BT_DEVERR_TIMEOUT the kernel clears them
- *             as well).
+ *             aligned; as for bt_gemv, its first 4096 bytes are counters that
+ *             must be zero before the first call and are left zero by every
+ *             call (also after one that reported BT_DEVERR_TIMEOUT); the rest
+ *             holds the chunk partials (N * K / 512 floats per matrix).
  *  dev_err    as for bt_gemv; a dependency or copy that does not arrive
  *             within a bounded time sets BT_DEVERR_TIMEOUT.
  * Matrices of different launches depend on one another through stream order.
@@ -227,13 +220,12 @@ bt_status bt_gemv_batched(int layout, const bt_gemv_problem* problems, int count
  * convenience of this library.
  * Arguments and results are those of bt_gemv without the workspace: the
  * scratch is an 8 MiB array in the library's own device memory, reserved on
- * every GPU that loads libbt.so until the process exits. Its first 2 MiB hold
- * the single-row kernel's counters and accumulators (zero at load, zero again
- * after every call); the other 6 MiB are scratch for the other kernels.
- * Requests needing more than their part (bt_gemv_workspace_bytes beyond
- * 2 MiB for single rows -- more than about 250000 output rows -- or beyond
- * 6 MiB otherwise, for example M >= 10 on 17408-row matrices) are rejected
- * with BT_ERR_WORKSPACE before anything is launched.
+ * every GPU that loads libbt.so until the process exits; its first 4096
+ * bytes are the single-row kernel's counters (zero at load, zero again after
+ * every call). Requests whose bt_gemv_workspace_bytes exceeds 8 MiB (for
+ * example M >= 10 on 17408-row matrices of K = 17408, or single rows with
+ * N * K / 128 beyond about two million) are rejected with BT_ERR_WORKSPACE
+ * before anything is launched.
  * The first call in a CUDA context looks up the array's device address
  * (for the usual primary context: once per device, with that device
  * current) and caches it for that context; a context created later on the

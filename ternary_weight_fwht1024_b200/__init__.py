@@ -26,12 +26,7 @@ DEVERR_INVALID_TRIT = 0x1
 DEVERR_INVALID_CODE = 0x2
 DEVERR_INVALID_PAD = 0x4
 DEVERR_TIMEOUT = 0x8
-DEVERR_RANGE = 0x10
 
-# Single-row calls that the persistent kernel serves keep zero-kept counters and
-# accumulators in their workspace; every other call uses its workspace as
-# scratch. The binding keeps one cached workspace of each kind.
-SINGLE_ROW_MAX_N = 258048
 # Exported entry points, as declared in include/bt.h.
 SYMBOLS = (
     "bt_status_string", "bt_version", "bt_codes_row_bytes", "bt_pack", "bt_unpack",
@@ -122,22 +117,17 @@ def codes_row_bytes(layout: int, K: int) -> int:
     return int(load().bt_codes_row_bytes(layout, K))
 
 
-def workspace(nbytes: int, device, single_row: bool = False) -> torch.Tensor:
-    """A cached uint8 workspace of at least nbytes on `device`, one per stream
-    and kind. Zero-filled when allocated: a single-row workspace must start
-    zeroed (the library keeps it so), a scratch one may hold anything."""
-    key = (torch.device(device), torch.cuda.current_stream(device).cuda_stream, bool(single_row))
+def workspace(nbytes: int, device) -> torch.Tensor:
+    """A cached uint8 workspace of at least nbytes on `device`, one per stream.
+
+    Zero-filled when allocated: its first 4096 bytes are counters that the
+    library keeps at zero between calls (include/bt.h)."""
+    key = (torch.device(device), torch.cuda.current_stream(device).cuda_stream)
     buf = _workspaces.get(key)
     if buf is None or buf.numel() < nbytes:
         buf = torch.zeros(max(nbytes, 4096), dtype=torch.uint8, device=device)
         _workspaces[key] = buf
     return buf
-
-
-def single_row_call(M: int, N: int, K: int, codes: torch.Tensor, scales: torch.Tensor) -> bool:
-    """Whether bt_gemv serves this call with the single-row kernel (zero-kept workspace)."""
-    return (M == 1 and K % 1024 == 0 and N <= SINGLE_ROW_MAX_N and codes.data_ptr() % 16 == 0
-            and scales.data_ptr() % 16 == 0)
 
 
 def new_workspace(nbytes: int, device) -> torch.Tensor:
@@ -204,7 +194,7 @@ def gemv(codes: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, sign: torch
         out = torch.empty((M, N), dtype=torch.float32 if y_dtype == F32 else torch.bfloat16, device=x.device)
     need = gemv_workspace_bytes(layout, M, N, K)
     if ws is None:
-        ws = workspace(need, x.device, single_row_call(M, N, K, codes, scales))
+        ws = workspace(need, x.device)
     _check("bt_gemv", load().bt_gemv(layout, _ptr(codes), _ptr(scales), _ptr(x), _x_dtype(x), _ptr(sign),
                                       M, N, K, y_dtype, _ptr(out), _ptr(ws), ws.numel(), _ptr(dev_err),
                                       _stream(x.device)))
@@ -248,7 +238,7 @@ def gemv_batched(problems, sign: torch.Tensor | None, layout: int = LAYOUT_B3, y
     arr = _problem_array(problems)
     need = int(load().bt_gemv_batched_workspace_bytes(layout, arr, len(problems)))
     if ws is None:
-        ws = workspace(need, dev, single_row=True)
+        ws = workspace(need, dev)
     _check("bt_gemv_batched", load().bt_gemv_batched(layout, arr, len(problems), _ptr(sign), y_dtype, _ptr(ws),
                                                       ws.numel(), _ptr(dev_err), _stream(dev)))
     return [p["y"] for p in problems]
@@ -260,8 +250,7 @@ def gemv_noalloc(codes: torch.Tensor, scales: torch.Tensor, x: torch.Tensor, sig
     """bt_gemv without a caller-provided workspace (scratch lives in libbt.so).
 
     For callers that cannot allocate device memory at call time. Calls share
-    one 8 MiB scratch array per GPU (2 MiB for single rows, 6 MiB for the
-    rest): calls that may overlap on the GPU race.
+    one 8 MiB scratch array per GPU: calls that may overlap on the GPU race.
     `out` may be passed to avoid allocating the result here as well.
     """
     _require_cuda(codes, scales, x, sign, out, dev_err)

@@ -12,8 +12,8 @@ size_t gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num
 cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales, const void* x,
                         int x_dtype, const int8_t* sign, int64_t M, int64_t N, int64_t K, int y_dtype,
                         void* y, void* workspace, int32_t* dev_err, int num_sms, cudaStream_t stream);
-size_t gemv_noalloc_max_bytes(bool single_row);
-cudaError_t gemv_noalloc_scratch(bool single_row, void** out);
+size_t gemv_noalloc_max_bytes();
+cudaError_t gemv_noalloc_scratch(void** out);
 struct DecodeProblem {
     const uint8_t* codes;
     const uint16_t* scales;
@@ -23,7 +23,7 @@ struct DecodeProblem {
     void* y;
     int64_t N, K;
 };
-size_t gemv1_workspace_bytes(const int64_t* Ns, int count);
+size_t gemv1_workspace_bytes(const int64_t* Ns, const int64_t* Ks, int count);
 bool gemv1_applies(int64_t M, int64_t N, int64_t K, const void* codes, const void* scales);
 int64_t gemv1_max_rows();
 cudaError_t launch_gemv1(int layout, const DecodeProblem* problems, int count, const int8_t* sign, int y_dtype,
@@ -189,9 +189,12 @@ bt_status bt_gemv(int layout, const uint8_t* codes, const uint16_t* scales, cons
 
 size_t bt_gemv_batched_workspace_bytes(int layout, const bt_gemv_problem* problems, int count) {
     if (!valid_layout(layout) || !problems || count < 1 || count > 256) return 0;
-    int64_t Ns[256];
-    for (int i = 0; i < count; ++i) Ns[i] = problems[i].N;
-    return bt::gemv1_workspace_bytes(Ns, count);
+    int64_t Ns[256], Ks[256];
+    for (int i = 0; i < count; ++i) {
+        Ns[i] = problems[i].N;
+        Ks[i] = problems[i].K;
+    }
+    return bt::gemv1_workspace_bytes(Ns, Ks, count);
 }
 
 bt_status bt_gemv_batched(int layout, const bt_gemv_problem* problems, int count, const int8_t* sign1024,
@@ -241,11 +244,9 @@ bt_status bt_gemv_noalloc(int layout, const uint8_t* codes, const uint16_t* scal
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (K == 0) return from_cuda(launch_zero(y, M * N * (y_dtype == BT_BF16 ? 2 : 4), s));
     const int sms = current_sm_count();
-    const bool single = bt::gemv1_applies(M, N, K, codes, scales);
-    const size_t need = single ? bt::gemv1_workspace_bytes(&N, 1) : bt::gemv_workspace_bytes(layout, M, N, K, sms);
-    if (need > bt::gemv_noalloc_max_bytes(single)) return BT_ERR_WORKSPACE;
+    if (bt::gemv_workspace_bytes(layout, M, N, K, sms) > bt::gemv_noalloc_max_bytes()) return BT_ERR_WORKSPACE;
     void* scratch = nullptr;
-    if (bt::gemv_noalloc_scratch(single, &scratch) != cudaSuccess) { cudaGetLastError(); return BT_ERR_CUDA; }
+    if (bt::gemv_noalloc_scratch(&scratch) != cudaSuccess) { cudaGetLastError(); return BT_ERR_CUDA; }
     return from_cuda(run_gemv(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y_dtype, y, scratch, dev_err,
                               sms, s));
 }

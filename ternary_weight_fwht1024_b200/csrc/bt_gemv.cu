@@ -1089,21 +1089,20 @@ static GemvPlan make_gemv_plan(int layout, int64_t M, int64_t N, int64_t K, int 
 }
 
 // Single rows that TMA can stream take the persistent table-lookup kernel
-// (bt_gemv_lut.cu), whose workspace is a zero-kept accumulator area; the
-// kernels of this file use their workspace as plain scratch after the
-// first kSyncBytes.
+// (bt_gemv_lut.cu). Every GEMV workspace starts with kSyncBytes of counters
+// that kernel keeps at zero between calls; the kernels of this file use only
+// the bytes after them, as plain scratch.
 constexpr size_t kSyncBytes = 4096;
-bool gemv1_applies(int64_t M, int64_t N, int64_t K, const void* codes, const void* scales);
-size_t gemv1_workspace_bytes(const int64_t* Ns, int count);
+size_t gemv1_workspace_bytes(const int64_t* Ns, const int64_t* Ks, int count);
 
 size_t gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num_sms) {
+    size_t need = kSyncBytes + make_gemv_plan(layout, M, N, K, num_sms).total;
     if (M == 1 && K % 1024 == 0) {
         // the single-row kernel's need (alignment of the pointers is not known here)
-        const size_t one = gemv1_workspace_bytes(&N, 1);
-        const size_t other = kSyncBytes + make_gemv_plan(layout, M, N, K, num_sms).total;
-        return one > other ? one : other;
+        const size_t one = gemv1_workspace_bytes(&N, &K, 1);
+        if (one > need) need = one;
     }
-    return kSyncBytes + make_gemv_plan(layout, M, N, K, num_sms).total;
+    return need;
 }
 
 // TMA-fed variant: applies to M <= 8, K % 1024 == 0, 16-byte aligned scales,
@@ -1317,14 +1316,10 @@ cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales
 // so it is cached per context (not per device ordinal): a context created
 // later on the same device -- after cudaDeviceReset, or a caller's own
 // non-primary context -- gets its own lookup, never a stale address.
-// The first 2 MiB serve the single-row kernel, whose counters and
-// accumulators must start at zero: the array starts zeroed and every
-// single-row call leaves its part zero again. The other 6 MiB are plain
-// scratch for the other kernels, so the two kinds of call never disturb one
-// another.
-constexpr size_t kNoAllocSingleBytes = size_t(2) << 20;  // single-row kernel: zero-kept accumulators
-constexpr size_t kNoAllocOtherBytes = size_t(6) << 20;   // the other kernels: plain scratch
-static __device__ __align__(256) uint8_t noalloc_scratch[kNoAllocSingleBytes + kNoAllocOtherBytes];
+// Its first 4096 bytes are the counters the single-row kernel keeps at zero
+// (the array starts zeroed); the rest is scratch.
+constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
+static __device__ __align__(256) uint8_t noalloc_scratch[kNoAllocScratchBytes];
 
 constexpr int kMaxContexts = 64;
 static std::mutex g_scratch_mutex;
@@ -1346,9 +1341,9 @@ static CtxGetCurrentFn ctx_get_current() {
     return fn;
 }
 
-size_t gemv_noalloc_max_bytes(bool single_row) { return single_row ? kNoAllocSingleBytes : kNoAllocOtherBytes; }
+size_t gemv_noalloc_max_bytes() { return kNoAllocScratchBytes; }
 
-cudaError_t gemv_noalloc_scratch(bool single_row, void** out) {
+cudaError_t gemv_noalloc_scratch(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -1358,7 +1353,7 @@ cudaError_t gemv_noalloc_scratch(bool single_row, void** out) {
         std::lock_guard<std::mutex> lock(g_scratch_mutex);
         for (int i = 0; i < g_scratch_used; ++i) {
             if (g_scratch_ctx[i] == ctx) {
-                *out = static_cast<uint8_t*>(g_scratch_ptr[i]) + (single_row ? 0 : kNoAllocSingleBytes);
+                *out = g_scratch_ptr[i];
                 return cudaSuccess;
             }
         }
@@ -1379,7 +1374,7 @@ cudaError_t gemv_noalloc_scratch(bool single_row, void** out) {
             ++g_scratch_used;
         }
     }
-    *out = static_cast<uint8_t*>(p) + (single_row ? 0 : kNoAllocSingleBytes);
+    *out = p;
     return cudaSuccess;
 }
 

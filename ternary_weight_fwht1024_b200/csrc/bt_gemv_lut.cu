@@ -25,16 +25,15 @@
 // input is an earlier matrix's output, the segment's weights are requested
 // first and the rotation waits until that output is complete.
 //
-// Reduction. A row's chunk partials come from several CTAs. Each is turned
-// into a 64-bit fixed-point integer (36 fraction bits) and added to the row's
-// accumulator with a fire-and-forget red.add: integer sums do not depend on
-// their order, so the result is deterministic with no second kernel. At the
-// end of its share of a phase a CTA counts the rows it streamed into 256-row
-// completion blocks (one atomic per block it touched, all in flight at
-// once); the CTA that completes a block converts its rows to y (one rounding
-// to FP32 or bf16), zeroes their accumulators and, when a later matrix reads
-// this output, counts the rows done. The accumulators and counters are thus
-// zero again after every call.
+// Reduction. A row's chunk partials come from several CTAs; each goes to the
+// workspace with a plain store. At the end of its share of a phase a CTA
+// counts the rows it streamed into 256-row completion blocks (one atomic per
+// block it touched, all in flight at once); the CTA that completes a block
+// adds each of its rows' partials in chunk order (one thread per row, the
+// loads in flight together), so results do not depend on the schedule, and
+// writes y (one rounding to FP32 or bf16); when a later matrix reads this
+// output it then counts the rows done. The completion counters are zero again
+// after every call.
 //
 // Phases. Matrices that do not read one another's outputs form one phase and
 // share the grid as one range; a matrix whose input is an earlier output
@@ -86,8 +85,6 @@ constexpr size_t kLutSyncBytes = 4096;               // counters at the start of
 constexpr int kLutSyncExit = 0, kLutSyncAbort = 1, kLutSyncDone = 2, kLutSyncBlocks = 16;
 constexpr int kLutMaxBlocks = (int)(kLutSyncBytes / 4) - kLutSyncBlocks;  // completion blocks per launch
 constexpr int kLutMaxLast = 64;                      // blocks a CTA converts per round at a phase end
-constexpr float kLutFix = 68719476736.0f;             // 2^36: the accumulators' fixed-point unit
-constexpr float kLutUnfix = 1.0f / 68719476736.0f;    // 2^-36 (exact)
 
 #ifndef BT_WAIT_NS
 #define BT_WAIT_NS 2000000000ull
@@ -101,7 +98,7 @@ struct LutProblem {
     int32_t N, K, G, RB, nchunk, x_bf16;
     int32_t dep;            // problem whose output x is (-1: none)
     int32_t has_dependents; // a later problem of the launch reads this y
-    int32_t acc_base;       // first accumulator (row) of this matrix
+    int64_t part_base;      // first chunk partial of this matrix: partials [chunk][row]
     int32_t blk_base;       // first completion block of this matrix
 };
 
@@ -112,7 +109,7 @@ struct LutParams {
     const int8_t* sign;                // NULL: x already rotated
     int32_t* dev_err;
     int* sync;                         // [exits, rows done per matrix ..., completion blocks ...]
-    unsigned long long* acc;           // fixed-point row sums
+    float* part;                       // chunk partials of every matrix
     int64_t phase_rc[kLutMaxProblems + 1];  // first item of every phase, then the launch's item count
     int nprob, nphase, y_bf16;
 };
@@ -383,10 +380,6 @@ __device__ __forceinline__ bool lut_poll(const int* p, int target) {
     }
 }
 
-__device__ __forceinline__ void red_add_u64(unsigned long long* p, unsigned long long v) {
-    asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" :: "l"(p), "l"(v) : "memory");
-}
-
 // One segment of a CTA's range: matrix p, chunk c, rows [n0, n1).
 struct LutSeg {
     int p, c, n0, n1;
@@ -463,7 +456,7 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_c
         while (lut_next_seg(P, rc, rc1, sg)) {
             const LutProblem& pr = P.p[sg.p];
             const int n0 = sg.n0, n1 = sg.n1;
-            unsigned long long* acc = P.acc + pr.acc_base;
+            float* part = P.part + pr.part_base + (int64_t)sg.c * pr.N;
             const int cb = sg.c * CB;
             const int cx = cb & ~15, coff = cb - cx;
             const int sx = (4 * sg.c) & ~7, soff = 2 * (4 * sg.c - sx);
@@ -541,18 +534,13 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_c
                     lut_issue_set(rg, &P.cmap[sg.p], &P.smap[sg.p], issued, cx, sx,
                                   n0 + (int64_t)kLutSet * (warp + kLutWarps * (q + kLutDepth)));
                 if (q + kLutDepth < my) ++issued;
-                if (L < kLutSet && r0 + L < n1) {
-                    // the row's chunk partial, in fixed point (36 fraction bits)
-                    if (!(fabsf(v) < 0x1p27f)) bad |= BT_DEVERR_RANGE;
-                    const long long f = __float2ll_rn(fminf(fmaxf(v, -0x1p27f), 0x1p27f) * kLutFix);
-                    red_add_u64(acc + r0 + L, static_cast<unsigned long long>(f));
-                }
+                if (L < kLutSet && r0 + L < n1) __stcg(part + r0 + L, v);  // the row's chunk partial
             }
         }
 
         // ---- phase end: count this CTA's rows into the completion blocks and
         // convert the blocks it completes
-        __threadfence();  // this thread's adds are performed before the counts below
+        __threadfence();  // this thread's partials are visible before the counts below
         if (threadIdx.x == 0) s_nlast = 0;
         __syncthreads();
         {
@@ -565,7 +553,7 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_c
                     const int b0 = b * kLutBlockRows, b1 = min(pr.N, b0 + kLutBlockRows);
                     const int part = min(b1, sg.n1) - max(b0, sg.n0);
                     if (atomicAdd(P.sync + kLutSyncBlocks + pr.blk_base + b, part) + part == (b1 - b0) * pr.nchunk) {
-                        __threadfence();  // every other CTA's adds to these rows are visible
+                        __threadfence();  // every other CTA's partials of these rows are visible
                         const int slot = atomicAdd(&s_nlast, 1);
                         if (slot < kLutMaxLast) s_last[slot] = (sg.p << 20) | b;
                         else bad |= BT_DEVERR_TIMEOUT;  // (cannot happen: a share touches few blocks)
@@ -575,16 +563,27 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_c
         }
         __syncthreads();
         const int nlast = min(s_nlast, kLutMaxLast);
+        // every row of a completed block: its chunk partials added in chunk
+        // order (one thread per row, the loads in flight together)
         for (int i = threadIdx.x; i < nlast * kLutBlockRows; i += kLutThreads) {
             const int e = s_last[i / kLutBlockRows];
             const LutProblem& pr = P.p[e >> 20];
             const int n = (e & 0xFFFFF) * kLutBlockRows + i % kLutBlockRows;
             if (n < pr.N) {
-                unsigned long long* a = P.acc + pr.acc_base + n;
-                const float v = __ll2float_rn(static_cast<long long>(__ldcg(a))) * kLutUnfix;
-                __stcg(a, 0ull);
-                if (P.y_bf16) reinterpret_cast<__nv_bfloat16*>(pr.y)[n] = __float2bfloat16_rn(v);
-                else reinterpret_cast<float*>(pr.y)[n] = v;
+                const float* pp = P.part + pr.part_base + n;
+                const int64_t stride = pr.N;
+                float sum = 0.f;
+                int c = 0;
+                for (; c + 8 <= pr.nchunk; c += 8) {
+                    float v8[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) v8[u] = __ldcg(pp + (int64_t)(c + u) * stride);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) sum += v8[u];
+                }
+                for (; c < pr.nchunk; ++c) sum += __ldcg(pp + (int64_t)c * stride);
+                if (P.y_bf16) reinterpret_cast<__nv_bfloat16*>(pr.y)[n] = __float2bfloat16_rn(sum);
+                else reinterpret_cast<float*>(pr.y)[n] = sum;
             }
         }
         __syncthreads();
@@ -612,8 +611,8 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_c
     __syncthreads();
 
     // Launch end: the last CTA resets the per-matrix counters. After a wait
-    // that ran out somewhere, it also clears every accumulator and completion
-    // counter of the launch, so the workspace is zero again either way.
+    // that ran out somewhere, it also clears every completion counter of the
+    // launch, so the counters are zero again either way.
     __shared__ int s_lastcta;
     if (threadIdx.x == 0) {
         __threadfence();
@@ -626,9 +625,7 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_c
         const bool aborted = *reinterpret_cast<volatile int*>(P.sync + kLutSyncAbort) != 0;
         if (aborted) {
             const LutProblem& lp = P.p[P.nprob - 1];
-            const int rows = lp.acc_base + lp.N;
             const int blocks = lp.blk_base + (lp.N + kLutBlockRows - 1) / kLutBlockRows;
-            for (int i = threadIdx.x; i < rows; i += blockDim.x) P.acc[i] = 0ull;
             for (int i = threadIdx.x; i < blocks; i += blockDim.x) P.sync[kLutSyncBlocks + i] = 0;
         }
         __syncthreads();
@@ -673,12 +670,12 @@ static void lut_for_each_launch(const int64_t* Ns, int count, F&& f) {
     }
 }
 
-size_t gemv1_workspace_bytes(const int64_t* Ns, int count) {
+size_t gemv1_workspace_bytes(const int64_t* Ns, const int64_t* Ks, int count) {
     size_t need = kLutSyncBytes;
     lut_for_each_launch(Ns, count, [&](int first, int n) {
-        size_t rows = 0;
-        for (int i = first; i < first + n; ++i) rows += (size_t)Ns[i];
-        const size_t w = kLutSyncBytes + lut_align(rows * 8, 256);
+        size_t parts = 0;
+        for (int i = first; i < first + n; ++i) parts += (size_t)Ns[i] * (size_t)(Ks[i] / kLutChunk);
+        const size_t w = kLutSyncBytes + lut_align(parts * sizeof(float), 256);
         if (w > need) need = w;
     });
     return need;
@@ -719,8 +716,8 @@ static cudaError_t lut_launch_group(int layout, const DecodeProblem* all, int fi
     if (!enc) return cudaErrorNotSupported;
     LutParams P{};
     const int gbytes = layout == BT_LAYOUT_B3 ? kB3GroupBytes : k2bGroupBytes;
-    int64_t rc = 0;
-    int rows = 0, blocks = 0;
+    int64_t rc = 0, parts = 0;
+    int blocks = 0;
     for (int i = 0; i < count; ++i) {
         const DecodeProblem& s = all[first + i];
         LutProblem& d = P.p[i];
@@ -730,7 +727,7 @@ static cudaError_t lut_launch_group(int layout, const DecodeProblem* all, int fi
         d.RB = d.G * gbytes;
         d.nchunk = static_cast<int32_t>(s.K / kLutChunk);
         d.rc_base = rc;
-        d.acc_base = rows;
+        d.part_base = parts;
         d.blk_base = blocks;
         d.y = s.y;
         d.has_dependents = 0;
@@ -745,7 +742,7 @@ static cudaError_t lut_launch_group(int layout, const DecodeProblem* all, int fi
             d.x_bf16 = s.x_from >= 0 ? y_bf16 : s.x_bf16;
         }
         rc += (int64_t)d.nchunk * d.N;
-        rows += d.N;
+        parts += (int64_t)d.nchunk * d.N;
         blocks += (d.N + kLutBlockRows - 1) / kLutBlockRows;
         const cuuint64_t cdim[2] = {static_cast<cuuint64_t>(d.RB), static_cast<cuuint64_t>(s.N)};
         const cuuint64_t cstr[1] = {static_cast<cuuint64_t>(d.RB)};
@@ -765,7 +762,7 @@ static cudaError_t lut_launch_group(int layout, const DecodeProblem* all, int fi
     P.sign = sign;
     P.dev_err = dev_err;
     P.sync = reinterpret_cast<int*>(ws);
-    P.acc = reinterpret_cast<unsigned long long*>(ws + kLutSyncBytes);
+    P.part = reinterpret_cast<float*>(ws + kLutSyncBytes);
     P.nprob = count;
     P.y_bf16 = y_bf16;
     // a matrix that reads an output of this launch starts a new phase

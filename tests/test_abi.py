@@ -143,4 +143,4 @@ def test_batched_validation(lib):
     assert lib.bt_gemv_batched(0, probs(), 0, None, 0, None, 0, None, None) == 0  # nothing to do
     arr = probs()
     need = lib.bt_gemv_batched_workspace_bytes(0, arr, 2)
-    assert need == 4096 + 256 * ((2 * 64 * 8 + 255) // 256)  # counters, then one 64-bit accumulator per row
+    assert need == 4096 + 256 * ((2 * 64 * 2 * 4 + 255) // 256)  # counters, then a float per (row, 512-chunk)
