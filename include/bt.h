@@ -123,10 +123,8 @@ bt_status bt_fwht1024(const uint16_t* x_bf16, const int8_t* sign1024, int64_t M,
  *            first (K % 1024 == 0). If sign1024 == NULL, x is already
  *            rotated, in x_dtype (BT_F32 or BT_BF16), K % 128 == 0.
  *  y         device [M][N] in y_dtype (BT_F32 or BT_BF16), 16-byte aligned
- *  workspace device, >= bt_gemv_workspace_bytes(...), 256-byte aligned. Its
- *            first 4096 bytes are counters of the single-row kernel: zero-
- *            fill them once, before the first call with this workspace;
- *            every call leaves them zero again. The rest is scratch.
+ *  workspace device, >= bt_gemv_workspace_bytes(...), 256-byte aligned;
+ *            scratch (no call expects particular contents).
  *  dev_err   nullable. When given, the packed codes are validated on the
  *            fly and invalid ones set BT_DEVERR_INVALID_CODE (their
  *            contribution is then unspecified but finite); when NULL the
@@ -134,11 +132,11 @@ bt_status bt_fwht1024(const uint16_t* x_bf16, const int8_t* sign1024, int64_t M,
  *            A copy that does not arrive within a bounded wait sets
  *            BT_DEVERR_TIMEOUT and the affected outputs are unspecified.
  * Kernels: single rows that TMA can stream (M = 1, K % 1024 == 0, 16-byte
- * aligned codes and scales, N <= 258048) run the persistent table-lookup
- * kernel of bt_gemv_batched: per-chunk tables of the 5- or 4-trit partial dot
- * products of x', one lookup per packed byte, FP32 throughout; the partials
- * of a row's 512-column chunks are added in chunk order by the CTA that
- * completes the row's block; one launch per call. Other shapes run a prep
+ * aligned codes and scales) run the table-lookup kernels of
+ * bt_gemv_batched: per-chunk tables of the 5- or 4-trit partial dot products
+ * of x', one lookup per packed byte, FP32 throughout, one partial per row and
+ * 512-column chunk; a second kernel adds a row's partials in chunk order.
+ * Other shapes run a prep
  * kernel (rotation, FP16 activation fragments) and an mma.sync kernel
  * (M <= 8 per launch; 9-16 rows take two launches).
  * Consecutive kernels of a call, and of consecutive calls, overlap through
@@ -165,8 +163,9 @@ bt_status bt_gemv(int layout, const uint8_t* codes, const uint16_t* scales,
 
 /*
  * bt_gemv_batched: the single-row (M = 1) product y_p = W_p (R x_p) for a list
- * of matrices, in one persistent launch per 12 matrices (or per 258048 output
- * rows). A matrix's activation is either given (x, x_dtype) or the output of
+ * of matrices: one persistent table-lookup kernel and one reduction kernel per
+ * 12 matrices (fewer where a matrix reads an output of the current group:
+ * it starts the next group). A matrix's activation is either given (x, x_dtype) or the output of
  * an earlier matrix of the list (x_from >= 0: the chained layers of a decode
  * step), so a whole token's stack of layers -- or matrices that share nothing
  * -- stream their weights without a gap between them. Every CTA takes an
@@ -184,16 +183,14 @@ bt_status bt_gemv(int layout, const uint8_t* codes, const uint16_t* scales,
  *             in y_dtype) is this activation; with sign1024 that y must be
  *             bf16 (y_dtype BT_BF16)
  *    y        device [1][N] in y_dtype, 16-byte aligned
- *    1 <= N <= 258048; K % 1024 == 0
+ *    1 <= N <= 2^24; 1024 <= K <= 2^30, K % 1024 == 0
  *  sign1024   as for bt_gemv (NULL: every x is already rotated)
  *  workspace  device, >= bt_gemv_batched_workspace_bytes(...), 256-byte
- *             aligned; as for bt_gemv, its first 4096 bytes are counters that
- *             must be zero before the first call and are left zero by every
- *             call (also after one that reported BT_DEVERR_TIMEOUT); the rest
- *             holds the chunk partials (N * K / 512 floats per matrix).
+ *             aligned; scratch for the chunk partials (N * K / 512 floats per
+ *             matrix of the largest group).
  *  dev_err    as for bt_gemv; a dependency or copy that does not arrive
  *             within a bounded time sets BT_DEVERR_TIMEOUT.
- * Matrices of different launches depend on one another through stream order.
+ * Successive groups depend on one another through stream order.
  * Numerics and determinism as for single-row bt_gemv calls.
  */
 typedef struct {
@@ -220,18 +217,17 @@ bt_status bt_gemv_batched(int layout, const bt_gemv_problem* problems, int count
  * convenience of this library.
  * Arguments and results are those of bt_gemv without the workspace: the
  * scratch is an 8 MiB array in the library's own device memory, reserved on
- * every GPU that loads libbt.so until the process exits; its first 4096
- * bytes are the single-row kernel's counters (zero at load, zero again after
- * every call). Requests whose bt_gemv_workspace_bytes exceeds 8 MiB (for
- * example M >= 10 on 17408-row matrices of K = 17408, or single rows with
- * N * K / 128 beyond about two million) are rejected with BT_ERR_WORKSPACE
+ * every GPU that loads libbt.so until the process exits. Requests whose
+ * bt_gemv_workspace_bytes exceeds 8 MiB (for example M >= 13 on 17408-row
+ * matrices of K = 17408, or single rows with N * K / 512 above 2^21: N = K =
+ * 32768 fits, N = K = 33792 does not) are rejected with BT_ERR_WORKSPACE
  * before anything is launched.
  * The first call in a CUDA context looks up the array's device address
  * (for the usual primary context: once per device, with that device
  * current) and caches it for that context; a context created later on the
  * same device -- after cudaDeviceReset, or a caller's own context -- gets a
  * lookup of its own. Make that first call before any stream capture. All calls share the one array and it keeps the last call's
- * contents (everything that must start at zero is cleared by the call), so
+ * contents (no call depends on them), so
  * calls that may overlap on the GPU -- on different streams, or from
  * different host threads -- race and must be serialised by the caller.
  * Never calls cudaMalloc, cudaFree or any allocating routine.

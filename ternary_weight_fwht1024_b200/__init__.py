@@ -118,21 +118,19 @@ def codes_row_bytes(layout: int, K: int) -> int:
 
 
 def workspace(nbytes: int, device) -> torch.Tensor:
-    """A cached uint8 workspace of at least nbytes on `device`, one per stream.
-
-    Zero-filled when allocated: its first 4096 bytes are counters that the
-    library keeps at zero between calls (include/bt.h)."""
+    """A cached uint8 workspace of at least nbytes on `device`, one per stream
+    (scratch: the library expects no particular contents)."""
     key = (torch.device(device), torch.cuda.current_stream(device).cuda_stream)
     buf = _workspaces.get(key)
     if buf is None or buf.numel() < nbytes:
-        buf = torch.zeros(max(nbytes, 4096), dtype=torch.uint8, device=device)
+        buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
         _workspaces[key] = buf
     return buf
 
 
 def new_workspace(nbytes: int, device) -> torch.Tensor:
-    """A workspace of its own (zero-filled, as every GEMV workspace must start)."""
-    return torch.zeros(max(nbytes, 4096), dtype=torch.uint8, device=device)
+    """A workspace of its own."""
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
 
 
 def pack(trits: torch.Tensor, layout: int = LAYOUT_B3, dev_err: torch.Tensor | None = None) -> torch.Tensor:

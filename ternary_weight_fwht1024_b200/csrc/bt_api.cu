@@ -14,18 +14,8 @@ cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales
                         void* y, void* workspace, int32_t* dev_err, int num_sms, cudaStream_t stream);
 size_t gemv_noalloc_max_bytes();
 cudaError_t gemv_noalloc_scratch(void** out);
-struct DecodeProblem {
-    const uint8_t* codes;
-    const uint16_t* scales;
-    const void* x;
-    int x_bf16;
-    int x_from;
-    void* y;
-    int64_t N, K;
-};
-size_t gemv1_workspace_bytes(const int64_t* Ns, const int64_t* Ks, int count);
-bool gemv1_applies(int64_t M, int64_t N, int64_t K, const void* codes, const void* scales);
-int64_t gemv1_max_rows();
+size_t gemv1_workspace_bytes(const DecodeProblem* problems, int count);
+bool gemv1_applies(int64_t M, int64_t K, const void* codes, const void* scales);
 cudaError_t launch_gemv1(int layout, const DecodeProblem* problems, int count, const int8_t* sign, int y_dtype,
                          void* workspace, int32_t* dev_err, int num_sms, cudaStream_t stream);
 size_t gemm_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num_sms);
@@ -161,7 +151,7 @@ size_t bt_gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K) {
 cudaError_t run_gemv(int layout, const uint8_t* codes, const uint16_t* scales, const void* x, int x_dtype,
                      const int8_t* sign1024, int64_t M, int64_t N, int64_t K, int y_dtype, void* y, void* ws,
                      int32_t* dev_err, int sms, cudaStream_t s) {
-    if (bt::gemv1_applies(M, N, K, codes, scales)) {
+    if (bt::gemv1_applies(M, K, codes, scales)) {
         bt::DecodeProblem p{codes, scales, x, x_dtype == BT_BF16 ? 1 : 0, -1, y, N, K};
         return bt::launch_gemv1(layout, &p, 1, sign1024, y_dtype, ws, dev_err, sms, s);
     }
@@ -189,12 +179,13 @@ bt_status bt_gemv(int layout, const uint8_t* codes, const uint16_t* scales, cons
 
 size_t bt_gemv_batched_workspace_bytes(int layout, const bt_gemv_problem* problems, int count) {
     if (!valid_layout(layout) || !problems || count < 1 || count > 256) return 0;
-    int64_t Ns[256], Ks[256];
+    bt::DecodeProblem dp[256];
     for (int i = 0; i < count; ++i) {
-        Ns[i] = problems[i].N;
-        Ks[i] = problems[i].K;
+        const bt_gemv_problem& q = problems[i];
+        if (q.N < 1 || q.K < 1024 || q.K % 1024 != 0) return 0;
+        dp[i] = bt::DecodeProblem{nullptr, nullptr, nullptr, 1, q.x_from, nullptr, q.N, q.K};
     }
-    return bt::gemv1_workspace_bytes(Ns, Ks, count);
+    return bt::gemv1_workspace_bytes(dp, count);
 }
 
 bt_status bt_gemv_batched(int layout, const bt_gemv_problem* problems, int count, const int8_t* sign1024,
@@ -207,7 +198,7 @@ bt_status bt_gemv_batched(int layout, const bt_gemv_problem* problems, int count
     bt::DecodeProblem dp[256];
     for (int i = 0; i < count; ++i) {
         const bt_gemv_problem& q = problems[i];
-        if (q.N < 1 || q.K < 1024 || q.K % 1024 != 0 || q.K > (int64_t(1) << 30) || q.N > bt::gemv1_max_rows())
+        if (q.N < 1 || q.K < 1024 || q.K % 1024 != 0 || q.K > (int64_t(1) << 30) || q.N > (int64_t(1) << 24))
             return BT_ERR_SHAPE;
         if (!q.codes || !q.scales || !q.y) return BT_ERR_INVALID_ARG;
         if (!aligned(q.codes, 16) || !aligned(q.scales, 16) || !aligned(q.y, 16)) return BT_ERR_ALIGN;
@@ -251,15 +242,10 @@ bt_status bt_gemv_noalloc(int layout, const uint8_t* codes, const uint16_t* scal
                               sms, s));
 }
 
-// Every workspace keeps its first kSyncBytes for the decode kernel's counters
-// (zero between calls); the GEMM's scratch follows them, so one buffer can
-// serve both entry points.
-constexpr size_t kSyncBytes = 4096;
-
 size_t bt_gemm_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K) {
     if (!valid_layout(layout) || M < 128 || M % 128 != 0 || N < 128 || N % 128 != 0 || K < 128 || K % 128 != 0)
         return 0;
-    return kSyncBytes + bt::gemm_workspace_bytes(layout, M, N, K, current_sm_count());
+    return bt::gemm_workspace_bytes(layout, M, N, K, current_sm_count());
 }
 
 bt_status bt_gemm(int layout, const uint8_t* codes, const uint16_t* scales, const void* x, int x_dtype,
@@ -273,11 +259,11 @@ bt_status bt_gemm(int layout, const uint8_t* codes, const uint16_t* scales, cons
     cudaStream_t s = static_cast<cudaStream_t>(stream);
     if (K == 0) return from_cuda(launch_zero(y_bf16, M * N * 2, s));
     const int sms = current_sm_count();
-    const size_t need = kSyncBytes + bt::gemm_workspace_bytes(layout, M, N, K, sms);
+    const size_t need = bt::gemm_workspace_bytes(layout, M, N, K, sms);
     if (!workspace || workspace_bytes < need) return BT_ERR_WORKSPACE;
     if (!aligned(workspace, 256)) return BT_ERR_ALIGN;
     return from_cuda(bt::launch_gemm(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y_bf16,
-                                     static_cast<uint8_t*>(workspace) + kSyncBytes, dev_err, sms, s));
+                                     workspace, dev_err, sms, s));
 }
 
 size_t bt_ternarize_workspace_bytes(int64_t N, int64_t K) {

@@ -1088,18 +1088,16 @@ static GemvPlan make_gemv_plan(int layout, int64_t M, int64_t N, int64_t K, int 
     return pl;
 }
 
-// Single rows that TMA can stream take the persistent table-lookup kernel
-// (bt_gemv_lut.cu). Every GEMV workspace starts with kSyncBytes of counters
-// that kernel keeps at zero between calls; the kernels of this file use only
-// the bytes after them, as plain scratch.
-constexpr size_t kSyncBytes = 4096;
-size_t gemv1_workspace_bytes(const int64_t* Ns, const int64_t* Ks, int count);
+// Single rows that TMA can stream take the table-lookup kernels
+// (bt_gemv_lut.cu); a workspace sized here serves either path.
+size_t gemv1_workspace_bytes(const DecodeProblem* problems, int count);
 
 size_t gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num_sms) {
-    size_t need = kSyncBytes + make_gemv_plan(layout, M, N, K, num_sms).total;
+    size_t need = make_gemv_plan(layout, M, N, K, num_sms).total;
     if (M == 1 && K % 1024 == 0) {
-        // the single-row kernel's need (alignment of the pointers is not known here)
-        const size_t one = gemv1_workspace_bytes(&N, &K, 1);
+        // the single-row kernels' need (alignment of the pointers is not known here)
+        const DecodeProblem p{nullptr, nullptr, nullptr, 1, -1, nullptr, N, K};
+        const size_t one = gemv1_workspace_bytes(&p, 1);
         if (one > need) need = one;
     }
     return need;
@@ -1213,7 +1211,7 @@ cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales
                         int x_dtype, const int8_t* sign, int64_t M, int64_t N, int64_t K, int y_dtype,
                         void* y, void* workspace, int32_t* dev_err, int num_sms,
                         cudaStream_t stream) {
-    uint8_t* ws = static_cast<uint8_t*>(workspace) + kSyncBytes;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
     const GemvPlan pl = make_gemv_plan(layout, M, N, K, num_sms);
 
     PrepArgs pa{};
@@ -1316,8 +1314,7 @@ cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales
 // so it is cached per context (not per device ordinal): a context created
 // later on the same device -- after cudaDeviceReset, or a caller's own
 // non-primary context -- gets its own lookup, never a stale address.
-// Its first 4096 bytes are the counters the single-row kernel keeps at zero
-// (the array starts zeroed); the rest is scratch.
+// Every call uses it as plain scratch: no call expects particular contents.
 constexpr size_t kNoAllocScratchBytes = size_t(8) << 20;  // 8 MiB
 static __device__ __align__(256) uint8_t noalloc_scratch[kNoAllocScratchBytes];
 

@@ -13,7 +13,7 @@
 // cost outside the product at batch 1, and decode is bound by weight bytes
 // (section 实测吞吐).
 //
-// Work. A phase's (matrix, 512-chunk, row) items, in that order, are cut
+// Work. A launch's (matrix, 512-chunk, row) items, in that order, are cut
 // into one contiguous range per CTA (one CTA per SM), so every CTA streams the
 // same number of row chunks. A range is a few segments (matrix p, chunk c,
 // rows n0..n1); per segment the CTA rotates the 1024-block holding the chunk
@@ -21,25 +21,17 @@
 // blog, sections 3.2 and 5.2) unless it already holds it, builds the chunk's
 // tables, and its 16 warps stream the rows in sets of 16 (set k to warp
 // k % 16), each warp with its own two-slot TMA ring ([16 rows][112 B] of codes,
-// x rounded down to 16 B, and [16 rows][8 halves] of scales). When matrix p's
-// input is an earlier matrix's output, the segment's weights are requested
-// first and the rotation waits until that output is complete.
+// x rounded down to 16 B, and [16 rows][8 halves] of scales). Each row's chunk
+// partial goes to the workspace with a plain store.
 //
-// Reduction. A row's chunk partials come from several CTAs; each goes to the
-// workspace with a plain store. At the end of its share of a phase a CTA
-// counts the rows it streamed into 256-row completion blocks (one atomic per
-// block it touched, all in flight at once); the CTA that completes a block
-// adds each of its rows' partials in chunk order (one thread per row, the
-// loads in flight together), so results do not depend on the schedule, and
-// writes y (one rounding to FP32 or bf16); when a later matrix reads this
-// output it then counts the rows done. The completion counters are zero again
-// after every call.
-//
-// Phases. Matrices that do not read one another's outputs form one phase and
-// share the grid as one range; a matrix whose input is an earlier output
-// starts a new phase, which every CTA joins after finishing its share of the
-// previous one (its weights are requested, and it waits for the input, at
-// the start of its first segment).
+// Reduction. A second kernel, launched as a programmatic dependent, adds each
+// row's partials in chunk order (one thread per row), so results do not
+// depend on the schedule, and writes y. (A single kernel that counts finished
+// rows and lets the last CTA of a row block add them was slower on B200: the
+// fences and atomics of CTAs that finish early queue behind the other CTAs'
+// weight stream, several microseconds each.) A list whose matrices read
+// earlier outputs runs as one launch pair per dependency level; stream order
+// carries the outputs from one to the next.
 //
 // Tables. Lane L of a warp reads code word L (bytes 4L..4L+3) of a row chunk,
 // so byte position p = 4L + k is only ever looked up by lane L: its table
@@ -53,6 +45,8 @@
 // one FP32 partial per row of its set in every lane and reduces the 32 x 16
 // block with a butterfly transpose (16 shuffles); lanes i and i + 16 then hold
 // row i.
+#include <algorithm>
+
 #include "bt_internal.cuh"
 
 namespace bt {
@@ -80,11 +74,7 @@ static_assert((kLutSet * kLutCBoxB3 + kLutSet * 16) % 128 == 0 && (kLutSet * kLu
               "slot sizes and the scale boxes inside them keep 128-byte alignment");
 
 constexpr int kLutMaxProblems = 12;                  // per launch (kernel parameters < 4 KB)
-constexpr int kLutBlockRows = 256;                   // rows per completion block
-constexpr size_t kLutSyncBytes = 4096;               // counters at the start of the workspace
-constexpr int kLutSyncExit = 0, kLutSyncAbort = 1, kLutSyncDone = 2, kLutSyncBlocks = 16;
-constexpr int kLutMaxBlocks = (int)(kLutSyncBytes / 4) - kLutSyncBlocks;  // completion blocks per launch
-constexpr int kLutMaxLast = 64;                      // blocks a CTA converts per round at a phase end
+constexpr int kLutReduceThreads = 256;
 
 #ifndef BT_WAIT_NS
 #define BT_WAIT_NS 2000000000ull
@@ -92,14 +82,11 @@ constexpr int kLutMaxLast = 64;                      // blocks a CTA converts pe
 constexpr uint64_t kLutWaitNs = BT_WAIT_NS;
 
 struct LutProblem {
-    const void* x;          // [1][K] bf16 or f32 (the output of problem `dep` when dep >= 0)
+    const void* x;          // [1][K] bf16 or f32
     void* y;                // [1][N]
     int64_t rc_base;        // first (chunk, row) item of this matrix in the launch's order
-    int32_t N, K, G, RB, nchunk, x_bf16;
-    int32_t dep;            // problem whose output x is (-1: none)
-    int32_t has_dependents; // a later problem of the launch reads this y
     int64_t part_base;      // first chunk partial of this matrix: partials [chunk][row]
-    int32_t blk_base;       // first completion block of this matrix
+    int32_t N, K, G, RB, nchunk, x_bf16;
 };
 
 struct LutParams {
@@ -108,10 +95,17 @@ struct LutParams {
     LutProblem p[kLutMaxProblems];
     const int8_t* sign;                // NULL: x already rotated
     int32_t* dev_err;
-    int* sync;                         // [exits, rows done per matrix ..., completion blocks ...]
     float* part;                       // chunk partials of every matrix
-    int64_t phase_rc[kLutMaxProblems + 1];  // first item of every phase, then the launch's item count
-    int nprob, nphase, y_bf16;
+    int64_t total_rc;
+    int nprob;
+};
+
+struct LutReduceParams {
+    const float* part;
+    void* y[kLutMaxProblems];
+    int64_t part_base[kLutMaxProblems];
+    int32_t N[kLutMaxProblems], nchunk[kLutMaxProblems], row_base[kLutMaxProblems];
+    int nprob, rows, y_bf16;
 };
 
 extern __shared__ __align__(1024) uint8_t lut_smem[];
@@ -368,18 +362,6 @@ __device__ __forceinline__ bool lut_wait(uint32_t bar, uint32_t parity) {
     }
 }
 
-// Wait until *p >= target (a counter other CTAs raise), bounded in time.
-__device__ __forceinline__ bool lut_poll(const int* p, int target) {
-    const uint64_t t0 = lut_ns();
-    for (;;) {
-        int v;
-        asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-        if (v >= target) return true;
-        if (lut_ns() - t0 > kLutWaitNs) return false;
-        __nanosleep(128);
-    }
-}
-
 // One segment of a CTA's range: matrix p, chunk c, rows [n0, n1).
 struct LutSeg {
     int p, c, n0, n1;
@@ -408,8 +390,6 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_c
     const uint32_t tab_s = smem_addr(lut_smem);
     float* xr = reinterpret_cast<float*>(lut_smem + kLutXrOffset);
     float* xs = reinterpret_cast<float*>(lut_smem + kLutXsOffset);
-    __shared__ int s_last[kLutMaxLast];   // blocks this CTA completed: (matrix << 20) | block
-    __shared__ int s_nlast, s_flag;
     const int warp = threadIdx.x >> 5, L = threadIdx.x & 31;
     const int CB = LAYOUT == BT_LAYOUT_B3 ? 4 * kB3GroupBytes : 4 * k2bGroupBytes;  // bytes per chunk row
     const bool lane_on = LAYOUT == BT_LAYOUT_B3 ? L < 26 : true;
@@ -438,259 +418,165 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_c
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncwarp();
-    pdl_launch_dependents();
     lut_zero_invalid<LAYOUT>(table);
-    pdl_wait();  // x, y, the accumulators and the counters belong to this launch from here on
+    pdl_wait();  // x may come from the preceding kernel, which may also still read the partials
+    pdl_launch_dependents();
 
     int bad = 0;
     uint32_t issued = 0, done = 0;  // sets requested / consumed by this warp
     bool ok = true;
     int cur_p = -1, cur_blk = -1;
-    for (int ph = 0; ph < P.nphase; ++ph) {
-        // this CTA's contiguous share of the phase's (matrix, chunk, row) items
-        const int64_t base = P.phase_rc[ph], span = P.phase_rc[ph + 1] - base;
-        const int64_t rc0 = base + span * blockIdx.x / gridDim.x;
-        const int64_t rc1 = base + span * (blockIdx.x + 1) / gridDim.x;
-        int64_t rc = rc0;
-        LutSeg sg;
-        while (lut_next_seg(P, rc, rc1, sg)) {
-            const LutProblem& pr = P.p[sg.p];
-            const int n0 = sg.n0, n1 = sg.n1;
-            float* part = P.part + pr.part_base + (int64_t)sg.c * pr.N;
-            const int cb = sg.c * CB;
-            const int cx = cb & ~15, coff = cb - cx;
-            const int sx = (4 * sg.c) & ~7, soff = 2 * (4 * sg.c - sx);
-            const int blk = (sg.c * kLutChunk) / kBlock;
-            const bool new_blk = sg.p != cur_p || blk != cur_blk;
-            const int nsets = (n1 - n0 + kLutSet - 1) / kLutSet;
-            const int my = warp < nsets ? (nsets - warp + kLutWarps - 1) / kLutWarps : 0;  // sets warp, warp + 16, ...
+    // this CTA's contiguous share of the launch's (matrix, chunk, row) items
+    const int64_t rc0 = P.total_rc * blockIdx.x / gridDim.x;
+    const int64_t rc1 = P.total_rc * (blockIdx.x + 1) / gridDim.x;
+    int64_t rc = rc0;
+    LutSeg sg;
+    while (lut_next_seg(P, rc, rc1, sg)) {
+        const LutProblem& pr = P.p[sg.p];
+        const int n0 = sg.n0, n1 = sg.n1;
+        float* part = P.part + pr.part_base + (int64_t)sg.c * pr.N;
+        const int cb = sg.c * CB;
+        const int cx = cb & ~15, coff = cb - cx;
+        const int sx = (4 * sg.c) & ~7, soff = 2 * (4 * sg.c - sx);
+        const int blk = (sg.c * kLutChunk) / kBlock;
+        const bool new_blk = sg.p != cur_p || blk != cur_blk;
+        const int nsets = (n1 - n0 + kLutSet - 1) / kLutSet;
+        const int my = warp < nsets ? (nsets - warp + kLutWarps - 1) / kLutWarps : 0;  // sets warp, warp + 16, ...
 
-            XFetch xf;
-            if (new_blk && warp == 0) {
-                if (sg.p != cur_p && pr.dep >= 0) {
-                    // the input is an earlier matrix's output: wait until all its rows are in
-                    int okw = 1;
-                    if (L == 0) okw = lut_poll(P.sync + kLutSyncDone + pr.dep, P.p[pr.dep].N) ? 1 : 0;
-                    if (!__shfl_sync(0xffffffffu, okw, 0)) bad |= BT_DEVERR_TIMEOUT;
-                }
-                lut_fetch_block(pr.x, pr.x_bf16, P.sign, blk, xf);
-            }
-            __syncthreads();  // the previous segment's lookups are done with table / xs
-            // This segment's first sets go out after warp 0 has issued its
-            // activation loads, so those loads do not queue behind the weight
-            // stream; the rotation and the table build run under the copies'
-            // latency.
-            if (L == 0 && ok)
-                for (int d = 0; d < kLutDepth && d < my; ++d)
-                    lut_issue_set(rg, &P.cmap[sg.p], &P.smap[sg.p], issued + d, cx, sx,
-                                  n0 + (int64_t)kLutSet * (warp + kLutWarps * d));
-            if (ok) issued += min(kLutDepth, my);
-            if (new_blk) {
-                if (warp == 0)
-                    lut_rotate_block(pr.x, pr.x_bf16, P.sign, blk, xf, xr,
-                                     reinterpret_cast<float*>(lut_smem + kLutTileOffset));
-                cur_p = sg.p;
-                cur_blk = blk;
-                __syncthreads();
-            }
-            lut_scatter<LAYOUT>(xr, (sg.c * kLutChunk - blk * kBlock) / kLutChunk, xs);
+        XFetch xf;
+        if (new_blk && warp == 0) lut_fetch_block(pr.x, pr.x_bf16, P.sign, blk, xf);
+        __syncthreads();  // the previous segment's lookups are done with table / xs
+        // This segment's first sets go out after warp 0 has issued its
+        // activation loads, so those loads do not queue behind the weight
+        // stream; the rotation and the table build run under the copies'
+        // latency.
+        if (L == 0 && ok)
+            for (int d = 0; d < kLutDepth && d < my; ++d)
+                lut_issue_set(rg, &P.cmap[sg.p], &P.smap[sg.p], issued + d, cx, sx,
+                              n0 + (int64_t)kLutSet * (warp + kLutWarps * d));
+        if (ok) issued += min(kLutDepth, my);
+        if (new_blk) {
+            if (warp == 0)
+                lut_rotate_block(pr.x, pr.x_bf16, P.sign, blk, xf, xr,
+                                 reinterpret_cast<float*>(lut_smem + kLutTileOffset));
+            cur_p = sg.p;
+            cur_blk = blk;
             __syncthreads();
-            lut_build<LAYOUT>(xs, table);
-            __syncthreads();
+        }
+        lut_scatter<LAYOUT>(xr, (sg.c * kLutChunk - blk * kBlock) / kLutChunk, xs);
+        __syncthreads();
+        lut_build<LAYOUT>(xs, table);
+        __syncthreads();
 
-            for (int q = 0; q < my && ok; ++q) {
-                const uint32_t n = done;
-                const uint32_t d = n % kLutDepth;
-                if (!lut_wait(rg.bar + 8 * d, (n / kLutDepth) & 1u)) {
-                    ok = false;
-                    bad |= BT_DEVERR_TIMEOUT;
-                    break;
-                }
-                ++done;
-                const uint32_t cslot = rg.ring + d * rg.slot_bytes + coff + 4 * wlane;
-                const uint32_t sslot = rg.ring + d * rg.slot_bytes + kLutSet * rg.cbox + soff;
-                float a16[kLutSet];
+        for (int q = 0; q < my && ok; ++q) {
+            const uint32_t n = done;
+            const uint32_t d = n % kLutDepth;
+            if (!lut_wait(rg.bar + 8 * d, (n / kLutDepth) & 1u)) {
+                ok = false;
+                bad |= BT_DEVERR_TIMEOUT;
+                break;
+            }
+            ++done;
+            const uint32_t cslot = rg.ring + d * rg.slot_bytes + coff + 4 * wlane;
+            const uint32_t sslot = rg.ring + d * rg.slot_bytes + kLutSet * rg.cbox + soff;
+            float a16[kLutSet];
 #pragma unroll
-                for (int i = 0; i < kLutSet; ++i) {
-                    const uint32_t cw = lds_u32(cslot + i * rg.cbox);
-                    if (CHECK && lane_on) bad |= lut_check<LAYOUT>(cw);
-                    const uint32_t o0 = prmt(cw, lanebytes, 0x6604u);
-                    const uint32_t o1 = prmt(cw, lanebytes, 0x6615u);
-                    const uint32_t o2 = prmt(cw, lanebytes, 0x6624u);
-                    const uint32_t o3 = prmt(cw, lanebytes, 0x6635u);
-                    const float e0 = lds_f32(tab_s + o0);
-                    const float e1 = lds_f32(tab_s + o1);
-                    const float e2 = lds_f32(tab_s + kLutRegion + o2);
-                    const float e3 = lds_f32(tab_s + kLutRegion + o3);
-                    const uint2 q4 = lds_u64(sslot + 16 * i);
-                    const uint32_t sp = prmt(q4.x, q4.y, ssel);
-                    const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&sp));
-                    a16[i] = fmaf(sf.y, e2 + e3, sf.x * (e0 + e1));
-                }
-                const int r0 = n0 + kLutSet * (warp + kLutWarps * q);
-                const float v = lut_transpose_reduce(a16);  // every value read from the slot is consumed here
-                __syncwarp();
-                if (L == 0 && q + kLutDepth < my)
-                    lut_issue_set(rg, &P.cmap[sg.p], &P.smap[sg.p], issued, cx, sx,
-                                  n0 + (int64_t)kLutSet * (warp + kLutWarps * (q + kLutDepth)));
-                if (q + kLutDepth < my) ++issued;
-                if (L < kLutSet && r0 + L < n1) __stcg(part + r0 + L, v);  // the row's chunk partial
+            for (int i = 0; i < kLutSet; ++i) {
+                const uint32_t cw = lds_u32(cslot + i * rg.cbox);
+                if (CHECK && lane_on) bad |= lut_check<LAYOUT>(cw);
+                const uint32_t o0 = prmt(cw, lanebytes, 0x6604u);
+                const uint32_t o1 = prmt(cw, lanebytes, 0x6615u);
+                const uint32_t o2 = prmt(cw, lanebytes, 0x6624u);
+                const uint32_t o3 = prmt(cw, lanebytes, 0x6635u);
+                const float e0 = lds_f32(tab_s + o0);
+                const float e1 = lds_f32(tab_s + o1);
+                const float e2 = lds_f32(tab_s + kLutRegion + o2);
+                const float e3 = lds_f32(tab_s + kLutRegion + o3);
+                const uint2 q4 = lds_u64(sslot + 16 * i);
+                const uint32_t sp = prmt(q4.x, q4.y, ssel);
+                const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&sp));
+                a16[i] = fmaf(sf.y, e2 + e3, sf.x * (e0 + e1));
             }
-        }
-
-        // ---- phase end: count this CTA's rows into the completion blocks and
-        // convert the blocks it completes
-        __threadfence();  // this thread's partials are visible before the counts below
-        if (threadIdx.x == 0) s_nlast = 0;
-        __syncthreads();
-        {
-            int pair = 0;
-            rc = rc0;
-            while (lut_next_seg(P, rc, rc1, sg)) {
-                const LutProblem& pr = P.p[sg.p];
-                for (int b = sg.n0 / kLutBlockRows; b * kLutBlockRows < sg.n1; ++b, ++pair) {
-                    if (pair % kLutThreads != (int)threadIdx.x) continue;
-                    const int b0 = b * kLutBlockRows, b1 = min(pr.N, b0 + kLutBlockRows);
-                    const int part = min(b1, sg.n1) - max(b0, sg.n0);
-                    if (atomicAdd(P.sync + kLutSyncBlocks + pr.blk_base + b, part) + part == (b1 - b0) * pr.nchunk) {
-                        __threadfence();  // every other CTA's partials of these rows are visible
-                        const int slot = atomicAdd(&s_nlast, 1);
-                        if (slot < kLutMaxLast) s_last[slot] = (sg.p << 20) | b;
-                        else bad |= BT_DEVERR_TIMEOUT;  // (cannot happen: a share touches few blocks)
-                    }
-                }
-            }
-        }
-        __syncthreads();
-        const int nlast = min(s_nlast, kLutMaxLast);
-        // every row of a completed block: its chunk partials added in chunk
-        // order (one thread per row, the loads in flight together)
-        for (int i = threadIdx.x; i < nlast * kLutBlockRows; i += kLutThreads) {
-            const int e = s_last[i / kLutBlockRows];
-            const LutProblem& pr = P.p[e >> 20];
-            const int n = (e & 0xFFFFF) * kLutBlockRows + i % kLutBlockRows;
-            if (n < pr.N) {
-                const float* pp = P.part + pr.part_base + n;
-                const int64_t stride = pr.N;
-                float sum = 0.f;
-                int c = 0;
-                for (; c + 8 <= pr.nchunk; c += 8) {
-                    float v8[8];
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) v8[u] = __ldcg(pp + (int64_t)(c + u) * stride);
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) sum += v8[u];
-                }
-                for (; c < pr.nchunk; ++c) sum += __ldcg(pp + (int64_t)c * stride);
-                if (P.y_bf16) reinterpret_cast<__nv_bfloat16*>(pr.y)[n] = __float2bfloat16_rn(sum);
-                else reinterpret_cast<float*>(pr.y)[n] = sum;
-            }
-        }
-        __syncthreads();
-        if ((int)threadIdx.x < nlast) {
-            const int e = s_last[threadIdx.x];
-            const LutProblem& pr = P.p[e >> 20];
-            const int b = e & 0xFFFFF;
-            P.sync[kLutSyncBlocks + pr.blk_base + b] = 0;
-            if (pr.has_dependents) {
-                __threadfence();  // the block's y is visible before it is counted
-                atomicAdd(P.sync + kLutSyncDone + (e >> 20), min(pr.N, (b + 1) * kLutBlockRows) - b * kLutBlockRows);
-            }
+            const int r0 = n0 + kLutSet * (warp + kLutWarps * q);
+            const float v = lut_transpose_reduce(a16);  // every value read from the slot is consumed here
+            __syncwarp();
+            if (L == 0 && q + kLutDepth < my)
+                lut_issue_set(rg, &P.cmap[sg.p], &P.smap[sg.p], issued, cx, sx,
+                              n0 + (int64_t)kLutSet * (warp + kLutWarps * (q + kLutDepth)));
+            if (q + kLutDepth < my) ++issued;
+            if (L < kLutSet && r0 + L < n1) part[r0 + L] = v;  // the row's chunk partial
         }
     }
     // after a timeout: let every copy still in flight land before exiting
     // (each wait is bounded; a set whose wait ran out does not stop the
     // waits on the sets requested after it)
     for (; done < issued; ++done) lut_wait(rg.bar + 8 * (done % kLutDepth), (done / kLutDepth) & 1u);
-
     bad = __reduce_or_sync(0xffffffffu, bad);
     if (L == 0 && bad) report(P.dev_err, bad);
-    if (threadIdx.x == 0) s_flag = 0;
-    __syncthreads();
-    if (L == 0 && (bad & BT_DEVERR_TIMEOUT)) atomicOr(&s_flag, 1);
-    __syncthreads();
+}
 
-    // Launch end: the last CTA resets the per-matrix counters. After a wait
-    // that ran out somewhere, it also clears every completion counter of the
-    // launch, so the counters are zero again either way.
-    __shared__ int s_lastcta;
-    if (threadIdx.x == 0) {
-        __threadfence();
-        if (s_flag) atomicOr(P.sync + kLutSyncAbort, 1);
-        s_lastcta = atomicAdd(P.sync + kLutSyncExit, 1) == (int)gridDim.x - 1;
-        if (s_lastcta) __threadfence();
+// y of every matrix of the launch: each row's chunk partials added in chunk
+// order (one thread per row; the loads of a row go out together).
+__global__ void __launch_bounds__(kLutReduceThreads) gemv_lut_reduce_kernel(const __grid_constant__ LutReduceParams R) {
+    pdl_wait();
+    pdl_launch_dependents();
+    const int row = blockIdx.x * kLutReduceThreads + threadIdx.x;
+    if (row >= R.rows) return;
+    int p = 0;
+    while (p + 1 < R.nprob && row >= R.row_base[p + 1]) ++p;
+    const int n = row - R.row_base[p];
+    const int N = R.N[p], nchunk = R.nchunk[p];
+    const float* pp = R.part + R.part_base[p] + n;
+    float sum = 0.f;
+    int c = 0;
+    for (; c + 8 <= nchunk; c += 8) {
+        float v8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) v8[u] = pp[(int64_t)(c + u) * N];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) sum += v8[u];
     }
-    __syncthreads();
-    if (s_lastcta) {
-        const bool aborted = *reinterpret_cast<volatile int*>(P.sync + kLutSyncAbort) != 0;
-        if (aborted) {
-            const LutProblem& lp = P.p[P.nprob - 1];
-            const int blocks = lp.blk_base + (lp.N + kLutBlockRows - 1) / kLutBlockRows;
-            for (int i = threadIdx.x; i < blocks; i += blockDim.x) P.sync[kLutSyncBlocks + i] = 0;
-        }
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            for (int i = 0; i < P.nprob; ++i) P.sync[kLutSyncDone + i] = 0;
-            P.sync[kLutSyncAbort] = 0;
-            P.sync[kLutSyncExit] = 0;
-            __threadfence();
-        }
-    }
+    for (; c < nchunk; ++c) sum += pp[(int64_t)c * N];
+    if (R.y_bf16) reinterpret_cast<__nv_bfloat16*>(R.y[p])[n] = __float2bfloat16_rn(sum);
+    else reinterpret_cast<float*>(R.y[p])[n] = sum;
 }
 
 // ---------------------------------------------------------------- host ----
 
-struct DecodeProblem {
-    const uint8_t* codes;
-    const uint16_t* scales;
-    const void* x;
-    int x_bf16;
-    int x_from;  // -1 or an earlier problem index
-    void* y;
-    int64_t N, K;
-};
-
 static size_t lut_align(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-// The launches a list is cut into: at most kLutMaxProblems matrices and
-// kLutMaxBlocks completion blocks each.
+// The launch pairs a list is cut into: at most kLutMaxProblems matrices each,
+// and a new pair wherever a matrix reads the output of a matrix of the
+// current pair.
 template <class F>
-static void lut_for_each_launch(const int64_t* Ns, int count, F&& f) {
+static void lut_for_each_launch(const DecodeProblem* pr, int count, F&& f) {
     int first = 0;
     while (first < count) {
-        int n = 0, blocks = 0;
-        while (first + n < count && n < kLutMaxProblems) {
-            const int b = (int)((Ns[first + n] + kLutBlockRows - 1) / kLutBlockRows);
-            if (n > 0 && blocks + b > kLutMaxBlocks) break;
-            blocks += b;
-            ++n;
-        }
+        int n = 1;
+        while (first + n < count && n < kLutMaxProblems && pr[first + n].x_from < first) ++n;
         f(first, n);
         first += n;
     }
 }
 
-size_t gemv1_workspace_bytes(const int64_t* Ns, const int64_t* Ks, int count) {
-    size_t need = kLutSyncBytes;
-    lut_for_each_launch(Ns, count, [&](int first, int n) {
-        size_t parts = 0;
-        for (int i = first; i < first + n; ++i) parts += (size_t)Ns[i] * (size_t)(Ks[i] / kLutChunk);
-        const size_t w = kLutSyncBytes + lut_align(parts * sizeof(float), 256);
-        if (w > need) need = w;
-    });
+static size_t lut_part_bytes(const DecodeProblem* pr, int first, int n) {
+    size_t parts = 0;
+    for (int i = first; i < first + n; ++i) parts += (size_t)pr[i].N * (size_t)(pr[i].K / kLutChunk);
+    return lut_align(parts * sizeof(float), 256);
+}
+
+size_t gemv1_workspace_bytes(const DecodeProblem* pr, int count) {
+    size_t need = 256;
+    lut_for_each_launch(pr, count, [&](int first, int n) { need = std::max(need, lut_part_bytes(pr, first, n)); });
     return need;
 }
 
 // Single rows whose weights TMA can stream: K a multiple of 1024 (so the
-// scale rows are whole 16-byte units), 16-byte aligned codes and scales, and
-// few enough rows for the completion counters of one launch.
-bool gemv1_applies(int64_t M, int64_t N, int64_t K, const void* codes, const void* scales) {
+// scale rows are whole 16-byte units), 16-byte aligned codes and scales.
+bool gemv1_applies(int64_t M, int64_t K, const void* codes, const void* scales) {
     return M == 1 && K > 0 && K % kBlock == 0 && (reinterpret_cast<uintptr_t>(scales) & 15) == 0 &&
-           (reinterpret_cast<uintptr_t>(codes) & 15) == 0 &&
-           (N + kLutBlockRows - 1) / kLutBlockRows <= kLutMaxBlocks;
+           (reinterpret_cast<uintptr_t>(codes) & 15) == 0;
 }
-
-int64_t gemv1_max_rows() { return (int64_t)kLutMaxBlocks * kLutBlockRows; }
 
 template <int LAYOUT, bool CHECK>
 static cudaError_t lut_launch_t(const LutParams& P, int grid, cudaStream_t stream) {
@@ -710,14 +596,15 @@ static cudaError_t lut_launch_t(const LutParams& P, int grid, cudaStream_t strea
     return cudaLaunchKernelEx(&cfg, kern, P);
 }
 
-static cudaError_t lut_launch_group(int layout, const DecodeProblem* all, int first, int count, const int8_t* sign,
-                                    int y_bf16, uint8_t* ws, int32_t* dev_err, int num_sms, cudaStream_t stream) {
+static cudaError_t lut_launch_pair(int layout, const DecodeProblem* all, int first, int count, const int8_t* sign,
+                                   int y_bf16, float* part, int32_t* dev_err, int num_sms, cudaStream_t stream) {
     EncodeTiledFn enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
     LutParams P{};
+    LutReduceParams R{};
     const int gbytes = layout == BT_LAYOUT_B3 ? kB3GroupBytes : k2bGroupBytes;
-    int64_t rc = 0, parts = 0;
-    int blocks = 0;
+    int64_t rc = 0;
+    int rows = 0;
     for (int i = 0; i < count; ++i) {
         const DecodeProblem& s = all[first + i];
         LutProblem& d = P.p[i];
@@ -727,23 +614,17 @@ static cudaError_t lut_launch_group(int layout, const DecodeProblem* all, int fi
         d.RB = d.G * gbytes;
         d.nchunk = static_cast<int32_t>(s.K / kLutChunk);
         d.rc_base = rc;
-        d.part_base = parts;
-        d.blk_base = blocks;
+        d.part_base = rc;  // one partial per (chunk, row) item
         d.y = s.y;
-        d.has_dependents = 0;
-        if (s.x_from >= first) {
-            d.dep = s.x_from - first;
-            d.x = all[s.x_from].y;
-            d.x_bf16 = y_bf16;
-            P.p[d.dep].has_dependents = 1;
-        } else {
-            d.dep = -1;
-            d.x = s.x_from >= 0 ? all[s.x_from].y : s.x;
-            d.x_bf16 = s.x_from >= 0 ? y_bf16 : s.x_bf16;
-        }
+        d.x = s.x_from >= 0 ? all[s.x_from].y : s.x;
+        d.x_bf16 = s.x_from >= 0 ? y_bf16 : s.x_bf16;
+        R.y[i] = s.y;
+        R.part_base[i] = rc;
+        R.N[i] = d.N;
+        R.nchunk[i] = d.nchunk;
+        R.row_base[i] = rows;
         rc += (int64_t)d.nchunk * d.N;
-        parts += (int64_t)d.nchunk * d.N;
-        blocks += (d.N + kLutBlockRows - 1) / kLutBlockRows;
+        rows += d.N;
         const cuuint64_t cdim[2] = {static_cast<cuuint64_t>(d.RB), static_cast<cuuint64_t>(s.N)};
         const cuuint64_t cstr[1] = {static_cast<cuuint64_t>(d.RB)};
         const cuuint32_t cbox[2] = {static_cast<cuuint32_t>(layout == BT_LAYOUT_B3 ? kLutCBoxB3 : kLutCBox2b), kLutSet};
@@ -761,33 +642,41 @@ static cudaError_t lut_launch_group(int layout, const DecodeProblem* all, int fi
     }
     P.sign = sign;
     P.dev_err = dev_err;
-    P.sync = reinterpret_cast<int*>(ws);
-    P.part = reinterpret_cast<float*>(ws + kLutSyncBytes);
+    P.part = part;
+    P.total_rc = rc;
     P.nprob = count;
-    P.y_bf16 = y_bf16;
-    // a matrix that reads an output of this launch starts a new phase
-    P.nphase = 0;
-    for (int i = 0; i < count; ++i)
-        if (i == 0 || P.p[i].dep >= 0) P.phase_rc[P.nphase++] = P.p[i].rc_base;
-    P.phase_rc[P.nphase] = rc;
+    R.part = part;
+    R.nprob = count;
+    R.rows = rows;
+    R.y_bf16 = y_bf16;
     // one CTA per SM, never more CTAs than (chunk, row) items
     const int grid = (int)(rc < num_sms ? rc : num_sms);
+    cudaError_t e;
     if (layout == BT_LAYOUT_B3)
-        return dev_err ? lut_launch_t<BT_LAYOUT_B3, true>(P, grid, stream)
-                       : lut_launch_t<BT_LAYOUT_B3, false>(P, grid, stream);
-    return dev_err ? lut_launch_t<BT_LAYOUT_2BIT, true>(P, grid, stream)
-                   : lut_launch_t<BT_LAYOUT_2BIT, false>(P, grid, stream);
+        e = dev_err ? lut_launch_t<BT_LAYOUT_B3, true>(P, grid, stream) : lut_launch_t<BT_LAYOUT_B3, false>(P, grid, stream);
+    else
+        e = dev_err ? lut_launch_t<BT_LAYOUT_2BIT, true>(P, grid, stream)
+                    : lut_launch_t<BT_LAYOUT_2BIT, false>(P, grid, stream);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3((unsigned)((rows + kLutReduceThreads - 1) / kLutReduceThreads));
+    cfg.blockDim = dim3(kLutReduceThreads);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, gemv_lut_reduce_kernel, R);
 }
 
 cudaError_t launch_gemv1(int layout, const DecodeProblem* problems, int count, const int8_t* sign, int y_dtype,
                          void* workspace, int32_t* dev_err, int num_sms, cudaStream_t stream) {
-    int64_t Ns[256];
-    for (int i = 0; i < count && i < 256; ++i) Ns[i] = problems[i].N;
     cudaError_t err = cudaSuccess;
-    lut_for_each_launch(Ns, count, [&](int first, int n) {
+    lut_for_each_launch(problems, count, [&](int first, int n) {
         if (err != cudaSuccess) return;
-        err = lut_launch_group(layout, problems, first, n, sign, y_dtype == BT_BF16,
-                               static_cast<uint8_t*>(workspace), dev_err, num_sms, stream);
+        err = lut_launch_pair(layout, problems, first, n, sign, y_dtype == BT_BF16, static_cast<float*>(workspace),
+                              dev_err, num_sms, stream);
     });
     return err;
 }

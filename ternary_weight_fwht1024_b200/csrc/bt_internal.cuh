@@ -24,6 +24,18 @@ constexpr int k2bGroupBytes = 32;  // 2-bit bytes per group
 constexpr int kB3Mmas = 9;
 constexpr int k2bMmas = 8;
 
+// One single-row product of a decode list, y = W (R x): x is either given or
+// the output of an earlier entry of the same list (x_from >= 0).
+struct DecodeProblem {
+    const uint8_t* codes;
+    const uint16_t* scales;
+    const void* x;
+    int x_bf16;
+    int x_from;  // -1, or the index of the entry whose y is this x
+    void* y;
+    int64_t N, K;
+};
+
 // ---------------------------------------------------------------- PTX ----
 
 __device__ __forceinline__ void pdl_wait() {

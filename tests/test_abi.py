@@ -134,7 +134,7 @@ def test_batched_validation(lib):
     assert call(probs()) == 4                       # fine but no workspace
     assert call(probs(K=1000)) == 2                 # K % 1024
     assert call(probs(K=76 * 1024)) == 4            # any K % 1024 == 0
-    assert call(probs(N=258049)) == 2               # beyond the rows of one launch's counters
+    assert call(probs(N=(1 << 24) + 1)) == 2         # rows beyond 2^24
     assert call(probs(x_from=1)) == 1               # only earlier outputs
     assert call(probs(x_from=0, K=1024, N=64)) == 2  # problem 0's N (64) is not this K
     assert call(probs(x_from=-2)) == 1
@@ -143,4 +143,8 @@ def test_batched_validation(lib):
     assert lib.bt_gemv_batched(0, probs(), 0, None, 0, None, 0, None, None) == 0  # nothing to do
     arr = probs()
     need = lib.bt_gemv_batched_workspace_bytes(0, arr, 2)
-    assert need == 4096 + 256 * ((2 * 64 * 2 * 4 + 255) // 256)  # counters, then a float per (row, 512-chunk)
+    assert need == 256 * ((2 * 64 * 2 * 4 + 255) // 256)  # a float per (row, 512-chunk) of the group
+    arr = probs(x_from=0, K=64 * 1024)
+    arr[0].N = 64 * 1024                              # problem 1 reads problem 0: two groups
+    need = lib.bt_gemv_batched_workspace_bytes(0, arr, 2)
+    assert need == max(64 * 1024 * 2, 64 * 128) * 4     # the larger group's partials

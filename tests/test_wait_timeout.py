@@ -6,9 +6,9 @@ lets the copies still in flight land and returns, so the context stays
 usable. These tests load the test-only twin of the library
 (libbt_waittest.so), in which the single-row kernel never requests one set of
 rows -- the second set of CTA 0's warp 0 -- and every wait gives up after
-20 ms. They check that the call returns with the timeout bit set, that the
-workspace's counters are zero again afterwards, and that the product library
-still matches the oracle in the same process. Nothing traps, faults or spins
+20 ms. They check that the call returns with the timeout bit set, that a
+second timed-out call behaves the same, and that the product library still
+matches the oracle in the same process. Nothing traps, faults or spins
 without a bound.
 """
 import ctypes
@@ -50,7 +50,7 @@ def test_withheld_copy_times_out_and_the_context_survives():
 
     lib = _waittest_lib()
     need = lib.bt_gemv_workspace_bytes(bt.LAYOUT_B3, 1, N, K)
-    ws = torch.zeros(need, dtype=torch.uint8, device=dev)  # counters start at zero
+    ws = torch.empty(need, dtype=torch.uint8, device=dev)
     stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
     vp = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
     st = lib.bt_gemv(bt.LAYOUT_B3, vp(codes), vp(scales), vp(x), bt.BF16, vp(sign), 1, N, K, bt.F32, vp(y),
@@ -69,7 +69,7 @@ def test_withheld_copy_times_out_and_the_context_survives():
     assert np.all(np.abs(y2.cpu().numpy().astype(np.float64) - y_ref) <= bound)
 
 
-def test_withheld_copy_twice_leaves_a_clean_workspace():
+def test_withheld_copy_twice_then_a_correct_call():
     dev = torch.device("cuda:0")
     N, K = 5120, 5120          # CTA 0's share: 346 rows of chunk 0, sets 0 and 16 for warp 0
     case = workloads.random_case(11100, 1, N, K)
@@ -82,17 +82,16 @@ def test_withheld_copy_twice_leaves_a_clean_workspace():
 
     lib = _waittest_lib()
     need = lib.bt_gemv_workspace_bytes(bt.LAYOUT_B3, 1, N, K)
-    ws = torch.zeros(need, dtype=torch.uint8, device=dev)  # counters start at zero
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device=dev)  # the workspace's contents do not matter
     stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
     vp = lambda t: ctypes.c_void_p(t.data_ptr())  # noqa: E731
-    for _ in range(2):         # the counters are back at zero after a call that timed out
+    for _ in range(2):
         err.zero_()
         st = lib.bt_gemv(bt.LAYOUT_B3, vp(codes), vp(scales), vp(x), bt.BF16, vp(sign), 1, N, K, bt.F32, vp(y),
                          vp(ws), need, vp(err), stream)
         assert st == 0
         torch.cuda.synchronize()
         assert int(err.item()) & bt.DEVERR_TIMEOUT
-    assert int(ws[:4096].count_nonzero().item()) == 0
 
     _, y_ref, bound = oracle.forward(case["trits"], case["scales"], case["x"], case["sign"])
     err.zero_()
