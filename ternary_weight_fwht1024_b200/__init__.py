@@ -204,12 +204,12 @@ def _problem_array(problems):
     for i, p in enumerate(problems):
         x = p.get("x")
         x_from = int(p.get("x_from", -1))
-        arr[i].codes = p["codes"].data_ptr()
-        arr[i].scales = p["scales"].data_ptr()
+        arr[i].codes = p["codes"].data_ptr() if "codes" in p else None  # sizes alone suffice for the workspace query
+        arr[i].scales = p["scales"].data_ptr() if "scales" in p else None
         arr[i].x = x.data_ptr() if (x is not None and x_from < 0) else None
         arr[i].x_dtype = _x_dtype(x) if (x is not None and x_from < 0) else BF16
         arr[i].x_from = x_from
-        arr[i].y = p["y"].data_ptr()
+        arr[i].y = p["y"].data_ptr() if "y" in p else None
         arr[i].N = int(p["N"])
         arr[i].K = int(p["K"])
     return arr
@@ -222,7 +222,9 @@ def gemv_batched_workspace_bytes(layout: int, problems) -> int:
 
 def gemv_batched(problems, sign: torch.Tensor | None, layout: int = LAYOUT_B3, y_dtype: int = F32,
                  ws: torch.Tensor | None = None, dev_err: torch.Tensor | None = None):
-    """y_p = W_p (R x_p) for a list of single-row problems in one launch (per 12).
+    """y_p = W_p (R x_p) for a list of single-row problems: one persistent
+    kernel per group of up to 12 matrices (a matrix reading an output of the
+    current group starts the next group), then the reductions that write y.
 
     Each problem is a dict with codes, scales, y ([1, N] of y_dtype), N, K and
     either x ([1, K] bf16, or f32 when sign is None) or x_from (the index of an

@@ -64,11 +64,15 @@ constexpr int kLutCBoxB3 = 112;                      // box bytes per row: 104 +
 constexpr int kLutCBox2b = 128;
 constexpr int kLutSlotMax = kLutSet * kLutCBox2b + kLutSet * 16;  // codes box + scale box (8 halves/row)
 constexpr int kLutTileOffset = kLutXsOffset + 5 * 4 * 32 * 4;   // FWHT exchange tile, 32 x 36 f32
-constexpr int kLutBarOffset = kLutTileOffset + 32 * kTileStride * 4;
+constexpr int kLutXstOffset = kLutTileOffset + 32 * kTileStride * 4;  // staged raw block of x (<= 4 KB)
+constexpr int kLutSgnOffset = kLutXstOffset + kBlock * 4;      // the 1024 signs of S
+constexpr int kLutBarOffset = kLutSgnOffset + kBlock;
 // TMA writes into the ring: every slot starts on a 128-byte boundary
 constexpr int kLutRingOffset = (kLutBarOffset + kLutWarps * kLutDepth * 8 + 127) & ~127;
 constexpr int kLutSmem = kLutRingOffset + kLutWarps * kLutDepth * kLutSlotMax;
 static_assert(kLutRingOffset % 128 == 0, "ring slots are TMA destinations");
+static_assert(kLutXstOffset % 16 == 0 && kLutSgnOffset % 16 == 0, "16-byte asynchronous copies land there");
+static_assert(kLutSmem <= 227 * 1024, "one CTA per SM");
 static_assert((kLutSet * kLutCBoxB3 + kLutSet * 16) % 128 == 0 && (kLutSet * kLutCBox2b + kLutSet * 16) % 128 == 0 &&
                   (kLutSet * kLutCBoxB3) % 128 == 0 && (kLutSet * kLutCBox2b) % 128 == 0,
               "slot sizes and the scale boxes inside them keep 128-byte alignment");
@@ -81,12 +85,15 @@ constexpr int kLutReduceThreads = 256;
 #endif
 constexpr uint64_t kLutWaitNs = BT_WAIT_NS;
 
+// Chunk partials: matrix p of a list keeps [nchunk][ld] floats (ld = N
+// rounded up to 4, so every 4-row piece of a chunk is one 16-byte load).
 struct LutProblem {
-    const void* x;          // [1][K] bf16 or f32
-    void* y;                // [1][N]
+    const void* x;          // [1][K] bf16 or f32; unused when src != NULL
+    const float* src;       // NULL, or the partials of the earlier matrix whose output is x
     int64_t rc_base;        // first (chunk, row) item of this matrix in the launch's order
-    int64_t part_base;      // first chunk partial of this matrix: partials [chunk][row]
-    int32_t N, K, G, RB, nchunk, x_bf16;
+    int64_t part_base;      // its own partials, from LutParams::part
+    int32_t N, ld, nchunk, x_bf16;
+    int32_t src_ld, src_nchunk;
 };
 
 struct LutParams {
@@ -95,17 +102,18 @@ struct LutParams {
     LutProblem p[kLutMaxProblems];
     const int8_t* sign;                // NULL: x already rotated
     int32_t* dev_err;
-    float* part;                       // chunk partials of every matrix
+    float* part;                       // chunk partials of every matrix of the list
     int64_t total_rc;
-    int nprob;
+    int nprob, y_bf16;
 };
+static_assert(sizeof(LutParams) <= 4096, "kernel parameters");
 
+// Sums of chunk partials for up to kLutMaxProblems matrices and where they go.
 struct LutReduceParams {
-    const float* part;
+    const float* part[kLutMaxProblems];
     void* y[kLutMaxProblems];
-    int64_t part_base[kLutMaxProblems];
-    int32_t N[kLutMaxProblems], nchunk[kLutMaxProblems], row_base[kLutMaxProblems];
-    int nprob, rows, y_bf16;
+    int32_t N[kLutMaxProblems], ld[kLutMaxProblems], nchunk[kLutMaxProblems];
+    int nprob, y_bf16;
 };
 
 extern __shared__ __align__(1024) uint8_t lut_smem[];
@@ -131,50 +139,57 @@ __device__ __forceinline__ float lds_f32(uint32_t addr) {
     return v;
 }
 
-// Raw words of one lane's 32 bf16 activations of a 1024-block and of its 32
-// sign bytes. Fetched before the first weight copies are requested, so that
-// the rotation does not queue behind them. (FP32 activations are read when
-// the block is rotated.)
-struct XFetch {
-    uint4 q[4];
-    uint4 sg[2];
-};
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
-__device__ __forceinline__ void lut_fetch_block(const void* x, int x_bf16, const int8_t* sign, int blk, XFetch& f) {
+// Warp 0 starts copying the raw 1024-block `blk` of x (bf16: 2 KB, f32:
+// 4 KB) into the staging buffer. Issued as soon as the block is known, so the
+// copy overlaps the stream of the segment before; x may be an output of an
+// earlier kernel, so only after the grid dependency is resolved.
+__device__ __forceinline__ void lut_stage_block(const void* x, int x_bf16, int blk, uint32_t xst) {
     const int lane = threadIdx.x & 31;
-    if (!x_bf16) return;
-    // L2 reads: x may be the output of an earlier matrix of the same launch
-    const uint4* src =
-        reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(x) + (size_t)blk * kBlock + 32 * lane);
-#pragma unroll
-    for (int q = 0; q < 4; ++q) f.q[q] = __ldcg(src + q);
-    if (sign) {
-        const uint4* sg = reinterpret_cast<const uint4*>(sign + 32 * lane);
-        f.sg[0] = __ldg(sg);
-        f.sg[1] = __ldg(sg + 1);
+    const int esz = x_bf16 ? 2 : 4;
+    const uint8_t* src = static_cast<const uint8_t*>(x) + (size_t)blk * kBlock * esz;
+    const int per_lane = esz * 2;  // 16-byte pieces per lane: 4 (bf16) or 8 (f32)
+#pragma unroll 4
+    for (int j = 0; j < per_lane; ++j) {
+        const int off = (lane * per_lane + j) * 16;  // lane l's pieces hold elements 32 l .. 32 l + 31
+        cp_async16(xst + off, src + off);
     }
+    cp_async_commit();
 }
 
-// The rotated (or, without S, copied) block into xr as FP32. Warp 0 only.
-__device__ __forceinline__ void lut_rotate_block(const void* x, int x_bf16, const int8_t* sign, int blk,
-                                                 const XFetch& f, float* xr, float* tile) {
+// The staged block, rotated (or, without S, copied) into xr as FP32. Warp 0
+// only, after every lane's staged copies have landed.
+__device__ __forceinline__ void lut_rotate_block(const uint8_t* xst, int x_bf16, const int8_t* sgn, bool has_sign,
+                                                 float* xr, float* tile) {
     const int lane = threadIdx.x & 31;
     float v[32];
     if (x_bf16) {
-        const uint32_t* w = reinterpret_cast<const uint32_t*>(f.q);
+        const uint4* src = reinterpret_cast<const uint4*>(xst + 64 * lane);
+        uint32_t w[16];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const uint4 t = src[q];
+            w[4 * q] = t.x; w[4 * q + 1] = t.y; w[4 * q + 2] = t.z; w[4 * q + 3] = t.w;
+        }
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = bf16_bits_to_f32((i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu));
     } else {
-        const float4* src = reinterpret_cast<const float4*>(static_cast<const float*>(x) + (size_t)blk * kBlock +
-                                                            32 * lane);
+        const float4* src = reinterpret_cast<const float4*>(xst + 128 * lane);
 #pragma unroll
         for (int q = 0; q < 8; ++q) {
-            const float4 t = __ldcg(src + q);
+            const float4 t = src[q];
             v[4 * q] = t.x; v[4 * q + 1] = t.y; v[4 * q + 2] = t.z; v[4 * q + 3] = t.w;
         }
     }
-    if (sign) {  // the ABI accepts S with bf16 activations only
-        const uint32_t* sw = reinterpret_cast<const uint32_t*>(f.sg);
+    if (has_sign) {  // the ABI accepts S with bf16 activations only
+        const uint4* sg = reinterpret_cast<const uint4*>(sgn + 32 * lane);
+        const uint4 s0 = sg[0], s1 = sg[1];
+        const uint32_t sw[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             // sign byte i: bit 7 set for negative entries
@@ -382,6 +397,49 @@ __device__ __forceinline__ bool lut_next_seg(const LutParams& P, int64_t& rc, in
     return true;
 }
 
+// Row n of matrix p of a group: its chunk partials added in chunk order, up
+// to UNROLL loads in flight. The partials were written by an earlier kernel
+// of the stream: read through L2.
+__device__ __forceinline__ float4 ldcg_f4(const float* p) { return __ldcg(reinterpret_cast<const float4*>(p)); }
+
+// Row n of a matrix whose partials ([nchunk][ld] floats) start at `part`:
+// its chunk partials added in chunk order, RPT rows (n, n + step, ...) at a
+// time with up to UNROLL loads of each row in flight together.
+template <int RPT, int UNROLL>
+__device__ __forceinline__ void lut_row_sums(const float* part, int64_t ld, int nchunk, int n, int step,
+                                             float (&sum)[RPT]) {
+#pragma unroll
+    for (int j = 0; j < RPT; ++j) sum[j] = 0.f;
+    for (int c0 = 0; c0 < nchunk; c0 += UNROLL) {
+        float v[RPT][UNROLL];
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u)
+#pragma unroll
+            for (int j = 0; j < RPT; ++j)
+                v[j][u] = c0 + u < nchunk ? __ldcg(part + (c0 + u) * ld + n + j * step) : 0.f;
+#pragma unroll
+        for (int u = 0; u < UNROLL; ++u)
+#pragma unroll
+            for (int j = 0; j < RPT; ++j)
+                if (c0 + u < nchunk) sum[j] += v[j][u];
+    }
+}
+
+// Block blk of the output of the matrix whose partials pr.src holds, as the
+// stored output reads (bf16-rounded when outputs are bf16), into the staging
+// buffer. All threads of the CTA, two rows each.
+__device__ __forceinline__ void lut_gather_block(const LutProblem& pr, int y_bf16, int blk, uint8_t* xst) {
+    static_assert(kBlock == 2 * kLutThreads, "two rows per thread");
+    float v[2];
+    lut_row_sums<2, 24>(pr.src, pr.src_ld, pr.src_nchunk, blk * kBlock + threadIdx.x, kLutThreads, v);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const int i = threadIdx.x + kLutThreads * j;
+        if (y_bf16) reinterpret_cast<__nv_bfloat16*>(xst)[i] = __float2bfloat16_rn(v[j]);
+        else reinterpret_cast<float*>(xst)[i] = v[j];
+    }
+}
+
 // ------------------------------------------------------------- kernel ----
 
 template <int LAYOUT, bool CHECK>
@@ -390,6 +448,9 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_c
     const uint32_t tab_s = smem_addr(lut_smem);
     float* xr = reinterpret_cast<float*>(lut_smem + kLutXrOffset);
     float* xs = reinterpret_cast<float*>(lut_smem + kLutXsOffset);
+    const uint8_t* xst = lut_smem + kLutXstOffset;
+    const uint32_t xst_s = smem_addr(xst);
+    int8_t* sgn = reinterpret_cast<int8_t*>(lut_smem + kLutSgnOffset);
     const int warp = threadIdx.x >> 5, L = threadIdx.x & 31;
     const int CB = LAYOUT == BT_LAYOUT_B3 ? 4 * kB3GroupBytes : 4 * k2bGroupBytes;  // bytes per chunk row
     const bool lane_on = LAYOUT == BT_LAYOUT_B3 ? L < 26 : true;
@@ -418,47 +479,76 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_c
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     __syncwarp();
+    if (P.sign && threadIdx.x < kBlock / 16)
+        reinterpret_cast<uint4*>(sgn)[threadIdx.x] = __ldg(reinterpret_cast<const uint4*>(P.sign) + threadIdx.x);
     lut_zero_invalid<LAYOUT>(table);
+
+    // This CTA's contiguous share of the launch's (matrix, chunk, row) items,
+    // cut into segments. Each warp requests its sets (warp, warp + 16, ... of
+    // every segment) in order through its own cursor, up to kLutDepth ahead of
+    // the set it works on, across segment boundaries. Weights, scales and S
+    // are never written by the kernels this launch may overlap, so the first
+    // sets go out before the grid dependency is resolved.
+    const int64_t rc0 = P.total_rc * blockIdx.x / gridDim.x;
+    const int64_t rc1 = P.total_rc * (blockIdx.x + 1) / gridDim.x;
+    uint32_t issued = 0, done = 0;  // sets requested / consumed by this warp
+    bool ok = true;
+    LutSeg is;
+    int64_t irc = rc0;
+    int iq = 0;
+    bool ihave = lut_next_seg(P, irc, rc1, is);
+    auto warp_sets = [&](const LutSeg& g) {
+        const int nsets = (g.n1 - g.n0 + kLutSet - 1) / kLutSet;
+        return warp < nsets ? (nsets - warp + kLutWarps - 1) / kLutWarps : 0;
+    };
+    auto issue_next = [&]() {
+        while (ihave && iq >= warp_sets(is)) {
+            ihave = lut_next_seg(P, irc, rc1, is);
+            iq = 0;
+        }
+        if (!ihave) return;
+        if (L == 0) {
+            const int cb = is.c * CB;
+            lut_issue_set(rg, &P.cmap[is.p], &P.smap[is.p], issued, cb & ~15, (4 * is.c) & ~7,
+                          is.n0 + (int64_t)kLutSet * (warp + kLutWarps * iq));
+        }
+        ++iq;
+        ++issued;
+    };
+    for (int d = 0; d < kLutDepth; ++d) issue_next();
+    int64_t rc = rc0;
+    LutSeg sg;
+    bool have = lut_next_seg(P, rc, rc1, sg);
+
     pdl_wait();  // x may come from the preceding kernel, which may also still read the partials
     pdl_launch_dependents();
 
     int bad = 0;
-    uint32_t issued = 0, done = 0;  // sets requested / consumed by this warp
-    bool ok = true;
     int cur_p = -1, cur_blk = -1;
-    // this CTA's contiguous share of the launch's (matrix, chunk, row) items
-    const int64_t rc0 = P.total_rc * blockIdx.x / gridDim.x;
-    const int64_t rc1 = P.total_rc * (blockIdx.x + 1) / gridDim.x;
-    int64_t rc = rc0;
-    LutSeg sg;
-    while (lut_next_seg(P, rc, rc1, sg)) {
+    if (have && warp == 0 && !P.p[sg.p].src)
+        lut_stage_block(P.p[sg.p].x, P.p[sg.p].x_bf16, (sg.c * kLutChunk) / kBlock, xst_s);
+    while (have) {
         const LutProblem& pr = P.p[sg.p];
         const int n0 = sg.n0, n1 = sg.n1;
-        float* part = P.part + pr.part_base + (int64_t)sg.c * pr.N;
-        const int cb = sg.c * CB;
-        const int cx = cb & ~15, coff = cb - cx;
-        const int sx = (4 * sg.c) & ~7, soff = 2 * (4 * sg.c - sx);
+        float* part = P.part + pr.part_base + (int64_t)sg.c * pr.ld;
+        const int coff = (sg.c * CB) & 15;
+        const int soff = 2 * ((4 * sg.c) & 7);
         const int blk = (sg.c * kLutChunk) / kBlock;
         const bool new_blk = sg.p != cur_p || blk != cur_blk;
-        const int nsets = (n1 - n0 + kLutSet - 1) / kLutSet;
-        const int my = warp < nsets ? (nsets - warp + kLutWarps - 1) / kLutWarps : 0;  // sets warp, warp + 16, ...
+        const int my = warp_sets(sg);
 
-        XFetch xf;
-        if (new_blk && warp == 0) lut_fetch_block(pr.x, pr.x_bf16, P.sign, blk, xf);
         __syncthreads();  // the previous segment's lookups are done with table / xs
-        // This segment's first sets go out after warp 0 has issued its
-        // activation loads, so those loads do not queue behind the weight
-        // stream; the rotation and the table build run under the copies'
-        // latency.
-        if (L == 0 && ok)
-            for (int d = 0; d < kLutDepth && d < my; ++d)
-                lut_issue_set(rg, &P.cmap[sg.p], &P.smap[sg.p], issued + d, cx, sx,
-                              n0 + (int64_t)kLutSet * (warp + kLutWarps * d));
-        if (ok) issued += min(kLutDepth, my);
         if (new_blk) {
-            if (warp == 0)
-                lut_rotate_block(pr.x, pr.x_bf16, P.sign, blk, xf, xr,
+            if (pr.src) {  // x is an earlier matrix's output: add up its partials
+                lut_gather_block(pr, P.y_bf16, blk, lut_smem + kLutXstOffset);
+                __syncthreads();
+            }
+            if (warp == 0) {
+                cp_async_wait_all();
+                __syncwarp();
+                lut_rotate_block(xst, pr.x_bf16, sgn, P.sign != nullptr, xr,
                                  reinterpret_cast<float*>(lut_smem + kLutTileOffset));
+            }
             cur_p = sg.p;
             cur_blk = blk;
             __syncthreads();
@@ -467,6 +557,16 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_c
         __syncthreads();
         lut_build<LAYOUT>(xs, table);
         __syncthreads();
+
+        // the next segment; its block of x is staged now if it is a new one
+        LutSeg nx;
+        int64_t nrc = rc;
+        const bool nhave = lut_next_seg(P, nrc, rc1, nx);
+        if (nhave && warp == 0) {
+            const int nb = (nx.c * kLutChunk) / kBlock;
+            if ((nx.p != sg.p || nb != blk) && !P.p[nx.p].src)
+                lut_stage_block(P.p[nx.p].x, P.p[nx.p].x_bf16, nb, xst_s);
+        }
 
         for (int q = 0; q < my && ok; ++q) {
             const uint32_t n = done;
@@ -500,45 +600,40 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_c
             const int r0 = n0 + kLutSet * (warp + kLutWarps * q);
             const float v = lut_transpose_reduce(a16);  // every value read from the slot is consumed here
             __syncwarp();
-            if (L == 0 && q + kLutDepth < my)
-                lut_issue_set(rg, &P.cmap[sg.p], &P.smap[sg.p], issued, cx, sx,
-                              n0 + (int64_t)kLutSet * (warp + kLutWarps * (q + kLutDepth)));
-            if (q + kLutDepth < my) ++issued;
+            issue_next();  // into the slot just freed
             if (L < kLutSet && r0 + L < n1) part[r0 + L] = v;  // the row's chunk partial
         }
+        sg = nx;
+        rc = nrc;
+        have = nhave;
     }
     // after a timeout: let every copy still in flight land before exiting
     // (each wait is bounded; a set whose wait ran out does not stop the
     // waits on the sets requested after it)
     for (; done < issued; ++done) lut_wait(rg.bar + 8 * (done % kLutDepth), (done / kLutDepth) & 1u);
+    cp_async_wait_all();
     bad = __reduce_or_sync(0xffffffffu, bad);
     if (L == 0 && bad) report(P.dev_err, bad);
 }
 
-// y of every matrix of the launch: each row's chunk partials added in chunk
-// order (one thread per row; the loads of a row go out together).
+// y of up to 12 matrices, one thread per row: its chunk partials added in
+// chunk order, up to 64 loads in flight together.
 __global__ void __launch_bounds__(kLutReduceThreads) gemv_lut_reduce_kernel(const __grid_constant__ LutReduceParams R) {
+    // the tile's matrix and first row, from the parameters, before the wait
+    int q = 0, k = blockIdx.x;
+    for (; q < R.nprob; ++q) {
+        const int t = (R.N[q] + kLutReduceThreads - 1) / kLutReduceThreads;
+        if (k < t) break;
+        k -= t;
+    }
     pdl_wait();
     pdl_launch_dependents();
-    const int row = blockIdx.x * kLutReduceThreads + threadIdx.x;
-    if (row >= R.rows) return;
-    int p = 0;
-    while (p + 1 < R.nprob && row >= R.row_base[p + 1]) ++p;
-    const int n = row - R.row_base[p];
-    const int N = R.N[p], nchunk = R.nchunk[p];
-    const float* pp = R.part + R.part_base[p] + n;
-    float sum = 0.f;
-    int c = 0;
-    for (; c + 8 <= nchunk; c += 8) {
-        float v8[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) v8[u] = pp[(int64_t)(c + u) * N];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) sum += v8[u];
-    }
-    for (; c < nchunk; ++c) sum += pp[(int64_t)c * N];
-    if (R.y_bf16) reinterpret_cast<__nv_bfloat16*>(R.y[p])[n] = __float2bfloat16_rn(sum);
-    else reinterpret_cast<float*>(R.y[p])[n] = sum;
+    const int n = k * kLutReduceThreads + threadIdx.x;
+    if (q >= R.nprob || n >= R.N[q]) return;
+    float v[1];
+    lut_row_sums<1, 64>(R.part[q], R.ld[q], R.nchunk[q], n, 0, v);
+    if (R.y_bf16) reinterpret_cast<__nv_bfloat16*>(R.y[q])[n] = __float2bfloat16_rn(v[0]);
+    else reinterpret_cast<float*>(R.y[q])[n] = v[0];
 }
 
 // ---------------------------------------------------------------- host ----
@@ -559,16 +654,20 @@ static void lut_for_each_launch(const DecodeProblem* pr, int count, F&& f) {
     }
 }
 
-static size_t lut_part_bytes(const DecodeProblem* pr, int first, int n) {
-    size_t parts = 0;
-    for (int i = first; i < first + n; ++i) parts += (size_t)pr[i].N * (size_t)(pr[i].K / kLutChunk);
-    return lut_align(parts * sizeof(float), 256);
-}
+// Partial floats of one matrix: [K / 512][N rounded up to 4].
+static int64_t lut_part_floats(const DecodeProblem& p) { return (p.K / kLutChunk) * ((p.N + 3) & ~3); }
 
+// Every matrix of a list keeps its partials until the list's reductions at
+// the end (a later group may read them as its input): their sum, each group
+// starting on a 256-byte boundary.
 size_t gemv1_workspace_bytes(const DecodeProblem* pr, int count) {
-    size_t need = 256;
-    lut_for_each_launch(pr, count, [&](int first, int n) { need = std::max(need, lut_part_bytes(pr, first, n)); });
-    return need;
+    size_t total = 0;
+    lut_for_each_launch(pr, count, [&](int first, int n) {
+        int64_t f = 0;
+        for (int i = first; i < first + n; ++i) f += lut_part_floats(pr[i]);
+        total += lut_align((size_t)f * sizeof(float), 256);
+    });
+    return std::max(total, (size_t)256);
 }
 
 // Single rows whose weights TMA can stream: K a multiple of 1024 (so the
@@ -596,40 +695,44 @@ static cudaError_t lut_launch_t(const LutParams& P, int grid, cudaStream_t strea
     return cudaLaunchKernelEx(&cfg, kern, P);
 }
 
-static cudaError_t lut_launch_pair(int layout, const DecodeProblem* all, int first, int count, const int8_t* sign,
-                                   int y_bf16, float* part, int32_t* dev_err, int num_sms, cudaStream_t stream) {
+// The partials and outputs of one group, as the reduction reads them.
+// The main kernel of group [first, first + count). base[i]: offset in floats
+// of matrix i's partials in the workspace `part`.
+static cudaError_t lut_launch_group(int layout, const DecodeProblem* all, const int64_t* base, int first, int count,
+                                    const int8_t* sign, int y_bf16, float* part, int32_t* dev_err, int num_sms,
+                                    cudaStream_t stream) {
     EncodeTiledFn enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
     LutParams P{};
-    LutReduceParams R{};
     const int gbytes = layout == BT_LAYOUT_B3 ? kB3GroupBytes : k2bGroupBytes;
     int64_t rc = 0;
-    int rows = 0;
     for (int i = 0; i < count; ++i) {
         const DecodeProblem& s = all[first + i];
         LutProblem& d = P.p[i];
+        const int64_t G = s.K / kGroup, RB = G * gbytes;
         d.N = static_cast<int32_t>(s.N);
-        d.K = static_cast<int32_t>(s.K);
-        d.G = static_cast<int32_t>(s.K / kGroup);
-        d.RB = d.G * gbytes;
+        d.ld = static_cast<int32_t>((s.N + 3) & ~3);
         d.nchunk = static_cast<int32_t>(s.K / kLutChunk);
         d.rc_base = rc;
-        d.part_base = rc;  // one partial per (chunk, row) item
-        d.y = s.y;
-        d.x = s.x_from >= 0 ? all[s.x_from].y : s.x;
-        d.x_bf16 = s.x_from >= 0 ? y_bf16 : s.x_bf16;
-        R.y[i] = s.y;
-        R.part_base[i] = rc;
-        R.N[i] = d.N;
-        R.nchunk[i] = d.nchunk;
-        R.row_base[i] = rows;
+        d.part_base = base[first + i];
+        if (s.x_from >= 0) {  // an earlier group's output: summed from its partials
+            const DecodeProblem& q = all[s.x_from];
+            d.src = part + base[s.x_from];
+            d.src_ld = static_cast<int32_t>((q.N + 3) & ~3);
+            d.src_nchunk = static_cast<int32_t>(q.K / kLutChunk);
+            d.x = nullptr;
+            d.x_bf16 = y_bf16;
+        } else {
+            d.src = nullptr;
+            d.x = s.x;
+            d.x_bf16 = s.x_bf16;
+        }
         rc += (int64_t)d.nchunk * d.N;
-        rows += d.N;
-        const cuuint64_t cdim[2] = {static_cast<cuuint64_t>(d.RB), static_cast<cuuint64_t>(s.N)};
-        const cuuint64_t cstr[1] = {static_cast<cuuint64_t>(d.RB)};
+        const cuuint64_t cdim[2] = {static_cast<cuuint64_t>(RB), static_cast<cuuint64_t>(s.N)};
+        const cuuint64_t cstr[1] = {static_cast<cuuint64_t>(RB)};
         const cuuint32_t cbox[2] = {static_cast<cuuint32_t>(layout == BT_LAYOUT_B3 ? kLutCBoxB3 : kLutCBox2b), kLutSet};
-        const cuuint64_t sdim[2] = {static_cast<cuuint64_t>(d.G), static_cast<cuuint64_t>(s.N)};
-        const cuuint64_t sstr[1] = {static_cast<cuuint64_t>(d.G) * 2};
+        const cuuint64_t sdim[2] = {static_cast<cuuint64_t>(G), static_cast<cuuint64_t>(s.N)};
+        const cuuint64_t sstr[1] = {static_cast<cuuint64_t>(G) * 2};
         const cuuint32_t sbox[2] = {8, kLutSet};
         const cuuint32_t one[2] = {1, 1};
         if (enc(&P.cmap[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(s.codes), cdim, cstr, cbox, one,
@@ -645,21 +748,34 @@ static cudaError_t lut_launch_pair(int layout, const DecodeProblem* all, int fir
     P.part = part;
     P.total_rc = rc;
     P.nprob = count;
-    R.part = part;
-    R.nprob = count;
-    R.rows = rows;
-    R.y_bf16 = y_bf16;
+    P.y_bf16 = y_bf16;
     // one CTA per SM, never more CTAs than (chunk, row) items
     const int grid = (int)(rc < num_sms ? rc : num_sms);
-    cudaError_t e;
     if (layout == BT_LAYOUT_B3)
-        e = dev_err ? lut_launch_t<BT_LAYOUT_B3, true>(P, grid, stream) : lut_launch_t<BT_LAYOUT_B3, false>(P, grid, stream);
-    else
-        e = dev_err ? lut_launch_t<BT_LAYOUT_2BIT, true>(P, grid, stream)
-                    : lut_launch_t<BT_LAYOUT_2BIT, false>(P, grid, stream);
-    if (e != cudaSuccess) return e;
+        return dev_err ? lut_launch_t<BT_LAYOUT_B3, true>(P, grid, stream)
+                       : lut_launch_t<BT_LAYOUT_B3, false>(P, grid, stream);
+    return dev_err ? lut_launch_t<BT_LAYOUT_2BIT, true>(P, grid, stream)
+                   : lut_launch_t<BT_LAYOUT_2BIT, false>(P, grid, stream);
+}
+
+// Outputs of matrices [first, first + count), count <= kLutMaxProblems.
+static cudaError_t lut_launch_reduce(const DecodeProblem* all, const int64_t* base, int first, int count, int y_bf16,
+                                     float* part, cudaStream_t stream) {
+    LutReduceParams R{};
+    R.nprob = count;
+    R.y_bf16 = y_bf16;
+    int tiles = 0;
+    for (int i = 0; i < count; ++i) {
+        const DecodeProblem& s = all[first + i];
+        R.part[i] = part + base[first + i];
+        R.y[i] = s.y;
+        R.N[i] = static_cast<int32_t>(s.N);
+        R.ld[i] = static_cast<int32_t>((s.N + 3) & ~3);
+        R.nchunk[i] = static_cast<int32_t>(s.K / kLutChunk);
+        tiles += (int)((s.N + kLutReduceThreads - 1) / kLutReduceThreads);
+    }
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3((unsigned)((rows + kLutReduceThreads - 1) / kLutReduceThreads));
+    cfg.gridDim = dim3((unsigned)tiles);
     cfg.blockDim = dim3(kLutReduceThreads);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
@@ -670,14 +786,32 @@ static cudaError_t lut_launch_pair(int layout, const DecodeProblem* all, int fir
     return cudaLaunchKernelEx(&cfg, gemv_lut_reduce_kernel, R);
 }
 
+// A list runs as one main kernel per group (a matrix that reads an output of
+// the current group starts the next one) and, at the end, the reductions
+// that write every output: a group reads its inputs from the partials of the
+// groups before it, so between groups there is nothing else to wait for.
 cudaError_t launch_gemv1(int layout, const DecodeProblem* problems, int count, const int8_t* sign, int y_dtype,
                          void* workspace, int32_t* dev_err, int num_sms, cudaStream_t stream) {
+    const int y_bf16 = y_dtype == BT_BF16;
+    float* part = static_cast<float*>(workspace);
+    int64_t base[256];
+    {
+        int64_t off = 0;
+        lut_for_each_launch(problems, count, [&](int first, int n) {
+            for (int i = first; i < first + n; ++i) {
+                base[i] = off;
+                off += lut_part_floats(problems[i]);
+            }
+            off = (int64_t)lut_align((size_t)off, 64);  // 256-byte boundary between groups
+        });
+    }
     cudaError_t err = cudaSuccess;
     lut_for_each_launch(problems, count, [&](int first, int n) {
-        if (err != cudaSuccess) return;
-        err = lut_launch_pair(layout, problems, first, n, sign, y_dtype == BT_BF16, static_cast<float*>(workspace),
-                              dev_err, num_sms, stream);
+        if (err == cudaSuccess)
+            err = lut_launch_group(layout, problems, base, first, n, sign, y_bf16, part, dev_err, num_sms, stream);
     });
+    for (int first = 0; first < count && err == cudaSuccess; first += kLutMaxProblems)
+        err = lut_launch_reduce(problems, base, first, std::min(kLutMaxProblems, count - first), y_bf16, part, stream);
     return err;
 }
 

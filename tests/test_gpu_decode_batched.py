@@ -231,3 +231,35 @@ def test_batched_zero_weights_exact_and_invalid_codes_flagged():
     torch.cuda.synchronize()
     assert int(err.item()) & bt.DEVERR_INVALID_CODE
     assert torch.isfinite(y).all()
+
+
+@pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
+def test_batched_outputs_feeding_later_matrices(layout):
+    # inputs from the previous group (summed from its partials inside the next
+    # kernel), from a group two launches back (read from memory) and given
+    # activations, mixed in one list: groups {A}, {B, C}, {D, E, F}
+    spec = [(1024, 2048, None), (2048, 1024, 0), (2048, 3072, 0), (1024, 1024, 1), (2048, 777, 0), (3072, 500, None)]
+    g = workloads.rng(12600 + layout)
+    sign_np = workloads.sign1024()
+    cases, probs = [], []
+    for K, N, src in spec:
+        c = {"K": K, "N": N, "trits": workloads.trits(g, N, K), "scales": workloads.scales_f16_bits(g, N, K),
+             "src": src}
+        codes, sc = _weights(c, layout)
+        p = dict(codes=codes, scales=sc, y=torch.empty((1, N), dtype=torch.bfloat16, device=DEV), N=N, K=K)
+        if src is None:
+            c["x"] = workloads.activations_bf16_bits(g, 1, K, True)
+            p["x"] = T(c["x"], "bf16")
+        else:
+            p["x_from"] = src
+        cases.append(c)
+        probs.append(p)
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    ys = bt.gemv_batched(probs, T(sign_np), layout, y_dtype=bt.BF16, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+    for c, y in zip(cases, ys):
+        xb = c["x"] if c["src"] is None else ys[c["src"]].view(torch.int16).cpu().numpy().view(np.uint16)
+        y_ref, b = oracle.gemv(c["trits"], c["scales"], oracle.rotate_bf16(xb, sign_np))
+        y64 = y.float().cpu().numpy().astype(np.float64)
+        check(y64, y_ref, b, bf16_half_ulp(y64))
