@@ -1,9 +1,9 @@
 """Benchmark: packed-ternary decode GEMV (with the FWHT-1024 rotation) on B200.
 
 One step = one decode token through the 5120x5120 / 5120x17408 / 17408x5120
-triple at M = 1: for each matrix, bt_gemv rotates the bf16 activation block-wise
-(R = H_1024 S / 32) and multiplies by the base-3 packed ternary weights with
-g128 FP16 scales. The weights are synthetic and seeded (the pages' 27B model
+triple at M = 1: one bt_gemv_batched call takes the three matrices, each with
+its own bf16 activation, rotates each activation block-wise (R = H_1024 S / 32)
+and multiplies by the base-3 packed ternary weights with g128 FP16 scales. The weights are synthetic and seeded (the pages' 27B model
 is not available); twelve distinct copies of the triple (537 MB, over four
 times the 126 MB L2) are used in turn so every step streams from HBM.
 
@@ -38,6 +38,7 @@ L2_BYTES = 126 * 1024 * 1024
 # three layers, from an ncu capture of the current kernel; None when the kernel
 # has changed since the counters were taken.
 TRAFFIC_PER_LAUNCH = None
+STEPS_PER_GRAPH = 4
 
 
 def _peaks():
@@ -167,25 +168,36 @@ def run_gpu(args, rank, world):
                for L in triple]
     xs = [h.to(dev).view(torch.bfloat16) for h in xs_host]
     ys = [torch.empty((M, L.N), dtype=torch.float32, device=dev) for L in triple]
-    ws = torch.zeros(max(bt.gemv_workspace_bytes(l, M, L.N, L.K) for L in triple for l in (0, 1)),
+    probs_of = lambda reps, r, xs_, ys_: [dict(codes=reps[r][i][0], scales=reps[r][i][1], x=xs_[i], y=ys_[i],  # noqa: E731
+                                               N=L.N, K=L.K) for i, L in enumerate(triple)]
+    ws = torch.empty(max([bt.gemv_workspace_bytes(l, M, L.N, L.K) for L in triple for l in (0, 1)] +
+                         [bt.gemv_batched_workspace_bytes(l, [dict(N=L.N, K=L.K) for L in triple]) for l in (0, 1)]),
                      dtype=torch.uint8, device=dev)
+
+    # Steps are replayed from CUDA graphs of STEPS_PER_GRAPH consecutive steps
+    # (each step its own bt_gemv_batched call on the next weight copy), so the
+    # host's graph launches keep ahead of the device.
+    spg = STEPS_PER_GRAPH if copies % STEPS_PER_GRAPH == 0 else 1
 
     def graphs_for(reps, layout, with_events=False):
         gs = []
         with torch.cuda.stream(stream):
-            for r in range(copies):
-                for i, L in enumerate(triple):  # warm the code path before capture
-                    bt.gemv(reps[r][i][0], reps[r][i][1], xs[i], sign, L.N, layout, out=ys[i], ws=ws)
+            for r in range(copies):  # warm the code path before capture
+                bt.gemv_batched(probs_of(reps, r, xs, ys), sign, layout, ws=ws)
             torch.cuda.synchronize()
-            for r in range(copies):
+            for r0 in range(0, copies, spg):
                 gr = torch.cuda.CUDAGraph()
                 with torch.cuda.graph(gr, stream=stream):
-                    for i, L in enumerate(triple):
-                        bt.gemv(reps[r][i][0], reps[r][i][1], xs[i], sign, L.N, layout, out=ys[i], ws=ws)
+                    for r in range(r0, r0 + spg):
+                        bt.gemv_batched(probs_of(reps, r, xs, ys), sign, layout, ws=ws)
                 gs.append(gr)
         return gs
 
-    def timed(gs, steps, warmup, per_call_events=False):
+    def timed(gs, steps, warmup, per_call_events=False, per_graph=1):
+        """K steps from graphs of `per_graph` steps each (K a multiple of it)."""
+        assert steps % per_graph == 0
+        warmup = -(-warmup // per_graph)
+        steps_r = steps // per_graph
         with torch.cuda.stream(stream):
             for w in range(warmup):
                 gs[w % len(gs)].replay()
@@ -196,23 +208,27 @@ def run_gpu(args, rank, world):
             st = torch.cuda.Event(enable_timing=True)
             en = torch.cuda.Event(enable_timing=True)
             st.record(stream)
-            for k in range(steps):
+            for k in range(steps_r):
                 gs[(warmup + k) % len(gs)].replay()
             en.record(stream)
             torch.cuda.synchronize()
         return max_over_ranks(st.elapsed_time(en) / steps, world, dist, dev)
+
+    if args.steps % spg:
+        spg = 1
 
     # ---- base-3 (headline) ----
     reps3 = build(0)
     gs3 = graphs_for(reps3, 0)
     with ClockSampler(dev.index) as clk:
         time.sleep(0.5)  # let the sampler start before the timed region
-        ms3 = timed(gs3, args.steps, args.warmup)
+        ms3 = timed(gs3, args.steps, args.warmup, per_graph=spg)
     bytes3 = sum(_weight_bytes(L, 0) for L in triple)
     io_bytes = sum(M * L.K * 2 + M * L.N * 4 for L in triple)
 
-    # per-call durations of the dominant call (one bt_gemv: main kernel + chunk reduction),
-    # from a CUDA graph of `copies` calls of one layer over the rotating weight copies
+    # per-call durations of single bt_gemv calls (context: each call is a main
+    # kernel and a reduction), from a CUDA graph of `copies` calls of one layer
+    # over the rotating weight copies
     per_layer_us = []
     with torch.cuda.stream(stream):
         for i, L in enumerate(triple):
@@ -237,8 +253,8 @@ def run_gpu(args, rank, world):
 
     # ---- e2e through the public API with host buffers ----
     # Each step copies the step's activations from pinned host memory, makes
-    # the three bt_gemv calls and reads the outputs back into pinned host
-    # memory. "graph": the step as a serving loop would run it, captured once
+    # the step's bt_gemv_batched call and reads the outputs back into pinned
+    # host memory. "graph": the step as a serving loop would run it, captured once
     # as a CUDA graph of those API calls and copies and replayed per step.
     # "eager": the same calls issued from Python every step.
     # one pinned host buffer per direction: a step is one H2D copy of the three
@@ -257,8 +273,7 @@ def run_gpu(args, rank, world):
 
     def e2e_step(r):
         x_dev_all.copy_(x_host_all, non_blocking=True)
-        for i, L in enumerate(triple):
-            bt.gemv(reps3[r][i][0], reps3[r][i][1], xs_e[i], sign, L.N, 0, out=ys_e[i], ws=ws)
+        bt.gemv_batched(probs_of(reps3, r, xs_e, ys_e), sign, 0, ws=ws)
         y_host_all.copy_(y_dev_all, non_blocking=True)
 
     def e2e_timed(run_step):
@@ -293,7 +308,7 @@ def run_gpu(args, rank, world):
     # ---- 2-bit layout twin ----
     reps2 = build(1)
     gs2 = graphs_for(reps2, 1)
-    ms2 = timed(gs2, args.steps, args.warmup)
+    ms2 = timed(gs2, args.steps, args.warmup, per_graph=spg)
     bytes2 = sum(_weight_bytes(L, 1) for L in triple)
     del gs2, reps2
 
@@ -324,8 +339,11 @@ def run_gpu(args, rank, world):
         fwht = {"error": str(e)[:200]}
 
     gbs = whole_job_rate(bytes3, ms3, world) / 1e9
-    dom_bytes = [(_weight_bytes(L, 0) + M * L.K * 2 + M * L.N * 4) for L in triple]
-    achieved = sum(dom_bytes) / (sum(per_layer_us) * 1e-6) / 1e9
+    # the dominant launch pair is the step's own bt_gemv_batched call: its
+    # algorithmic bytes are the triple's weights and scales plus activations in
+    # and outputs out; its duration is the device time of the step
+    dom_bytes = sum(_weight_bytes(L, 0) + M * L.K * 2 + M * L.N * 4 for L in triple)
+    achieved = dom_bytes / (ms3 * 1e-3) / 1e9
     out = {
         "metric": METRIC,
         "value": round(gbs, 2),
@@ -343,7 +361,8 @@ def run_gpu(args, rank, world):
                                "FWHT-1024 fused",
                    "M": M, "layout": "base-3 5 trits/byte, 26 B + 2 B scale per 128 weights",
                    "l2": f"{copies} distinct weight copies rotated ({copies * bytes3 / 1e6:.0f} MB > 126 MB L2)",
-                   "graph": "each step is one CUDA graph replay of three bt_gemv calls",
+                   "graph": f"each step is one bt_gemv_batched call (the three matrices); {spg} consecutive steps per "
+                            "CUDA graph replay",
                    "parallelism": f"replicas x{world}" if world > 1 else "single GPU"},
         "pct_of_hbm_peak": round(100 * gbs / world / peaks["hbm_gbs"], 2),
         "per_call_us": {L.name: round(u, 2) for L, u in zip(triple, per_layer_us)},
@@ -362,13 +381,14 @@ def run_gpu(args, rank, world):
                           "ms_per_step": round(e2e_eager_ms, 5)}},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 2), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                      "frac": round(achieved / peaks["hbm_gbs"], 4),
-                     # dram__bytes_read.sum + dram__bytes_write.sum of the GEMV kernel per launch, mean
-                     # over the three layers (one ncu capture of this kernel build)
+                     # dram__bytes_read.sum + dram__bytes_write.sum of the table-lookup kernel per
+                     # launch (one ncu capture of this kernel build)
                      "traffic": TRAFFIC_PER_LAUNCH,
-                     "algorithmic_bytes_per_launch": int(sum(dom_bytes) / len(dom_bytes)),
-                     "kernel": "bt_gemv call (table-lookup GEMV kernel + chunk reduction), weighted over the three layers",
+                     "algorithmic_bytes_per_launch": int(dom_bytes),
+                     "kernel": "the step's bt_gemv_batched call: gemv_lut_kernel over the three matrices "
+                               "and gemv_lut_reduce_kernel, timed together (CUDA events on the launching stream)",
                      "peak_kind": f"HBM copy, {peaks['src']}"},
-        "gpu_launches": args.steps * len(triple) * 2,  # GEMV + chunk-sum kernels per bt_gemv call
+        "gpu_launches": args.steps * 2,  # table-lookup kernel + reduction kernel per bt_gemv_batched call
         "clocks": clk.summary(),
     }
     if rank == 0 and not args.no_cpu_baseline:
@@ -453,8 +473,14 @@ def run_fwht_sweep(bt, torch, dev, stream, sign):
 def run_sweep(bt, torch, dev, stream, sign, args, world, dist, layout=0):
     """Decode token through 64 stacks x 2 triples (384 matrices, 26.2e9 weights, 5.7 GB
     base-3 / 7.0 GB 2-bit): one seeded triple generated on the host and cloned on the
-    device to 128 distinct copies at distinct addresses; one token step = 384 bt_gemv
-    calls replayed from CUDA graphs."""
+    device to 128 distinct copies at distinct addresses.
+
+    M = 1: the chained decode step -- each matrix's bf16 output is the next matrix's
+    input (5120 -> 5120 -> 17408 -> 5120 -> 5120 -> ...), as in a layer stack: two
+    bt_gemv_batched calls of 192 chained matrices (the second starts from the first's
+    last output), captured in one CUDA graph per token.
+    M = 4, 16: 384 bt_gemv calls per token, the three activations of the triple reused,
+    replayed from CUDA graphs."""
     import workloads
     triple = workloads.TRIPLE
     uniq = []
@@ -468,12 +494,65 @@ def run_sweep(bt, torch, dev, stream, sign, args, world, dist, layout=0):
     weight_bytes = n_triples * sum(_weight_bytes(L, layout) for L in triple)
     out = {"weights": int(n_triples * sum(L.N * L.K for L in triple)), "bytes_per_token": weight_bytes,
            "matrices": 3 * n_triples}
-    for M in (1, 4, 16):
+
+    def time_graphs(graphs, tokens=3):
+        with torch.cuda.stream(stream):
+            for gr in graphs:
+                gr.replay()
+            torch.cuda.synchronize()
+            if world > 1:
+                dist.barrier()
+            a_ = torch.cuda.Event(enable_timing=True)
+            b_ = torch.cuda.Event(enable_timing=True)
+            a_.record(stream)
+            for _ in range(tokens):
+                for gr in graphs:
+                    gr.replay()
+            b_.record(stream)
+            torch.cuda.synchronize()
+        return max_over_ranks(a_.elapsed_time(b_) / tokens, world, dist, dev)
+
+    # ---- M = 1, chained
+    n_mat = 3 * n_triples
+    per_call = n_mat // 2
+    g = workloads.rng(3 * 1_000_003 + 1000 + 1)
+    x0 = torch.from_numpy(workloads.activations_bf16_bits(g, 1, triple[0].K, True).view(np.int16)).to(dev) \
+        .view(torch.bfloat16)
+    ychain = [torch.empty((1, triple[j % 3].N), dtype=torch.bfloat16, device=dev) for j in range(n_mat)]
+    calls = []
+    for c0 in range(0, n_mat, per_call):
+        probs = []
+        for j in range(c0, c0 + per_call):
+            L = triple[j % 3]
+            p = dict(codes=mats[j // 3][j % 3][0], scales=mats[j // 3][j % 3][1], y=ychain[j], N=L.N, K=L.K)
+            if j == c0:
+                p["x"] = x0 if j == 0 else ychain[j - 1]
+            else:
+                p["x_from"] = j - 1 - c0
+            probs.append(p)
+        calls.append(probs)
+    wsc = torch.empty(max(bt.gemv_batched_workspace_bytes(layout, pr) for pr in calls), dtype=torch.uint8, device=dev)
+    with torch.cuda.stream(stream):
+        for pr in calls:
+            bt.gemv_batched(pr, sign, layout, y_dtype=bt.BF16, ws=wsc)
+        torch.cuda.synchronize()
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=stream):
+            for pr in calls:
+                bt.gemv_batched(pr, sign, layout, y_dtype=bt.BF16, ws=wsc)
+    ms = time_graphs([gr])
+    out["M1"] = {"ms_per_token_step": round(ms, 3), "tokens_per_s": round(whole_job_rate(1, ms, world), 1),
+                 "weight_GB/s": round(whole_job_rate(weight_bytes, ms, world) / 1e9, 1),
+                 "chained": True, "calls_per_token": len(calls)}
+    del gr, wsc, ychain
+
+    # ---- M = 4, 16
+    for M in (4, 16):
         g = workloads.rng(3 * 1_000_003 + 1000 + M)
         xs = [torch.from_numpy(workloads.activations_bf16_bits(g, M, L.K, True).view(np.int16)).to(dev)
               .view(torch.bfloat16) for L in triple]
         ys = [torch.empty((M, L.N), device=dev) for L in triple]
-        ws = torch.zeros(max(bt.gemv_workspace_bytes(layout, M, L.N, L.K) for L in triple), dtype=torch.uint8,
+        ws = torch.empty(max(bt.gemv_workspace_bytes(layout, M, L.N, L.K) for L in triple), dtype=torch.uint8,
                          device=dev)
         graphs = []
         with torch.cuda.stream(stream):
@@ -488,25 +567,12 @@ def run_sweep(bt, torch, dev, stream, sign, args, world, dist, layout=0):
                         for i, L in enumerate(triple):
                             bt.gemv(mats[t][i][0], mats[t][i][1], xs[i], sign, L.N, layout, out=ys[i], ws=ws)
                 graphs.append(gr)
-            for gr in graphs:
-                gr.replay()
-            torch.cuda.synchronize()
-            if world > 1:
-                dist.barrier()
-            a_ = torch.cuda.Event(enable_timing=True)
-            b_ = torch.cuda.Event(enable_timing=True)
-            tokens = 3
-            a_.record(stream)
-            for _ in range(tokens):
-                for gr in graphs:
-                    gr.replay()
-            b_.record(stream)
-            torch.cuda.synchronize()
-        ms = max_over_ranks(a_.elapsed_time(b_) / tokens, world, dist, dev)
+        ms = time_graphs(graphs)
         out[f"M{M}"] = {"ms_per_token_step": round(ms, 3), "tokens_per_s": round(whole_job_rate(M, ms, world), 1),
                         "weight_GB/s": round(whole_job_rate(weight_bytes, ms, world) / 1e9, 1)}
         del graphs
     out["roofline_tokens_per_s_M1"] = round(_peaks()["hbm_gbs"] * 1e9 / weight_bytes, 1)
+    out["M1_frac_of_roofline"] = round(out["M1"]["tokens_per_s"] / world / out["roofline_tokens_per_s_M1"], 4)
     del mats
     return out
 
