@@ -15,7 +15,10 @@ cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales
 size_t gemv_noalloc_max_bytes();
 cudaError_t gemv_noalloc_scratch(void** out);
 size_t gemv1_workspace_bytes(const DecodeProblem* problems, int count);
-bool gemv1_applies(int64_t M, int64_t K, const void* codes, const void* scales);
+bool gemv_lut_applies(int64_t M, int64_t K, const void* codes, const void* scales);
+cudaError_t launch_gemv_lut(int layout, const uint8_t* codes, const uint16_t* scales, const void* x, int x_bf16,
+                            const int8_t* sign, int M, int64_t N, int64_t K, int y_dtype, void* y, void* workspace,
+                            int32_t* dev_err, int num_sms, cudaStream_t stream);
 cudaError_t launch_gemv1(int layout, const DecodeProblem* problems, int count, const int8_t* sign, int y_dtype,
                          void* workspace, int32_t* dev_err, int num_sms, cudaStream_t stream);
 size_t gemm_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num_sms);
@@ -146,15 +149,20 @@ size_t bt_gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K) {
     return bt::gemv_workspace_bytes(layout, M, N, K, current_sm_count());
 }
 
-// One GEMV call on a validated workspace: single rows that TMA can stream
-// take the persistent table-lookup kernel, the rest the kernels of bt_gemv.cu.
+// One GEMV call on a validated workspace: products whose weights TMA can
+// stream take the persistent kernels of bt_gemv_lut.cu (table lookup for
+// M = 1, tensor cores above), the rest the kernels of bt_gemv.cu.
 cudaError_t run_gemv(int layout, const uint8_t* codes, const uint16_t* scales, const void* x, int x_dtype,
                      const int8_t* sign1024, int64_t M, int64_t N, int64_t K, int y_dtype, void* y, void* ws,
                      int32_t* dev_err, int sms, cudaStream_t s) {
-    if (bt::gemv1_applies(M, K, codes, scales)) {
-        bt::DecodeProblem p{codes, scales, x, x_dtype == BT_BF16 ? 1 : 0, -1, y, N, K};
-        return bt::launch_gemv1(layout, &p, 1, sign1024, y_dtype, ws, dev_err, sms, s);
-    }
+    // Base-3 weights at 2 <= M <= 8 stay on the TMA-fed kernel of bt_gemv.cu,
+    // which was measured faster there (27B-equivalent sweep at M = 4); above
+    // M = 8, and for the 2-bit layout, the tensor-core kernel of
+    // bt_gemv_lut.cu streams the weights once for all rows.
+    const bool old_path = layout == BT_LAYOUT_B3 && M >= 2 && M <= 8;
+    if (!old_path && bt::gemv_lut_applies(M, K, codes, scales))
+        return bt::launch_gemv_lut(layout, codes, scales, x, x_dtype == BT_BF16 ? 1 : 0, sign1024, (int)M, N, K,
+                                   y_dtype, y, ws, dev_err, sms, s);
     return bt::launch_gemv(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y_dtype, y, ws, dev_err, sms, s);
 }
 

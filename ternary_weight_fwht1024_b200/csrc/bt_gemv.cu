@@ -1088,17 +1088,15 @@ static GemvPlan make_gemv_plan(int layout, int64_t M, int64_t N, int64_t K, int 
     return pl;
 }
 
-// Single rows that TMA can stream take the table-lookup kernels
-// (bt_gemv_lut.cu); a workspace sized here serves either path.
-size_t gemv1_workspace_bytes(const DecodeProblem* problems, int count);
+// Products whose weights TMA can stream take the kernels of bt_gemv_lut.cu;
+// a workspace sized here serves either path.
+size_t gemv_lut_workspace_bytes(int64_t M, int64_t N, int64_t K);
 
 size_t gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num_sms) {
     size_t need = make_gemv_plan(layout, M, N, K, num_sms).total;
-    if (M == 1 && K % 1024 == 0) {
-        // the single-row kernels' need (alignment of the pointers is not known here)
-        const DecodeProblem p{nullptr, nullptr, nullptr, 1, -1, nullptr, N, K};
-        const size_t one = gemv1_workspace_bytes(&p, 1);
-        if (one > need) need = one;
+    if (K % 1024 == 0) {  // (alignment of the pointers is not known here)
+        const size_t lut = gemv_lut_workspace_bytes(M, N, K);
+        if (lut > need) need = lut;
     }
     return need;
 }

@@ -48,6 +48,7 @@
 #include <algorithm>
 
 #include "bt_internal.cuh"
+#include "bt_slots.cuh"
 
 namespace bt {
 
@@ -105,14 +106,19 @@ struct LutParams {
     float* part;                       // chunk partials of every matrix of the list
     int64_t total_rc;
     int nprob, y_bf16;
+    int M;                             // activation rows (1 for the table-lookup kernel)
+    const void* frag;                  // M > 1: the prep kernel's fragment words and group constants
+    const void* meta;
 };
 static_assert(sizeof(LutParams) <= 4096, "kernel parameters");
 
 // Sums of chunk partials for up to kLutMaxProblems matrices and where they go.
+// Partials of a matrix with M activation rows: [nchunk][ld][M] (a 16-row set
+// of a chunk writes 16 M contiguous floats).
 struct LutReduceParams {
     const float* part[kLutMaxProblems];
     void* y[kLutMaxProblems];
-    int32_t N[kLutMaxProblems], ld[kLutMaxProblems], nchunk[kLutMaxProblems];
+    int32_t N[kLutMaxProblems], ld[kLutMaxProblems], nchunk[kLutMaxProblems], M[kLutMaxProblems];
     int nprob, y_bf16;
 };
 
@@ -128,6 +134,12 @@ __device__ __forceinline__ uint2 lds_u64(uint32_t addr) {
     uint2 v;
     asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(addr) : "memory");
     return v;
+}
+
+__device__ __forceinline__ uint32_t lds_u16(uint32_t addr) {
+    uint16_t r;
+    asm volatile("ld.shared.u16 %0, [%1];" : "=h"(r) : "r"(addr) : "memory");
+    return r;
 }
 
 // Table lookup at a shared-window byte address. The ring reads above carry a
@@ -616,24 +628,375 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_c
     if (L == 0 && bad) report(P.dev_err, bad);
 }
 
-// y of up to 12 matrices, one thread per row: its chunk partials added in
-// chunk order, up to 64 loads in flight together.
-__global__ void __launch_bounds__(kLutReduceThreads) gemv_lut_reduce_kernel(const __grid_constant__ LutReduceParams R) {
+// y of up to 12 matrices, one thread per output: its chunk partials added in
+// chunk order, up to UNROLL loads in flight together.
+template <int UNROLL>
+__global__ void __launch_bounds__(kLutReduceThreads, UNROLL >= 64 ? 1 : 4)
+gemv_lut_reduce_kernel(const __grid_constant__ LutReduceParams R) {
     // the tile's matrix and first row, from the parameters, before the wait
     int q = 0, k = blockIdx.x;
     for (; q < R.nprob; ++q) {
-        const int t = (R.N[q] + kLutReduceThreads - 1) / kLutReduceThreads;
+        const int t = (int)(((int64_t)R.M[q] * R.N[q] + kLutReduceThreads - 1) / kLutReduceThreads);
         if (k < t) break;
         k -= t;
     }
     pdl_wait();
     pdl_launch_dependents();
-    const int n = k * kLutReduceThreads + threadIdx.x;
-    if (q >= R.nprob || n >= R.N[q]) return;
+    if (q >= R.nprob) return;
+    const int64_t idx = (int64_t)k * kLutReduceThreads + threadIdx.x;  // n * M + m: partial (n, m) of a chunk
+    if (idx >= (int64_t)R.M[q] * R.N[q]) return;
+    const int n = (int)(idx / R.M[q]), m = (int)(idx - (int64_t)n * R.M[q]);
     float v[1];
-    lut_row_sums<1, 64>(R.part[q], R.ld[q], R.nchunk[q], n, 0, v);
-    if (R.y_bf16) reinterpret_cast<__nv_bfloat16*>(R.y[q])[n] = __float2bfloat16_rn(v[0]);
-    else reinterpret_cast<float*>(R.y[q])[n] = v[0];
+    lut_row_sums<1, UNROLL>(R.part[q], (int64_t)R.M[q] * R.ld[q], R.nchunk[q], (int)idx, 0, v);
+    const int64_t yi = (int64_t)m * R.N[q] + n;
+    if (R.y_bf16) reinterpret_cast<__nv_bfloat16*>(R.y[q])[yi] = __float2bfloat16_rn(v[0]);
+    else reinterpret_cast<float*>(R.y[q])[yi] = v[0];
+}
+
+// ------------------------------------------------- M = 2..16: tensor cores ----
+//
+// Several activation rows share every weight byte, so the bytes are decoded
+// once into FP16 digit fields (bt_slots.cuh) and multiplied on the tensor
+// cores (m16n8k16: 16 weight rows x 16 k by 8 activation rows, two n8 blocks
+// for M > 8) instead of being looked up per row. A prep kernel rotates x and
+// writes, per 128-group and activation row, the fragment words in slot order
+// and the group constants; the main kernel keeps the table-lookup kernel's
+// work split, TMA ring and chunk partials, and copies each segment's chunk of
+// fragments into shared memory (the next one while it streams the current).
+
+template <int LAYOUT>
+struct MmaGeom {
+    static constexpr int NT = LAYOUT == BT_LAYOUT_B3 ? kB3Mmas : k2bMmas;
+    static constexpr int kCBox = LAYOUT == BT_LAYOUT_B3 ? kLutCBoxB3 : kLutCBox2b;
+    static constexpr int kSlot = kLutSet * kCBox + kLutSet * 16;
+    static constexpr int kLut = LAYOUT == BT_LAYOUT_B3 ? kB3LutBytes : 0;      // decode table
+    static constexpr int kRing = kLut;
+    // per chunk: fragment words [4 q][NT t][M m][4 c][2 hp] (the 32 lanes of a
+    // load, m = lane / 4, c = lane % 4, read 256 contiguous bytes) and group
+    // constants [4 q][M m] (corr, 2^e); two buffers
+    static constexpr int kFragBytes = 4 * NT * 16 * 32;
+    static constexpr int kMetaBytes = 4 * 16 * 8;
+    static constexpr int kBuf = kRing + kLutWarps * kLutDepth * kSlot;
+    static constexpr int kBufBytes = kFragBytes + kMetaBytes;
+    static constexpr int kBar = kBuf + 2 * kBufBytes;
+    static constexpr int kSmem = kBar + kLutWarps * kLutDepth * 8;
+    static_assert(kRing % 128 == 0 && kSlot % 128 == 0, "ring slots are TMA destinations");
+    static_assert(kBuf % 16 == 0 && kBufBytes % 16 == 0, "16-byte asynchronous copies land in the buffers");
+    static_assert(kSmem <= 227 * 1024, "one CTA per SM");
+};
+
+struct MmaLut {  // the decode table at the start of dynamic shared memory
+    __device__ __forceinline__ static uint32_t ld(uint32_t off) { return lds_u32(smem_addr(lut_smem) + off); }
+};
+
+// The k (0..127, or -1: empty) and digit field of every half of a group's
+// activation fragment words, word w = 8 t + 2 c + hp, half u: the slot maps of
+// bt_slots.cuh tabulated once at compile time.
+struct SlotTable {
+    int8_t k[2][kB3Mmas * 8 * 2];
+    int8_t f[2][kB3Mmas * 8 * 2];
+};
+constexpr SlotTable make_slot_table() {
+    SlotTable T{};
+    for (int l = 0; l < 2; ++l)
+        for (int w = 0; w < kB3Mmas * 8; ++w)
+            for (int u = 0; u < 2; ++u) {
+                const int t = w / 8, c = (w % 8) / 2, hp = w % 2;
+                int field = 0, k = -1;
+                if (l == 0) k = b3_slot(t, c, 2 * hp + u, &field);
+                else if (t < k2bMmas) k = tb_slot(t, c, 2 * hp + u, &field);
+                T.k[l][2 * w + u] = static_cast<int8_t>(k);
+                T.f[l][2 * w + u] = static_cast<int8_t>(k >= 0 ? field : 0);
+            }
+    return T;
+}
+static __constant__ SlotTable c_slots = make_slot_table();
+
+// Activation fragments and group constants of row m, group q of the chunk
+// (the chunk's 128 x' values at xg), by one warp: per-group exponent e from
+// the largest |x'|, fragment words FP16(x' 2^(24 - 2i - e)) in slot order
+// (every lane writes some of the NT * 8 words), and corr = 2^e times the
+// tensor-core sum with every digit 1, by the same MMA chain the stream runs,
+// so zero trits give exactly 0.
+// dst: the word (t = 0, c = 0, hp = 0) of this group and row; word (t, c, hp)
+// at dst[t * tstride + c * 2 + hp]. tab: (k, field) pairs of the slot table.
+template <int LAYOUT>
+__device__ __forceinline__ void mma_build_group(const float* xg, uint32_t* dst, int tstride, float2* meta,
+                                                const int8_t* tab) {
+    constexpr int NT = MmaGeom<LAYOUT>::NT;
+    const int lane = threadIdx.x & 31;
+    float amax = 0.f;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) amax = fmaxf(amax, fabsf(xg[32 * r + lane]));
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, s));
+    int E = amax > 0.f ? ilogbf(amax) + 1 : -100;  // amax < 2^E
+    E = max(-100, min(100, E));
+    const int e = 9 + E;
+#pragma unroll
+    for (int w = lane; w < NT * 8; w += 32) {  // w = 8 t + 2 c + hp
+        uint32_t word = 0;
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int k = tab[4 * w + 2 * u], i = tab[4 * w + 2 * u + 1];
+            if (k >= 0) {
+                const __half hv = __float2half_rn(xg[k] * exp2i(24 - 2 * i - e));
+                word |= static_cast<uint32_t>(__half_as_ushort(hv)) << (16 * u);
+            }
+        }
+        dst[(w >> 3) * tstride + (w & 7)] = word;
+    }
+    __syncwarp();
+    uint32_t bf[NT][2];
+#pragma unroll
+    for (int t = 0; t < NT; ++t)
+#pragma unroll
+        for (int hp = 0; hp < 2; ++hp) bf[t][hp] = lane < 4 ? dst[t * tstride + lane * 2 + hp] : 0u;  // column 0
+    uint32_t Rg[16], Rh[16];
+    float d[4];
+    if constexpr (LAYOUT == BT_LAYOUT_B3) {
+        uint32_t QG[3], QH[3];
+        b3_ones_tile(lane & 3, Rg, Rh, QG, QH);
+        b3_group_mma(Rg, Rh, QG, QH, bf, d);
+    } else {
+        tb_ones_tile(Rg, Rh);
+        tb_group_mma(Rg, Rh, bf, d);
+    }
+    if (lane == 0) *meta = make_float2(d[0] * exp2i(e), exp2i(e));
+}
+
+// Prep: one CTA of 8 warps per (activation row m, 1024-block b). Warp 0
+// rotates the block (S, then H_1024 / 32) or copies it when x is already
+// rotated; warp q then writes group 8 b + q's fragment words and constants.
+// Output layout, per 128-group g: words [g][NT][M][4][2], constants [g][M].
+struct MmaPrepArgs {
+    const void* x;
+    const int8_t* sign;  // NULL: x already rotated
+    uint32_t* frag;
+    float2* meta;
+    int x_bf16, M, K;
+};
+
+template <int LAYOUT>
+__global__ void __launch_bounds__(256) gemv_mma_prep_kernel(const MmaPrepArgs a) {
+    constexpr int NT = MmaGeom<LAYOUT>::NT;
+    __shared__ __align__(16) float xs[32 * kTileStride];
+    __shared__ int8_t tab[NT * 8 * 2 * 2];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nblk = a.K / kBlock;
+    const int m = blockIdx.x / nblk, b = blockIdx.x % nblk;
+    if (threadIdx.x < NT * 8 * 2) {
+        constexpr int lt = LAYOUT == BT_LAYOUT_B3 ? 0 : 1;
+        tab[2 * threadIdx.x] = c_slots.k[lt][threadIdx.x];
+        tab[2 * threadIdx.x + 1] = c_slots.f[lt][threadIdx.x];
+    }
+    pdl_wait();  // x may be the previous kernel's output
+    pdl_launch_dependents();
+    if (warp == 0) {
+        float v[32];
+        const int64_t off = (int64_t)m * a.K + (int64_t)b * kBlock;
+        if (a.sign) {
+            load_signed_bf16_block(static_cast<const uint16_t*>(a.x) + off, a.sign, v);
+            fwht1024_warp(v, xs);
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < 32; ++j) xs[32 * j + lane] = v[j];  // lane holds element 32 j + lane
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const int64_t i = off + 32 * j + lane;
+                xs[32 * j + lane] = a.x_bf16 ? bf16_bits_to_f32(static_cast<const uint16_t*>(a.x)[i])
+                                             : static_cast<const float*>(a.x)[i];
+            }
+        }
+    }
+    __syncthreads();
+    const int g = 8 * b + warp;
+    mma_build_group<LAYOUT>(xs + kGroup * warp, a.frag + ((int64_t)g * NT * a.M + m) * 8, a.M * 8,
+                            a.meta + (int64_t)g * a.M + m, tab);
+}
+
+template <int LAYOUT, int NB, bool CHECK>
+__global__ void __launch_bounds__(kLutThreads, 1) gemv_mma_kernel(const __grid_constant__ LutParams P) {
+    using GE = MmaGeom<LAYOUT>;
+    constexpr int NT = GE::NT;
+    const int warp = threadIdx.x >> 5, L = threadIdx.x & 31;
+    const int g = L >> 2, c = L & 3;
+    const int M = P.M;
+    const int CB = LAYOUT == BT_LAYOUT_B3 ? 4 * kB3GroupBytes : 4 * k2bGroupBytes;  // bytes per chunk row
+    LutRing rg;
+    rg.cbox = GE::kCBox;
+    rg.slot_bytes = GE::kSlot;
+    rg.ring = smem_addr(lut_smem + GE::kRing) + warp * kLutDepth * rg.slot_bytes;
+    rg.bar = smem_addr(lut_smem + GE::kBar) + warp * kLutDepth * 8;
+    const uint32_t buf_s = smem_addr(lut_smem + GE::kBuf);
+    // words and constants of a chunk, in global memory: contiguous
+    const int fwords = 4 * NT * M * 8, mbytes = 4 * M * 8;
+    const uint32_t* frag = reinterpret_cast<const uint32_t*>(P.frag);
+    const float2* gmeta = reinterpret_cast<const float2*>(P.meta);
+    // all threads: the chunk c's fragments and constants into buffer `bi`
+    auto fetch_chunk = [&](int chunk, int bi) {
+        const uint32_t dst = buf_s + bi * GE::kBufBytes;
+        const uint8_t* src = reinterpret_cast<const uint8_t*>(frag + (int64_t)chunk * fwords);
+        for (int i = threadIdx.x; i < fwords / 4; i += kLutThreads) cp_async16(dst + 16 * i, src + 16 * i);
+        const uint8_t* msrc = reinterpret_cast<const uint8_t*>(gmeta + (int64_t)chunk * 4 * M);
+        for (int i = threadIdx.x; i < mbytes / 16; i += kLutThreads)
+            cp_async16(dst + GE::kFragBytes + 16 * i, msrc + 16 * i);
+        cp_async_commit();
+    };
+
+    if (L == 0) {
+        for (int d = 0; d < kLutDepth; ++d) mbar_init(rg.bar + 8 * d, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncwarp();
+    if constexpr (LAYOUT == BT_LAYOUT_B3) b3_lut_fill(lut_smem, threadIdx.x, kLutThreads);
+
+    const int64_t rc0 = P.total_rc * blockIdx.x / gridDim.x;
+    const int64_t rc1 = P.total_rc * (blockIdx.x + 1) / gridDim.x;
+    uint32_t issued = 0, done = 0;
+    bool ok = true;
+    LutSeg is;
+    int64_t irc = rc0;
+    int iq = 0;
+    bool ihave = lut_next_seg(P, irc, rc1, is);
+    auto warp_sets = [&](const LutSeg& sgm) {
+        const int nsets = (sgm.n1 - sgm.n0 + kLutSet - 1) / kLutSet;
+        return warp < nsets ? (nsets - warp + kLutWarps - 1) / kLutWarps : 0;
+    };
+    auto issue_next = [&]() {
+        while (ihave && iq >= warp_sets(is)) {
+            ihave = lut_next_seg(P, irc, rc1, is);
+            iq = 0;
+        }
+        if (!ihave) return;
+        if (L == 0) {
+            const int cb = is.c * CB;
+            lut_issue_set(rg, &P.cmap[is.p], &P.smap[is.p], issued, cb & ~15, (4 * is.c) & ~7,
+                          is.n0 + (int64_t)kLutSet * (warp + kLutWarps * iq));
+        }
+        ++iq;
+        ++issued;
+    };
+    for (int d = 0; d < kLutDepth; ++d) issue_next();
+    int64_t rc = rc0;
+    LutSeg sg;
+    bool have = lut_next_seg(P, rc, rc1, sg);
+    uint32_t mG[3] = {0u, 0u, 0u}, mH[3] = {0u, 0u, 0u};
+    if constexpr (LAYOUT == BT_LAYOUT_B3) b3_pair12_masks(c, mG, mH);
+    const uint32_t lane4 = static_cast<uint32_t>(L) * 4u;
+
+    pdl_wait();  // the prep kernel's fragments
+    pdl_launch_dependents();
+
+    uint32_t err = 0;
+    int bad = 0;
+    int bi = 0;
+    if (have) fetch_chunk(sg.c, 0);
+    while (have) {
+        const LutProblem& pr = P.p[sg.p];
+        const int n0 = sg.n0, n1 = sg.n1;
+        float* part = P.part + pr.part_base + (int64_t)sg.c * M * pr.ld;
+        const int coff = (sg.c * CB) & 15;
+        const int soff = 2 * ((4 * sg.c) & 7);
+        const int my = warp_sets(sg);
+        cp_async_wait_all();
+        __syncthreads();  // this chunk's fragments are in buffer bi; the other buffer is free
+        LutSeg nx;
+        int64_t nrc = rc;
+        const bool nhave = lut_next_seg(P, nrc, rc1, nx);
+        if (nhave) fetch_chunk(nx.c, bi ^ 1);  // overlaps this segment's stream
+        const uint32_t slots_s = buf_s + bi * GE::kBufBytes, meta_s = slots_s + GE::kFragBytes;
+
+        for (int qs = 0; qs < my && ok; ++qs) {
+            const uint32_t n = done;
+            const uint32_t d = n % kLutDepth;
+            if (!lut_wait(rg.bar + 8 * d, (n / kLutDepth) & 1u)) {
+                ok = false;
+                bad |= BT_DEVERR_TIMEOUT;
+                break;
+            }
+            ++done;
+            const uint32_t cs = rg.ring + d * rg.slot_bytes + coff;       // row 0 of the chunk in the slot
+            const uint32_t ss = rg.ring + d * rg.slot_bytes + kLutSet * rg.cbox + soff;
+            const uint32_t rowg = cs + g * rg.cbox, rowh = cs + (g + 8) * rg.cbox;
+            float acc[NB][4];
+#pragma unroll
+            for (int b = 0; b < NB; ++b) acc[b][0] = acc[b][1] = acc[b][2] = acc[b][3] = 0.f;
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                uint32_t Rg[16], Rh[16], QG[3], QH[3];
+                if constexpr (LAYOUT == BT_LAYOUT_B3) {
+                    // the lane's bytes 6c .. 6c + 5 of group q, from the aligned word below them
+                    const uint32_t Ag = rowg + q * kB3GroupBytes + 6 * c, Ah = rowh + q * kB3GroupBytes + 6 * c;
+                    const uint32_t o8 = (Ag & 3u) * 8u;  // rows are 112 B apart: the same shift for both
+                    const uint32_t w12 = lds_u16(cs + (c < 2 ? g : g + 8) * rg.cbox + q * kB3GroupBytes + 24);
+                    b3_decode_tile<CHECK, MmaLut>(lds_u32(Ag & ~3u), lds_u32((Ag & ~3u) + 4), lds_u32(Ah & ~3u),
+                                                  lds_u32((Ah & ~3u) + 4), w12, o8, lane4, mG, mH, Rg, Rh, QG, QH,
+                                                  err);
+                } else {
+                    const uint2 x0 = lds_u64(rowg + q * k2bGroupBytes + 8 * c);
+                    const uint2 x1 = lds_u64(rowh + q * k2bGroupBytes + 8 * c);
+                    tb_decode_tile<CHECK>(x0, x1, Rg, Rh, err);
+#pragma unroll
+                    for (int k = 0; k < 3; ++k) QG[k] = QH[k] = 0u;
+                }
+                const float sgv = f16_bits_to_f32(lds_u16(ss + g * 16 + 2 * q));
+                const float shv = f16_bits_to_f32(lds_u16(ss + (g + 8) * 16 + 2 * q));
+#pragma unroll
+                for (int b = 0; b < NB; ++b) {
+                    const int m = 8 * b + g;  // this lane's activation row in the B fragment
+                    uint32_t bf[NT][2];
+                    const uint32_t ba = slots_s + (uint32_t)(((q * NT) * M + m) * 32 + c * 8);
+#pragma unroll
+                    for (int t = 0; t < NT; ++t) {
+                        uint2 v = make_uint2(0u, 0u);
+                        if (m < M) v = lds_u64(ba + (uint32_t)(t * M * 32));
+                        bf[t][0] = v.x;
+                        bf[t][1] = v.y;
+                    }
+                    float d4[4];
+                    if constexpr (LAYOUT == BT_LAYOUT_B3) b3_group_mma(Rg, Rh, QG, QH, bf, d4);
+                    else tb_group_mma(Rg, Rh, bf, d4);
+                    // D columns 2c, 2c + 1 of this block are activation rows 8 b + 2c (+1)
+                    const int m0 = 8 * b + 2 * c;
+                    const uint2 md0 = m0 < M ? lds_u64(meta_s + (uint32_t)((q * M + m0) * 8)) : make_uint2(0u, 0u);
+                    const uint2 md1 = m0 + 1 < M ? lds_u64(meta_s + (uint32_t)((q * M + m0 + 1) * 8))
+                                                 : make_uint2(0u, 0u);
+                    const float c0 = __uint_as_float(md0.x), p0 = __uint_as_float(md0.y);
+                    const float c1 = __uint_as_float(md1.x), p1 = __uint_as_float(md1.y);
+                    acc[b][0] = fmaf(sgv, fmaf(d4[0], p0, -c0), acc[b][0]);
+                    acc[b][1] = fmaf(sgv, fmaf(d4[1], p1, -c1), acc[b][1]);
+                    acc[b][2] = fmaf(shv, fmaf(d4[2], p0, -c0), acc[b][2]);
+                    acc[b][3] = fmaf(shv, fmaf(d4[3], p1, -c1), acc[b][3]);
+                }
+            }
+            __syncwarp();
+            issue_next();  // into the slot just freed
+            const int r0 = n0 + kLutSet * (warp + kLutWarps * qs);
+#pragma unroll
+            for (int b = 0; b < NB; ++b) {
+                const int m0 = 8 * b + 2 * c;
+#pragma unroll
+                for (int r = 0; r < 4; ++r) {
+                    const int m = m0 + (r & 1), row = r0 + g + 8 * (r >> 1);
+                    if (m < M && row < n1) part[(int64_t)row * M + m] = acc[b][r];
+                }
+            }
+        }
+        sg = nx;
+        rc = nrc;
+        have = nhave;
+        bi ^= 1;
+    }
+    for (; done < issued; ++done) lut_wait(rg.bar + 8 * (done % kLutDepth), (done / kLutDepth) & 1u);
+    cp_async_wait_all();
+    if (CHECK) {
+        if (LAYOUT == BT_LAYOUT_B3) { if (err >> 31) bad |= BT_DEVERR_INVALID_CODE; }
+        else if (err & 0x55555555u) bad |= BT_DEVERR_INVALID_CODE;
+    }
+    bad = __reduce_or_sync(0xffffffffu, bad);
+    if (L == 0 && bad) report(P.dev_err, bad);
 }
 
 // ---------------------------------------------------------------- host ----
@@ -670,22 +1033,32 @@ size_t gemv1_workspace_bytes(const DecodeProblem* pr, int count) {
     return std::max(total, (size_t)256);
 }
 
-// Single rows whose weights TMA can stream: K a multiple of 1024 (so the
-// scale rows are whole 16-byte units), 16-byte aligned codes and scales.
-bool gemv1_applies(int64_t M, int64_t K, const void* codes, const void* scales) {
-    return M == 1 && K > 0 && K % kBlock == 0 && (reinterpret_cast<uintptr_t>(scales) & 15) == 0 &&
+// Products whose weights TMA can stream: K a multiple of 1024 (so the scale
+// rows are whole 16-byte units), 16-byte aligned codes and scales.
+bool gemv_lut_applies(int64_t M, int64_t K, const void* codes, const void* scales) {
+    return M >= 1 && M <= 16 && K > 0 && K % kBlock == 0 && (reinterpret_cast<uintptr_t>(scales) & 15) == 0 &&
            (reinterpret_cast<uintptr_t>(codes) & 15) == 0;
 }
 
-template <int LAYOUT, bool CHECK>
-static cudaError_t lut_launch_t(const LutParams& P, int grid, cudaStream_t stream) {
-    auto kern = gemv_lut_kernel<LAYOUT, CHECK>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kLutSmem);
+// Workspace of one product with M activation rows: for M > 1 the prep
+// kernel's fragment words (M x K/128 x 9 x 32 bytes) and group constants
+// (M x K/128 x 8 bytes) first, then the partials [K/512][N rounded up to 4][M].
+static size_t mma_frag_bytes(int64_t M, int64_t K) { return lut_align((size_t)M * (K / kGroup) * kB3Mmas * 32, 256); }
+static size_t mma_meta_bytes(int64_t M, int64_t K) { return lut_align((size_t)M * (K / kGroup) * 8, 256); }
+
+size_t gemv_lut_workspace_bytes(int64_t M, int64_t N, int64_t K) {
+    const size_t part = lut_align((size_t)(K / kLutChunk) * (size_t)M * (size_t)((N + 3) & ~3) * sizeof(float), 256);
+    return std::max((M > 1 ? mma_frag_bytes(M, K) + mma_meta_bytes(M, K) : 0) + part, (size_t)256);
+}
+
+template <class Kern>
+static cudaError_t lut_launch_k(Kern kern, int smem, const LutParams& P, int grid, cudaStream_t stream) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(grid);
     cfg.blockDim = dim3(kLutThreads);
-    cfg.dynamicSmemBytes = kLutSmem;
+    cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -696,11 +1069,20 @@ static cudaError_t lut_launch_t(const LutParams& P, int grid, cudaStream_t strea
 }
 
 // The partials and outputs of one group, as the reduction reads them.
-// The main kernel of group [first, first + count). base[i]: offset in floats
-// of matrix i's partials in the workspace `part`.
+template <int LAYOUT, bool CHECK>
+static cudaError_t lut_launch_t(const LutParams& P, int grid, cudaStream_t stream) {
+    if (P.M == 1) return lut_launch_k(gemv_lut_kernel<LAYOUT, CHECK>, kLutSmem, P, grid, stream);
+    if (P.M <= 8) return lut_launch_k(gemv_mma_kernel<LAYOUT, 1, CHECK>, MmaGeom<LAYOUT>::kSmem, P, grid, stream);
+    return lut_launch_k(gemv_mma_kernel<LAYOUT, 2, CHECK>, MmaGeom<LAYOUT>::kSmem, P, grid, stream);
+}
+
+// The main kernel of group [first, first + count), M activation rows (M > 1:
+// one matrix). base[i]: offset in floats of matrix i's partials in the
+// workspace `part`.
 static cudaError_t lut_launch_group(int layout, const DecodeProblem* all, const int64_t* base, int first, int count,
-                                    const int8_t* sign, int y_bf16, float* part, int32_t* dev_err, int num_sms,
-                                    cudaStream_t stream) {
+                                    int M, const int8_t* sign, int y_bf16, float* part, int32_t* dev_err,
+                                    int num_sms, cudaStream_t stream, const void* frag = nullptr,
+                                    const void* meta = nullptr) {
     EncodeTiledFn enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
     LutParams P{};
@@ -749,6 +1131,9 @@ static cudaError_t lut_launch_group(int layout, const DecodeProblem* all, const 
     P.total_rc = rc;
     P.nprob = count;
     P.y_bf16 = y_bf16;
+    P.M = M;
+    P.frag = frag;
+    P.meta = meta;
     // one CTA per SM, never more CTAs than (chunk, row) items
     const int grid = (int)(rc < num_sms ? rc : num_sms);
     if (layout == BT_LAYOUT_B3)
@@ -759,8 +1144,8 @@ static cudaError_t lut_launch_group(int layout, const DecodeProblem* all, const 
 }
 
 // Outputs of matrices [first, first + count), count <= kLutMaxProblems.
-static cudaError_t lut_launch_reduce(const DecodeProblem* all, const int64_t* base, int first, int count, int y_bf16,
-                                     float* part, cudaStream_t stream) {
+static cudaError_t lut_launch_reduce(const DecodeProblem* all, const int64_t* base, int first, int count, int M,
+                                     int y_bf16, float* part, cudaStream_t stream) {
     LutReduceParams R{};
     R.nprob = count;
     R.y_bf16 = y_bf16;
@@ -772,7 +1157,8 @@ static cudaError_t lut_launch_reduce(const DecodeProblem* all, const int64_t* ba
         R.N[i] = static_cast<int32_t>(s.N);
         R.ld[i] = static_cast<int32_t>((s.N + 3) & ~3);
         R.nchunk[i] = static_cast<int32_t>(s.K / kLutChunk);
-        tiles += (int)((s.N + kLutReduceThreads - 1) / kLutReduceThreads);
+        R.M[i] = M;
+        tiles += (int)((M * s.N + kLutReduceThreads - 1) / kLutReduceThreads);
     }
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3((unsigned)tiles);
@@ -783,7 +1169,10 @@ static cudaError_t lut_launch_reduce(const DecodeProblem* all, const int64_t* ba
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    return cudaLaunchKernelEx(&cfg, gemv_lut_reduce_kernel, R);
+    // single rows: few outputs, every load of a row in flight at once; several
+    // rows: many outputs, four CTAs per SM
+    return M == 1 ? cudaLaunchKernelEx(&cfg, gemv_lut_reduce_kernel<64>, R)
+                  : cudaLaunchKernelEx(&cfg, gemv_lut_reduce_kernel<16>, R);
 }
 
 // A list runs as one main kernel per group (a matrix that reads an output of
@@ -808,11 +1197,49 @@ cudaError_t launch_gemv1(int layout, const DecodeProblem* problems, int count, c
     cudaError_t err = cudaSuccess;
     lut_for_each_launch(problems, count, [&](int first, int n) {
         if (err == cudaSuccess)
-            err = lut_launch_group(layout, problems, base, first, n, sign, y_bf16, part, dev_err, num_sms, stream);
+            err = lut_launch_group(layout, problems, base, first, n, 1, sign, y_bf16, part, dev_err, num_sms, stream);
     });
     for (int first = 0; first < count && err == cudaSuccess; first += kLutMaxProblems)
-        err = lut_launch_reduce(problems, base, first, std::min(kLutMaxProblems, count - first), y_bf16, part, stream);
+        err = lut_launch_reduce(problems, base, first, std::min(kLutMaxProblems, count - first), 1, y_bf16, part,
+                                stream);
     return err;
+}
+
+// One product with 1 <= M <= 16 activation rows (x [M][K], y [M][N]): the
+// table-lookup kernel for M = 1, the tensor-core kernel above it, then the
+// reduction.
+cudaError_t launch_gemv_lut(int layout, const uint8_t* codes, const uint16_t* scales, const void* x, int x_bf16,
+                            const int8_t* sign, int M, int64_t N, int64_t K, int y_dtype, void* y, void* workspace,
+                            int32_t* dev_err, int num_sms, cudaStream_t stream) {
+    const DecodeProblem p{codes, scales, x, x_bf16, -1, y, N, K};
+    const int64_t base[1] = {0};
+    const int y_bf16 = y_dtype == BT_BF16;
+    uint8_t* ws = static_cast<uint8_t*>(workspace);
+    void* frag = nullptr;
+    void* meta = nullptr;
+    if (M > 1) {
+        frag = ws;
+        meta = ws + mma_frag_bytes(M, K);
+        ws += mma_frag_bytes(M, K) + mma_meta_bytes(M, K);
+        MmaPrepArgs a{x, sign, static_cast<uint32_t*>(frag), static_cast<float2*>(meta), x_bf16, M, (int)K};
+        cudaLaunchConfig_t cfg{};
+        cfg.gridDim = dim3((unsigned)(M * (K / kBlock)));
+        cfg.blockDim = dim3(256);
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        const cudaError_t e = layout == BT_LAYOUT_B3 ? cudaLaunchKernelEx(&cfg, gemv_mma_prep_kernel<BT_LAYOUT_B3>, a)
+                                                     : cudaLaunchKernelEx(&cfg, gemv_mma_prep_kernel<BT_LAYOUT_2BIT>, a);
+        if (e != cudaSuccess) return e;
+    }
+    float* part = reinterpret_cast<float*>(ws);
+    cudaError_t err = lut_launch_group(layout, &p, base, 0, 1, M, sign, y_bf16, part, dev_err, num_sms, stream,
+                                       frag, meta);
+    if (err != cudaSuccess) return err;
+    return lut_launch_reduce(&p, base, 0, 1, M, y_bf16, part, stream);
 }
 
 }  // namespace bt

@@ -25,7 +25,7 @@ __host__ __device__ constexpr uint32_t fmask(int i) {
     return (3u << (2 * i)) | (3u << (2 * i + 16));
 }
 
-__device__ __forceinline__ int b3_slot(int t, int c, int h, int* field) {
+__host__ __device__ constexpr int b3_slot(int t, int c, int h, int* field) {
     // lane c decodes byte pairs 3c, 3c+1, 3c+2 (bytes 6c..6c+5) into registers
     // rho = 5 q + i; pair 12 (bytes 24, 25) is shared by lanes c (fields
     // {0,1,2} for even c, {3,4} for odd c) and appears as registers Q0..Q2.
@@ -47,7 +47,7 @@ __device__ __forceinline__ int b3_slot(int t, int c, int h, int* field) {
     return k;
 }
 
-__device__ __forceinline__ int tb_slot(int t, int c, int h, int* field) {
+__host__ __device__ constexpr int tb_slot(int t, int c, int h, int* field) {
     // lane c holds bytes 8c..8c+7 = two words of 16 trits; register
     // rho = 8 w + f holds trits f and 8 + f of word w (f < 6 directly, f = 6, 7
     // after a 12-bit shift, then as field f - 6).
