@@ -34,10 +34,11 @@ import numpy as np  # noqa: E402
 
 METRIC = "packed-ternary GEMV weight GB/s (% of HBM peak); pp512 GEMM TFLOP/s"
 L2_BYTES = 126 * 1024 * 1024
-# DRAM bytes (read + write) per launch of the timed GEMV kernel, mean over the
-# three layers, from an ncu capture of the current kernel; None when the kernel
+# DRAM bytes (read + write) per launch of the table-lookup kernel over the
+# decode triple (one bt_gemv_batched call), from an ncu capture of the current
+# kernel (dram__bytes_read.sum + dram__bytes_write.sum); None when the kernel
 # has changed since the counters were taken.
-TRAFFIC_PER_LAUNCH = None
+TRAFFIC_PER_LAUNCH = 44_844_288
 STEPS_PER_GRAPH = 4
 
 
