@@ -28,6 +28,7 @@ _lib = None
 
 LAYOUT_BASE3 = 0
 LAYOUT_2BIT = 1
+LAYOUT_BASE3_CONT = 2
 GROUP = 128
 BLOCK = 1024
 
@@ -55,6 +56,8 @@ def _load():
             P = ctypes.c_void_p
             I64 = ctypes.c_int64
             lib.oracle_bytes_per_group.argtypes = [ctypes.c_int]
+            lib.oracle_row_bytes.argtypes = [ctypes.c_int, I64]
+            lib.oracle_row_bytes.restype = I64
             lib.oracle_pack.argtypes = [ctypes.c_int, P, I64, I64, P]
             lib.oracle_unpack.argtypes = [ctypes.c_int, P, I64, I64, P]
             lib.oracle_hadamard.argtypes = [I64, P]
@@ -99,10 +102,19 @@ def bytes_per_group(layout: int) -> int:
     return _load().oracle_bytes_per_group(layout)
 
 
+def row_bytes(layout: int, K: int) -> int:
+    """Bytes of one packed row: K/128 groups of 26 (base-3) or 32 (2-bit), or
+    ceil(K/5) rounded up to 16 (continuous base-3)."""
+    return int(_load().oracle_row_bytes(layout, K))
+
+
 def pack(trits: np.ndarray, layout: int = LAYOUT_BASE3) -> np.ndarray:
     t = np.ascontiguousarray(trits, dtype=np.int8)
     N, K = t.shape
-    codes = np.zeros((N, (K // GROUP) * bytes_per_group(layout)), dtype=np.uint8)
+    rb = row_bytes(layout, K)
+    if rb < 0:
+        _check(BAD_SHAPE, "pack")
+    codes = np.zeros((N, rb), dtype=np.uint8)
     _check(_load().oracle_pack(layout, _ptr(t), N, K, _ptr(codes)), "pack")
     return codes
 

@@ -18,6 +18,15 @@
  *    group's last 3 trits and two zero-valued pad trits (digit 1).
  *    The plain 2-bit layout stores digit t+1 in bits [2i, 2i+1] of byte
  *    i/4, 32 bytes per group; digit 3 is invalid.
+ *    The continuous base-3 layout packs a row's trits five to a byte with no
+ *    break at group boundaries (byte j holds trits 5j .. 5j+4 of the row, so
+ *    a byte may hold trits of two groups): ceil(K/5) bytes, the last byte's
+ *    trits past K are pads (digit 1), and the row is padded with zero bytes
+ *    to a multiple of 16 bytes. This is the accounting behind the release
+ *    summary's 1.72 bit for ternary + g128 (section 三值权重怎么压缩到 1.76
+ *    bit): 8/5 bit per trit plus 16/128 for the scales, 1.725 bit at
+ *    K = 5120; the per-group layout above spends 26 + 2 bytes per 128
+ *    weights, 1.75 bit.
  *
  *  - oracle_hadamard: H[i][j] = (-1)^popcount(i & j), the closed form of the
  *    Sylvester recursion H_2n = [[H, H], [H, -H]] printed (with H4) in the
@@ -63,7 +72,7 @@
 #define ORACLE_GROUP 128
 #define ORACLE_BLOCK 1024
 
-enum { ORACLE_LAYOUT_BASE3 = 0, ORACLE_LAYOUT_2BIT = 1 };
+enum { ORACLE_LAYOUT_BASE3 = 0, ORACLE_LAYOUT_2BIT = 1, ORACLE_LAYOUT_BASE3_CONT = 2 };
 
 enum {
     ORACLE_OK = 0,
@@ -126,9 +135,68 @@ static int pow3(int i)
     return p;
 }
 
+/* bytes of one packed row */
+int64_t oracle_row_bytes(int layout, int64_t K)
+{
+    if (K % ORACLE_GROUP != 0 || K < 0) return -1;
+    if (layout == ORACLE_LAYOUT_BASE3_CONT) {
+        int64_t used = (K + 4) / 5;
+        return (used + 15) / 16 * 16;
+    }
+    int bpg = oracle_bytes_per_group(layout);
+    return bpg < 0 ? -1 : K / ORACLE_GROUP * bpg;
+}
+
+static int pack_cont(const int8_t* trits, int64_t N, int64_t K, uint8_t* codes)
+{
+    int64_t rb = oracle_row_bytes(ORACLE_LAYOUT_BASE3_CONT, K), used = (K + 4) / 5;
+    for (int64_t i = 0; i < N * K; ++i)
+        if (trits[i] < -1 || trits[i] > 1) return ORACLE_BAD_TRIT;
+    for (int64_t n = 0; n < N; ++n) {
+        const int8_t* t = trits + n * K;
+        uint8_t* out = codes + n * rb;
+        for (int64_t j = 0; j < rb; ++j) {
+            int code = 0;
+            if (j < used)
+                for (int i = 0; i < 5; ++i) {
+                    int64_t k = 5 * j + i;
+                    int trit = k < K ? t[k] : 0;
+                    code += (trit + 1) * pow3(i);
+                }
+            out[j] = (uint8_t)code;
+        }
+    }
+    return ORACLE_OK;
+}
+
+static int unpack_cont(const uint8_t* codes, int64_t N, int64_t K, int8_t* trits)
+{
+    int64_t rb = oracle_row_bytes(ORACLE_LAYOUT_BASE3_CONT, K), used = (K + 4) / 5;
+    for (int64_t n = 0; n < N; ++n) {
+        const uint8_t* in = codes + n * rb;
+        int8_t* t = trits + n * K;
+        for (int64_t j = 0; j < rb; ++j) {
+            int code = in[j];
+            if (j >= used) {
+                if (code != 0) return ORACLE_BAD_PAD;
+                continue;
+            }
+            if (code >= 243) return ORACLE_BAD_CODE;
+            for (int i = 0; i < 5; ++i) {
+                int digit = (code / pow3(i)) % 3;
+                int64_t k = 5 * j + i;
+                if (k < K) t[k] = (int8_t)(digit - 1);
+                else if (digit != 1) return ORACLE_BAD_PAD;
+            }
+        }
+    }
+    return ORACLE_OK;
+}
+
 int oracle_pack(int layout, const int8_t* trits, int64_t N, int64_t K, uint8_t* codes)
 {
     if (K % ORACLE_GROUP != 0 || N < 0 || K < 0) return ORACLE_BAD_SHAPE;
+    if (layout == ORACLE_LAYOUT_BASE3_CONT) return pack_cont(trits, N, K, codes);
     int bpg = oracle_bytes_per_group(layout);
     if (bpg < 0) return ORACLE_BAD_LAYOUT;
     int64_t groups = K / ORACLE_GROUP;
@@ -165,6 +233,7 @@ int oracle_pack(int layout, const int8_t* trits, int64_t N, int64_t K, uint8_t* 
 int oracle_unpack(int layout, const uint8_t* codes, int64_t N, int64_t K, int8_t* trits)
 {
     if (K % ORACLE_GROUP != 0 || N < 0 || K < 0) return ORACLE_BAD_SHAPE;
+    if (layout == ORACLE_LAYOUT_BASE3_CONT) return unpack_cont(codes, N, K, trits);
     int bpg = oracle_bytes_per_group(layout);
     if (bpg < 0) return ORACLE_BAD_LAYOUT;
     int64_t groups = K / ORACLE_GROUP;

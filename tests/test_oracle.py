@@ -116,6 +116,67 @@ def test_pack_rejects_invalid():
         oracle.pack(np.zeros((1, 100), dtype=np.int8))
 
 
+def _digits_by_divmod(code):
+    # base-3 digits of a byte, least significant first, by repeated division
+    out = []
+    for _ in range(5):
+        code, d = divmod(code, 3)
+        out.append(d)
+    return out
+
+
+@pytest.mark.parametrize("K", [128, 640, 1024, 5120, 17408])
+def test_pack_continuous_layout(K):
+    # byte j holds trits 5j .. 5j+4 of the row across group boundaries; read
+    # back here by plain division, independently of the oracle's unpack
+    g = workloads.rng(9 + K)
+    t = workloads.trits(g, 3, K)
+    codes = oracle.pack(t, oracle.LAYOUT_BASE3_CONT)
+    used = -(-K // 5)
+    assert codes.shape == (3, -(-used // 16) * 16)
+    for n in range(3):
+        flat = []
+        for j in range(used):
+            flat += [d - 1 for d in _digits_by_divmod(int(codes[n, j]))]
+        assert flat[:K] == t[n].tolist()
+        assert all(v == 0 for v in flat[K:])             # pad trits: digit 1
+        assert not codes[n, used:].any()                # row padding: zero bytes
+    assert np.array_equal(oracle.unpack(codes, K, oracle.LAYOUT_BASE3_CONT), t)
+
+
+def test_pack_continuous_worked_example_and_bits():
+    rows = dict((r[0], r[1:]) for r in _read_golden("pack_example.txt"))
+    example = [int(v) for v in rows["trits"]]
+    t = np.zeros((1, 5120), dtype=np.int8)
+    t[0, :5] = example
+    codes = oracle.pack(t, oracle.LAYOUT_BASE3_CONT)
+    assert int(codes[0, 0]) == 183
+    # the release summary's accounting: 1.6 bit per trit + 16 bit per 128 = 1.725 bit at K = 5120
+    K = 5120
+    bits = (oracle.row_bytes(oracle.LAYOUT_BASE3_CONT, K) * 8 + (K // 128) * 16) / K
+    assert bits == 1.725
+    assert (oracle.row_bytes(oracle.LAYOUT_BASE3, K) * 8 + (K // 128) * 16) / K == 1.75
+    # a group boundary inside a byte: trits 125..129 share byte 25
+    t2 = np.zeros((1, 256), dtype=np.int8)
+    t2[0, 125:130] = [1, -1, 1, -1, 1]
+    c2 = oracle.pack(t2, oracle.LAYOUT_BASE3_CONT)
+    assert _digits_by_divmod(int(c2[0, 25])) == [2, 0, 2, 0, 2]
+
+
+def test_pack_continuous_rejects_invalid():
+    ok = oracle.pack(np.zeros((1, 128), dtype=np.int8), oracle.LAYOUT_BASE3_CONT)  # 26 bytes used of 32
+    assert ok.shape == (1, 32)
+    c = ok.copy()
+    c[0, 4] = 243
+    assert oracle.unpack_status(c, 128, oracle.LAYOUT_BASE3_CONT) == oracle.BAD_CODE
+    c = ok.copy()
+    c[0, 25] = 121 - 27                                   # a pad trit of the last byte that is not 0
+    assert oracle.unpack_status(c, 128, oracle.LAYOUT_BASE3_CONT) == oracle.BAD_PAD
+    c = ok.copy()
+    c[0, 30] = 1                                          # row padding must be zero
+    assert oracle.unpack_status(c, 128, oracle.LAYOUT_BASE3_CONT) == oracle.BAD_PAD
+
+
 # ------------------------------------------------------ number formats -----
 
 def test_f16_conversion_all_patterns():
