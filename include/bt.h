@@ -64,7 +64,16 @@ typedef enum {
     BT_LAYOUT_B3 = 0,
     /* Plain 2 bits per trit: digit t + 1 in bits [2i, 2i+1] of byte i/4 (4
      * trits per byte, lowest k in the low bits); 32 bytes per group. */
-    BT_LAYOUT_2BIT = 1
+    BT_LAYOUT_2BIT = 1,
+    /* Continuous base-3: the row's trits five to a byte with no break at
+     * group boundaries (byte j holds trits 5j .. 5j+4, code as for
+     * BT_LAYOUT_B3; a byte may hold trits of two groups); ceil(K/5) bytes,
+     * the last byte's trits past K are pads of value 0, and the row is padded
+     * with zero bytes to a multiple of 16. 1.725 bit per weight with the g128
+     * scales at K = 5120, the release summary's 1.72-bit accounting (section
+     * 三值权重怎么压缩到 1.76 bit). bt_pack, bt_unpack, and the single-row
+     * products (bt_gemv at M = 1, bt_gemv_batched) take it; bt_gemm does not. */
+    BT_LAYOUT_B3C = 2
 } bt_layout;
 
 typedef enum { BT_F32 = 0, BT_BF16 = 1 } bt_dtype;
@@ -72,9 +81,9 @@ typedef enum { BT_F32 = 0, BT_BF16 = 1 } bt_dtype;
 const char* bt_status_string(int status);
 int bt_version(void);
 
-/* Bytes of one packed row: K/128 * 26 (base-3) or K/128 * 32 (2-bit).
- * -1 if K is not a positive multiple of 128 or layout is unknown. Every
- * packed row is therefore a multiple of 2 bytes (base-3) or 32 bytes. */
+/* Bytes of one packed row: K/128 * 26 (base-3), K/128 * 32 (2-bit), or
+ * ceil(K/5) rounded up to 16 (continuous base-3). -1 if K is not a positive
+ * multiple of 128 or layout is unknown. */
 int64_t bt_codes_row_bytes(int layout, int64_t K);
 
 /*

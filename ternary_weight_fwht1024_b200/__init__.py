@@ -19,6 +19,7 @@ LIB_PATH = os.path.join(HERE, "libbt.so")
 
 LAYOUT_B3 = 0
 LAYOUT_2BIT = 1
+LAYOUT_B3C = 2   # continuous base-3 (no per-group byte padding); bt_pack/unpack and single-row products
 F32 = 0
 BF16 = 1
 

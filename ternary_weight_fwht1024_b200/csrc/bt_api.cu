@@ -14,8 +14,8 @@ cudaError_t launch_gemv(int layout, const uint8_t* codes, const uint16_t* scales
                         void* y, void* workspace, int32_t* dev_err, int num_sms, cudaStream_t stream);
 size_t gemv_noalloc_max_bytes();
 cudaError_t gemv_noalloc_scratch(void** out);
-size_t gemv1_workspace_bytes(const DecodeProblem* problems, int count);
-bool gemv_lut_applies(int64_t M, int64_t K, const void* codes, const void* scales);
+size_t gemv1_workspace_bytes(int layout, const DecodeProblem* problems, int count);
+bool gemv_lut_applies(int layout, int64_t M, int64_t K, const void* codes, const void* scales);
 cudaError_t launch_gemv_lut(int layout, const uint8_t* codes, const uint16_t* scales, const void* x, int x_bf16,
                             const int8_t* sign, int M, int64_t N, int64_t K, int y_dtype, void* y, void* workspace,
                             int32_t* dev_err, int num_sms, cudaStream_t stream);
@@ -46,7 +46,7 @@ int current_sm_count() {
 }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
-bool valid_layout(int layout) { return layout == BT_LAYOUT_B3 || layout == BT_LAYOUT_2BIT; }
+bool valid_layout(int layout) { return layout == BT_LAYOUT_B3 || layout == BT_LAYOUT_2BIT || layout == BT_LAYOUT_B3C; }
 bool valid_dtype(int d) { return d == BT_F32 || d == BT_BF16; }
 int64_t group_bytes(int layout) { return layout == BT_LAYOUT_B3 ? 26 : 32; }
 
@@ -110,6 +110,7 @@ int bt_version(void) { return kVersion; }
 
 int64_t bt_codes_row_bytes(int layout, int64_t K) {
     if (!valid_layout(layout) || K <= 0 || K % 128 != 0) return -1;
+    if (layout == BT_LAYOUT_B3C) return ((K + 4) / 5 + 15) / 16 * 16;
     return (K / 128) * group_bytes(layout);
 }
 
@@ -144,8 +145,18 @@ bt_status bt_fwht1024(const uint16_t* x_bf16, const int8_t* sign1024, int64_t M,
                                          static_cast<cudaStream_t>(stream)));
 }
 
+// The continuous base-3 layout runs on the single-row table-lookup kernel
+// only: M = 1, K % 1024 == 0, codes and scales on 16-byte boundaries.
+bt_status check_b3c(int layout, int64_t M, int64_t K, const void* codes, const void* scales) {
+    if (layout != BT_LAYOUT_B3C) return BT_OK;
+    if (M > 1 || K % 1024 != 0) return BT_ERR_SHAPE;
+    if (!aligned(codes, 16) || !aligned(scales, 16)) return BT_ERR_ALIGN;
+    return BT_OK;
+}
+
 size_t bt_gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K) {
     if (!valid_layout(layout) || M < 1 || M > 16 || N < 1 || K < 128 || K % 128 != 0) return 0;
+    if (layout == BT_LAYOUT_B3C && (M > 1 || K % 1024 != 0)) return 0;
     return bt::gemv_workspace_bytes(layout, M, N, K, current_sm_count());
 }
 
@@ -160,7 +171,7 @@ cudaError_t run_gemv(int layout, const uint8_t* codes, const uint16_t* scales, c
     // M = 8, and for the 2-bit layout, the tensor-core kernel of
     // bt_gemv_lut.cu streams the weights once for all rows.
     const bool old_path = layout == BT_LAYOUT_B3 && M >= 2 && M <= 8;
-    if (!old_path && bt::gemv_lut_applies(M, K, codes, scales))
+    if (!old_path && bt::gemv_lut_applies(layout, M, K, codes, scales))
         return bt::launch_gemv_lut(layout, codes, scales, x, x_dtype == BT_BF16 ? 1 : 0, sign1024, (int)M, N, K,
                                    y_dtype, y, ws, dev_err, sms, s);
     return bt::launch_gemv(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y_dtype, y, ws, dev_err, sms, s);
@@ -173,6 +184,7 @@ bt_status bt_gemv(int layout, const uint8_t* codes, const uint16_t* scales, cons
     if (st != BT_OK) return st;
     if (!valid_dtype(y_dtype)) return BT_ERR_INVALID_ARG;
     if (M > 16) return BT_ERR_SHAPE;
+    if ((st = check_b3c(layout, M, K, codes, scales)) != BT_OK) return st;
     if (M == 0 || N == 0) return BT_OK;
     if (!aligned(dev_err, 4)) return BT_ERR_ALIGN;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -193,7 +205,7 @@ size_t bt_gemv_batched_workspace_bytes(int layout, const bt_gemv_problem* proble
         if (q.N < 1 || q.K < 1024 || q.K % 1024 != 0) return 0;
         dp[i] = bt::DecodeProblem{nullptr, nullptr, nullptr, 1, q.x_from, nullptr, q.N, q.K};
     }
-    return bt::gemv1_workspace_bytes(dp, count);
+    return bt::gemv1_workspace_bytes(layout, dp, count);
 }
 
 bt_status bt_gemv_batched(int layout, const bt_gemv_problem* problems, int count, const int8_t* sign1024,
@@ -238,6 +250,7 @@ bt_status bt_gemv_noalloc(int layout, const uint8_t* codes, const uint16_t* scal
     if (st != BT_OK) return st;
     if (!valid_dtype(y_dtype)) return BT_ERR_INVALID_ARG;
     if (M > 16) return BT_ERR_SHAPE;
+    if ((st = check_b3c(layout, M, K, codes, scales)) != BT_OK) return st;
     if (M == 0 || N == 0) return BT_OK;
     if (!aligned(dev_err, 4)) return BT_ERR_ALIGN;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
@@ -251,7 +264,7 @@ bt_status bt_gemv_noalloc(int layout, const uint8_t* codes, const uint16_t* scal
 }
 
 size_t bt_gemm_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K) {
-    if (!valid_layout(layout) || M < 128 || M % 128 != 0 || N < 128 || N % 128 != 0 || K < 128 || K % 128 != 0)
+    if (!valid_layout(layout) || layout == BT_LAYOUT_B3C || M < 128 || M % 128 != 0 || N < 128 || N % 128 != 0 || K < 128 || K % 128 != 0)
         return 0;
     return bt::gemm_workspace_bytes(layout, M, N, K, current_sm_count());
 }
@@ -261,6 +274,7 @@ bt_status bt_gemm(int layout, const uint8_t* codes, const uint16_t* scales, cons
                   void* workspace, size_t workspace_bytes, int32_t* dev_err, void* stream) {
     bt_status st = check_product_args(layout, codes, scales, x, x_dtype, sign1024, M, N, K, y_bf16);
     if (st != BT_OK) return st;
+    if (layout == BT_LAYOUT_B3C) return BT_ERR_INVALID_ARG;  // the prefill GEMM reads group-aligned bytes
     if (M == 0 || N == 0) return BT_OK;
     if (M % 128 != 0 || N % 128 != 0) return BT_ERR_SHAPE;
     if (!aligned(dev_err, 4)) return BT_ERR_ALIGN;

@@ -1090,12 +1090,14 @@ static GemvPlan make_gemv_plan(int layout, int64_t M, int64_t N, int64_t K, int 
 
 // Products whose weights TMA can stream take the kernels of bt_gemv_lut.cu;
 // a workspace sized here serves either path.
-size_t gemv_lut_workspace_bytes(int64_t M, int64_t N, int64_t K);
+size_t gemv_lut_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K);
 
 size_t gemv_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num_sms) {
+    // the continuous layout has the table-lookup kernel only
+    if (layout == BT_LAYOUT_B3C) return gemv_lut_workspace_bytes(layout, M, N, K);
     size_t need = make_gemv_plan(layout, M, N, K, num_sms).total;
     if (K % 1024 == 0) {  // (alignment of the pointers is not known here)
-        const size_t lut = gemv_lut_workspace_bytes(M, N, K);
+        const size_t lut = gemv_lut_workspace_bytes(layout, M, N, K);
         if (lut > need) need = lut;
     }
     return need;

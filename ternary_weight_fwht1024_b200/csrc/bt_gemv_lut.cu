@@ -54,29 +54,50 @@ namespace bt {
 
 constexpr int kLutWarps = 16;                        // streaming warps
 constexpr int kLutThreads = kLutWarps * 32;
-constexpr int kLutChunk = 512;                      // k per table set
+constexpr int kLutChunk = 512;                      // k per table set (group-aligned layouts)
+constexpr int kLutChunkC = 640;                     // k per table set, continuous base-3: 128 bytes, 5 groups
 constexpr int kLutRegion = 256 * 64 * 4;            // [256 codes][64 slots] f32
 constexpr int kLutTableBytes = 2 * kLutRegion;
-constexpr int kLutXrOffset = kLutTableBytes;         // rotated block, 1024 f32
-constexpr int kLutXsOffset = kLutXrOffset + kBlock * 4;  // [5][4][32] f32 slot inputs
 constexpr int kLutSet = 16;                          // rows per set (one TMA box, one reduction)
 constexpr int kLutDepth = 2;                         // sets in flight per warp
 constexpr int kLutCBoxB3 = 112;                      // box bytes per row: 104 + up to 8 of alignment
 constexpr int kLutCBox2b = 128;
-constexpr int kLutSlotMax = kLutSet * kLutCBox2b + kLutSet * 16;  // codes box + scale box (8 halves/row)
-constexpr int kLutTileOffset = kLutXsOffset + 5 * 4 * 32 * 4;   // FWHT exchange tile, 32 x 36 f32
-constexpr int kLutXstOffset = kLutTileOffset + 32 * kTileStride * 4;  // staged raw block of x (<= 4 KB)
-constexpr int kLutSgnOffset = kLutXstOffset + kBlock * 4;      // the 1024 signs of S
-constexpr int kLutBarOffset = kLutSgnOffset + kBlock;
-// TMA writes into the ring: every slot starts on a 128-byte boundary
-constexpr int kLutRingOffset = (kLutBarOffset + kLutWarps * kLutDepth * 8 + 127) & ~127;
-constexpr int kLutSmem = kLutRingOffset + kLutWarps * kLutDepth * kLutSlotMax;
-static_assert(kLutRingOffset % 128 == 0, "ring slots are TMA destinations");
-static_assert(kLutXstOffset % 16 == 0 && kLutSgnOffset % 16 == 0, "16-byte asynchronous copies land there");
-static_assert(kLutSmem <= 227 * 1024, "one CTA per SM");
-static_assert((kLutSet * kLutCBoxB3 + kLutSet * 16) % 128 == 0 && (kLutSet * kLutCBox2b + kLutSet * 16) % 128 == 0 &&
-                  (kLutSet * kLutCBoxB3) % 128 == 0 && (kLutSet * kLutCBox2b) % 128 == 0,
-              "slot sizes and the scale boxes inside them keep 128-byte alignment");
+
+// Continuous base-3 rows: the chunk's bytes 25, 51, 76 and 102 hold trits of
+// two groups; their second-group parts come from four extra tables, looked
+// up by lanes 6, 12, 19 and 25 (byte 1, 3, 0 and 2 of their word).
+__host__ __device__ constexpr int split_byte(int s) { return s == 0 ? 25 : s == 1 ? 51 : s == 2 ? 76 : 102; }
+
+// Shared memory of the table-lookup kernel, per layout: tables, [continuous:
+// extra tables + a zero word], the chunk's rotated activations, the slot
+// inputs, the signs of S, the ring barriers, a staging area for raw x
+// (continuous: two blocks; f32 staging overlaps the FWHT tile, which only a
+// bf16 rotation uses) and the per-warp TMA rings.
+template <int LAYOUT>
+struct LutGeom {
+    static constexpr bool kCont = LAYOUT == BT_LAYOUT_B3C;
+    static constexpr int kChunk = kCont ? kLutChunkC : kLutChunk;
+    static constexpr int kCB = kCont ? 128 : (LAYOUT == BT_LAYOUT_B3 ? 4 * kB3GroupBytes : 4 * k2bGroupBytes);
+    static constexpr int kCBox = LAYOUT == BT_LAYOUT_B3 ? kLutCBoxB3 : 128;
+    static constexpr int kSBox = kCont ? 16 : 8;     // scale halves per row in a set's scale box
+    static constexpr int kSlot = kLutSet * kCBox + kLutSet * kSBox * 2;
+    static constexpr int kExtra = kLutTableBytes;
+    static constexpr int kExtraBytes = kCont ? 256 * 16 + 16 : 0;
+    static constexpr int kXr = kExtra + kExtraBytes;
+    static constexpr int kXrBytes = (kCont ? kLutChunkC : kBlock) * 4;
+    static constexpr int kXs = kXr + kXrBytes;       // [5][4][32] f32 slot inputs
+    static constexpr int kSgn = kXs + 5 * 4 * 32 * 4;
+    static constexpr int kBar = kSgn + kBlock;
+    static constexpr int kStage = kBar + kLutWarps * kLutDepth * 8;
+    static constexpr int kTile = kStage + kBlock * 4;  // FWHT exchange tile, 32 x 36 f32
+    static constexpr int kRing = (kTile + 32 * kTileStride * 4 + 127) & ~127;
+    static constexpr int kSmem = kRing + kLutWarps * kLutDepth * kSlot;
+    static_assert(kRing % 128 == 0 && kSlot % 128 == 0 && (kLutSet * kCBox) % 128 == 0,
+                  "ring slots and the scale boxes inside them are TMA destinations");
+    static_assert(kStage % 16 == 0 && kSgn % 16 == 0, "16-byte asynchronous copies land there");
+    static_assert(!kCont || kTile + 32 * kTileStride * 4 >= kStage + 2 * kBlock * 4, "two f32 blocks fit");
+    static_assert(kSmem <= 227 * 1024, "one CTA per SM");
+};
 
 constexpr int kLutMaxProblems = 12;                  // per launch (kernel parameters < 4 KB)
 constexpr int kLutReduceThreads = 256;
@@ -95,6 +116,7 @@ struct LutProblem {
     int64_t part_base;      // its own partials, from LutParams::part
     int32_t N, ld, nchunk, x_bf16;
     int32_t src_ld, src_nchunk;
+    int32_t K;              // (the last continuous chunk may be partial)
 };
 
 struct LutParams {
@@ -219,13 +241,18 @@ __device__ __forceinline__ void lut_rotate_block(const uint8_t* xst, int x_bf16,
 
 // Slot inputs of chunk half `h` of the block in xr: xs[i][k][L] = x' of trit i
 // of byte 4L + k (zero past the group's last trit and for unused lanes).
+// Continuous base-3: xr holds the chunk's own x' (kvalid of them, zeros past
+// K); a byte that holds trits of two groups keeps only its first group's here.
 template <int LAYOUT>
-__device__ __forceinline__ void lut_scatter(const float* xr, int h, float* xs) {
+__device__ __forceinline__ void lut_scatter(const float* xr, int h, float* xs, int kvalid = 0) {
     for (int t = threadIdx.x; t < 5 * 4 * 32; t += kLutThreads) {
         const int i = t >> 7, k = (t >> 5) & 3, L = t & 31;
         const int p = 4 * L + k;
         float v = 0.f;
-        if (LAYOUT == BT_LAYOUT_B3) {
+        if (LAYOUT == BT_LAYOUT_B3C) {
+            const int j = 5 * p + i;
+            if (j < kvalid && j / kGroup == (5 * p) / kGroup) v = xr[j];
+        } else if (LAYOUT == BT_LAYOUT_B3) {
             if (L < 26) {
                 const int g = p / 26, b = p - 26 * g, j = 5 * b + i;
                 if (j < kGroup) v = xr[h * kLutChunk + g * kGroup + j];
@@ -242,7 +269,11 @@ __device__ __forceinline__ void lut_scatter(const float* xr, int h, float* xs) {
 // checked kernel reports it). They never change: zeroed once per launch.
 template <int LAYOUT>
 __device__ __forceinline__ void lut_zero_invalid(float* table) {
-    if (LAYOUT == BT_LAYOUT_B3) {
+    if (LAYOUT == BT_LAYOUT_B3C) {  // the extra tables' invalid codes and the zero word too
+        float* extra = table + kLutTableBytes / 4;
+        for (int t = threadIdx.x; t < 13 * 4 + 4; t += kLutThreads) extra[243 * 4 + t] = 0.f;
+    }
+    if (LAYOUT == BT_LAYOUT_B3 || LAYOUT == BT_LAYOUT_B3C) {
         for (int t = threadIdx.x; t < 2 * 13 * 64; t += kLutThreads) {
             const int r = t / (13 * 64), u = t - r * 13 * 64;
             table[r * (kLutRegion / 4) + 243 * 64 + u] = 0.f;
@@ -268,7 +299,7 @@ __device__ __forceinline__ void lut_build(const float* xs, float* table) {
     const float x0 = xs[(0 * 4 + k) * 32 + L], x1 = xs[(1 * 4 + k) * 32 + L], x2 = xs[(2 * 4 + k) * 32 + L],
                 x3 = xs[(3 * 4 + k) * 32 + L];
     float* col = table + (k >> 1) * (kLutRegion / 4) + L + 32 * (k & 1);
-    if (LAYOUT == BT_LAYOUT_B3) {
+    if (LAYOUT == BT_LAYOUT_B3 || LAYOUT == BT_LAYOUT_B3C) {
         const float x4 = xs[(4 * 4 + k) * 32 + L];
         for (int b = q; b < 9; b += 4) {
             const float base = (float)(b % 3 - 1) * x3 + (float)(b / 3 - 1) * x4;
@@ -302,6 +333,26 @@ __device__ __forceinline__ void lut_build(const float* xs, float* table) {
     }
 }
 
+// Continuous base-3: the second-group parts of the four split bytes,
+// extra[code][s] = sum_i (d_i(code) - 1) x'_i over the byte's trits in the
+// later group (kvalid as for lut_scatter).
+__device__ __forceinline__ void lut_build_extra(const float* xr, float* extra, int kvalid) {
+    for (int t = threadIdx.x; t < 4 * 243; t += kLutThreads) {
+        const int sidx = t / 243, code = t - 243 * sidx;
+        const int p = split_byte(sidx);
+        float v = 0.f;
+        int c = code;
+#pragma unroll
+        for (int i = 0; i < 5; ++i) {
+            const int d = c % 3;
+            c /= 3;
+            const int j = 5 * p + i;
+            if (j < kvalid && j / kGroup != (5 * p) / kGroup) v += (float)(d - 1) * xr[j];
+        }
+        extra[code * 4 + sidx] = v;
+    }
+}
+
 // acc[j] (j = 0..15, one row each) summed over the warp: halving exchanges on
 // lane bits 3..0 leave lane L with row L % 16 summed over 16 lanes, and one
 // more exchange adds the other half-warp. Lanes i and i + 16 return row i.
@@ -323,7 +374,7 @@ __device__ __forceinline__ float lut_transpose_reduce(float (&acc)[kLutSet]) {
 // A base-3 byte >= 243, or a 2-bit field holding 3.
 template <int LAYOUT>
 __device__ __forceinline__ uint32_t lut_check(uint32_t w) {
-    if (LAYOUT == BT_LAYOUT_B3) return __vcmpgeu4(w, 0xF3F3F3F3u) ? BT_DEVERR_INVALID_CODE : 0u;
+    if (LAYOUT != BT_LAYOUT_2BIT) return __vcmpgeu4(w, 0xF3F3F3F3u) ? BT_DEVERR_INVALID_CODE : 0u;
     return (w & (w >> 1) & 0x55555555u) ? BT_DEVERR_INVALID_CODE : 0u;
 }
 
@@ -356,7 +407,7 @@ __device__ __forceinline__ void lut_issue_set(const LutRing& rg, const CUtensorM
     const uint32_t d = n % kLutDepth;
     const uint32_t dst = rg.ring + d * rg.slot_bytes;
     const uint32_t bar = rg.bar + 8 * d;
-    mbar_arrive_tx(bar, (uint32_t)(kLutSet * rg.cbox + kLutSet * 16));
+    mbar_arrive_tx(bar, (uint32_t)rg.slot_bytes);  // codes box + scale box
     tma_load_2d(dst, cmap, cx, (int)r0, bar);
     tma_load_2d(dst + kLutSet * rg.cbox, smap, sx, (int)r0, bar);
 }
@@ -454,23 +505,83 @@ __device__ __forceinline__ void lut_gather_block(const LutProblem& pr, int y_bf1
 
 // ------------------------------------------------------------- kernel ----
 
+// Continuous base-3: warp 0 rotates (or copies) the staged blocks b0 and b1
+// (b1 < 0: one block) and keeps the chunk's kvalid values of x' in xr.
+__device__ __forceinline__ void lut_rotate_chunk(const uint8_t* xst, int x_bf16, const int8_t* sgn, bool has_sign,
+                                                 int64_t k0, int b0, int b1, int kvalid, float* xr, float* tile) {
+    const int lane = threadIdx.x & 31;
+    const int esz = x_bf16 ? 2 : 4;
+    for (int u = 0; u < 2; ++u) {
+        const int bb = u == 0 ? b0 : b1;
+        if (bb < 0) break;
+        float v[32];
+        const uint8_t* raw = xst + u * kBlock * esz;
+        if (x_bf16) {
+            const uint4* src = reinterpret_cast<const uint4*>(raw + 64 * lane);
+            uint32_t w[16];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint4 t = src[q];
+                w[4 * q] = t.x; w[4 * q + 1] = t.y; w[4 * q + 2] = t.z; w[4 * q + 3] = t.w;
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = bf16_bits_to_f32((i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu));
+        } else {
+            const float4* src = reinterpret_cast<const float4*>(raw + 128 * lane);
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                const float4 t = src[q];
+                v[4 * q] = t.x; v[4 * q + 1] = t.y; v[4 * q + 2] = t.z; v[4 * q + 3] = t.w;
+            }
+        }
+        const int64_t e0 = (int64_t)bb * kBlock - k0;  // chunk position of the block's element 0
+        if (has_sign) {
+            const uint4* sg = reinterpret_cast<const uint4*>(sgn + 32 * lane);
+            const uint4 s0 = sg[0], s1 = sg[1];
+            const uint32_t sw[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const uint32_t sbit = (sw[i >> 2] >> (8 * (i & 3))) & 0x80u;
+                v[i] = __uint_as_float(__float_as_uint(v[i]) ^ (sbit << 24));
+            }
+            fwht1024_warp(v, tile);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {  // lane holds element 32 j + lane
+                const int64_t kk = e0 + 32 * j + lane;
+                if (kk >= 0 && kk < kvalid) xr[kk] = v[j];
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const int64_t kk = e0 + 32 * lane + i;
+                if (kk >= 0 && kk < kvalid) xr[kk] = v[i];
+            }
+        }
+    }
+}
+
 template <int LAYOUT, bool CHECK>
 __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_constant__ LutParams P) {
+    using GE = LutGeom<LAYOUT>;
+    constexpr bool CONT = GE::kCont;
+    constexpr int CHUNK = GE::kChunk;
     float* table = reinterpret_cast<float*>(lut_smem);
     const uint32_t tab_s = smem_addr(lut_smem);
-    float* xr = reinterpret_cast<float*>(lut_smem + kLutXrOffset);
-    float* xs = reinterpret_cast<float*>(lut_smem + kLutXsOffset);
-    const uint8_t* xst = lut_smem + kLutXstOffset;
+    float* xr = reinterpret_cast<float*>(lut_smem + GE::kXr);
+    float* xs = reinterpret_cast<float*>(lut_smem + GE::kXs);
+    const uint8_t* xst = lut_smem + GE::kStage;
     const uint32_t xst_s = smem_addr(xst);
-    int8_t* sgn = reinterpret_cast<int8_t*>(lut_smem + kLutSgnOffset);
+    int8_t* sgn = reinterpret_cast<int8_t*>(lut_smem + GE::kSgn);
+    float* tile = reinterpret_cast<float*>(lut_smem + GE::kTile);
+    const uint32_t extra_s = smem_addr(lut_smem + GE::kExtra);
     const int warp = threadIdx.x >> 5, L = threadIdx.x & 31;
-    const int CB = LAYOUT == BT_LAYOUT_B3 ? 4 * kB3GroupBytes : 4 * k2bGroupBytes;  // bytes per chunk row
+    const int CB = GE::kCB;  // bytes per chunk row
     const bool lane_on = LAYOUT == BT_LAYOUT_B3 ? L < 26 : true;
     LutRing rg;
-    rg.cbox = LAYOUT == BT_LAYOUT_B3 ? kLutCBoxB3 : kLutCBox2b;
-    rg.slot_bytes = kLutSet * rg.cbox + kLutSet * 16;
-    rg.ring = smem_addr(lut_smem + kLutRingOffset) + warp * kLutDepth * rg.slot_bytes;
-    rg.bar = smem_addr(lut_smem + kLutBarOffset) + warp * kLutDepth * 8;
+    rg.cbox = GE::kCBox;
+    rg.slot_bytes = GE::kSlot;
+    rg.ring = smem_addr(lut_smem + GE::kRing) + warp * kLutDepth * rg.slot_bytes;
+    rg.bar = smem_addr(lut_smem + GE::kBar) + warp * kLutDepth * 8;
 
     // lane constants: table byte offsets and scale selectors
     const uint32_t lanebytes = (uint32_t)(4 * L) | ((uint32_t)(4 * L + 128) << 8);
@@ -478,6 +589,9 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_c
     if (LAYOUT == BT_LAYOUT_B3) {
         ga = lane_on ? (4 * L) / 26 : 3;
         gb = lane_on ? (4 * L + 3) / 26 : 3;
+    } else if (CONT) {
+        ga = (20 * L) / kGroup;       // the groups of the lane's first and last trit
+        gb = (20 * L + 19) / kGroup;
     } else {
         ga = gb = L >> 3;
     }
@@ -485,6 +599,22 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_c
     // lanes past the 26 words of a base-3 chunk row read lane 25's word; their
     // table slots hold zeros
     const int wlane = LAYOUT == BT_LAYOUT_B3 ? (L < 26 ? L : 25) : L;
+    // continuous base-3: which bytes of the lane's word count for its first
+    // group (the split byte's first-group part among them), and where its
+    // extra lookup goes (the zero word for lanes without a split byte)
+    float wa[4] = {1.f, 1.f, 1.f, 1.f};
+    uint32_t exsh = 0, exmul = 0, exadd = 256 * 16;
+    if (CONT) {
+        const int sidx = L == 6 ? 0 : L == 12 ? 1 : L == 19 ? 2 : L == 25 ? 3 : -1;
+        if (sidx >= 0) {
+            const int sb = split_byte(sidx) - 4 * L;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) wa[i] = i <= sb ? 1.f : 0.f;
+            exsh = 8u * sb;
+            exmul = 16u;
+            exadd = 4u * sidx;
+        }
+    }
 
     if (L == 0) {
         for (int d = 0; d < kLutDepth; ++d) mbar_init(rg.bar + 8 * d, 1);
@@ -521,7 +651,8 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_c
         if (!ihave) return;
         if (L == 0) {
             const int cb = is.c * CB;
-            lut_issue_set(rg, &P.cmap[is.p], &P.smap[is.p], issued, cb & ~15, (4 * is.c) & ~7,
+            const int sx = CONT ? (5 * is.c) & ~7 : (4 * is.c) & ~7;
+            lut_issue_set(rg, &P.cmap[is.p], &P.smap[is.p], issued, cb & ~15, sx,
                           is.n0 + (int64_t)kLutSet * (warp + kLutWarps * iq));
         }
         ++iq;
@@ -532,52 +663,80 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_c
     LutSeg sg;
     bool have = lut_next_seg(P, rc, rc1, sg);
 
+    // the raw blocks of x a segment needs (continuous: the one or two blocks
+    // its 640 columns touch), staged by warp 0
+    auto seg_blocks = [&](const LutSeg& g, int& b0, int& b1) {
+        const int64_t k0 = (int64_t)g.c * CHUNK;
+        b0 = (int)(k0 / kBlock);
+        b1 = -1;
+        if (CONT) {
+            const int64_t K = (int64_t)P.p[g.p].K;
+            const int64_t kend = min(k0 + CHUNK, K) - 1;
+            if (kend / kBlock != b0) b1 = (int)(kend / kBlock);
+        }
+    };
+    auto stage = [&](const LutSeg& g) {
+        const LutProblem& q = P.p[g.p];
+        int b0, b1;
+        seg_blocks(g, b0, b1);
+        lut_stage_block(q.x, q.x_bf16, b0, xst_s);
+        if (b1 >= 0) lut_stage_block(q.x, q.x_bf16, b1, xst_s + kBlock * (q.x_bf16 ? 2 : 4));
+    };
+
     pdl_wait();  // x may come from the preceding kernel, which may also still read the partials
     pdl_launch_dependents();
 
     int bad = 0;
     int cur_p = -1, cur_blk = -1;
-    if (have && warp == 0 && !P.p[sg.p].src)
-        lut_stage_block(P.p[sg.p].x, P.p[sg.p].x_bf16, (sg.c * kLutChunk) / kBlock, xst_s);
+    if (have && warp == 0 && !P.p[sg.p].src) stage(sg);
     while (have) {
         const LutProblem& pr = P.p[sg.p];
         const int n0 = sg.n0, n1 = sg.n1;
         float* part = P.part + pr.part_base + (int64_t)sg.c * pr.ld;
         const int coff = (sg.c * CB) & 15;
-        const int soff = 2 * ((4 * sg.c) & 7);
-        const int blk = (sg.c * kLutChunk) / kBlock;
-        const bool new_blk = sg.p != cur_p || blk != cur_blk;
+        const int soff = CONT ? 2 * ((5 * sg.c) & 7) : 2 * ((4 * sg.c) & 7);  // bytes into a scale row
+        int b0, b1;
+        seg_blocks(sg, b0, b1);
+        const int blk = b0;
+        // continuous chunks always rebuild xr from their own one or two blocks
+        const bool new_blk = CONT || sg.p != cur_p || blk != cur_blk;
+        const int kvalid = CONT ? (int)min((int64_t)CHUNK, (int64_t)pr.K - (int64_t)sg.c * CHUNK) : 0;
         const int my = warp_sets(sg);
 
         __syncthreads();  // the previous segment's lookups are done with table / xs
         if (new_blk) {
             if (pr.src) {  // x is an earlier matrix's output: add up its partials
-                lut_gather_block(pr, P.y_bf16, blk, lut_smem + kLutXstOffset);
+                lut_gather_block(pr, P.y_bf16, b0, lut_smem + GE::kStage);
+                if (b1 >= 0) lut_gather_block(pr, P.y_bf16, b1, lut_smem + GE::kStage + kBlock * (P.y_bf16 ? 2 : 4));
                 __syncthreads();
             }
             if (warp == 0) {
                 cp_async_wait_all();
                 __syncwarp();
-                lut_rotate_block(xst, pr.x_bf16, sgn, P.sign != nullptr, xr,
-                                 reinterpret_cast<float*>(lut_smem + kLutTileOffset));
+                if (CONT)
+                    lut_rotate_chunk(xst, pr.x_bf16, sgn, P.sign != nullptr, (int64_t)sg.c * CHUNK, b0, b1, kvalid,
+                                     xr, tile);
+                else
+                    lut_rotate_block(xst, pr.x_bf16, sgn, P.sign != nullptr, xr, tile);
             }
             cur_p = sg.p;
             cur_blk = blk;
             __syncthreads();
         }
-        lut_scatter<LAYOUT>(xr, (sg.c * kLutChunk - blk * kBlock) / kLutChunk, xs);
+        if (CONT) lut_scatter<LAYOUT>(xr, 0, xs, kvalid);
+        else lut_scatter<LAYOUT>(xr, (sg.c * CHUNK - blk * kBlock) / CHUNK, xs);
         __syncthreads();
         lut_build<LAYOUT>(xs, table);
+        if (CONT) lut_build_extra(xr, reinterpret_cast<float*>(lut_smem + GE::kExtra), kvalid);
         __syncthreads();
 
-        // the next segment; its block of x is staged now if it is a new one
+        // the next segment; its block(s) of x are staged now if needed
         LutSeg nx;
         int64_t nrc = rc;
         const bool nhave = lut_next_seg(P, nrc, rc1, nx);
         if (nhave && warp == 0) {
-            const int nb = (nx.c * kLutChunk) / kBlock;
-            if ((nx.p != sg.p || nb != blk) && !P.p[nx.p].src)
-                lut_stage_block(P.p[nx.p].x, P.p[nx.p].x_bf16, nb, xst_s);
+            const int nb = (int)(((int64_t)nx.c * CHUNK) / kBlock);
+            if ((CONT || nx.p != sg.p || nb != blk) && !P.p[nx.p].src) stage(nx);
         }
 
         for (int q = 0; q < my && ok; ++q) {
@@ -604,10 +763,20 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_c
                 const float e1 = lds_f32(tab_s + o1);
                 const float e2 = lds_f32(tab_s + kLutRegion + o2);
                 const float e3 = lds_f32(tab_s + kLutRegion + o3);
-                const uint2 q4 = lds_u64(sslot + 16 * i);
-                const uint32_t sp = prmt(q4.x, q4.y, ssel);
-                const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&sp));
-                a16[i] = fmaf(sf.y, e2 + e3, sf.x * (e0 + e1));
+                if (CONT) {
+                    const float ex = lds_f32(extra_s + ((cw >> exsh) & 0xFFu) * exmul + exadd);
+                    const float sa = f16_bits_to_f32(lds_u16(sslot + GE::kSBox * 2 * i + 2 * ga));
+                    const float sbv = f16_bits_to_f32(lds_u16(sslot + GE::kSBox * 2 * i + 2 * gb));
+                    const float A = fmaf(wa[3], e3, fmaf(wa[2], e2, fmaf(wa[1], e1, wa[0] * e0)));
+                    const float B = fmaf(1.f - wa[3], e3, fmaf(1.f - wa[2], e2, fmaf(1.f - wa[1], e1,
+                                                                                      fmaf(1.f - wa[0], e0, ex))));
+                    a16[i] = fmaf(sbv, B, sa * A);
+                } else {
+                    const uint2 q4 = lds_u64(sslot + 16 * i);
+                    const uint32_t sp = prmt(q4.x, q4.y, ssel);
+                    const float2 sf = __half22float2(*reinterpret_cast<const __half2*>(&sp));
+                    a16[i] = fmaf(sf.y, e2 + e3, sf.x * (e0 + e1));
+                }
             }
             const int r0 = n0 + kLutSet * (warp + kLutWarps * q);
             const float v = lut_transpose_reduce(a16);  // every value read from the slot is consumed here
@@ -1017,17 +1186,31 @@ static void lut_for_each_launch(const DecodeProblem* pr, int count, F&& f) {
     }
 }
 
-// Partial floats of one matrix: [K / 512][N rounded up to 4].
-static int64_t lut_part_floats(const DecodeProblem& p) { return (p.K / kLutChunk) * ((p.N + 3) & ~3); }
+// Chunks of a row: 512 columns, or 640 (128 bytes) in the continuous layout
+// (the last one may be partial).
+static int64_t lut_nchunk(int layout, int64_t K) {
+    return layout == BT_LAYOUT_B3C ? (K + kLutChunkC - 1) / kLutChunkC : K / kLutChunk;
+}
+
+// Bytes of one packed row.
+static int64_t lut_row_bytes(int layout, int64_t K) {
+    if (layout == BT_LAYOUT_B3C) return ((K + 4) / 5 + 15) / 16 * 16;
+    return (K / kGroup) * (layout == BT_LAYOUT_B3 ? kB3GroupBytes : k2bGroupBytes);
+}
+
+// Partial floats of one matrix: [chunks][N rounded up to 4].
+static int64_t lut_part_floats(int layout, const DecodeProblem& p) {
+    return lut_nchunk(layout, p.K) * ((p.N + 3) & ~3);
+}
 
 // Every matrix of a list keeps its partials until the list's reductions at
 // the end (a later group may read them as its input): their sum, each group
 // starting on a 256-byte boundary.
-size_t gemv1_workspace_bytes(const DecodeProblem* pr, int count) {
+size_t gemv1_workspace_bytes(int layout, const DecodeProblem* pr, int count) {
     size_t total = 0;
     lut_for_each_launch(pr, count, [&](int first, int n) {
         int64_t f = 0;
-        for (int i = first; i < first + n; ++i) f += lut_part_floats(pr[i]);
+        for (int i = first; i < first + n; ++i) f += lut_part_floats(layout, pr[i]);
         total += lut_align((size_t)f * sizeof(float), 256);
     });
     return std::max(total, (size_t)256);
@@ -1035,9 +1218,9 @@ size_t gemv1_workspace_bytes(const DecodeProblem* pr, int count) {
 
 // Products whose weights TMA can stream: K a multiple of 1024 (so the scale
 // rows are whole 16-byte units), 16-byte aligned codes and scales.
-bool gemv_lut_applies(int64_t M, int64_t K, const void* codes, const void* scales) {
-    return M >= 1 && M <= 16 && K > 0 && K % kBlock == 0 && (reinterpret_cast<uintptr_t>(scales) & 15) == 0 &&
-           (reinterpret_cast<uintptr_t>(codes) & 15) == 0;
+bool gemv_lut_applies(int layout, int64_t M, int64_t K, const void* codes, const void* scales) {
+    return M >= 1 && M <= (layout == BT_LAYOUT_B3C ? 1 : 16) && K > 0 && K % kBlock == 0 &&
+           (reinterpret_cast<uintptr_t>(scales) & 15) == 0 && (reinterpret_cast<uintptr_t>(codes) & 15) == 0;
 }
 
 // Workspace of one product with M activation rows: for M > 1 the prep
@@ -1046,8 +1229,9 @@ bool gemv_lut_applies(int64_t M, int64_t K, const void* codes, const void* scale
 static size_t mma_frag_bytes(int64_t M, int64_t K) { return lut_align((size_t)M * (K / kGroup) * kB3Mmas * 32, 256); }
 static size_t mma_meta_bytes(int64_t M, int64_t K) { return lut_align((size_t)M * (K / kGroup) * 8, 256); }
 
-size_t gemv_lut_workspace_bytes(int64_t M, int64_t N, int64_t K) {
-    const size_t part = lut_align((size_t)(K / kLutChunk) * (size_t)M * (size_t)((N + 3) & ~3) * sizeof(float), 256);
+size_t gemv_lut_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K) {
+    const size_t part =
+        lut_align((size_t)lut_nchunk(layout, K) * (size_t)M * (size_t)((N + 3) & ~3) * sizeof(float), 256);
     return std::max((M > 1 ? mma_frag_bytes(M, K) + mma_meta_bytes(M, K) : 0) + part, (size_t)256);
 }
 
@@ -1071,9 +1255,13 @@ static cudaError_t lut_launch_k(Kern kern, int smem, const LutParams& P, int gri
 // The partials and outputs of one group, as the reduction reads them.
 template <int LAYOUT, bool CHECK>
 static cudaError_t lut_launch_t(const LutParams& P, int grid, cudaStream_t stream) {
-    if (P.M == 1) return lut_launch_k(gemv_lut_kernel<LAYOUT, CHECK>, kLutSmem, P, grid, stream);
-    if (P.M <= 8) return lut_launch_k(gemv_mma_kernel<LAYOUT, 1, CHECK>, MmaGeom<LAYOUT>::kSmem, P, grid, stream);
-    return lut_launch_k(gemv_mma_kernel<LAYOUT, 2, CHECK>, MmaGeom<LAYOUT>::kSmem, P, grid, stream);
+    if (P.M == 1) return lut_launch_k(gemv_lut_kernel<LAYOUT, CHECK>, LutGeom<LAYOUT>::kSmem, P, grid, stream);
+    if constexpr (LAYOUT == BT_LAYOUT_B3C) {
+        return cudaErrorInvalidValue;  // single rows only
+    } else {
+        if (P.M <= 8) return lut_launch_k(gemv_mma_kernel<LAYOUT, 1, CHECK>, MmaGeom<LAYOUT>::kSmem, P, grid, stream);
+        return lut_launch_k(gemv_mma_kernel<LAYOUT, 2, CHECK>, MmaGeom<LAYOUT>::kSmem, P, grid, stream);
+    }
 }
 
 // The main kernel of group [first, first + count), M activation rows (M > 1:
@@ -1086,22 +1274,23 @@ static cudaError_t lut_launch_group(int layout, const DecodeProblem* all, const 
     EncodeTiledFn enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
     LutParams P{};
-    const int gbytes = layout == BT_LAYOUT_B3 ? kB3GroupBytes : k2bGroupBytes;
+    const bool cont = layout == BT_LAYOUT_B3C;
     int64_t rc = 0;
     for (int i = 0; i < count; ++i) {
         const DecodeProblem& s = all[first + i];
         LutProblem& d = P.p[i];
-        const int64_t G = s.K / kGroup, RB = G * gbytes;
+        const int64_t G = s.K / kGroup, RB = lut_row_bytes(layout, s.K);
         d.N = static_cast<int32_t>(s.N);
+        d.K = static_cast<int32_t>(s.K);
         d.ld = static_cast<int32_t>((s.N + 3) & ~3);
-        d.nchunk = static_cast<int32_t>(s.K / kLutChunk);
+        d.nchunk = static_cast<int32_t>(lut_nchunk(layout, s.K));
         d.rc_base = rc;
         d.part_base = base[first + i];
         if (s.x_from >= 0) {  // an earlier group's output: summed from its partials
             const DecodeProblem& q = all[s.x_from];
             d.src = part + base[s.x_from];
             d.src_ld = static_cast<int32_t>((q.N + 3) & ~3);
-            d.src_nchunk = static_cast<int32_t>(q.K / kLutChunk);
+            d.src_nchunk = static_cast<int32_t>(lut_nchunk(layout, q.K));
             d.x = nullptr;
             d.x_bf16 = y_bf16;
         } else {
@@ -1115,7 +1304,7 @@ static cudaError_t lut_launch_group(int layout, const DecodeProblem* all, const 
         const cuuint32_t cbox[2] = {static_cast<cuuint32_t>(layout == BT_LAYOUT_B3 ? kLutCBoxB3 : kLutCBox2b), kLutSet};
         const cuuint64_t sdim[2] = {static_cast<cuuint64_t>(G), static_cast<cuuint64_t>(s.N)};
         const cuuint64_t sstr[1] = {static_cast<cuuint64_t>(G) * 2};
-        const cuuint32_t sbox[2] = {8, kLutSet};
+        const cuuint32_t sbox[2] = {cont ? 16u : 8u, kLutSet};
         const cuuint32_t one[2] = {1, 1};
         if (enc(&P.cmap[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(s.codes), cdim, cstr, cbox, one,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -1139,13 +1328,16 @@ static cudaError_t lut_launch_group(int layout, const DecodeProblem* all, const 
     if (layout == BT_LAYOUT_B3)
         return dev_err ? lut_launch_t<BT_LAYOUT_B3, true>(P, grid, stream)
                        : lut_launch_t<BT_LAYOUT_B3, false>(P, grid, stream);
+    if (layout == BT_LAYOUT_B3C)
+        return dev_err ? lut_launch_t<BT_LAYOUT_B3C, true>(P, grid, stream)
+                       : lut_launch_t<BT_LAYOUT_B3C, false>(P, grid, stream);
     return dev_err ? lut_launch_t<BT_LAYOUT_2BIT, true>(P, grid, stream)
                    : lut_launch_t<BT_LAYOUT_2BIT, false>(P, grid, stream);
 }
 
 // Outputs of matrices [first, first + count), count <= kLutMaxProblems.
-static cudaError_t lut_launch_reduce(const DecodeProblem* all, const int64_t* base, int first, int count, int M,
-                                     int y_bf16, float* part, cudaStream_t stream) {
+static cudaError_t lut_launch_reduce(int layout, const DecodeProblem* all, const int64_t* base, int first, int count,
+                                     int M, int y_bf16, float* part, cudaStream_t stream) {
     LutReduceParams R{};
     R.nprob = count;
     R.y_bf16 = y_bf16;
@@ -1156,7 +1348,7 @@ static cudaError_t lut_launch_reduce(const DecodeProblem* all, const int64_t* ba
         R.y[i] = s.y;
         R.N[i] = static_cast<int32_t>(s.N);
         R.ld[i] = static_cast<int32_t>((s.N + 3) & ~3);
-        R.nchunk[i] = static_cast<int32_t>(s.K / kLutChunk);
+        R.nchunk[i] = static_cast<int32_t>(lut_nchunk(layout, s.K));
         R.M[i] = M;
         tiles += (int)((M * s.N + kLutReduceThreads - 1) / kLutReduceThreads);
     }
@@ -1189,7 +1381,7 @@ cudaError_t launch_gemv1(int layout, const DecodeProblem* problems, int count, c
         lut_for_each_launch(problems, count, [&](int first, int n) {
             for (int i = first; i < first + n; ++i) {
                 base[i] = off;
-                off += lut_part_floats(problems[i]);
+                off += lut_part_floats(layout, problems[i]);
             }
             off = (int64_t)lut_align((size_t)off, 64);  // 256-byte boundary between groups
         });
@@ -1200,8 +1392,8 @@ cudaError_t launch_gemv1(int layout, const DecodeProblem* problems, int count, c
             err = lut_launch_group(layout, problems, base, first, n, 1, sign, y_bf16, part, dev_err, num_sms, stream);
     });
     for (int first = 0; first < count && err == cudaSuccess; first += kLutMaxProblems)
-        err = lut_launch_reduce(problems, base, first, std::min(kLutMaxProblems, count - first), 1, y_bf16, part,
-                                stream);
+        err = lut_launch_reduce(layout, problems, base, first, std::min(kLutMaxProblems, count - first), 1, y_bf16,
+                                part, stream);
     return err;
 }
 
@@ -1239,7 +1431,7 @@ cudaError_t launch_gemv_lut(int layout, const uint8_t* codes, const uint16_t* sc
     cudaError_t err = lut_launch_group(layout, &p, base, 0, 1, M, sign, y_bf16, part, dev_err, num_sms, stream,
                                        frag, meta);
     if (err != cudaSuccess) return err;
-    return lut_launch_reduce(&p, base, 0, 1, M, y_bf16, part, stream);
+    return lut_launch_reduce(layout, &p, base, 0, 1, M, y_bf16, part, stream);
 }
 
 }  // namespace bt

@@ -7,6 +7,7 @@ import re
 
 import pytest
 
+import oracle
 import ternary_weight_fwht1024_b200 as bt
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -51,6 +52,10 @@ def test_codes_row_bytes(lib):
     assert bt.codes_row_bytes(bt.LAYOUT_B3, 100) == -1
     assert bt.codes_row_bytes(bt.LAYOUT_B3, 0) == -1
     assert bt.codes_row_bytes(5, 1024) == -1
+    # continuous base-3: ceil(K/5) bytes rounded up to 16, as the oracle lays them out
+    for K in (128, 640, 1024, 5120, 17408):
+        assert bt.codes_row_bytes(bt.LAYOUT_B3C, K) == oracle.row_bytes(oracle.LAYOUT_BASE3_CONT, K)
+    assert bt.codes_row_bytes(bt.LAYOUT_B3C, 5120) == 1024 and bt.codes_row_bytes(bt.LAYOUT_B3C, 17408) == 3488
 
 
 P = ctypes.c_void_p
@@ -99,6 +104,12 @@ def test_gemv_validation(lib):
     assert lib.bt_gemv(*args(ws=_fake((1 << 24) + 16), wsb=need)) == 3
     assert lib.bt_gemv(*args(M=0)) == 0
     assert lib.bt_gemv_workspace_bytes(0, 17, 256, 1024) == 0
+    # continuous base-3: single rows only, K % 1024 == 0, 16-byte aligned codes and scales
+    assert lib.bt_gemv(*args(layout=2, M=2)) == 2
+    assert lib.bt_gemv(*args(layout=2, K=1152, sign=None)) == 2
+    assert lib.bt_gemv(*args(layout=2)) == 4          # fine, but no workspace
+    assert lib.bt_gemv_workspace_bytes(2, 2, 256, 1024) == 0
+    assert lib.bt_gemv_workspace_bytes(2, 1, 256, 1024) == 256 * 2 * 4  # two 640-column chunks of partials
 
 
 def test_gemm_validation(lib):
@@ -111,6 +122,8 @@ def test_gemm_validation(lib):
     assert lib.bt_gemm(*args()) == 4
     assert lib.bt_gemm_workspace_bytes(0, 512, 5120, 5120) > 0
     assert lib.bt_gemm_workspace_bytes(0, 100, 5120, 5120) == 0
+    assert lib.bt_gemm(*args(layout=2)) == 1           # the prefill GEMM reads group-aligned bytes only
+    assert lib.bt_gemm_workspace_bytes(2, 512, 5120, 5120) == 0
 
 
 def test_binding_refuses_cpu_tensors():

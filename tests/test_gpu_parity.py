@@ -260,10 +260,9 @@ def test_gemv_bf16_output():
 def test_gemv_special_cases_m1_exact(layout, t, K):
     # M = 1 runs the table-lookup kernel. A byte of zero trits has the table
     # entry 0 exactly and a byte with one non-zero trit the entry +-x'_k
-    # exactly, and chunk partials are added as exact integers (2^-36 units),
-    # so all-zero weights give y = 0 exactly and a single trit gives
-    # y[n] = t * fl(s * x'_k) (|s x'_k| >= 2^-13 here, so the fixed-point unit
-    # does not round it), with x' the library's own FP32 rotation
+    # exactly; every other term of the row, and every other chunk partial, is
+    # an exact zero, so all-zero weights give y = 0 exactly and a single trit
+    # gives y[n] = t * fl(s * x'_k), with x' the library's own FP32 rotation
     # (bt_fwht1024 runs the same warp transform).
     N = 64
     case = workloads.random_case(5000, 1, N, K)
