@@ -136,6 +136,8 @@ def _layer_tensors(bt, torch, dev, layout, idx, L, with_x=False):
 
 
 def _weight_bytes(L, layout):
+    if layout == 2:  # continuous base-3: ceil(K/5) bytes rounded up to 16, plus the scales
+        return L.N * (((L.K + 4) // 5 + 15) // 16 * 16 + (L.K // 128) * 2)
     per_group = (26 if layout == 0 else 32) + 2
     return L.N * (L.K // 128) * per_group
 
@@ -313,6 +315,21 @@ def run_gpu(args, rank, world):
     bytes2 = sum(_weight_bytes(L, 1) for L in triple)
     del gs2, reps2
 
+    # ---- continuous base-3 twin (1.725 bit: no per-group byte padding) ----
+    reps_c = build(2)
+    gs_c = graphs_for(reps_c, 2)
+    ms_c = timed(gs_c, args.steps, args.warmup, per_graph=spg)
+    bytes_c = sum(_weight_bytes(L, 2) for L in triple)
+    del gs_c, reps_c
+
+    # ---- GEMV / GEMM crossover on the triple (base-3) ----
+    crossover = None
+    if not args.no_sweep:
+        try:
+            crossover = run_crossover(bt, torch, dev, stream, sign)
+        except Exception as e:
+            crossover = {"error": str(e)[:200]}
+
     # ---- prefill GEMM pp512, both layouts (seeded C3 / C4 inputs) ----
     gemm = {}
     for layout, cfg, name in ((0, "C3", "base-3"), (1, "C4", "2-bit")):
@@ -369,6 +386,10 @@ def run_gpu(args, rank, world):
         "per_call_us": {L.name: round(u, 2) for L, u in zip(triple, per_layer_us)},
         "layout_2bit": {"value": round(bytes2 / (ms2 * 1e-3) / 1e9 * world, 2), "unit": "GB/s",
                         "ms_per_step": round(ms2, 5), "bytes_per_step": bytes2},
+        "layout_b3_continuous": {"value": round(bytes_c / (ms_c * 1e-3) / 1e9 * world, 2), "unit": "GB/s",
+                                 "ms_per_step": round(ms_c, 5), "bytes_per_step": bytes_c,
+                                 "bits_per_weight": round(8 * bytes_c / sum(L.N * L.K for L in triple), 4)},
+        "crossover_gemv_gemm": crossover,
         "tokens_per_s_triple": round(1e3 / ms3 * world, 1),
         "gemm": gemm.get("base-3"),
         "gemm_2bit": gemm.get("2-bit"),
@@ -428,6 +449,79 @@ def run_gemm(bt, torch, dev, stream, sign, layout, cfg, args, timed, peaks):
             "frac_of_peak": round(tf / peaks["bf16_tflops"], 4), "peak": peaks["bf16_tflops"],
             "peak_kind": f"bf16 burst, {peaks['src']}",
             "l2": "weights (21-26 MB per matrix) re-read from L2 across steps; the activations dominate traffic"}
+
+
+def run_crossover(bt, torch, dev, stream, sign):
+    """Decode GEMV against the prefill GEMM on the base-3 triple for M = 1 .. 64
+    activation rows: the GEMV at M = 1 (one batched call) and M = 2, 4, 8, 16
+    (three bt_gemv calls), above 16 as M / 16 such calls; the GEMM at M = 128,
+    the smallest M it takes (a caller pads M rows up to it). Device time per
+    triple from CUDA graphs over weight copies that exceed L2; tokens/s = M /
+    time. The crossover is the smallest M at which the padded GEMM is faster."""
+    import workloads
+    triple = workloads.TRIPLE
+    copies = max(4, math.ceil(4 * L2_BYTES / sum(_weight_bytes(L, 0) for L in triple)))
+    base = [_layer_tensors(bt, torch, dev, 0, i, L)[:2] for i, L in enumerate(triple)]
+    reps = [[(c.clone(), s.clone()) for c, s in base] for _ in range(copies)]
+    del base
+
+    def per_triple_us(step):
+        with torch.cuda.stream(stream):
+            for r in range(copies):
+                step(r)
+            torch.cuda.synchronize()
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=stream):
+                for r in range(copies):
+                    step(r)
+            for _ in range(3):
+                gr.replay()
+            torch.cuda.synchronize()
+            a_ = torch.cuda.Event(enable_timing=True)
+            b_ = torch.cuda.Event(enable_timing=True)
+            n = 10
+            a_.record(stream)
+            for _ in range(n):
+                gr.replay()
+            b_.record(stream)
+            torch.cuda.synchronize()
+        return a_.elapsed_time(b_) * 1e3 / (n * copies)
+
+    g = workloads.rng(4 * 1_000_003 + 7)
+    gemv_us = {}
+    for M in (1, 2, 4, 8, 16):
+        xs = [torch.from_numpy(workloads.activations_bf16_bits(g, M, L.K, True).view(np.int16)).to(dev)
+              .view(torch.bfloat16) for L in triple]
+        ys = [torch.empty((M, L.N), device=dev) for L in triple]
+        if M == 1:
+            ws = torch.empty(bt.gemv_batched_workspace_bytes(0, [dict(N=L.N, K=L.K) for L in triple]),
+                             dtype=torch.uint8, device=dev)
+            step = lambda r: bt.gemv_batched([dict(codes=reps[r][i][0], scales=reps[r][i][1], x=xs[i], y=ys[i],  # noqa: E731
+                                                   N=L.N, K=L.K) for i, L in enumerate(triple)], sign, 0, ws=ws)
+        else:
+            ws = torch.empty(max(bt.gemv_workspace_bytes(0, M, L.N, L.K) for L in triple), dtype=torch.uint8,
+                             device=dev)
+            step = lambda r: [bt.gemv(reps[r][i][0], reps[r][i][1], xs[i], sign, L.N, 0, out=ys[i], ws=ws)  # noqa: E731
+                              for i, L in enumerate(triple)]
+        gemv_us[M] = per_triple_us(step)
+    Mg = 128
+    Xg = [torch.from_numpy(workloads.activations_bf16_bits(g, Mg, L.K, True).view(np.int16)).to(dev)
+          .view(torch.bfloat16) for L in triple]
+    Yg = [torch.empty((Mg, L.N), dtype=torch.bfloat16, device=dev) for L in triple]
+    wsg = torch.empty(max(bt.gemm_workspace_bytes(0, Mg, L.N, L.K) for L in triple), dtype=torch.uint8, device=dev)
+    gemm_us = per_triple_us(lambda r: [bt.gemm(reps[r][i][0], reps[r][i][1], Xg[i], sign, L.N, 0, out=Yg[i], ws=wsg)
+                                       for i, L in enumerate(triple)])
+    del reps
+    rows = {}
+    cross = None
+    for M in (1, 2, 4, 8, 16, 32, 64):
+        gv = gemv_us[M] if M <= 16 else gemv_us[16] * (M // 16)
+        rows[f"M{M}"] = {"gemv_us": round(gv, 2), "gemm_padded_us": round(gemm_us, 2),
+                         "gemv_tokens_per_s": round(M / gv * 1e6, 1), "gemm_tokens_per_s": round(M / gemm_us * 1e6, 1)}
+        if cross is None and gemm_us <= gv:
+            cross = M
+    return {"triple": "5120x5120 / 5120x17408 / 17408x5120, base-3", "gemm_M": Mg, "rows": rows,
+            "crossover_M": cross, "note": "GEMV above M = 16 is M/16 calls of 16 rows"}
 
 
 def run_fwht_sweep(bt, torch, dev, stream, sign):
