@@ -14,8 +14,9 @@
 // (section 实测吞吐).
 //
 // Work. A launch's (matrix, 512-chunk, row) items, in that order, are cut
-// into one contiguous range per CTA (one CTA per SM), so every CTA streams the
-// same number of row chunks. A range is a few segments (matrix p, chunk c,
+// into one contiguous range per CTA (one CTA per SM), balanced so that every
+// CTA streams about the same number of row chunks once the chunk starts it
+// takes on are counted (each costs about 256 rows of streaming). A range is a few segments (matrix p, chunk c,
 // rows n0..n1); per segment the CTA rotates the 1024-block holding the chunk
 // (the warp FWHT of the Sylvester H_1024, S applied first, 1/32; TensorSharp
 // blog, sections 3.2 and 5.2) unless it already holds it, builds the chunk's
@@ -445,6 +446,34 @@ struct LutSeg {
     int p, c, n0, n1;
 };
 
+// A CTA's share of the launch's (matrix, chunk, row) items. Starting a chunk
+// (rotation, scatter, table build) costs about kLutHead rows of streaming, so
+// the items are laid on a cost line where every chunk start takes kLutHead
+// units before its rows; CTA b takes the items of cost range
+// [C b / G, C (b + 1) / G). A share that crosses a chunk start gets that many
+// fewer rows; consecutive shares meet exactly.
+constexpr int kLutHead = 256;
+
+__device__ __forceinline__ int64_t lut_item_at_cost(const LutParams& P, int64_t x) {
+    for (int p = 0; p < P.nprob; ++p) {
+        const int64_t per = kLutHead + (int64_t)P.p[p].N;
+        const int64_t span = per * P.p[p].nchunk;
+        if (x < span) {
+            const int64_t c = x / per, w = x - c * per;
+            return P.p[p].rc_base + c * P.p[p].N + (w > kLutHead ? w - kLutHead : 0);
+        }
+        x -= span;
+    }
+    return P.total_rc;
+}
+
+__device__ __forceinline__ void lut_share(const LutParams& P, int64_t& rc0, int64_t& rc1) {
+    int64_t C = 0;
+    for (int p = 0; p < P.nprob; ++p) C += (kLutHead + (int64_t)P.p[p].N) * P.p[p].nchunk;
+    rc0 = lut_item_at_cost(P, C * blockIdx.x / gridDim.x);
+    rc1 = lut_item_at_cost(P, C * (blockIdx.x + 1) / gridDim.x);
+}
+
 __device__ __forceinline__ bool lut_next_seg(const LutParams& P, int64_t& rc, int64_t rc1, LutSeg& s) {
     if (rc >= rc1) return false;
     int p = 0;
@@ -625,14 +654,14 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_lut_kernel(const __grid_c
         reinterpret_cast<uint4*>(sgn)[threadIdx.x] = __ldg(reinterpret_cast<const uint4*>(P.sign) + threadIdx.x);
     lut_zero_invalid<LAYOUT>(table);
 
-    // This CTA's contiguous share of the launch's (matrix, chunk, row) items,
-    // cut into segments. Each warp requests its sets (warp, warp + 16, ... of
+    // This CTA's contiguous share of the launch's (matrix, chunk, row) items
+    // (lut_share), cut into segments. Each warp requests its sets (warp, warp + 16, ... of
     // every segment) in order through its own cursor, up to kLutDepth ahead of
     // the set it works on, across segment boundaries. Weights, scales and S
     // are never written by the kernels this launch may overlap, so the first
     // sets go out before the grid dependency is resolved.
-    const int64_t rc0 = P.total_rc * blockIdx.x / gridDim.x;
-    const int64_t rc1 = P.total_rc * (blockIdx.x + 1) / gridDim.x;
+    int64_t rc0, rc1;
+    lut_share(P, rc0, rc1);
     uint32_t issued = 0, done = 0;  // sets requested / consumed by this warp
     bool ok = true;
     LutSeg is;
@@ -1021,8 +1050,8 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_mma_kernel(const __grid_c
     __syncwarp();
     if constexpr (LAYOUT == BT_LAYOUT_B3) b3_lut_fill(lut_smem, threadIdx.x, kLutThreads);
 
-    const int64_t rc0 = P.total_rc * blockIdx.x / gridDim.x;
-    const int64_t rc1 = P.total_rc * (blockIdx.x + 1) / gridDim.x;
+    int64_t rc0, rc1;
+    lut_share(P, rc0, rc1);
     uint32_t issued = 0, done = 0;
     bool ok = true;
     LutSeg is;

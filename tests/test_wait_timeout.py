@@ -37,7 +37,7 @@ def _waittest_lib():
 
 def test_withheld_copy_times_out_and_the_context_survives():
     dev = torch.device("cuda:0")
-    # 152 chunks of 512: CTA 0's share starts with 1000 rows of chunk 0, so its
+    # 152 chunks of 512: CTA 0's share is the 1000 rows of chunk 0, so its
     # warp 0 streams sets 0, 16, 32 and 48 and the second of them is left out
     N, K = 1000, 76 * 1024
     case = workloads.random_case(11000, 1, N, K)
@@ -71,7 +71,7 @@ def test_withheld_copy_times_out_and_the_context_survives():
 
 def test_withheld_copy_twice_then_a_correct_call():
     dev = torch.device("cuda:0")
-    N, K = 5120, 5120          # CTA 0's share: 346 rows of chunk 0, sets 0 and 16 for warp 0
+    N, K = 17408, 5120         # CTA 0's share: over 900 rows of chunk 0, so warp 0 has sets 0, 16, 32, ...
     case = workloads.random_case(11100, 1, N, K)
     codes = bt.pack(torch.from_numpy(case["trits"]).to(dev))
     scales = torch.from_numpy(case["scales"].view(np.int16)).to(dev)
