@@ -297,30 +297,66 @@ __global__ void __launch_bounds__(kGemmPrepWarps * 32) gemm_prep_kernel(GemmPrep
     const int m = blockIdx.x;
     const int nblocks = (a.K + kBlock - 1) / kBlock;
     float amax = 0.f;
-    for (int b = warp; b < nblocks; b += kGemmPrepWarps) {
-        const int64_t k0 = (int64_t)b * kBlock;
-        float v[32];
-        if (a.sign) {
-            load_signed_bf16_block(reinterpret_cast<const uint16_t*>(a.x) + (int64_t)m * a.K + k0, a.sign, v);
+    if (a.sign) {
+        // bf16 blocks with S: the next block's raw words are loaded while the
+        // current one is rotated, so the row's loads overlap
+        const uint16_t* xrow = reinterpret_cast<const uint16_t*>(a.x) + (int64_t)m * a.K;
+        const uint4* sg = reinterpret_cast<const uint4*>(a.sign + 32 * lane);
+        const uint4 s0 = __ldg(sg), s1 = __ldg(sg + 1);
+        const uint32_t sw[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+        uint4 nxt[4];
+        int b = warp;
+        if (b < nblocks) {
+            const uint4* src = reinterpret_cast<const uint4*>(xrow + (int64_t)b * kBlock + 32 * lane);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) nxt[q] = __ldg(src + q);
+        }
+        for (; b < nblocks; b += kGemmPrepWarps) {
+            uint4 cur[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) cur[q] = nxt[q];
+            if (b + kGemmPrepWarps < nblocks) {
+                const uint4* src =
+                    reinterpret_cast<const uint4*>(xrow + (int64_t)(b + kGemmPrepWarps) * kBlock + 32 * lane);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) nxt[q] = __ldg(src + q);
+            }
+            float v[32];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                const uint32_t ww[4] = {cur[q].x, cur[q].y, cur[q].z, cur[q].w};
+#pragma unroll
+                for (int h = 0; h < 4; ++h)
+#pragma unroll
+                    for (int half = 0; half < 2; ++half) {
+                        const int i = 8 * q + 2 * h + half;
+                        const uint32_t bits = half ? (ww[h] & 0xFFFF0000u) : (ww[h] << 16);
+                        const uint32_t sbyte = (sw[i >> 2] >> (8 * (i & 3))) & 0x80u;  // bit 7: negative
+                        v[i] = __uint_as_float(bits ^ (sbyte << 24));
+                    }
+            }
             fwht1024_warp(v, tiles + warp * 32 * kTileStride);
-        } else {
+            const int64_t k0 = (int64_t)b * kBlock;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                rowbuf[k0 + 32 * j + lane] = v[j];
+                amax = fmaxf(amax, fabsf(v[j]));
+            }
+        }
+    } else {
+        for (int b = warp; b < nblocks; b += kGemmPrepWarps) {
+            const int64_t k0 = (int64_t)b * kBlock;
 #pragma unroll
             for (int j = 0; j < 32; ++j) {
                 const int64_t idx = k0 + 32 * j + lane;
-                float val = 0.f;
                 if (idx < a.K) {
                     const int64_t off = (int64_t)m * a.K + idx;
-                    val = a.x_bf16 ? bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(a.x)[off])
-                                   : reinterpret_cast<const float*>(a.x)[off];
+                    const float val = a.x_bf16 ? bf16_bits_to_f32(reinterpret_cast<const uint16_t*>(a.x)[off])
+                                               : reinterpret_cast<const float*>(a.x)[off];
+                    rowbuf[idx] = val;
+                    amax = fmaxf(amax, fabsf(val));
                 }
-                v[j] = val;
             }
-        }
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            const int64_t idx = k0 + 32 * j + lane;
-            if (idx < a.K) rowbuf[idx] = v[j];
-            amax = fmaxf(amax, fabsf(v[j]));
         }
     }
 #pragma unroll
@@ -334,10 +370,18 @@ __global__ void __launch_bounds__(kGemmPrepWarps * 32) gemm_prep_kernel(GemmPrep
     e = max(-110, min(110, e));
     const float inv = __int_as_float((127 - e) << 23);
     if (threadIdx.x == 0) a.rowscale[m] = __int_as_float((127 + e) << 23);
-    __half* dst = a.xt + (int64_t)m * a.K;
-    for (int idx = threadIdx.x; idx < a.K; idx += blockDim.x) {
-        const int g = idx >> 7, slot = idx & 127;
-        dst[idx] = __float2half_rn(rowbuf[g * kGroup + gemm_slot_k(a.layout, slot)] * inv);
+    // eight consecutive slots per thread, one 16-byte store (K % 128 == 0)
+    uint4* dst = reinterpret_cast<uint4*>(a.xt + (int64_t)m * a.K);
+    for (int o = threadIdx.x; o < a.K / 8; o += blockDim.x) {
+        const int idx = 8 * o, g = idx >> 7, slot0 = idx & 127;
+        uint32_t w4[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const __half lo = __float2half_rn(rowbuf[g * kGroup + gemm_slot_k(a.layout, slot0 + 2 * u)] * inv);
+            const __half hi = __float2half_rn(rowbuf[g * kGroup + gemm_slot_k(a.layout, slot0 + 2 * u + 1)] * inv);
+            w4[u] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+        }
+        dst[o] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
     }
 }
 
