@@ -1141,21 +1141,30 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_mma_kernel(const __grid_c
                 }
                 const float sgv = f16_bits_to_f32(lds_u16(ss + g * 16 + 2 * q));
                 const float shv = f16_bits_to_f32(lds_u16(ss + (g + 8) * 16 + 2 * q));
+                // B fragments of this lane's activation rows g (block 0) and 8 + g (block 1)
+                uint32_t bf[NB][NT][2];
 #pragma unroll
                 for (int b = 0; b < NB; ++b) {
-                    const int m = 8 * b + g;  // this lane's activation row in the B fragment
-                    uint32_t bf[NT][2];
+                    const int m = 8 * b + g;
                     const uint32_t ba = slots_s + (uint32_t)(((q * NT) * M + m) * 32 + c * 8);
 #pragma unroll
                     for (int t = 0; t < NT; ++t) {
                         uint2 v = make_uint2(0u, 0u);
                         if (m < M) v = lds_u64(ba + (uint32_t)(t * M * 32));
-                        bf[t][0] = v.x;
-                        bf[t][1] = v.y;
+                        bf[b][t][0] = v.x;
+                        bf[b][t][1] = v.y;
                     }
-                    float d4[4];
-                    if constexpr (LAYOUT == BT_LAYOUT_B3) b3_group_mma(Rg, Rh, QG, QH, bf, d4);
-                    else tb_group_mma(Rg, Rh, bf, d4);
+                }
+                float d4[NB][4];
+                if constexpr (NB == 2) {
+                    group_mma2<LAYOUT == BT_LAYOUT_B3>(Rg, Rh, QG, QH, bf[0], bf[1], d4[0], d4[1]);
+                } else if constexpr (LAYOUT == BT_LAYOUT_B3) {
+                    b3_group_mma(Rg, Rh, QG, QH, bf[0], d4[0]);
+                } else {
+                    tb_group_mma(Rg, Rh, bf[0], d4[0]);
+                }
+#pragma unroll
+                for (int b = 0; b < NB; ++b) {
                     // D columns 2c, 2c + 1 of this block are activation rows 8 b + 2c (+1)
                     const int m0 = 8 * b + 2 * c;
                     const uint2 md0 = m0 < M ? lds_u64(meta_s + (uint32_t)((q * M + m0) * 8)) : make_uint2(0u, 0u);
@@ -1163,10 +1172,10 @@ __global__ void __launch_bounds__(kLutThreads, 1) gemv_mma_kernel(const __grid_c
                                                  : make_uint2(0u, 0u);
                     const float c0 = __uint_as_float(md0.x), p0 = __uint_as_float(md0.y);
                     const float c1 = __uint_as_float(md1.x), p1 = __uint_as_float(md1.y);
-                    acc[b][0] = fmaf(sgv, fmaf(d4[0], p0, -c0), acc[b][0]);
-                    acc[b][1] = fmaf(sgv, fmaf(d4[1], p1, -c1), acc[b][1]);
-                    acc[b][2] = fmaf(shv, fmaf(d4[2], p0, -c0), acc[b][2]);
-                    acc[b][3] = fmaf(shv, fmaf(d4[3], p1, -c1), acc[b][3]);
+                    acc[b][0] = fmaf(sgv, fmaf(d4[b][0], p0, -c0), acc[b][0]);
+                    acc[b][1] = fmaf(sgv, fmaf(d4[b][1], p1, -c1), acc[b][1]);
+                    acc[b][2] = fmaf(shv, fmaf(d4[b][2], p0, -c0), acc[b][2]);
+                    acc[b][3] = fmaf(shv, fmaf(d4[b][3], p1, -c1), acc[b][3]);
                 }
             }
             __syncwarp();

@@ -200,6 +200,41 @@ __device__ __forceinline__ void b3_group_mma(const uint32_t (&Rg)[16], const uin
     for (int r = 0; r < 4; ++r) d[r] += e4[r];
 }
 
+// The same chains for two n8 blocks of B that share the A registers, issued
+// interleaved so each block's MMA hides the other's latency; each block's D is
+// bitwise what b3_group_mma / tb_group_mma would give it.
+template <bool B3, int NB>
+__device__ __forceinline__ void group_mma2(const uint32_t (&Rg)[16], const uint32_t (&Rh)[16],
+                                           const uint32_t (&QG)[3], const uint32_t (&QH)[3],
+                                           const uint32_t (&b0)[NB][2], const uint32_t (&b1)[NB][2], float (&d0)[4],
+                                           float (&d1)[4]) {
+    float e0[4] = {0.f, 0.f, 0.f, 0.f}, e1[4] = {0.f, 0.f, 0.f, 0.f};
+    d0[0] = d0[1] = d0[2] = d0[3] = 0.f;
+    d1[0] = d1[1] = d1[2] = d1[3] = 0.f;
+    constexpr int T = B3 ? 7 : 8;
+#pragma unroll
+    for (int t = 0; t < T; ++t) {
+        if (t & 1) {
+            mma_f16_16816(e0, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1], b0[t][0], b0[t][1], e0);
+            mma_f16_16816(e1, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1], b1[t][0], b1[t][1], e1);
+        } else {
+            mma_f16_16816(d0, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1], b0[t][0], b0[t][1], d0);
+            mma_f16_16816(d1, Rg[2 * t], Rh[2 * t], Rg[2 * t + 1], Rh[2 * t + 1], b1[t][0], b1[t][1], d1);
+        }
+    }
+    if constexpr (B3) {
+        mma_f16_16816(e0, Rg[14], Rh[14], QG[0], QH[0], b0[7][0], b0[7][1], e0);
+        mma_f16_16816(e1, Rg[14], Rh[14], QG[0], QH[0], b1[7][0], b1[7][1], e1);
+        mma_f16_16816(d0, QG[1], QH[1], QG[2], QH[2], b0[8][0], b0[8][1], d0);
+        mma_f16_16816(d1, QG[1], QH[1], QG[2], QH[2], b1[8][0], b1[8][1], d1);
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        d0[r] += e0[r];
+        d1[r] += e1[r];
+    }
+}
+
 template <int NB>
 __device__ __forceinline__ void tb_group_mma(const uint32_t (&Rg)[16], const uint32_t (&Rh)[16],
                                              const uint32_t (&bf)[NB][2], float (&d)[4]) {
