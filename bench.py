@@ -38,7 +38,7 @@ L2_BYTES = 126 * 1024 * 1024
 # decode triple (one bt_gemv_batched call), from an ncu capture of the current
 # kernel (dram__bytes_read.sum + dram__bytes_write.sum); None when the kernel
 # has changed since the counters were taken.
-TRAFFIC_PER_LAUNCH = 44_844_288
+TRAFFIC_PER_LAUNCH = 44_860_160
 STEPS_PER_GRAPH = 4
 
 
