@@ -227,10 +227,10 @@ bt_status bt_gemv_batched(int layout, const bt_gemv_problem* problems, int count
  * Arguments and results are those of bt_gemv without the workspace: the
  * scratch is an 8 MiB array in the library's own device memory, reserved on
  * every GPU that loads libbt.so until the process exits. Requests whose
- * bt_gemv_workspace_bytes exceeds 8 MiB (for example M >= 13 on 17408-row
- * matrices of K = 17408, or single rows with N * K / 512 above 2^21: N = K =
- * 32768 fits, N = K = 33792 does not) are rejected with BT_ERR_WORKSPACE
- * before anything is launched.
+ * bt_gemv_workspace_bytes exceeds 8 MiB return BT_ERR_WORKSPACE before
+ * anything is launched. On the decode shapes, M <= 16 fits on 5120x5120,
+ * M <= 11 on 5120x17408 and 17408x5120, M <= 3 on 17408x17408; single rows fit
+ * up to N * K / 512 = 2^21 (N = K = 32768 fits, N = K = 33792 does not).
  * The first call in a CUDA context looks up the array's device address
  * (for the usual primary context: once per device, with that device
  * current) and caches it for that context; a context created later on the

@@ -161,3 +161,15 @@ def test_batched_validation(lib):
     arr[0].N = 64 * 1024                              # problem 1 reads problem 0: two groups
     need = lib.bt_gemv_batched_workspace_bytes(0, arr, 2)
     assert need == (64 * 1024 * 2 + 64 * 128) * 4       # every matrix keeps its partials until the end
+
+
+def test_noalloc_limits_stated_in_the_header(lib):
+    # the 8 MiB built-in scratch: the largest M that fits on each decode shape, as bt.h states it
+    lim = 8 << 20
+    for layout in (bt.LAYOUT_B3, bt.LAYOUT_2BIT):
+        for (N, K), mmax in (((5120, 5120), 16), ((5120, 17408), 11), ((17408, 5120), 11), ((17408, 17408), 3)):
+            assert lib.bt_gemv_workspace_bytes(layout, mmax, N, K) <= lim
+            if mmax < 16:
+                assert lib.bt_gemv_workspace_bytes(layout, mmax + 1, N, K) > lim
+    assert lib.bt_gemv_workspace_bytes(0, 1, 32768, 32768) <= lim
+    assert lib.bt_gemv_workspace_bytes(0, 1, 33792, 33792) > lim
