@@ -1,4 +1,6 @@
 // C ABI of libbt.so: host-side validation and dispatch (declared in include/bt.h).
+#include <atomic>
+
 #include "bt_internal.cuh"
 
 namespace bt {
@@ -35,13 +37,28 @@ namespace {
 constexpr int kVersion = 1;
 constexpr int kDefaultSms = 148;   // B200; used when no device can be queried
 
+// SM count of the current device, looked up once per device ordinal. Without
+// a usable device (a build or test machine) every query would retry the
+// driver's initialisation, so a failed query is remembered too.
 int current_sm_count() {
+    static std::atomic<int> no_device{0};
+    static std::atomic<int> cached[64];
+    if (no_device.load(std::memory_order_relaxed)) return kDefaultSms;
     int dev = 0, sms = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) { cudaGetLastError(); return kDefaultSms; }
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        cudaGetLastError();
+        no_device.store(1, std::memory_order_relaxed);
+        return kDefaultSms;
+    }
+    if (dev >= 0 && dev < 64) {
+        const int c = cached[dev].load(std::memory_order_relaxed);
+        if (c > 0) return c;
+    }
     if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
         cudaGetLastError();
         return kDefaultSms;
     }
+    if (dev >= 0 && dev < 64) cached[dev].store(sms, std::memory_order_relaxed);
     return sms;
 }
 
