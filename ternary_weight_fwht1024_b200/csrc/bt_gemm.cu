@@ -126,6 +126,33 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+        "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]),
+          "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// NC accumulator columns of one row scaled by rs, rounded to bf16 and stored
+template <int NC>
+__device__ __forceinline__ void epi_store(const uint32_t (&r)[NC], float rs, __nv_bfloat16* dst) {
+    uint32_t packed[NC / 2];
+#pragma unroll
+    for (int j = 0; j < NC / 2; ++j) {
+        const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[2 * j]) * rs,
+                                                        __uint_as_float(r[2 * j + 1]) * rs);
+        packed[j] = *reinterpret_cast<const uint32_t*>(&b2);
+    }
+    uint4* out = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+    for (int v = 0; v < NC / 8; ++v)
+        out[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+}
+
 __device__ __forceinline__ uint32_t hfma2_u32(uint32_t a, uint32_t b, uint32_t c) {
     uint32_t r;
     asm("fma.rn.f16x2 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(c));
@@ -404,12 +431,14 @@ struct GemmArgs {
 #define BT_GEMM_BSTAGES 3
 #endif
 
-template <int LAYOUT, int BN, int STAGES, int ASTAGES = BT_GEMM_ASTAGES>
+template <int LAYOUT, int BN, int STAGES, int ASTAGES = BT_GEMM_ASTAGES, int MT = 1>
 struct GemmSmem {
-    // activation ring (TMA) and ring of decoded weight tiles (BN rows each)
+    // activation ring (TMA; MT tiles of 128 rows per stage) and ring of
+    // decoded weight tiles (BN rows each)
     static constexpr int kAStages = ASTAGES;
     static constexpr int kBStages = STAGES;
-    static constexpr int kA = kGemmBM * kGemmBK * 2;   // 32 KB: two 64-column panels
+    static constexpr int kA1 = kGemmBM * kGemmBK * 2;  // 32 KB per 128-row tile: two 64-column panels
+    static constexpr int kA = MT * kA1;
     static constexpr int kB = BN * kGemmBK * 2;
     static constexpr int kLut = LAYOUT == BT_LAYOUT_B3 ? kGemmLutBytes : 0;
     static constexpr int kBars = 1024;                  // barriers, TMEM address, flags
@@ -424,11 +453,19 @@ struct GemmSmem {
 // leader's barrier; the peer's decoders arrive on their own barrier, which
 // one relay thread forwards to the leader's; each commit arrives on the
 // barrier pair in both CTAs.
-template <int LAYOUT, int BN, int STAGES, int ASTAGES = BT_GEMM_ASTAGES, bool PAIR = false>
+//
+// MT = 2 (pairs only): the pair takes two 256-row activation tiles against the
+// same weight tile, so each decoded weight row serves 512 activation rows; the
+// two accumulators sit side by side in TMEM (columns 0 .. BN - 1 and
+// BN .. 2 BN - 1) and every stage issues the MMAs of both.
+template <int LAYOUT, int BN, int STAGES, int ASTAGES = BT_GEMM_ASTAGES, bool PAIR = false, int MT = 1>
 __global__ void __launch_bounds__(gemm_threads(PAIR ? BN / 2 : BN), 1)
 gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
+    static_assert(MT == 1 || PAIR, "several activation tiles per CTA only in pairs");
+    static_assert(BN % 16 == 0 && (PAIR ? BN / 2 : BN) % 8 == 0, "tile width");
     constexpr int BL = PAIR ? BN / 2 : BN;             // weight rows decoded by this CTA
-    using SM = GemmSmem<LAYOUT, BL, STAGES, ASTAGES>;
+    using SM = GemmSmem<LAYOUT, BL, STAGES, ASTAGES, MT>;
+    constexpr uint32_t kTmemCols = MT * BN <= 128 ? 128 : (MT * BN <= 256 ? 256 : 512);
     extern __shared__ uint8_t gsm_raw[];
     uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(gsm_raw) + 1023) & ~uintptr_t(1023));
     constexpr int SA = SM::kAStages, SB = SM::kBStages;
@@ -447,7 +484,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     // a CTA pair sits along x, so that its two CTAs take the two halves of a
     // 256-row activation tile against the same weight tile
-    const int m0 = (PAIR ? blockIdx.x : blockIdx.y) * kGemmBM, n0 = (PAIR ? blockIdx.y : blockIdx.x) * BN;
+    // a pair's CTA of rank r holds rows r * 128 .. r * 128 + 127 of each of its
+    // MT 256-row activation tiles; m0 is its first tile's
+    const int m0 = PAIR ? ((int)(blockIdx.x >> 1) * MT * 2 + (int)(blockIdx.x & 1)) * kGemmBM
+                        : (int)blockIdx.y * kGemmBM;
+    const int n0 = (PAIR ? blockIdx.y : blockIdx.x) * BN;
     const int ktiles = a.G;
     const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
     const bool leader = rank == 0;
@@ -483,11 +524,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
     if (warp == 1) {
         if constexpr (PAIR) {
             asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
-                         :: "r"(smem_addr(tmem_slot)), "r"(BN <= 128 ? 128 : 256) : "memory");
+                         :: "r"(smem_addr(tmem_slot)), "r"(kTmemCols) : "memory");
             asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
         } else {
             asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                         :: "r"(smem_addr(tmem_slot)), "r"(BN <= 128 ? 128 : 256) : "memory");
+                         :: "r"(smem_addr(tmem_slot)), "r"(kTmemCols) : "memory");
             asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
         }
     }
@@ -511,8 +552,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
                 if constexpr (PAIR) {
                     // the leader's barrier counts both CTAs' activation bytes
                     if (leader) mbar_arrive_tx(smem_addr(fullA + s), 2 * SM::kA);
-                    tma_load_2d_pair(dst, &amap, kt * kGemmBK, m0, smem_addr(fullA + s));
-                    tma_load_2d_pair(dst + SM::kA / 2, &amap, kt * kGemmBK + 64, m0, smem_addr(fullA + s));
+#pragma unroll
+                    for (int j = 0; j < MT; ++j) {
+                        const uint32_t dj = dst + j * SM::kA1;
+                        const int mj = m0 + j * 2 * kGemmBM;
+                        tma_load_2d_pair(dj, &amap, kt * kGemmBK, mj, smem_addr(fullA + s));
+                        tma_load_2d_pair(dj + SM::kA1 / 2, &amap, kt * kGemmBK + 64, mj, smem_addr(fullA + s));
+                    }
                 } else {
                     mbar_arrive_tx(smem_addr(fullA + s), SM::kA);
                     tma_load_2d(dst, &amap, kt * kGemmBK, m0, smem_addr(fullA + s));
@@ -537,12 +583,16 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
                 const uint32_t sb = smem_addr(b_ring + s_b * SM::kB);
 #pragma unroll
                 for (int k = 0; k < kGemmBK / 16; ++k) {
-                    const uint32_t pa = sa + (k >> 2) * (SM::kA / 2) + (k & 3) * 32;
                     const uint32_t pb = sb + (k >> 2) * (SM::kB / 2) + (k & 3) * 32;
-                    if constexpr (PAIR)
-                        tc_mma_pair(tmem, smem_desc_sw128(pa), smem_desc_sw128(pb), idesc, (kt > 0 || k > 0) ? 1u : 0u);
-                    else
-                        tc_mma(tmem, smem_desc_sw128(pa), smem_desc_sw128(pb), idesc, (kt > 0 || k > 0) ? 1u : 0u);
+#pragma unroll
+                    for (int j = 0; j < MT; ++j) {
+                        const uint32_t pa = sa + j * SM::kA1 + (k >> 2) * (SM::kA1 / 2) + (k & 3) * 32;
+                        if constexpr (PAIR)
+                            tc_mma_pair(tmem + j * BN, smem_desc_sw128(pa), smem_desc_sw128(pb), idesc,
+                                        (kt > 0 || k > 0) ? 1u : 0u);
+                        else
+                            tc_mma(tmem, smem_desc_sw128(pa), smem_desc_sw128(pb), idesc, (kt > 0 || k > 0) ? 1u : 0u);
+                    }
                 }
                 if constexpr (PAIR) {
                     tc_commit_pair(smem_addr(emptyA + s_a));
@@ -575,7 +625,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
         // ---------------- decoders: thread (part qq, row t) decodes the 128 /
         // TPR slots of weight row t with index 128 qq / TPR and up; they lie
         // in panel h (64-slot halves of the group)
-        constexpr int TPR = kGemmTpr;
         constexpr int WPT = GemmPart<LAYOUT>::WPT;      // 32-bit words per thread
         const int tt = threadIdx.x - 64;                // 0 .. TPR BL - 1
         const int qq = tt / BL, t = tt - qq * BL;
@@ -692,24 +741,22 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
         tc_fence_after();
         const int quarter = warp & 3;
         const bool do_epi = warp >= 2 && warp < 6 && !*abort_flag;   // one warp per TMEM lane quarter
-        if (do_epi) {
-            const int m = m0 + quarter * 32 + lane;
-            const float rs = a.rowscale[m];
 #pragma unroll 1
-            for (int c0 = 0; c0 < BN; c0 += 32) {
+        for (int j = 0; j < MT && do_epi; ++j) {
+            const int m = m0 + j * 2 * kGemmBM + quarter * 32 + lane;
+            const float rs = a.rowscale[m];
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + j * BN;
+            __nv_bfloat16* yrow = a.y + (int64_t)m * a.N + n0;
+#pragma unroll 1
+            for (int c0 = 0; c0 + 32 <= BN; c0 += 32) {
                 uint32_t r[32];
-                tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + c0, r);
-                uint32_t packed[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) {
-                    const __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(r[2 * j]) * rs,
-                                                                    __uint_as_float(r[2 * j + 1]) * rs);
-                    packed[j] = *reinterpret_cast<const uint32_t*>(&b2);
-                }
-                uint4* out = reinterpret_cast<uint4*>(a.y + (int64_t)m * a.N + n0 + c0);
-#pragma unroll
-                for (int v = 0; v < 4; ++v)
-                    out[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+                tmem_ld32(taddr + c0, r);
+                epi_store<32>(r, rs, yrow + c0);
+            }
+            if constexpr (BN % 32 == 16) {   // 80-wide tiles: the last 16 columns
+                uint32_t r[16];
+                tmem_ld16(taddr + BN - 16, r);
+                epi_store<16>(r, rs, yrow + BN - 16);
             }
         }
     }
@@ -721,11 +768,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
         cluster_sync_all();   // both CTAs are done with the pair's TMEM and barriers
         if (warp == 1)
             asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;"
-                         :: "r"(tmem), "r"(BN <= 128 ? 128 : 256) : "memory");
+                         :: "r"(tmem), "r"(kTmemCols) : "memory");
     } else {
         if (warp == 1)
             asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;"
-                         :: "r"(tmem), "r"(BN <= 128 ? 128 : 256) : "memory");
+                         :: "r"(tmem), "r"(kTmemCols) : "memory");
     }
 }
 
@@ -808,15 +855,16 @@ static cudaError_t launch_gemm_t(const CUtensorMap& amap, const GemmArgs& ga, cu
 #ifndef BT_GEMM_PAIR_SA256
 #define BT_GEMM_PAIR_SA256 3
 #endif
-template <int LAYOUT, int BN, int SB, int SA>
+template <int LAYOUT, int BN, int SB, int SA, int MT = 1>
 static cudaError_t launch_gemm_pair_t(const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t stream) {
-    using SM = GemmSmem<LAYOUT, BN / 2, SB, SA>;
+    using SM = GemmSmem<LAYOUT, BN / 2, SB, SA, MT>;
     static_assert(SM::kTotal <= 227 * 1024, "shared memory");
-    auto kern = gemm_kernel<LAYOUT, BN, SB, SA, true>;
+    static_assert(MT * BN <= 512, "TMEM columns");
+    auto kern = gemm_kernel<LAYOUT, BN, SB, SA, true, MT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kTotal);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(ga.M / kGemmBM, ga.N / BN);
+    cfg.gridDim = dim3(ga.M / (kGemmBM * MT), ga.N / BN);
     cfg.blockDim = dim3(gemm_threads(BN / 2));
     cfg.dynamicSmemBytes = SM::kTotal;
     cfg.stream = stream;
@@ -832,10 +880,56 @@ static cudaError_t launch_gemm_pair_t(const CUtensorMap& amap, const GemmArgs& g
     return cudaLaunchKernelEx(&cfg, kern, amap, ga);
 }
 
+// Two 256-row activation tiles per pair (MT = 2) against one weight tile:
+// each decoded weight row meets 512 activation rows, half the decode work per
+// FLOP. The activation ring keeps two 64 KB stages; TMEM holds both
+// accumulators side by side. Tiles 256 wide (N = 17408), or for the 2-bit
+// layout 80 wide (N = 5120, where 160-wide tiles with one activation tile per
+// pair give the same grid), are taken when they fill the SMs as well as the
+// one-tile choice does. On B200 at M = 512 the 256-wide tiles took the
+// 17408 x 5120 layer from 830 to 950 TFLOP/s (base-3) and from 930 to 1210
+// (2-bit); the 80-wide ones took the 2-bit 5120 x 17408 layer from 576 to 599
+// TFLOP/s, and base-3 from 546 to 547 (its 5120 x 5120 layer lost 4 %, so
+// base-3 keeps the 160-wide tiles there).
+struct GemmTile {
+    int bn, mt;
+};
+
+#ifndef BT_GEMM_PAIR_SB80
+#define BT_GEMM_PAIR_SB80 4
+#endif
+
+static GemmTile pick_tile(int layout, int64_t M, int64_t N, int num_sms) {
+    const GemmTile one{pick_bn(M, N, num_sms), 1};
+#if defined(BT_GEMM_NO_PAIR) || defined(BT_GEMM_NO_MT2)
+    (void)layout;
+    return one;
+#else
+    if (!gemm_pairs(M) || M % (4 * kGemmBM) != 0) return one;
+    auto eff = [&](int64_t ctas) {
+        const int64_t waves = (ctas + num_sms - 1) / num_sms;
+        return (double)ctas / (double)(waves * num_sms);
+    };
+    const double e1 = eff((M / kGemmBM) * (N / one.bn));
+    for (int bn : {256, 80}) {
+        if (N % bn || (bn == 80 && layout != BT_LAYOUT_2BIT)) continue;
+        if (eff((M / (2 * kGemmBM)) * (N / bn)) >= e1 - 1e-9) return GemmTile{bn, 2};
+    }
+    return one;
+#endif
+}
+
 template <int LAYOUT>
-static cudaError_t dispatch_gemm(int bn, const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t s) {
+static cudaError_t dispatch_gemm(GemmTile tile, const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t s) {
+    const int bn = tile.bn;
 #ifndef BT_GEMM_NO_PAIR
     if (gemm_pairs(ga.M)) {
+        if (tile.mt == 2 && bn == 256)
+            return launch_gemm_pair_t<LAYOUT, 256, LAYOUT == BT_LAYOUT_B3 ? 2 : 3, 2, 2>(amap, ga, s);
+        if constexpr (LAYOUT == BT_LAYOUT_2BIT) {
+            if (tile.mt == 2 && bn == 80)
+                return launch_gemm_pair_t<LAYOUT, 80, BT_GEMM_PAIR_SB80, 2, 2>(amap, ga, s);
+        }
         if (bn == 256) return launch_gemm_pair_t<LAYOUT, 256, BT_GEMM_PAIR_SB256, BT_GEMM_PAIR_SA256>(amap, ga, s);
         if (bn == 160) return launch_gemm_pair_t<LAYOUT, 160, BT_GEMM_PAIR_SB160, BT_GEMM_PAIR_SA160>(amap, ga, s);
         return launch_gemm_pair_t<LAYOUT, 128, 4, 3>(amap, ga, s);
@@ -899,9 +993,9 @@ cudaError_t launch_gemm(int layout, const uint8_t* codes, const uint16_t* scales
     ga.G = static_cast<int>(K / kGroup);
     ga.row_bytes = (K / kGroup) * (layout == BT_LAYOUT_B3 ? kB3GroupBytes : k2bGroupBytes);
     ga.dev_err = dev_err;
-    const int bn = pick_bn(M, N, num_sms);
-    return layout == BT_LAYOUT_B3 ? dispatch_gemm<BT_LAYOUT_B3>(bn, amap, ga, stream)
-                                  : dispatch_gemm<BT_LAYOUT_2BIT>(bn, amap, ga, stream);
+    const GemmTile tile = pick_tile(layout, M, N, num_sms);
+    return layout == BT_LAYOUT_B3 ? dispatch_gemm<BT_LAYOUT_B3>(tile, amap, ga, stream)
+                                  : dispatch_gemm<BT_LAYOUT_2BIT>(tile, amap, ga, stream);
 }
 
 }  // namespace bt

@@ -8,6 +8,8 @@ rotation against |x' - x'_ref| <= 1e-6 * sum_j |x_j| / 32 + 1e-7 per element
 of the value actually returned (bf16 keeps 8 significant bits, so that is
 2^(floor(log2 |y|) - 8), between 2^-9 |y| and 2^-8 |y|).
 """
+import functools
+
 import numpy as np
 import pytest
 import torch
@@ -397,6 +399,40 @@ def test_gemm_prerotated_ragged_blocks(layout, M):
     y_ref, b = oracle.gemv(case["trits"], case["scales"], xr32)
     y = run_gemm(case["trits"], case["scales"], None, None, layout, x_f32=xr32)
     check_bf16(y, y_ref, b)
+
+
+@functools.lru_cache(maxsize=2)
+def _two_tile_case(N):
+    # at M = 512, N = 17408 takes 256-wide weight tiles with two 256-row
+    # activation tiles per CTA pair, and so does N = 5120 in the 2-bit layout
+    # with 80-wide tiles (base-3: 160-wide tiles, one activation tile per
+    # pair); K = 1152 keeps the whole output cheap for the oracle (and has an
+    # odd number of K groups)
+    M, K = 512, 1152
+    case = workloads.random_case(8550 + N, M, N, K)
+    xr = workloads.rng(8551 + N).standard_normal((M, K)) * 2.0
+    xr32 = xr.astype(np.float32).astype(np.float64)
+    y_ref, b = oracle.gemv(case["trits"], case["scales"], xr32)
+    return case, xr32, y_ref, b
+
+
+@pytest.mark.parametrize("N", [17408, 5120])
+@pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
+def test_gemm_two_tiles_per_pair_full(layout, N):
+    case, xr32, y_ref, b = _two_tile_case(N)
+    y = run_gemm(case["trits"], case["scales"], None, None, layout, x_f32=xr32)
+    check_bf16(y, y_ref, b)
+
+
+def test_gemm_two_tiles_per_pair_two_pairs_sampled_rows():
+    # M = 1024: two pairs along M, each with two activation tiles
+    M, N, K = 1024, 17408, 2048
+    case = workloads.random_case(8560, M, N, K)
+    y = run_gemm(case["trits"], case["scales"], case["x"], case["sign"])
+    rows = tile_rows(M, 8561)
+    xr = oracle.rotate_bf16(case["x"][rows], case["sign"])
+    y_ref, b = oracle.gemv(case["trits"], case["scales"], xr)
+    check_bf16(y[rows], y_ref, b)
 
 
 @pytest.mark.parametrize("M", [128, 256])
