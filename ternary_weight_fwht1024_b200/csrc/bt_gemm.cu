@@ -300,6 +300,8 @@ struct GemmPrepArgs {
     int layout;
     __half* xt;           // [M][K] FP16, slot order within each group
     float* rowscale;      // [M] 2^e_m
+    int32_t* tile_cnt;    // nullable: split-K arrival counters, zeroed here
+    int n_cnt;
 };
 
 __device__ __forceinline__ int gemm_slot_k(int layout, int slot) {
@@ -320,6 +322,10 @@ __global__ void __launch_bounds__(kGemmPrepWarps * 32) gemm_prep_kernel(GemmPrep
     __shared__ float red[kGemmPrepWarps];
     pdl_launch_dependents();
     pdl_wait();
+    // the preceding GEMM of the stream is complete here, and the GEMM that
+    // follows reads the counters only after this kernel has finished
+    if (a.tile_cnt && blockIdx.x == 0)
+        for (int i = threadIdx.x; i < a.n_cnt; i += blockDim.x) a.tile_cnt[i] = 0;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int m = blockIdx.x;
     const int nblocks = (a.K + kBlock - 1) / kBlock;
@@ -422,6 +428,8 @@ struct GemmArgs {
     int M, N, K, G;
     int64_t row_bytes;
     int32_t* dev_err;
+    float* part;          // split-K: [2][M][N] FP32 partial products
+    int32_t* tile_cnt;    // split-K: [tiles][4] arrivals per epilogue warp
 };
 
 #ifndef BT_GEMM_ASTAGES
@@ -458,10 +466,17 @@ struct GemmSmem {
 // same weight tile, so each decoded weight row serves 512 activation rows; the
 // two accumulators sit side by side in TMEM (columns 0 .. BN - 1 and
 // BN .. 2 BN - 1) and every stage issues the MMAs of both.
-template <int LAYOUT, int BN, int STAGES, int ASTAGES = BT_GEMM_ASTAGES, bool PAIR = false, int MT = 1>
+//
+// KS = 2 or 3 (split K): blockIdx.z takes 1 / KS of the K groups. Each
+// epilogue warp stores its chunks' FP32 partial products, then counts itself
+// in on its tile; the warp that arrives last adds the KS partials in split
+// order, scales and writes the bf16 rows. Nobody waits for anybody.
+template <int LAYOUT, int BN, int STAGES, int ASTAGES = BT_GEMM_ASTAGES, bool PAIR = false, int MT = 1,
+          int KS = 1>
 __global__ void __launch_bounds__(gemm_threads(PAIR ? BN / 2 : BN), 1)
 gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
     static_assert(MT == 1 || PAIR, "several activation tiles per CTA only in pairs");
+    static_assert(KS >= 1 && KS <= 3 && (KS == 1 || BN % 32 == 0), "K splits");
     static_assert(BN % 16 == 0 && (PAIR ? BN / 2 : BN) % 8 == 0, "tile width");
     constexpr int BL = PAIR ? BN / 2 : BN;             // weight rows decoded by this CTA
     using SM = GemmSmem<LAYOUT, BL, STAGES, ASTAGES, MT>;
@@ -489,7 +504,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
     const int m0 = PAIR ? ((int)(blockIdx.x >> 1) * MT * 2 + (int)(blockIdx.x & 1)) * kGemmBM
                         : (int)blockIdx.y * kGemmBM;
     const int n0 = (PAIR ? blockIdx.y : blockIdx.x) * BN;
-    const int ktiles = a.G;
+    // K groups [kbase, kbase + ktiles) of this CTA
+    const int kbase = KS == 1 ? 0 : (int)blockIdx.z * a.G / KS;
+    const int ktiles = KS == 1 ? a.G : ((int)blockIdx.z + 1) * a.G / KS - kbase;
     const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
     const bool leader = rank == 0;
 
@@ -556,13 +573,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
                     for (int j = 0; j < MT; ++j) {
                         const uint32_t dj = dst + j * SM::kA1;
                         const int mj = m0 + j * 2 * kGemmBM;
-                        tma_load_2d_pair(dj, &amap, kt * kGemmBK, mj, smem_addr(fullA + s));
-                        tma_load_2d_pair(dj + SM::kA1 / 2, &amap, kt * kGemmBK + 64, mj, smem_addr(fullA + s));
+                        const int kx = (kbase + kt) * kGemmBK;
+                        tma_load_2d_pair(dj, &amap, kx, mj, smem_addr(fullA + s));
+                        tma_load_2d_pair(dj + SM::kA1 / 2, &amap, kx + 64, mj, smem_addr(fullA + s));
                     }
                 } else {
                     mbar_arrive_tx(smem_addr(fullA + s), SM::kA);
-                    tma_load_2d(dst, &amap, kt * kGemmBK, m0, smem_addr(fullA + s));
-                    tma_load_2d(dst + SM::kA / 2, &amap, kt * kGemmBK + 64, m0, smem_addr(fullA + s));
+                    tma_load_2d(dst, &amap, (kbase + kt) * kGemmBK, m0, smem_addr(fullA + s));
+                    tma_load_2d(dst + SM::kA / 2, &amap, (kbase + kt) * kGemmBK + 64, m0, smem_addr(fullA + s));
                 }
             }
         }
@@ -647,6 +665,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
         const int p_lo = (WPT * qq) / 5;
         auto load_group = [&](int kt, uint32_t (&dst)[NW], uint32_t& sc) {
             if (kt >= ktiles) return;
+            kt += kbase;
             if constexpr (LAYOUT == BT_LAYOUT_B3) {
                 // the 2 NW bytes from pair p_lo through the 8-byte aligned
                 // window that holds them (alignment taken from the address:
@@ -736,27 +755,114 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
         }
         if (LAYOUT == BT_LAYOUT_B3 ? (err >> 31) : (err != 0)) bad |= BT_DEVERR_INVALID_CODE;
 
-        // ---------------- epilogue: TMEM -> bf16 Y (rows m0 + 32 (warp % 4) + lane)
+        // ---------------- epilogue: TMEM -> bf16 Y. Every decoder warp takes
+        // part: warp w reads TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31, i.e. rows
+        // m0 + 256 j + 32 (w % 4) + lane, and the warps of one lane quarter
+        // share its MT x NCH column chunks of 32 (16 for the last one when
+        // BN % 32 == 16) round-robin
         if (!*abort_flag && !mbar_wait(smem_addr(accf), 0)) { bad |= BT_DEVERR_TIMEOUT; *abort_flag = 1; }
         tc_fence_after();
+        constexpr int NDW = gemm_dec_warps(BL);
+        static_assert(NDW >= 4, "a decoder warp for every TMEM lane quarter");
+        constexpr int NCH = (BN + 31) / 32;
         const int quarter = warp & 3;
-        const bool do_epi = warp >= 2 && warp < 6 && !*abort_flag;   // one warp per TMEM lane quarter
+        const int w0 = 2 + ((quarter + 2) & 3);        // this quarter's first decoder warp
+        const int slot = (warp - w0) >> 2;
+        const int nslot = (NDW + 1 - w0) / 4 + 1;
+        const uint32_t tq = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        // the decision is the whole warp's: TMEM loads and shuffles are warp-collective
+        const bool do_epi = __all_sync(0xffffffffu, !*abort_flag);
+        if constexpr (KS == 1) {
 #pragma unroll 1
-        for (int j = 0; j < MT && do_epi; ++j) {
-            const int m = m0 + j * 2 * kGemmBM + quarter * 32 + lane;
-            const float rs = a.rowscale[m];
-            const uint32_t taddr = tmem + (static_cast<uint32_t>(quarter * 32) << 16) + j * BN;
-            __nv_bfloat16* yrow = a.y + (int64_t)m * a.N + n0;
-#pragma unroll 1
-            for (int c0 = 0; c0 + 32 <= BN; c0 += 32) {
-                uint32_t r[32];
-                tmem_ld32(taddr + c0, r);
-                epi_store<32>(r, rs, yrow + c0);
+            for (int u = slot; u < MT * NCH && do_epi; u += nslot) {
+                const int j = u / NCH, c0 = (u - j * NCH) * 32;
+                const int m = m0 + j * 2 * kGemmBM + quarter * 32 + lane;
+                const float rs = a.rowscale[m];
+                __nv_bfloat16* yrow = a.y + (int64_t)m * a.N + n0 + c0;
+                if (BN % 32 == 16 && c0 + 32 > BN) {
+                    uint32_t r[16];
+                    tmem_ld16(tq + j * BN + c0, r);
+                    epi_store<16>(r, rs, yrow);
+                } else {
+                    uint32_t r[32];
+                    tmem_ld32(tq + j * BN + c0, r);
+                    epi_store<32>(r, rs, yrow);
+                }
             }
-            if constexpr (BN % 32 == 16) {   // 80-wide tiles: the last 16 columns
-                uint32_t r[16];
-                tmem_ld16(taddr + BN - 16, r);
-                epi_store<16>(r, rs, yrow + BN - 16);
+        } else if (do_epi) {
+            // split K: store this split's FP32 partial products, count in; the
+            // warp arriving last (the KS-th, for this warp's chunks of this
+            // tile) adds the KS partials in split order, so the bits do not
+            // depend on who finishes when. Partials move through a per-warp
+            // 32 x 33 shared-memory transpose (the drained activation ring), so
+            // that each global access of the warp covers four whole 128-byte
+            // rows of a chunk instead of 16 bytes of 32 rows.
+            const size_t plane = (size_t)a.M * a.N;
+            const int z = (int)blockIdx.z;
+            float* tb = reinterpret_cast<float*>(a_ring) + (warp - 2) * (32 * 33);
+            const int prow = lane >> 3, pcol = (lane & 7) * 4;   // coalesced role: rows 4 i + prow
+#pragma unroll 1
+            for (int u = slot; u < MT * NCH; u += nslot) {
+                const int j = u / NCH, c0 = (u - j * NCH) * 32;
+                float* base = a.part + z * plane + (int64_t)(m0 + j * 2 * kGemmBM + quarter * 32) * a.N + n0 + c0;
+                uint32_t r[32];
+                tmem_ld32(tq + j * BN + c0, r);
+#pragma unroll
+                for (int c = 0; c < 32; ++c) tb[lane * 33 + c] = __uint_as_float(r[c]);
+                __syncwarp();
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float* t = tb + (4 * i + prow) * 33 + pcol;
+                    *reinterpret_cast<float4*>(base + (int64_t)(4 * i + prow) * a.N + pcol) =
+                        make_float4(t[0], t[1], t[2], t[3]);
+                }
+                __syncwarp();
+            }
+            __threadfence();
+            __syncwarp();
+            int arrived = 0;
+            if (lane == 0)
+                arrived = atomicAdd(a.tile_cnt + ((int)blockIdx.y * (int)gridDim.x + (int)blockIdx.x) * NDW + (warp - 2), 1);
+            arrived = __shfl_sync(0xffffffffu, arrived, 0);
+            if (arrived == KS - 1) {
+                __threadfence();   // the other splits' stores, made visible by their fences, are seen
+#pragma unroll 1
+                for (int u = slot; u < MT * NCH; u += nslot) {
+                    const int j = u / NCH, c0 = (u - j * NCH) * 32;
+                    const int mb = m0 + j * 2 * kGemmBM + quarter * 32;
+                    const int64_t off = (int64_t)mb * a.N + n0 + c0;
+                    float acc[32];
+#pragma unroll
+                    for (int zz = 0; zz < KS; ++zz) {
+                        if (zz == z) {   // warp-uniform
+                            uint32_t r[32];
+                            tmem_ld32(tq + j * BN + c0, r);
+#pragma unroll
+                            for (int c = 0; c < 32; ++c)
+                                acc[c] = zz == 0 ? __uint_as_float(r[c]) : acc[c] + __uint_as_float(r[c]);
+                        } else {
+                            const float* src = a.part + zz * plane + off;
+                            float4 q[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i)
+                                q[i] = __ldcg(reinterpret_cast<const float4*>(src + (int64_t)(4 * i + prow) * a.N + pcol));
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                float* t = tb + (4 * i + prow) * 33 + pcol;
+                                t[0] = q[i].x; t[1] = q[i].y; t[2] = q[i].z; t[3] = q[i].w;
+                            }
+                            __syncwarp();
+#pragma unroll
+                            for (int c = 0; c < 32; ++c)
+                                acc[c] = zz == 0 ? tb[lane * 33 + c] : acc[c] + tb[lane * 33 + c];
+                            __syncwarp();
+                        }
+                    }
+                    uint32_t r[32];
+#pragma unroll
+                    for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(acc[c]);
+                    epi_store<32>(r, a.rowscale[mb + lane], a.y + off + (int64_t)lane * a.N);
+                }
             }
         }
     }
@@ -780,9 +886,6 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
 
 static size_t gemm_align(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
-size_t gemm_workspace_bytes(int, int64_t M, int64_t, int64_t K, int) {
-    return gemm_align((size_t)M * K * 2, 256) + gemm_align((size_t)M * 4, 256);
-}
 
 static bool gemm_pairs(int64_t M) {
 #ifdef BT_GEMM_NO_PAIR
@@ -855,16 +958,16 @@ static cudaError_t launch_gemm_t(const CUtensorMap& amap, const GemmArgs& ga, cu
 #ifndef BT_GEMM_PAIR_SA256
 #define BT_GEMM_PAIR_SA256 3
 #endif
-template <int LAYOUT, int BN, int SB, int SA, int MT = 1>
+template <int LAYOUT, int BN, int SB, int SA, int MT = 1, int KS = 1>
 static cudaError_t launch_gemm_pair_t(const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t stream) {
     using SM = GemmSmem<LAYOUT, BN / 2, SB, SA, MT>;
     static_assert(SM::kTotal <= 227 * 1024, "shared memory");
     static_assert(MT * BN <= 512, "TMEM columns");
-    auto kern = gemm_kernel<LAYOUT, BN, SB, SA, true, MT>;
+    auto kern = gemm_kernel<LAYOUT, BN, SB, SA, true, MT, KS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kTotal);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(ga.M / (kGemmBM * MT), ga.N / BN);
+    cfg.gridDim = dim3(ga.M / (kGemmBM * MT), ga.N / BN, KS);
     cfg.blockDim = dim3(gemm_threads(BN / 2));
     cfg.dynamicSmemBytes = SM::kTotal;
     cfg.stream = stream;
@@ -883,26 +986,31 @@ static cudaError_t launch_gemm_pair_t(const CUtensorMap& amap, const GemmArgs& g
 // Two 256-row activation tiles per pair (MT = 2) against one weight tile:
 // each decoded weight row meets 512 activation rows, half the decode work per
 // FLOP. The activation ring keeps two 64 KB stages; TMEM holds both
-// accumulators side by side. Tiles 256 wide (N = 17408), or for the 2-bit
-// layout 80 wide (N = 5120, where 160-wide tiles with one activation tile per
-// pair give the same grid), are taken when they fill the SMs as well as the
-// one-tile choice does. On B200 at M = 512 the 256-wide tiles took the
-// 17408 x 5120 layer from 830 to 950 TFLOP/s (base-3) and from 930 to 1210
-// (2-bit); the 80-wide ones took the 2-bit 5120 x 17408 layer from 576 to 599
-// TFLOP/s, and base-3 from 546 to 547 (its 5120 x 5120 layer lost 4 %, so
-// base-3 keeps the 160-wide tiles there).
+// accumulators side by side. Candidates, in order, each taken when its grid
+// fills the SMs as well as the one-tile choice does:
+//  - 256 wide (N = 17408 at M = 512: 136 CTAs). On B200 the 17408 x 5120
+//    layer went from 830 to 950 TFLOP/s (base-3), 930 to 1210 (2-bit).
+//  - 160 wide with K split in two (N = 5120 at M = 512: 2 x 64 CTAs, the
+//    same grid as one tile per pair without the split). Half the K groups per
+//    CTA and twice the MMAs per decoded group; the halves meet through FP32
+//    partials in the workspace. 5120 x 17408 went from 546 to 756 TFLOP/s
+//    (base-3) and 576 to 830 (2-bit); 5120 x 5120 from 453 to 487 and 498 to
+//    541. Splitting K in three over 256-wide tiles (120 CTAs, fewer activation
+//    reads) lost: the CTA arriving last adds two partial tiles of 256 KB
+//    alone, which left a 20-30 us tail.
+//  - 80 wide, 2-bit only, where K is too short to split.
 struct GemmTile {
-    int bn, mt;
+    int bn, mt, ks;   // weight tile width, activation tiles per pair, K splits
 };
 
 #ifndef BT_GEMM_PAIR_SB80
 #define BT_GEMM_PAIR_SB80 4
 #endif
 
-static GemmTile pick_tile(int layout, int64_t M, int64_t N, int num_sms) {
-    const GemmTile one{pick_bn(M, N, num_sms), 1};
+static GemmTile pick_tile(int layout, int64_t M, int64_t N, int64_t K, int num_sms) {
+    const GemmTile one{pick_bn(M, N, num_sms), 1, 1};
 #if defined(BT_GEMM_NO_PAIR) || defined(BT_GEMM_NO_MT2)
-    (void)layout;
+    (void)layout; (void)K;
     return one;
 #else
     if (!gemm_pairs(M) || M % (4 * kGemmBM) != 0) return one;
@@ -911,12 +1019,39 @@ static GemmTile pick_tile(int layout, int64_t M, int64_t N, int num_sms) {
         return (double)ctas / (double)(waves * num_sms);
     };
     const double e1 = eff((M / kGemmBM) * (N / one.bn));
-    for (int bn : {256, 80}) {
-        if (N % bn || (bn == 80 && layout != BT_LAYOUT_2BIT)) continue;
-        if (eff((M / (2 * kGemmBM)) * (N / bn)) >= e1 - 1e-9) return GemmTile{bn, 2};
+    const GemmTile cands[] = {{256, 2, 1}, {160, 2, 2}, {80, 2, 1}};
+    for (const GemmTile& c : cands) {
+        if (N % c.bn || (c.bn == 80 && layout != BT_LAYOUT_2BIT)) continue;
+        if (c.ks > 1 && K / kGroup < 8 * c.ks) continue;   // each half keeps a pipeline's worth of K groups
+#ifdef BT_GEMM_NO_SPLITK
+        if (c.ks > 1) continue;
+#endif
+        if (eff((M / (2 * kGemmBM)) * (N / c.bn) * c.ks) >= e1 - 1e-9) return c;
     }
     return one;
 #endif
+}
+
+// workspace: the rotated FP16 activations, the row scales and, for split K,
+// the arrival counters and both halves' FP32 partial products
+struct GemmWs {
+    size_t xt, rowscale, cnt, part, total;
+    int n_cnt;
+};
+
+static GemmWs gemm_ws_layout(const GemmTile& t, int64_t M, int64_t N, int64_t K) {
+    GemmWs w{};
+    w.xt = 0;
+    w.rowscale = gemm_align((size_t)M * K * 2, 256);
+    w.cnt = w.rowscale + gemm_align((size_t)M * 4, 256);
+    w.n_cnt = t.ks > 1 ? (int)((M / (kGemmBM * t.mt)) * (N / t.bn) * gemm_dec_warps(t.bn / 2)) : 0;
+    w.part = w.cnt + gemm_align((size_t)w.n_cnt * 4, 256);
+    w.total = w.part + (t.ks > 1 ? (size_t)t.ks * M * N * 4 : 0);
+    return w;
+}
+
+size_t gemm_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num_sms) {
+    return gemm_ws_layout(pick_tile(layout, M, N, K, num_sms), M, N, K).total;
 }
 
 template <int LAYOUT>
@@ -924,8 +1059,10 @@ static cudaError_t dispatch_gemm(GemmTile tile, const CUtensorMap& amap, const G
     const int bn = tile.bn;
 #ifndef BT_GEMM_NO_PAIR
     if (gemm_pairs(ga.M)) {
-        if (tile.mt == 2 && bn == 256)
+        if (tile.mt == 2 && bn == 256 && tile.ks == 1)
             return launch_gemm_pair_t<LAYOUT, 256, LAYOUT == BT_LAYOUT_B3 ? 2 : 3, 2, 2>(amap, ga, s);
+        if (tile.mt == 2 && bn == 160 && tile.ks == 2)
+            return launch_gemm_pair_t<LAYOUT, 160, LAYOUT == BT_LAYOUT_B3 ? 3 : 4, 2, 2, 2>(amap, ga, s);
         if constexpr (LAYOUT == BT_LAYOUT_2BIT) {
             if (tile.mt == 2 && bn == 80)
                 return launch_gemm_pair_t<LAYOUT, 80, BT_GEMM_PAIR_SB80, 2, 2>(amap, ga, s);
@@ -950,9 +1087,12 @@ cudaError_t launch_gemm(int layout, const uint8_t* codes, const uint16_t* scales
                         int32_t* dev_err, int num_sms, cudaStream_t stream) {
     EncodeTiledFn enc = tensor_map_encoder();
     if (!enc) return cudaErrorNotSupported;
+    const GemmTile tile = pick_tile(layout, M, N, K, num_sms);
+    const GemmWs wl = gemm_ws_layout(tile, M, N, K);
     uint8_t* ws = static_cast<uint8_t*>(workspace);
-    __half* xt = reinterpret_cast<__half*>(ws);
-    float* rowscale = reinterpret_cast<float*>(ws + gemm_align((size_t)M * K * 2, 256));
+    __half* xt = reinterpret_cast<__half*>(ws + wl.xt);
+    float* rowscale = reinterpret_cast<float*>(ws + wl.rowscale);
+    int32_t* tile_cnt = wl.n_cnt ? reinterpret_cast<int32_t*>(ws + wl.cnt) : nullptr;
 
     GemmPrepArgs pa{};
     pa.x = x;
@@ -964,6 +1104,8 @@ cudaError_t launch_gemm(int layout, const uint8_t* codes, const uint16_t* scales
     pa.layout = layout;
     pa.xt = xt;
     pa.rowscale = rowscale;
+    pa.tile_cnt = tile_cnt;
+    pa.n_cnt = wl.n_cnt;
     const size_t prep_smem = (size_t)K * 4 + (size_t)kGemmPrepWarps * 32 * kTileStride * 4;
     cudaError_t e = cudaFuncSetAttribute(gemm_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)prep_smem);
@@ -993,7 +1135,8 @@ cudaError_t launch_gemm(int layout, const uint8_t* codes, const uint16_t* scales
     ga.G = static_cast<int>(K / kGroup);
     ga.row_bytes = (K / kGroup) * (layout == BT_LAYOUT_B3 ? kB3GroupBytes : k2bGroupBytes);
     ga.dev_err = dev_err;
-    const GemmTile tile = pick_tile(layout, M, N, num_sms);
+    ga.part = wl.n_cnt ? reinterpret_cast<float*>(ws + wl.part) : nullptr;
+    ga.tile_cnt = tile_cnt;
     return layout == BT_LAYOUT_B3 ? dispatch_gemm<BT_LAYOUT_B3>(tile, amap, ga, stream)
                                   : dispatch_gemm<BT_LAYOUT_2BIT>(tile, amap, ga, stream);
 }

@@ -126,6 +126,28 @@ def test_gemm_validation(lib):
     assert lib.bt_gemm_workspace_bytes(2, 512, 5120, 5120) == 0
 
 
+def test_gemm_workspace_sizes(lib):
+    # without a GPU the tile choice assumes B200's 148 SMs. The rotated FP16
+    # activations and the row scales, each rounded up to 256 bytes ...
+    def base(M, K):
+        return -(-M * K * 2 // 256) * 256 + -(-M * 4 // 256) * 256
+    # ... are all that 17408 x 5120 needs (256-wide tiles, two activation
+    # tiles per pair, 136 CTAs)
+    assert lib.bt_gemm_workspace_bytes(0, 512, 17408, 5120) == base(512, 5120)
+    # N = 5120 at M = 512 splits K in two over 160-wide tiles: 64 tiles x 10
+    # decoder warps of arrival counters, then both halves' FP32 partials
+    cnt = 64 * 10 * 4
+    for K in (2176, 5120, 17408):
+        for layout in (0, 1):
+            assert lib.bt_gemm_workspace_bytes(layout, 512, 5120, K) == base(512, K) + cnt + 2 * 512 * 5120 * 4
+    # 15 K groups are too few to split: 2-bit takes 80-wide tiles, base-3
+    # 160-wide ones with one activation tile per pair
+    for layout in (0, 1):
+        assert lib.bt_gemm_workspace_bytes(layout, 512, 5120, 1920) == base(512, 1920)
+    # M = 256: one activation tile per pair, nothing but the activations
+    assert lib.bt_gemm_workspace_bytes(0, 256, 5120, 5120) == base(256, 5120)
+
+
 def test_binding_refuses_cpu_tensors():
     import torch
     with pytest.raises(ValueError):

@@ -402,13 +402,14 @@ def test_gemm_prerotated_ragged_blocks(layout, M):
 
 
 @functools.lru_cache(maxsize=2)
-def _two_tile_case(N):
+def _two_tile_case(N, K):
     # at M = 512, N = 17408 takes 256-wide weight tiles with two 256-row
-    # activation tiles per CTA pair, and so does N = 5120 in the 2-bit layout
-    # with 80-wide tiles (base-3: 160-wide tiles, one activation tile per
-    # pair); K = 1152 keeps the whole output cheap for the oracle (and has an
-    # odd number of K groups)
-    M, K = 512, 1152
+    # activation tiles per CTA pair; N = 5120 takes 160-wide tiles with two
+    # activation tiles per pair and K split in two (17 K groups: halves of 8
+    # and 9), the CTA finishing second adding the partial products. Small K
+    # keeps the whole output cheap for the oracle; both have odd numbers of
+    # K groups.
+    M = 512
     case = workloads.random_case(8550 + N, M, N, K)
     xr = workloads.rng(8551 + N).standard_normal((M, K)) * 2.0
     xr32 = xr.astype(np.float32).astype(np.float64)
@@ -416,12 +417,15 @@ def _two_tile_case(N):
     return case, xr32, y_ref, b
 
 
-@pytest.mark.parametrize("N", [17408, 5120])
+@pytest.mark.parametrize("N,K", [(17408, 1152), (5120, 2176)])
 @pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
-def test_gemm_two_tiles_per_pair_full(layout, N):
-    case, xr32, y_ref, b = _two_tile_case(N)
+def test_gemm_two_tiles_per_pair_full(layout, N, K):
+    case, xr32, y_ref, b = _two_tile_case(N, K)
     y = run_gemm(case["trits"], case["scales"], None, None, layout, x_f32=xr32)
     check_bf16(y, y_ref, b)
+    # the splits meet in whichever order they finish: same bits each call
+    y2 = run_gemm(case["trits"], case["scales"], None, None, layout, x_f32=xr32)
+    assert np.array_equal(y, y2)
 
 
 def test_gemm_two_tiles_per_pair_two_pairs_sampled_rows():
