@@ -467,16 +467,16 @@ struct GemmSmem {
 // two accumulators sit side by side in TMEM (columns 0 .. BN - 1 and
 // BN .. 2 BN - 1) and every stage issues the MMAs of both.
 //
-// KS = 2 or 3 (split K): blockIdx.z takes 1 / KS of the K groups. Each
+// SPLIT (split K): blockIdx.z takes 1 / gridDim.z of the K groups. Each
 // epilogue warp stores its chunks' FP32 partial products, then counts itself
-// in on its tile; the warp that arrives last adds the KS partials in split
+// in on its tile; the warp that arrives last adds the partials in split
 // order, scales and writes the bf16 rows. Nobody waits for anybody.
 template <int LAYOUT, int BN, int STAGES, int ASTAGES = BT_GEMM_ASTAGES, bool PAIR = false, int MT = 1,
-          int KS = 1>
+          bool SPLIT = false>
 __global__ void __launch_bounds__(gemm_threads(PAIR ? BN / 2 : BN), 1)
 gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
     static_assert(MT == 1 || PAIR, "several activation tiles per CTA only in pairs");
-    static_assert(KS >= 1 && KS <= 3 && (KS == 1 || BN % 32 == 0), "K splits");
+    static_assert(!SPLIT || BN % 32 == 0, "K splits");
     static_assert(BN % 16 == 0 && (PAIR ? BN / 2 : BN) % 8 == 0, "tile width");
     constexpr int BL = PAIR ? BN / 2 : BN;             // weight rows decoded by this CTA
     using SM = GemmSmem<LAYOUT, BL, STAGES, ASTAGES, MT>;
@@ -505,8 +505,9 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
                         : (int)blockIdx.y * kGemmBM;
     const int n0 = (PAIR ? blockIdx.y : blockIdx.x) * BN;
     // K groups [kbase, kbase + ktiles) of this CTA
-    const int kbase = KS == 1 ? 0 : (int)blockIdx.z * a.G / KS;
-    const int ktiles = KS == 1 ? a.G : ((int)blockIdx.z + 1) * a.G / KS - kbase;
+    const int ks = SPLIT ? (int)gridDim.z : 1;
+    const int kbase = SPLIT ? (int)blockIdx.z * a.G / ks : 0;
+    const int ktiles = SPLIT ? ((int)blockIdx.z + 1) * a.G / ks - kbase : a.G;
     const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
     const bool leader = rank == 0;
 
@@ -772,7 +773,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
         const uint32_t tq = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
         // the decision is the whole warp's: TMEM loads and shuffles are warp-collective
         const bool do_epi = __all_sync(0xffffffffu, !*abort_flag);
-        if constexpr (KS == 1) {
+        if constexpr (!SPLIT) {
 #pragma unroll 1
             for (int u = slot; u < MT * NCH && do_epi; u += nslot) {
                 const int j = u / NCH, c0 = (u - j * NCH) * 32;
@@ -791,12 +792,13 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
             }
         } else if (do_epi) {
             // split K: store this split's FP32 partial products, count in; the
-            // warp arriving last (the KS-th, for this warp's chunks of this
-            // tile) adds the KS partials in split order, so the bits do not
+            // warp arriving last (the ks-th, for this warp's chunks of this
+            // tile) adds the ks partials in split order, so the bits do not
             // depend on who finishes when. Partials move through a per-warp
             // 32 x 33 shared-memory transpose (the drained activation ring), so
             // that each global access of the warp covers four whole 128-byte
             // rows of a chunk instead of 16 bytes of 32 rows.
+            static_assert(!SPLIT || NDW * 32 * 33 * 4 <= SA * SM::kA + SB * SM::kB, "transpose buffers");
             const size_t plane = (size_t)a.M * a.N;
             const int z = (int)blockIdx.z;
             float* tb = reinterpret_cast<float*>(a_ring) + (warp - 2) * (32 * 33);
@@ -824,7 +826,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
             if (lane == 0)
                 arrived = atomicAdd(a.tile_cnt + ((int)blockIdx.y * (int)gridDim.x + (int)blockIdx.x) * NDW + (warp - 2), 1);
             arrived = __shfl_sync(0xffffffffu, arrived, 0);
-            if (arrived == KS - 1) {
+            if (arrived == ks - 1) {
                 __threadfence();   // the other splits' stores, made visible by their fences, are seen
 #pragma unroll 1
                 for (int u = slot; u < MT * NCH; u += nslot) {
@@ -832,8 +834,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
                     const int mb = m0 + j * 2 * kGemmBM + quarter * 32;
                     const int64_t off = (int64_t)mb * a.N + n0 + c0;
                     float acc[32];
-#pragma unroll
-                    for (int zz = 0; zz < KS; ++zz) {
+#pragma unroll 1
+                    for (int zz = 0; zz < ks; ++zz) {
                         if (zz == z) {   // warp-uniform
                             uint32_t r[32];
                             tmem_ld32(tq + j * BN + c0, r);
@@ -842,14 +844,17 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
                                 acc[c] = zz == 0 ? __uint_as_float(r[c]) : acc[c] + __uint_as_float(r[c]);
                         } else {
                             const float* src = a.part + zz * plane + off;
-                            float4 q[8];
 #pragma unroll
-                            for (int i = 0; i < 8; ++i)
-                                q[i] = __ldcg(reinterpret_cast<const float4*>(src + (int64_t)(4 * i + prow) * a.N + pcol));
+                            for (int i0 = 0; i0 < 8; i0 += 4) {   // two rounds of four loads in flight
+                                float4 q[4];
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) {
-                                float* t = tb + (4 * i + prow) * 33 + pcol;
-                                t[0] = q[i].x; t[1] = q[i].y; t[2] = q[i].z; t[3] = q[i].w;
+                                for (int i = 0; i < 4; ++i)
+                                    q[i] = __ldcg(reinterpret_cast<const float4*>(src + (int64_t)(4 * (i0 + i) + prow) * a.N + pcol));
+#pragma unroll
+                                for (int i = 0; i < 4; ++i) {
+                                    float* t = tb + (4 * (i0 + i) + prow) * 33 + pcol;
+                                    t[0] = q[i].x; t[1] = q[i].y; t[2] = q[i].z; t[3] = q[i].w;
+                                }
                             }
                             __syncwarp();
 #pragma unroll
@@ -919,14 +924,14 @@ static int pick_bn(int64_t M, int64_t N, int num_sms) {
     return best;
 }
 
-template <int LAYOUT, int BN, int STAGES>
-static cudaError_t launch_gemm_t(const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t stream) {
+template <int LAYOUT, int BN, int STAGES, bool SPLIT = false>
+static cudaError_t launch_gemm_t(const CUtensorMap& amap, const GemmArgs& ga, int ks, cudaStream_t stream) {
     using SM = GemmSmem<LAYOUT, BN, STAGES>;
-    auto kern = gemm_kernel<LAYOUT, BN, STAGES>;
+    auto kern = gemm_kernel<LAYOUT, BN, STAGES, BT_GEMM_ASTAGES, false, 1, SPLIT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kTotal);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(ga.N / BN, ga.M / kGemmBM);
+    cfg.gridDim = dim3(ga.N / BN, ga.M / kGemmBM, SPLIT ? ks : 1);
     cfg.blockDim = dim3(gemm_threads(BN));
     cfg.dynamicSmemBytes = SM::kTotal;
     cfg.stream = stream;
@@ -958,16 +963,16 @@ static cudaError_t launch_gemm_t(const CUtensorMap& amap, const GemmArgs& ga, cu
 #ifndef BT_GEMM_PAIR_SA256
 #define BT_GEMM_PAIR_SA256 3
 #endif
-template <int LAYOUT, int BN, int SB, int SA, int MT = 1, int KS = 1>
-static cudaError_t launch_gemm_pair_t(const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t stream) {
+template <int LAYOUT, int BN, int SB, int SA, int MT = 1, bool SPLIT = false>
+static cudaError_t launch_gemm_pair_t(const CUtensorMap& amap, const GemmArgs& ga, int ks, cudaStream_t stream) {
     using SM = GemmSmem<LAYOUT, BN / 2, SB, SA, MT>;
     static_assert(SM::kTotal <= 227 * 1024, "shared memory");
     static_assert(MT * BN <= 512, "TMEM columns");
-    auto kern = gemm_kernel<LAYOUT, BN, SB, SA, true, MT, KS>;
+    auto kern = gemm_kernel<LAYOUT, BN, SB, SA, true, MT, SPLIT>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, SM::kTotal);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg{};
-    cfg.gridDim = dim3(ga.M / (kGemmBM * MT), ga.N / BN, KS);
+    cfg.gridDim = dim3(ga.M / (kGemmBM * MT), ga.N / BN, SPLIT ? ks : 1);
     cfg.blockDim = dim3(gemm_threads(BN / 2));
     cfg.dynamicSmemBytes = SM::kTotal;
     cfg.stream = stream;
@@ -1000,33 +1005,56 @@ static cudaError_t launch_gemm_pair_t(const CUtensorMap& amap, const GemmArgs& g
 //    alone, which left a 20-30 us tail.
 //  - 80 wide, 2-bit only, where K is too short to split.
 struct GemmTile {
-    int bn, mt, ks;   // weight tile width, activation tiles per pair, K splits
+    int bn, mt, ks;   // weight tile width, activation tiles per CTA (pair), K splits
+    bool pair;        // CTA pairs (cta_group::2) along M
 };
 
 #ifndef BT_GEMM_PAIR_SB80
 #define BT_GEMM_PAIR_SB80 4
 #endif
 
-static GemmTile pick_tile(int layout, int64_t M, int64_t N, int64_t K, int num_sms) {
-    const GemmTile one{pick_bn(M, N, num_sms), 1, 1};
-#if defined(BT_GEMM_NO_PAIR) || defined(BT_GEMM_NO_MT2)
-    (void)layout; (void)K;
-    return one;
+static double wave_eff(int64_t ctas, int num_sms) {
+    const int64_t waves = (ctas + num_sms - 1) / num_sms;
+    return (double)ctas / (double)(waves * num_sms);
+}
+
+// Small grids (M = 128 or 256 against N = 5120: 32-80 CTAs) split K over the
+// single-CTA kernel, 2 to 4 ways, keeping at least 8 K groups per split; a
+// split is taken when it fills the SMs clearly better (by 5 % of a wave).
+static GemmTile pick_small_split(const GemmTile& one, int64_t M, int64_t N, int64_t K, int num_sms) {
+    GemmTile best = one;
+#ifndef BT_GEMM_NO_SPLITK
+    double best_e = wave_eff((M / kGemmBM) * (N / one.bn), num_sms);
+    for (int bn : {160, 128}) {
+        if (N % bn) continue;
+        const int64_t ctas = (M / kGemmBM) * (N / bn);
+        for (int ks = 2; ks <= 4 && K / kGroup >= 8 * ks; ++ks) {
+            const double e = wave_eff(ctas * ks, num_sms);
+            if (e > best_e + 0.05) { best = GemmTile{bn, 1, ks, false}; best_e = e; }
+        }
+    }
 #else
-    if (!gemm_pairs(M) || M % (4 * kGemmBM) != 0) return one;
-    auto eff = [&](int64_t ctas) {
-        const int64_t waves = (ctas + num_sms - 1) / num_sms;
-        return (double)ctas / (double)(waves * num_sms);
-    };
-    const double e1 = eff((M / kGemmBM) * (N / one.bn));
-    const GemmTile cands[] = {{256, 2, 1}, {160, 2, 2}, {80, 2, 1}};
+    (void)M; (void)N; (void)K; (void)num_sms;
+#endif
+    return best;
+}
+
+static GemmTile pick_tile(int layout, int64_t M, int64_t N, int64_t K, int num_sms) {
+    const GemmTile one{pick_bn(M, N, num_sms), 1, 1, gemm_pairs(M)};
+#if defined(BT_GEMM_NO_PAIR) || defined(BT_GEMM_NO_MT2)
+    (void)layout;
+    return pick_small_split(one, M, N, K, num_sms);
+#else
+    if (!gemm_pairs(M) || M % (4 * kGemmBM) != 0) return pick_small_split(one, M, N, K, num_sms);
+    const double e1 = wave_eff((M / kGemmBM) * (N / one.bn), num_sms);
+    const GemmTile cands[] = {{256, 2, 1, true}, {160, 2, 2, true}, {80, 2, 1, true}};
     for (const GemmTile& c : cands) {
         if (N % c.bn || (c.bn == 80 && layout != BT_LAYOUT_2BIT)) continue;
         if (c.ks > 1 && K / kGroup < 8 * c.ks) continue;   // each half keeps a pipeline's worth of K groups
 #ifdef BT_GEMM_NO_SPLITK
         if (c.ks > 1) continue;
 #endif
-        if (eff((M / (2 * kGemmBM)) * (N / c.bn) * c.ks) >= e1 - 1e-9) return c;
+        if (wave_eff((M / (2 * kGemmBM)) * (N / c.bn) * c.ks, num_sms) >= e1 - 1e-9) return c;
     }
     return one;
 #endif
@@ -1044,7 +1072,7 @@ static GemmWs gemm_ws_layout(const GemmTile& t, int64_t M, int64_t N, int64_t K)
     w.xt = 0;
     w.rowscale = gemm_align((size_t)M * K * 2, 256);
     w.cnt = w.rowscale + gemm_align((size_t)M * 4, 256);
-    w.n_cnt = t.ks > 1 ? (int)((M / (kGemmBM * t.mt)) * (N / t.bn) * gemm_dec_warps(t.bn / 2)) : 0;
+    w.n_cnt = t.ks > 1 ? (int)((M / (kGemmBM * t.mt)) * (N / t.bn) * gemm_dec_warps(t.pair ? t.bn / 2 : t.bn)) : 0;
     w.part = w.cnt + gemm_align((size_t)w.n_cnt * 4, 256);
     w.total = w.part + (t.ks > 1 ? (size_t)t.ks * M * N * 4 : 0);
     return w;
@@ -1058,28 +1086,31 @@ template <int LAYOUT>
 static cudaError_t dispatch_gemm(GemmTile tile, const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t s) {
     const int bn = tile.bn;
 #ifndef BT_GEMM_NO_PAIR
-    if (gemm_pairs(ga.M)) {
-        if (tile.mt == 2 && bn == 256 && tile.ks == 1)
-            return launch_gemm_pair_t<LAYOUT, 256, LAYOUT == BT_LAYOUT_B3 ? 2 : 3, 2, 2>(amap, ga, s);
-        if (tile.mt == 2 && bn == 160 && tile.ks == 2)
-            return launch_gemm_pair_t<LAYOUT, 160, LAYOUT == BT_LAYOUT_B3 ? 3 : 4, 2, 2, 2>(amap, ga, s);
+    if (tile.pair) {
+        if (tile.mt == 2 && bn == 256)
+            return launch_gemm_pair_t<LAYOUT, 256, LAYOUT == BT_LAYOUT_B3 ? 2 : 3, 2, 2>(amap, ga, 1, s);
+        if (tile.mt == 2 && bn == 160 && tile.ks > 1)
+            return launch_gemm_pair_t<LAYOUT, 160, LAYOUT == BT_LAYOUT_B3 ? 3 : 4, 2, 2, true>(amap, ga, tile.ks, s);
         if constexpr (LAYOUT == BT_LAYOUT_2BIT) {
             if (tile.mt == 2 && bn == 80)
-                return launch_gemm_pair_t<LAYOUT, 80, BT_GEMM_PAIR_SB80, 2, 2>(amap, ga, s);
+                return launch_gemm_pair_t<LAYOUT, 80, BT_GEMM_PAIR_SB80, 2, 2>(amap, ga, 1, s);
         }
-        if (bn == 256) return launch_gemm_pair_t<LAYOUT, 256, BT_GEMM_PAIR_SB256, BT_GEMM_PAIR_SA256>(amap, ga, s);
-        if (bn == 160) return launch_gemm_pair_t<LAYOUT, 160, BT_GEMM_PAIR_SB160, BT_GEMM_PAIR_SA160>(amap, ga, s);
-        return launch_gemm_pair_t<LAYOUT, 128, 4, 3>(amap, ga, s);
+        if (bn == 256) return launch_gemm_pair_t<LAYOUT, 256, BT_GEMM_PAIR_SB256, BT_GEMM_PAIR_SA256>(amap, ga, 1, s);
+        if (bn == 160) return launch_gemm_pair_t<LAYOUT, 160, BT_GEMM_PAIR_SB160, BT_GEMM_PAIR_SA160>(amap, ga, 1, s);
+        return launch_gemm_pair_t<LAYOUT, 128, 4, 3>(amap, ga, 1, s);
     }
 #endif
+    if (tile.ks > 1)
+        return bn == 160 ? launch_gemm_t<LAYOUT, 160, BT_GEMM_BSTAGES, true>(amap, ga, tile.ks, s)
+                         : launch_gemm_t<LAYOUT, 128, BT_GEMM_BSTAGES, true>(amap, ga, tile.ks, s);
     // BN = 256: two weight stages (64 KB each) fit beside the activation ring;
     // with four decoder threads per row its CTA would exceed 1024 threads, and
     // pick_bn does not choose it
     if constexpr (gemm_threads(256) <= 1024) {
-        if (bn == 256) return launch_gemm_t<LAYOUT, 256, 2>(amap, ga, s);
+        if (bn == 256) return launch_gemm_t<LAYOUT, 256, 2>(amap, ga, 1, s);
     }
-    return bn == 160 ? launch_gemm_t<LAYOUT, 160, BT_GEMM_BSTAGES>(amap, ga, s)
-                     : launch_gemm_t<LAYOUT, 128, BT_GEMM_BSTAGES>(amap, ga, s);
+    return bn == 160 ? launch_gemm_t<LAYOUT, 160, BT_GEMM_BSTAGES>(amap, ga, 1, s)
+                     : launch_gemm_t<LAYOUT, 128, BT_GEMM_BSTAGES>(amap, ga, 1, s);
 }
 
 cudaError_t launch_gemm(int layout, const uint8_t* codes, const uint16_t* scales, const void* x, int x_dtype,

@@ -144,8 +144,15 @@ def test_gemm_workspace_sizes(lib):
     # 160-wide ones with one activation tile per pair
     for layout in (0, 1):
         assert lib.bt_gemm_workspace_bytes(layout, 512, 5120, 1920) == base(512, 1920)
-    # M = 256: one activation tile per pair, nothing but the activations
-    assert lib.bt_gemm_workspace_bytes(0, 256, 5120, 5120) == base(256, 5120)
+    # M = 128 and 256 against N = 5120 fill the SMs by splitting K over the
+    # single-CTA kernel with 160-wide tiles (20 decoder warps): 4 ways for
+    # 32 tiles, 2 ways for 64
+    assert lib.bt_gemm_workspace_bytes(0, 128, 5120, 5120) == base(128, 5120) + 32 * 20 * 4 + 4 * 128 * 5120 * 4
+    assert lib.bt_gemm_workspace_bytes(0, 256, 5120, 5120) == base(256, 5120) + 64 * 20 * 4 + 2 * 256 * 5120 * 4
+    # 24 K groups allow 3 splits at most
+    assert lib.bt_gemm_workspace_bytes(1, 128, 5120, 3072) == base(128, 3072) + 32 * 20 * 4 + 3 * 128 * 5120 * 4
+    # 17408 columns fill the SMs without a split
+    assert lib.bt_gemm_workspace_bytes(0, 128, 17408, 5120) == base(128, 5120)
 
 
 def test_binding_refuses_cpu_tensors():

@@ -428,6 +428,22 @@ def test_gemm_two_tiles_per_pair_full(layout, N, K):
     assert np.array_equal(y, y2)
 
 
+@pytest.mark.parametrize("M,K", [(128, 4096), (256, 2176)])
+@pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
+def test_gemm_small_m_split_k_full(layout, M, K):
+    # M = 128 and 256 against N = 5120 split K over the single-CTA kernel:
+    # 32 K groups in four (8 each), 17 in two (8 and 9)
+    N = 5120
+    case = workloads.random_case(8570 + M, M, N, K)
+    xr = workloads.rng(8571 + M).standard_normal((M, K)) * 2.0
+    xr32 = xr.astype(np.float32).astype(np.float64)
+    y_ref, b = oracle.gemv(case["trits"], case["scales"], xr32)
+    y = run_gemm(case["trits"], case["scales"], None, None, layout, x_f32=xr32)
+    check_bf16(y, y_ref, b)
+    y2 = run_gemm(case["trits"], case["scales"], None, None, layout, x_f32=xr32)
+    assert np.array_equal(y, y2)
+
+
 def test_gemm_two_tiles_per_pair_two_pairs_sampled_rows():
     # M = 1024: two pairs along M, each with two activation tiles
     M, N, K = 1024, 17408, 2048
