@@ -882,15 +882,20 @@ def run_case(case: str, reps: int):
         for _ in range(reps):
             bt.gemv_batched(probs, sign, layout)
     elif case.startswith("gemm"):
-        # gemm_<layout>: pp512 on the 5120x5120 layer
+        # gemm[_2bit]: pp512 on the 5120x5120 layer; gemm_triple[_2bit]: on
+        # all three layers, one bt_gemm call each per rep
         layout = 1 if case.endswith("2bit") else 0
-        L = workloads.TRIPLE[0]
-        inp = workloads.layer_inputs("C3", L, M=512, index=0)
-        codes = bt.pack(torch.from_numpy(inp["trits"]).to(dev), layout)
-        sc = torch.from_numpy(inp["scales"].view(np.int16)).to(dev)
-        x = torch.from_numpy(inp["x"].view(np.int16)).to(dev).view(torch.bfloat16)
+        idxs = range(len(workloads.TRIPLE)) if "triple" in case else [0]
+        calls = []
+        for i in idxs:
+            L = workloads.TRIPLE[i]
+            inp = workloads.layer_inputs("C3", L, M=512, index=i)
+            calls.append((bt.pack(torch.from_numpy(inp["trits"]).to(dev), layout),
+                          torch.from_numpy(inp["scales"].view(np.int16)).to(dev),
+                          torch.from_numpy(inp["x"].view(np.int16)).to(dev).view(torch.bfloat16), L.N))
         for _ in range(reps):
-            bt.gemm(codes, sc, x, sign, L.N, layout)
+            for codes, sc, x, n in calls:
+                bt.gemm(codes, sc, x, sign, n, layout)
     elif case == "fwht":
         # 512 x 17408 (53 MB in + out) over distinct buffers: 10 of them exceed 4x L2
         g = workloads.rng(77)
@@ -919,7 +924,7 @@ def main():
     ap.add_argument("--no-sweep", action="store_true", help="skip the 384-matrix 27B-equivalent sweep")
     ap.add_argument("--case", default=None,
                     help="run one small workload for a profiler capture (gemv_m<M>[_2bit], batched[_2bit], "
-                         "gemm[_2bit], fwht)")
+                         "gemm[_triple][_2bit], fwht)")
     ap.add_argument("--reps", type=int, default=3)
     args = ap.parse_args()
     if args.case:

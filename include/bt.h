@@ -258,10 +258,17 @@ bt_status bt_gemv_noalloc(int layout, const uint8_t* codes, const uint16_t* scal
  *  order), then the tensor-core kernel, chained by programmatic dependent
  *  launch. With M % 256 == 0 the output tiles run as clusters of two CTAs
  *  that share each decoded weight tile (tcgen05 cta_group::2, M = 256 per
- *  instruction); otherwise one CTA per 128-row tile. Both forms add the same
- *  products in the same order per output, and repeated calls give
- *  bit-identical results. Waits are bounded: one that runs out sets
- *  BT_DEVERR_TIMEOUT and the affected outputs are unspecified.
+ *  instruction; with M % 512 == 0 a pair can take two 256-row tiles);
+ *  otherwise one CTA per 128-row tile. Grids too small for the SMs split K
+ *  (2-4 ways): each split stores FP32 partial products in the workspace and
+ *  the last to finish adds them in split order. The form is a function of
+ *  (layout, M, N, K, SM count), so repeated calls give bit-identical results;
+ *  different forms differ only in FP32 summation order.
+ *  The workspace (>= bt_gemm_workspace_bytes, which includes the partials
+ *  and arrival counters when K is split; the call zeroes the counters) is
+ *  scratch, as for bt_gemv.
+ *  Waits are bounded: one that runs out sets BT_DEVERR_TIMEOUT and the
+ *  affected outputs are unspecified.
  * Source: pp512 prompt processing, release summary, section 实测吞吐.
  */
 size_t bt_gemm_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K);

@@ -28,9 +28,9 @@
 //                   exact -- and store them in the tensor cores' K-major
 //                   128-byte-swizzled layout: BT_GEMM_TPR (4) threads per
 //                   weight row, each one 128 / TPR-slot part of the group
-//                   (BN TPR / 32 warps); then warps 2-5
-//                   read the accumulator back (tcgen05.ld) and write bf16 Y
-//                   scaled by 2^e_m.
+//                   (BN TPR / 32 warps); then all of them read the
+//                   accumulator back (tcgen05.ld) and write bf16 Y scaled by
+//                   2^e_m (or, with K split, FP32 partials first).
 //     A group's 128 trits are laid out in "slot" order: slot 2w + h holds
 //     half h of decoded word w. For base-3, word w < 60 is digit w % 5 of
 //     bytes (2p, 2p+1), p = w / 5; words 60-62 are digits 0-2 of bytes
@@ -429,7 +429,7 @@ struct GemmArgs {
     int64_t row_bytes;
     int32_t* dev_err;
     float* part;          // split-K: [2][M][N] FP32 partial products
-    int32_t* tile_cnt;    // split-K: [tiles][4] arrivals per epilogue warp
+    int32_t* tile_cnt;    // split-K: [tiles][decoder warps] arrivals
 };
 
 #ifndef BT_GEMM_ASTAGES
