@@ -61,12 +61,16 @@ constexpr int kGemmBK = 128;             // one weight group per stage
 constexpr int kGemmTpr = BT_GEMM_TPR;
 __host__ __device__ constexpr int gemm_dec_warps(int bn) { return bn * kGemmTpr / 32; }
 __host__ __device__ constexpr int gemm_threads(int bn) { return (2 + gemm_dec_warps(bn)) * 32; }
-// Base-3 decode table: per code, one 32-bit word per lane (each lane reads
-// only its own bank, so lookups never conflict) holding the code's five
-// base-3 digits as 2-bit fields plus the FP16 exponent bits of 1024 (0x6400)
-// in both halves; bit 31 marks codes 243-255.
+// -DBT_GEMM_B3_LUT: base-3 digits from a decode table in shared memory
+// instead of b3_pair_fields' arithmetic. Per code, one 32-bit word per lane
+// (each lane reads only its own bank, so lookups never conflict) holding the
+// code's five base-3 digits as 2-bit fields plus the FP16 exponent bits of
+// 1024 (0x6400) in both halves; bit 31 marks codes 243-255. The 32 KB it
+// takes cost a weight stage.
+#ifdef BT_GEMM_B3_LUT
 constexpr int kGemmLutRow = 32 * 4;                       // bytes per code
 constexpr int kGemmLutBytes = 256 * kGemmLutRow;
+#endif
 
 // ---------------------------------------------------------------- helpers ----
 
@@ -236,6 +240,25 @@ struct GemmPart {
     static constexpr int NW = LAYOUT == BT_LAYOUT_B3 ? (kGemmTpr == 2 ? 7 : 4) : WPT / 8;
 };
 
+// Base-3 digits of a byte pair, computed: bytes 2p (low half) and 2p + 1
+// (high half) of pr become the 2-bit digit fields of both codes with the FP16
+// exponent bits of 1024 in each half. floor(c / 3) = (171 c) >> 9 for
+// c < 256, and one 32-bit multiply serves both halves (171 c < 2^16, and the
+// mask drops what the high half shifts down). Codes 243-255 set bit 8 or 24
+// of err.
+__device__ __forceinline__ uint32_t b3_pair_fields(uint32_t pr, uint32_t& err) {
+    uint32_t x = prmt(pr, 0u, 0x4140u);                  // [byte 2p, 0, byte 2p+1, 0]
+    err |= (x + 0x000D000Du) & 0x01000100u;
+    uint32_t f = 0x64006400u;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const uint32_t q = ((x * 171u) >> 9) & 0x007F007Fu;
+        f |= (x - 3u * q) << (2 * i);
+        x = q;
+    }
+    return f | (x << 8);
+}
+
 // Decode part QQ of one group (WPT words of FP16 pairs s t, slot order) from
 // the part's packed words. Base-3 word w < 60 is digit w % 5 of byte pair
 // w / 5; words 60-62 are digits 0-2 of pair 12, word 63 digits 3-4 of byte
@@ -254,10 +277,16 @@ __device__ __forceinline__ void gemm_decode_part(const uint32_t (&cw)[GemmPart<L
             const int p = P0 + j;
             if (p > 12) continue;
             const uint32_t pr = cw[j];
+#ifdef BT_GEMM_B3_LUT
             const uint32_t va = *reinterpret_cast<const uint32_t*>(lut_lane + (pr & 0xFFu) * kGemmLutRow);
             const uint32_t vb = *reinterpret_cast<const uint32_t*>(lut_lane + (pr >> 8) * kGemmLutRow);
             err |= (va | vb) & 0x80000000u;
             const uint32_t x = prmt(va, vb, 0x7610u);   // byte 2p's fields low, byte 2p+1's high
+#else
+            (void)lut_lane;
+            const uint32_t x = b3_pair_fields(pr, err);
+            const uint32_t va = x;                      // byte 2p's fields in the low half
+#endif
             const int nw = p < 12 ? 5 : 3;
 #pragma unroll
             for (int i = 0; i < nw; ++i) {
@@ -448,7 +477,11 @@ struct GemmSmem {
     static constexpr int kA1 = kGemmBM * kGemmBK * 2;  // 32 KB per 128-row tile: two 64-column panels
     static constexpr int kA = MT * kA1;
     static constexpr int kB = BN * kGemmBK * 2;
+#ifdef BT_GEMM_B3_LUT
     static constexpr int kLut = LAYOUT == BT_LAYOUT_B3 ? kGemmLutBytes : 0;
+#else
+    static constexpr int kLut = 0;                      // base-3 digits are computed
+#endif
     static constexpr int kBars = 1024;                  // barriers, TMEM address, flags
     static constexpr int kTotal = kAStages * kA + kBStages * kB + kLut + kBars + 1024;  // + alignment slack
 };
@@ -525,6 +558,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
         *abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+#ifdef BT_GEMM_B3_LUT
     if (LAYOUT == BT_LAYOUT_B3) {
         // digits of each code as 2-bit fields with the FP16 exponent bits of
         // 1024 (0x6400), in both halves, so that field i masked out of a half
@@ -539,6 +573,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
             reinterpret_cast<uint32_t*>(lut)[idx] = f | (f << 16) | (code < 243 ? 0u : 0x80000000u);
         }
     }
+#endif
     if (warp == 1) {
         if constexpr (PAIR) {
             asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -754,7 +789,11 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
             if (!stage(kt + 1, bufB, sB)) break;
             load_group(kt + 3, bufB, sB);
         }
+#ifdef BT_GEMM_B3_LUT
         if (LAYOUT == BT_LAYOUT_B3 ? (err >> 31) : (err != 0)) bad |= BT_DEVERR_INVALID_CODE;
+#else
+        if (err != 0) bad |= BT_DEVERR_INVALID_CODE;
+#endif
 
         // ---------------- epilogue: TMEM -> bf16 Y. Every decoder warp takes
         // part: warp w reads TMEM lanes 32 (w % 4) .. 32 (w % 4) + 31, i.e. rows
@@ -1085,12 +1124,14 @@ size_t gemm_workspace_bytes(int layout, int64_t M, int64_t N, int64_t K, int num
 template <int LAYOUT>
 static cudaError_t dispatch_gemm(GemmTile tile, const CUtensorMap& amap, const GemmArgs& ga, cudaStream_t s) {
     const int bn = tile.bn;
+    // a decode table in shared memory leaves room for one weight stage less
+    constexpr bool kTableLayout = GemmSmem<LAYOUT, 128, 1>::kLut > 0;
 #ifndef BT_GEMM_NO_PAIR
     if (tile.pair) {
         if (tile.mt == 2 && bn == 256)
-            return launch_gemm_pair_t<LAYOUT, 256, LAYOUT == BT_LAYOUT_B3 ? 2 : 3, 2, 2>(amap, ga, 1, s);
+            return launch_gemm_pair_t<LAYOUT, 256, kTableLayout ? 2 : 3, 2, 2>(amap, ga, 1, s);
         if (tile.mt == 2 && bn == 160 && tile.ks > 1)
-            return launch_gemm_pair_t<LAYOUT, 160, LAYOUT == BT_LAYOUT_B3 ? 3 : 4, 2, 2, true>(amap, ga, tile.ks, s);
+            return launch_gemm_pair_t<LAYOUT, 160, kTableLayout ? 3 : 4, 2, 2, true>(amap, ga, tile.ks, s);
         if constexpr (LAYOUT == BT_LAYOUT_2BIT) {
             if (tile.mt == 2 && bn == 80)
                 return launch_gemm_pair_t<LAYOUT, 80, BT_GEMM_PAIR_SB80, 2, 2>(amap, ga, 1, s);

@@ -455,6 +455,26 @@ def test_gemm_two_tiles_per_pair_two_pairs_sampled_rows():
     check_bf16(y[rows], y_ref, b)
 
 
+@pytest.mark.parametrize("M", [128, 512])   # 512: the split-K pair kernel at N = 5120
+@pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
+def test_gemm_flags_invalid_codes(layout, M):
+    N, K = (128, 1024) if M == 128 else (5120, 2048)
+    case = workloads.random_case(8650 + M, M, N, K)
+    codes = oracle.pack(case["trits"], layout)
+    codes[N - 3, 40] = 247 if layout == bt.LAYOUT_B3 else 0xC3
+    err = torch.zeros(1, dtype=torch.int32, device=DEV)
+    y = bt.gemm(T(codes), T(case["scales"]), T(case["x"], "bf16"), T(case["sign"]), N, layout, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) & bt.DEVERR_INVALID_CODE
+    assert torch.isfinite(y.float()).all()
+    # and a clean call on the same shape reports nothing
+    err.zero_()
+    bt.gemm(T(oracle.pack(case["trits"], layout)), T(case["scales"]), T(case["x"], "bf16"), T(case["sign"]), N,
+            layout, dev_err=err)
+    torch.cuda.synchronize()
+    assert int(err.item()) == 0
+
+
 @pytest.mark.parametrize("M", [128, 256])
 def test_gemm_special_cases(M):
     N, K = 128, 1024
