@@ -130,6 +130,13 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void gemm_cp_async16(uint32_t dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" :: "r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void gemm_cp_async_wait_all() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_all;" ::: "memory");
+}
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
@@ -867,45 +874,100 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
             arrived = __shfl_sync(0xffffffffu, arrived, 0);
             if (arrived == ks - 1) {
                 __threadfence();   // the other splits' stores, made visible by their fences, are seen
+                // The other splits' 32 x 32 chunks land in this warp's slots of the
+                // drained rings by cp.async, a batch of whole units at a time, so
+                // that a batch costs one round trip to L2. A slot is [32 rows][32 f32]
+                // with row r's 16-byte pieces rotated by r % 8, so that the row-per-
+                // lane reads below do not conflict.
+                constexpr int kRingBytes = SA * SM::kA + SB * SM::kB;
+                constexpr int kTbBytes = NDW * 32 * 33 * 4;
+                constexpr int kSlots = (kRingBytes - kTbBytes) / NDW / 4096;
+                const int per = ks - 1;
+                const int upb = per <= kSlots ? kSlots / per : 0;   // units per batch
+                const uint32_t land = smem_addr(a_ring) + kTbBytes + (warp - 2) * kSlots * 4096;
+                const float* land_f = reinterpret_cast<const float*>(a_ring + kTbBytes + (warp - 2) * kSlots * 4096);
 #pragma unroll 1
-                for (int u = slot; u < MT * NCH; u += nslot) {
-                    const int j = u / NCH, c0 = (u - j * NCH) * 32;
-                    const int mb = m0 + j * 2 * kGemmBM + quarter * 32;
-                    const int64_t off = (int64_t)mb * a.N + n0 + c0;
-                    float acc[32];
+                for (int ub = slot; ub < MT * NCH; ub += (upb > 0 ? upb : 1) * nslot) {
+                    if (upb > 0) {
+                        int t = 0;
 #pragma unroll 1
-                    for (int zz = 0; zz < ks; ++zz) {
-                        if (zz == z) {   // warp-uniform
-                            uint32_t r[32];
-                            tmem_ld32(tq + j * BN + c0, r);
+                        for (int u = ub; u < MT * NCH && t < upb; u += nslot, ++t) {
+                            const int j = u / NCH, c0 = (u - j * NCH) * 32;
+                            const int64_t off = (int64_t)(m0 + j * 2 * kGemmBM + quarter * 32) * a.N + n0 + c0;
+                            int pz = 0;
+#pragma unroll 1
+                            for (int zz = 0; zz < ks; ++zz) {
+                                if (zz == z) continue;
+                                const float* src = a.part + zz * plane + off;
+                                const uint32_t dst = land + (t * per + pz) * 4096;
 #pragma unroll
-                            for (int c = 0; c < 32; ++c)
-                                acc[c] = zz == 0 ? __uint_as_float(r[c]) : acc[c] + __uint_as_float(r[c]);
-                        } else {
-                            const float* src = a.part + zz * plane + off;
-#pragma unroll
-                            for (int i0 = 0; i0 < 8; i0 += 4) {   // two rounds of four loads in flight
-                                float4 q[4];
-#pragma unroll
-                                for (int i = 0; i < 4; ++i)
-                                    q[i] = __ldcg(reinterpret_cast<const float4*>(src + (int64_t)(4 * (i0 + i) + prow) * a.N + pcol));
-#pragma unroll
-                                for (int i = 0; i < 4; ++i) {
-                                    float* t = tb + (4 * (i0 + i) + prow) * 33 + pcol;
-                                    t[0] = q[i].x; t[1] = q[i].y; t[2] = q[i].z; t[3] = q[i].w;
+                                for (int i = 0; i < 8; ++i) {
+                                    const int row = 4 * i + prow;
+                                    gemm_cp_async16(dst + row * 128 + ((((pcol >> 2) ^ (row & 7))) << 4),
+                                                    src + (int64_t)row * a.N + pcol);
                                 }
+                                ++pz;
                             }
-                            __syncwarp();
-#pragma unroll
-                            for (int c = 0; c < 32; ++c)
-                                acc[c] = zz == 0 ? tb[lane * 33 + c] : acc[c] + tb[lane * 33 + c];
-                            __syncwarp();
                         }
+                        gemm_cp_async_wait_all();
+                        __syncwarp();
                     }
-                    uint32_t r[32];
+                    int t = 0;
+#pragma unroll 1
+                    for (int u = ub; u < MT * NCH && t < (upb > 0 ? upb : 1); u += nslot, ++t) {
+                        const int j = u / NCH, c0 = (u - j * NCH) * 32;
+                        const int mb = m0 + j * 2 * kGemmBM + quarter * 32;
+                        const int64_t off = (int64_t)mb * a.N + n0 + c0;
+                        float acc[32];
+                        int pz = 0;
+#pragma unroll 1
+                        for (int zz = 0; zz < ks; ++zz) {
+                            if (zz == z) {   // warp-uniform
+                                uint32_t r[32];
+                                tmem_ld32(tq + j * BN + c0, r);
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(acc[c]);
-                    epi_store<32>(r, a.rowscale[mb + lane], a.y + off + (int64_t)lane * a.N);
+                                for (int c = 0; c < 32; ++c)
+                                    acc[c] = zz == 0 ? __uint_as_float(r[c]) : acc[c] + __uint_as_float(r[c]);
+                            } else if (upb > 0) {
+                                const float4* rowp = reinterpret_cast<const float4*>(land_f + (t * per + pz) * 1024 + lane * 32);
+#pragma unroll
+                                for (int c4 = 0; c4 < 8; ++c4) {
+                                    const float4 v = rowp[c4 ^ (lane & 7)];
+                                    acc[4 * c4] = zz == 0 ? v.x : acc[4 * c4] + v.x;
+                                    acc[4 * c4 + 1] = zz == 0 ? v.y : acc[4 * c4 + 1] + v.y;
+                                    acc[4 * c4 + 2] = zz == 0 ? v.z : acc[4 * c4 + 2] + v.z;
+                                    acc[4 * c4 + 3] = zz == 0 ? v.w : acc[4 * c4 + 3] + v.w;
+                                }
+                                ++pz;
+                            } else {
+                                // no room for a unit's pieces: through the transpose
+                                // buffer, one partial chunk at a time
+                                const float* src = a.part + zz * plane + off;
+#pragma unroll
+                                for (int i0 = 0; i0 < 8; i0 += 4) {
+                                    float4 q[4];
+#pragma unroll
+                                    for (int i = 0; i < 4; ++i)
+                                        q[i] = __ldcg(reinterpret_cast<const float4*>(src + (int64_t)(4 * (i0 + i) + prow) * a.N + pcol));
+#pragma unroll
+                                    for (int i = 0; i < 4; ++i) {
+                                        float* tp = tb + (4 * (i0 + i) + prow) * 33 + pcol;
+                                        tp[0] = q[i].x; tp[1] = q[i].y; tp[2] = q[i].z; tp[3] = q[i].w;
+                                    }
+                                }
+                                __syncwarp();
+#pragma unroll
+                                for (int c = 0; c < 32; ++c)
+                                    acc[c] = zz == 0 ? tb[lane * 33 + c] : acc[c] + tb[lane * 33 + c];
+                                __syncwarp();
+                            }
+                        }
+                        uint32_t r[32];
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) r[c] = __float_as_uint(acc[c]);
+                        epi_store<32>(r, a.rowscale[mb + lane], a.y + off + (int64_t)lane * a.N);
+                    }
+                    __syncwarp();   // the batch's slots are read before the next batch lands
                 }
             }
         }
