@@ -222,7 +222,7 @@ bt_status bt_gemv_batched(int layout, const bt_gemv_problem* problems, int count
  * code that runs where cudaMalloc is unavailable or not allowed (inside a
  * custom allocator or memory-pool callback, in a runtime that has handed all
  * device memory to its own arena, or under a fixed memory budget decided
- * before the call). The paper has no counterpart; it is an interface
+ * before the call). The method has no counterpart; it is an interface
  * convenience of this library.
  * Arguments and results are those of bt_gemv without the workspace: the
  * scratch is an 8 MiB array in the library's own device memory, reserved on
