@@ -201,9 +201,21 @@ __device__ __forceinline__ void tc_mma_pair(uint32_t tmem_d, uint64_t a, uint64_
 }
 // arrive once on the barrier at this offset in both CTAs of the pair when the
 // pair's MMAs issued so far complete
-__device__ __forceinline__ void tc_commit_pair(uint32_t bar) {
+// commit to the barrier at this offset in both CTAs of the pair (cluster
+// ranks `pair_base` and pair_base + 1)
+__device__ __forceinline__ void tc_commit_pair(uint32_t bar, uint32_t pair_base) {
     asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;"
-                 :: "r"(bar), "h"((uint16_t)3) : "memory");
+                 :: "r"(bar), "h"((uint16_t)(3u << pair_base)) : "memory");
+}
+// this CTA's shared-memory address `a` as seen from the cluster, in CTA `rank`
+__device__ __forceinline__ uint32_t cluster_map(uint32_t a, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ void st_cluster_v4(uint32_t a, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+    asm volatile("st.shared::cluster.v4.b32 [%0], {%1, %2, %3, %4};" :: "r"(a), "r"(x), "r"(y), "r"(z), "r"(w)
+                 : "memory");
 }
 // arrive on the barrier at this offset in CTA `rank` of the cluster
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar, uint32_t rank) {
@@ -548,7 +560,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
     const int ks = SPLIT ? (int)gridDim.z : 1;
     const int kbase = SPLIT ? (int)blockIdx.z * a.G / ks : 0;
     const int ktiles = SPLIT ? ((int)blockIdx.z + 1) * a.G / ks - kbase : a.G;
-    const uint32_t rank = PAIR ? cluster_ctarank() : 0u;
+    // cluster ranks: pairs are (0, 1) and, when the two K halves of a split
+    // share the cluster, (2, 3); the even rank of a pair leads
+    const uint32_t crank = PAIR ? cluster_ctarank() : 0u;
+    const uint32_t rank = crank & 1u, pair_base = crank & ~1u;
     const bool leader = rank == 0;
 
     if (threadIdx.x == 0) {
@@ -656,14 +671,14 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
                     }
                 }
                 if constexpr (PAIR) {
-                    tc_commit_pair(smem_addr(emptyA + s_a));
-                    tc_commit_pair(smem_addr(emptyB + s_b));
+                    tc_commit_pair(smem_addr(emptyA + s_a), pair_base);
+                    tc_commit_pair(smem_addr(emptyB + s_b), pair_base);
                 } else {
                     tc_commit(smem_addr(emptyA + s_a));
                     tc_commit(smem_addr(emptyB + s_b));
                 }
             }
-            if constexpr (PAIR) tc_commit_pair(smem_addr(accf));
+            if constexpr (PAIR) tc_commit_pair(smem_addr(accf), pair_base);
             else tc_commit(smem_addr(accf));
         }
         if constexpr (PAIR) {
@@ -678,7 +693,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
                         bad = BT_DEVERR_TIMEOUT; *abort_flag = 1; break;
                     }
                     if (*abort_flag) break;
-                    mbar_arrive_cluster(smem_addr(fullB + s_b), 0u);
+                    mbar_arrive_cluster(smem_addr(fullB + s_b), pair_base);
                 }
             }
         }
@@ -836,6 +851,8 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
                     epi_store<32>(r, rs, yrow);
                 }
             }
+        } else if (PAIR) {
+            // the pair's two K halves meet through the cluster, after the role branches
         } else if (do_epi) {
             // split K: store this split's FP32 partial products, count in; the
             // warp arriving last (the ks-th, for this warp's chunks of this
@@ -974,6 +991,62 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
     }
     bad = __reduce_or_sync(0xffffffffu, bad);
     if (lane == 0) report(a.dev_err, bad);
+    if constexpr (PAIR && SPLIT) {
+        // K split in two across the cluster: the pair of cluster ranks (0, 1)
+        // has the first half of the K groups, (2, 3) the second, for the same
+        // rows and columns. Split z finishes activation tile j = z: it sends
+        // its partial products of tile 1 - z to the CTA of rank crank ^ 2
+        // (through distributed shared memory, into that CTA's drained
+        // activation ring) and adds the partials it receives to its own,
+        // split 0's first (a + b: the same bits either way round). Every
+        // thread of the cluster passes both barriers.
+        static_assert(MT == 2, "one activation tile per split");
+        constexpr int kXs = BN + 4;   // row stride (floats) of the exchange buffer
+        static_assert(kGemmBM * kXs * 4 <= SA * SM::kA, "exchange buffer in the activation ring");
+        constexpr int NDW = gemm_dec_warps(BL);
+        constexpr int NCH = BN / 32;
+        const bool dec = warp >= 2;
+        const int quarter = warp & 3;
+        const int w0 = 2 + ((quarter + 2) & 3);
+        const int slot = (warp - w0) >> 2;
+        const int nslot = (NDW + 1 - w0) / 4 + 1;
+        const uint32_t tq = tmem + (static_cast<uint32_t>(quarter * 32) << 16);
+        const int z = (int)blockIdx.z;
+        const int row = quarter * 32 + lane;   // this lane's TMEM lane
+        cluster_sync_all();                    // every MMA of the cluster is complete: the rings are free
+        const bool go = dec && __all_sync(0xffffffffu, !*abort_flag);
+        if (go) {
+            const uint32_t rb = cluster_map(smem_addr(a_ring), crank ^ 2u) + (uint32_t)(row * kXs * 4);
+#pragma unroll 1
+            for (int u = slot; u < NCH; u += nslot) {
+                uint32_t r[32];
+                tmem_ld32(tq + (1 - z) * BN + u * 32, r);
+#pragma unroll
+                for (int v = 0; v < 8; ++v)
+                    st_cluster_v4(rb + (uint32_t)((u * 32 + 4 * v) * 4), r[4 * v], r[4 * v + 1], r[4 * v + 2], r[4 * v + 3]);
+            }
+        }
+        cluster_sync_all();                    // the other split's half is in this CTA's ring
+        if (go) {
+            const int m = m0 + z * 2 * kGemmBM + row;
+            const float rs = a.rowscale[m];
+            const float4* rp = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(a_ring) + row * kXs);
+#pragma unroll 1
+            for (int u = slot; u < NCH; u += nslot) {
+                uint32_t r[32];
+                tmem_ld32(tq + z * BN + u * 32, r);
+#pragma unroll
+                for (int v = 0; v < 8; ++v) {
+                    const float4 o = rp[u * 8 + v];
+                    r[4 * v] = __float_as_uint(__uint_as_float(r[4 * v]) + o.x);
+                    r[4 * v + 1] = __float_as_uint(__uint_as_float(r[4 * v + 1]) + o.y);
+                    r[4 * v + 2] = __float_as_uint(__uint_as_float(r[4 * v + 2]) + o.z);
+                    r[4 * v + 3] = __float_as_uint(__uint_as_float(r[4 * v + 3]) + o.w);
+                }
+                epi_store<32>(r, rs, a.y + (int64_t)m * a.N + n0 + u * 32);
+            }
+        }
+    }
     tc_fence_before();
     __syncthreads();
     if constexpr (PAIR) {
@@ -1083,7 +1156,7 @@ static cudaError_t launch_gemm_pair_t(const CUtensorMap& amap, const GemmArgs& g
     attr[1].id = cudaLaunchAttributeClusterDimension;
     attr[1].val.clusterDim.x = 2;
     attr[1].val.clusterDim.y = 1;
-    attr[1].val.clusterDim.z = 1;
+    attr[1].val.clusterDim.z = SPLIT ? ks : 1;   // the K halves of a tile share a cluster
     cfg.attrs = attr;
     cfg.numAttrs = 2;
     return cudaLaunchKernelEx(&cfg, kern, amap, ga);
@@ -1098,12 +1171,13 @@ static cudaError_t launch_gemm_pair_t(const CUtensorMap& amap, const GemmArgs& g
 //    layer went from 830 to 950 TFLOP/s (base-3), 930 to 1210 (2-bit).
 //  - 160 wide with K split in two (N = 5120 at M = 512: 2 x 64 CTAs, the
 //    same grid as one tile per pair without the split). Half the K groups per
-//    CTA and twice the MMAs per decoded group; the halves meet through FP32
-//    partials in the workspace. 5120 x 17408 went from 546 to 756 TFLOP/s
-//    (base-3) and 576 to 830 (2-bit); 5120 x 5120 from 453 to 487 and 498 to
-//    541. Splitting K in three over 256-wide tiles (120 CTAs, fewer activation
-//    reads) lost: the CTA arriving last adds two partial tiles of 256 KB
-//    alone, which left a 20-30 us tail.
+//    CTA and twice the MMAs per decoded group. The two pairs of a tile form
+//    one cluster of four CTAs and swap halves through distributed shared
+//    memory (each finishes one activation tile). 5120 x 17408 went from 546
+//    to 771 TFLOP/s (base-3); 5120 x 5120 from 453 to 540. Exchanging FP32
+//    partials through the workspace instead, with the CTA finishing second
+//    adding them, left a 10-15 us tail per layer. Splitting K in three over
+//    256-wide tiles (120 CTAs, fewer activation reads) lost the same way.
 //  - 80 wide, 2-bit only, where K is too short to split.
 struct GemmTile {
     int bn, mt, ks;   // weight tile width, activation tiles per CTA (pair), K splits
@@ -1161,8 +1235,8 @@ static GemmTile pick_tile(int layout, int64_t M, int64_t N, int64_t K, int num_s
 #endif
 }
 
-// workspace: the rotated FP16 activations, the row scales and, for split K,
-// the arrival counters and both halves' FP32 partial products
+// workspace: the rotated FP16 activations, the row scales and, for K split
+// over single CTAs, the arrival counters and the splits' FP32 partial products
 struct GemmWs {
     size_t xt, rowscale, cnt, part, total;
     int n_cnt;
@@ -1173,9 +1247,11 @@ static GemmWs gemm_ws_layout(const GemmTile& t, int64_t M, int64_t N, int64_t K)
     w.xt = 0;
     w.rowscale = gemm_align((size_t)M * K * 2, 256);
     w.cnt = w.rowscale + gemm_align((size_t)M * 4, 256);
-    w.n_cnt = t.ks > 1 ? (int)((M / (kGemmBM * t.mt)) * (N / t.bn) * gemm_dec_warps(t.pair ? t.bn / 2 : t.bn)) : 0;
+    // (split pairs exchange their halves inside the cluster and need neither)
+    const bool global_split = t.ks > 1 && !t.pair;
+    w.n_cnt = global_split ? (int)((M / kGemmBM) * (N / t.bn) * gemm_dec_warps(t.bn)) : 0;
     w.part = w.cnt + gemm_align((size_t)w.n_cnt * 4, 256);
-    w.total = w.part + (t.ks > 1 ? (size_t)t.ks * M * N * 4 : 0);
+    w.total = w.part + (global_split ? (size_t)t.ks * M * N * 4 : 0);
     return w;
 }
 
@@ -1192,7 +1268,7 @@ static cudaError_t dispatch_gemm(GemmTile tile, const CUtensorMap& amap, const G
     if (tile.pair) {
         if (tile.mt == 2 && bn == 256)
             return launch_gemm_pair_t<LAYOUT, 256, kTableLayout ? 2 : 3, 2, 2>(amap, ga, 1, s);
-        if (tile.mt == 2 && bn == 160 && tile.ks > 1)
+        if (tile.mt == 2 && bn == 160 && tile.ks == 2)   // the kernel pairs split z with cluster rank ^ 2
             return launch_gemm_pair_t<LAYOUT, 160, kTableLayout ? 3 : 4, 2, 2, true>(amap, ga, tile.ks, s);
         if constexpr (LAYOUT == BT_LAYOUT_2BIT) {
             if (tile.mt == 2 && bn == 80)

@@ -134,12 +134,11 @@ def test_gemm_workspace_sizes(lib):
     # ... are all that 17408 x 5120 needs (256-wide tiles, two activation
     # tiles per pair, 136 CTAs)
     assert lib.bt_gemm_workspace_bytes(0, 512, 17408, 5120) == base(512, 5120)
-    # N = 5120 at M = 512 splits K in two over 160-wide tiles: 64 tiles x 10
-    # decoder warps of arrival counters, then both halves' FP32 partials
-    cnt = 64 * 10 * 4
+    # N = 5120 at M = 512 splits K in two over 160-wide tiles; the two pairs
+    # of a tile share a cluster and swap halves in shared memory: nothing more
     for K in (2176, 5120, 17408):
         for layout in (0, 1):
-            assert lib.bt_gemm_workspace_bytes(layout, 512, 5120, K) == base(512, K) + cnt + 2 * 512 * 5120 * 4
+            assert lib.bt_gemm_workspace_bytes(layout, 512, 5120, K) == base(512, K)
     # 15 K groups are too few to split: 2-bit takes 80-wide tiles, base-3
     # 160-wide ones with one activation tile per pair
     for layout in (0, 1):

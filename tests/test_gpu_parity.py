@@ -406,9 +406,9 @@ def _two_tile_case(N, K):
     # at M = 512, N = 17408 takes 256-wide weight tiles with two 256-row
     # activation tiles per CTA pair; N = 5120 takes 160-wide tiles with two
     # activation tiles per pair and K split in two (17 K groups: halves of 8
-    # and 9), the CTA finishing second adding the partial products. Small K
-    # keeps the whole output cheap for the oracle; both have odd numbers of
-    # K groups.
+    # and 9), the two pairs of a tile sharing a cluster and swapping halves in
+    # shared memory. Small K keeps the whole output cheap for the oracle; both
+    # have odd numbers of K groups.
     M = 512
     case = workloads.random_case(8550 + N, M, N, K)
     xr = workloads.rng(8551 + N).standard_normal((M, K)) * 2.0
@@ -423,7 +423,7 @@ def test_gemm_two_tiles_per_pair_full(layout, N, K):
     case, xr32, y_ref, b = _two_tile_case(N, K)
     y = run_gemm(case["trits"], case["scales"], None, None, layout, x_f32=xr32)
     check_bf16(y, y_ref, b)
-    # the splits meet in whichever order they finish: same bits each call
+    # the splits meet whatever their timing: same bits each call
     y2 = run_gemm(case["trits"], case["scales"], None, None, layout, x_f32=xr32)
     assert np.array_equal(y, y2)
 
