@@ -259,14 +259,16 @@ bt_status bt_gemv_noalloc(int layout, const uint8_t* codes, const uint16_t* scal
  *  launch. With M % 256 == 0 the output tiles run as clusters of two CTAs
  *  that share each decoded weight tile (tcgen05 cta_group::2, M = 256 per
  *  instruction; with M % 512 == 0 a pair can take two 256-row tiles);
- *  otherwise one CTA per 128-row tile. Grids too small for the SMs split K
- *  (2-4 ways): each split stores FP32 partial products in the workspace and
- *  the last to finish adds them in split order. The form is a function of
+ *  otherwise one CTA per 128-row tile. Grids too small for the SMs split K:
+ *  in two for pairs (the two pairs of a tile form a cluster of four CTAs and
+ *  swap halves in shared memory), 2-4 ways for single CTAs (each split stores
+ *  FP32 partial products in the workspace and the last to finish adds them
+ *  in split order). The form is a function of
  *  (layout, M, N, K, SM count), so repeated calls give bit-identical results;
  *  different forms differ only in FP32 summation order.
  *  The workspace (>= bt_gemm_workspace_bytes, which includes the partials
- *  and arrival counters when K is split; the call zeroes the counters) is
- *  scratch, as for bt_gemv.
+ *  and arrival counters when K is split over single CTAs; the call zeroes
+ *  the counters) is scratch, as for bt_gemv.
  *  Waits are bounded: one that runs out sets BT_DEVERR_TIMEOUT and the
  *  affected outputs are unspecified.
  * Source: pp512 prompt processing, release summary, section 实测吞吐.
