@@ -44,7 +44,16 @@
 //     With M % 256 == 0 the tiles run as CTA pairs (clusters of two along
 //     M): both CTAs decode half of a BN-row weight tile each, and the pair
 //     leader issues tcgen05.mma.cta_group::2 (M 256) over both CTAs' shared
-//     memory, so each decoded weight row serves 256 activation rows.
+//     memory, so each decoded weight row serves 256 activation rows. With
+//     M % 512 == 0 a pair can take two 256-row activation tiles (512 rows
+//     per decoded weight row), and where that leaves too few CTAs the K
+//     groups are split in two between two pairs of one cluster of four CTAs,
+//     which swap halves through distributed shared memory at the end. Small
+//     grids of single CTAs split K 2-4 ways through FP32 partials in the
+//     workspace instead (the tile forms and their measurements are listed
+//     above pick_tile).
+// Base-3 digits are computed per byte pair (b3_pair_fields) rather than read
+// from a table, which leaves shared memory for one more weight stage.
 // Waits on barriers are bounded: a wait that runs out sets BT_DEVERR_TIMEOUT,
 // the CTA skips the rest of its work and still releases its TMEM.
 #include "bt_internal.cuh"
