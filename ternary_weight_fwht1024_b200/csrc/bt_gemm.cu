@@ -620,7 +620,10 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
     if constexpr (PAIR) cluster_sync_all();   // both CTAs' barriers exist before any remote arrival
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    pdl_wait();  // the activations come from the prep kernel
+    // the activations and row scales come from the prep kernel: the TMA and
+    // MMA warps wait for it here, the decoders once their first weight loads
+    // (never written by a kernel this one may overlap) are in flight
+    if (warp < 2) pdl_wait();
 
     int bad = 0;
     if (warp == 0) {
@@ -813,6 +816,7 @@ gemm_kernel(const __grid_constant__ CUtensorMap amap, GemmArgs a) {
         uint32_t bufA[NW], bufB[NW], sA = 0, sB = 0;
         load_group(0, bufA, sA);
         load_group(1, bufB, sB);
+        pdl_wait();
         for (int kt = 0; kt < ktiles; kt += 2) {
             if (!stage(kt, bufA, sA)) break;
             load_group(kt + 2, bufA, sA);
