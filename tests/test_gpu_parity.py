@@ -444,6 +444,19 @@ def test_gemm_small_m_split_k_full(layout, M, K):
     assert np.array_equal(y, y2)
 
 
+@pytest.mark.parametrize("layout", [bt.LAYOUT_B3, bt.LAYOUT_2BIT])
+def test_gemm_split_clusters_two_pairs_along_m_sampled_rows(layout):
+    # M = 1024 against N = 5120: two clusters along M, each of two pairs with
+    # two activation tiles and one half of K (24 K groups, rotated input)
+    M, N, K = 1024, 5120, 3072
+    case = workloads.random_case(8580 + layout, M, N, K)
+    y = run_gemm(case["trits"], case["scales"], case["x"], case["sign"], layout)
+    rows = tile_rows(M, 8581)
+    xr = oracle.rotate_bf16(case["x"][rows], case["sign"])
+    y_ref, b = oracle.gemv(case["trits"], case["scales"], xr)
+    check_bf16(y[rows], y_ref, b)
+
+
 def test_gemm_two_tiles_per_pair_two_pairs_sampled_rows():
     # M = 1024: two pairs along M, each with two activation tiles
     M, N, K = 1024, 17408, 2048
